@@ -1,0 +1,417 @@
+"""Benchmark of the WHALE attention-fusion forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step is one pass of the whole hot path (every layer of the stack: RMSNorm + projections,
+split-L cross-attention, Fusion MLP, SwiGLU FFN) over one batch of synthetic inputs that are
+already resident in HBM. The default workload is the 15k-history stack (B=64 examples,
+N=32 Wukong tokens, d=512, 8 heads, 8 layers, lognormal history lengths in [64, 15000]).
+Every layer reads its own 0.4 GB state slab, larger than the 126 MB L2, so no L2 flush is
+needed between steps. Under torchrun each rank runs its own batch (weak scaling, examples are
+independent: no data-path collective); the step time is the max over ranks.
+
+Prints one JSON line (rank 0). `--impl reference` times the fp64 CPU oracle instead (the
+reference arm of this repository), on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from wukong_hstu_cross_b200 import inputs as I  # noqa: E402
+
+METRIC = "WHALE fusion-layer examples/s @15k jagged history; % of HBM/TC roofline"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            p = json.load(fh)
+        return p, "measured"
+    except Exception:
+        return PEAKS_FALLBACK, "fallback"
+
+
+# ------------------------------------------------------------------------------------------------
+# algorithmic work per step (bf16 storage)
+# ------------------------------------------------------------------------------------------------
+def step_work(w: I.Workload, total_L: int) -> dict:
+    """FLOPs and bytes per kernel family for one layer (no re-reads, no partials)."""
+    B, N, d, H, Fh = w.batch, w.n_tokens, w.d, w.ffn_hidden, w.fusion_hidden
+    rows = B * N
+    e = 2
+    return {
+        "kv_proj": {"flops": 2.0 * total_L * d * 2 * d, "bytes": e * (total_L * d + total_L * 2 * d + 2 * d * d)},
+        "attention": {"flops": 4.0 * rows * 0 + 4.0 * N * total_L * d,   # 2 matmuls of N x L x d per example
+                      "bytes": e * (total_L * 2 * d + 2 * rows * d)},
+        "q_proj": {"flops": 2.0 * rows * d * d, "bytes": e * (2 * rows * d + d * d)},
+        "fusion_mlp": {"flops": 2.0 * rows * (2 * d * Fh + Fh * d), "bytes": e * (3 * rows * d + 2 * rows * Fh + 3 * d * Fh)},
+        "swiglu_ffn": {"flops": 2.0 * rows * (d * 2 * H + H * d), "bytes": e * (3 * rows * d + 2 * rows * H + 3 * d * H)},
+    }
+
+
+def launches_per_step(w: I.Workload) -> int:
+    # once: residual-stream set-up; per layer: weight fold, Q GEMM, K|V GEMM, attention, combine,
+    # Fusion GEMM(s), up|gate GEMM, down GEMM
+    return 1 + w.n_layers * (8 + (1 if w.fusion_hidden > 0 else 0))
+
+
+# ------------------------------------------------------------------------------------------------
+# clocks sampled while the timed region runs
+# ------------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"whale_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.fh,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None:
+            return None
+        try:
+            rows = [r.split(",") for r in open(self.path).read().strip().splitlines() if r.strip()]
+        except Exception:
+            return None
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+                for k, v in zip(names, r[5:9]):
+                    if v.strip() == "Active":
+                        reasons.add(k)
+            except Exception:
+                continue
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU baseline: the oracle on a bounded sample of the workload
+# ------------------------------------------------------------------------------------------------
+def oracle_sample(w: I.Workload, budget_s: float = 15.0, max_examples: int = 64):
+    from oracle import whale_oracle as O
+    L = I.draw_lengths(w)
+    lws = I.make_all_weights(w)
+    done, t_oracle = 0, 0.0
+    toks = 0
+    sample_tokens = w.n_tokens
+    if w.candidates:   # serving workload: time 64 of the request's candidate tokens, scale per example
+        sample_tokens = 64
+    for b in range(min(w.batch, max_examples)):
+        x = I.tokens_of_example(w, b)[:sample_tokens]
+        slabs = [I.states_of_example(w, l, b, int(L[b])) for l in range(w.n_layers)]
+        t0 = time.perf_counter()
+        O.fusion_stack_example(x, slabs, lws, w.n_heads, w.eps)
+        t_oracle += time.perf_counter() - t0
+        done += 1
+        toks += sample_tokens
+        if t_oracle >= budget_s:
+            break
+    cores = len(os.sched_getaffinity(0))
+    if w.candidates:
+        # per-token cost excluding nothing: the sampled tokens share the K/V projections (amortised as in serving)
+        value = 1.0 / (t_oracle * (w.n_tokens / toks))
+        desc = f"{done} request(s), {sample_tokens} of {w.n_tokens} candidate tokens timed, scaled per request"
+    else:
+        value = done / t_oracle
+        desc = f"first {done} of {w.batch} examples (all {w.n_layers} layers, all {w.n_tokens} tokens each)"
+    return {"value": value, "unit": "examples/s", "cores": cores, "kind": "oracle",
+            "sample": desc + f"; fp64 numpy, {t_oracle:.1f} s of CPU time"}
+
+
+# ------------------------------------------------------------------------------------------------
+def dist_setup(n_gpus):
+    import torch
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    from wukong_hstu_cross_b200 import dist as D
+    return D.max_over_ranks(x, world, device="cuda")
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = I.WORKLOADS[args.workload]
+    t0 = time.time()
+    vals = []
+    steps = max(args.steps, 1)
+    for _ in range(steps):
+        cb = oracle_sample(w, budget_s=args.ref_budget)
+        vals.append(cb["value"])
+    value = statistics.median(vals)
+    cb["value"] = value
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "examples/s", "n_gpus": args.gpus,
+            "steps": steps, "warmup": 0, "ms_per_step": 1e3 * w.batch / value if value else None,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "n_tokens": w.n_tokens, "d": w.d, "heads": w.n_heads,
+                       "layers": w.n_layers},
+            "cpu_baseline": cb, "e2e": {"value": value, "unit": "examples/s", "h2d_bytes_per_step": 0,
+                                        "d2h_bytes_per_step": 0},
+            "wall_s": time.time() - t0}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_kernel_case(args):
+    """One step entry point (K|V projection or attention) on one layer, for ncu captures.
+    Prints the average device time per launch; not a benchmark line."""
+    import torch
+    from wukong_hstu_cross_b200 import build
+    build.build()
+    from wukong_hstu_cross_b200 import harness as Hn
+    from wukong_hstu_cross_b200 import whale as Wb
+    w = I.WORKLOADS[args.workload].replace(n_layers=1)
+    if args.batch:
+        w = w.replace(batch=args.batch)
+    p = Hn.build_problem(w, device="cuda")
+    T = p.total_L
+    kv = torch.empty(T, 2 * w.d, dtype=torch.bfloat16, device="cuda")
+    q = torch.empty(w.batch * w.n_tokens, w.d, dtype=torch.bfloat16, device="cuda")
+    a = torch.empty_like(q)
+    lw = p.weights[0]
+    Wb.whale_project_queries(p.cfg, q.shape[0], p.tokens, lw["g_q"], lw["w_q"], q, p.workspace)
+    Wb.whale_project_kv(p.cfg, T, p.states[0], lw["g_kv"], lw["w_kv"], kv, p.workspace)
+
+    def step():
+        if args.kernel_case == "kv":
+            Wb.whale_project_kv(p.cfg, T, p.states[0], lw["g_kv"], lw["w_kv"], kv, p.workspace)
+        else:
+            Wb.whale_cross_attention(p.cfg, q, kv, p.offsets_t, a, p.hint, p.workspace)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    work = step_work(w, T)["kv_proj" if args.kernel_case == "kv" else "attention"]
+    print(json.dumps({"kernel_case": args.kernel_case, "workload": w.name, "total_L": T, "ms_per_launch": ms,
+                      "tflops": work["flops"] / ms / 1e9, "gbs": work["bytes"] / ms / 1e6}), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="hist15k_d512", choices=list(I.WORKLOADS))
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--ref-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel-case", choices=["kv", "attn"], default=None,
+                    help="profiling aid: run only one step entry point on one layer of the workload")
+    ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (kernel cases)")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.kernel_case:
+        return run_kernel_case(args)
+
+    import torch
+    rank, world, local = dist_setup(args.gpus)
+    from wukong_hstu_cross_b200 import build
+    if rank == 0:
+        build.build()
+    barrier(world)
+    from wukong_hstu_cross_b200 import harness as Hn
+    from wukong_hstu_cross_b200 import whale as Wb
+
+    from wukong_hstu_cross_b200 import dist as D
+    w = D.shard_workload(I.WORKLOADS[args.workload], rank, world)   # this rank's own examples
+    p = Hn.build_problem(w, device="cuda")
+    stream = torch.cuda.current_stream()
+    total_L = p.total_L
+
+    # ---------------- device-resident timed region: the whole stack per step ----------------
+    for _ in range(args.warmup):
+        Hn.run_forward(p, stream)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            Hn.run_forward(p, stream)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    ms = ev0.elapsed_time(ev1) / args.steps
+    ms = max_over_ranks(ms, world)
+    value = world * w.batch / (ms / 1e3)
+
+    # ---------------- per-kernel timing of the two heavy steps (same stream, CUDA events) ------
+    work = step_work(w, total_L)
+    Hn_ws = p.workspace
+    kv = torch.empty(total_L, 2 * w.d, dtype=torch.bfloat16, device="cuda")
+    q = torch.empty(w.batch * w.n_tokens, w.d, dtype=torch.bfloat16, device="cuda")
+    a = torch.empty_like(q)
+    reps = max(args.steps, 3)
+
+    def timed(fn, n):
+        for l in range(min(2, w.n_layers)):
+            fn(l)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        cnt = 0
+        for _ in range(n):
+            for l in range(w.n_layers):
+                fn(l)
+                cnt += 1
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / cnt
+
+    def kv_step(l):
+        Wb.whale_project_kv(p.cfg, total_L, p.states[l], p.weights[l]["g_kv"], p.weights[l]["w_kv"], kv, Hn_ws,
+                            stream=stream)
+
+    def attn_step(l):
+        Wb.whale_cross_attention(p.cfg, q, kv, p.offsets_t, a, p.hint, Hn_ws, stream=stream)
+
+    kv_step(0)
+    Wb.whale_project_queries(p.cfg, q.shape[0], p.tokens, p.weights[0]["g_q"], p.weights[0]["w_q"], q, Hn_ws,
+                             stream=stream)
+    torch.cuda.synchronize()
+    t_kv = timed(kv_step, reps)
+    t_attn = timed(attn_step, reps)
+    peaks, peak_src = load_peaks()
+    kv_tflops = work["kv_proj"]["flops"] / (t_kv * 1e-3) / 1e12
+    attn_gbs = work["attention"]["bytes"] / (t_attn * 1e-3) / 1e9
+    layer_ms = ms / w.n_layers
+    share_kv, share_attn = t_kv / layer_ms, t_attn / layer_ms
+    if share_kv >= share_attn:
+        roof = {"kernel": "K|V projection GEMM (tcgen05, RMSNorm row factor fused)", "bound": "tensor",
+                "achieved": kv_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": kv_tflops / peaks["bf16_tflops"], "traffic": None,
+                "algorithmic_per_launch": work["kv_proj"]["flops"], "avg_launch_ms": t_kv,
+                "peak_source": f"{peak_src} bf16 burst"}
+    else:
+        roof = {"kernel": "split-L cross-attention + combine", "bound": "hbm", "achieved": attn_gbs,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": attn_gbs / peaks["hbm_gbs"], "traffic": None,
+                "algorithmic_per_launch": work["attention"]["bytes"], "avg_launch_ms": t_attn,
+                "peak_source": f"{peak_src} HBM copy"}
+    # roofline of the whole step: sum over kernels of max(flops / TC peak, bytes / HBM peak)
+    t_star = 0.0
+    for k, v in work.items():
+        t_star += max(v["flops"] / (peaks["bf16_tflops"] * 1e12), v["bytes"] / (peaks["hbm_gbs"] * 1e9))
+    t_star *= w.n_layers * 1e3
+
+    # ---------------- end to end: host buffers through the C ABI, copies inside the timed region -----
+    e2e = None
+    if args.e2e_steps > 0:
+        hs = p.states.cpu().pin_memory()
+        ht = p.tokens.cpu().pin_memory()
+        ho = torch.empty_like(ht).pin_memory()
+        hoff = torch.from_numpy(p.offsets).pin_memory()
+        hws = torch.empty(Wb.whale_host_workspace_size(p.cfg, p.hint), dtype=torch.uint8, device="cuda")
+        del p.workspace
+        Wb.whale_fusion_forward_host(p.cfg, ht, hs, hoff, p.weights, ho, p.hint, hws, stream=stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            Wb.whale_fusion_forward_host(p.cfg, ht, hs, hoff, p.weights, ho, p.hint, hws, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world)
+        h2d = hs.numel() * hs.element_size() + ht.numel() * ht.element_size() + hoff.numel() * 4
+        d2h = ho.numel() * ho.element_size()
+        e2e = {"value": world * w.batch / (e_ms / 1e3), "unit": "examples/s", "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_sample(w, budget_s=args.ref_budget)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "examples/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) states and tokens, Xavier weights)",
+            "config": {"workload": w.name, "batch": w.batch, "n_tokens": w.n_tokens, "d": w.d, "heads": w.n_heads,
+                       "layers": w.n_layers, "total_L": total_L, "max_L": int(p.lengths.max()),
+                       "parallelism": f"dp{world} (independent examples per rank, no collective)",
+                       "l2": "inputs larger than L2 (each layer reads its own "
+                             f"{total_L * w.d * 2 / 1e6:.0f} MB state slab), no flush"},
+            "roofline": roof,
+            "step_roofline": {"t_star_ms": t_star, "frac": t_star / ms, "per_layer_ms": layer_ms,
+                              "kv_proj_ms": t_kv, "attention_ms": t_attn,
+                              "peaks": f"{peak_src}: {peaks['hbm_gbs']} GB/s, {peaks['bf16_tflops']} TFLOP/s"},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step(w) * args.steps,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

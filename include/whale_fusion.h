@@ -1,0 +1,185 @@
+/*
+ * whale_fusion.h — C ABI of the B200 (sm_100a) WHALE attention-fusion forward.
+ *
+ * What is computed. WHALE stacks layers; in each, a fusion module lets the Wukong
+ * branch's interaction tokens query the HSTU branch's per-position behavior states
+ * (gist.science technical summary of WHALE, section 2.1 "Core Architecture",
+ * Attention-Based Fusion Module; pith.science verdict, "key_machinery"):
+ *
+ *   Q    = RMSNorm(H_w; g_q)  W_Q^T                     queries from Wukong tokens
+ *   K|V  = RMSNorm(H_s; g_kv) [W_K ; W_V]^T             keys/values from HSTU states
+ *   A    = per-head softmax(Q K^T / sqrt(d_head)) V      Eq. (4), over the example's own
+ *                                                       jagged history, no mask, no bias
+ *   F    = H_w + W_F2 SiLU(W_F1 [A ; H_w])              Eq. (5), residual Fusion MLP
+ *   H_f  = F + W_down (SiLU(W_gate n) * (W_up n)),      pre-norm SwiGLU FFN, n = RMSNorm(F; g_ffn),
+ *                                                       up|gate run as ONE concatenated GEMM
+ *   H_f feeds the next layer's query side (identity Wukong stand-in); layer l reads its
+ *   own H_s slab (section 2.1 "Propagation").
+ *
+ * Conventions (all entry points):
+ *  - Matrices are row-major. Weights use the nn.Linear layout [out, in].
+ *  - "device" pointers are CUDA global memory on the current device; "host" pointers
+ *    are ordinary (preferably pinned) host memory. The caller owns every buffer and
+ *    the stream. No entry point allocates device memory: scratch lives in the
+ *    caller's workspace (size from whale_workspace_size).
+ *  - Element type of tokens, states, weights and outputs is cfg->dtype (bf16 or fp32).
+ *    Gains g_* are always fp32 [d]. Offsets are int32.
+ *  - All GPU work is enqueued on `stream` and is asynchronous; return codes report
+ *    host-detectable errors only (bad arguments, unsupported shapes, launch errors).
+ *    Nothing inside a forward synchronises the device or copies device->host: the
+ *    shape hint carries the sizes the host needs (the pages' "shape hint tensors",
+ *    gist.science section 2.2, Inference Optimizations).
+ *  - Offsets must satisfy offsets[0] = 0, offsets[b] <= offsets[b+1],
+ *    offsets[B] <= hint->total_L and offsets[b+1]-offsets[b] <= hint->max_L. Kernels
+ *    clamp every history row index to [0, total_L), so a violation never reads out of
+ *    bounds, but it gives wrong results; with WHALE_DEBUG the forward also checks the
+ *    offsets on the device and records WHALE_DEVERR_OFFSETS, read by
+ *    whale_get_device_error.
+ *  - Device-side waits are bounded; a wait that runs out records WHALE_DEVERR_TIMEOUT
+ *    and the kernel returns.
+ */
+#ifndef WHALE_FUSION_H_
+#define WHALE_FUSION_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* whale_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  WHALE_OK = 0,
+  WHALE_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, inconsistent config */
+  WHALE_ERR_UNSUPPORTED = 2,   /* valid but not implemented shape (see whale_config) */
+  WHALE_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed (launch, encode) */
+  WHALE_ERR_WORKSPACE = 4,     /* workspace null or smaller than whale_workspace_size */
+  WHALE_ERR_DEVICE_CHECK = 5   /* whale_get_device_error found a recorded device error */
+} whale_status;
+
+typedef enum { WHALE_FP32 = 0, WHALE_BF16 = 1 } whale_dtype;
+
+/* cfg->flags */
+#define WHALE_SHARED_KV 1u  /* K = V: w_kv is W_K alone [d, d] (gist.science 2.2 "Shared Key-Value") */
+#define WHALE_TIED_GATE 2u  /* W_gate = W_up: w_upgate is W_up alone [H, d] (gist.science 2.2 "Shared-Gate SwiGLU") */
+#define WHALE_DEBUG 4u      /* validate offsets on the device before the forward */
+
+/* device error bits (whale_get_device_error) */
+#define WHALE_DEVERR_TIMEOUT 1
+#define WHALE_DEVERR_OFFSETS 2
+
+typedef struct {
+  int n_layers;       /* stacked fusion layers (>= 1) */
+  int d;              /* width of tokens and states */
+  int n_heads;        /* attention heads; d_head = d / n_heads */
+  int n_tokens;       /* N: Wukong tokens (queries) per example */
+  int ffn_hidden;     /* SwiGLU hidden width H (4d in the pages' setting) */
+  int fusion_hidden;  /* Fusion MLP hidden width (2d); 0 = one linear map W_F [d, 2d] */
+  int dtype;          /* whale_dtype */
+  unsigned flags;     /* WHALE_SHARED_KV | WHALE_TIED_GATE | WHALE_DEBUG */
+  float eps;          /* RMSNorm epsilon */
+} whale_config;
+/* Supported: fp32 — any d with d % n_heads == 0, d_head <= 128 (SIMT correctness path).
+ *            bf16 — d % 64 == 0, d_head in {32, 64}, n_heads / (heads per CTA) integral
+ *            (heads per CTA = min(n_heads, 8), its d_head multiple of 64 columns),
+ *            ffn_hidden % 64 == 0, fusion_hidden % 64 == 0. Any n_tokens >= 1. */
+
+/* Per-layer weights: device pointers. Element type cfg->dtype, gains fp32. */
+typedef struct {
+  const float* g_q;      /* [d]   RMSNorm gain before W_Q */
+  const float* g_kv;     /* [d]   RMSNorm gain before W_K, W_V */
+  const void* w_q;       /* [d, d] */
+  const void* w_kv;      /* [2d, d] = [W_K ; W_V]   ([d, d] with WHALE_SHARED_KV) */
+  const void* w_f1;      /* [fusion_hidden, 2d], columns 0..d-1 read A, d..2d-1 read H_w (unused if fusion_hidden 0) */
+  const void* w_f2;      /* [d, fusion_hidden]      ([d, 2d] = W_F if fusion_hidden 0) */
+  const float* g_ffn;    /* [d]   RMSNorm gain before the SwiGLU FFN */
+  const void* w_upgate;  /* [2H, d] = [W_up ; W_gate] ([H, d] with WHALE_TIED_GATE) */
+  const void* w_down;    /* [d, H] */
+} whale_layer_weights;
+
+/* Host-side sizes, so no device->host read is needed to launch.
+ * B: examples; max_L: an upper bound of every history length; total_L: rows of each
+ * H_s slab (>= offsets[B]). */
+typedef struct {
+  int B;
+  int max_L;
+  long long total_L;
+} whale_shape_hint;
+
+/* Human-readable name of a status code (static string). */
+const char* whale_status_string(whale_status s);
+
+/* Bytes of device workspace needed by every entry point below for this config and
+ * shape (0 if cfg/hint are invalid or unsupported). */
+size_t whale_workspace_size(const whale_config* cfg, const whale_shape_hint* hint);
+
+/* Whole stack (all n_layers) on device buffers.
+ *   wukong_tokens  device [B, N, d]            H_w of layer 0
+ *   seq_states     device [n_layers, total_L, d]  H_s slab of each layer
+ *   seq_offsets    device int32 [B+1]
+ *   weights        HOST array of n_layers whale_layer_weights (device pointers inside)
+ *   out            device [B, N, d]            H_f of the last layer; must not alias inputs
+ *   workspace      device, >= whale_workspace_size bytes, 256-byte aligned */
+whale_status whale_fusion_forward(const whale_config* cfg, const void* wukong_tokens, const void* seq_states,
+                                  const int* seq_offsets, const whale_layer_weights* weights, void* out,
+                                  const whale_shape_hint* hint, void* workspace, size_t workspace_bytes,
+                                  whale_stream_t stream);
+
+/* Same computation from HOST buffers: copies each layer's inputs host->device inside the
+ * call (overlapped with the previous layer's compute) and the result device->host.
+ * host_tokens [B,N,d], host_seq_states [n_layers,total_L,d], host_offsets int32 [B+1],
+ * host_out [B,N,d] are host pointers (pin them for asynchronous copies); weights as above.
+ * The workspace must hold whale_host_workspace_size bytes. Returns after enqueueing;
+ * synchronise `stream` before reading host_out. */
+size_t whale_host_workspace_size(const whale_config* cfg, const whale_shape_hint* hint);
+whale_status whale_fusion_forward_host(const whale_config* cfg, const void* host_tokens,
+                                       const void* host_seq_states, const int* host_offsets,
+                                       const whale_layer_weights* weights, void* host_out,
+                                       const whale_shape_hint* hint, void* workspace, size_t workspace_bytes,
+                                       whale_stream_t stream);
+
+/* One layer: tokens_in/out device [B, N, d], layer_states device [total_L, d]. */
+whale_status whale_fusion_layer_forward(const whale_config* cfg, const void* tokens_in, const void* layer_states,
+                                        const int* seq_offsets, const whale_layer_weights* layer_weights,
+                                        void* tokens_out, const whale_shape_hint* hint, void* workspace,
+                                        size_t workspace_bytes, whale_stream_t stream);
+
+/* ---- single steps of one layer (for step-level tests and composition) ---------------- */
+
+/* Q = RMSNorm(x; g_q) W_Q^T.  x, q: device [rows, d]. */
+whale_status whale_project_queries(const whale_config* cfg, long long rows, const void* x, const float* g_q,
+                                   const void* w_q, void* q, void* workspace, size_t workspace_bytes,
+                                   whale_stream_t stream);
+
+/* K|V = RMSNorm(s; g_kv) [W_K ; W_V]^T.  s: device [rows, d]; kv: device [rows, 2d]
+ * (K in columns 0..d-1, V in d..2d-1; [rows, d] = K with WHALE_SHARED_KV). */
+whale_status whale_project_kv(const whale_config* cfg, long long rows, const void* s, const float* g_kv,
+                              const void* w_kv, void* kv, void* workspace, size_t workspace_bytes,
+                              whale_stream_t stream);
+
+/* Eq. (4): q device [B*N, d] (row b*N+n), kv device [total_L, 2d] (or [total_L, d] shared),
+ * offsets device int32 [B+1] -> a device [B*N, d]. Empty histories give a = 0. */
+whale_status whale_cross_attention(const whale_config* cfg, const void* q, const void* kv, const int* seq_offsets,
+                                   void* a, const whale_shape_hint* hint, void* workspace, size_t workspace_bytes,
+                                   whale_stream_t stream);
+
+/* Eq. (5): f = x + W_F2 SiLU(W_F1 [a ; x]) (or x + W_F [a ; x]).  a, x, f: device [rows, d]. */
+whale_status whale_fusion_mlp(const whale_config* cfg, long long rows, const void* a, const void* x,
+                              const void* w_f1, const void* w_f2, void* f, void* workspace, size_t workspace_bytes,
+                              whale_stream_t stream);
+
+/* y = f + W_down (SiLU(W_gate n) * W_up n), n = RMSNorm(f; g_ffn).  f, y: device [rows, d]. */
+whale_status whale_swiglu_ffn(const whale_config* cfg, long long rows, const void* f, const float* g_ffn,
+                              const void* w_upgate, const void* w_down, void* y, void* workspace,
+                              size_t workspace_bytes, whale_stream_t stream);
+
+/* Synchronises `stream`, then reads and clears the device error word of the current
+ * device (bits WHALE_DEVERR_*). Returns WHALE_ERR_DEVICE_CHECK if any bit was set. */
+whale_status whale_get_device_error(whale_stream_t stream, int* code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WHALE_FUSION_H_ */

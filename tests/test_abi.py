@@ -1,0 +1,93 @@
+"""The C-ABI library loads, exports every function include/whale_fusion.h declares, and its
+host-side checks return the documented status codes. No GPU work: every call below
+returns before any CUDA call is made."""
+import ctypes
+
+import pytest
+
+from wukong_hstu_cross_b200 import build
+
+build.build()
+from wukong_hstu_cross_b200 import whale as W  # noqa: E402
+from wukong_hstu_cross_b200 import inputs as I  # noqa: E402
+from wukong_hstu_cross_b200 import harness as Hn  # noqa: E402
+
+EXPECTED = {
+    "whale_status_string", "whale_workspace_size", "whale_fusion_forward", "whale_host_workspace_size",
+    "whale_fusion_forward_host", "whale_fusion_layer_forward", "whale_project_queries", "whale_project_kv",
+    "whale_cross_attention", "whale_fusion_mlp", "whale_swiglu_ffn", "whale_get_device_error",
+}
+
+
+def test_library_exports_every_declared_symbol():
+    declared = set(W.header_functions())
+    assert EXPECTED <= declared, EXPECTED - declared
+    lib = ctypes.CDLL(W.LIB_PATH)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_status_strings():
+    for code in range(6):
+        assert W.whale_status_string(code) and W.whale_status_string(code) != "unknown status"
+    assert W.whale_status_string(99) == "unknown status"
+
+
+def _cfg(name, **kw):
+    w = I.WORKLOADS[name].replace(**kw) if kw else I.WORKLOADS[name]
+    return w, Hn.config_of(w)
+
+
+def test_workspace_size_scales_and_rejects_invalid():
+    w, cfg = _cfg("stack_d256")
+    small = W.whale_workspace_size(cfg, W.make_hint(4, 100, 400))
+    large = W.whale_workspace_size(cfg, W.make_hint(128, 6000, 576000))
+    assert 0 < small < large
+    # K|V buffer alone (total_L x 2d bf16) must fit
+    assert large > 576000 * 2 * w.d * 2
+    bad = Hn.config_of(w.replace(n_heads=3))           # d % heads != 0
+    assert W.whale_workspace_size(bad, W.make_hint(4, 100, 400)) == 0
+    unsup = Hn.config_of(w.replace(d=96, n_heads=3))   # bf16 needs d % 64 == 0
+    assert W.whale_workspace_size(unsup, W.make_hint(4, 100, 400)) == 0
+    assert W.whale_workspace_size(cfg, W.make_hint(-1, 100, 400)) == 0
+
+
+def test_host_side_errors_are_reported_without_gpu_work():
+    w, cfg = _cfg("stack_d128")
+    hint = W.make_hint(2, 10, 20)
+    ws = W.whale_workspace_size(cfg, hint)
+    fake = 1 << 20  # never dereferenced: every call below fails validation first
+    wts = [dict.fromkeys(["g_q", "g_kv", "w_q", "w_kv", "w_f1", "w_f2", "g_ffn", "w_upgate", "w_down"], fake)] * 4
+    # null tokens
+    assert W.whale_fusion_forward(cfg, None, fake, fake, wts, fake, hint, fake, ws, stream=0, raw=True) == 1
+    # workspace too small / null
+    assert W.whale_fusion_forward(cfg, fake, fake, fake, wts, fake, hint, fake, ws - 1, stream=0, raw=True) == 4
+    assert W.whale_fusion_forward(cfg, fake, fake, fake, wts, fake, hint, None, ws, stream=0, raw=True) == 4
+    # missing weight pointer
+    wts2 = [dict(wts[0], w_down=None)] + wts[1:]
+    assert W.whale_fusion_forward(cfg, fake, fake, fake, wts2, fake, hint, fake, ws, stream=0, raw=True) == 1
+    # invalid config / unsupported shape
+    bad = Hn.config_of(w.replace(n_heads=3))
+    assert W.whale_fusion_forward(bad, fake, fake, fake, wts, fake, hint, fake, ws, stream=0, raw=True) == 1
+    unsup = Hn.config_of(w.replace(d=128, n_heads=1))   # d_head 128 not in the bf16 path
+    assert W.whale_fusion_forward(unsup, fake, fake, fake, wts, fake, hint, fake, ws, stream=0, raw=True) == 2
+    # bad hint
+    assert W.whale_fusion_forward(cfg, fake, fake, fake, wts, fake, W.make_hint(2, 10, -5), fake, ws, stream=0,
+                                  raw=True) == 1
+    # misaligned tokens pointer
+    assert W.whale_fusion_forward(cfg, fake + 2, fake, fake, wts, fake, hint, fake, ws, stream=0, raw=True) == 1
+    # step entry points
+    assert W.whale_project_kv(cfg, 10, None, fake, fake, fake, fake, 1 << 20, stream=0, raw=True) == 1
+    assert W.whale_project_kv(cfg, 10, fake, fake, fake, fake, fake, 16, stream=0, raw=True) == 4
+    assert W.whale_cross_attention(cfg, fake, fake, None, fake, hint, fake, 1 << 30, stream=0, raw=True) == 1
+    assert W.whale_swiglu_ffn(cfg, 10, fake, fake, fake, fake, fake, None, 0, stream=0, raw=True) == 4
+
+
+def test_empty_batch_is_a_no_op():
+    w, cfg = _cfg("stack_d128")
+    hint = W.make_hint(0, 0, 0)
+    ws = W.whale_workspace_size(cfg, hint)
+    assert ws > 0
+    fake = 1 << 20
+    wts = [dict.fromkeys(["g_q", "g_kv", "w_q", "w_kv", "w_f1", "w_f2", "g_ffn", "w_upgate", "w_down"], fake)] * 4
+    assert W.whale_fusion_forward(cfg, fake, fake, fake, wts, fake, hint, fake, ws, stream=0, raw=True) == 0

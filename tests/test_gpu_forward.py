@@ -1,0 +1,160 @@
+"""Whole-layer and whole-stack parity of the CUDA path against the fp64 oracle through
+whale_fusion_forward / whale_fusion_layer_forward / whale_fusion_forward_host: every example
+of reduced copies of the workloads (ragged lengths, an empty history, every variant flag),
+then the full-size workloads in the benchmark's launch configuration, checked on sampled
+examples and tokens the oracle recomputes one by one (tokens of an example are independent
+given its history). Also batch-reordering invariance and the debug offset check."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import whale_oracle as O
+from tests.gpu_util import assert_parity
+from wukong_hstu_cross_b200 import inputs as I
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    from wukong_hstu_cross_b200 import build
+    build.build()
+    from wukong_hstu_cross_b200 import harness as Hn
+    from wukong_hstu_cross_b200 import whale as W
+
+
+def _oracle_all(p, examples=None, token_idx=None):
+    w = p.w
+    flags = p.flags
+    res = {}
+    for b in (range(w.batch) if examples is None else examples):
+        x = I.tokens_of_example(w, b)
+        if token_idx is not None:
+            x = x[token_idx]
+        res[b] = O.fusion_stack_example(x, Hn.states_of_example_host(p, b), p.host_weights, w.n_heads, w.eps, **flags)
+    return res
+
+
+def _check(p, out, examples=None, token_idx=None, rms_rel=2e-2):
+    ref = _oracle_all(p, examples, token_idx)
+    o = out.float().cpu().numpy()
+    for b, r in ref.items():
+        g = o[b] if token_idx is None else o[b][token_idx]
+        assert_parity(g, r, p.w.dtype, rms_rel=rms_rel if p.w.dtype == "bf16" else None, what=f"example {b}")
+
+
+REDUCED = {
+    "tiny_fp32": dict(),
+    "tiny_as_bf16": dict(dtype="bf16"),
+    "stack_d128": dict(batch=6, lengths=("uniform", 1, 700)),
+    "stack_d256": dict(batch=4, lengths=("uniform", 100, 1500)),
+    "hist15k_d512": dict(batch=3, n_layers=2, lengths=("lognormal", 1500.0, 0.5, 64, 3000)),
+    "serve_15k": dict(n_tokens=16 * 64, n_layers=2, lengths=("fixed", 3000)),
+}
+
+
+@pytest.mark.parametrize("name", list(REDUCED))
+def test_stack_reduced_workloads(name):
+    base = "tiny_fp32" if name.startswith("tiny") else name
+    w = I.WORKLOADS[base].replace(**REDUCED[name])
+    L = I.draw_lengths(w)
+    if name == "stack_d128":
+        L[2] = 0  # an empty history inside the batch
+    p = Hn.build_problem(w, gains="random", lengths=L)
+    out = Hn.run_forward(p)
+    torch.cuda.synchronize()
+    if name == "serve_15k":
+        idx = np.random.default_rng(0).choice(w.n_tokens, 64, replace=False)
+        _check(p, out, token_idx=idx)
+    else:
+        _check(p, out)
+
+
+@pytest.mark.parametrize("shared_kv,tied_gate,fusion_mult", [(True, False, 2), (False, True, 2), (True, True, 0),
+                                                              (False, False, 0)])
+def test_variants(shared_kv, tied_gate, fusion_mult):
+    w = I.WORKLOADS["stack_d256"].replace(batch=3, n_layers=2, lengths=("uniform", 1, 900), fusion_mult=fusion_mult)
+    p = Hn.build_problem(w, gains="random", shared_kv=shared_kv, tied_gate=tied_gate)
+    out = Hn.run_forward(p)
+    torch.cuda.synchronize()
+    _check(p, out)
+
+
+def test_fp32_variants():
+    w = I.WORKLOADS["tiny_fp32"].replace(batch=3, n_layers=2, fusion_mult=0)
+    p = Hn.build_problem(w, gains="random", shared_kv=True, tied_gate=True)
+    out = Hn.run_forward(p)
+    torch.cuda.synchronize()
+    _check(p, out)
+
+
+def test_layer_entry_point_and_batch_reordering():
+    w = I.WORKLOADS["stack_d128"].replace(batch=5, n_layers=1, lengths=("uniform", 1, 800))
+    p = Hn.build_problem(w, gains="random")
+    y = torch.empty_like(p.tokens)
+    W.whale_fusion_layer_forward(p.cfg, p.tokens, p.states[0], p.offsets_t, p.weights[0], y, p.hint, p.workspace)
+    out = Hn.run_forward(p)
+    torch.cuda.synchronize()
+    assert torch.equal(y, out)
+    _check(p, y)
+    # reorder the examples (same total and max length): each example's output follows it exactly
+    perm = np.array([3, 0, 4, 2, 1])
+    L2 = p.lengths[perm]
+    off2 = I.offsets_of(L2)
+    rows = [p.states[0, p.offsets[b]:p.offsets[b + 1]] for b in perm]
+    states2 = torch.cat(rows).unsqueeze(0).contiguous()
+    tok2 = p.tokens[torch.from_numpy(perm).cuda()].contiguous()
+    y2 = torch.empty_like(tok2)
+    W.whale_fusion_forward(p.cfg, tok2, states2, torch.from_numpy(off2).cuda(), p.weights, y2, p.hint, p.workspace)
+    torch.cuda.synchronize()
+    assert torch.equal(y2, out[torch.from_numpy(perm).cuda()])
+
+
+def test_host_buffer_entry_point_matches_device_entry_point():
+    w = I.WORKLOADS["stack_d256"].replace(batch=4, n_layers=3, lengths=("uniform", 10, 1200))
+    p = Hn.build_problem(w, gains="random")
+    out = Hn.run_forward(p).clone()
+    hs = p.states.cpu().pin_memory()
+    ht = p.tokens.cpu().pin_memory()
+    ho = torch.empty_like(ht).pin_memory()
+    hoff = torch.from_numpy(p.offsets).pin_memory()
+    ws = torch.empty(W.whale_host_workspace_size(p.cfg, p.hint), dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        ho.zero_()
+        W.whale_fusion_forward_host(p.cfg, ht, hs, hoff, p.weights, ho, p.hint, ws)
+        torch.cuda.synchronize()
+        assert torch.equal(ho, out.cpu())
+
+
+def test_debug_mode_flags_bad_offsets():
+    w = I.WORKLOADS["stack_d128"].replace(batch=3, n_layers=1, lengths=("uniform", 10, 50))
+    p = Hn.build_problem(w, debug=True)
+    Hn.run_forward(p)
+    assert W.whale_get_device_error() == 0
+    bad = torch.tensor([0, 40, 20, int(p.offsets[-1])], dtype=torch.int32, device="cuda")  # decreasing: invalid
+    W.whale_fusion_forward(p.cfg, p.tokens, p.states, bad, p.weights, p.out, p.hint, p.workspace)
+    assert W.whale_get_device_error() & W.WHALE_DEVERR_OFFSETS
+    assert W.whale_get_device_error() == 0  # cleared by the read
+
+
+# ------------------------------------------------------------------------------------------
+# full-size workloads, as the benchmark launches them; sampled outputs
+# ------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("name", ["stack_d128", "stack_d256", "hist15k_d512", "serve_15k"])
+def test_full_size_sampled(name):
+    w = I.WORKLOADS[name]
+    p = Hn.build_problem(w)
+    out = Hn.run_forward(p)
+    torch.cuda.synchronize()
+    if name == "serve_15k":
+        idx = np.random.default_rng(1).choice(w.n_tokens, 48, replace=False)
+        _check(p, out, examples=[0], token_idx=idx)
+    else:
+        L = p.lengths
+        ex = sorted({int(np.argmax(L)), int(np.argmin(L)), 0, w.batch - 1})
+        _check(p, out, examples=ex, token_idx=np.arange(min(w.n_tokens, 8)))
+    assert torch.isfinite(out.float()).all()
+    # determinism: a second run gives bitwise the same output
+    out2 = Hn.run_forward(p).clone()
+    torch.cuda.synchronize()
+    out3 = Hn.run_forward(p)
+    torch.cuda.synchronize()
+    assert torch.equal(out2, out3)

@@ -1,0 +1,291 @@
+// gemm_tc.cuh — bf16 GEMM on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+//   out[M, N'] = epilogue( sum_k A[m, k] * W[n, k] ),  A = [A0 | A1] (two K sources),
+//   W row-major [N, K0 + K1] (nn.Linear layout), fp32 accumulation in tensor memory.
+//
+// Operand precision. With SPLIT, each A source is given as a pair of bf16 tensors (hi, lo)
+// with A = hi + lo (about 16 mantissa bits), and every k-step issues two MMAs, hi*W and lo*W,
+// into the same accumulator. The weights are bf16 values, so the product is then as precise
+// as an fp32 activation times the weight. The token-side (residual-stream) GEMMs use this;
+// the history-side K|V projection reads bf16 states directly.
+//
+// One CTA computes one 128 x BN tile. Warp roles (192 threads):
+//   warp 0      TMA producer: A (hi, lo) and W tiles (64 columns = 128 B, 128-byte swizzle)
+//               into a STAGES-deep ring of shared-memory stages, completion on `full[s]`.
+//   warp 1      allocates BN TMEM columns; one thread issues tcgen05.mma (M=128, N=BN,
+//               K=16 per instruction) and commits each stage back to `empty[s]`.
+//   warps 2..5  epilogue: thread i of the warp with quadrant q = warp % 4 owns output row
+//               32q + i (= TMEM lane). With ROWNORM they also read their row of every A stage
+//               from shared memory while the MMAs run and accumulate sum(x^2), so RMSNorm's
+//               row factor r = 1/sqrt(mean(x^2) + eps) costs no extra pass over A:
+//               RMSNorm(x; g) W^T = r * (x (W diag(g))^T), with diag(g) folded into W beforehand.
+// Epilogue value per element (fp32): STORE r*acc; SILU silu(acc); RESID acc + resid32;
+// SWIGLU (W rows packed in blocks of 32 = 16 up rows then the 16 matching gate rows)
+// silu(r*gate) * r*up; SWIGLU_TIED (W_gate = W_up) silu(r*u) * r*u. It is then written to
+// any of: out32 (fp32), out_hi (bf16 rounding), out_lo (bf16 of the rounding residue).
+#pragma once
+
+#include "ptx.cuh"
+
+namespace whale {
+
+enum GemmEpi : int { EPI_STORE = 0, EPI_SILU = 1, EPI_RESID = 2, EPI_SWIGLU = 3, EPI_SWIGLU_TIED = 4 };
+
+struct GemmArgs {
+  int M;                       // rows of A and of the output
+  int N;                       // accumulator columns (rows of W), multiple of 32
+  int kb0;                     // 64-column K blocks taken from A0
+  int kb1;                     // 64-column K blocks taken from A1 (0: single source)
+  int tiles_n;                 // N / BN
+  float inv_k;                 // 1 / (K of the normalised source), ROWNORM only
+  float eps;                   // RMSNorm epsilon, ROWNORM only
+  __nv_bfloat16* out_hi;       // bf16 output (may be null)
+  __nv_bfloat16* out_lo;       // bf16 residue of out_hi (may be null)
+  float* out32;                // fp32 output (may be null)
+  long long ldo;               // output row stride (elements), shared by the three outputs
+  const float* resid32;        // EPI_RESID: fp32 residual [M, N]
+  long long ldr;
+};
+
+constexpr int kGemmThreads = 192;
+
+template <int BN, bool SPLIT>
+struct GemmSmem {
+  static constexpr int BM = 128, BK = 64;
+  static constexpr uint32_t A_BYTES = BM * BK * 2;
+  static constexpr uint32_t A_ALL = SPLIT ? 2 * A_BYTES : A_BYTES;
+  static constexpr uint32_t B_BYTES = BN * BK * 2;
+  static constexpr uint32_t STAGE_BYTES = A_ALL + B_BYTES;
+  static constexpr int STAGES = (196608 / STAGE_BYTES) > 8 ? 8 : (196608 / STAGE_BYTES);
+  static constexpr size_t BYTES = 1024 /*alignment slack*/ + STAGES * (size_t)STAGE_BYTES + 256 /*barriers*/;
+};
+
+__device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* f) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 t = __bfloat1622float2(h[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+
+// Write NV consecutive fp32 values (NV multiple of 8) of one row to the requested outputs.
+template <int NV>
+__device__ __forceinline__ void store_row_chunk(const GemmArgs& g, long long off, const float* x) {
+  if (g.out32) {
+    float4* d = reinterpret_cast<float4*>(g.out32 + off);
+#pragma unroll
+    for (int i = 0; i < NV / 4; ++i) d[i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+  }
+  if (g.out_hi) {
+    uint32_t hi[NV / 2], lo[NV / 2];
+#pragma unroll
+    for (int j = 0; j < NV / 2; ++j) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * j], x[2 * j + 1]);
+      hi[j] = *reinterpret_cast<const uint32_t*>(&h);
+      const float2 hf = __bfloat1622float2(h);
+      lo[j] = pack_bf16x2(x[2 * j] - hf.x, x[2 * j + 1] - hf.y);
+    }
+    uint4* dh = reinterpret_cast<uint4*>(g.out_hi + off);
+#pragma unroll
+    for (int i = 0; i < NV / 8; ++i) dh[i] = make_uint4(hi[4 * i], hi[4 * i + 1], hi[4 * i + 2], hi[4 * i + 3]);
+    if (g.out_lo) {
+      uint4* dl = reinterpret_cast<uint4*>(g.out_lo + off);
+#pragma unroll
+      for (int i = 0; i < NV / 8; ++i) dl[i] = make_uint4(lo[4 * i], lo[4 * i + 1], lo[4 * i + 2], lo[4 * i + 3]);
+    }
+  }
+}
+
+template <int BN, int EPI, bool ROWNORM, bool SPLIT>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA0lo,
+                   const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmA1lo,
+                   const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
+  using L = GemmSmem<BN, SPLIT>;
+  constexpr int STAGES = L::STAGES;
+  constexpr uint32_t TMEM_COLS = BN;  // 64, 128 or 256: a power of two >= 32
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // stage s: [A hi | A lo (SPLIT) | W]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * L::STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* accf = empty + STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile_n = blockIdx.x % args.tiles_n;
+  const int tile_m = blockIdx.x / args.tiles_n;
+  const int m0 = tile_m * L::BM, n0 = tile_n * BN;
+  const int KB = args.kb0 + args.kb1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1 + (ROWNORM ? 4 : 0));
+    }
+    mbar_init(accf, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA0);
+    tma_prefetch_desc(&tmB);
+    if (SPLIT) tma_prefetch_desc(&tmA0lo);
+    if (args.kb1 > 0) {
+      tma_prefetch_desc(&tmA1);
+      if (SPLIT) tma_prefetch_desc(&tmA1lo);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int issued = 0;
+      for (int kb = 0; kb < KB; ++kb) {
+        const int s = kb % STAGES, u = kb / STAGES;
+        if (kb >= STAGES && !mbar_wait(&empty[s], (u - 1) & 1, abort_flag)) break;
+        uint8_t* st = smem + s * L::STAGE_BYTES;
+        mbar_arrive_expect_tx(&full[s], L::STAGE_BYTES);
+        const bool first = kb < args.kb0;
+        const int kc = (first ? kb : kb - args.kb0) * L::BK;
+        tma_load_2d(st, first ? &tmA0 : &tmA1, kc, m0, &full[s]);
+        if (SPLIT) tma_load_2d(st + L::A_BYTES, first ? &tmA0lo : &tmA1lo, kc, m0, &full[s]);
+        tma_load_2d(st + L::A_ALL, &tmB, kb * L::BK, n0, &full[s]);
+        issued = kb + 1;
+      }
+      if (*abort_flag) {
+        // Unwinding after a timeout: let the copies this thread started land before the CTA exits.
+        volatile int quiet = 0;
+        for (int kb = (issued > STAGES ? issued - STAGES : 0); kb < issued; ++kb)
+          mbar_wait(&full[kb % STAGES], (kb / STAGES) & 1, &quiet);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
+      for (int kb = 0; kb < KB; ++kb) {
+        const int s = kb % STAGES, u = kb / STAGES;
+        if (!mbar_wait(&full[s], u & 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(smem + s * L::STAGE_BYTES);
+        const uint32_t b_base = a_base + L::A_ALL;
+#pragma unroll
+        for (int kk = 0; kk < L::BK / 16; ++kk) {
+          const uint64_t bdesc = sdesc_k_sw128(b_base + kk * 32);
+          umma_f16(tmem_base, sdesc_k_sw128(a_base + kk * 32), bdesc, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          if (SPLIT) umma_f16(tmem_base, sdesc_k_sw128(a_base + L::A_BYTES + kk * 32), bdesc, idesc, 1u);
+        }
+        umma_commit(&empty[s]);
+      }
+      umma_commit(accf);  // also on abort: arrives once all issued MMAs are done
+    }
+  } else {
+    // ---------------- row statistics + epilogue (warps 2..5) ----------------
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    float ss = 0.f;
+    if (ROWNORM) {
+      for (int kb = 0; kb < KB; ++kb) {
+        const int s = kb % STAGES, u = kb / STAGES;
+        if (!mbar_wait(&full[s], u & 1, abort_flag)) break;
+        if (kb < args.kb0) {
+          // The row's 128 bytes are contiguous; the 128-byte swizzle stores its logical 16-byte
+          // chunk c at position c ^ (row % 8) (identically in the hi and lo tiles). Summing in
+          // logical order keeps the row factor independent of the row's position in the tile.
+          const uint8_t* st = smem + s * L::STAGE_BYTES + row * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const int pc = c ^ (row & 7);
+            float f[8];
+            bf16x8_to_f32(reinterpret_cast<const uint4*>(st)[pc], f);
+            if (SPLIT) {
+              float fl[8];
+              bf16x8_to_f32(reinterpret_cast<const uint4*>(st + L::A_BYTES)[pc], fl);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) f[j] += fl[j];
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) ss = fmaf(f[j], f[j], ss);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+      }
+    }
+    const bool ok = mbar_wait(accf, 0, abort_flag);
+    tc_fence_after();
+    const float r = ROWNORM ? rsqrtf(ss * args.inv_k + args.eps) : 1.0f;
+    const long long gm = (long long)m0 + row;
+    const bool row_ok = ok && gm < args.M;
+    const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16);
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(t_row + c * 32, v);
+      tmem_ld_wait();
+      const int col = n0 + c * 32;
+      if (!row_ok || col >= args.N) continue;
+      float x[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(v[j]) * r;
+      if (EPI == EPI_SWIGLU) {
+        float h[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) h[j] = silu_f(x[16 + j]) * x[j];
+        store_row_chunk<16>(args, gm * args.ldo + col / 2, h);
+      } else {
+        if (EPI == EPI_RESID) {
+          const float4* rp = reinterpret_cast<const float4*>(args.resid32 + gm * args.ldr + col);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 t = rp[i];
+            x[4 * i] += t.x;
+            x[4 * i + 1] += t.y;
+            x[4 * i + 2] += t.z;
+            x[4 * i + 3] += t.w;
+          }
+        } else if (EPI == EPI_SILU) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) x[j] = silu_f(x[j]);
+        } else if (EPI == EPI_SWIGLU_TIED) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) x[j] = silu_f(x[j]) * x[j];
+        }
+        store_row_chunk<32>(args, gm * args.ldo + col, x);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// Residual-stream tensor from a bf16 input: x32 = x, lo = 0 (x itself serves as hi).
+__global__ void pair_from_bf16_kernel(const __nv_bfloat16* __restrict__ x, float* __restrict__ x32,
+                                      __nv_bfloat16* __restrict__ lo, long long n) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    if (x32) x32[i] = __bfloat162float(x[i]);
+    if (lo) lo[i] = __float2bfloat16_rn(0.f);
+  }
+}
+
+}  // namespace whale

@@ -1,0 +1,968 @@
+// whale_fusion.cu — C ABI of the WHALE attention-fusion forward (see include/whale_fusion.h).
+//
+// Host side: argument checks, workspace layout, TMA descriptor encoding and the launch
+// sequence of one layer (all on the caller's stream, no device->host sync):
+//   bf16:  fold gains into W_Q, [W_K;W_V], [W_up;W_gate] (+ SwiGLU packing)
+//          S1 Q   = r(H_w) * H_w W_Q'^T                      tcgen05 GEMM, row-norm epilogue
+//          S2 K|V = r(H_s) * H_s [W_K;W_V]'^T                tcgen05 GEMM, row-norm epilogue
+//          S3 A   = attention (split-L) + log-sum-exp combine
+//          S4 G   = SiLU([A | H_w] W_F1^T),  F = H_w + G W_F2^T   (two-source GEMM, SiLU / residual)
+//          S5 U   = SiLU(gate) * up of r(F) * F W_ug'^T,  H_f = F + U W_down^T
+//   Precision policy (bf16 mode): weights, states, Q, K, V and P are bf16 tensor-core operands;
+//   the residual stream (H_w between layers, F, H_f) is kept in fp32, and every token-side
+//   activation that feeds a GEMM (H_w, A, G, F, U) is carried as a bf16 hi/lo pair whose two
+//   MMAs per k-step give ~16-bit operand precision. Only the final H_f is rounded to bf16.
+//   fp32:  the same steps with SIMT kernels (correctness mode).
+#include "whale_fusion.h"
+
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <functional>
+#include <mutex>
+
+#include "aux_kernels.cuh"
+#include "attention.cuh"
+#include "fp32_path.cuh"
+#include "gemm_persistent.cuh"
+#include "gemm_tc.cuh"
+#include "ptx.cuh"
+
+using namespace whale;
+
+namespace {
+
+#define WCHECK(x)                          \
+  do {                                     \
+    whale_status _s = (x);                 \
+    if (_s != WHALE_OK) return _s;         \
+  } while (0)
+#define CUCHECK(x)                         \
+  do {                                     \
+    cudaError_t _e = (x);                  \
+    if (_e != cudaSuccess) {               \
+      (void)cudaGetLastError();            \
+      return WHALE_ERR_CUDA;               \
+    }                                      \
+  } while (0)
+
+constexpr int kNumSM = 148;
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+template <class T>
+inline T cdiv(T a, T b) { return (a + b - 1) / b; }
+
+// ------------------------------------------------------------------------------------------
+// TMA descriptor encoding through the driver entry point (no link-time dependency on libcuda)
+// ------------------------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+whale_status get_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode ? WHALE_OK : WHALE_ERR_CUDA;
+}
+
+// 2-D bf16 row-major tensor [rows, cols] with row stride ld, box [box_rows, 64 columns], 128-B swizzle.
+whale_status tmap_bf16(CUtensorMap* tm, const void* base, long long rows, long long cols, long long ld, int box_rows) {
+  WCHECK(get_encoder());
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || (ld * 2) % 16 || rows <= 0 || cols <= 0) return WHALE_ERR_INVALID_ARG;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+  cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1u, 1u};
+  CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? WHALE_OK : WHALE_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------------------------------
+// Validated shape
+// ------------------------------------------------------------------------------------------
+struct Shape {
+  bool bf16;
+  int layers, d, h, dh, N, H, Fh;
+  bool shared_kv, tied, debug;
+  float eps;
+  int kvw;  // kv row width: 2d, or d with shared K = V
+  int ugw;  // rows of the up|gate matrix: 2H, or H with a tied gate
+  size_t es;  // element size
+};
+
+whale_status validate(const whale_config* c, Shape* s) {
+  if (!c || !s) return WHALE_ERR_INVALID_ARG;
+  if (c->n_layers < 1 || c->d < 1 || c->n_heads < 1 || c->n_tokens < 1 || c->ffn_hidden < 1 ||
+      c->fusion_hidden < 0 || !(c->eps >= 0.f) || (c->dtype != WHALE_FP32 && c->dtype != WHALE_BF16) ||
+      (c->flags & ~(WHALE_SHARED_KV | WHALE_TIED_GATE | WHALE_DEBUG)) || c->d % c->n_heads)
+    return WHALE_ERR_INVALID_ARG;
+  s->bf16 = c->dtype == WHALE_BF16;
+  s->layers = c->n_layers;
+  s->d = c->d;
+  s->h = c->n_heads;
+  s->dh = c->d / c->n_heads;
+  s->N = c->n_tokens;
+  s->H = c->ffn_hidden;
+  s->Fh = c->fusion_hidden;
+  s->shared_kv = c->flags & WHALE_SHARED_KV;
+  s->tied = c->flags & WHALE_TIED_GATE;
+  s->debug = c->flags & WHALE_DEBUG;
+  s->eps = c->eps;
+  s->kvw = s->shared_kv ? s->d : 2 * s->d;
+  s->ugw = s->tied ? s->H : 2 * s->H;
+  s->es = s->bf16 ? 2 : 4;
+  if (s->bf16) {
+    const int hg = s->h < 8 ? s->h : 8;
+    if (s->d % 64 || (s->dh != 32 && s->dh != 64) || s->h % hg || (hg * s->dh) % 64 || (hg != 2 && hg != 4 && hg != 8) ||
+        s->H % 64 || s->Fh % 64)
+      return WHALE_ERR_UNSUPPORTED;
+  } else {
+    if (s->dh != 8 && s->dh != 16 && s->dh != 32 && s->dh != 64 && s->dh != 128) return WHALE_ERR_UNSUPPORTED;
+  }
+  return WHALE_OK;
+}
+
+whale_status check_hint(const whale_shape_hint* h) {
+  if (!h || h->B < 0 || h->max_L < 0 || h->total_L < 0 || h->total_L >= (1ll << 31)) return WHALE_ERR_INVALID_ARG;
+  return WHALE_OK;
+}
+
+// ------------------------------------------------------------------------------------------
+// Attention plan (bf16 split-L kernel)
+// ------------------------------------------------------------------------------------------
+struct AttnPlan {
+  int QT, QB, nqb, T, HG, G;
+  size_t po_elems, pml_elems;
+};
+
+AttnPlan plan_attention(const Shape& s, int B, long long total_L) {
+  AttnPlan p{};
+  p.QT = s.N <= 16 ? 1 : (s.N <= 32 ? 2 : 4);
+  p.QB = 16 * p.QT;
+  p.nqb = cdiv(s.N, p.QB);
+  p.T = (s.dh == 64 || p.QT == 4) ? 32 : 64;
+  p.HG = s.h < 8 ? s.h : 8;
+  // one CTA per SM (the stage ring takes most of shared memory); each CTA streams an equal
+  // slice of the flattened work rows, at least a few tiles of them
+  const long long work_rows = total_L * p.nqb;
+  long long G = cdiv<long long>(work_rows, 4ll * p.T);
+  if (G > kNumSM) G = kNumSM;
+  if (G < 1) G = 1;
+  p.G = (int)G;
+  const size_t slots = (size_t)B * p.nqb + p.G;
+  p.pml_elems = slots * s.h * p.QB * 2;
+  p.po_elems = slots * s.h * p.QB * s.dh;
+  return p;
+}
+
+// ------------------------------------------------------------------------------------------
+// Workspace layout of the forward (the step entry points use prefixes of their own)
+// ------------------------------------------------------------------------------------------
+struct Layout {
+  size_t wq, wkv, wug;   // prepared weights (bf16)
+  size_t po, pml;        // attention partials (bf16)
+  size_t r;              // row factors (fp32 path)
+  size_t q, kv, a, g, f, u, ug, x0, x1;   // fp32 path, and q / kv of the bf16 path
+  // bf16 path: lo halves of the token-side operand pairs and the fp32 residual stream
+  size_t a_lo, g_lo, f_lo, u_lo, f32, x32[2], xhi[2], xlo[2];
+  size_t total;
+};
+
+Layout make_layout(const Shape& s, const whale_shape_hint& hint) {
+  Layout L{};
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = o;
+    o = align_up(o + bytes);
+    return at;
+  };
+  const size_t rows = (size_t)hint.B * s.N;
+  const size_t tl = (size_t)hint.total_L;
+  if (s.bf16) {
+    L.wq = take((size_t)s.d * s.d * 2);
+    L.wkv = take((size_t)s.kvw * s.d * 2);
+    L.wug = take((size_t)s.ugw * s.d * 2);
+    AttnPlan p = plan_attention(s, hint.B, hint.total_L);
+    L.po = take(p.po_elems * 4);
+    L.pml = take(p.pml_elems * 4);
+  } else {
+    L.r = take((rows > tl ? rows : tl) * 4);
+  }
+  L.q = take(rows * s.d * s.es);
+  L.kv = take(tl * s.kvw * s.es);
+  L.a = take(rows * s.d * s.es);
+  L.g = take(rows * (size_t)s.Fh * s.es);
+  L.f = take(rows * s.d * s.es);
+  L.u = take(rows * (size_t)s.H * s.es);
+  if (s.bf16) {
+    L.a_lo = take(rows * s.d * 2);
+    L.g_lo = take(rows * (size_t)s.Fh * 2);
+    L.f_lo = take(rows * s.d * 2);
+    L.u_lo = take(rows * (size_t)s.H * 2);
+    L.f32 = take(rows * s.d * 4);
+    for (int i = 0; i < 2; ++i) {
+      L.x32[i] = take(rows * s.d * 4);
+      L.xhi[i] = take(rows * s.d * 2);
+      L.xlo[i] = take(rows * s.d * 2);
+    }
+  } else {
+    L.ug = take(rows * (size_t)s.ugw * 4);
+    L.x0 = take(rows * s.d * s.es);
+    L.x1 = take(rows * s.d * s.es);
+  }
+  L.total = o;
+  return L;
+}
+
+inline char* at(void* ws, size_t off) { return static_cast<char*>(ws) + off; }
+
+// ------------------------------------------------------------------------------------------
+// bf16 tcgen05 GEMM dispatch
+// ------------------------------------------------------------------------------------------
+// A GEMM operand: bf16 rows [M, K] with row stride ld; `lo` (optional) is the second half of
+// a hi/lo pair (SPLIT mode).
+struct Opnd {
+  const void* hi;
+  const void* lo;
+  long long ld;
+  int K;
+};
+// Where the epilogue writes (any may be null): bf16 hi, bf16 residue lo, fp32.
+struct Outs {
+  void* hi;
+  void* lo;
+  float* f32;
+  long long ld;
+};
+
+template <int BN, int EPI, bool RN, bool SPLIT>
+whale_status launch_gemm_t(const CUtensorMap* tm, const GemmArgs& g, long long tiles, cudaStream_t st) {
+  const size_t smem = GemmSmem<BN, SPLIT>::BYTES;
+  auto kern = gemm_tc_kernel<BN, EPI, RN, SPLIT>;
+  CUCHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  kern<<<(unsigned)tiles, kGemmThreads, smem, st>>>(tm[0], tm[1], tm[2], tm[3], tm[4], g);
+  CUCHECK(cudaGetLastError());
+  return WHALE_OK;
+}
+
+template <int BN>
+whale_status launch_gemm_bn(int epi, bool rn, bool split, const CUtensorMap* tm, const GemmArgs& g, long long tiles,
+                            cudaStream_t st) {
+  if (rn && epi == EPI_STORE && !split) return launch_gemm_t<BN, EPI_STORE, true, false>(tm, g, tiles, st);
+  if (rn && epi == EPI_STORE && split) return launch_gemm_t<BN, EPI_STORE, true, true>(tm, g, tiles, st);
+  if (!split) return WHALE_ERR_UNSUPPORTED;
+  if (rn && epi == EPI_SWIGLU) return launch_gemm_t<BN, EPI_SWIGLU, true, true>(tm, g, tiles, st);
+  if (rn && epi == EPI_SWIGLU_TIED) return launch_gemm_t<BN, EPI_SWIGLU_TIED, true, true>(tm, g, tiles, st);
+  if (!rn && epi == EPI_SILU) return launch_gemm_t<BN, EPI_SILU, false, true>(tm, g, tiles, st);
+  if (!rn && epi == EPI_RESID) return launch_gemm_t<BN, EPI_RESID, false, true>(tm, g, tiles, st);
+  return WHALE_ERR_UNSUPPORTED;
+}
+
+template <int BN>
+whale_status launch_persistent_t(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
+                                 const PGemmArgs& g, cudaStream_t st) {
+  const size_t smem = PGemmSmem<BN>::BYTES;
+  auto kern = gemm_rownorm_persistent_kernel<BN>;
+  CUCHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  const int grid = g.num_tiles < kNumSM ? g.num_tiles : kNumSM;
+  kern<<<grid, kPGemmThreads, smem, st>>>(ta, tb, to, g);
+  CUCHECK(cudaGetLastError());
+  return WHALE_OK;
+}
+
+// out = r(A) * (A W^T) in bf16, persistent over 128 x BN tiles (BN = 256 when N allows).
+whale_status gemm_rownorm_persistent(const Opnd& a0, const void* W, int N, const Outs& out, long long M, float eps,
+                                     cudaStream_t st) {
+  const int bn = (N % 256 == 0) ? 256 : 128;
+  CUtensorMap ta, tb, to;
+  WCHECK(tmap_bf16(&ta, a0.hi, M, a0.K, a0.ld, 128));
+  WCHECK(tmap_bf16(&tb, W, N, a0.K, a0.K, bn));
+  WCHECK(tmap_bf16(&to, out.hi, M, N, out.ld, 32));
+  PGemmArgs g{};
+  g.M = (int)M;
+  g.N = N;
+  g.kb = a0.K / 64;
+  g.tiles_n = N / bn;
+  g.num_tiles = (int)(cdiv<long long>(M, 128) * g.tiles_n);
+  g.inv_k = 1.0f / (float)a0.K;
+  g.eps = eps;
+  if (bn == 256) return launch_persistent_t<256>(ta, tb, to, g, st);
+  return launch_persistent_t<128>(ta, tb, to, g, st);
+}
+
+// out = epi([A0 | A1] W^T), W [N, K0+K1] bf16; SPLIT when the operands carry lo halves.
+whale_status gemm_bf16(const Opnd& a0, const Opnd& a1, const void* W, int N, const Outs& out, const float* resid32,
+                       long long ldr, long long M, int epi, bool rn, float eps, cudaStream_t st) {
+  if (M <= 0) return WHALE_OK;
+  if (M >= (1ll << 31)) return WHALE_ERR_UNSUPPORTED;
+  const bool split = a0.lo != nullptr;
+  if (a0.K % 64 || a1.K % 64 || N % 64 || (a1.K > 0 && (a1.lo != nullptr) != split)) return WHALE_ERR_UNSUPPORTED;
+  const long long tm = cdiv<long long>(M, 128);
+  // Large single-source row-norm projections (the history-side K|V GEMM): persistent kernel.
+  if (!split && rn && epi == EPI_STORE && a1.K == 0 && out.hi && !out.lo && !out.f32 && N % 128 == 0 &&
+      tm * (N / 128) >= 2 * kNumSM)
+    return gemm_rownorm_persistent(a0, W, N, out, M, eps, st);
+  int bn = 64;
+  if (N % 256 == 0 && tm * (N / 256) >= kNumSM) bn = 256;
+  else if (N % 128 == 0 && tm * (N / 128) >= kNumSM) bn = 128;
+  CUtensorMap maps[5];
+  WCHECK(tmap_bf16(&maps[0], a0.hi, M, a0.K, a0.ld, 128));
+  if (split) WCHECK(tmap_bf16(&maps[1], a0.lo, M, a0.K, a0.ld, 128));
+  else maps[1] = maps[0];
+  if (a1.K > 0) {
+    WCHECK(tmap_bf16(&maps[2], a1.hi, M, a1.K, a1.ld, 128));
+    if (split) WCHECK(tmap_bf16(&maps[3], a1.lo, M, a1.K, a1.ld, 128));
+    else maps[3] = maps[2];
+  } else {
+    maps[2] = maps[0];
+    maps[3] = maps[1];
+  }
+  WCHECK(tmap_bf16(&maps[4], W, N, a0.K + a1.K, a0.K + a1.K, bn));
+  GemmArgs g{};
+  g.M = (int)M;
+  g.N = N;
+  g.kb0 = a0.K / 64;
+  g.kb1 = a1.K / 64;
+  g.tiles_n = N / bn;
+  g.inv_k = 1.0f / (float)a0.K;
+  g.eps = eps;
+  g.out_hi = static_cast<__nv_bfloat16*>(out.hi);
+  g.out_lo = static_cast<__nv_bfloat16*>(out.lo);
+  g.out32 = out.f32;
+  g.ldo = out.ld;
+  g.resid32 = resid32;
+  g.ldr = ldr;
+  const long long tiles = tm * g.tiles_n;
+  if (bn == 256) return launch_gemm_bn<256>(epi, rn, split, maps, g, tiles, st);
+  if (bn == 128) return launch_gemm_bn<128>(epi, rn, split, maps, g, tiles, st);
+  return launch_gemm_bn<64>(epi, rn, split, maps, g, tiles, st);
+}
+
+inline Opnd opnd(const void* hi, const void* lo, long long ld, int K) { return Opnd{hi, lo, ld, K}; }
+inline Opnd no_opnd() { return Opnd{nullptr, nullptr, 0, 0}; }
+
+whale_status pair_from_bf16(const void* x, float* x32, void* lo, long long n, cudaStream_t st) {
+  if (n <= 0) return WHALE_OK;
+  const unsigned grid = (unsigned)std::min<long long>(cdiv<long long>(n, 256), 8 * kNumSM);
+  pair_from_bf16_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), x32,
+                                              static_cast<__nv_bfloat16*>(lo), n);
+  CUCHECK(cudaGetLastError());
+  return WHALE_OK;
+}
+
+// ------------------------------------------------------------------------------------------
+// bf16 steps
+// ------------------------------------------------------------------------------------------
+whale_status fold_weights(const Shape& s, const __nv_bfloat16* wq, const float* gq, const __nv_bfloat16* wkv,
+                          const float* gkv, const __nv_bfloat16* wug, const float* gffn, __nv_bfloat16* oq,
+                          __nv_bfloat16* okv, __nv_bfloat16* oug, cudaStream_t st) {
+  FoldJobs jobs{};
+  long long maxe = 0;
+  auto add = [&](const __nv_bfloat16* w, const float* g, __nv_bfloat16* out, int rows, int mode) {
+    if (!w || !out) return;
+    FoldJob& j = jobs.job[jobs.n++];
+    j.w = w;
+    j.g = g;
+    j.out = out;
+    j.rows = rows;
+    j.cols = s.d;
+    j.mode = mode;
+    j.H = s.H;
+    maxe = std::max(maxe, (long long)rows * s.d);
+  };
+  add(wq, gq, oq, s.d, 0);
+  add(wkv, gkv, okv, s.kvw, 0);
+  add(wug, gffn, oug, s.ugw, s.tied ? 0 : 1);
+  if (jobs.n == 0) return WHALE_OK;
+  const unsigned gx = (unsigned)std::min<long long>(cdiv<long long>(maxe, 256), 4 * kNumSM);
+  fold_weights_kernel<<<dim3(gx, jobs.n), 256, 0, st>>>(jobs);
+  CUCHECK(cudaGetLastError());
+  return WHALE_OK;
+}
+
+template <int DH, int QT, int HG>
+whale_status launch_attn_t(const CUtensorMap& tm, const AttnArgs& a, dim3 grid, cudaStream_t st) {
+  constexpr int T = (DH == 64 || QT == 4) ? 32 : 64;
+  using C = AttnCfg<DH, QT, T, HG>;
+  constexpr int stage = 2 * C::KV_BYTES;
+  constexpr int ST = (196608 / stage) > 4 ? 4 : ((196608 / stage) < 2 ? 2 : (196608 / stage));
+  const size_t smem = 1024 + (size_t)ST * stage + 256;
+  auto kern = attn_splitl_kernel<DH, QT, T, HG, ST>;
+  CUCHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  kern<<<grid, C::THREADS, smem, st>>>(tm, a);
+  CUCHECK(cudaGetLastError());
+  return WHALE_OK;
+}
+
+template <int DH, int QT>
+whale_status launch_attn_hg(int hg, const CUtensorMap& tm, const AttnArgs& a, dim3 grid, cudaStream_t st) {
+  if (hg == 8) return launch_attn_t<DH, QT, 8>(tm, a, grid, st);
+  if (hg == 4) return launch_attn_t<DH, QT, 4>(tm, a, grid, st);
+  if (hg == 2) return launch_attn_t<DH, QT, 2>(tm, a, grid, st);
+  return WHALE_ERR_UNSUPPORTED;
+}
+
+whale_status attention_bf16(const Shape& s, const void* q, const void* kv, const int* offsets, void* out,
+                            void* out_lo, int B, int max_L, long long total_L, float* po, float* pml,
+                            cudaStream_t st) {
+  (void)max_L;
+  if (B == 0) return WHALE_OK;
+  const AttnPlan p = plan_attention(s, B, total_L);
+  AttnArgs a{};
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.offsets = offsets;
+  a.part_o = po;
+  a.part_ml = pml;
+  a.B = B;
+  a.N = s.N;
+  a.QB = p.QB;
+  a.n_qblocks = p.nqb;
+  a.d = s.d;
+  a.n_heads = s.h;
+  a.v_col0 = s.shared_kv ? 0 : s.d;
+  a.shared_kv = s.shared_kv ? 1 : 0;
+  a.G = p.G;
+  a.total_L = total_L;
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)s.dh));
+  if ((long long)B * p.nqb > (1ll << 31) - 1) return WHALE_ERR_UNSUPPORTED;
+  if (total_L > 0) {
+    CUtensorMap tm;
+    WCHECK(tmap_bf16(&tm, kv, total_L, s.kvw, s.kvw, p.T));
+    const dim3 grid(p.G, s.h / p.HG);
+    whale_status r = WHALE_ERR_UNSUPPORTED;
+    if (s.dh == 32) {
+      if (p.QT == 1) r = launch_attn_hg<32, 1>(p.HG, tm, a, grid, st);
+      else if (p.QT == 2) r = launch_attn_hg<32, 2>(p.HG, tm, a, grid, st);
+      else r = launch_attn_hg<32, 4>(p.HG, tm, a, grid, st);
+    } else {
+      if (p.QT == 1) r = launch_attn_hg<64, 1>(p.HG, tm, a, grid, st);
+      else if (p.QT == 2) r = launch_attn_hg<64, 2>(p.HG, tm, a, grid, st);
+      else r = launch_attn_hg<64, 4>(p.HG, tm, a, grid, st);
+    }
+    WCHECK(r);
+  }
+  if ((long long)B * p.nqb > 0x7fffffffll || s.h > 65535) return WHALE_ERR_UNSUPPORTED;
+  const dim3 cgrid((unsigned)(B * p.nqb), s.h);
+  auto* o_hi = static_cast<__nv_bfloat16*>(out);
+  auto* o_lo = static_cast<__nv_bfloat16*>(out_lo);
+  if (s.dh == 32) attn_combine_kernel<32><<<cgrid, 256, 0, st>>>(a, o_hi, o_lo);
+  else attn_combine_kernel<64><<<cgrid, 256, 0, st>>>(a, o_hi, o_lo);
+  CUCHECK(cudaGetLastError());
+  return WHALE_OK;
+}
+
+// ------------------------------------------------------------------------------------------
+// fp32 steps
+// ------------------------------------------------------------------------------------------
+whale_status row_rms(const float* x, long long rows, int d, float eps, float* r, cudaStream_t st) {
+  if (rows <= 0) return WHALE_OK;
+  row_rms_f32<<<(unsigned)cdiv<long long>(rows, 8), 256, 0, st>>>(x, d, rows, d, eps, r);
+  CUCHECK(cudaGetLastError());
+  return WHALE_OK;
+}
+
+whale_status gemm_f32(const float* A0, int K0, const float* A1, int K1, const float* rn, const float* gn,
+                      const float* W, int N, float* C, long long M, int epi, const float* R, cudaStream_t st) {
+  if (M <= 0) return WHALE_OK;
+  const long long gy = cdiv<long long>(M, 64);
+  if (gy > 65535) return WHALE_ERR_UNSUPPORTED;
+  gemm_f32_kernel<<<dim3(cdiv(N, 64), (unsigned)gy), 256, 0, st>>>(A0, K0, K0, A1, K1, K1, rn, gn, W, C, N, M, N, epi,
+                                                                    R, N);
+  CUCHECK(cudaGetLastError());
+  return WHALE_OK;
+}
+
+whale_status attention_f32(const Shape& s, const float* q, const float* kv, const int* offsets, float* a, int B,
+                           long long total_L, cudaStream_t st) {
+  const long long warps = (long long)B * s.N * s.h;
+  if (warps == 0) return WHALE_OK;
+  const unsigned grid = (unsigned)cdiv<long long>(warps, 4);
+  const float scale = (float)(1.0 / std::sqrt((double)s.dh));
+  const int v0 = s.shared_kv ? 0 : s.d;
+#define ATT32(DH) attn_f32_kernel<DH><<<grid, 128, 0, st>>>(q, kv, s.kvw, v0, offsets, a, B, s.N, s.d, s.h, total_L, scale)
+  switch (s.dh) {
+    case 8: ATT32(8); break;
+    case 16: ATT32(16); break;
+    case 32: ATT32(32); break;
+    case 64: ATT32(64); break;
+    case 128: ATT32(128); break;
+    default: return WHALE_ERR_UNSUPPORTED;
+  }
+#undef ATT32
+  CUCHECK(cudaGetLastError());
+  return WHALE_OK;
+}
+
+whale_status swiglu_f32(const Shape& s, const float* f, const float* gffn, const float* wug, const float* wdown,
+                        float* y, long long rows, float* r, float* ug, float* u, cudaStream_t st) {
+  WCHECK(row_rms(f, rows, s.d, s.eps, r, st));
+  WCHECK(gemm_f32(f, s.d, nullptr, 0, r, gffn, wug, s.ugw, ug, rows, F32_NONE, nullptr, st));
+  if (rows > 0) {
+    swiglu_f32_kernel<<<(unsigned)cdiv<long long>(rows * s.H, 256), 256, 0, st>>>(ug, s.ugw, u, rows, s.H, s.tied);
+    CUCHECK(cudaGetLastError());
+  }
+  return gemm_f32(u, s.H, nullptr, 0, nullptr, nullptr, wdown, s.d, y, rows, F32_RESID, f, st);
+}
+
+// fp32 Fusion MLP (correctness path).
+whale_status fusion_mlp_f32(const Shape& s, long long rows, const float* a, const float* x, const float* wf1,
+                            const float* wf2, float* f, float* gbuf, cudaStream_t st) {
+  if (s.Fh > 0) {
+    WCHECK(gemm_f32(a, s.d, x, s.d, nullptr, nullptr, wf1, s.Fh, gbuf, rows, F32_SILU, nullptr, st));
+    return gemm_f32(gbuf, s.Fh, nullptr, 0, nullptr, nullptr, wf2, s.d, f, rows, F32_RESID, x, st);
+  }
+  return gemm_f32(a, s.d, x, s.d, nullptr, nullptr, wf2, s.d, f, rows, F32_RESID, x, st);
+}
+
+bool weights_ok(const Shape& s, const whale_layer_weights* w) {
+  return w && w->g_q && w->g_kv && w->g_ffn && w->w_q && w->w_kv && w->w_f2 && w->w_upgate && w->w_down &&
+         (s.Fh == 0 || w->w_f1);
+}
+
+// A token-side tensor of the bf16 path: fp32 value plus its bf16 hi/lo pair (any may be null
+// for an output that is not needed).
+struct Stream3 {
+  float* f32;
+  void* hi;
+  void* lo;
+};
+
+// S4 + S5 of the bf16 path, shared by the layer and by the step entry points:
+//   F = X + W_F2 SiLU(W_F1 [A ; X])  (or X + W_F [A ; X]);  Y = F + W_down (SiLU(gate) * up)
+whale_status fusion_bf16(const Shape& s, long long rows, const Opnd& A, const Opnd& X, const float* x32,
+                         const void* wf1, const void* wf2, void* g, void* g_lo, const Stream3& F, cudaStream_t st) {
+  const Outs fo{F.hi, F.lo, F.f32, s.d};
+  if (s.Fh > 0) {
+    WCHECK(gemm_bf16(A, X, wf1, s.Fh, Outs{g, g_lo, nullptr, s.Fh}, nullptr, 0, rows, EPI_SILU, false, 0.f, st));
+    return gemm_bf16(opnd(g, g_lo, s.Fh, s.Fh), no_opnd(), wf2, s.d, fo, x32, s.d, rows, EPI_RESID, false, 0.f, st);
+  }
+  return gemm_bf16(A, X, wf2, s.d, fo, x32, s.d, rows, EPI_RESID, false, 0.f, st);
+}
+
+whale_status ffn_bf16(const Shape& s, long long rows, const Opnd& F, const float* f32, const void* wug_folded,
+                      const void* wdown, void* u, void* u_lo, const Stream3& Y, cudaStream_t st) {
+  WCHECK(gemm_bf16(F, no_opnd(), wug_folded, s.ugw, Outs{u, u_lo, nullptr, s.H}, nullptr, 0, rows,
+                   s.tied ? EPI_SWIGLU_TIED : EPI_SWIGLU, true, s.eps, st));
+  return gemm_bf16(opnd(u, u_lo, s.H, s.H), no_opnd(), wdown, s.d, Outs{Y.hi, Y.lo, Y.f32, s.d}, f32, s.d, rows,
+                   EPI_RESID, false, 0.f, st);
+}
+
+// One bf16 layer. `in` is the residual-stream tensor (f32, hi, lo all set), `out` receives
+// H_f in the forms requested.
+whale_status layer_bf16(const Shape& s, const Stream3& in, const void* slab, const int* offsets,
+                        const whale_layer_weights& w, const Stream3& out, const whale_shape_hint& hint, void* ws,
+                        const Layout& L, cudaStream_t st) {
+  const long long rows = (long long)hint.B * s.N;
+  auto* wq = at(ws, L.wq);
+  auto* wkv = at(ws, L.wkv);
+  auto* wug = at(ws, L.wug);
+  WCHECK(fold_weights(s, static_cast<const __nv_bfloat16*>(w.w_q), w.g_q, static_cast<const __nv_bfloat16*>(w.w_kv),
+                      w.g_kv, static_cast<const __nv_bfloat16*>(w.w_upgate), w.g_ffn,
+                      reinterpret_cast<__nv_bfloat16*>(wq), reinterpret_cast<__nv_bfloat16*>(wkv),
+                      reinterpret_cast<__nv_bfloat16*>(wug), st));
+  const Opnd X = opnd(in.hi, in.lo, s.d, s.d);
+  // S1 queries, S2 keys|values
+  WCHECK(gemm_bf16(X, no_opnd(), wq, s.d, Outs{at(ws, L.q), nullptr, nullptr, s.d}, nullptr, 0, rows, EPI_STORE, true,
+                   s.eps, st));
+  WCHECK(gemm_bf16(opnd(slab, nullptr, s.d, s.d), no_opnd(), wkv, s.kvw, Outs{at(ws, L.kv), nullptr, nullptr, s.kvw},
+                   nullptr, 0, hint.total_L, EPI_STORE, true, s.eps, st));
+  // S3 attention -> A as a hi/lo pair
+  WCHECK(attention_bf16(s, at(ws, L.q), at(ws, L.kv), offsets, at(ws, L.a), at(ws, L.a_lo), hint.B, hint.max_L,
+                        hint.total_L, reinterpret_cast<float*>(at(ws, L.po)), reinterpret_cast<float*>(at(ws, L.pml)),
+                        st));
+  // S4 Fusion MLP -> F (fp32 + pair)
+  auto* f32 = reinterpret_cast<float*>(at(ws, L.f32));
+  WCHECK(fusion_bf16(s, rows, opnd(at(ws, L.a), at(ws, L.a_lo), s.d, s.d), X, in.f32, w.w_f1, w.w_f2, at(ws, L.g),
+                     at(ws, L.g_lo), Stream3{f32, at(ws, L.f), at(ws, L.f_lo)}, st));
+  // S5 SwiGLU FFN -> H_f
+  return ffn_bf16(s, rows, opnd(at(ws, L.f), at(ws, L.f_lo), s.d, s.d), f32, wug, w.w_down, at(ws, L.u),
+                  at(ws, L.u_lo), out, st);
+}
+
+// One fp32 layer (SIMT correctness path).
+whale_status layer_f32(const Shape& s, const void* x_in, const void* slab, const int* offsets,
+                       const whale_layer_weights& w, void* x_out, const whale_shape_hint& hint, void* ws,
+                       const Layout& L, cudaStream_t st) {
+  const long long rows = (long long)hint.B * s.N;
+  auto F = [&](size_t off) { return reinterpret_cast<float*>(at(ws, off)); };
+  const float* xf = static_cast<const float*>(x_in);
+  const float* sf = static_cast<const float*>(slab);
+  WCHECK(row_rms(xf, rows, s.d, s.eps, F(L.r), st));
+  WCHECK(gemm_f32(xf, s.d, nullptr, 0, F(L.r), w.g_q, static_cast<const float*>(w.w_q), s.d, F(L.q), rows, F32_NONE,
+                  nullptr, st));
+  WCHECK(row_rms(sf, hint.total_L, s.d, s.eps, F(L.r), st));
+  WCHECK(gemm_f32(sf, s.d, nullptr, 0, F(L.r), w.g_kv, static_cast<const float*>(w.w_kv), s.kvw, F(L.kv),
+                  hint.total_L, F32_NONE, nullptr, st));
+  WCHECK(attention_f32(s, F(L.q), F(L.kv), offsets, F(L.a), hint.B, hint.total_L, st));
+  WCHECK(fusion_mlp_f32(s, rows, F(L.a), xf, static_cast<const float*>(w.w_f1), static_cast<const float*>(w.w_f2),
+                        F(L.f), F(L.g), st));
+  return swiglu_f32(s, F(L.f), w.g_ffn, static_cast<const float*>(w.w_upgate), static_cast<const float*>(w.w_down),
+                    static_cast<float*>(x_out), rows, F(L.r), F(L.ug), F(L.u), st);
+}
+
+// The stack over device buffers: tokens (layer-0 H_w) -> out (last H_f).
+// `hook(l, before)` (optional) runs on the host before and after layer l is enqueued.
+using LayerHook = std::function<whale_status(int, bool)>;
+whale_status stack_impl(const Shape& s, const void* tokens, const void* seq_states, const int* offsets,
+                        const whale_layer_weights* weights, int first_layer, int n_layers, void* out,
+                        const whale_shape_hint& hint, void* ws, const Layout& L, cudaStream_t st,
+                        const void* const* slabs /* per layer, or null: seq_states + l * slab */,
+                        const LayerHook& hook = nullptr) {
+  const size_t slab_bytes = (size_t)hint.total_L * s.d * s.es;
+  auto slab_of = [&](int l) -> const void* {
+    if (slabs) return slabs[l];
+    return seq_states ? static_cast<const char*>(seq_states) + (size_t)(first_layer + l) * slab_bytes : nullptr;
+  };
+  const long long rows = (long long)hint.B * s.N;
+  if (!s.bf16) {
+    const void* x = tokens;
+    for (int l = 0; l < n_layers; ++l) {
+      void* y = (l == n_layers - 1) ? out : at(ws, (l & 1) ? L.x1 : L.x0);
+      if (hook) WCHECK(hook(l, true));
+      WCHECK(layer_f32(s, x, slab_of(l), offsets, weights[first_layer + l], y, hint, ws, L, st));
+      if (hook) WCHECK(hook(l, false));
+      x = y;
+    }
+    return WHALE_OK;
+  }
+  auto buf = [&](int i) {
+    return Stream3{reinterpret_cast<float*>(at(ws, L.x32[i])), at(ws, L.xhi[i]), at(ws, L.xlo[i])};
+  };
+  Stream3 in = buf(0);
+  in.hi = const_cast<void*>(tokens);  // bf16 tokens are their own hi half; lo = 0
+  WCHECK(pair_from_bf16(tokens, in.f32, in.lo, rows * s.d, st));
+  for (int l = 0; l < n_layers; ++l) {
+    const Stream3 y = (l == n_layers - 1) ? Stream3{nullptr, out, nullptr} : buf((l + 1) & 1);
+    if (hook) WCHECK(hook(l, true));
+    WCHECK(layer_bf16(s, in, slab_of(l), offsets, weights[first_layer + l], y, hint, ws, L, st));
+    if (hook) WCHECK(hook(l, false));
+    in = y;
+  }
+  return WHALE_OK;
+}
+
+whale_status common_checks(const whale_config* cfg, const whale_shape_hint* hint, Shape* s, void* ws, size_t ws_bytes,
+                           Layout* L) {
+  WCHECK(validate(cfg, s));
+  WCHECK(check_hint(hint));
+  *L = make_layout(*s, *hint);
+  if (!ws || ws_bytes < L->total || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1))) return WHALE_ERR_WORKSPACE;
+  return WHALE_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+whale_status debug_check(const Shape& s, const int* offsets, const whale_shape_hint& hint, cudaStream_t st) {
+  if (!s.debug) return WHALE_OK;
+  check_offsets_kernel<<<cdiv(hint.B + 1, 256), 256, 0, st>>>(offsets, hint.B, hint.max_L, hint.total_L);
+  CUCHECK(cudaGetLastError());
+  return WHALE_OK;
+}
+
+// Per-device copy stream and events of the host-buffer forward (created once, kept).
+struct HostPipe {
+  cudaStream_t copy = nullptr;
+  cudaEvent_t copied[2] = {nullptr, nullptr}, consumed[2] = {nullptr, nullptr};
+};
+std::mutex g_pipe_mu;
+HostPipe g_pipes[64];
+
+whale_status host_pipe(HostPipe** out) {
+  int dev = 0;
+  CUCHECK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return WHALE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_pipe_mu);
+  HostPipe& p = g_pipes[dev];
+  if (!p.copy) {
+    CUCHECK(cudaStreamCreateWithFlags(&p.copy, cudaStreamNonBlocking));
+    for (int i = 0; i < 2; ++i) {
+      CUCHECK(cudaEventCreateWithFlags(&p.copied[i], cudaEventDisableTiming));
+      CUCHECK(cudaEventCreateWithFlags(&p.consumed[i], cudaEventDisableTiming));
+    }
+  }
+  *out = &p;
+  return WHALE_OK;
+}
+
+size_t host_staging_bytes(const Shape& s, const whale_shape_hint& h, size_t* o_tok, size_t* o_slab0, size_t* o_slab1,
+                          size_t* o_off, size_t* o_out) {
+  const size_t rows = (size_t)h.B * s.N;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    size_t a = o;
+    o = align_up(o + bytes);
+    return a;
+  };
+  *o_tok = take(rows * s.d * s.es);
+  *o_slab0 = take((size_t)h.total_L * s.d * s.es);
+  *o_slab1 = take((size_t)h.total_L * s.d * s.es);
+  *o_off = take(((size_t)h.B + 1) * 4);
+  *o_out = take(rows * s.d * s.es);
+  return o;
+}
+
+}  // namespace
+
+// ============================================================================================
+// C ABI
+// ============================================================================================
+extern "C" {
+
+const char* whale_status_string(whale_status s) {
+  switch (s) {
+    case WHALE_OK: return "ok";
+    case WHALE_ERR_INVALID_ARG: return "invalid argument";
+    case WHALE_ERR_UNSUPPORTED: return "unsupported shape or configuration";
+    case WHALE_ERR_CUDA: return "CUDA error";
+    case WHALE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case WHALE_ERR_DEVICE_CHECK: return "device-side check recorded an error";
+  }
+  return "unknown status";
+}
+
+size_t whale_workspace_size(const whale_config* cfg, const whale_shape_hint* hint) {
+  Shape s;
+  if (validate(cfg, &s) != WHALE_OK || check_hint(hint) != WHALE_OK) return 0;
+  return make_layout(s, *hint).total;
+}
+
+whale_status whale_fusion_layer_forward(const whale_config* cfg, const void* tokens_in, const void* layer_states,
+                                        const int* seq_offsets, const whale_layer_weights* w, void* tokens_out,
+                                        const whale_shape_hint* hint, void* ws, size_t ws_bytes,
+                                        whale_stream_t stream) {
+  Shape s;
+  Layout L;
+  WCHECK(common_checks(cfg, hint, &s, ws, ws_bytes, &L));
+  if (hint->B == 0) return WHALE_OK;
+  if (!tokens_in || !tokens_out || !seq_offsets || !weights_ok(s, w) || (hint->total_L > 0 && !layer_states))
+    return WHALE_ERR_INVALID_ARG;
+  if (!aligned16(tokens_in) || !aligned16(tokens_out) || (layer_states && !aligned16(layer_states)))
+    return WHALE_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  WCHECK(debug_check(s, seq_offsets, *hint, st));
+  const void* slabs[1] = {layer_states};
+  return stack_impl(s, tokens_in, nullptr, seq_offsets, w, 0, 1, tokens_out, *hint, ws, L, st, slabs);
+}
+
+whale_status whale_fusion_forward(const whale_config* cfg, const void* tokens, const void* seq_states,
+                                  const int* seq_offsets, const whale_layer_weights* weights, void* out,
+                                  const whale_shape_hint* hint, void* ws, size_t ws_bytes, whale_stream_t stream) {
+  Shape s;
+  Layout L;
+  WCHECK(common_checks(cfg, hint, &s, ws, ws_bytes, &L));
+  if (hint->B == 0) return WHALE_OK;
+  if (!tokens || !out || !seq_offsets || !weights || (hint->total_L > 0 && !seq_states)) return WHALE_ERR_INVALID_ARG;
+  for (int l = 0; l < s.layers; ++l)
+    if (!weights_ok(s, &weights[l])) return WHALE_ERR_INVALID_ARG;
+  if (!aligned16(tokens) || !aligned16(out) || (seq_states && !aligned16(seq_states))) return WHALE_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  WCHECK(debug_check(s, seq_offsets, *hint, st));
+  return stack_impl(s, tokens, seq_states, seq_offsets, weights, 0, s.layers, out, *hint, ws, L, st, nullptr);
+}
+
+size_t whale_host_workspace_size(const whale_config* cfg, const whale_shape_hint* hint) {
+  Shape s;
+  if (validate(cfg, &s) != WHALE_OK || check_hint(hint) != WHALE_OK) return 0;
+  size_t a, b, c, d, e;
+  return align_up(host_staging_bytes(s, *hint, &a, &b, &c, &d, &e)) + make_layout(s, *hint).total;
+}
+
+whale_status whale_fusion_forward_host(const whale_config* cfg, const void* host_tokens, const void* host_states,
+                                       const int* host_offsets, const whale_layer_weights* weights, void* host_out,
+                                       const whale_shape_hint* hint, void* ws, size_t ws_bytes,
+                                       whale_stream_t stream) {
+  Shape s;
+  WCHECK(validate(cfg, &s));
+  WCHECK(check_hint(hint));
+  size_t o_tok, o_s0, o_s1, o_off, o_out;
+  const size_t staging = align_up(host_staging_bytes(s, *hint, &o_tok, &o_s0, &o_s1, &o_off, &o_out));
+  const Layout L = make_layout(s, *hint);
+  if (!ws || ws_bytes < staging + L.total || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)))
+    return WHALE_ERR_WORKSPACE;
+  if (hint->B == 0) return WHALE_OK;
+  if (!host_tokens || !host_out || !host_offsets || !weights || (hint->total_L > 0 && !host_states))
+    return WHALE_ERR_INVALID_ARG;
+  for (int l = 0; l < s.layers; ++l)
+    if (!weights_ok(s, &weights[l])) return WHALE_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  HostPipe* pipe = nullptr;
+  WCHECK(host_pipe(&pipe));
+  void* fws = at(ws, staging);
+  const size_t rows = (size_t)hint->B * s.N;
+  const size_t tok_bytes = rows * s.d * s.es;
+  const size_t slab_bytes = (size_t)hint->total_L * s.d * s.es;
+  void* d_tok = at(ws, o_tok);
+  void* d_slab[2] = {at(ws, o_s0), at(ws, o_s1)};
+  int* d_off = reinterpret_cast<int*>(at(ws, o_off));
+  void* d_out = at(ws, o_out);
+  CUCHECK(cudaMemcpyAsync(d_off, host_offsets, ((size_t)hint->B + 1) * 4, cudaMemcpyHostToDevice, st));
+  CUCHECK(cudaMemcpyAsync(d_tok, host_tokens, tok_bytes, cudaMemcpyHostToDevice, st));
+  WCHECK(debug_check(s, d_off, *hint, st));
+  // The copy stream starts after everything already queued on `stream` (earlier users of the
+  // staging buffers); slab l+1 is copied while layer l computes, into the other buffer.
+  CUCHECK(cudaEventRecord(pipe->consumed[0], st));
+  CUCHECK(cudaEventRecord(pipe->consumed[1], st));
+  auto copy_slab = [&](int l) -> whale_status {
+    CUCHECK(cudaStreamWaitEvent(pipe->copy, pipe->consumed[l & 1], 0));
+    if (slab_bytes)
+      CUCHECK(cudaMemcpyAsync(d_slab[l & 1], static_cast<const char*>(host_states) + (size_t)l * slab_bytes,
+                              slab_bytes, cudaMemcpyHostToDevice, pipe->copy));
+    CUCHECK(cudaEventRecord(pipe->copied[l & 1], pipe->copy));
+    return WHALE_OK;
+  };
+  WCHECK(copy_slab(0));
+  const void* slabs[64];
+  if (s.layers > 64) return WHALE_ERR_UNSUPPORTED;
+  for (int l = 0; l < s.layers; ++l) slabs[l] = slab_bytes ? d_slab[l & 1] : nullptr;
+  auto hook = [&](int l, bool before) -> whale_status {
+    if (before) {
+      if (l + 1 < s.layers) WCHECK(copy_slab(l + 1));
+      CUCHECK(cudaStreamWaitEvent(st, pipe->copied[l & 1], 0));
+    } else {
+      CUCHECK(cudaEventRecord(pipe->consumed[l & 1], st));
+    }
+    return WHALE_OK;
+  };
+  WCHECK(stack_impl(s, d_tok, nullptr, d_off, weights, 0, s.layers, d_out, *hint, fws, L, st, slabs, hook));
+  CUCHECK(cudaMemcpyAsync(host_out, d_out, tok_bytes, cudaMemcpyDeviceToHost, st));
+  return WHALE_OK;
+}
+
+whale_status whale_project_queries(const whale_config* cfg, long long rows, const void* x, const float* g_q,
+                                   const void* w_q, void* q, void* ws, size_t ws_bytes, whale_stream_t stream) {
+  Shape s;
+  WCHECK(validate(cfg, &s));
+  if (rows < 0 || !x || !g_q || !w_q || !q) return WHALE_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (s.bf16) {
+    if (!ws || ws_bytes < (size_t)s.d * s.d * 2) return WHALE_ERR_WORKSPACE;
+    auto* wq = static_cast<__nv_bfloat16*>(ws);
+    WCHECK(fold_weights(s, static_cast<const __nv_bfloat16*>(w_q), g_q, nullptr, nullptr, nullptr, nullptr, wq, nullptr,
+                        nullptr, st));
+    return gemm_bf16(opnd(x, nullptr, s.d, s.d), no_opnd(), wq, s.d, Outs{q, nullptr, nullptr, s.d}, nullptr, 0, rows,
+                     EPI_STORE, true, s.eps, st);
+  }
+  if (!ws || ws_bytes < (size_t)rows * 4) return WHALE_ERR_WORKSPACE;
+  float* r = static_cast<float*>(ws);
+  WCHECK(row_rms(static_cast<const float*>(x), rows, s.d, s.eps, r, st));
+  return gemm_f32(static_cast<const float*>(x), s.d, nullptr, 0, r, g_q, static_cast<const float*>(w_q), s.d,
+                  static_cast<float*>(q), rows, F32_NONE, nullptr, st);
+}
+
+whale_status whale_project_kv(const whale_config* cfg, long long rows, const void* sx, const float* g_kv,
+                              const void* w_kv, void* kv, void* ws, size_t ws_bytes, whale_stream_t stream) {
+  Shape s;
+  WCHECK(validate(cfg, &s));
+  if (rows < 0 || !sx || !g_kv || !w_kv || !kv) return WHALE_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (s.bf16) {
+    if (!ws || ws_bytes < (size_t)s.kvw * s.d * 2) return WHALE_ERR_WORKSPACE;
+    auto* wkv = static_cast<__nv_bfloat16*>(ws);
+    WCHECK(fold_weights(s, nullptr, nullptr, static_cast<const __nv_bfloat16*>(w_kv), g_kv, nullptr, nullptr, nullptr,
+                        wkv, nullptr, st));
+    return gemm_bf16(opnd(sx, nullptr, s.d, s.d), no_opnd(), wkv, s.kvw, Outs{kv, nullptr, nullptr, s.kvw}, nullptr,
+                     0, rows, EPI_STORE, true, s.eps, st);
+  }
+  if (!ws || ws_bytes < (size_t)rows * 4) return WHALE_ERR_WORKSPACE;
+  float* r = static_cast<float*>(ws);
+  WCHECK(row_rms(static_cast<const float*>(sx), rows, s.d, s.eps, r, st));
+  return gemm_f32(static_cast<const float*>(sx), s.d, nullptr, 0, r, g_kv, static_cast<const float*>(w_kv), s.kvw,
+                  static_cast<float*>(kv), rows, F32_NONE, nullptr, st);
+}
+
+whale_status whale_cross_attention(const whale_config* cfg, const void* q, const void* kv, const int* seq_offsets,
+                                   void* a, const whale_shape_hint* hint, void* ws, size_t ws_bytes,
+                                   whale_stream_t stream) {
+  Shape s;
+  WCHECK(validate(cfg, &s));
+  WCHECK(check_hint(hint));
+  if (hint->B == 0) return WHALE_OK;
+  if (!q || !a || !seq_offsets || (hint->total_L > 0 && !kv)) return WHALE_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (s.bf16) {
+    const AttnPlan p = plan_attention(s, hint->B, hint->total_L);
+    const size_t po = align_up(p.po_elems * 4);
+    if (!ws || ws_bytes < po + p.pml_elems * 4 || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)))
+      return WHALE_ERR_WORKSPACE;
+    WCHECK(debug_check(s, seq_offsets, *hint, st));
+    return attention_bf16(s, q, kv, seq_offsets, a, nullptr, hint->B, hint->max_L, hint->total_L,
+                          static_cast<float*>(ws), reinterpret_cast<float*>(at(ws, po)), st);
+  }
+  WCHECK(debug_check(s, seq_offsets, *hint, st));
+  return attention_f32(s, static_cast<const float*>(q), static_cast<const float*>(kv), seq_offsets,
+                       static_cast<float*>(a), hint->B, hint->total_L, st);
+}
+
+whale_status whale_fusion_mlp(const whale_config* cfg, long long rows, const void* a, const void* x, const void* w_f1,
+                              const void* w_f2, void* f, void* ws, size_t ws_bytes, whale_stream_t stream) {
+  Shape s;
+  WCHECK(validate(cfg, &s));
+  if (rows < 0 || !a || !x || !w_f2 || !f || (s.Fh > 0 && !w_f1)) return WHALE_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (!s.bf16) {
+    if (s.Fh > 0 && (!ws || ws_bytes < (size_t)rows * s.Fh * 4)) return WHALE_ERR_WORKSPACE;
+    return fusion_mlp_f32(s, rows, static_cast<const float*>(a), static_cast<const float*>(x),
+                          static_cast<const float*>(w_f1), static_cast<const float*>(w_f2), static_cast<float*>(f),
+                          static_cast<float*>(ws), st);
+  }
+  // workspace: x (fp32) | zero lo half | G pair
+  const size_t o_z = align_up((size_t)rows * s.d * 4), o_g = o_z + align_up((size_t)rows * s.d * 2);
+  const size_t o_gl = o_g + align_up((size_t)rows * s.Fh * 2), need = o_gl + (size_t)rows * s.Fh * 2;
+  if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1))) return WHALE_ERR_WORKSPACE;
+  auto* x32 = static_cast<float*>(ws);
+  void* zlo = at(ws, o_z);
+  WCHECK(pair_from_bf16(x, x32, zlo, rows * s.d, st));
+  return fusion_bf16(s, rows, opnd(a, zlo, s.d, s.d), opnd(x, zlo, s.d, s.d), x32, w_f1, w_f2, at(ws, o_g),
+                     at(ws, o_gl), Stream3{nullptr, f, nullptr}, st);
+}
+
+whale_status whale_swiglu_ffn(const whale_config* cfg, long long rows, const void* f, const float* g_ffn,
+                              const void* w_upgate, const void* w_down, void* y, void* ws, size_t ws_bytes,
+                              whale_stream_t stream) {
+  Shape s;
+  WCHECK(validate(cfg, &s));
+  if (rows < 0 || !f || !g_ffn || !w_upgate || !w_down || !y) return WHALE_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (s.bf16) {
+    // workspace: folded up|gate | f (fp32) | zero lo half | U pair
+    const size_t o_f = align_up((size_t)s.ugw * s.d * 2), o_z = o_f + align_up((size_t)rows * s.d * 4);
+    const size_t o_u = o_z + align_up((size_t)rows * s.d * 2), o_ul = o_u + align_up((size_t)rows * s.H * 2);
+    const size_t need = o_ul + (size_t)rows * s.H * 2;
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1))) return WHALE_ERR_WORKSPACE;
+    auto* wug = static_cast<__nv_bfloat16*>(ws);
+    WCHECK(fold_weights(s, nullptr, nullptr, nullptr, nullptr, static_cast<const __nv_bfloat16*>(w_upgate), g_ffn,
+                        nullptr, nullptr, wug, st));
+    auto* f32 = reinterpret_cast<float*>(at(ws, o_f));
+    void* zlo = at(ws, o_z);
+    WCHECK(pair_from_bf16(f, f32, zlo, rows * s.d, st));
+    return ffn_bf16(s, rows, opnd(f, zlo, s.d, s.d), f32, wug, w_down, at(ws, o_u), at(ws, o_ul),
+                    Stream3{nullptr, y, nullptr}, st);
+  }
+  const size_t rb = align_up((size_t)rows * 4), ugb = align_up((size_t)rows * s.ugw * 4);
+  if (!ws || ws_bytes < rb + ugb + (size_t)rows * s.H * 4) return WHALE_ERR_WORKSPACE;
+  float* r = static_cast<float*>(ws);
+  float* ug = reinterpret_cast<float*>(at(ws, rb));
+  float* u = reinterpret_cast<float*>(at(ws, rb + ugb));
+  return swiglu_f32(s, static_cast<const float*>(f), g_ffn, static_cast<const float*>(w_upgate),
+                    static_cast<const float*>(w_down), static_cast<float*>(y), rows, r, ug, u, st);
+}
+
+whale_status whale_get_device_error(whale_stream_t stream, int* code) {
+  if (!code) return WHALE_ERR_INVALID_ARG;
+  CUCHECK(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
+  unsigned v = 0, zero = 0;
+  CUCHECK(cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)));
+  CUCHECK(cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)));
+  *code = (int)v;
+  return v ? WHALE_ERR_DEVICE_CHECK : WHALE_OK;
+}
+
+}  // extern "C"

@@ -62,6 +62,7 @@ class Workload:
     fusion_mult: int = 2  # Fusion MLP hidden = fusion_mult * d (0: single linear)
     candidates: int = 0   # serving workload: candidates per request (N = candidates * tokens)
     eps: float = 1e-6
+    weight_seed: int | None = None   # weights' seed when it differs from `seed` (per-rank shards)
 
     @property
     def d_head(self) -> int:
@@ -216,14 +217,15 @@ def make_layer_weights(w: Workload, layer: int, gains: str = "ones", shared_kv: 
     Gains g_q, g_kv, g_ffn are float32 [d]: ones, or U[0.5, 1.5] when gains == "random".
     """
     d, H, Fh = w.d, w.ffn_hidden, w.fusion_hidden
+    wseed = w.seed if w.weight_seed is None else w.weight_seed
 
     def mat(name: str, fan_out: int, fan_in: int) -> np.ndarray:
-        return _store(xavier_uniform(_rng(w.seed, _S_WEIGHTS, layer, _W_IDS[name]), fan_out, fan_in), w.dtype)
+        return _store(xavier_uniform(_rng(wseed, _S_WEIGHTS, layer, _W_IDS[name]), fan_out, fan_in), w.dtype)
 
     def gain(name: str) -> np.ndarray:
         if gains == "ones":
             return np.ones(d, dtype=np.float32)
-        return _rng(w.seed, _S_GAINS, layer, _G_IDS[name]).uniform(0.5, 1.5, size=d).astype(np.float32)
+        return _rng(wseed, _S_GAINS, layer, _G_IDS[name]).uniform(0.5, 1.5, size=d).astype(np.float32)
 
     lw = {"g_q": gain("g_q"), "g_kv": gain("g_kv"), "g_ffn": gain("g_ffn"), "w_q": mat("w_q", d, d)}
     wk = mat("w_k", d, d)

@@ -1,0 +1,233 @@
+"""Thin ctypes binding of libwhale_fusion.so (include/whale_fusion.h), same names.
+
+Argument marshalling only: every step of the forward runs in the library's CUDA kernels.
+Tensors are torch tensors (device memory and streams come from PyTorch); a plain int is
+taken as a raw pointer. Importing this module loads the library and raises ImportError
+if it has not been built (python -m wukong_hstu_cross_b200.build) — there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from ctypes import POINTER, c_float, c_int, c_longlong, c_size_t, c_uint, c_void_p
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwhale_fusion.so")
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "whale_fusion.h")
+
+WHALE_FP32, WHALE_BF16 = 0, 1
+WHALE_SHARED_KV, WHALE_TIED_GATE, WHALE_DEBUG = 1, 2, 4
+WHALE_DEVERR_TIMEOUT, WHALE_DEVERR_OFFSETS = 1, 2
+STATUS = {0: "WHALE_OK", 1: "WHALE_ERR_INVALID_ARG", 2: "WHALE_ERR_UNSUPPORTED", 3: "WHALE_ERR_CUDA",
+          4: "WHALE_ERR_WORKSPACE", 5: "WHALE_ERR_DEVICE_CHECK"}
+
+
+class whale_config(ctypes.Structure):
+    _fields_ = [("n_layers", c_int), ("d", c_int), ("n_heads", c_int), ("n_tokens", c_int),
+                ("ffn_hidden", c_int), ("fusion_hidden", c_int), ("dtype", c_int), ("flags", c_uint),
+                ("eps", c_float)]
+
+
+_WNAMES = ("g_q", "g_kv", "w_q", "w_kv", "w_f1", "w_f2", "g_ffn", "w_upgate", "w_down")
+
+
+class whale_layer_weights(ctypes.Structure):
+    _fields_ = [(n, c_void_p) for n in _WNAMES]
+
+
+class whale_shape_hint(ctypes.Structure):
+    _fields_ = [("B", c_int), ("max_L", c_int), ("total_L", c_longlong)]
+
+
+class WhaleError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+        self.status = status
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m wukong_hstu_cross_b200.build`")
+_lib = ctypes.CDLL(LIB_PATH)
+
+_P = c_void_p
+_SIGS = {
+    "whale_status_string": ([c_int], ctypes.c_char_p),
+    "whale_workspace_size": ([POINTER(whale_config), POINTER(whale_shape_hint)], c_size_t),
+    "whale_host_workspace_size": ([POINTER(whale_config), POINTER(whale_shape_hint)], c_size_t),
+    "whale_fusion_forward": ([POINTER(whale_config), _P, _P, _P, POINTER(whale_layer_weights), _P,
+                              POINTER(whale_shape_hint), _P, c_size_t, _P], c_int),
+    "whale_fusion_forward_host": ([POINTER(whale_config), _P, _P, _P, POINTER(whale_layer_weights), _P,
+                                   POINTER(whale_shape_hint), _P, c_size_t, _P], c_int),
+    "whale_fusion_layer_forward": ([POINTER(whale_config), _P, _P, _P, POINTER(whale_layer_weights), _P,
+                                    POINTER(whale_shape_hint), _P, c_size_t, _P], c_int),
+    "whale_project_queries": ([POINTER(whale_config), c_longlong, _P, _P, _P, _P, _P, c_size_t, _P], c_int),
+    "whale_project_kv": ([POINTER(whale_config), c_longlong, _P, _P, _P, _P, _P, c_size_t, _P], c_int),
+    "whale_cross_attention": ([POINTER(whale_config), _P, _P, _P, _P, POINTER(whale_shape_hint), _P, c_size_t,
+                               _P], c_int),
+    "whale_fusion_mlp": ([POINTER(whale_config), c_longlong, _P, _P, _P, _P, _P, _P, c_size_t, _P], c_int),
+    "whale_swiglu_ffn": ([POINTER(whale_config), c_longlong, _P, _P, _P, _P, _P, _P, c_size_t, _P], c_int),
+    "whale_get_device_error": ([_P, POINTER(c_int)], c_int),
+}
+for _name, (_args, _res) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.argtypes, _f.restype = _args, _res
+
+
+def header_functions() -> list:
+    """Names of the functions include/whale_fusion.h declares."""
+    with open(HEADER) as fh:
+        text = fh.read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(whale_\w+)\s*\(", text, flags=re.M)))
+
+
+# ------------------------------------------------------------------------------------------------
+# marshalling helpers
+# ------------------------------------------------------------------------------------------------
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise WhaleError(status, where)
+
+
+def make_config(n_layers, d, n_heads, n_tokens, ffn_hidden, fusion_hidden, dtype, flags=0, eps=1e-6) -> whale_config:
+    return whale_config(n_layers, d, n_heads, n_tokens, ffn_hidden, fusion_hidden, dtype, flags, eps)
+
+
+def make_hint(B, max_L, total_L) -> whale_shape_hint:
+    return whale_shape_hint(int(B), int(max_L), int(total_L))
+
+
+def layer_weights(lw) -> whale_layer_weights:
+    """A whale_layer_weights from a dict of tensors (None allowed for w_f1)."""
+    if isinstance(lw, whale_layer_weights):
+        return lw
+    return whale_layer_weights(*[_ptr(lw.get(n)) for n in _WNAMES])
+
+
+def weights_array(layers) -> ctypes.Array:
+    arr = (whale_layer_weights * len(layers))()
+    for i, lw in enumerate(layers):
+        arr[i] = layer_weights(lw)
+    return arr
+
+
+# ------------------------------------------------------------------------------------------------
+# entry points (same names as the C ABI)
+# ------------------------------------------------------------------------------------------------
+def whale_status_string(status: int) -> str:
+    return _lib.whale_status_string(status).decode()
+
+
+def whale_workspace_size(cfg: whale_config, hint: whale_shape_hint) -> int:
+    return int(_lib.whale_workspace_size(ctypes.byref(cfg), ctypes.byref(hint)))
+
+
+def whale_host_workspace_size(cfg: whale_config, hint: whale_shape_hint) -> int:
+    return int(_lib.whale_host_workspace_size(ctypes.byref(cfg), ctypes.byref(hint)))
+
+
+def _ws_bytes(workspace, nbytes):
+    if nbytes is not None:
+        return int(nbytes)
+    if workspace is None:
+        return 0
+    return workspace.numel() * workspace.element_size()
+
+
+def whale_fusion_forward(cfg, wukong_tokens, seq_states, seq_offsets, weights, out, hint, workspace,
+                         workspace_bytes=None, stream=None, raw=False):
+    w = weights if isinstance(weights, ctypes.Array) else weights_array(weights)
+    st = _lib.whale_fusion_forward(ctypes.byref(cfg), _ptr(wukong_tokens), _ptr(seq_states), _ptr(seq_offsets), w,
+                                   _ptr(out), ctypes.byref(hint), _ptr(workspace),
+                                   _ws_bytes(workspace, workspace_bytes), _stream(stream))
+    if raw:
+        return st
+    _check(st, "whale_fusion_forward")
+
+
+def whale_fusion_forward_host(cfg, host_tokens, host_seq_states, host_offsets, weights, host_out, hint, workspace,
+                              workspace_bytes=None, stream=None, raw=False):
+    w = weights if isinstance(weights, ctypes.Array) else weights_array(weights)
+    st = _lib.whale_fusion_forward_host(ctypes.byref(cfg), _ptr(host_tokens), _ptr(host_seq_states),
+                                        _ptr(host_offsets), w, _ptr(host_out), ctypes.byref(hint), _ptr(workspace),
+                                        _ws_bytes(workspace, workspace_bytes), _stream(stream))
+    if raw:
+        return st
+    _check(st, "whale_fusion_forward_host")
+
+
+def whale_fusion_layer_forward(cfg, tokens_in, layer_states, seq_offsets, layer_weights_, tokens_out, hint, workspace,
+                               workspace_bytes=None, stream=None, raw=False):
+    lw = layer_weights(layer_weights_)
+    st = _lib.whale_fusion_layer_forward(ctypes.byref(cfg), _ptr(tokens_in), _ptr(layer_states), _ptr(seq_offsets),
+                                         ctypes.byref(lw), _ptr(tokens_out), ctypes.byref(hint), _ptr(workspace),
+                                         _ws_bytes(workspace, workspace_bytes), _stream(stream))
+    if raw:
+        return st
+    _check(st, "whale_fusion_layer_forward")
+
+
+def whale_project_queries(cfg, rows, x, g_q, w_q, q, workspace, workspace_bytes=None, stream=None, raw=False):
+    st = _lib.whale_project_queries(ctypes.byref(cfg), int(rows), _ptr(x), _ptr(g_q), _ptr(w_q), _ptr(q),
+                                    _ptr(workspace), _ws_bytes(workspace, workspace_bytes), _stream(stream))
+    if raw:
+        return st
+    _check(st, "whale_project_queries")
+
+
+def whale_project_kv(cfg, rows, s, g_kv, w_kv, kv, workspace, workspace_bytes=None, stream=None, raw=False):
+    st = _lib.whale_project_kv(ctypes.byref(cfg), int(rows), _ptr(s), _ptr(g_kv), _ptr(w_kv), _ptr(kv),
+                               _ptr(workspace), _ws_bytes(workspace, workspace_bytes), _stream(stream))
+    if raw:
+        return st
+    _check(st, "whale_project_kv")
+
+
+def whale_cross_attention(cfg, q, kv, seq_offsets, a, hint, workspace, workspace_bytes=None, stream=None, raw=False):
+    st = _lib.whale_cross_attention(ctypes.byref(cfg), _ptr(q), _ptr(kv), _ptr(seq_offsets), _ptr(a),
+                                    ctypes.byref(hint), _ptr(workspace), _ws_bytes(workspace, workspace_bytes),
+                                    _stream(stream))
+    if raw:
+        return st
+    _check(st, "whale_cross_attention")
+
+
+def whale_fusion_mlp(cfg, rows, a, x, w_f1, w_f2, f, workspace, workspace_bytes=None, stream=None, raw=False):
+    st = _lib.whale_fusion_mlp(ctypes.byref(cfg), int(rows), _ptr(a), _ptr(x), _ptr(w_f1), _ptr(w_f2), _ptr(f),
+                               _ptr(workspace), _ws_bytes(workspace, workspace_bytes), _stream(stream))
+    if raw:
+        return st
+    _check(st, "whale_fusion_mlp")
+
+
+def whale_swiglu_ffn(cfg, rows, f, g_ffn, w_upgate, w_down, y, workspace, workspace_bytes=None, stream=None,
+                     raw=False):
+    st = _lib.whale_swiglu_ffn(ctypes.byref(cfg), int(rows), _ptr(f), _ptr(g_ffn), _ptr(w_upgate), _ptr(w_down),
+                               _ptr(y), _ptr(workspace), _ws_bytes(workspace, workspace_bytes), _stream(stream))
+    if raw:
+        return st
+    _check(st, "whale_swiglu_ffn")
+
+
+def whale_get_device_error(stream=None) -> int:
+    code = c_int(0)
+    st = _lib.whale_get_device_error(_stream(stream), ctypes.byref(code))
+    if st not in (0, 5):
+        _check(st, "whale_get_device_error")
+    return code.value
