@@ -95,7 +95,9 @@ def test_layer_entry_point_and_batch_reordering():
     torch.cuda.synchronize()
     assert torch.equal(y, out)
     _check(p, y)
-    # reorder the examples (same total and max length): each example's output follows it exactly
+    # reorder the examples (same total and max length): each example's output follows it. The
+    # attention's load-balanced split points depend on where an example sits in the batch, so the
+    # order of the fp32 partial merges (not the result) may change: compare within 1e-2*(1+|y|).
     perm = np.array([3, 0, 4, 2, 1])
     L2 = p.lengths[perm]
     off2 = I.offsets_of(L2)
@@ -105,7 +107,8 @@ def test_layer_entry_point_and_batch_reordering():
     y2 = torch.empty_like(tok2)
     W.whale_fusion_forward(p.cfg, tok2, states2, torch.from_numpy(off2).cuda(), p.weights, y2, p.hint, p.workspace)
     torch.cuda.synchronize()
-    assert torch.equal(y2, out[torch.from_numpy(perm).cuda()])
+    ref = out[torch.from_numpy(perm).cuda()].float()
+    assert bool(((y2.float() - ref).abs() <= 1e-2 * (1 + ref.abs())).all())
 
 
 def test_host_buffer_entry_point_matches_device_entry_point():

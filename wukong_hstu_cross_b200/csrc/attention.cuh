@@ -14,7 +14,9 @@
 // m, sum l and unnormalised output o in registers (online softmax in base 2), computing q k^T
 // and p v with warp-level bf16 tensor-core MMAs fed by ldmatrix from the swizzled stages; row
 // max / sum reductions are warp shuffles across the 4 threads that share a query row. A last
-// warp issues the TMA. attn_combine merges the partials of each item with log-sum-exp.
+// warp issues the TMA. An item that lies inside one slice is finished in place; otherwise every
+// slice writes a partial, counts itself done on the item's counter, and the CTA that completes
+// the item merges the partials with log-sum-exp and writes A (no separate combine pass).
 // At the workloads' query counts the path is HBM-bound (N flops per byte of K|V); the tensor
 // cores only need to keep up with the stream.
 #pragma once
@@ -39,6 +41,9 @@ struct AttnArgs {
   int G;                   // CTAs per head group in the flattened schedule
   long long total_L;       // rows of the kv tensor
   float scale_log2;        // log2(e) / sqrt(DH)
+  int* counters;           // [B * n_qblocks] finished-slice counts, zero at launch
+  __nv_bfloat16* out;      // A [B*N, d] (bf16)
+  __nv_bfloat16* out_lo;   // bf16 residue of A (may be null)
 };
 
 // Offsets clamped into the slab [0, total_L]: example b owns rows [lo_b, hi_b).
@@ -96,6 +101,27 @@ __device__ __forceinline__ bool attn_next_segment(const AttnArgs& a, long long& 
   return true;
 }
 
+// CTA whose slice contains flat position p.
+__device__ __forceinline__ int attn_cta_of(long long p, long long P0, long long W, int G) {
+  int c = (int)(((p - P0) * G) / W);
+  if (c < 0) c = 0;
+  if (c > G - 1) c = G - 1;
+  while (c + 1 < G && slice_start(P0, W, G, c + 1) <= p) ++c;
+  while (c > 0 && slice_start(P0, W, G, c) > p) --c;
+  return c;
+}
+
+// Number of CTAs whose (non-empty) slices hold rows of an item that starts at flat position F and
+// has L rows, and the first / last of them.
+__device__ __forceinline__ int attn_item_ctas(long long F, long long L, long long P0, long long W, int G, int& c0,
+                                              int& c1) {
+  c0 = attn_cta_of(F, P0, W, G);
+  c1 = attn_cta_of(F + L - 1, P0, W, G);
+  int n = 0;
+  for (int k = c0; k <= c1; ++k) n += slice_start(P0, W, G, k) < slice_start(P0, W, G, k + 1);
+  return n;
+}
+
 template <int DH, int QT, int T, int HG>
 struct AttnCfg {
   static constexpr int NBOX = HG * DH / 64;           // 64-column TMA boxes per K (or V) tile
@@ -117,9 +143,24 @@ __global__ void __launch_bounds__(32 * (HG + 1), 1)
   uint64_t* empty = full + STAGES;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + STAGES);
 
+  volatile int* last_flag = reinterpret_cast<volatile int*>(empty + STAGES) + 1;
+
   const int cta = blockIdx.x, hg = blockIdx.y;
   long long P0, W;
   flat_extent(a, P0, W);
+  // Items with an empty history get A = 0 here (no slice covers them).
+  for (int item = cta; item < a.B * a.n_qblocks; item += a.G) {
+    const int b = item / a.n_qblocks, qb = item % a.n_qblocks;
+    if (clamp_off(a, b + 1) > clamp_off(a, b)) continue;
+    for (int idx = threadIdx.x; idx < a.QB * HG * DH; idx += blockDim.x) {
+      const int nl = idx / (HG * DH), col = hg * HG * DH + idx % (HG * DH);
+      const int n = qb * a.QB + nl;
+      if (n >= a.N) continue;
+      const long long oi = ((long long)b * a.N + n) * a.d + col;
+      a.out[oi] = __float2bfloat16_rn(0.f);
+      if (a.out_lo) a.out_lo[oi] = __float2bfloat16_rn(0.f);
+    }
+  }
   const long long p_begin = slice_start(P0, W, a.G, cta), p_end = slice_start(P0, W, a.G, cta + 1);
   if (p_begin >= p_end) return;  // uniform across the CTA
 
@@ -245,9 +286,14 @@ __global__ void __launch_bounds__(32 * (HG + 1), 1)
         }
       }
 
-      // online softmax (base 2); rows past the segment end are masked out
+      // online softmax (base 2); rows past the segment end are masked out. The reference max
+      // m_run (scaled log2 units) moves only when some row's max exceeds it by more than 8, so the
+      // O / l rescale is skipped on most tiles; p = 2^(s*scale - m_run) <= 2^8 stays exact in fp32
+      // and well inside bf16 range. The decision is warp-uniform.
       const bool partial = trow0 + T > sg.t1;
       uint32_t pa[QT][T / 16][4];
+      float mxs[QT][2];
+      bool need = false;
 #pragma unroll
       for (int mt = 0; mt < QT; ++mt) {
 #pragma unroll
@@ -257,33 +303,49 @@ __global__ void __launch_bounds__(32 * (HG + 1), 1)
           for (int nt = 0; nt < T / 8; ++nt) {
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-              float v = sc[mt][nt][2 * hr + j] * a.scale_log2;
-              if (partial && trow0 + nt * 8 + 2 * qd + j >= sg.t1) v = -INFINITY;
-              sc[mt][nt][2 * hr + j] = v;
-              mx = fmaxf(mx, v);
+              if (partial && trow0 + nt * 8 + 2 * qd + j >= sg.t1) sc[mt][nt][2 * hr + j] = -INFINITY;
+              mx = fmaxf(mx, sc[mt][nt][2 * hr + j]);
             }
           }
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-          const float m_new = fmaxf(m_run[mt][hr], mx);
-          const float corr = fast_exp2(m_run[mt][hr] - m_new);
-          m_run[mt][hr] = m_new;
+          mxs[mt][hr] = mx * a.scale_log2;
+          need |= mxs[mt][hr] > m_run[mt][hr] + 8.0f;
+        }
+      }
+      if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+        for (int mt = 0; mt < QT; ++mt) {
+#pragma unroll
+          for (int hr = 0; hr < 2; ++hr) {
+            const float m_new = fmaxf(m_run[mt][hr], mxs[mt][hr]);
+            const float corr = fast_exp2(m_run[mt][hr] - m_new);
+            m_run[mt][hr] = m_new;
+            l_run[mt][hr] *= corr;
+#pragma unroll
+            for (int nt = 0; nt < DH / 8; ++nt) {
+              o[mt][nt][2 * hr] *= corr;
+              o[mt][nt][2 * hr + 1] *= corr;
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int mt = 0; mt < QT; ++mt) {
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          const float neg_m = -m_run[mt][hr];
           float sum = 0.f;
 #pragma unroll
           for (int nt = 0; nt < T / 8; ++nt) {
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-              const float pv = fast_exp2(sc[mt][nt][2 * hr + j] - m_new);
+              const float pv = fast_exp2(fmaf(sc[mt][nt][2 * hr + j], a.scale_log2, neg_m));
               sc[mt][nt][2 * hr + j] = pv;
               sum += pv;
             }
           }
-          l_run[mt][hr] = l_run[mt][hr] * corr + sum;
-#pragma unroll
-          for (int nt = 0; nt < DH / 8; ++nt) {
-            o[mt][nt][2 * hr] *= corr;
-            o[mt][nt][2 * hr + 1] *= corr;
-          }
+          l_run[mt][hr] += sum;
         }
 #pragma unroll
         for (int kt = 0; kt < T / 16; ++kt) {
@@ -317,87 +379,116 @@ __global__ void __launch_bounds__(32 * (HG + 1), 1)
     }
     if (!ok) break;
 
-    // partial of this segment: slot = item + cta (unique and increasing along the slices)
-    const long long slot = (long long)sg.item + cta;
+    // ---- end of a segment: quad-reduced row sums, then either the final A (the item lies in this
+    // CTA's slice alone) or a partial; the CTA that completes an item merges all of its partials.
+    float lq[QT][2];
 #pragma unroll
-    for (int mt = 0; mt < QT; ++mt) {
+    for (int mt = 0; mt < QT; ++mt)
 #pragma unroll
       for (int hr = 0; hr < 2; ++hr) {
         float l = l_run[mt][hr];
         l += __shfl_xor_sync(0xffffffffu, l, 1);
         l += __shfl_xor_sync(0xffffffffu, l, 2);
-        const int nl = mt * 16 + g + 8 * hr;
-        if (sg.qb * a.QB + nl >= a.N) continue;
-        const long long base = (slot * a.n_heads + head) * a.QB + nl;
-        if (qd == 0) {
-          a.part_ml[2 * base] = m_run[mt][hr];
-          a.part_ml[2 * base + 1] = l;
-        }
-        float* po = a.part_o + base * DH;
+        lq[mt][hr] = l;
+      }
+    const long long lo_b = clamp_off(a, sg.b);
+    const long long Lb = clamp_off(a, sg.b + 1) - lo_b;
+    int c0, c1;
+    const int nseg = attn_item_ctas((long long)a.n_qblocks * lo_b + (long long)sg.qb * Lb, Lb, P0, W, a.G, c0, c1);
+    bool finish = nseg <= 1;
+    if (!finish) {
+      // partial of this segment: slot = item + cta (unique and increasing along the slices)
+      const long long slot = (long long)sg.item + cta;
 #pragma unroll
-        for (int nt = 0; nt < DH / 8; ++nt)
-          *reinterpret_cast<float2*>(po + nt * 8 + 2 * qd) = make_float2(o[mt][nt][2 * hr], o[mt][nt][2 * hr + 1]);
+      for (int mt = 0; mt < QT; ++mt) {
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          const int nl = mt * 16 + g + 8 * hr;
+          if (sg.qb * a.QB + nl >= a.N) continue;
+          const long long base = (slot * a.n_heads + head) * a.QB + nl;
+          if (qd == 0) {
+            a.part_ml[2 * base] = m_run[mt][hr];
+            a.part_ml[2 * base + 1] = lq[mt][hr];
+          }
+          float* po = a.part_o + base * DH;
+#pragma unroll
+          for (int nt = 0; nt < DH / 8; ++nt)
+            *reinterpret_cast<float2*>(po + nt * 8 + 2 * qd) = make_float2(o[mt][nt][2 * hr], o[mt][nt][2 * hr + 1]);
+        }
+      }
+      __threadfence();
+      asm volatile("bar.sync 1, %0;" ::"n"(HG * 32) : "memory");  // compute warps only
+      if (threadIdx.x == 0) {
+        const int prev = atomicAdd(a.counters + sg.item, 1);
+        *last_flag = (prev == nseg - 1);
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(HG * 32) : "memory");
+      finish = *last_flag != 0;
+      if (finish) {
+        __threadfence();
+        // Merge every slice's partial (this CTA's own included, re-read) in slot order from an
+        // empty state, so the result does not depend on which CTA finishes the item. Partials
+        // written by other SMs are read through L2.
+#pragma unroll
+        for (int mt = 0; mt < QT; ++mt)
+#pragma unroll
+          for (int hr = 0; hr < 2; ++hr) {
+            m_run[mt][hr] = -INFINITY;
+            lq[mt][hr] = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < DH / 8; ++nt) o[mt][nt][2 * hr] = o[mt][nt][2 * hr + 1] = 0.f;
+          }
+        for (int k = c0; k <= c1; ++k) {
+          if (slice_start(P0, W, a.G, k) >= slice_start(P0, W, a.G, k + 1)) continue;
+          const long long slot_k = (long long)sg.item + k;
+#pragma unroll
+          for (int mt = 0; mt < QT; ++mt) {
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+              const int nl = mt * 16 + g + 8 * hr;
+              if (sg.qb * a.QB + nl >= a.N) continue;
+              const long long base = (slot_k * a.n_heads + head) * a.QB + nl;
+              const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part_ml + 2 * base));
+              const float m_new = fmaxf(m_run[mt][hr], ml.x);
+              const float w_acc = fast_exp2(m_run[mt][hr] - m_new), w_k = fast_exp2(ml.x - m_new);
+              m_run[mt][hr] = m_new;
+              lq[mt][hr] = lq[mt][hr] * w_acc + ml.y * w_k;
+              const float* po = a.part_o + base * DH;
+#pragma unroll
+              for (int nt = 0; nt < DH / 8; ++nt) {
+                const float2 ov = __ldcg(reinterpret_cast<const float2*>(po + nt * 8 + 2 * qd));
+                o[mt][nt][2 * hr] = o[mt][nt][2 * hr] * w_acc + ov.x * w_k;
+                o[mt][nt][2 * hr + 1] = o[mt][nt][2 * hr + 1] * w_acc + ov.y * w_k;
+              }
+            }
+          }
+        }
       }
     }
-  }
-}
-
-// CTA whose slice contains flat position p.
-__device__ __forceinline__ int attn_cta_of(long long p, long long P0, long long W, int G) {
-  int c = (int)(((p - P0) * G) / W);
-  if (c < 0) c = 0;
-  if (c > G - 1) c = G - 1;
-  while (c + 1 < G && slice_start(P0, W, G, c + 1) <= p) ++c;
-  while (c > 0 && slice_start(P0, W, G, c) > p) --c;
-  return c;
-}
-
-// Merge the segments of each item: m* = max m_s, o = sum 2^(m_s - m*) o_s / sum 2^(m_s - m*) l_s.
-// grid = (item, head); empty histories give 0. Writes bf16 `out` and, if out_lo is not null,
-// the bf16 residue out_lo = bf16(o - out) (the pair carries ~16 mantissa bits).
-template <int DH>
-__global__ void attn_combine_kernel(const AttnArgs a, __nv_bfloat16* out, __nv_bfloat16* out_lo) {
-  const int item = blockIdx.x, head = blockIdx.y;
-  const int b = item / a.n_qblocks, qb = item % a.n_qblocks;
-  long long P0, W;
-  flat_extent(a, P0, W);
-  const long long lo_b = clamp_off(a, b);
-  long long hi_b = clamp_off(a, b + 1);
-  if (hi_b < lo_b) hi_b = lo_b;
-  const long long L = hi_b - lo_b;
-  int c0 = 0, c1 = -1;
-  if (L > 0 && W > 0) {
-    const long long F = (long long)a.n_qblocks * lo_b + (long long)qb * L;
-    c0 = attn_cta_of(F, P0, W, a.G);
-    c1 = attn_cta_of(F + L - 1, P0, W, a.G);
-  }
-  for (int idx = threadIdx.x; idx < a.QB * DH; idx += blockDim.x) {
-    const int nl = idx / DH, c = idx % DH;
-    const int n = qb * a.QB + nl;
-    if (n >= a.N) continue;
-    float res = 0.f;
-    if (c1 >= c0) {
-      // (CTAs with an empty slice, possible when W < G, wrote nothing and are skipped)
-      float mmax = -INFINITY;
-      for (int k = c0; k <= c1; ++k) {
-        if (slice_start(P0, W, a.G, k) >= slice_start(P0, W, a.G, k + 1)) continue;
-        const long long base = (((long long)item + k) * a.n_heads + head) * a.QB + nl;
-        mmax = fmaxf(mmax, a.part_ml[2 * base]);
+    if (finish) {
+      // A = o / l as bf16 (and its bf16 residue)
+#pragma unroll
+      for (int mt = 0; mt < QT; ++mt) {
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          const int nl = mt * 16 + g + 8 * hr;
+          const int n = sg.qb * a.QB + nl;
+          if (n >= a.N) continue;
+          const float inv = 1.0f / lq[mt][hr];
+          const long long row = ((long long)sg.b * a.N + n) * a.d + head * DH;
+#pragma unroll
+          for (int nt = 0; nt < DH / 8; ++nt) {
+            const float x0 = o[mt][nt][2 * hr] * inv, x1 = o[mt][nt][2 * hr + 1] * inv;
+            const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+            *reinterpret_cast<__nv_bfloat162*>(a.out + row + nt * 8 + 2 * qd) = h;
+            if (a.out_lo) {
+              const float2 hf = __bfloat1622float2(h);
+              *reinterpret_cast<uint32_t*>(a.out_lo + row + nt * 8 + 2 * qd) = pack_bf16x2(x0 - hf.x, x1 - hf.y);
+            }
+          }
+        }
       }
-      float l = 0.f, acc = 0.f;
-      for (int k = c0; k <= c1; ++k) {
-        if (slice_start(P0, W, a.G, k) >= slice_start(P0, W, a.G, k + 1)) continue;
-        const long long base = (((long long)item + k) * a.n_heads + head) * a.QB + nl;
-        const float w = fast_exp2(a.part_ml[2 * base] - mmax);
-        l += w * a.part_ml[2 * base + 1];
-        acc += w * a.part_o[base * DH + c];
-      }
-      res = acc / l;
     }
-    const long long oi = ((long long)b * a.N + n) * a.d + head * DH + c;
-    const __nv_bfloat16 hi = __float2bfloat16_rn(res);
-    out[oi] = hi;
-    if (out_lo) out_lo[oi] = __float2bfloat16_rn(res - __bfloat162float(hi));
   }
 }
 

@@ -21,21 +21,38 @@ struct FoldJobs {
   int n;
 };
 
+// One thread per 8 consecutive columns (16-byte loads and stores; cols % 8 == 0).
 __global__ void fold_weights_kernel(const FoldJobs jobs) {
   if ((int)blockIdx.y >= jobs.n) return;
   const FoldJob j = jobs.job[blockIdx.y];
-  const long long total = (long long)j.rows * j.cols;
-  for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
-       idx += (long long)gridDim.x * blockDim.x) {
-    const int r = (int)(idx / j.cols), c = (int)(idx % j.cols);
+  const int cols8 = j.cols >> 3;
+  const int total8 = j.rows * cols8;
+  for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < total8; idx += gridDim.x * blockDim.x) {
+    const int r = idx / cols8, c8 = idx - r * cols8;
     int src = r;
     if (j.mode == 1) {
       const int p = r >> 5, w = r & 31;
       src = (w < 16) ? (16 * p + w) : (j.H + 16 * p + (w - 16));
     }
-    float v = __bfloat162float(j.w[(long long)src * j.cols + c]);
-    if (j.g) v *= j.g[c];
-    j.out[idx] = __float2bfloat16_rn(v);
+    const uint4 wv = *reinterpret_cast<const uint4*>(j.w + (size_t)src * j.cols + c8 * 8);
+    const __nv_bfloat162* wh = reinterpret_cast<const __nv_bfloat162*>(&wv);
+    float g[8];
+    if (j.g) {
+      const float4 g0 = *reinterpret_cast<const float4*>(j.g + c8 * 8);
+      const float4 g1 = *reinterpret_cast<const float4*>(j.g + c8 * 8 + 4);
+      g[0] = g0.x; g[1] = g0.y; g[2] = g0.z; g[3] = g0.w; g[4] = g1.x; g[5] = g1.y; g[6] = g1.z; g[7] = g1.w;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) g[i] = 1.f;
+    }
+    uint4 ov;
+    uint32_t* op = reinterpret_cast<uint32_t*>(&ov);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(wh[i]);
+      op[i] = pack_bf16x2(f.x * g[2 * i], f.y * g[2 * i + 1]);
+    }
+    *reinterpret_cast<uint4*>(j.out + (size_t)idx * 8) = ov;
   }
 }
 

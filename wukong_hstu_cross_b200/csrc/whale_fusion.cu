@@ -19,6 +19,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <functional>
 #include <mutex>
@@ -26,6 +27,7 @@
 #include "aux_kernels.cuh"
 #include "attention.cuh"
 #include "fp32_path.cuh"
+#include "gemm_2sm.cuh"
 #include "gemm_persistent.cuh"
 #include "gemm_tc.cuh"
 #include "ptx.cuh"
@@ -49,6 +51,11 @@ namespace {
   } while (0)
 
 constexpr int kNumSM = 148;
+// The 2-SM (cta_group::2) K|V GEMM is opt-in: WHALE_GEMM_2SM=1 in the environment (read per call).
+inline bool gemm_2sm_enabled() {
+  const char* e = std::getenv("WHALE_GEMM_2SM");
+  return e && e[0] == '1';
+}
 constexpr size_t kAlign = 256;
 inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 template <class T>
@@ -140,7 +147,12 @@ whale_status check_hint(const whale_shape_hint* h) {
 // ------------------------------------------------------------------------------------------
 struct AttnPlan {
   int QT, QB, nqb, T, HG, G;
-  size_t po_elems, pml_elems;
+  size_t po_elems, pml_elems, cnt_elems;
+  // scratch layout: partial o | partial (m, l) | per-item counters
+  size_t po_off() const { return 0; }
+  size_t pml_off() const { return align_up(po_elems * 4); }
+  size_t cnt_off() const { return pml_off() + align_up(pml_elems * 4); }
+  size_t bytes() const { return cnt_off() + cnt_elems * 4; }
 };
 
 AttnPlan plan_attention(const Shape& s, int B, long long total_L) {
@@ -160,6 +172,7 @@ AttnPlan plan_attention(const Shape& s, int B, long long total_L) {
   const size_t slots = (size_t)B * p.nqb + p.G;
   p.pml_elems = slots * s.h * p.QB * 2;
   p.po_elems = slots * s.h * p.QB * s.dh;
+  p.cnt_elems = (size_t)B * p.nqb;
   return p;
 }
 
@@ -191,8 +204,8 @@ Layout make_layout(const Shape& s, const whale_shape_hint& hint) {
     L.wkv = take((size_t)s.kvw * s.d * 2);
     L.wug = take((size_t)s.ugw * s.d * 2);
     AttnPlan p = plan_attention(s, hint.B, hint.total_L);
-    L.po = take(p.po_elems * 4);
-    L.pml = take(p.pml_elems * 4);
+    L.po = take(p.bytes());
+    L.pml = 0;
   } else {
     L.r = take((rows > tl ? rows : tl) * 4);
   }
@@ -278,6 +291,59 @@ whale_status launch_persistent_t(const CUtensorMap& ta, const CUtensorMap& tb, c
   return WHALE_OK;
 }
 
+// Co-resident 2-CTA clusters of the 2-SM GEMM on the current device (cached per device).
+whale_status g2_max_pairs(int* pairs) {
+  static std::mutex mu;
+  static int cache[64];
+  int dev = 0;
+  CUCHECK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return WHALE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(mu);
+  if (cache[dev] == 0) {
+    auto kern = gemm_rownorm_2sm_kernel;
+    CUCHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)G2Smem::BYTES));
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(2 * kNumSM / 2, 1, 1);
+    lc.blockDim = dim3(kG2Threads, 1, 1);
+    lc.dynamicSmemBytes = G2Smem::BYTES;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    int n = 0;
+    CUCHECK(cudaOccupancyMaxActiveClusters(&n, kern, &lc));
+    cache[dev] = n > 0 ? n : -1;
+  }
+  *pairs = cache[dev];
+  return WHALE_OK;
+}
+
+// out = r(A) * (A W^T) in bf16 on 256 x 256 tiles, one persistent CTA pair per two SMs.
+whale_status gemm_rownorm_2sm(const Opnd& a0, const void* W, int N, const Outs& out, long long M, float eps,
+                              int pairs, cudaStream_t st) {
+  CUtensorMap ta, tb, to;
+  WCHECK(tmap_bf16(&ta, a0.hi, M, a0.K, a0.ld, 128));
+  WCHECK(tmap_bf16(&tb, W, N, a0.K, a0.K, 128));
+  WCHECK(tmap_bf16(&to, out.hi, M, N, out.ld, 32));
+  G2Args g{};
+  g.M = (int)M;
+  g.N = N;
+  g.kb = a0.K / 64;
+  g.tiles_n = N / 256;
+  g.num_tiles = (int)(cdiv<long long>(M, 256) * g.tiles_n);
+  g.inv_k = 1.0f / (float)a0.K;
+  g.eps = eps;
+  if (pairs > g.num_tiles) pairs = g.num_tiles;
+  auto kern = gemm_rownorm_2sm_kernel;
+  CUCHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)G2Smem::BYTES));
+  kern<<<2 * pairs, kG2Threads, G2Smem::BYTES, st>>>(ta, tb, to, g);
+  CUCHECK(cudaGetLastError());
+  return WHALE_OK;
+}
+
 // out = r(A) * (A W^T) in bf16, persistent over 128 x BN tiles (BN = 256 when N allows).
 whale_status gemm_rownorm_persistent(const Opnd& a0, const void* W, int N, const Outs& out, long long M, float eps,
                                      cudaStream_t st) {
@@ -308,8 +374,12 @@ whale_status gemm_bf16(const Opnd& a0, const Opnd& a1, const void* W, int N, con
   const long long tm = cdiv<long long>(M, 128);
   // Large single-source row-norm projections (the history-side K|V GEMM): persistent kernel.
   if (!split && rn && epi == EPI_STORE && a1.K == 0 && out.hi && !out.lo && !out.f32 && N % 128 == 0 &&
-      tm * (N / 128) >= 2 * kNumSM)
+      tm * (N / 128) >= 2 * kNumSM) {
+    int pairs = 0;
+    if (N % 256 == 0 && gemm_2sm_enabled()) WCHECK(g2_max_pairs(&pairs));
+    if (pairs > 0) return gemm_rownorm_2sm(a0, W, N, out, M, eps, pairs, st);
     return gemm_rownorm_persistent(a0, W, N, out, M, eps, st);
+  }
   int bn = 64;
   if (N % 256 == 0 && tm * (N / 256) >= kNumSM) bn = 256;
   else if (N % 128 == 0 && tm * (N / 128) >= kNumSM) bn = 128;
@@ -382,7 +452,7 @@ whale_status fold_weights(const Shape& s, const __nv_bfloat16* wq, const float* 
   add(wkv, gkv, okv, s.kvw, 0);
   add(wug, gffn, oug, s.ugw, s.tied ? 0 : 1);
   if (jobs.n == 0) return WHALE_OK;
-  const unsigned gx = (unsigned)std::min<long long>(cdiv<long long>(maxe, 256), 4 * kNumSM);
+  const unsigned gx = (unsigned)std::min<long long>(cdiv<long long>(maxe / 8, 256), 8 * kNumSM);
   fold_weights_kernel<<<dim3(gx, jobs.n), 256, 0, st>>>(jobs);
   CUCHECK(cudaGetLastError());
   return WHALE_OK;
@@ -411,16 +481,23 @@ whale_status launch_attn_hg(int hg, const CUtensorMap& tm, const AttnArgs& a, di
 }
 
 whale_status attention_bf16(const Shape& s, const void* q, const void* kv, const int* offsets, void* out,
-                            void* out_lo, int B, int max_L, long long total_L, float* po, float* pml,
-                            cudaStream_t st) {
-  (void)max_L;
+                            void* out_lo, int B, long long total_L, void* scratch, cudaStream_t st) {
   if (B == 0) return WHALE_OK;
   const AttnPlan p = plan_attention(s, B, total_L);
+  const size_t rows = (size_t)B * s.N;
+  if (total_L <= 0) {  // every history is empty: A = 0
+    CUCHECK(cudaMemsetAsync(out, 0, rows * s.d * 2, st));
+    if (out_lo) CUCHECK(cudaMemsetAsync(out_lo, 0, rows * s.d * 2, st));
+    return WHALE_OK;
+  }
   AttnArgs a{};
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.offsets = offsets;
-  a.part_o = po;
-  a.part_ml = pml;
+  a.part_o = reinterpret_cast<float*>(at(scratch, p.po_off()));
+  a.part_ml = reinterpret_cast<float*>(at(scratch, p.pml_off()));
+  a.counters = reinterpret_cast<int*>(at(scratch, p.cnt_off()));
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.out_lo = static_cast<__nv_bfloat16*>(out_lo);
   a.B = B;
   a.N = s.N;
   a.QB = p.QB;
@@ -432,31 +509,22 @@ whale_status attention_bf16(const Shape& s, const void* q, const void* kv, const
   a.G = p.G;
   a.total_L = total_L;
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)s.dh));
-  if ((long long)B * p.nqb > (1ll << 31) - 1) return WHALE_ERR_UNSUPPORTED;
-  if (total_L > 0) {
-    CUtensorMap tm;
-    WCHECK(tmap_bf16(&tm, kv, total_L, s.kvw, s.kvw, p.T));
-    const dim3 grid(p.G, s.h / p.HG);
-    whale_status r = WHALE_ERR_UNSUPPORTED;
-    if (s.dh == 32) {
-      if (p.QT == 1) r = launch_attn_hg<32, 1>(p.HG, tm, a, grid, st);
-      else if (p.QT == 2) r = launch_attn_hg<32, 2>(p.HG, tm, a, grid, st);
-      else r = launch_attn_hg<32, 4>(p.HG, tm, a, grid, st);
-    } else {
-      if (p.QT == 1) r = launch_attn_hg<64, 1>(p.HG, tm, a, grid, st);
-      else if (p.QT == 2) r = launch_attn_hg<64, 2>(p.HG, tm, a, grid, st);
-      else r = launch_attn_hg<64, 4>(p.HG, tm, a, grid, st);
-    }
-    WCHECK(r);
+  if ((long long)B * p.nqb > (1ll << 30)) return WHALE_ERR_UNSUPPORTED;
+  CUCHECK(cudaMemsetAsync(a.counters, 0, p.cnt_elems * 4, st));
+  CUtensorMap tm;
+  WCHECK(tmap_bf16(&tm, kv, total_L, s.kvw, s.kvw, p.T));
+  const dim3 grid(p.G, s.h / p.HG);
+  whale_status r = WHALE_ERR_UNSUPPORTED;
+  if (s.dh == 32) {
+    if (p.QT == 1) r = launch_attn_hg<32, 1>(p.HG, tm, a, grid, st);
+    else if (p.QT == 2) r = launch_attn_hg<32, 2>(p.HG, tm, a, grid, st);
+    else r = launch_attn_hg<32, 4>(p.HG, tm, a, grid, st);
+  } else {
+    if (p.QT == 1) r = launch_attn_hg<64, 1>(p.HG, tm, a, grid, st);
+    else if (p.QT == 2) r = launch_attn_hg<64, 2>(p.HG, tm, a, grid, st);
+    else r = launch_attn_hg<64, 4>(p.HG, tm, a, grid, st);
   }
-  if ((long long)B * p.nqb > 0x7fffffffll || s.h > 65535) return WHALE_ERR_UNSUPPORTED;
-  const dim3 cgrid((unsigned)(B * p.nqb), s.h);
-  auto* o_hi = static_cast<__nv_bfloat16*>(out);
-  auto* o_lo = static_cast<__nv_bfloat16*>(out_lo);
-  if (s.dh == 32) attn_combine_kernel<32><<<cgrid, 256, 0, st>>>(a, o_hi, o_lo);
-  else attn_combine_kernel<64><<<cgrid, 256, 0, st>>>(a, o_hi, o_lo);
-  CUCHECK(cudaGetLastError());
-  return WHALE_OK;
+  return r;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -523,8 +591,10 @@ whale_status fusion_mlp_f32(const Shape& s, long long rows, const float* a, cons
 }
 
 bool weights_ok(const Shape& s, const whale_layer_weights* w) {
+  auto al = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
   return w && w->g_q && w->g_kv && w->g_ffn && w->w_q && w->w_kv && w->w_f2 && w->w_upgate && w->w_down &&
-         (s.Fh == 0 || w->w_f1);
+         (s.Fh == 0 || w->w_f1) && al(w->g_q) && al(w->g_kv) && al(w->g_ffn) && al(w->w_q) && al(w->w_kv) &&
+         al(w->w_f1) && al(w->w_f2) && al(w->w_upgate) && al(w->w_down);
 }
 
 // A token-side tensor of the bf16 path: fp32 value plus its bf16 hi/lo pair (any may be null
@@ -575,9 +645,8 @@ whale_status layer_bf16(const Shape& s, const Stream3& in, const void* slab, con
   WCHECK(gemm_bf16(opnd(slab, nullptr, s.d, s.d), no_opnd(), wkv, s.kvw, Outs{at(ws, L.kv), nullptr, nullptr, s.kvw},
                    nullptr, 0, hint.total_L, EPI_STORE, true, s.eps, st));
   // S3 attention -> A as a hi/lo pair
-  WCHECK(attention_bf16(s, at(ws, L.q), at(ws, L.kv), offsets, at(ws, L.a), at(ws, L.a_lo), hint.B, hint.max_L,
-                        hint.total_L, reinterpret_cast<float*>(at(ws, L.po)), reinterpret_cast<float*>(at(ws, L.pml)),
-                        st));
+  WCHECK(attention_bf16(s, at(ws, L.q), at(ws, L.kv), offsets, at(ws, L.a), at(ws, L.a_lo), hint.B, hint.total_L,
+                        at(ws, L.po), st));
   // S4 Fusion MLP -> F (fp32 + pair)
   auto* f32 = reinterpret_cast<float*>(at(ws, L.f32));
   WCHECK(fusion_bf16(s, rows, opnd(at(ws, L.a), at(ws, L.a_lo), s.d, s.d), X, in.f32, w.w_f1, w.w_f2, at(ws, L.g),
@@ -889,12 +958,9 @@ whale_status whale_cross_attention(const whale_config* cfg, const void* q, const
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (s.bf16) {
     const AttnPlan p = plan_attention(s, hint->B, hint->total_L);
-    const size_t po = align_up(p.po_elems * 4);
-    if (!ws || ws_bytes < po + p.pml_elems * 4 || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)))
-      return WHALE_ERR_WORKSPACE;
+    if (!ws || ws_bytes < p.bytes() || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1))) return WHALE_ERR_WORKSPACE;
     WCHECK(debug_check(s, seq_offsets, *hint, st));
-    return attention_bf16(s, q, kv, seq_offsets, a, nullptr, hint->B, hint->max_L, hint->total_L,
-                          static_cast<float*>(ws), reinterpret_cast<float*>(at(ws, po)), st);
+    return attention_bf16(s, q, kv, seq_offsets, a, nullptr, hint->B, hint->total_L, ws, st);
   }
   WCHECK(debug_check(s, seq_offsets, *hint, st));
   return attention_f32(s, static_cast<const float*>(q), static_cast<const float*>(kv), seq_offsets,
