@@ -174,6 +174,29 @@ whale_status whale_swiglu_ffn(const whale_config* cfg, long long rows, const voi
                               const void* w_upgate, const void* w_down, void* y, void* workspace,
                               size_t workspace_bytes, whale_stream_t stream);
 
+/* Eq. (4) like whale_cross_attention, for callers that cannot allocate device memory.
+ * No counterpart in the paper: this is a deployment convenience. Some callers cannot call
+ * cudaMalloc or hand out a workspace: code embedded in a host framework that owns every byte of
+ * device memory through its own allocator or a fixed pre-reserved pool, and latency-critical
+ * serving loops where a cudaMalloc (which may synchronise the device) is not acceptable. This
+ * entry point takes no workspace: the attention partials live in one file-scope device array of
+ * WHALE_NOALLOC_SCRATCH_BYTES (32 MiB) that every GPU which loads this library holds until the
+ * process exits. It allocates nothing itself.
+ *  - Limit: the partials of a call, (B * ceil(N / QB) + G) * n_heads * QB * (d_head + 2) * 4 bytes
+ *    (QB = 16, 32 or 64 queries per block, G <= 148), must fit; a larger shape returns
+ *    WHALE_ERR_WORKSPACE before any GPU work. The 15k-history stack (B 64, N 32, d 512, 8 heads)
+ *    needs 14 MB; the 16384-query serving shape needs 28 MB.
+ *  - The first call on a device looks up the array's device address (once per device, with that
+ *    device current); make that first call before any stream capture.
+ *  - Every call shares the one array and overwrites it; nothing in it needs to start at zero (each
+ *    partial is written before it is read within the same call). Calls whose kernels overlap on
+ *    the GPU (other streams, other host threads) race on the array: serialise them.
+ *  - fp32 mode uses no scratch and simply runs the fp32 attention. */
+#define WHALE_NOALLOC_SCRATCH_BYTES (32u << 20)
+whale_status whale_cross_attention_noalloc(const whale_config* cfg, const void* q, const void* kv,
+                                           const int* seq_offsets, void* a, const whale_shape_hint* hint,
+                                           whale_stream_t stream);
+
 /* Synchronises `stream`, then reads and clears the device error word of the current
  * device (bits WHALE_DEVERR_*). Returns WHALE_ERR_DEVICE_CHECK if any bit was set. */
 whale_status whale_get_device_error(whale_stream_t stream, int* code);

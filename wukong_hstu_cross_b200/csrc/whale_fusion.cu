@@ -1021,6 +1021,57 @@ whale_status whale_swiglu_ffn(const whale_config* cfg, long long rows, const voi
                     static_cast<const float*>(w_down), static_cast<float*>(y), rows, r, ug, u, st);
 }
 
+}  // extern "C"
+
+// ------------------------------------------------------------------------------------------
+// Allocation-free attention entry point: partials in a fixed file-scope device array.
+// ------------------------------------------------------------------------------------------
+namespace {
+__device__ __align__(256) unsigned char g_noalloc_scratch[WHALE_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on the current device, looked up once per device (the
+// name is only a host-side stand-in for the array; kernels must get the real address).
+whale_status noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[64];
+  int dev = 0;
+  CUCHECK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return WHALE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    CUCHECK(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return WHALE_OK;
+}
+}  // namespace
+
+extern "C" {
+
+whale_status whale_cross_attention_noalloc(const whale_config* cfg, const void* q, const void* kv,
+                                           const int* seq_offsets, void* a, const whale_shape_hint* hint,
+                                           whale_stream_t stream) {
+  Shape s;
+  WCHECK(validate(cfg, &s));
+  WCHECK(check_hint(hint));
+  if (hint->B == 0) return WHALE_OK;
+  if (!q || !a || !seq_offsets || (hint->total_L > 0 && !kv)) return WHALE_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (!s.bf16) {
+    WCHECK(debug_check(s, seq_offsets, *hint, st));
+    return attention_f32(s, static_cast<const float*>(q), static_cast<const float*>(kv), seq_offsets,
+                         static_cast<float*>(a), hint->B, hint->total_L, st);
+  }
+  const AttnPlan p = plan_attention(s, hint->B, hint->total_L);
+  if (p.bytes() > (size_t)WHALE_NOALLOC_SCRATCH_BYTES) return WHALE_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  WCHECK(noalloc_scratch(&scratch));
+  WCHECK(debug_check(s, seq_offsets, *hint, st));
+  return attention_bf16(s, q, kv, seq_offsets, a, nullptr, hint->B, hint->total_L, scratch, st);
+}
+
 whale_status whale_get_device_error(whale_stream_t stream, int* code) {
   if (!code) return WHALE_ERR_INVALID_ARG;
   CUCHECK(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));

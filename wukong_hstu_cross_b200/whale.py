@@ -18,6 +18,7 @@ HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))
 WHALE_FP32, WHALE_BF16 = 0, 1
 WHALE_SHARED_KV, WHALE_TIED_GATE, WHALE_DEBUG = 1, 2, 4
 WHALE_DEVERR_TIMEOUT, WHALE_DEVERR_OFFSETS = 1, 2
+WHALE_NOALLOC_SCRATCH_BYTES = 32 << 20
 STATUS = {0: "WHALE_OK", 1: "WHALE_ERR_INVALID_ARG", 2: "WHALE_ERR_UNSUPPORTED", 3: "WHALE_ERR_CUDA",
           4: "WHALE_ERR_WORKSPACE", 5: "WHALE_ERR_DEVICE_CHECK"}
 
@@ -67,6 +68,7 @@ _SIGS = {
     "whale_fusion_mlp": ([POINTER(whale_config), c_longlong, _P, _P, _P, _P, _P, _P, c_size_t, _P], c_int),
     "whale_swiglu_ffn": ([POINTER(whale_config), c_longlong, _P, _P, _P, _P, _P, _P, c_size_t, _P], c_int),
     "whale_get_device_error": ([_P, POINTER(c_int)], c_int),
+    "whale_cross_attention_noalloc": ([POINTER(whale_config), _P, _P, _P, _P, POINTER(whale_shape_hint), _P], c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -206,6 +208,16 @@ def whale_cross_attention(cfg, q, kv, seq_offsets, a, hint, workspace, workspace
     if raw:
         return st
     _check(st, "whale_cross_attention")
+
+
+def whale_cross_attention_noalloc(cfg, q, kv, seq_offsets, a, hint, stream=None, raw=False):
+    """Eq. (4) without a workspace: the partials live in the library's fixed device array
+    (WHALE_NOALLOC_SCRATCH_BYTES); see include/whale_fusion.h."""
+    st = _lib.whale_cross_attention_noalloc(ctypes.byref(cfg), _ptr(q), _ptr(kv), _ptr(seq_offsets), _ptr(a),
+                                            ctypes.byref(hint), _stream(stream))
+    if raw:
+        return st
+    _check(st, "whale_cross_attention_noalloc")
 
 
 def whale_fusion_mlp(cfg, rows, a, x, w_f1, w_f2, f, workspace, workspace_bytes=None, stream=None, raw=False):
