@@ -31,6 +31,11 @@ sys.path.insert(0, ROOT)
 from wukong_hstu_cross_b200 import inputs as I  # noqa: E402
 
 METRIC = "WHALE fusion-layer examples/s @15k jagged history; % of HBM/TC roofline"
+# DRAM bytes per launch measured by ncu (dram__bytes_read.sum + dram__bytes_write.sum), per
+# history row, from the committed summary profiles/kv_proj_gemm_hist15k.md (one-SM K|V kernel,
+# d = 512). Reported only for that kernel and width; null otherwise.
+KV_TRAFFIC_BYTES_PER_ROW_D512 = (113.375488e6 + 168.328960e6) / 109605
+
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
 
 
@@ -46,25 +51,28 @@ def load_peaks():
 # ------------------------------------------------------------------------------------------------
 # algorithmic work per step (bf16 storage)
 # ------------------------------------------------------------------------------------------------
-def step_work(w: I.Workload, total_L: int) -> dict:
-    """FLOPs and bytes per kernel family for one layer (no re-reads, no partials)."""
+def step_work(w: I.Workload, total_L: int, shared_kv: bool = False, tied_gate: bool = False) -> dict:
+    """FLOPs and bytes per kernel family for one layer (no re-reads, no partials; the hi/lo
+    operand halves of the token-side GEMMs are not counted: algorithmic work only)."""
     B, N, d, H, Fh = w.batch, w.n_tokens, w.d, w.ffn_hidden, w.fusion_hidden
     rows = B * N
     e = 2
+    kvw = d if shared_kv else 2 * d
+    ugw = H if tied_gate else 2 * H
     return {
-        "kv_proj": {"flops": 2.0 * total_L * d * 2 * d, "bytes": e * (total_L * d + total_L * 2 * d + 2 * d * d)},
-        "attention": {"flops": 4.0 * rows * 0 + 4.0 * N * total_L * d,   # 2 matmuls of N x L x d per example
-                      "bytes": e * (total_L * 2 * d + 2 * rows * d)},
+        "kv_proj": {"flops": 2.0 * total_L * d * kvw, "bytes": e * (total_L * d + total_L * kvw + kvw * d)},
+        "attention": {"flops": 4.0 * N * total_L * d,   # q k^T and p v: 2 x (2 N L d) per example
+                      "bytes": e * (total_L * kvw + 2 * rows * d)},
         "q_proj": {"flops": 2.0 * rows * d * d, "bytes": e * (2 * rows * d + d * d)},
         "fusion_mlp": {"flops": 2.0 * rows * (2 * d * Fh + Fh * d), "bytes": e * (3 * rows * d + 2 * rows * Fh + 3 * d * Fh)},
-        "swiglu_ffn": {"flops": 2.0 * rows * (d * 2 * H + H * d), "bytes": e * (3 * rows * d + 2 * rows * H + 3 * d * H)},
+        "swiglu_ffn": {"flops": 2.0 * rows * (d * ugw + H * d), "bytes": e * (3 * rows * d + 2 * rows * H + (ugw + H) * d)},
     }
 
 
-def launches_per_step(w: I.Workload) -> int:
-    # once: residual-stream set-up; per layer: weight fold, Q GEMM, K|V GEMM, attention (split
+def launches_per_step(w: I.Workload, fold_per_call: bool) -> int:
+    # once: residual-stream set-up; per layer: [weight fold,] Q GEMM, K|V GEMM, attention (split
     # merge fused in), Fusion GEMM(s), up|gate GEMM, down GEMM
-    return 1 + w.n_layers * (7 + (1 if w.fusion_hidden > 0 else 0))
+    return 1 + w.n_layers * (6 + (1 if fold_per_call else 0) + (1 if w.fusion_hidden > 0 else 0))
 
 
 # ------------------------------------------------------------------------------------------------
@@ -229,11 +237,18 @@ def run_kernel_case(args):
     Wb.whale_project_queries(p.cfg, q.shape[0], p.tokens, lw["g_q"], lw["w_q"], q, p.workspace)
     Wb.whale_project_kv(p.cfg, T, p.states[0], lw["g_kv"], lw["w_kv"], kv, p.workspace)
 
+    rows = w.batch * w.n_tokens
+    f_out = torch.empty_like(q)
+
     def step():
         if args.kernel_case == "kv":
             Wb.whale_project_kv(p.cfg, T, p.states[0], lw["g_kv"], lw["w_kv"], kv, p.workspace)
-        else:
+        elif args.kernel_case == "attn":
             Wb.whale_cross_attention(p.cfg, q, kv, p.offsets_t, a, p.hint, p.workspace)
+        elif args.kernel_case == "ffn":     # up|gate GEMM (SwiGLU epilogue) + down GEMM
+            Wb.whale_swiglu_ffn(p.cfg, rows, q, lw["g_ffn"], lw["w_upgate"], lw["w_down"], f_out, p.workspace)
+        else:                               # Fusion MLP: two GEMMs
+            Wb.whale_fusion_mlp(p.cfg, rows, a, q, lw["w_f1"], lw["w_f2"], f_out, p.workspace)
     step()  # compile / first-use work outside the timed loop
     for _ in range(args.warmup):
         step()
@@ -245,7 +260,8 @@ def run_kernel_case(args):
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / args.steps
-    work = step_work(w, T)["kv_proj" if args.kernel_case == "kv" else "attention"]
+    work = step_work(w, T)[{"kv": "kv_proj", "attn": "attention", "ffn": "swiglu_ffn",
+                             "fusion": "fusion_mlp"}[args.kernel_case]]
     print(json.dumps({"kernel_case": args.kernel_case, "workload": w.name, "total_L": T, "ms_per_launch": ms,
                       "tflops": work["flops"] / ms / 1e9, "gbs": work["bytes"] / ms / 1e6}), flush=True)
     return 0
@@ -261,9 +277,13 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--ref-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel-case", choices=["kv", "attn"], default=None,
+    ap.add_argument("--kernel-case", choices=["kv", "attn", "ffn", "fusion"], default=None,
                     help="profiling aid: run only one step entry point on one layer of the workload")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (kernel cases)")
+    ap.add_argument("--shared-kv", action="store_true", help="variant: K = V (one W_K), the pages' shared key/value")
+    ap.add_argument("--tied-gate", action="store_true", help="variant: W_gate = W_up, the pages' shared-gate SwiGLU")
+    ap.add_argument("--fold-per-call", action="store_true",
+                    help="fold the RMSNorm gains into the weights inside every forward instead of once at load")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
@@ -282,7 +302,10 @@ def main():
 
     from wukong_hstu_cross_b200 import dist as D
     w = D.shard_workload(I.WORKLOADS[args.workload], rank, world)   # this rank's own examples
-    p = Hn.build_problem(w, device="cuda")
+    p = Hn.build_problem(w, device="cuda", shared_kv=args.shared_kv, tied_gate=args.tied_gate)
+    raw_weights = p.weights
+    if not args.fold_per_call:
+        Hn.prepare_weights(p)   # gains folded into the weights once, as at model load
     stream = torch.cuda.current_stream()
     total_L = p.total_L
 
@@ -305,9 +328,9 @@ def main():
     value = world * w.batch / (ms / 1e3)
 
     # ---------------- per-kernel timing of the two heavy steps (same stream, CUDA events) ------
-    work = step_work(w, total_L)
+    work = step_work(w, total_L, args.shared_kv, args.tied_gate)
     Hn_ws = p.workspace
-    kv = torch.empty(total_L, 2 * w.d, dtype=torch.bfloat16, device="cuda")
+    kv = torch.empty(total_L, (1 if args.shared_kv else 2) * w.d, dtype=torch.bfloat16, device="cuda")
     q = torch.empty(w.batch * w.n_tokens, w.d, dtype=torch.bfloat16, device="cuda")
     a = torch.empty_like(q)
     reps = max(args.steps, 3)
@@ -328,14 +351,14 @@ def main():
         return e0.elapsed_time(e1) / cnt
 
     def kv_step(l):
-        Wb.whale_project_kv(p.cfg, total_L, p.states[l], p.weights[l]["g_kv"], p.weights[l]["w_kv"], kv, Hn_ws,
+        Wb.whale_project_kv(p.cfg, total_L, p.states[l], raw_weights[l]["g_kv"], raw_weights[l]["w_kv"], kv, Hn_ws,
                             stream=stream)
 
     def attn_step(l):
         Wb.whale_cross_attention(p.cfg, q, kv, p.offsets_t, a, p.hint, Hn_ws, stream=stream)
 
     kv_step(0)
-    Wb.whale_project_queries(p.cfg, q.shape[0], p.tokens, p.weights[0]["g_q"], p.weights[0]["w_q"], q, Hn_ws,
+    Wb.whale_project_queries(p.cfg, q.shape[0], p.tokens, raw_weights[0]["g_q"], raw_weights[0]["w_q"], q, Hn_ws,
                              stream=stream)
     torch.cuda.synchronize()
     t_kv = timed(kv_step, reps)
@@ -345,10 +368,14 @@ def main():
     attn_gbs = work["attention"]["bytes"] / (t_attn * 1e-3) / 1e9
     layer_ms = ms / w.n_layers
     share_kv, share_attn = t_kv / layer_ms, t_attn / layer_ms
+    kv_traffic = None
+    if w.d == 512 and os.environ.get("WHALE_GEMM_1SM", "0") == "1":
+        kv_traffic = KV_TRAFFIC_BYTES_PER_ROW_D512 * total_L
     if share_kv >= share_attn:
         roof = {"kernel": "K|V projection GEMM (tcgen05, RMSNorm row factor fused)", "bound": "tensor",
                 "achieved": kv_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": kv_tflops / peaks["bf16_tflops"], "traffic": None,
+                "frac": kv_tflops / peaks["bf16_tflops"], "traffic": kv_traffic,
+                "traffic_source": "ncu capture scaled by rows (profiles/kv_proj_gemm_hist15k.md)",
                 "algorithmic_per_launch": work["kv_proj"]["flops"], "avg_launch_ms": t_kv,
                 "peak_source": f"{peak_src} bf16 burst"}
     else:
@@ -398,13 +425,17 @@ def main():
             "config": {"workload": w.name, "batch": w.batch, "n_tokens": w.n_tokens, "d": w.d, "heads": w.n_heads,
                        "layers": w.n_layers, "total_L": total_L, "max_L": int(p.lengths.max()),
                        "parallelism": f"dp{world} (independent examples per rank, no collective)",
+                       "variant": ("shared K=V " if args.shared_kv else "") + ("tied gate" if args.tied_gate else "")
+                                  or "separate W_K, W_V; untied up|gate",
+                       "weights": ("gains folded per forward" if args.fold_per_call else
+                                   "gains folded into the weights once at load (whale_prepare_weights)"),
                        "l2": "inputs larger than L2 (each layer reads its own "
                              f"{total_L * w.d * 2 / 1e6:.0f} MB state slab), no flush"},
             "roofline": roof,
             "step_roofline": {"t_star_ms": t_star, "frac": t_star / ms, "per_layer_ms": layer_ms,
                               "kv_proj_ms": t_kv, "attention_ms": t_attn,
                               "peaks": f"{peak_src}: {peaks['hbm_gbs']} GB/s, {peaks['bf16_tflops']} TFLOP/s"},
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step(w) * args.steps,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step(w, args.fold_per_call) * args.steps,
             "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)

@@ -64,6 +64,8 @@ typedef enum { WHALE_FP32 = 0, WHALE_BF16 = 1 } whale_dtype;
 #define WHALE_SHARED_KV 1u  /* K = V: w_kv is W_K alone [d, d] (gist.science 2.2 "Shared Key-Value") */
 #define WHALE_TIED_GATE 2u  /* W_gate = W_up: w_upgate is W_up alone [H, d] (gist.science 2.2 "Shared-Gate SwiGLU") */
 #define WHALE_DEBUG 4u      /* validate offsets on the device before the forward */
+#define WHALE_PREPARED_WEIGHTS 8u  /* bf16: w_q, w_kv, w_upgate come from whale_prepare_weights (gains
+                                      already folded in, up|gate rows packed); g_* are not read */
 
 /* device error bits (whale_get_device_error) */
 #define WHALE_DEVERR_TIMEOUT 1
@@ -113,6 +115,18 @@ const char* whale_status_string(whale_status s);
 /* Bytes of device workspace needed by every entry point below for this config and
  * shape (0 if cfg/hint are invalid or unsupported). */
 size_t whale_workspace_size(const whale_config* cfg, const whale_shape_hint* hint);
+
+/* One-time weight preparation (bf16 mode). RMSNorm(x; g) W^T = r(x) * (x (W diag(g))^T), so the
+ * gains can live in the weights: this folds g_q into W_Q, g_kv into [W_K ; W_V] and g_ffn into
+ * [W_up ; W_gate], re-packing the up|gate rows in blocks of 32 (16 up rows, then the 16 matching
+ * gate rows) for the fused SwiGLU epilogue. The results go to `prepared` (device, at least
+ * whale_prepared_weights_size bytes, 256-byte aligned, owned by the caller), and `out_weights`
+ * (host array of n_layers) receives the input pointers with w_q, w_kv, w_upgate replaced by the
+ * prepared copies. Forwards given out_weights with cfg->flags | WHALE_PREPARED_WEIGHTS skip the
+ * per-call fold. Asynchronous on `stream`; the inputs must stay valid until it completes. */
+size_t whale_prepared_weights_size(const whale_config* cfg);
+whale_status whale_prepare_weights(const whale_config* cfg, const whale_layer_weights* weights, void* prepared,
+                                   size_t prepared_bytes, whale_layer_weights* out_weights, whale_stream_t stream);
 
 /* Whole stack (all n_layers) on device buffers.
  *   wukong_tokens  device [B, N, d]            H_w of layer 0

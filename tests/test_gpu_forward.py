@@ -111,6 +111,21 @@ def test_layer_entry_point_and_batch_reordering():
     assert bool(((y2.float() - ref).abs() <= 1e-2 * (1 + ref.abs())).all())
 
 
+def test_prepared_weights_match_per_call_fold():
+    w = I.WORKLOADS["stack_d256"].replace(batch=3, n_layers=2, lengths=("uniform", 1, 900))
+    for tied in (False, True):
+        p = Hn.build_problem(w, gains="random", tied_gate=tied)
+        ref = Hn.run_forward(p).clone()
+        buf = torch.empty(W.whale_prepared_weights_size(p.cfg), dtype=torch.uint8, device="cuda")
+        pw = W.whale_prepare_weights(p.cfg, p.weights, buf)
+        cfg = W.make_config(p.cfg.n_layers, p.cfg.d, p.cfg.n_heads, p.cfg.n_tokens, p.cfg.ffn_hidden,
+                            p.cfg.fusion_hidden, p.cfg.dtype, p.cfg.flags | W.WHALE_PREPARED_WEIGHTS, p.cfg.eps)
+        out = torch.empty_like(p.out)
+        W.whale_fusion_forward(cfg, p.tokens, p.states, p.offsets_t, pw, out, p.hint, p.workspace)
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref)
+
+
 def test_host_buffer_entry_point_matches_device_entry_point():
     w = I.WORKLOADS["stack_d256"].replace(batch=4, n_layers=3, lengths=("uniform", 10, 1200))
     p = Hn.build_problem(w, gains="random")

@@ -182,21 +182,28 @@ def test_swiglu_ffn(rows, d, tied):
     assert_parity(y, O.swiglu_ffn(f, g, wug, wd, 1e-6, tied_gate=tied), "bf16", rms_rel=1e-2, what="Y")
 
 
-def test_project_kv_two_sm_kernel():
-    """The 2-SM (cta_group::2) K|V GEMM, selected with WHALE_GEMM_2SM=1, on a ragged large M."""
+def test_project_kv_one_and_two_sm_kernels():
+    """Both persistent K|V GEMMs on a ragged large M: the 2-SM (cta_group::2) default and the
+    one-SM kernel selected with WHALE_GEMM_1SM=1; they must agree bitwise (same fp32 sums)."""
     import os
     rng = np.random.default_rng(77)
     rows, d = 70001, 512
     x = bf16_randn(rng, rows, d)
     g = rng.uniform(0.5, 1.5, d).astype(np.float32)
     wkv = I.bf16_round(np.concatenate([I.xavier_uniform(rng, d, d), I.xavier_uniform(rng, d, d)]))
-    kv = torch.empty(rows, 2 * d, dtype=torch.bfloat16, device=DEV)
-    os.environ["WHALE_GEMM_2SM"] = "1"
-    try:
-        W.whale_project_kv(_cfg(d, 8), rows, _t(x), _g(g), _t(wkv), kv, _ws(64 << 20))
-        torch.cuda.synchronize()
-    finally:
-        os.environ.pop("WHALE_GEMM_2SM", None)
+    outs = []
+    for one_sm in (False, True):
+        kv = torch.empty(rows, 2 * d, dtype=torch.bfloat16, device=DEV)
+        if one_sm:
+            os.environ["WHALE_GEMM_1SM"] = "1"
+        try:
+            W.whale_project_kv(_cfg(d, 8), rows, _t(x), _g(g), _t(wkv), kv, _ws(64 << 20))
+            torch.cuda.synchronize()
+        finally:
+            os.environ.pop("WHALE_GEMM_1SM", None)
+        outs.append(kv)
     sel = np.r_[0:300, rows - 300:rows]
     ref = O.linear(O.rms_norm(x[sel], g, 1e-6), wkv)
-    assert_parity(kv[torch.from_numpy(sel).to(DEV)], ref, "bf16", rms_rel=1e-2, what="KV (2-SM)")
+    for kv, name in zip(outs, ("2-SM", "1-SM")):
+        assert_parity(kv[torch.from_numpy(sel).to(DEV)], ref, "bf16", rms_rel=1e-2, what=f"KV ({name})")
+    assert torch.equal(outs[0], outs[1])

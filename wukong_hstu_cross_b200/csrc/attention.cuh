@@ -146,6 +146,8 @@ __global__ void __launch_bounds__(32 * (HG + 1), 1)
   volatile int* last_flag = reinterpret_cast<volatile int*>(empty + STAGES) + 1;
 
   const int cta = blockIdx.x, hg = blockIdx.y;
+  pdl_wait();
+  pdl_trigger();
   long long P0, W;
   flat_extent(a, P0, W);
   // Items with an empty history get A = 0 here (no slice covers them).

@@ -23,6 +23,8 @@ struct FoldJobs {
 
 // One thread per 8 consecutive columns (16-byte loads and stores; cols % 8 == 0).
 __global__ void fold_weights_kernel(const FoldJobs jobs) {
+  pdl_wait();
+  pdl_trigger();
   if ((int)blockIdx.y >= jobs.n) return;
   const FoldJob j = jobs.job[blockIdx.y];
   const int cols8 = j.cols >> 3;

@@ -8,15 +8,16 @@
 // MMA work — half the operand bytes per FLOP of a one-SM 128 x 256 tile — so six stages cover
 // twice the load latency.
 //
-// Per CTA (352 threads): warp 0 TMA producer (both CTAs; completion counted on the even CTA's
+// Per CTA (480 threads): warp 0 TMA producer (both CTAs; completion counted on the even CTA's
 // `full` barrier), warp 1 TMEM allocation (2 x 256 columns: two accumulators) and, in the even
-// CTA, the MMA thread, warps 2..5 epilogue (TMEM -> row factor -> bf16 -> swizzled staging ->
-// TMA store), warps 6..9 row statistics (sum of squares of each row of A from the staged tiles),
-// warp 10 (even CTA) relays "stage s landed" to both CTAs' `ready[s]`, so the statistic warps of
-// the odd CTA, whose bytes are counted on the even CTA's barrier, know when to read.
+// CTA, the MMA thread, warps 2..9 epilogue (two warps per TMEM lane quadrant, 128 columns each:
+// TMEM -> row factor -> bf16 -> swizzled staging -> TMA store), warps 10..13 row statistics (sum
+// of squares of each row of A from the staged tiles), warp 14 (even CTA) relays "stage s landed"
+// to both CTAs' `ready[s]`, so the statistic warps of the odd CTA, whose bytes are counted on the
+// even CTA's barrier, know when to read.
 // Barriers (same offsets in both CTAs): full[s] (even only), ready[s], empty[s] (MMA commit
 // multicast to both + 4 local statistic warps), tfull[2] (commit multicast), tempty[2] (even
-// only: 4 + 4 epilogue warps), nfull[2], edone[2] (local). Every wait is bounded; every thread of
+// only: 8 + 8 epilogue warps), nfull[2], edone[2] (local). Every wait is bounded; every thread of
 // both CTAs reaches the closing cluster barrier on every path.
 #pragma once
 
@@ -38,13 +39,13 @@ struct G2Smem {
   static constexpr uint32_t A_BYTES = 128 * BK * 2;   // this CTA's 128 rows of A
   static constexpr uint32_t B_BYTES = 128 * BK * 2;   // this CTA's 128 rows of W
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr uint32_t EPI_BYTES = 4 * 2 * 32 * 128;
+  static constexpr uint32_t EPI_BYTES = 8 * 32 * 128;  // one 32 x 64 bf16 staging tile per epilogue warp
   static constexpr int FIXED = 1024 + EPI_BYTES + 2 * 128 * 4 + 512;
   static constexpr int STAGES = (232448 - FIXED) / (int)STAGE_BYTES > 8 ? 8 : (232448 - FIXED) / (int)STAGE_BYTES;
   static constexpr size_t BYTES = FIXED + STAGES * (size_t)STAGE_BYTES;
 };
 
-constexpr int kG2Threads = 352;
+constexpr int kG2Threads = 480;
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
     gemm_rownorm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -80,9 +81,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 8);
+      mbar_init(&tempty[i], 16);
       mbar_init(&nfull[i], 4);
-      mbar_init(&edone[i], 4);
+      mbar_init(&edone[i], 8);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -102,6 +103,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
   cluster_sync_all();  // both CTAs' barriers exist before any remote arrive or counted copy
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 0) {
     // ---------------- TMA producer (both CTAs) ----------------
@@ -113,7 +116,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
         const int n0 = (tile % args.tiles_n) * 256 + (int)rank * 128;
         for (int kb = 0; kb < KB; ++kb, ++kg) {
           const int s = kg % ST, u = kg / ST;
-          if (kg >= ST && !mbar_wait_cluster(&empty[s], (u - 1) & 1, abort_flag)) {
+          if (kg >= ST && !mbar_wait(&empty[s], (u - 1) & 1, abort_flag)) {
             stop = true;
             break;
           }
@@ -133,12 +136,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
       bool stop = false;
       for (int tile = pair; tile < args.num_tiles && !stop; tile += npairs, ++it) {
         const int acc = it & 1, ua = it >> 1;
-        if (it >= 2 && !mbar_wait_cluster(&tempty[acc], (ua - 1) & 1, abort_flag)) break;
+        if (it >= 2 && !mbar_wait(&tempty[acc], (ua - 1) & 1, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * 256;
         for (int kb = 0; kb < KB; ++kb, ++kg) {
           const int s = kg % ST, u = kg / ST;
-          if (!mbar_wait_cluster(&full[s], u & 1, abort_flag)) {
+          if (!mbar_wait(&full[s], u & 1, abort_flag)) {
             stop = true;
             break;
           }
@@ -154,7 +157,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
         umma_commit_cg2_mc(&tfull[acc], 0x3);
       }
     }
-  } else if (warp == 10) {
+  } else if (warp == 14) {
     // ---------------- relay (even CTA): "stage s landed" to both CTAs' statistic warps ----------
     // (kept off the MMA thread: the cluster-scope release of the remote arrive is a fence)
     if (leader && lane == 0) {
@@ -162,12 +165,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
       const int total = ((args.num_tiles - pair + npairs - 1) / npairs) * KB;
       for (int kg = 0; kg < total; ++kg) {
         const int s = kg % ST, u = kg / ST;
-        if (!mbar_wait_cluster(&full[s], u & 1, abort_flag)) break;
+        if (!mbar_wait(&full[s], u & 1, abort_flag)) break;
         mbar_arrive(&ready[s]);
         mbar_arrive_cluster(peer_ready0 + s * 8);
       }
     }
-  } else if (warp >= 6) {
+  } else if (warp >= 10) {
     // ---------------- row statistics (both CTAs) ----------------
     const int row = (warp & 3) * 32 + lane;
     int kg = 0, it = 0;
@@ -177,7 +180,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
       bool ok = true;
       for (int kb = 0; kb < KB; ++kb, ++kg) {
         const int s = kg % ST, u = kg / ST;
-        if (!mbar_wait_cluster(&ready[s], u & 1, abort_flag)) {
+        if (!mbar_wait(&ready[s], u & 1, abort_flag)) {
           ok = false;
           break;
         }
@@ -199,28 +202,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kG2Threads, 1)
       if (lane == 0) mbar_arrive(&nfull[acc]);
     }
   } else {
-    // ---------------- epilogue (warps 2..5, both CTAs) ----------------
+    // ---------------- epilogue (warps 2..9, both CTAs): two warps per TMEM lane quadrant ----------
     const int q = warp & 3;
+    const int half = (warp - 2) >> 2;  // columns [128 * half, 128 * half + 128) of the tile
     const int row = q * 32 + lane;
-    uint8_t* stage0 = epi + (warp - 2) * 2 * 4096;
+    uint8_t* sbuf = epi + (warp - 2) * 4096;
     const uint32_t tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
     int it = 0, nstore = 0;
     for (int tile = pair; tile < args.num_tiles; tile += npairs, ++it) {
       const int acc = it & 1, ua = it >> 1;
       const int m0 = (tile / args.tiles_n) * 256 + (int)rank * 128, n0 = (tile % args.tiles_n) * 256;
-      if (!mbar_wait_cluster(&tfull[acc], ua & 1, abort_flag)) break;
+      if (!mbar_wait(&tfull[acc], ua & 1, abort_flag)) break;
       if (!mbar_wait(&nfull[acc], ua & 1, abort_flag)) break;
       tc_fence_after();
       const float r = rbuf[acc * 128 + row];
       const uint32_t t_row = tmem_base + acc * 256 + ((uint32_t)(q * 32) << 16);
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c, ++nstore) {
+      for (int cc = 0; cc < 2; ++cc, ++nstore) {
+        const int c = 2 * half + cc;
         uint32_t v0[32], v1[32];
         tmem_ld_32x32b_x32(t_row + c * 64, v0);
         tmem_ld_32x32b_x32(t_row + c * 64 + 32, v1);
         tmem_ld_wait();
-        uint8_t* sb = stage0 + (nstore & 1) * 4096;
-        if (lane == 0) bulk_wait_read<1>();
+        uint8_t* sb = sbuf;
+        // the TMA store issued from this buffer for the previous chunk must have read it
+        if (lane == 0) bulk_wait_read<0>();
         __syncwarp();
         uint4* dst = reinterpret_cast<uint4*>(sb + lane * 128);
 #pragma unroll

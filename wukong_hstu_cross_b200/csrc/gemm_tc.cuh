@@ -150,6 +150,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -282,6 +284,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // Residual-stream tensor from a bf16 input: x32 = x, lo = 0 (x itself serves as hi).
 __global__ void pair_from_bf16_kernel(const __nv_bfloat16* __restrict__ x, float* __restrict__ x32,
                                       __nv_bfloat16* __restrict__ lo, long long n) {
+  pdl_wait();
+  pdl_trigger();
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
     if (x32) x32[i] = __bfloat162float(x[i]);
     if (lo) lo[i] = __float2bfloat16_rn(0.f);

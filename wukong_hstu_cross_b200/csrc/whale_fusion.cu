@@ -22,6 +22,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <functional>
+#include <utility>
 #include <mutex>
 
 #include "aux_kernels.cuh"
@@ -51,15 +52,43 @@ namespace {
   } while (0)
 
 constexpr int kNumSM = 148;
-// The 2-SM (cta_group::2) K|V GEMM is opt-in: WHALE_GEMM_2SM=1 in the environment (read per call).
+// The 2-SM (cta_group::2) K|V GEMM is the default; WHALE_GEMM_1SM=1 in the environment selects the
+// one-SM persistent kernel instead (read per call; comparison runs and tests).
 inline bool gemm_2sm_enabled() {
-  const char* e = std::getenv("WHALE_GEMM_2SM");
-  return e && e[0] == '1';
+  const char* e = std::getenv("WHALE_GEMM_1SM");
+  return !(e && e[0] == '1');
 }
 constexpr size_t kAlign = 256;
 inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 template <class T>
 inline T cdiv(T a, T b) { return (a + b - 1) / b; }
+
+// ------------------------------------------------------------------------------------------
+// Launch with programmatic dependent launch (PDL): the kernel may start while the previous kernel
+// of the stream drains; it waits (griddepcontrol.wait) before touching global memory. Plain
+// launches when WHALE_NO_PDL=1 is set (comparison runs).
+// ------------------------------------------------------------------------------------------
+inline bool pdl_enabled() {
+  const char* e = std::getenv("WHALE_NO_PDL");
+  return !(e && e[0] == '1');
+}
+
+template <typename... KArgs, typename... Args>
+whale_status launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                        Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  CUCHECK(cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...));
+  return WHALE_OK;
+}
 
 // ------------------------------------------------------------------------------------------
 // TMA descriptor encoding through the driver entry point (no link-time dependency on libcuda)
@@ -98,7 +127,7 @@ whale_status tmap_bf16(CUtensorMap* tm, const void* base, long long rows, long l
 struct Shape {
   bool bf16;
   int layers, d, h, dh, N, H, Fh;
-  bool shared_kv, tied, debug;
+  bool shared_kv, tied, debug, prepared;
   float eps;
   int kvw;  // kv row width: 2d, or d with shared K = V
   int ugw;  // rows of the up|gate matrix: 2H, or H with a tied gate
@@ -109,7 +138,7 @@ whale_status validate(const whale_config* c, Shape* s) {
   if (!c || !s) return WHALE_ERR_INVALID_ARG;
   if (c->n_layers < 1 || c->d < 1 || c->n_heads < 1 || c->n_tokens < 1 || c->ffn_hidden < 1 ||
       c->fusion_hidden < 0 || !(c->eps >= 0.f) || (c->dtype != WHALE_FP32 && c->dtype != WHALE_BF16) ||
-      (c->flags & ~(WHALE_SHARED_KV | WHALE_TIED_GATE | WHALE_DEBUG)) || c->d % c->n_heads)
+      (c->flags & ~(WHALE_SHARED_KV | WHALE_TIED_GATE | WHALE_DEBUG | WHALE_PREPARED_WEIGHTS)) || c->d % c->n_heads)
     return WHALE_ERR_INVALID_ARG;
   s->bf16 = c->dtype == WHALE_BF16;
   s->layers = c->n_layers;
@@ -122,6 +151,7 @@ whale_status validate(const whale_config* c, Shape* s) {
   s->shared_kv = c->flags & WHALE_SHARED_KV;
   s->tied = c->flags & WHALE_TIED_GATE;
   s->debug = c->flags & WHALE_DEBUG;
+  s->prepared = (c->flags & WHALE_PREPARED_WEIGHTS) && c->dtype == WHALE_BF16;
   s->eps = c->eps;
   s->kvw = s->shared_kv ? s->d : 2 * s->d;
   s->ugw = s->tied ? s->H : 2 * s->H;
@@ -261,9 +291,7 @@ whale_status launch_gemm_t(const CUtensorMap* tm, const GemmArgs& g, long long t
   const size_t smem = GemmSmem<BN, SPLIT>::BYTES;
   auto kern = gemm_tc_kernel<BN, EPI, RN, SPLIT>;
   CUCHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  kern<<<(unsigned)tiles, kGemmThreads, smem, st>>>(tm[0], tm[1], tm[2], tm[3], tm[4], g);
-  CUCHECK(cudaGetLastError());
-  return WHALE_OK;
+  return launch_pdl(kern, dim3((unsigned)tiles), dim3(kGemmThreads), smem, st, tm[0], tm[1], tm[2], tm[3], tm[4], g);
 }
 
 template <int BN>
@@ -286,9 +314,7 @@ whale_status launch_persistent_t(const CUtensorMap& ta, const CUtensorMap& tb, c
   auto kern = gemm_rownorm_persistent_kernel<BN>;
   CUCHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   const int grid = g.num_tiles < kNumSM ? g.num_tiles : kNumSM;
-  kern<<<grid, kPGemmThreads, smem, st>>>(ta, tb, to, g);
-  CUCHECK(cudaGetLastError());
-  return WHALE_OK;
+  return launch_pdl(kern, dim3(grid), dim3(kPGemmThreads), smem, st, ta, tb, to, g);
 }
 
 // Co-resident 2-CTA clusters of the 2-SM GEMM on the current device (cached per device).
@@ -339,9 +365,7 @@ whale_status gemm_rownorm_2sm(const Opnd& a0, const void* W, int N, const Outs& 
   if (pairs > g.num_tiles) pairs = g.num_tiles;
   auto kern = gemm_rownorm_2sm_kernel;
   CUCHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)G2Smem::BYTES));
-  kern<<<2 * pairs, kG2Threads, G2Smem::BYTES, st>>>(ta, tb, to, g);
-  CUCHECK(cudaGetLastError());
-  return WHALE_OK;
+  return launch_pdl(kern, dim3(2 * pairs), dim3(kG2Threads), G2Smem::BYTES, st, ta, tb, to, g);
 }
 
 // out = r(A) * (A W^T) in bf16, persistent over 128 x BN tiles (BN = 256 when N allows).
@@ -380,9 +404,20 @@ whale_status gemm_bf16(const Opnd& a0, const Opnd& a1, const void* W, int N, con
     if (pairs > 0) return gemm_rownorm_2sm(a0, W, N, out, M, eps, pairs, st);
     return gemm_rownorm_persistent(a0, W, N, out, M, eps, st);
   }
+  // Tile width by a small cost model (cycles): waves over the SMs x (per-CTA fixed cost + per
+  // 64-deep K block the larger of the MMA time and the operand bytes at ~80 B/clk, the rate
+  // one latency-bound CTA streams from L2).
+  const int KB = (a0.K + a1.K) / 64;
+  auto cost = [&](int bn) -> double {
+    if (N % bn) return 1e300;
+    const double waves = (double)cdiv<long long>(tm * (N / bn), kNumSM);
+    const double mma = (split ? 4.0 : 2.0) * bn;
+    const double bytes = (split ? 32768.0 : 16384.0) + bn * 128.0;
+    return waves * (5600.0 + KB * std::max(mma, bytes / 80.0));
+  };
   int bn = 64;
-  if (N % 256 == 0 && tm * (N / 256) >= kNumSM) bn = 256;
-  else if (N % 128 == 0 && tm * (N / 128) >= kNumSM) bn = 128;
+  for (int cand : {128, 256})
+    if (cost(cand) < cost(bn)) bn = cand;
   CUtensorMap maps[5];
   WCHECK(tmap_bf16(&maps[0], a0.hi, M, a0.K, a0.ld, 128));
   if (split) WCHECK(tmap_bf16(&maps[1], a0.lo, M, a0.K, a0.ld, 128));
@@ -422,10 +457,8 @@ inline Opnd no_opnd() { return Opnd{nullptr, nullptr, 0, 0}; }
 whale_status pair_from_bf16(const void* x, float* x32, void* lo, long long n, cudaStream_t st) {
   if (n <= 0) return WHALE_OK;
   const unsigned grid = (unsigned)std::min<long long>(cdiv<long long>(n, 256), 8 * kNumSM);
-  pair_from_bf16_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), x32,
-                                              static_cast<__nv_bfloat16*>(lo), n);
-  CUCHECK(cudaGetLastError());
-  return WHALE_OK;
+  return launch_pdl(pair_from_bf16_kernel, dim3(grid), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(x), x32,
+                    static_cast<__nv_bfloat16*>(lo), n);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -453,9 +486,7 @@ whale_status fold_weights(const Shape& s, const __nv_bfloat16* wq, const float* 
   add(wug, gffn, oug, s.ugw, s.tied ? 0 : 1);
   if (jobs.n == 0) return WHALE_OK;
   const unsigned gx = (unsigned)std::min<long long>(cdiv<long long>(maxe / 8, 256), 8 * kNumSM);
-  fold_weights_kernel<<<dim3(gx, jobs.n), 256, 0, st>>>(jobs);
-  CUCHECK(cudaGetLastError());
-  return WHALE_OK;
+  return launch_pdl(fold_weights_kernel, dim3(gx, jobs.n), dim3(256), 0, st, jobs);
 }
 
 template <int DH, int QT, int HG>
@@ -467,9 +498,7 @@ whale_status launch_attn_t(const CUtensorMap& tm, const AttnArgs& a, dim3 grid, 
   const size_t smem = 1024 + (size_t)ST * stage + 256;
   auto kern = attn_splitl_kernel<DH, QT, T, HG, ST>;
   CUCHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  kern<<<grid, C::THREADS, smem, st>>>(tm, a);
-  CUCHECK(cudaGetLastError());
-  return WHALE_OK;
+  return launch_pdl(kern, grid, dim3(C::THREADS), smem, st, tm, a);
 }
 
 template <int DH, int QT>
@@ -592,7 +621,8 @@ whale_status fusion_mlp_f32(const Shape& s, long long rows, const float* a, cons
 
 bool weights_ok(const Shape& s, const whale_layer_weights* w) {
   auto al = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
-  return w && w->g_q && w->g_kv && w->g_ffn && w->w_q && w->w_kv && w->w_f2 && w->w_upgate && w->w_down &&
+  const bool gains = s.prepared || (w && w->g_q && w->g_kv && w->g_ffn);
+  return w && gains && w->w_q && w->w_kv && w->w_f2 && w->w_upgate && w->w_down &&
          (s.Fh == 0 || w->w_f1) && al(w->g_q) && al(w->g_kv) && al(w->g_ffn) && al(w->w_q) && al(w->w_kv) &&
          al(w->w_f1) && al(w->w_f2) && al(w->w_upgate) && al(w->w_down);
 }
@@ -631,13 +661,18 @@ whale_status layer_bf16(const Shape& s, const Stream3& in, const void* slab, con
                         const whale_layer_weights& w, const Stream3& out, const whale_shape_hint& hint, void* ws,
                         const Layout& L, cudaStream_t st) {
   const long long rows = (long long)hint.B * s.N;
-  auto* wq = at(ws, L.wq);
-  auto* wkv = at(ws, L.wkv);
-  auto* wug = at(ws, L.wug);
-  WCHECK(fold_weights(s, static_cast<const __nv_bfloat16*>(w.w_q), w.g_q, static_cast<const __nv_bfloat16*>(w.w_kv),
-                      w.g_kv, static_cast<const __nv_bfloat16*>(w.w_upgate), w.g_ffn,
-                      reinterpret_cast<__nv_bfloat16*>(wq), reinterpret_cast<__nv_bfloat16*>(wkv),
-                      reinterpret_cast<__nv_bfloat16*>(wug), st));
+  const void* wq = w.w_q;
+  const void* wkv = w.w_kv;
+  const void* wug = w.w_upgate;
+  if (!s.prepared) {
+    wq = at(ws, L.wq);
+    wkv = at(ws, L.wkv);
+    wug = at(ws, L.wug);
+    WCHECK(fold_weights(s, static_cast<const __nv_bfloat16*>(w.w_q), w.g_q, static_cast<const __nv_bfloat16*>(w.w_kv),
+                        w.g_kv, static_cast<const __nv_bfloat16*>(w.w_upgate), w.g_ffn,
+                        reinterpret_cast<__nv_bfloat16*>(at(ws, L.wq)), reinterpret_cast<__nv_bfloat16*>(at(ws, L.wkv)),
+                        reinterpret_cast<__nv_bfloat16*>(at(ws, L.wug)), st));
+  }
   const Opnd X = opnd(in.hi, in.lo, s.d, s.d);
   // S1 queries, S2 keys|values
   WCHECK(gemm_bf16(X, no_opnd(), wq, s.d, Outs{at(ws, L.q), nullptr, nullptr, s.d}, nullptr, 0, rows, EPI_STORE, true,
@@ -795,6 +830,45 @@ const char* whale_status_string(whale_status s) {
     case WHALE_ERR_DEVICE_CHECK: return "device-side check recorded an error";
   }
   return "unknown status";
+}
+
+size_t whale_prepared_weights_size(const whale_config* cfg) {
+  Shape s;
+  if (validate(cfg, &s) != WHALE_OK || !s.bf16) return 0;
+  return (size_t)s.layers *
+         (align_up((size_t)s.d * s.d * 2) + align_up((size_t)s.kvw * s.d * 2) + align_up((size_t)s.ugw * s.d * 2));
+}
+
+whale_status whale_prepare_weights(const whale_config* cfg, const whale_layer_weights* weights, void* prepared,
+                                   size_t prepared_bytes, whale_layer_weights* out_weights, whale_stream_t stream) {
+  Shape s;
+  WCHECK(validate(cfg, &s));
+  if (!s.bf16) return WHALE_ERR_UNSUPPORTED;
+  if (!weights || !out_weights) return WHALE_ERR_INVALID_ARG;
+  s.prepared = false;  // the inputs carry their gains
+  for (int l = 0; l < s.layers; ++l)
+    if (!weights_ok(s, &weights[l])) return WHALE_ERR_INVALID_ARG;
+  if (!prepared || prepared_bytes < whale_prepared_weights_size(cfg) ||
+      (reinterpret_cast<uintptr_t>(prepared) & (kAlign - 1)))
+    return WHALE_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  size_t o = 0;
+  for (int l = 0; l < s.layers; ++l) {
+    const whale_layer_weights& w = weights[l];
+    auto* oq = reinterpret_cast<__nv_bfloat16*>(at(prepared, o));
+    o += align_up((size_t)s.d * s.d * 2);
+    auto* okv = reinterpret_cast<__nv_bfloat16*>(at(prepared, o));
+    o += align_up((size_t)s.kvw * s.d * 2);
+    auto* oug = reinterpret_cast<__nv_bfloat16*>(at(prepared, o));
+    o += align_up((size_t)s.ugw * s.d * 2);
+    WCHECK(fold_weights(s, static_cast<const __nv_bfloat16*>(w.w_q), w.g_q, static_cast<const __nv_bfloat16*>(w.w_kv),
+                        w.g_kv, static_cast<const __nv_bfloat16*>(w.w_upgate), w.g_ffn, oq, okv, oug, st));
+    out_weights[l] = w;
+    out_weights[l].w_q = oq;
+    out_weights[l].w_kv = okv;
+    out_weights[l].w_upgate = oug;
+  }
+  return WHALE_OK;
 }
 
 size_t whale_workspace_size(const whale_config* cfg, const whale_shape_hint* hint) {

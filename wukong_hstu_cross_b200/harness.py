@@ -65,6 +65,7 @@ class Problem:
     out: torch.Tensor
     workspace: torch.Tensor
     flags: dict
+    prepared_buf: torch.Tensor | None = None
 
     @property
     def total_L(self) -> int:
@@ -98,6 +99,17 @@ def build_problem(w: I.Workload, device="cuda", gains="ones", shared_kv=False, t
     out = torch.empty_like(tokens)
     return Problem(w, L, off, lws, tokens, states, torch.from_numpy(off).to(device), weights_to_device(lws, w, device),
                    cfg, hint, out, workspace, {"shared_kv": shared_kv, "tied_gate": tied_gate})
+
+
+def prepare_weights(p: Problem) -> None:
+    """Fold the gains into the weights once (whale_prepare_weights) and switch the problem's
+    config to WHALE_PREPARED_WEIGHTS (bf16 only): what a deployment does at load time."""
+    if p.w.dtype != "bf16":
+        return
+    p.prepared_buf = torch.empty(W.whale_prepared_weights_size(p.cfg), dtype=torch.uint8, device=p.out.device)
+    p.weights = W.whale_prepare_weights(p.cfg, p.weights, p.prepared_buf)
+    p.cfg = W.make_config(p.cfg.n_layers, p.cfg.d, p.cfg.n_heads, p.cfg.n_tokens, p.cfg.ffn_hidden,
+                          p.cfg.fusion_hidden, p.cfg.dtype, p.cfg.flags | W.WHALE_PREPARED_WEIGHTS, p.cfg.eps)
 
 
 def run_forward(p: Problem, stream=None) -> torch.Tensor:

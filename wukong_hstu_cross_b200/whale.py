@@ -16,7 +16,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwhale_fu
 HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "whale_fusion.h")
 
 WHALE_FP32, WHALE_BF16 = 0, 1
-WHALE_SHARED_KV, WHALE_TIED_GATE, WHALE_DEBUG = 1, 2, 4
+WHALE_SHARED_KV, WHALE_TIED_GATE, WHALE_DEBUG, WHALE_PREPARED_WEIGHTS = 1, 2, 4, 8
 WHALE_DEVERR_TIMEOUT, WHALE_DEVERR_OFFSETS = 1, 2
 WHALE_NOALLOC_SCRATCH_BYTES = 32 << 20
 STATUS = {0: "WHALE_OK", 1: "WHALE_ERR_INVALID_ARG", 2: "WHALE_ERR_UNSUPPORTED", 3: "WHALE_ERR_CUDA",
@@ -68,6 +68,9 @@ _SIGS = {
     "whale_fusion_mlp": ([POINTER(whale_config), c_longlong, _P, _P, _P, _P, _P, _P, c_size_t, _P], c_int),
     "whale_swiglu_ffn": ([POINTER(whale_config), c_longlong, _P, _P, _P, _P, _P, _P, c_size_t, _P], c_int),
     "whale_get_device_error": ([_P, POINTER(c_int)], c_int),
+    "whale_prepared_weights_size": ([POINTER(whale_config)], c_size_t),
+    "whale_prepare_weights": ([POINTER(whale_config), POINTER(whale_layer_weights), _P, c_size_t,
+                               POINTER(whale_layer_weights), _P], c_int),
     "whale_cross_attention_noalloc": ([POINTER(whale_config), _P, _P, _P, _P, POINTER(whale_shape_hint), _P], c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
@@ -150,6 +153,23 @@ def _ws_bytes(workspace, nbytes):
     if workspace is None:
         return 0
     return workspace.numel() * workspace.element_size()
+
+
+def whale_prepared_weights_size(cfg: whale_config) -> int:
+    return int(_lib.whale_prepared_weights_size(ctypes.byref(cfg)))
+
+
+def whale_prepare_weights(cfg, weights, prepared, prepared_bytes=None, stream=None, raw=False):
+    """Fold gains / pack up|gate once; returns the ctypes array of prepared layer weights (use it
+    with cfg.flags | WHALE_PREPARED_WEIGHTS). Keep `prepared` alive while it is used."""
+    w = weights if isinstance(weights, ctypes.Array) else weights_array(weights)
+    out = (whale_layer_weights * len(w))()
+    st = _lib.whale_prepare_weights(ctypes.byref(cfg), w, _ptr(prepared), _ws_bytes(prepared, prepared_bytes), out,
+                                    _stream(stream))
+    if raw:
+        return st
+    _check(st, "whale_prepare_weights")
+    return out
 
 
 def whale_fusion_forward(cfg, wukong_tokens, seq_states, seq_offsets, weights, out, hint, workspace,
