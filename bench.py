@@ -32,9 +32,10 @@ from wukong_hstu_cross_b200 import inputs as I  # noqa: E402
 
 METRIC = "WHALE fusion-layer examples/s @15k jagged history; % of HBM/TC roofline"
 # DRAM bytes per launch measured by ncu (dram__bytes_read.sum + dram__bytes_write.sum), per
-# history row, from the committed summary profiles/kv_proj_gemm_hist15k.md (one-SM K|V kernel,
-# d = 512). Reported only for that kernel and width; null otherwise.
-KV_TRAFFIC_BYTES_PER_ROW_D512 = (113.375488e6 + 168.328960e6) / 109605
+# history row, from the committed summary profiles/kv_proj_gemm_hist15k.md (d = 512; the 2-SM
+# default kernel and the one-SM kernel). Reported only for that width; null otherwise.
+KV_TRAFFIC_BYTES_PER_ROW_D512 = {"2sm": (113.380864e6 + 169.296896e6) / 109605,
+                                 "1sm": (113.375488e6 + 168.328960e6) / 109605}
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
 
@@ -369,13 +370,15 @@ def main():
     layer_ms = ms / w.n_layers
     share_kv, share_attn = t_kv / layer_ms, t_attn / layer_ms
     kv_traffic = None
-    if w.d == 512 and os.environ.get("WHALE_GEMM_1SM", "0") == "1":
-        kv_traffic = KV_TRAFFIC_BYTES_PER_ROW_D512 * total_L
+    if w.d == 512 and not args.shared_kv:
+        kv_traffic = KV_TRAFFIC_BYTES_PER_ROW_D512[
+            "1sm" if os.environ.get("WHALE_GEMM_1SM", "0") == "1" else "2sm"] * total_L
     if share_kv >= share_attn:
         roof = {"kernel": "K|V projection GEMM (tcgen05, RMSNorm row factor fused)", "bound": "tensor",
                 "achieved": kv_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": kv_tflops / peaks["bf16_tflops"], "traffic": kv_traffic,
                 "traffic_source": "ncu capture scaled by rows (profiles/kv_proj_gemm_hist15k.md)",
+                "frac_of_sustained": kv_tflops / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
                 "algorithmic_per_launch": work["kv_proj"]["flops"], "avg_launch_ms": t_kv,
                 "peak_source": f"{peak_src} bf16 burst"}
     else:
