@@ -34,7 +34,7 @@ METRIC = "WHALE fusion-layer examples/s @15k jagged history; % of HBM/TC rooflin
 # DRAM bytes per launch measured by ncu (dram__bytes_read.sum + dram__bytes_write.sum), per
 # history row, from the committed summary profiles/kv_proj_gemm_hist15k.md (d = 512; the 2-SM
 # default kernel and the one-SM kernel). Reported only for that width; null otherwise.
-KV_TRAFFIC_BYTES_PER_ROW_D512 = {"2sm": (113.380864e6 + 169.296896e6) / 109605,
+KV_TRAFFIC_BYTES_PER_ROW_D512 = {"2sm": (113.378816e6 + 169.603840e6) / 109605,
                                  "1sm": (113.375488e6 + 168.328960e6) / 109605}
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
