@@ -9,16 +9,19 @@
 // as an fp32 activation times the weight. The token-side (residual-stream) GEMMs use this;
 // the history-side K|V projection reads bf16 states directly.
 //
-// One CTA computes one 128 x BN tile. Warp roles (192 threads):
+// Persistent: CTA c walks the 128 x BN tiles c, c + gridDim.x, ... (N-tiles of a row block are
+// adjacent, so A is re-read from L2, not HBM). Warp roles (192 threads, 320 with ROWNORM):
 //   warp 0      TMA producer: A (hi, lo) and W tiles (64 columns = 128 B, 128-byte swizzle)
 //               into a STAGES-deep ring of shared-memory stages, completion on `full[s]`.
-//   warp 1      allocates BN TMEM columns; one thread issues tcgen05.mma (M=128, N=BN,
-//               K=16 per instruction) and commits each stage back to `empty[s]`.
+//   warp 1      allocates 2 x BN TMEM columns (two accumulators: tile i uses buffer i % 2, so the
+//               epilogue of tile i overlaps the MMAs of tile i+1); one thread issues tcgen05.mma
+//               (M=128, N=BN, K=16 per instruction) and commits each stage back to `empty[s]`.
 //   warps 2..5  epilogue: thread i of the warp with quadrant q = warp % 4 owns output row
-//               32q + i (= TMEM lane). With ROWNORM they also read their row of every A stage
-//               from shared memory while the MMAs run and accumulate sum(x^2), so RMSNorm's
-//               row factor r = 1/sqrt(mean(x^2) + eps) costs no extra pass over A:
-//               RMSNorm(x; g) W^T = r * (x (W diag(g))^T), with diag(g) folded into W beforehand.
+//               32q + i (= TMEM lane).
+//   warps 6..9  (ROWNORM) read their row of every A stage from shared memory while the MMAs run
+//               and accumulate sum(x^2), so RMSNorm's row factor r = 1/sqrt(mean(x^2) + eps)
+//               costs no extra pass over A: RMSNorm(x; g) W^T = r * (x (W diag(g))^T), with
+//               diag(g) folded into W beforehand.
 // Epilogue value per element (fp32): STORE r*acc; SILU silu(acc); RESID acc + resid32;
 // SWIGLU (W rows packed in blocks of 32 = 16 up rows then the 16 matching gate rows)
 // silu(r*gate) * r*up; SWIGLU_TIED (W_gate = W_up) silu(r*u) * r*u. It is then written to
@@ -37,6 +40,7 @@ struct GemmArgs {
   int kb0;                     // 64-column K blocks taken from A0
   int kb1;                     // 64-column K blocks taken from A1 (0: single source)
   int tiles_n;                 // N / BN
+  int num_tiles;               // ceil(M / 128) * tiles_n (CTAs walk tiles blockIdx.x + i * gridDim.x)
   float inv_k;                 // 1 / (K of the normalised source), ROWNORM only
   float eps;                   // RMSNorm epsilon, ROWNORM only
   __nv_bfloat16* out_hi;       // bf16 output (may be null)
@@ -47,7 +51,6 @@ struct GemmArgs {
   long long ldr;
 };
 
-constexpr int kGemmThreads = 192;
 
 template <int BN, bool SPLIT>
 struct GemmSmem {
@@ -57,7 +60,8 @@ struct GemmSmem {
   static constexpr uint32_t B_BYTES = BN * BK * 2;
   static constexpr uint32_t STAGE_BYTES = A_ALL + B_BYTES;
   static constexpr int STAGES = (196608 / STAGE_BYTES) > 8 ? 8 : (196608 / STAGE_BYTES);
-  static constexpr size_t BYTES = 1024 /*alignment slack*/ + STAGES * (size_t)STAGE_BYTES + 256 /*barriers*/;
+  static constexpr size_t BYTES = 1024 /*alignment slack*/ + STAGES * (size_t)STAGE_BYTES + 2 * 128 * 4 /*row factors*/ +
+                                  256 /*barriers*/;
 };
 
 __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
@@ -100,27 +104,33 @@ __device__ __forceinline__ void store_row_chunk(const GemmArgs& g, long long off
   }
 }
 
+template <bool ROWNORM>
+constexpr int gemm_threads() {
+  return ROWNORM ? 320 : 192;
+}
+
 template <int BN, int EPI, bool ROWNORM, bool SPLIT>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA0lo,
                    const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmA1lo,
                    const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
   using L = GemmSmem<BN, SPLIT>;
   constexpr int STAGES = L::STAGES;
-  constexpr uint32_t TMEM_COLS = BN;  // 64, 128 or 256: a power of two >= 32
+  constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators: 128, 256 or 512 columns
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  // stage s: [A hi | A lo (SPLIT) | W]
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * L::STAGE_BYTES);
+  // stage s: [A hi | A lo (SPLIT) | W]; then row factors [2][128]; then barriers
+  float* rbuf = reinterpret_cast<float*>(smem + STAGES * L::STAGE_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(rbuf + 2 * 128);
   uint64_t* empty = full + STAGES;
-  uint64_t* accf = empty + STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  uint64_t* tfull = empty + STAGES;  // [2] accumulator ready (MMA commit)
+  uint64_t* tempty = tfull + 2;      // [2] accumulator drained (4 epilogue warps)
+  uint64_t* nfull = tempty + 2;      // [2] row factors ready (4 statistic warps)
+  uint64_t* edone = nfull + 2;       // [2] row factors consumed (4 epilogue warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(edone + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile_n = blockIdx.x % args.tiles_n;
-  const int tile_m = blockIdx.x / args.tiles_n;
-  const int m0 = tile_m * L::BM, n0 = tile_n * BN;
   const int KB = args.kb0 + args.kb1;
 
   if (threadIdx.x == 0) {
@@ -128,7 +138,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1 + (ROWNORM ? 4 : 0));
     }
-    mbar_init(accf, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 4);
+      mbar_init(&nfull[i], 4);
+      mbar_init(&edone[i], 4);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -154,121 +169,167 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   pdl_trigger();
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
+    // ---------------- TMA producer: every K block of every tile of this CTA ----------------
     if (lane == 0) {
-      int issued = 0;
-      for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % STAGES, u = kb / STAGES;
-        if (kb >= STAGES && !mbar_wait(&empty[s], (u - 1) & 1, abort_flag)) break;
-        uint8_t* st = smem + s * L::STAGE_BYTES;
-        mbar_arrive_expect_tx(&full[s], L::STAGE_BYTES);
-        const bool first = kb < args.kb0;
-        const int kc = (first ? kb : kb - args.kb0) * L::BK;
-        tma_load_2d(st, first ? &tmA0 : &tmA1, kc, m0, &full[s]);
-        if (SPLIT) tma_load_2d(st + L::A_BYTES, first ? &tmA0lo : &tmA1lo, kc, m0, &full[s]);
-        tma_load_2d(st + L::A_ALL, &tmB, kb * L::BK, n0, &full[s]);
-        issued = kb + 1;
+      int kg = 0;
+      bool stop = false;
+      for (int tile = blockIdx.x; tile < args.num_tiles && !stop; tile += gridDim.x) {
+        const int m0 = (tile / args.tiles_n) * L::BM, n0 = (tile % args.tiles_n) * BN;
+        for (int kb = 0; kb < KB; ++kb, ++kg) {
+          const int s = kg % STAGES, u = kg / STAGES;
+          if (kg >= STAGES && !mbar_wait(&empty[s], (u - 1) & 1, abort_flag)) {
+            stop = true;
+            break;
+          }
+          uint8_t* st = smem + s * L::STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[s], L::STAGE_BYTES);
+          const bool first = kb < args.kb0;
+          const int kc = (first ? kb : kb - args.kb0) * L::BK;
+          tma_load_2d(st, first ? &tmA0 : &tmA1, kc, m0, &full[s]);
+          if (SPLIT) tma_load_2d(st + L::A_BYTES, first ? &tmA0lo : &tmA1lo, kc, m0, &full[s]);
+          tma_load_2d(st + L::A_ALL, &tmB, kb * L::BK, n0, &full[s]);
+        }
       }
       if (*abort_flag) {
         // Unwinding after a timeout: let the copies this thread started land before the CTA exits.
         volatile int quiet = 0;
-        for (int kb = (issued > STAGES ? issued - STAGES : 0); kb < issued; ++kb)
-          mbar_wait(&full[kb % STAGES], (kb / STAGES) & 1, &quiet);
+        for (int k = (kg > STAGES ? kg - STAGES : 0); k < kg; ++k)
+          mbar_wait(&full[k % STAGES], (k / STAGES) & 1, &quiet);
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
+    // ---------------- MMA issuer: tile i accumulates into buffer i % 2 ----------------
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
-      for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % STAGES, u = kb / STAGES;
-        if (!mbar_wait(&full[s], u & 1, abort_flag)) break;
+      int kg = 0, it = 0;
+      bool stop = false;
+      for (int tile = blockIdx.x; tile < args.num_tiles && !stop; tile += gridDim.x, ++it) {
+        const int acc = it & 1, ua = it >> 1;
+        if (it >= 2 && !mbar_wait(&tempty[acc], (ua - 1) & 1, abort_flag)) break;
         tc_fence_after();
-        const uint32_t a_base = smem_u32(smem + s * L::STAGE_BYTES);
-        const uint32_t b_base = a_base + L::A_ALL;
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < KB; ++kb, ++kg) {
+          const int s = kg % STAGES, u = kg / STAGES;
+          if (!mbar_wait(&full[s], u & 1, abort_flag)) {
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + s * L::STAGE_BYTES);
+          const uint32_t b_base = a_base + L::A_ALL;
 #pragma unroll
-        for (int kk = 0; kk < L::BK / 16; ++kk) {
-          const uint64_t bdesc = sdesc_k_sw128(b_base + kk * 32);
-          umma_f16(tmem_base, sdesc_k_sw128(a_base + kk * 32), bdesc, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
-          if (SPLIT) umma_f16(tmem_base, sdesc_k_sw128(a_base + L::A_BYTES + kk * 32), bdesc, idesc, 1u);
+          for (int kk = 0; kk < L::BK / 16; ++kk) {
+            const uint64_t bdesc = sdesc_k_sw128(b_base + kk * 32);
+            umma_f16(d_tmem, sdesc_k_sw128(a_base + kk * 32), bdesc, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            if (SPLIT) umma_f16(d_tmem, sdesc_k_sw128(a_base + L::A_BYTES + kk * 32), bdesc, idesc, 1u);
+          }
+          umma_commit(&empty[s]);
         }
-        umma_commit(&empty[s]);
+        umma_commit(&tfull[acc]);  // also on abort: arrives once all issued MMAs are done
       }
-      umma_commit(accf);  // also on abort: arrives once all issued MMAs are done
+    }
+  } else if (warp >= 6) {
+    // ---------------- row statistics (ROWNORM): sum of squares of each A row ----------------
+    if (ROWNORM) {
+      const int row = (warp & 3) * 32 + lane;
+      int kg = 0, it = 0;
+      for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x, ++it) {
+        const int acc = it & 1, ua = it >> 1;
+        float ss = 0.f;
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb, ++kg) {
+          const int s = kg % STAGES, u = kg / STAGES;
+          if (!mbar_wait(&full[s], u & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          if (kb < args.kb0) {
+            // The row's 128 bytes are contiguous; the 128-byte swizzle stores its logical 16-byte
+            // chunk c at position c ^ (row % 8) (identically in the hi and lo tiles). Summing in
+            // logical order keeps the row factor independent of the row's position in the tile.
+            const uint8_t* st = smem + s * L::STAGE_BYTES + row * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const int pc = c ^ (row & 7);
+              float f[8];
+              bf16x8_to_f32(reinterpret_cast<const uint4*>(st)[pc], f);
+              if (SPLIT) {
+                float fl[8];
+                bf16x8_to_f32(reinterpret_cast<const uint4*>(st + L::A_BYTES)[pc], fl);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) f[j] += fl[j];
+              }
+#pragma unroll
+              for (int j = 0; j < 8; ++j) ss = fmaf(f[j], f[j], ss);
+            }
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[s]);
+        }
+        if (!ok) break;
+        if (it >= 2 && !mbar_wait(&edone[acc], (ua - 1) & 1, abort_flag)) break;
+        rbuf[acc * 128 + row] = rsqrtf(ss * args.inv_k + args.eps);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&nfull[acc]);
+      }
     }
   } else {
-    // ---------------- row statistics + epilogue (warps 2..5) ----------------
+    // ---------------- epilogue (warps 2..5): thread i of quadrant q owns row 32q + i ----------------
     const int q = warp & 3;
     const int row = q * 32 + lane;
-    float ss = 0.f;
-    if (ROWNORM) {
-      for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % STAGES, u = kb / STAGES;
-        if (!mbar_wait(&full[s], u & 1, abort_flag)) break;
-        if (kb < args.kb0) {
-          // The row's 128 bytes are contiguous; the 128-byte swizzle stores its logical 16-byte
-          // chunk c at position c ^ (row % 8) (identically in the hi and lo tiles). Summing in
-          // logical order keeps the row factor independent of the row's position in the tile.
-          const uint8_t* st = smem + s * L::STAGE_BYTES + row * 128;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const int pc = c ^ (row & 7);
-            float f[8];
-            bf16x8_to_f32(reinterpret_cast<const uint4*>(st)[pc], f);
-            if (SPLIT) {
-              float fl[8];
-              bf16x8_to_f32(reinterpret_cast<const uint4*>(st + L::A_BYTES)[pc], fl);
-#pragma unroll
-              for (int j = 0; j < 8; ++j) f[j] += fl[j];
-            }
-#pragma unroll
-            for (int j = 0; j < 8; ++j) ss = fmaf(f[j], f[j], ss);
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
-      }
-    }
-    const bool ok = mbar_wait(accf, 0, abort_flag);
-    tc_fence_after();
-    const float r = ROWNORM ? rsqrtf(ss * args.inv_k + args.eps) : 1.0f;
-    const long long gm = (long long)m0 + row;
-    const bool row_ok = ok && gm < args.M;
-    const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16);
+    int it = 0;
+    for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x, ++it) {
+      const int acc = it & 1, ua = it >> 1;
+      const int m0 = (tile / args.tiles_n) * L::BM, n0 = (tile % args.tiles_n) * BN;
+      if (!mbar_wait(&tfull[acc], ua & 1, abort_flag)) break;
+      if (ROWNORM && !mbar_wait(&nfull[acc], ua & 1, abort_flag)) break;
+      tc_fence_after();
+      const float r = ROWNORM ? rbuf[acc * 128 + row] : 1.0f;
+      const long long gm = (long long)m0 + row;
+      const bool row_ok = gm < args.M;
+      const uint32_t t_row = tmem_base + acc * BN + ((uint32_t)(q * 32) << 16);
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(t_row + c * 32, v);
-      tmem_ld_wait();
-      const int col = n0 + c * 32;
-      if (!row_ok || col >= args.N) continue;
-      float x[32];
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(t_row + c * 32, v);
+        tmem_ld_wait();
+        const int col = n0 + c * 32;
+        if (!row_ok || col >= args.N) continue;
+        float x[32];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(v[j]) * r;
-      if (EPI == EPI_SWIGLU) {
-        float h[16];
+        for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(v[j]) * r;
+        if (EPI == EPI_SWIGLU) {
+          float h[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) h[j] = silu_f(x[16 + j]) * x[j];
-        store_row_chunk<16>(args, gm * args.ldo + col / 2, h);
-      } else {
-        if (EPI == EPI_RESID) {
-          const float4* rp = reinterpret_cast<const float4*>(args.resid32 + gm * args.ldr + col);
+          for (int j = 0; j < 16; ++j) h[j] = silu_f(x[16 + j]) * x[j];
+          store_row_chunk<16>(args, gm * args.ldo + col / 2, h);
+        } else {
+          if (EPI == EPI_RESID) {
+            const float4* rp = reinterpret_cast<const float4*>(args.resid32 + gm * args.ldr + col);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float4 t = rp[i];
-            x[4 * i] += t.x;
-            x[4 * i + 1] += t.y;
-            x[4 * i + 2] += t.z;
-            x[4 * i + 3] += t.w;
+            for (int i = 0; i < 8; ++i) {
+              const float4 t = rp[i];
+              x[4 * i] += t.x;
+              x[4 * i + 1] += t.y;
+              x[4 * i + 2] += t.z;
+              x[4 * i + 3] += t.w;
+            }
+          } else if (EPI == EPI_SILU) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) x[j] = silu_f(x[j]);
+          } else if (EPI == EPI_SWIGLU_TIED) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) x[j] = silu_f(x[j]) * x[j];
           }
-        } else if (EPI == EPI_SILU) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) x[j] = silu_f(x[j]);
-        } else if (EPI == EPI_SWIGLU_TIED) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) x[j] = silu_f(x[j]) * x[j];
+          store_row_chunk<32>(args, gm * args.ldo + col, x);
         }
-        store_row_chunk<32>(args, gm * args.ldo + col, x);
+      }
+      // this accumulator buffer and its row factors may be reused
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&tempty[acc]);
+        mbar_arrive(&edone[acc]);
       }
     }
   }

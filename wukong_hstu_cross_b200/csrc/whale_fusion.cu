@@ -291,7 +291,8 @@ whale_status launch_gemm_t(const CUtensorMap* tm, const GemmArgs& g, long long t
   const size_t smem = GemmSmem<BN, SPLIT>::BYTES;
   auto kern = gemm_tc_kernel<BN, EPI, RN, SPLIT>;
   CUCHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  return launch_pdl(kern, dim3((unsigned)tiles), dim3(kGemmThreads), smem, st, tm[0], tm[1], tm[2], tm[3], tm[4], g);
+  const unsigned grid = (unsigned)(tiles < kNumSM ? tiles : kNumSM);
+  return launch_pdl(kern, dim3(grid), dim3(gemm_threads<RN>()), smem, st, tm[0], tm[1], tm[2], tm[3], tm[4], g);
 }
 
 template <int BN>
@@ -404,16 +405,16 @@ whale_status gemm_bf16(const Opnd& a0, const Opnd& a1, const void* W, int N, con
     if (pairs > 0) return gemm_rownorm_2sm(a0, W, N, out, M, eps, pairs, st);
     return gemm_rownorm_persistent(a0, W, N, out, M, eps, st);
   }
-  // Tile width by a small cost model (cycles): waves over the SMs x (per-CTA fixed cost + per
-  // 64-deep K block the larger of the MMA time and the operand bytes at ~80 B/clk, the rate
+  // Tile width by a small cost model (cycles): per-CTA fixed cost + tiles per persistent CTA x
+  // (per 64-deep K block the larger of the MMA time and the operand bytes at ~80 B/clk, the rate
   // one latency-bound CTA streams from L2).
   const int KB = (a0.K + a1.K) / 64;
   auto cost = [&](int bn) -> double {
     if (N % bn) return 1e300;
-    const double waves = (double)cdiv<long long>(tm * (N / bn), kNumSM);
+    const double per_cta = (double)cdiv<long long>(tm * (N / bn), kNumSM);  // tiles per persistent CTA
     const double mma = (split ? 4.0 : 2.0) * bn;
     const double bytes = (split ? 32768.0 : 16384.0) + bn * 128.0;
-    return waves * (5600.0 + KB * std::max(mma, bytes / 80.0));
+    return 5600.0 + per_cta * KB * std::max(mma, bytes / 80.0);
   };
   int bn = 64;
   for (int cand : {128, 256})
@@ -437,6 +438,7 @@ whale_status gemm_bf16(const Opnd& a0, const Opnd& a1, const void* W, int N, con
   g.kb0 = a0.K / 64;
   g.kb1 = a1.K / 64;
   g.tiles_n = N / bn;
+  g.num_tiles = (int)(tm * g.tiles_n);
   g.inv_k = 1.0f / (float)a0.K;
   g.eps = eps;
   g.out_hi = static_cast<__nv_bfloat16*>(out.hi);
