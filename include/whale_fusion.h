@@ -64,8 +64,11 @@ typedef enum { WHALE_FP32 = 0, WHALE_BF16 = 1 } whale_dtype;
 #define WHALE_SHARED_KV 1u  /* K = V: w_kv is W_K alone [d, d] (gist.science 2.2 "Shared Key-Value") */
 #define WHALE_TIED_GATE 2u  /* W_gate = W_up: w_upgate is W_up alone [H, d] (gist.science 2.2 "Shared-Gate SwiGLU") */
 #define WHALE_DEBUG 4u      /* validate offsets on the device before the forward */
-#define WHALE_PREPARED_WEIGHTS 8u  /* bf16: w_q, w_kv, w_upgate come from whale_prepare_weights (gains
-                                      already folded in, up|gate rows packed); g_* are not read */
+#define WHALE_PREPARED_WEIGHTS 8u  /* bf16: w_q, w_kv, w_upgate (and w_kabs) come from
+                                      whale_prepare_weights (gains already folded in, up|gate rows
+                                      packed); g_* are not read */
+#define WHALE_MATERIALIZED_KV 16u  /* bf16: always project K|V and attend over them, even where the
+                                      absorbed path (below) applies */
 
 /* device error bits (whale_get_device_error) */
 #define WHALE_DEVERR_TIMEOUT 1
@@ -79,13 +82,24 @@ typedef struct {
   int ffn_hidden;     /* SwiGLU hidden width H (4d in the pages' setting) */
   int fusion_hidden;  /* Fusion MLP hidden width (2d); 0 = one linear map W_F [d, 2d] */
   int dtype;          /* whale_dtype */
-  unsigned flags;     /* WHALE_SHARED_KV | WHALE_TIED_GATE | WHALE_DEBUG */
+  unsigned flags;     /* WHALE_SHARED_KV | WHALE_TIED_GATE | WHALE_DEBUG | WHALE_PREPARED_WEIGHTS |
+                         WHALE_MATERIALIZED_KV */
   float eps;          /* RMSNorm epsilon */
 } whale_config;
 /* Supported: fp32 — any d with d % n_heads == 0, d_head <= 128 (SIMT correctness path).
  *            bf16 — d % 64 == 0, d_head in {32, 64}, n_heads / (heads per CTA) integral
  *            (heads per CTA = min(n_heads, 8), its d_head multiple of 64 columns),
- *            ffn_hidden % 64 == 0, fusion_hidden % 64 == 0. Any n_tokens >= 1. */
+ *            ffn_hidden % 64 == 0, fusion_hidden % 64 == 0. Any n_tokens >= 1.
+ *
+ * Absorbed attention (bf16, the default where it applies: n_tokens * n_heads == 256, d_head == 64,
+ * d in {256, 512}, WHALE_MATERIALIZED_KV not set). The key and value projections are folded into
+ * the queries, which is exact algebra for Eq. (4) with RMSNorm'd states:
+ *   q_j . K_t,j = r_t * (H_t . qa),  qa = diag(g_kv) W_K,j^T q_j;   sum_t p_t V_t,j = z W'_V,j^T,
+ *   z = sum_t p_t r_t H_t,  W'_V = W_V diag(g_kv),
+ * so the history states are read twice and no K|V tensor is formed: 2 (N h) d instead of 2 d^2
+ * multiply-adds per history row. Results agree with the materialising path to bf16 rounding, not
+ * bit for bit. It assumes finite states: the last 256-row unit of an example multiplies the zero
+ * weights of its padding columns with the following rows of the slab. */
 
 /* Per-layer weights: device pointers. Element type cfg->dtype, gains fp32. */
 typedef struct {
@@ -98,6 +112,8 @@ typedef struct {
   const float* g_ffn;    /* [d]   RMSNorm gain before the SwiGLU FFN */
   const void* w_upgate;  /* [2H, d] = [W_up ; W_gate] ([H, d] with WHALE_TIED_GATE) */
   const void* w_down;    /* [d, H] */
+  const void* w_kabs;    /* prepared weights only (may be null): per-head absorbed key weights from
+                            whale_prepare_weights, [n_heads * d, d_head]; null = formed per call */
 } whale_layer_weights;
 
 /* Host-side sizes, so no device->host read is needed to launch.
@@ -122,8 +138,11 @@ size_t whale_workspace_size(const whale_config* cfg, const whale_shape_hint* hin
  * gate rows) for the fused SwiGLU epilogue. The results go to `prepared` (device, at least
  * whale_prepared_weights_size bytes, 256-byte aligned, owned by the caller), and `out_weights`
  * (host array of n_layers) receives the input pointers with w_q, w_kv, w_upgate replaced by the
- * prepared copies. Forwards given out_weights with cfg->flags | WHALE_PREPARED_WEIGHTS skip the
- * per-call fold. Asynchronous on `stream`; the inputs must stay valid until it completes. */
+ * prepared copies. Where the absorbed attention applies (see whale_config) it also forms the
+ * per-head absorbed key weights w_kabs[j*d + n][k] = W_K[j*d_head + k][n] g_kv[n] log2(e)/sqrt(d_head)
+ * and sets out_weights[l].w_kabs (null otherwise). Forwards given out_weights with
+ * cfg->flags | WHALE_PREPARED_WEIGHTS skip the per-call fold. Asynchronous on `stream`; the inputs
+ * must stay valid until it completes. */
 size_t whale_prepared_weights_size(const whale_config* cfg);
 whale_status whale_prepare_weights(const whale_config* cfg, const whale_layer_weights* weights, void* prepared,
                                    size_t prepared_bytes, whale_layer_weights* out_weights, whale_stream_t stream);

@@ -1,0 +1,761 @@
+// absorbed.cuh — Eq. (4) of WHALE with the key and value projections folded into the queries
+// (gist.science technical summary of WHALE, section 2.1 "Core Architecture", Attention-Based
+// Fusion Module; pith.science verdict, "key_machinery"). For query q = (head j, token n) of
+// example b and history row t with RMSNorm row factor r_t = 1/sqrt(mean(H_t^2) + eps):
+//
+//   q_j . K_{t,j} / sqrt(d_h) = r_t * (H_t . qa_q),     qa_q = diag(g_kv) W_K,j^T q_j / sqrt(d_h)
+//   sum_t p_{q,t} V_{t,j}     = (sum_t p_{q,t} r_t H_t) . diag(g_kv) W_V,j^T = z_q W'_V,j^T
+//
+// which is exact algebra. Per history row this costs 2 * (N h) * d multiply-adds instead of the
+// 2 d^2 of projecting K and V (and no K|V tensor is written or re-read), so it is the path taken
+// when N h <= d. Work is done in units of 256 history rows of one example by a CTA pair (cluster
+// of two, cta_group::2 MMAs; CTA r holds queries [128 r, 128 r + 128) of the example's 256):
+//
+//   pass A  S = qa H_u^T (M = 256 queries, N = 256 rows, K = d), r_t applied per column, online
+//           softmax per query in base 2 with a lazy reference (raised only when a tile maximum
+//           exceeds it by kAbsLazy): writes pw = p * r_t (bf16), the reference of every unit, and
+//           (m, l) of every segment.
+//   pass B  z += pw_u H_u (M = 256 queries, N = d, K = 256 rows; H as an MN-major operand),
+//           rescaling the TMEM accumulator whenever pass A raised a reference; writes z / l of
+//           examples held by one pair, or an unnormalised partial.
+//   merge   combines the partials of examples split across pairs (log-sum-exp weights).
+//
+// Both passes give the P pairs contiguous ranges of the flattened unit index (units of example b
+// are [ustart[b], ustart[b+1])); a range cut inside an example makes a partial segment, stored
+// in slot 2p (the range's first segment) or 2p + 1 (its last).
+#pragma once
+
+#include "gemm_tc.cuh"
+#include "ptx.cuh"
+
+namespace whale {
+
+constexpr int kAbsRows = 256;      // history rows per unit
+constexpr int kAbsQ = 256;         // absorbed queries per example (N * h)
+constexpr float kAbsLazy = 8.0f;   // log2 headroom before the softmax reference is raised
+
+struct AbsArgs {
+  const int* offsets;       // [B+1]
+  const int* ustart;        // [B+1] first unit of each example; ustart[B] = number of units
+  int B, N, d;              // examples, tokens per example, width
+  int n_pairs;
+  long long total_L;
+  float inv_d, eps;
+  float* mref;              // [units_max, 256] softmax reference of each unit (log2 units)
+  float* stats_whole;       // [B, 256] (m, l) of examples held by one pair
+  float* stats_part;        // [2 * n_pairs, 256] (m, l) of partial segments
+  float* part_z;            // [2 * n_pairs, 256, d] unnormalised z of partial segments
+  __nv_bfloat16* z_hi;      // [h, B*N, d] z / l, bf16 pair (row j*B*N + b*N + n)
+  __nv_bfloat16* z_lo;
+};
+
+__device__ __forceinline__ long long abs_off(const AbsArgs& a, int b) {
+  long long o = a.offsets[b];
+  return o < 0 ? 0 : (o > a.total_L ? a.total_L : o);
+}
+
+__device__ __forceinline__ int abs_range_start(int U, int P, int p) { return (int)(((long long)U * p) / P); }
+
+// Pair whose range holds unit u (0 <= u < U).
+__device__ __forceinline__ int abs_pair_of(int u, int U, int P) {
+  int p = (int)(((long long)u * P) / U);
+  if (p > P - 1) p = P - 1;
+  while (p + 1 < P && abs_range_start(U, P, p + 1) <= u) ++p;
+  while (p > 0 && abs_range_start(U, P, p) > u) --p;
+  return p;
+}
+
+// Walk over the units [u0, u1) of one pair, tracking the example they belong to.
+struct AbsWalk {
+  int u, u0, u1, p;
+  int b, ub, ub1;  // example of u and its unit range
+  __device__ __forceinline__ void init(const AbsArgs& a, int p_) {
+    p = p_;
+    const int U = a.ustart[a.B];
+    u0 = abs_range_start(U, a.n_pairs, p);
+    u1 = abs_range_start(U, a.n_pairs, p + 1);
+    u = u0;
+    b = 0;
+    ub = ub1 = 0;
+    if (u < u1) {
+      int lo = 0, hi = a.B - 1;  // largest b with ustart[b] <= u (non-empty since u < ustart[B])
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (a.ustart[mid] <= u) lo = mid;
+        else hi = mid - 1;
+      }
+      b = lo;
+      ub = a.ustart[b];
+      ub1 = a.ustart[b + 1];
+    }
+  }
+  __device__ __forceinline__ bool valid() const { return u < u1; }
+  __device__ __forceinline__ void next(const AbsArgs& a) {
+    ++u;
+    if (u < u1 && u >= ub1) {
+      do {
+        ++b;
+      } while (a.ustart[b + 1] <= u);
+      ub = a.ustart[b];
+      ub1 = a.ustart[b + 1];
+    }
+  }
+};
+
+struct AbsUnit {
+  int b, t, nvalid, pcol0, slot;
+  long long row0;            // first history row of the unit
+  bool first, last, whole;   // first / last unit of its segment; segment = the whole example
+};
+
+__device__ __forceinline__ AbsUnit abs_unit(const AbsArgs& a, const AbsWalk& w) {
+  AbsUnit un;
+  un.b = w.b;
+  un.t = w.u - w.ub;
+  const long long lo = abs_off(a, w.b);
+  long long hi = abs_off(a, w.b + 1);
+  if (hi < lo) hi = lo;
+  un.row0 = lo + (long long)kAbsRows * un.t;
+  const long long nv = hi - un.row0;
+  un.nvalid = nv > kAbsRows ? kAbsRows : (nv < 1 ? 1 : (int)nv);
+  un.pcol0 = w.u * kAbsRows;
+  un.first = (w.u == w.u0) || (un.t == 0);
+  un.last = (w.u == w.u1 - 1) || (w.u == w.ub1 - 1);
+  un.whole = (w.u0 <= w.ub) && (w.u1 >= w.ub1);
+  un.slot = (w.u0 >= w.ub) ? 2 * w.p : 2 * w.p + 1;
+  return un;
+}
+
+// ustart[b] = sum_{b' < b} ceil(L_b' / 256), capped at units_max (only inconsistent offsets reach
+// the cap; they lose rows, never index past the buffers). One block of 1024 threads.
+__global__ void __launch_bounds__(1024) abs_units_kernel(const int* __restrict__ offsets, int B, long long total_L,
+                                                         int units_max, int* __restrict__ ustart) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ int part[1024];
+  const int per = (B + 1023) / 1024;
+  const int b0 = threadIdx.x * per, b1 = min(B, b0 + per);
+  auto clampo = [&](int b) -> long long {
+    long long o = offsets[b];
+    return o < 0 ? 0 : (o > total_L ? total_L : o);
+  };
+  long long sum = 0;
+  for (int b = b0; b < b1; ++b) {
+    const long long L = clampo(b + 1) - clampo(b);
+    if (L > 0) sum += (L + kAbsRows - 1) / kAbsRows;
+  }
+  part[threadIdx.x] = (int)(sum < units_max ? sum : units_max);
+  __syncthreads();
+  for (int off = 1; off < 1024; off <<= 1) {  // inclusive scan (values capped, no overflow)
+    const int v = threadIdx.x >= off ? part[threadIdx.x - off] : 0;
+    __syncthreads();
+    part[threadIdx.x] = min(part[threadIdx.x] + v, units_max);
+    __syncthreads();
+  }
+  long long run = threadIdx.x > 0 ? part[threadIdx.x - 1] : 0;
+  for (int b = b0; b < b1; ++b) {
+    ustart[b] = (int)run;
+    const long long L = clampo(b + 1) - clampo(b);
+    if (L > 0) run += (L + kAbsRows - 1) / kAbsRows;
+    if (run > units_max) run = units_max;
+  }
+  if (threadIdx.x == 1023) ustart[B] = part[1023];
+}
+
+// ================================================================================================
+// pass A: S = qa H^T, online softmax, pw = p * r
+// ================================================================================================
+struct AbsASmem {
+  static constexpr int BK = 64;
+  static constexpr uint32_t A_BYTES = 128 * BK * 2;   // 128 absorbed queries (this CTA's)
+  static constexpr uint32_t B_BYTES = 128 * BK * 2;   // this CTA's 128 history rows of the unit
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t EPI_BYTES = 8 * 4096;     // one 32 x 64 bf16 staging tile per epilogue warp
+  static constexpr int XCH = 2 * 256 * 4 + 2 * 2 * 128 * 4 + 2 * 128 * 4;  // r[2][256], max[2][2][128], l[2][128]
+  static constexpr int FIXED = 1024 + EPI_BYTES + XCH + 512;
+  static constexpr int STAGES = (232448 - FIXED) / (int)STAGE_BYTES > 8 ? 8 : (232448 - FIXED) / (int)STAGE_BYTES;
+  static constexpr size_t BYTES = FIXED + STAGES * (size_t)STAGE_BYTES;
+};
+constexpr int kAbsAThreads = 480;
+
+// warps: 0 TMA producer (both CTAs), 1 TMEM (2 x 256 columns) + MMA issue (even CTA), 2..9 softmax
+// epilogue (two warps per lane quadrant, 128 columns each), 10..13 row statistics of this CTA's 128
+// history rows (r of all 256 columns reaches both CTAs through distributed shared memory), 14 relay
+// of "stage landed" (even CTA) as in the 2-SM projection GEMM.
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
+    abs_scores_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmH,
+                      const __grid_constant__ CUtensorMap tmP, const AbsArgs a) {
+  using L = AbsASmem;
+  constexpr int ST = L::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* epi = smem + ST * L::STAGE_BYTES;
+  float* rbuf = reinterpret_cast<float*>(epi + L::EPI_BYTES);  // [2][256]
+  float* xmax = rbuf + 2 * 256;                                // [2 acc][2 half][128]
+  float* xsum = xmax + 2 * 2 * 128;                            // [2 half][128]
+  uint64_t* full = reinterpret_cast<uint64_t*>(xsum + 2 * 128);
+  uint64_t* ready = full + ST;
+  uint64_t* empty = ready + ST;
+  uint64_t* tfull = empty + ST;   // [2]
+  uint64_t* tempty = tfull + 2;   // [2] (even CTA: 8 + 8 epilogue warps)
+  uint64_t* nfull = tempty + 2;   // [2] 4 local + 4 peer statistic warps
+  uint64_t* edone = nfull + 2;    // [2] 8 local + 8 peer epilogue warps
+  uint64_t* xbar = edone + 2;     // [4 quadrants][2 acc] tile maxima of both half-warps written
+  uint64_t* lbar = xbar + 8;      // [4 quadrants] segment sums of both half-warps written
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lbar + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int KB = a.d / 64;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&ready[s], 1);
+      mbar_init(&empty[s], 1 + 4);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 16);
+      mbar_init(&nfull[i], 8);
+      mbar_init(&edone[i], 16);
+    }
+    for (int i = 0; i < 8; ++i) mbar_init(&xbar[i], 2);
+    for (int i = 0; i < 4; ++i) mbar_init(&lbar[i], 2);
+    *abort_flag = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmH);
+    tma_prefetch_desc(&tmP);
+  }
+  if (warp == 1) {
+    tmem_alloc_cg2(tmem_slot, 512);
+    tmem_relinquish_cg2();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
+
+  AbsWalk wk;
+  wk.init(a, pair);
+
+  if (warp == 0) {
+    // ---------------- TMA producer (both CTAs) ----------------
+    if (lane == 0) {
+      int kg = 0;
+      bool stop = false;
+      for (; wk.valid() && !stop; wk.next(a)) {
+        const AbsUnit un = abs_unit(a, wk);
+        const int qrow = un.b * kAbsQ + (int)rank * 128;
+        const int hrow = (int)un.row0 + (int)rank * 128;
+        for (int kb = 0; kb < KB; ++kb, ++kg) {
+          const int s = kg % ST, u = kg / ST;
+          if (kg >= ST && !mbar_wait(&empty[s], (u - 1) & 1, abort_flag)) {
+            stop = true;
+            break;
+          }
+          uint8_t* st = smem + s * L::STAGE_BYTES;
+          const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
+          if (leader) mbar_arrive_expect_tx(&full[s], 2 * L::STAGE_BYTES);
+          tma_load_2d_cg2(st, &tmQ, kb * L::BK, qrow, bar);
+          tma_load_2d_cg2(st + L::A_BYTES, &tmH, kb * L::BK, hrow, bar);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (even CTA) ----------------
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(256, 256);
+      int kg = 0, it = 0;
+      bool stop = false;
+      for (; wk.valid() && !stop; wk.next(a), ++it) {
+        const int acc = it & 1, ua = it >> 1;
+        if (it >= 2 && !mbar_wait(&tempty[acc], (ua - 1) & 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * 256;
+        for (int kb = 0; kb < KB; ++kb, ++kg) {
+          const int s = kg % ST, u = kg / ST;
+          if (!mbar_wait(&full[s], u & 1, abort_flag)) {
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + s * L::STAGE_BYTES);
+          const uint32_t b_base = a_base + L::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < L::BK / 16; ++kk)
+            umma_f16_cg2(d_tmem, sdesc_k_sw128(a_base + kk * 32), sdesc_k_sw128(b_base + kk * 32), idesc,
+                         (kb > 0 || kk > 0) ? 1u : 0u);
+          umma_commit_cg2_mc(&empty[s], 0x3);
+        }
+        umma_commit_cg2_mc(&tfull[acc], 0x3);
+      }
+    }
+  } else if (warp == 14) {
+    // ---------------- relay (even CTA) ----------------
+    if (leader && lane == 0) {
+      const uint32_t peer_ready0 = mapa_shared(smem_u32(&ready[0]), 1);
+      const int total = (wk.u1 - wk.u0) * KB;
+      for (int kg = 0; kg < total; ++kg) {
+        const int s = kg % ST, u = kg / ST;
+        if (!mbar_wait(&full[s], u & 1, abort_flag)) break;
+        mbar_arrive(&ready[s]);
+        mbar_arrive_cluster(peer_ready0 + s * 8);
+      }
+    }
+  } else if (warp >= 10) {
+    // ---------------- row statistics of this CTA's 128 history rows (both CTAs) ----------------
+    const int row = (warp & 3) * 32 + lane;
+    const uint32_t rb_peer = mapa_shared(smem_u32(rbuf), rank ^ 1);
+    const uint32_t nfull_peer0 = mapa_shared(smem_u32(&nfull[0]), rank ^ 1);
+    int kg = 0, it = 0;
+    for (; wk.valid(); wk.next(a), ++it) {
+      const int acc = it & 1, ua = it >> 1;
+      float ss = 0.f;
+      bool ok = true;
+      for (int kb = 0; kb < KB; ++kb, ++kg) {
+        const int s = kg % ST, u = kg / ST;
+        if (!mbar_wait(&ready[s], u & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const uint4* rp = reinterpret_cast<const uint4*>(smem + s * L::STAGE_BYTES + L::A_BYTES + row * 128);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          float f[8];
+          bf16x8_to_f32(rp[c ^ (row & 7)], f);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) ss = fmaf(f[j], f[j], ss);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+      }
+      if (!ok) break;
+      // both CTAs' epilogues must be done with this buffer before either side rewrites it
+      if (it >= 2 && !mbar_wait_cluster(&edone[acc], (ua - 1) & 1, abort_flag)) break;
+      const float rv = rsqrtf(ss * a.inv_d + a.eps);
+      const int idx = acc * 256 + (int)rank * 128 + row;
+      rbuf[idx] = rv;
+      st_shared_cluster_f32(rb_peer + idx * 4, rv);
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&nfull[acc]);
+        mbar_arrive_cluster_release(nfull_peer0 + acc * 8);
+      }
+    }
+  } else {
+    // ---------------- softmax epilogue (warps 2..9, both CTAs) ----------------
+    const int qd = warp & 3;
+    const int hf = (warp - 2) >> 2;  // columns [128 hf, 128 hf + 128) of the unit
+    const int row = qd * 32 + lane;
+    const int qg = (int)rank * 128 + row;
+    uint8_t* sbuf = epi + (warp - 2) * 4096;
+    const uint32_t tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
+    const uint32_t edone_peer0 = mapa_shared(smem_u32(&edone[0]), rank ^ 1);
+    float m_run = 0.f, l_part = 0.f;
+    int it = 0, nseg = 0;
+    for (; wk.valid(); wk.next(a), ++it) {
+      const AbsUnit un = abs_unit(a, wk);
+      const int acc = it & 1, ua = it >> 1;
+      if (!mbar_wait(&tfull[acc], ua & 1, abort_flag)) break;
+      if (!mbar_wait_cluster(&nfull[acc], ua & 1, abort_flag)) break;
+      tc_fence_after();
+      const float* r = rbuf + acc * 256 + hf * 128;
+      const uint32_t t0 = tmem_base + acc * 256 + hf * 128 + ((uint32_t)(qd * 32) << 16);
+      const int nv = un.nvalid - hf * 128;  // valid columns of this warp's half (may be <= 0)
+      // tile maximum of r_t * s over the valid columns
+      float mx = -INFINITY;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(t0 + c * 32, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (c * 32 + j < nv) mx = fmaxf(mx, __uint_as_float(v[j]) * r[c * 32 + j]);
+      }
+      // exchange with the other half-warp of this quadrant (bounded wait: no named barrier that a
+      // partner leaving on a timeout could strand)
+      xmax[(acc * 2 + hf) * 128 + row] = mx;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&xbar[qd * 2 + acc]);
+      if (!mbar_wait(&xbar[qd * 2 + acc], ua & 1, abort_flag)) break;
+      const float mt = fmaxf(xmax[(acc * 2) * 128 + row], xmax[(acc * 2 + 1) * 128 + row]);
+      if (un.first) {
+        m_run = mt;
+        l_part = 0.f;
+      } else if (mt > m_run + kAbsLazy) {
+        l_part *= fast_exp2(m_run - mt);
+        m_run = mt;
+      }
+      // weights p = 2^(r s - m), written as pw = p * r (bf16) through the staging tile
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t v[32];
+        if (lane == 0) bulk_wait_read<0>();  // the previous store from this buffer has read it
+        __syncwarp();
+        uint4* dst = reinterpret_cast<uint4*>(sbuf + lane * 128);
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int c0 = cc * 64 + h2 * 32;
+          tmem_ld_32x32b_x32(t0 + c0, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j8 = 0; j8 < 4; ++j8) {
+            float w[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int col = c0 + 8 * j8 + j;
+              const float rr = r[col];
+              const float p = col < nv ? fast_exp2(fmaf(__uint_as_float(v[8 * j8 + j]), rr, -m_run)) : 0.f;
+              l_part += p;
+              w[j] = p * rr;
+            }
+            uint4 pk;
+            pk.x = pack_bf16x2(w[0], w[1]);
+            pk.y = pack_bf16x2(w[2], w[3]);
+            pk.z = pack_bf16x2(w[4], w[5]);
+            pk.w = pack_bf16x2(w[6], w[7]);
+            dst[(h2 * 4 + j8) ^ (lane & 7)] = pk;
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmP, sbuf, un.pcol0 + hf * 128 + cc * 64, (int)rank * 128 + qd * 32);
+          bulk_commit();
+        }
+      }
+      if (hf == 0) a.mref[(size_t)wk.u * kAbsQ + qg] = m_run;
+      if (un.last) {
+        xsum[hf * 128 + row] = l_part;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&lbar[qd]);
+        if (!mbar_wait(&lbar[qd], nseg & 1, abort_flag)) break;
+        ++nseg;
+        if (hf == 0) {
+          const float l = xsum[row] + xsum[128 + row];
+          float2* st = un.whole ? reinterpret_cast<float2*>(a.stats_whole) + (size_t)un.b * kAbsQ + qg
+                                : reinterpret_cast<float2*>(a.stats_part) + (size_t)un.slot * kAbsQ + qg;
+          *st = make_float2(m_run, l);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_cluster(tempty0 + acc * 8);  // the even CTA's MMA may reuse this accumulator
+        mbar_arrive(&edone[acc]);
+        mbar_arrive_cluster_release(edone_peer0 + acc * 8);
+      }
+    }
+    if (lane == 0) bulk_wait<0>();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_cg2(tmem_base, 512);
+  }
+}
+
+// ================================================================================================
+// pass B: z += pw H
+// ================================================================================================
+template <int E>  // d = 256 E
+struct AbsBSmem {
+  static constexpr uint32_t A_BYTES = 128 * 64 * 2;       // pw: this CTA's 128 queries x 64 rows
+  static constexpr uint32_t BOX_BYTES = 64 * 64 * 2;      // 64 rows x 64 columns of H
+  static constexpr uint32_t B_BYTES = E * 2 * BOX_BYTES;  // this CTA's 128 columns of each 256-column half
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int FIXED = 1024 + 512;
+  static constexpr int STAGES = (232448 - FIXED) / (int)STAGE_BYTES > 8 ? 8 : (232448 - FIXED) / (int)STAGE_BYTES;
+  static constexpr size_t BYTES = FIXED + STAGES * (size_t)STAGE_BYTES;
+};
+constexpr int kAbsBThreads = 320;
+
+// warps: 0 TMA producer (both CTAs), 1 TMEM (256 E columns: z of this CTA's 128 queries) + MMA issue
+// (even CTA), 2..9 correction and drain (two warps per lane quadrant, half of the columns each).
+// Per unit: the correction warps compare pass A's references of consecutive units; where one
+// was raised they wait for the previous unit's MMAs, scale their rows of z in TMEM and only then
+// release the unit to the MMA issuer (`cready`, 8 + 8 warps). They run at most two units ahead
+// (`udone` of unit - 2), so the two `cready` phases never alias.
+template <int E>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsBThreads, 1)
+    abs_values_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmH,
+                      const AbsArgs a) {
+  using L = AbsBSmem<E>;
+  constexpr int ST = L::STAGES;
+  constexpr uint32_t TMEM_COLS = 256 * E;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * L::STAGE_BYTES);
+  uint64_t* empty = full + ST;
+  uint64_t* udone = empty + ST;   // [2] MMAs of a unit complete (commit to both CTAs)
+  uint64_t* cready = udone + 2;   // [2] even CTA: unit released by 8 + 8 correction warps
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cready + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&udone[i], 1);
+      mbar_init(&cready[i], 16);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmP);
+    tma_prefetch_desc(&tmH);
+  }
+  if (warp == 1) {
+    tmem_alloc_cg2(tmem_slot, TMEM_COLS);
+    tmem_relinquish_cg2();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
+
+  AbsWalk wk;
+  wk.init(a, pair);
+
+  if (warp == 0) {
+    // ---------------- TMA producer (both CTAs): only the 64-row chunks holding valid rows ----------
+    if (lane == 0) {
+      int kg = 0;
+      bool stop = false;
+      for (; wk.valid() && !stop; wk.next(a)) {
+        const AbsUnit un = abs_unit(a, wk);
+        const int nch = (un.nvalid + 63) / 64;
+        for (int c = 0; c < nch; ++c, ++kg) {
+          const int s = kg % ST, u = kg / ST;
+          if (kg >= ST && !mbar_wait(&empty[s], (u - 1) & 1, abort_flag)) {
+            stop = true;
+            break;
+          }
+          uint8_t* st = smem + s * L::STAGE_BYTES;
+          const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
+          if (leader) mbar_arrive_expect_tx(&full[s], 2 * L::STAGE_BYTES);
+          tma_load_2d_cg2(st, &tmP, un.pcol0 + 64 * c, (int)rank * 128, bar);
+          const int hrow = (int)un.row0 + 64 * c;
+#pragma unroll
+          for (int e = 0; e < E; ++e)
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+              tma_load_2d_cg2(st + L::A_BYTES + (e * 2 + j) * L::BOX_BYTES, &tmH, e * 256 + (int)rank * 128 + j * 64,
+                              hrow, bar);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (even CTA) ----------------
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(256, 256) | kIdescBMnMajor;
+      int kg = 0, it = 0;
+      bool stop = false;
+      for (; wk.valid() && !stop; wk.next(a), ++it) {
+        const AbsUnit un = abs_unit(a, wk);
+        if (!mbar_wait_cluster(&cready[it & 1], (it >> 1) & 1, abort_flag)) break;
+        tc_fence_after();
+        const int nch = (un.nvalid + 63) / 64;
+        for (int c = 0; c < nch; ++c, ++kg) {
+          const int s = kg % ST, u = kg / ST;
+          if (!mbar_wait(&full[s], u & 1, abort_flag)) {
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + s * L::STAGE_BYTES);
+          const uint32_t b_base = a_base + L::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+              umma_f16_cg2(tmem_base + e * 256, sdesc_k_sw128(a_base + kk * 32),
+                           sdesc_mn_sw128(b_base + e * 2 * L::BOX_BYTES + kk * 2048, L::BOX_BYTES, 1024), idesc,
+                           (un.first && c == 0 && kk == 0) ? 0u : 1u);
+          umma_commit_cg2_mc(&empty[s], 0x3);
+        }
+        umma_commit_cg2_mc(&udone[it & 1], 0x3);
+      }
+    }
+  } else {
+    // ---------------- correction and drain (warps 2..9, both CTAs) ----------------
+    const int qd = warp & 3;
+    const int hf = (warp - 2) >> 2;
+    constexpr int NC = E * 128;  // z columns of this warp: [NC hf, NC hf + NC)
+    const int row = qd * 32 + lane;
+    const int qg = (int)rank * 128 + row;
+    const int head = qg / a.N, n = qg % a.N;
+    const uint32_t cready0 = mapa_shared(smem_u32(&cready[0]), 0);
+    const uint32_t t0 = tmem_base + hf * NC + ((uint32_t)(qd * 32) << 16);
+    int it = 0;
+    for (; wk.valid(); wk.next(a), ++it) {
+      const AbsUnit un = abs_unit(a, wk);
+      if (it >= 2 && !mbar_wait(&udone[it & 1], ((it - 2) >> 1) & 1, abort_flag)) break;
+      if (!un.first) {
+        const float mp = a.mref[(size_t)(wk.u - 1) * kAbsQ + qg];
+        const float mc = a.mref[(size_t)wk.u * kAbsQ + qg];
+        if (__any_sync(0xffffffffu, mc != mp)) {
+          if (!mbar_wait(&udone[(it - 1) & 1], ((it - 1) >> 1) & 1, abort_flag)) break;
+          tc_fence_after();
+          const float f = mc != mp ? fast_exp2(mp - mc) : 1.0f;
+#pragma unroll 1
+          for (int c = 0; c < NC / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(t0 + c * 32, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * f);
+            tmem_st_32x32b_x32(t0 + c * 32, v);
+          }
+          tmem_st_wait();
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader) mbar_arrive(&cready[it & 1]);
+        else mbar_arrive_cluster_release(cready0 + (it & 1) * 8);
+      }
+      if (un.last) {
+        if (!mbar_wait(&udone[it & 1], (it >> 1) & 1, abort_flag)) break;
+        tc_fence_after();
+        if (un.whole) {
+          const float inv = 1.0f / reinterpret_cast<const float2*>(a.stats_whole)[(size_t)un.b * kAbsQ + qg].y;
+          const size_t zrow = ((size_t)head * a.B + un.b) * a.N + n;
+#pragma unroll 1
+          for (int c = 0; c < NC / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(t0 + c * 32, v);
+            tmem_ld_wait();
+            uint32_t hi[16], lo[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float x0 = __uint_as_float(v[2 * j]) * inv, x1 = __uint_as_float(v[2 * j + 1]) * inv;
+              const __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
+              hi[j] = *reinterpret_cast<const uint32_t*>(&hb);
+              const float2 hf2 = __bfloat1622float2(hb);
+              lo[j] = pack_bf16x2(x0 - hf2.x, x1 - hf2.y);
+            }
+            uint4* dh = reinterpret_cast<uint4*>(a.z_hi + zrow * a.d + hf * NC + c * 32);
+            uint4* dl = reinterpret_cast<uint4*>(a.z_lo + zrow * a.d + hf * NC + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              dh[i] = make_uint4(hi[4 * i], hi[4 * i + 1], hi[4 * i + 2], hi[4 * i + 3]);
+              dl[i] = make_uint4(lo[4 * i], lo[4 * i + 1], lo[4 * i + 2], lo[4 * i + 3]);
+            }
+          }
+        } else {
+          float* dz = a.part_z + ((size_t)un.slot * kAbsQ + qg) * a.d + hf * NC;
+#pragma unroll 1
+          for (int c = 0; c < NC / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(t0 + c * 32, v);
+            tmem_ld_wait();
+            float4* d4 = reinterpret_cast<float4*>(dz + c * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              d4[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                  __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+          }
+        }
+        tc_fence_before();
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_cg2(tmem_base, TMEM_COLS);
+  }
+}
+
+// ================================================================================================
+// merge of examples split across pairs; zero z for empty histories
+// ================================================================================================
+// grid (B, 256 / 8), 256 threads: one warp per absorbed query.
+__global__ void __launch_bounds__(256) abs_merge_kernel(const AbsArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  const int b = blockIdx.x;
+  const int q = blockIdx.y * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (q >= kAbsQ) return;
+  const int U = a.ustart[a.B];
+  const int ub = a.ustart[b], ub1 = a.ustart[b + 1];
+  const int head = q / a.N, n = q % a.N;
+  const size_t zrow = ((size_t)head * a.B + b) * a.N + n;
+  uint2* zh = reinterpret_cast<uint2*>(a.z_hi + zrow * a.d);
+  uint2* zl = reinterpret_cast<uint2*>(a.z_lo + zrow * a.d);
+  if (ub >= ub1) {  // empty history: the attention output is the empty sum
+    for (int c = lane; c < a.d / 4; c += 32) {
+      zh[c] = make_uint2(0u, 0u);
+      zl[c] = make_uint2(0u, 0u);
+    }
+    return;
+  }
+  const int P = a.n_pairs;
+  const int p0 = abs_pair_of(ub, U, P), p1 = abs_pair_of(ub1 - 1, U, P);
+  if (p0 == p1) return;  // finished by pass B
+  auto slot_of = [&](int p) { return abs_range_start(U, P, p) >= ub ? 2 * p : 2 * p + 1; };
+  auto nonempty = [&](int p) { return abs_range_start(U, P, p) < abs_range_start(U, P, p + 1); };
+  const float2* st = reinterpret_cast<const float2*>(a.stats_part);
+  float M = -INFINITY;
+  for (int p = p0; p <= p1; ++p)
+    if (nonempty(p)) M = fmaxf(M, st[(size_t)slot_of(p) * kAbsQ + q].x);
+  float l = 0.f;
+  for (int p = p0; p <= p1; ++p)
+    if (nonempty(p)) {
+      const float2 ml = st[(size_t)slot_of(p) * kAbsQ + q];
+      l += fast_exp2(ml.x - M) * ml.y;
+    }
+  const float inv = 1.0f / l;
+  for (int c = lane; c < a.d / 4; c += 32) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int p = p0; p <= p1; ++p) {
+      if (!nonempty(p)) continue;
+      const int sl = slot_of(p);
+      const float w = fast_exp2(st[(size_t)sl * kAbsQ + q].x - M);
+      const float4 z = __ldcg(reinterpret_cast<const float4*>(a.part_z + ((size_t)sl * kAbsQ + q) * a.d) + c);
+      acc.x = fmaf(w, z.x, acc.x);
+      acc.y = fmaf(w, z.y, acc.y);
+      acc.z = fmaf(w, z.z, acc.z);
+      acc.w = fmaf(w, z.w, acc.w);
+    }
+    const float x[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
+    const __nv_bfloat162 h0 = __floats2bfloat162_rn(x[0], x[1]), h1 = __floats2bfloat162_rn(x[2], x[3]);
+    const float2 f0 = __bfloat1622float2(h0), f1 = __bfloat1622float2(h1);
+    zh[c] = make_uint2(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1));
+    zl[c] = make_uint2(pack_bf16x2(x[0] - f0.x, x[1] - f0.y), pack_bf16x2(x[2] - f1.x, x[3] - f1.y));
+  }
+}
+
+}  // namespace whale

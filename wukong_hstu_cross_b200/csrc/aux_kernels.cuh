@@ -10,14 +10,17 @@ namespace whale {
 // mode 1 (SwiGLU packing for the fused up|gate epilogue): rows in blocks of 32, block p holds
 //         W_up rows 16p..16p+15 then W_gate rows 16p..16p+15, where W = [W_up ; W_gate] and
 //         W_gate starts at row H.
+// mode 2 (absorbed keys): W = W_K [d, d], out has rows = h*d (row j*d + n) and cols = d_head (H
+//         holds d_head, `src_cols` holds d): out[j*d + n, k] = bf16(W[j*d_head + k, n] * g[n] * scale).
 struct FoldJob {
   const __nv_bfloat16* w;
   const float* g;
   __nv_bfloat16* out;
-  int rows, cols, mode, H;
+  int rows, cols, mode, H, src_cols;
+  float scale;
 };
 struct FoldJobs {
-  FoldJob job[3];
+  FoldJob job[4];
   int n;
 };
 
@@ -31,6 +34,19 @@ __global__ void fold_weights_kernel(const FoldJobs jobs) {
   const int total8 = j.rows * cols8;
   for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < total8; idx += gridDim.x * blockDim.x) {
     const int r = idx / cols8, c8 = idx - r * cols8;
+    if (j.mode == 2) {
+      const int dsrc = j.src_cols, head = r / dsrc, n = r - head * dsrc;
+      const float gn = (j.g ? j.g[n] : 1.f) * j.scale;
+      uint4 ov;
+      uint32_t* op = reinterpret_cast<uint32_t*>(&ov);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const size_t k0 = (size_t)head * j.H + c8 * 8 + 2 * i;
+        op[i] = pack_bf16x2(__bfloat162float(j.w[k0 * dsrc + n]) * gn, __bfloat162float(j.w[(k0 + 1) * dsrc + n]) * gn);
+      }
+      *reinterpret_cast<uint4*>(j.out + (size_t)idx * 8) = ov;
+      continue;
+    }
     int src = r;
     if (j.mode == 1) {
       const int p = r >> 5, w = r & 31;

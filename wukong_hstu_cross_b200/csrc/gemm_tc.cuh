@@ -24,15 +24,16 @@
 //               diag(g) folded into W beforehand.
 // Epilogue value per element (fp32): STORE r*acc; SILU silu(acc); RESID acc + resid32;
 // SWIGLU (W rows packed in blocks of 32 = 16 up rows then the 16 matching gate rows)
-// silu(r*gate) * r*up; SWIGLU_TIED (W_gate = W_up) silu(r*u) * r*u. It is then written to
-// any of: out32 (fp32), out_hi (bf16 rounding), out_lo (bf16 of the rounding residue).
+// silu(r*gate) * r*up; SWIGLU_TIED (W_gate = W_up) silu(r*u) * r*u; QABS acc, written to a
+// per-head row order (see GemmArgs). It is then written to any of: out32 (fp32), out_hi (bf16
+// rounding), out_lo (bf16 of the rounding residue).
 #pragma once
 
 #include "ptx.cuh"
 
 namespace whale {
 
-enum GemmEpi : int { EPI_STORE = 0, EPI_SILU = 1, EPI_RESID = 2, EPI_SWIGLU = 3, EPI_SWIGLU_TIED = 4 };
+enum GemmEpi : int { EPI_STORE = 0, EPI_SILU = 1, EPI_RESID = 2, EPI_SWIGLU = 3, EPI_SWIGLU_TIED = 4, EPI_QABS = 5 };
 
 struct GemmArgs {
   int M;                       // rows of A and of the output
@@ -49,6 +50,15 @@ struct GemmArgs {
   long long ldo;               // output row stride (elements), shared by the three outputs
   const float* resid32;        // EPI_RESID: fp32 residual [M, N]
   long long ldr;
+  // Per-head GEMMs in one launch (head_tiles > 0): output columns come in head blocks of
+  // head_tiles n-tiles; the tiles of head j read A from K block j * a_kb_step (block-diagonal W)
+  // and from row j * a_row_step (a stack of per-head A matrices).
+  int head_tiles;
+  int a_kb_step;
+  long long a_row_step;
+  // EPI_QABS: the accumulator row m = b * qabs_N + n of head block j (qabs_d columns) is written to
+  // row b * qabs_rows + j * qabs_N + n, columns relative to the head block.
+  int qabs_N, qabs_d, qabs_rows;
 };
 
 
@@ -184,9 +194,14 @@ __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
           uint8_t* st = smem + s * L::STAGE_BYTES;
           mbar_arrive_expect_tx(&full[s], L::STAGE_BYTES);
           const bool first = kb < args.kb0;
-          const int kc = (first ? kb : kb - args.kb0) * L::BK;
-          tma_load_2d(st, first ? &tmA0 : &tmA1, kc, m0, &full[s]);
-          if (SPLIT) tma_load_2d(st + L::A_BYTES, first ? &tmA0lo : &tmA1lo, kc, m0, &full[s]);
+          int kc = (first ? kb : kb - args.kb0) * L::BK, ma = m0;
+          if (args.head_tiles > 0) {
+            const int head = (tile % args.tiles_n) / args.head_tiles;
+            kc += head * args.a_kb_step * L::BK;
+            ma += (int)(head * args.a_row_step);
+          }
+          tma_load_2d(st, first ? &tmA0 : &tmA1, kc, ma, &full[s]);
+          if (SPLIT) tma_load_2d(st + L::A_BYTES, first ? &tmA0lo : &tmA1lo, kc, ma, &full[s]);
           tma_load_2d(st + L::A_ALL, &tmB, kb * L::BK, n0, &full[s]);
         }
       }
@@ -321,7 +336,14 @@ __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) x[j] = silu_f(x[j]) * x[j];
           }
-          store_row_chunk<32>(args, gm * args.ldo + col, x);
+          if (EPI == EPI_QABS) {
+            const int head = col / args.qabs_d;
+            const long long orow =
+                (gm / args.qabs_N) * args.qabs_rows + (long long)head * args.qabs_N + gm % args.qabs_N;
+            store_row_chunk<32>(args, orow * args.ldo + (col - head * args.qabs_d), x);
+          } else {
+            store_row_chunk<32>(args, gm * args.ldo + col, x);
+          }
         }
       }
       // this accumulator buffer and its row factors may be reused

@@ -25,6 +25,7 @@
 #include <utility>
 #include <mutex>
 
+#include "absorbed.cuh"
 #include "aux_kernels.cuh"
 #include "attention.cuh"
 #include "fp32_path.cuh"
@@ -128,17 +129,25 @@ struct Shape {
   bool bf16;
   int layers, d, h, dh, N, H, Fh;
   bool shared_kv, tied, debug, prepared;
+  bool absorbed;  // bf16 attention with K and V folded into the queries (absorbed.cuh)
   float eps;
   int kvw;  // kv row width: 2d, or d with shared K = V
   int ugw;  // rows of the up|gate matrix: 2H, or H with a tied gate
   size_t es;  // element size
 };
 
+// Shapes the absorbed attention handles: 256 absorbed queries per example (two CTAs of 128), one
+// 64-column K block per head for the query-side GEMM, d a multiple of the 256-column MMA.
+bool absorbed_shape(const Shape& s) {
+  return s.bf16 && (long long)s.N * s.h == kAbsQ && s.dh == 64 && (s.d == 256 || s.d == 512);
+}
+
 whale_status validate(const whale_config* c, Shape* s) {
   if (!c || !s) return WHALE_ERR_INVALID_ARG;
   if (c->n_layers < 1 || c->d < 1 || c->n_heads < 1 || c->n_tokens < 1 || c->ffn_hidden < 1 ||
       c->fusion_hidden < 0 || !(c->eps >= 0.f) || (c->dtype != WHALE_FP32 && c->dtype != WHALE_BF16) ||
-      (c->flags & ~(WHALE_SHARED_KV | WHALE_TIED_GATE | WHALE_DEBUG | WHALE_PREPARED_WEIGHTS)) || c->d % c->n_heads)
+      (c->flags & ~(WHALE_SHARED_KV | WHALE_TIED_GATE | WHALE_DEBUG | WHALE_PREPARED_WEIGHTS | WHALE_MATERIALIZED_KV)) ||
+      c->d % c->n_heads)
     return WHALE_ERR_INVALID_ARG;
   s->bf16 = c->dtype == WHALE_BF16;
   s->layers = c->n_layers;
@@ -156,6 +165,7 @@ whale_status validate(const whale_config* c, Shape* s) {
   s->kvw = s->shared_kv ? s->d : 2 * s->d;
   s->ugw = s->tied ? s->H : 2 * s->H;
   s->es = s->bf16 ? 2 : 4;
+  s->absorbed = absorbed_shape(*s) && !(c->flags & WHALE_MATERIALIZED_KV);
   if (s->bf16) {
     const int hg = s->h < 8 ? s->h : 8;
     if (s->d % 64 || (s->dh != 32 && s->dh != 64) || s->h % hg || (hg * s->dh) % 64 || (hg != 2 && hg != 4 && hg != 8) ||
@@ -216,8 +226,17 @@ struct Layout {
   size_t q, kv, a, g, f, u, ug, x0, x1;   // fp32 path, and q / kv of the bf16 path
   // bf16 path: lo halves of the token-side operand pairs and the fp32 residual stream
   size_t a_lo, g_lo, f_lo, u_lo, f32, x32[2], xhi[2], xlo[2];
+  // absorbed attention: folded key weights, absorbed queries, weights pw, unit references,
+  // segment statistics, partial z, unit starts, z as a bf16 pair
+  size_t wkabs, qa, pw, mref, stw, stp, pz, ust, zh, zl;
+  long long units_max, pw_cols;
   size_t total;
 };
+
+constexpr int kMaxPairs = kNumSM / 2;
+
+// Units of 256 history rows: sum_b ceil(L_b / 256) <= ceil(total_L / 256) + B.
+long long abs_units_max(const whale_shape_hint& h) { return cdiv<long long>(h.total_L, kAbsRows) + h.B; }
 
 Layout make_layout(const Shape& s, const whale_shape_hint& hint) {
   Layout L{};
@@ -233,14 +252,28 @@ Layout make_layout(const Shape& s, const whale_shape_hint& hint) {
     L.wq = take((size_t)s.d * s.d * 2);
     L.wkv = take((size_t)s.kvw * s.d * 2);
     L.wug = take((size_t)s.ugw * s.d * 2);
-    AttnPlan p = plan_attention(s, hint.B, hint.total_L);
+    AttnPlan p = plan_attention(s, hint.B, hint.total_L);  // also the step entry points' scratch
     L.po = take(p.bytes());
     L.pml = 0;
   } else {
     L.r = take((rows > tl ? rows : tl) * 4);
   }
   L.q = take(rows * s.d * s.es);
-  L.kv = take(tl * s.kvw * s.es);
+  L.kv = s.absorbed ? 0 : take(tl * s.kvw * s.es);
+  if (s.absorbed) {
+    L.units_max = abs_units_max(hint);
+    L.pw_cols = L.units_max * kAbsRows;
+    L.wkabs = take((size_t)s.h * s.d * s.dh * 2);
+    L.qa = take((size_t)hint.B * kAbsQ * s.d * 2);
+    L.pw = take((size_t)kAbsQ * L.pw_cols * 2);
+    L.mref = take((size_t)L.units_max * kAbsQ * 4);
+    L.stw = take((size_t)hint.B * kAbsQ * 8);
+    L.stp = take((size_t)2 * kMaxPairs * kAbsQ * 8);
+    L.pz = take((size_t)2 * kMaxPairs * kAbsQ * s.d * 4);
+    L.ust = take(((size_t)hint.B + 1) * 4);
+    L.zh = take((size_t)hint.B * kAbsQ * s.d * 2);
+    L.zl = take((size_t)hint.B * kAbsQ * s.d * 2);
+  }
   L.a = take(rows * s.d * s.es);
   L.g = take(rows * (size_t)s.Fh * s.es);
   L.f = take(rows * s.d * s.es);
@@ -466,26 +499,36 @@ whale_status pair_from_bf16(const void* x, float* x32, void* lo, long long n, cu
 // ------------------------------------------------------------------------------------------
 // bf16 steps
 // ------------------------------------------------------------------------------------------
+// Log2(e) / sqrt(d_head): the attention scale in base-2 units.
+inline float scale_log2_of(const Shape& s) { return (float)(1.4426950408889634 / std::sqrt((double)s.dh)); }
+
+// Fold the gains into the weights (one launch for all jobs). `okabs` (optional) receives the
+// absorbed key weights from W_K = the first d rows of `wkv_kabs` with gain `gkv_kabs`.
 whale_status fold_weights(const Shape& s, const __nv_bfloat16* wq, const float* gq, const __nv_bfloat16* wkv,
                           const float* gkv, const __nv_bfloat16* wug, const float* gffn, __nv_bfloat16* oq,
-                          __nv_bfloat16* okv, __nv_bfloat16* oug, cudaStream_t st) {
+                          __nv_bfloat16* okv, __nv_bfloat16* oug, cudaStream_t st,
+                          const __nv_bfloat16* wkv_kabs = nullptr, const float* gkv_kabs = nullptr,
+                          __nv_bfloat16* okabs = nullptr) {
   FoldJobs jobs{};
   long long maxe = 0;
-  auto add = [&](const __nv_bfloat16* w, const float* g, __nv_bfloat16* out, int rows, int mode) {
+  auto add = [&](const __nv_bfloat16* w, const float* g, __nv_bfloat16* out, int rows, int cols, int mode) {
     if (!w || !out) return;
     FoldJob& j = jobs.job[jobs.n++];
     j.w = w;
     j.g = g;
     j.out = out;
     j.rows = rows;
-    j.cols = s.d;
+    j.cols = cols;
     j.mode = mode;
-    j.H = s.H;
-    maxe = std::max(maxe, (long long)rows * s.d);
+    j.H = mode == 2 ? s.dh : s.H;
+    j.src_cols = s.d;
+    j.scale = mode == 2 ? scale_log2_of(s) : 1.f;
+    maxe = std::max(maxe, (long long)rows * cols);
   };
-  add(wq, gq, oq, s.d, 0);
-  add(wkv, gkv, okv, s.kvw, 0);
-  add(wug, gffn, oug, s.ugw, s.tied ? 0 : 1);
+  add(wq, gq, oq, s.d, s.d, 0);
+  add(wkv, gkv, okv, s.kvw, s.d, 0);
+  add(wug, gffn, oug, s.ugw, s.d, s.tied ? 0 : 1);
+  add(wkv_kabs, gkv_kabs, okabs, s.h * s.d, s.dh, 2);
   if (jobs.n == 0) return WHALE_OK;
   const unsigned gx = (unsigned)std::min<long long>(cdiv<long long>(maxe / 8, 256), 8 * kNumSM);
   return launch_pdl(fold_weights_kernel, dim3(gx, jobs.n), dim3(256), 0, st, jobs);
@@ -559,6 +602,163 @@ whale_status attention_bf16(const Shape& s, const void* q, const void* kv, const
 }
 
 // ------------------------------------------------------------------------------------------
+// absorbed attention (bf16; absorbed.cuh)
+// ------------------------------------------------------------------------------------------
+// Co-resident clusters of both passes (cached per device): their shared memory allows one CTA per SM.
+whale_status abs_max_pairs(int E, int* pairs) {
+  static std::mutex mu;
+  static int cache[64][2];
+  int dev = 0;
+  CUCHECK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return WHALE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(mu);
+  int& c = cache[dev][E - 1];
+  if (c == 0) {
+    auto query = [&](const void* kern, size_t smem, int threads, int* n) -> whale_status {
+      CUCHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+      cudaLaunchConfig_t lc = {};
+      lc.gridDim = dim3(kNumSM, 1, 1);
+      lc.blockDim = dim3(threads, 1, 1);
+      lc.dynamicSmemBytes = smem;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      lc.attrs = attr;
+      lc.numAttrs = 1;
+      CUCHECK(cudaOccupancyMaxActiveClusters(n, kern, &lc));
+      return WHALE_OK;
+    };
+    int na = 0, nb = 0;
+    WCHECK(query(reinterpret_cast<const void*>(abs_scores_kernel), AbsASmem::BYTES, kAbsAThreads, &na));
+    if (E == 1) WCHECK(query(reinterpret_cast<const void*>(abs_values_kernel<1>), AbsBSmem<1>::BYTES, kAbsBThreads, &nb));
+    else WCHECK(query(reinterpret_cast<const void*>(abs_values_kernel<2>), AbsBSmem<2>::BYTES, kAbsBThreads, &nb));
+    const int n = std::min(std::min(na, nb), kMaxPairs);
+    c = n > 0 ? n : -1;
+  }
+  *pairs = c;
+  return c > 0 ? WHALE_OK : WHALE_ERR_UNSUPPORTED;
+}
+
+// qa[b*256 + j*N + n, :] = q[b*N + n, j*64 : j*64 + 64] W~_j^T with W~ [h*d, 64] (one K block per
+// head: a block-diagonal GEMM over the h*d output columns, rows scattered per head).
+whale_status gemm_qabs(const Shape& s, const void* q, const void* wkabs, void* qa, long long rows, cudaStream_t st) {
+  constexpr int BN = 256;
+  if (s.d % BN || s.dh != 64) return WHALE_ERR_UNSUPPORTED;
+  CUtensorMap maps[5];
+  WCHECK(tmap_bf16(&maps[0], q, rows, s.d, s.d, 128));
+  maps[1] = maps[2] = maps[3] = maps[0];
+  WCHECK(tmap_bf16(&maps[4], wkabs, (long long)s.h * s.d, s.dh, s.dh, BN));
+  GemmArgs g{};
+  g.M = (int)rows;
+  g.N = s.h * s.d;
+  g.kb0 = s.dh / 64;
+  g.kb1 = 0;
+  g.tiles_n = g.N / BN;
+  const long long tiles = cdiv<long long>(rows, 128) * g.tiles_n;
+  g.num_tiles = (int)tiles;
+  g.out_hi = static_cast<__nv_bfloat16*>(qa);
+  g.ldo = s.d;
+  g.head_tiles = s.d / BN;
+  g.a_kb_step = s.dh / 64;
+  g.a_row_step = 0;
+  g.qabs_N = s.N;
+  g.qabs_d = s.d;
+  g.qabs_rows = kAbsQ;
+  return launch_gemm_t<BN, EPI_QABS, false, false>(maps, g, tiles, st);
+}
+
+// A[:, j*64 : j*64 + 64] = z_j W'_V,j^T for every head j in one launch: z is the stack
+// [h, rows, d] (bf16 pair), W'_V the gain-folded [d, d] value weights (row j*64 + c).
+whale_status gemm_vabs(const Shape& s, const void* zh, const void* zl, const void* wv, void* a, void* a_lo,
+                       long long rows, cudaStream_t st) {
+  if (s.dh != 64) return WHALE_ERR_UNSUPPORTED;
+  CUtensorMap maps[5];
+  WCHECK(tmap_bf16(&maps[0], zh, (long long)s.h * rows, s.d, s.d, 128));
+  WCHECK(tmap_bf16(&maps[1], zl, (long long)s.h * rows, s.d, s.d, 128));
+  maps[2] = maps[0];
+  maps[3] = maps[1];
+  WCHECK(tmap_bf16(&maps[4], wv, s.d, s.d, s.d, 64));
+  GemmArgs g{};
+  g.M = (int)rows;
+  g.N = s.d;
+  g.kb0 = s.d / 64;
+  g.kb1 = 0;
+  g.tiles_n = s.d / 64;
+  const long long tiles = cdiv<long long>(rows, 128) * g.tiles_n;
+  g.num_tiles = (int)tiles;
+  g.out_hi = static_cast<__nv_bfloat16*>(a);
+  g.out_lo = static_cast<__nv_bfloat16*>(a_lo);
+  g.ldo = s.d;
+  g.head_tiles = 1;
+  g.a_kb_step = 0;
+  g.a_row_step = rows;
+  return launch_gemm_t<64, EPI_STORE, false, true>(maps, g, tiles, st);
+}
+
+// Unit starts of the batch (once per forward: the offsets are shared by every layer).
+whale_status abs_units(const Shape& s, const int* offsets, const whale_shape_hint& hint, void* ws, const Layout& L,
+                       cudaStream_t st) {
+  if (!s.absorbed || hint.B == 0) return WHALE_OK;
+  if (L.units_max >= (1ll << 31) / kAbsRows) return WHALE_ERR_UNSUPPORTED;
+  return launch_pdl(abs_units_kernel, dim3(1), dim3(1024), 0, st, offsets, hint.B, (long long)hint.total_L,
+                    (int)L.units_max, reinterpret_cast<int*>(at(ws, L.ust)));
+}
+
+// S3 through the absorbed path: q (bf16 [B*N, d]) -> A (bf16 pair [B*N, d]).
+whale_status attention_absorbed(const Shape& s, const void* q, const void* slab, const int* offsets,
+                                const void* wkabs, const void* wv, void* out, void* out_lo, const whale_shape_hint& hint,
+                                void* ws, const Layout& L, cudaStream_t st) {
+  if (hint.B == 0) return WHALE_OK;
+  const long long rows = (long long)hint.B * s.N;
+  const int E = s.d / 256;
+  WCHECK(gemm_qabs(s, q, wkabs, at(ws, L.qa), rows, st));
+  AbsArgs a{};
+  a.offsets = offsets;
+  a.ustart = reinterpret_cast<const int*>(at(ws, L.ust));
+  a.B = hint.B;
+  a.N = s.N;
+  a.d = s.d;
+  a.total_L = hint.total_L;
+  a.inv_d = 1.0f / (float)s.d;
+  a.eps = s.eps;
+  a.mref = reinterpret_cast<float*>(at(ws, L.mref));
+  a.stats_whole = reinterpret_cast<float*>(at(ws, L.stw));
+  a.stats_part = reinterpret_cast<float*>(at(ws, L.stp));
+  a.part_z = reinterpret_cast<float*>(at(ws, L.pz));
+  a.z_hi = reinterpret_cast<__nv_bfloat16*>(at(ws, L.zh));
+  a.z_lo = reinterpret_cast<__nv_bfloat16*>(at(ws, L.zl));
+  int pairs = 0;
+  WCHECK(abs_max_pairs(E, &pairs));
+  a.n_pairs = (int)std::max<long long>(1, std::min<long long>(pairs, L.units_max));
+  if (hint.total_L > 0) {
+    CUtensorMap tq, th, tps;
+    WCHECK(tmap_bf16(&tq, at(ws, L.qa), (long long)hint.B * kAbsQ, s.d, s.d, 128));
+    WCHECK(tmap_bf16(&th, slab, hint.total_L, s.d, s.d, 128));
+    WCHECK(tmap_bf16(&tps, at(ws, L.pw), kAbsQ, L.pw_cols, L.pw_cols, 32));
+    CUCHECK(cudaFuncSetAttribute(abs_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AbsASmem::BYTES));
+    WCHECK(launch_pdl(abs_scores_kernel, dim3(2 * a.n_pairs), dim3(kAbsAThreads), AbsASmem::BYTES, st, tq, th, tps, a));
+    CUtensorMap tpl, th64;
+    WCHECK(tmap_bf16(&tpl, at(ws, L.pw), kAbsQ, L.pw_cols, L.pw_cols, 128));
+    WCHECK(tmap_bf16(&th64, slab, hint.total_L, s.d, s.d, 64));
+    if (E == 1) {
+      CUCHECK(cudaFuncSetAttribute(abs_values_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)AbsBSmem<1>::BYTES));
+      WCHECK(launch_pdl(abs_values_kernel<1>, dim3(2 * a.n_pairs), dim3(kAbsBThreads), AbsBSmem<1>::BYTES, st, tpl,
+                        th64, a));
+    } else {
+      CUCHECK(cudaFuncSetAttribute(abs_values_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)AbsBSmem<2>::BYTES));
+      WCHECK(launch_pdl(abs_values_kernel<2>, dim3(2 * a.n_pairs), dim3(kAbsBThreads), AbsBSmem<2>::BYTES, st, tpl,
+                        th64, a));
+    }
+  }
+  WCHECK(launch_pdl(abs_merge_kernel, dim3(hint.B, kAbsQ / 8), dim3(256), 0, st, a));
+  return gemm_vabs(s, at(ws, L.zh), at(ws, L.zl), wv, out, out_lo, rows, st);
+}
+
+// ------------------------------------------------------------------------------------------
 // fp32 steps
 // ------------------------------------------------------------------------------------------
 whale_status row_rms(const float* x, long long rows, int d, float eps, float* r, cudaStream_t st) {
@@ -626,7 +826,7 @@ bool weights_ok(const Shape& s, const whale_layer_weights* w) {
   const bool gains = s.prepared || (w && w->g_q && w->g_kv && w->g_ffn);
   return w && gains && w->w_q && w->w_kv && w->w_f2 && w->w_upgate && w->w_down &&
          (s.Fh == 0 || w->w_f1) && al(w->g_q) && al(w->g_kv) && al(w->g_ffn) && al(w->w_q) && al(w->w_kv) &&
-         al(w->w_f1) && al(w->w_f2) && al(w->w_upgate) && al(w->w_down);
+         al(w->w_f1) && al(w->w_f2) && al(w->w_upgate) && al(w->w_down) && al(w->w_kabs);
 }
 
 // A token-side tensor of the bf16 path: fp32 value plus its bf16 hi/lo pair (any may be null
@@ -666,24 +866,39 @@ whale_status layer_bf16(const Shape& s, const Stream3& in, const void* slab, con
   const void* wq = w.w_q;
   const void* wkv = w.w_kv;
   const void* wug = w.w_upgate;
+  const void* wkabs = s.absorbed ? w.w_kabs : nullptr;
+  auto* wkabs_ws = reinterpret_cast<__nv_bfloat16*>(s.absorbed ? at(ws, L.wkabs) : nullptr);
   if (!s.prepared) {
     wq = at(ws, L.wq);
     wkv = at(ws, L.wkv);
     wug = at(ws, L.wug);
+    wkabs = wkabs_ws;
     WCHECK(fold_weights(s, static_cast<const __nv_bfloat16*>(w.w_q), w.g_q, static_cast<const __nv_bfloat16*>(w.w_kv),
                         w.g_kv, static_cast<const __nv_bfloat16*>(w.w_upgate), w.g_ffn,
                         reinterpret_cast<__nv_bfloat16*>(at(ws, L.wq)), reinterpret_cast<__nv_bfloat16*>(at(ws, L.wkv)),
-                        reinterpret_cast<__nv_bfloat16*>(at(ws, L.wug)), st));
+                        reinterpret_cast<__nv_bfloat16*>(at(ws, L.wug)), st,
+                        s.absorbed ? static_cast<const __nv_bfloat16*>(w.w_kv) : nullptr, w.g_kv, wkabs_ws));
+  } else if (s.absorbed && !wkabs) {  // prepared weights without the absorbed keys: form them from W_K'
+    wkabs = wkabs_ws;
+    WCHECK(fold_weights(s, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, st,
+                        static_cast<const __nv_bfloat16*>(w.w_kv), nullptr, wkabs_ws));
   }
   const Opnd X = opnd(in.hi, in.lo, s.d, s.d);
-  // S1 queries, S2 keys|values
+  // S1 queries
   WCHECK(gemm_bf16(X, no_opnd(), wq, s.d, Outs{at(ws, L.q), nullptr, nullptr, s.d}, nullptr, 0, rows, EPI_STORE, true,
                    s.eps, st));
-  WCHECK(gemm_bf16(opnd(slab, nullptr, s.d, s.d), no_opnd(), wkv, s.kvw, Outs{at(ws, L.kv), nullptr, nullptr, s.kvw},
-                   nullptr, 0, hint.total_L, EPI_STORE, true, s.eps, st));
-  // S3 attention -> A as a hi/lo pair
-  WCHECK(attention_bf16(s, at(ws, L.q), at(ws, L.kv), offsets, at(ws, L.a), at(ws, L.a_lo), hint.B, hint.total_L,
-                        at(ws, L.po), st));
+  if (s.absorbed) {
+    // S2 + S3 with K and V folded into the queries -> A as a hi/lo pair
+    const void* wv = s.shared_kv ? wkv : static_cast<const char*>(wkv) + (size_t)s.d * s.d * 2;
+    WCHECK(attention_absorbed(s, at(ws, L.q), slab, offsets, wkabs, wv, at(ws, L.a), at(ws, L.a_lo), hint, ws, L,
+                              st));
+  } else {
+    // S2 keys|values, S3 attention -> A as a hi/lo pair
+    WCHECK(gemm_bf16(opnd(slab, nullptr, s.d, s.d), no_opnd(), wkv, s.kvw,
+                     Outs{at(ws, L.kv), nullptr, nullptr, s.kvw}, nullptr, 0, hint.total_L, EPI_STORE, true, s.eps, st));
+    WCHECK(attention_bf16(s, at(ws, L.q), at(ws, L.kv), offsets, at(ws, L.a), at(ws, L.a_lo), hint.B, hint.total_L,
+                          at(ws, L.po), st));
+  }
   // S4 Fusion MLP -> F (fp32 + pair)
   auto* f32 = reinterpret_cast<float*>(at(ws, L.f32));
   WCHECK(fusion_bf16(s, rows, opnd(at(ws, L.a), at(ws, L.a_lo), s.d, s.d), X, in.f32, w.w_f1, w.w_f2, at(ws, L.g),
@@ -745,6 +960,7 @@ whale_status stack_impl(const Shape& s, const void* tokens, const void* seq_stat
   Stream3 in = buf(0);
   in.hi = const_cast<void*>(tokens);  // bf16 tokens are their own hi half; lo = 0
   WCHECK(pair_from_bf16(tokens, in.f32, in.lo, rows * s.d, st));
+  WCHECK(abs_units(s, offsets, hint, ws, L, st));
   for (int l = 0; l < n_layers; ++l) {
     const Stream3 y = (l == n_layers - 1) ? Stream3{nullptr, out, nullptr} : buf((l + 1) & 1);
     if (hook) WCHECK(hook(l, true));
@@ -837,8 +1053,9 @@ const char* whale_status_string(whale_status s) {
 size_t whale_prepared_weights_size(const whale_config* cfg) {
   Shape s;
   if (validate(cfg, &s) != WHALE_OK || !s.bf16) return 0;
-  return (size_t)s.layers *
-         (align_up((size_t)s.d * s.d * 2) + align_up((size_t)s.kvw * s.d * 2) + align_up((size_t)s.ugw * s.d * 2));
+  const size_t kabs = absorbed_shape(s) ? align_up((size_t)s.h * s.d * s.dh * 2) : 0;
+  return (size_t)s.layers * (align_up((size_t)s.d * s.d * 2) + align_up((size_t)s.kvw * s.d * 2) +
+                             align_up((size_t)s.ugw * s.d * 2) + kabs);
 }
 
 whale_status whale_prepare_weights(const whale_config* cfg, const whale_layer_weights* weights, void* prepared,
@@ -863,12 +1080,19 @@ whale_status whale_prepare_weights(const whale_config* cfg, const whale_layer_we
     o += align_up((size_t)s.kvw * s.d * 2);
     auto* oug = reinterpret_cast<__nv_bfloat16*>(at(prepared, o));
     o += align_up((size_t)s.ugw * s.d * 2);
+    __nv_bfloat16* okabs = nullptr;
+    if (absorbed_shape(s)) {
+      okabs = reinterpret_cast<__nv_bfloat16*>(at(prepared, o));
+      o += align_up((size_t)s.h * s.d * s.dh * 2);
+    }
     WCHECK(fold_weights(s, static_cast<const __nv_bfloat16*>(w.w_q), w.g_q, static_cast<const __nv_bfloat16*>(w.w_kv),
-                        w.g_kv, static_cast<const __nv_bfloat16*>(w.w_upgate), w.g_ffn, oq, okv, oug, st));
+                        w.g_kv, static_cast<const __nv_bfloat16*>(w.w_upgate), w.g_ffn, oq, okv, oug, st,
+                        okabs ? static_cast<const __nv_bfloat16*>(w.w_kv) : nullptr, w.g_kv, okabs));
     out_weights[l] = w;
     out_weights[l].w_q = oq;
     out_weights[l].w_kv = okv;
     out_weights[l].w_upgate = oug;
+    out_weights[l].w_kabs = okabs;
   }
   return WHALE_OK;
 }

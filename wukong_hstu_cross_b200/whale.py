@@ -17,6 +17,7 @@ HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))
 
 WHALE_FP32, WHALE_BF16 = 0, 1
 WHALE_SHARED_KV, WHALE_TIED_GATE, WHALE_DEBUG, WHALE_PREPARED_WEIGHTS = 1, 2, 4, 8
+WHALE_MATERIALIZED_KV = 16
 WHALE_DEVERR_TIMEOUT, WHALE_DEVERR_OFFSETS = 1, 2
 WHALE_NOALLOC_SCRATCH_BYTES = 32 << 20
 STATUS = {0: "WHALE_OK", 1: "WHALE_ERR_INVALID_ARG", 2: "WHALE_ERR_UNSUPPORTED", 3: "WHALE_ERR_CUDA",
@@ -29,7 +30,7 @@ class whale_config(ctypes.Structure):
                 ("eps", c_float)]
 
 
-_WNAMES = ("g_q", "g_kv", "w_q", "w_kv", "w_f1", "w_f2", "g_ffn", "w_upgate", "w_down")
+_WNAMES = ("g_q", "g_kv", "w_q", "w_kv", "w_f1", "w_f2", "g_ffn", "w_upgate", "w_down", "w_kabs")
 
 
 class whale_layer_weights(ctypes.Structure):
