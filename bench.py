@@ -37,6 +37,10 @@ METRIC = "WHALE fusion-layer examples/s @15k jagged history; % of HBM/TC rooflin
 KV_TRAFFIC_BYTES_PER_ROW_D512 = {"2sm": (113.378816e6 + 169.603840e6) / 109605,
                                  "1sm": (113.375488e6 + 168.328960e6) / 109605}
 
+# DRAM bytes per history row of one whale_attend_states call (pass A + pass B + the small kernels),
+# from the committed summary profiles/absorbed_attention_hist15k.md; None until captured.
+ABS_TRAFFIC_BYTES_PER_ROW_D512 = None
+
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
 
 
@@ -52,28 +56,45 @@ def load_peaks():
 # ------------------------------------------------------------------------------------------------
 # algorithmic work per step (bf16 storage)
 # ------------------------------------------------------------------------------------------------
-def step_work(w: I.Workload, total_L: int, shared_kv: bool = False, tied_gate: bool = False) -> dict:
+def step_work(w: I.Workload, total_L: int, shared_kv: bool = False, tied_gate: bool = False,
+              absorbed: bool = False) -> dict:
     """FLOPs and bytes per kernel family for one layer (no re-reads, no partials; the hi/lo
-    operand halves of the token-side GEMMs are not counted: algorithmic work only)."""
+    operand halves of the token-side GEMMs are not counted: algorithmic work only).
+
+    absorbed: S2 + S3 with K and V folded into the queries (one family): the scores of the N*h
+    absorbed queries against every history row and the weighted row sums, 2 x (2 N h L d), plus the
+    per-head query and output GEMMs (2 rows d d_head h = 2 rows d^2 each); its algorithmic bytes
+    are the states read once plus q, A and the two weight matrices."""
     B, N, d, H, Fh = w.batch, w.n_tokens, w.d, w.ffn_hidden, w.fusion_hidden
     rows = B * N
     e = 2
     kvw = d if shared_kv else 2 * d
     ugw = H if tied_gate else 2 * H
+    if absorbed:
+        nq = N * w.n_heads
+        history = {"attention_absorbed": {"flops": 4.0 * nq * total_L * d + 4.0 * rows * d * d,
+                                          "bytes": e * (total_L * d + 2 * rows * d + 2 * d * d)}}
+    else:
+        history = {
+            "kv_proj": {"flops": 2.0 * total_L * d * kvw, "bytes": e * (total_L * d + total_L * kvw + kvw * d)},
+            "attention": {"flops": 4.0 * N * total_L * d,   # q k^T and p v: 2 x (2 N L d) per example
+                          "bytes": e * (total_L * kvw + 2 * rows * d)},
+        }
     return {
-        "kv_proj": {"flops": 2.0 * total_L * d * kvw, "bytes": e * (total_L * d + total_L * kvw + kvw * d)},
-        "attention": {"flops": 4.0 * N * total_L * d,   # q k^T and p v: 2 x (2 N L d) per example
-                      "bytes": e * (total_L * kvw + 2 * rows * d)},
+        **history,
         "q_proj": {"flops": 2.0 * rows * d * d, "bytes": e * (2 * rows * d + d * d)},
         "fusion_mlp": {"flops": 2.0 * rows * (2 * d * Fh + Fh * d), "bytes": e * (3 * rows * d + 2 * rows * Fh + 3 * d * Fh)},
         "swiglu_ffn": {"flops": 2.0 * rows * (d * ugw + H * d), "bytes": e * (3 * rows * d + 2 * rows * H + (ugw + H) * d)},
     }
 
 
-def launches_per_step(w: I.Workload, fold_per_call: bool) -> int:
-    # once: residual-stream set-up; per layer: [weight fold,] Q GEMM, K|V GEMM, attention (split
-    # merge fused in), Fusion GEMM(s), up|gate GEMM, down GEMM
-    return 1 + w.n_layers * (6 + (1 if fold_per_call else 0) + (1 if w.fusion_hidden > 0 else 0))
+def launches_per_step(w: I.Workload, fold_per_call: bool, absorbed: bool) -> int:
+    # once: residual-stream set-up (+ unit starts of the absorbed path); per layer: [weight fold,]
+    # Q GEMM, then either K|V GEMM + attention (split merge fused in) or absorbed-query GEMM + pass A +
+    # pass B + merge + W_V GEMM; Fusion GEMM(s), up|gate GEMM, down GEMM
+    history = 5 if absorbed else 2
+    return 1 + (1 if absorbed else 0) + w.n_layers * (
+        1 + history + 3 + (1 if fold_per_call else 0) + (1 if w.fusion_hidden > 0 else 0))
 
 
 # ------------------------------------------------------------------------------------------------
@@ -219,7 +240,8 @@ def run_reference(args):
 
 
 def run_kernel_case(args):
-    """One step entry point (K|V projection or attention) on one layer, for ncu captures.
+    """One step entry point (K|V projection, attention, absorbed attention, SwiGLU FFN or Fusion MLP)
+    on one layer, for ncu captures.
     Prints the average device time per launch; not a benchmark line."""
     import torch
     from wukong_hstu_cross_b200 import build
@@ -230,13 +252,17 @@ def run_kernel_case(args):
     if args.batch:
         w = w.replace(batch=args.batch)
     p = Hn.build_problem(w, device="cuda")
+    lw = p.weights[0]
+    if args.kernel_case == "absorbed":
+        Hn.prepare_weights(p)   # as the forward runs it: gains folded, absorbed keys formed at load
     T = p.total_L
     kv = torch.empty(T, 2 * w.d, dtype=torch.bfloat16, device="cuda")
     q = torch.empty(w.batch * w.n_tokens, w.d, dtype=torch.bfloat16, device="cuda")
     a = torch.empty_like(q)
-    lw = p.weights[0]
-    Wb.whale_project_queries(p.cfg, q.shape[0], p.tokens, lw["g_q"], lw["w_q"], q, p.workspace)
-    Wb.whale_project_kv(p.cfg, T, p.states[0], lw["g_kv"], lw["w_kv"], kv, p.workspace)
+    raw = Hn.config_of(w)
+    Wb.whale_project_queries(raw, q.shape[0], p.tokens, lw["g_q"], lw["w_q"], q, p.workspace)
+    if args.kernel_case != "absorbed":
+        Wb.whale_project_kv(p.cfg, T, p.states[0], lw["g_kv"], lw["w_kv"], kv, p.workspace)
 
     rows = w.batch * w.n_tokens
     f_out = torch.empty_like(q)
@@ -246,6 +272,8 @@ def run_kernel_case(args):
             Wb.whale_project_kv(p.cfg, T, p.states[0], lw["g_kv"], lw["w_kv"], kv, p.workspace)
         elif args.kernel_case == "attn":
             Wb.whale_cross_attention(p.cfg, q, kv, p.offsets_t, a, p.hint, p.workspace)
+        elif args.kernel_case == "absorbed":  # S2 + S3 without K|V: query GEMM, pass A, pass B, merge, W_V GEMM
+            Wb.whale_attend_states(p.cfg, q, p.states[0], p.offsets_t, p.weights[0], a, p.hint, p.workspace)
         elif args.kernel_case == "ffn":     # up|gate GEMM (SwiGLU epilogue) + down GEMM
             Wb.whale_swiglu_ffn(p.cfg, rows, q, lw["g_ffn"], lw["w_upgate"], lw["w_down"], f_out, p.workspace)
         else:                               # Fusion MLP: two GEMMs
@@ -261,8 +289,9 @@ def run_kernel_case(args):
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / args.steps
-    work = step_work(w, T)[{"kv": "kv_proj", "attn": "attention", "ffn": "swiglu_ffn",
-                             "fusion": "fusion_mlp"}[args.kernel_case]]
+    work = step_work(w, T, absorbed=args.kernel_case == "absorbed")[
+        {"kv": "kv_proj", "attn": "attention", "ffn": "swiglu_ffn", "fusion": "fusion_mlp",
+         "absorbed": "attention_absorbed"}[args.kernel_case]]
     print(json.dumps({"kernel_case": args.kernel_case, "workload": w.name, "total_L": T, "ms_per_launch": ms,
                       "tflops": work["flops"] / ms / 1e9, "gbs": work["bytes"] / ms / 1e6}), flush=True)
     return 0
@@ -278,13 +307,15 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--ref-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel-case", choices=["kv", "attn", "ffn", "fusion"], default=None,
+    ap.add_argument("--kernel-case", choices=["kv", "attn", "ffn", "fusion", "absorbed"], default=None,
                     help="profiling aid: run only one step entry point on one layer of the workload")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (kernel cases)")
     ap.add_argument("--shared-kv", action="store_true", help="variant: K = V (one W_K), the pages' shared key/value")
     ap.add_argument("--tied-gate", action="store_true", help="variant: W_gate = W_up, the pages' shared-gate SwiGLU")
     ap.add_argument("--fold-per-call", action="store_true",
                     help="fold the RMSNorm gains into the weights inside every forward instead of once at load")
+    ap.add_argument("--materialized-kv", action="store_true",
+                    help="project K|V and attend over them even where the absorbed attention applies")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
@@ -303,7 +334,9 @@ def main():
 
     from wukong_hstu_cross_b200 import dist as D
     w = D.shard_workload(I.WORKLOADS[args.workload], rank, world)   # this rank's own examples
-    p = Hn.build_problem(w, device="cuda", shared_kv=args.shared_kv, tied_gate=args.tied_gate)
+    p = Hn.build_problem(w, device="cuda", shared_kv=args.shared_kv, tied_gate=args.tied_gate,
+                         materialized_kv=args.materialized_kv)
+    absorbed = Hn.absorbed_applies(w, args.materialized_kv)
     raw_weights = p.weights
     if not args.fold_per_call:
         Hn.prepare_weights(p)   # gains folded into the weights once, as at model load
@@ -328,8 +361,8 @@ def main():
     ms = max_over_ranks(ms, world)
     value = world * w.batch / (ms / 1e3)
 
-    # ---------------- per-kernel timing of the two heavy steps (same stream, CUDA events) ------
-    work = step_work(w, total_L, args.shared_kv, args.tied_gate)
+    # ---------------- per-kernel timing of the heavy steps (same stream, CUDA events) ------
+    work = step_work(w, total_L, args.shared_kv, args.tied_gate, absorbed)
     Hn_ws = p.workspace
     kv = torch.empty(total_L, (1 if args.shared_kv else 2) * w.d, dtype=torch.bfloat16, device="cuda")
     q = torch.empty(w.batch * w.n_tokens, w.d, dtype=torch.bfloat16, device="cuda")
@@ -358,22 +391,45 @@ def main():
     def attn_step(l):
         Wb.whale_cross_attention(p.cfg, q, kv, p.offsets_t, a, p.hint, Hn_ws, stream=stream)
 
-    kv_step(0)
-    Wb.whale_project_queries(p.cfg, q.shape[0], p.tokens, raw_weights[0]["g_q"], raw_weights[0]["w_q"], q, Hn_ws,
+    def absorbed_step(l):  # the forward's own S2 + S3 call sequence, prepared weights as loaded
+        Wb.whale_attend_states(p.cfg, q, p.states[l], p.offsets_t, p.weights[l], a, p.hint, Hn_ws, stream=stream)
+
+    raw_cfg = Hn.config_of(w)
+    Wb.whale_project_queries(raw_cfg, q.shape[0], p.tokens, raw_weights[0]["g_q"], raw_weights[0]["w_q"], q, Hn_ws,
                              stream=stream)
-    torch.cuda.synchronize()
-    t_kv = timed(kv_step, reps)
-    t_attn = timed(attn_step, reps)
     peaks, peak_src = load_peaks()
-    kv_tflops = work["kv_proj"]["flops"] / (t_kv * 1e-3) / 1e12
-    attn_gbs = work["attention"]["bytes"] / (t_attn * 1e-3) / 1e9
     layer_ms = ms / w.n_layers
-    share_kv, share_attn = t_kv / layer_ms, t_attn / layer_ms
-    kv_traffic = None
-    if w.d == 512 and not args.shared_kv:
-        kv_traffic = KV_TRAFFIC_BYTES_PER_ROW_D512[
-            "1sm" if os.environ.get("WHALE_GEMM_1SM", "0") == "1" else "2sm"] * total_L
-    if share_kv >= share_attn:
+    t_kv = t_attn = t_abs = None
+    if absorbed:
+        torch.cuda.synchronize()
+        t_abs = timed(absorbed_step, reps)
+        abs_tflops = work["attention_absorbed"]["flops"] / (t_abs * 1e-3) / 1e12
+        abs_traffic = None
+        if w.d == 512 and not args.shared_kv and ABS_TRAFFIC_BYTES_PER_ROW_D512 is not None:
+            abs_traffic = ABS_TRAFFIC_BYTES_PER_ROW_D512 * total_L
+        roof = {"kernel": "absorbed attention (pass A scores+softmax, pass B values: tcgen05 2-SM; with the "
+                          "absorbed-query GEMM, merge and W_V GEMM of the same call)",
+                "bound": "tensor", "achieved": abs_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": abs_tflops / peaks["bf16_tflops"], "traffic": abs_traffic,
+                "traffic_source": "ncu capture scaled by rows (profiles/absorbed_attention_hist15k.md)",
+                "frac_of_sustained": abs_tflops / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
+                "algorithmic_per_launch": work["attention_absorbed"]["flops"], "avg_launch_ms": t_abs,
+                "peak_source": f"{peak_src} bf16 burst"}
+    else:
+        kv_step(0)
+        torch.cuda.synchronize()
+        t_kv = timed(kv_step, reps)
+        t_attn = timed(attn_step, reps)
+        kv_tflops = work["kv_proj"]["flops"] / (t_kv * 1e-3) / 1e12
+        attn_gbs = work["attention"]["bytes"] / (t_attn * 1e-3) / 1e9
+        share_kv, share_attn = t_kv / layer_ms, t_attn / layer_ms
+        kv_traffic = None
+        if w.d == 512 and not args.shared_kv:
+            kv_traffic = KV_TRAFFIC_BYTES_PER_ROW_D512[
+                "1sm" if os.environ.get("WHALE_GEMM_1SM", "0") == "1" else "2sm"] * total_L
+    if absorbed:
+        pass
+    elif share_kv >= share_attn:
         roof = {"kernel": "K|V projection GEMM (tcgen05, RMSNorm row factor fused)", "bound": "tensor",
                 "achieved": kv_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": kv_tflops / peaks["bf16_tflops"], "traffic": kv_traffic,
@@ -436,9 +492,10 @@ def main():
                              f"{total_L * w.d * 2 / 1e6:.0f} MB state slab), no flush"},
             "roofline": roof,
             "step_roofline": {"t_star_ms": t_star, "frac": t_star / ms, "per_layer_ms": layer_ms,
-                              "kv_proj_ms": t_kv, "attention_ms": t_attn,
+                              "path": "absorbed" if absorbed else "materialized K|V",
+                              "kv_proj_ms": t_kv, "attention_ms": t_attn, "absorbed_attention_ms": t_abs,
                               "peaks": f"{peak_src}: {peaks['hbm_gbs']} GB/s, {peaks['bf16_tflops']} TFLOP/s"},
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step(w, args.fold_per_call) * args.steps,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step(w, args.fold_per_call, absorbed) * args.steps,
             "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)

@@ -207,6 +207,17 @@ whale_status whale_swiglu_ffn(const whale_config* cfg, long long rows, const voi
                               const void* w_upgate, const void* w_down, void* y, void* workspace,
                               size_t workspace_bytes, whale_stream_t stream);
 
+/* S2 + S3 in absorbed form (see whale_config): A from the projected queries and the raw history
+ * states, without forming K|V. q device [B*N, d] bf16 (whale_project_queries), layer_states device
+ * [total_L, d], offsets device int32 [B+1]; from `w` it reads g_kv and w_kv (raw), or with
+ * WHALE_PREPARED_WEIGHTS the prepared w_kv and w_kabs (w_kabs may be null). a device [B*N, d] bf16.
+ * Workspace: whale_workspace_size. WHALE_ERR_UNSUPPORTED where the absorbed path does not apply
+ * (fp32, other shapes, WHALE_MATERIALIZED_KV). Empty histories give a = 0. */
+whale_status whale_attend_states(const whale_config* cfg, const void* q, const void* layer_states,
+                                 const int* seq_offsets, const whale_layer_weights* w, void* a,
+                                 const whale_shape_hint* hint, void* workspace, size_t workspace_bytes,
+                                 whale_stream_t stream);
+
 /* Eq. (4) like whale_cross_attention, for callers that cannot allocate device memory.
  * No counterpart in the paper: this is a deployment convenience. Some callers cannot call
  * cudaMalloc or hand out a workspace: code embedded in a host framework that owns every byte of

@@ -16,6 +16,7 @@ EXPECTED = {
     "whale_status_string", "whale_workspace_size", "whale_fusion_forward", "whale_host_workspace_size",
     "whale_fusion_forward_host", "whale_fusion_layer_forward", "whale_project_queries", "whale_project_kv",
     "whale_cross_attention", "whale_fusion_mlp", "whale_swiglu_ffn", "whale_get_device_error",
+    "whale_attend_states", "whale_prepare_weights", "whale_prepared_weights_size", "whale_cross_attention_noalloc",
 }
 
 
@@ -91,3 +92,27 @@ def test_empty_batch_is_a_no_op():
     fake = 1 << 20
     wts = [dict.fromkeys(["g_q", "g_kv", "w_q", "w_kv", "w_f1", "w_f2", "g_ffn", "w_upgate", "w_down"], fake)] * 4
     assert W.whale_fusion_forward(cfg, fake, fake, fake, wts, fake, hint, fake, ws, stream=0, raw=True) == 0
+
+
+def test_absorbed_path_selection_and_step_checks():
+    fake = 1 << 20
+    lw = dict.fromkeys(["g_q", "g_kv", "w_q", "w_kv", "w_f1", "w_f2", "g_ffn", "w_upgate", "w_down"], fake)
+    # 15k workload: N*h = 256, d_head = 64 -> absorbed; its workspace holds no K|V tensor
+    w, cfg = _cfg("hist15k_d512")
+    hint = W.make_hint(64, 15000, 403481)
+    cfg_m = W.make_config(cfg.n_layers, cfg.d, cfg.n_heads, cfg.n_tokens, cfg.ffn_hidden, cfg.fusion_hidden,
+                          cfg.dtype, cfg.flags | W.WHALE_MATERIALIZED_KV, cfg.eps)
+    ws_abs, ws_mat = W.whale_workspace_size(cfg, hint), W.whale_workspace_size(cfg_m, hint)
+    assert ws_abs > 0 and ws_mat > 403481 * 2 * w.d * 2
+    assert W.whale_attend_states(cfg, None, fake, fake, lw, fake, hint, fake, ws_abs, stream=0, raw=True) == 1
+    assert W.whale_attend_states(cfg, fake, fake, fake, lw, fake, hint, fake, ws_abs - 1, stream=0, raw=True) == 4
+    assert W.whale_attend_states(cfg_m, fake, fake, fake, lw, fake, hint, fake, ws_mat, stream=0, raw=True) == 2
+    # shapes outside the absorbed path: d_head 32 (stack_d256), fp32
+    for name in ("stack_d256", "tiny_fp32"):
+        w2, cfg2 = _cfg(name)
+        h2 = W.make_hint(2, 10, 20)
+        ws2 = W.whale_workspace_size(cfg2, h2)
+        assert W.whale_attend_states(cfg2, fake, fake, fake, lw, fake, h2, fake, ws2, stream=0, raw=True) == 2
+    # prepared weights carry the absorbed keys only where the path applies
+    assert W.whale_prepared_weights_size(cfg) > W.whale_prepared_weights_size(
+        Hn.config_of(w.replace(n_tokens=16)))

@@ -1,8 +1,9 @@
 """Step-level parity of the CUDA path against the fp64 oracle, through the C ABI:
 S1 query projection, S2 K|V projection (tcgen05 GEMMs with the fused RMSNorm row factor),
 S3 cross-attention (split-L kernel + combine, and the fp32 kernel), S4 Fusion MLP, S5 SwiGLU
-FFN. Shapes cross 128-row tiles with ragged tails, several K/V splits, empty and one-row
-histories, query counts that are not multiples of 16, and each BN tile width."""
+FFN, and S2 + S3 in absorbed form (whale_attend_states). Shapes cross 128-row tiles with ragged
+tails, several K/V splits, empty and one-row histories, query counts that are not multiples of 16,
+and each BN tile width."""
 import numpy as np
 import pytest
 import torch
@@ -207,3 +208,36 @@ def test_project_kv_one_and_two_sm_kernels():
     for kv, name in zip(outs, ("2-SM", "1-SM")):
         assert_parity(kv[torch.from_numpy(sel).to(DEV)], ref, "bf16", rms_rel=1e-2, what=f"KV ({name})")
     assert torch.equal(outs[0], outs[1])
+
+
+ABS_CASES = [
+    # (N, d, heads, lengths): N * heads = 256 absorbed queries, d_head = 64
+    (32, 512, 8, [1, 255, 256, 257, 0, 1024, 777, 3000]),
+    (64, 256, 4, [300, 1, 2048, 129, 0]),
+]
+
+
+@pytest.mark.parametrize("N,d,h,lengths", ABS_CASES)
+@pytest.mark.parametrize("shared", [False, True])
+def test_attend_states_absorbed(N, d, h, lengths, shared):
+    rng = np.random.default_rng(N * 7 + d + shared)
+    L = np.array(lengths, dtype=np.int64)
+    off = I.offsets_of(L)
+    B, total = len(L), int(off[-1])
+    q = bf16_randn(rng, B * N, d)
+    s = bf16_randn(rng, max(total, 1), d)
+    g = rng.uniform(0.5, 1.5, d).astype(np.float32)
+    wkv = I.bf16_round(I.xavier_uniform(rng, d, d)) if shared else \
+        np.concatenate([I.bf16_round(I.xavier_uniform(rng, d, d)), I.bf16_round(I.xavier_uniform(rng, d, d))])
+    cfg = _cfg(d, h, N=N, flags=W.WHALE_SHARED_KV if shared else 0)
+    hint = W.make_hint(B, int(L.max()), total)
+    a = torch.empty(B * N, d, dtype=torch.bfloat16, device=DEV)
+    ws = _ws(W.whale_workspace_size(cfg, hint))
+    W.whale_attend_states(cfg, _t(q), _t(s), torch.from_numpy(off).to(DEV), {"g_kv": _g(g), "w_kv": _t(wkv)}, a,
+                          hint, ws)
+    torch.cuda.synchronize()
+    k, v = O.project_kv(s[:total], g, wkv, 1e-6, shared_kv=shared)
+    ref = np.zeros((B, N, d))
+    for b in range(B):
+        ref[b] = O.cross_attention(q[b * N:(b + 1) * N], k[off[b]:off[b + 1]], v[off[b]:off[b + 1]], h)
+    assert_parity(a, ref.reshape(-1, d), "bf16", rms_rel=1e-2, what="A (absorbed)")

@@ -20,6 +20,8 @@
 //           examples held by one pair, or an unnormalised partial.
 //   merge   combines the partials of examples split across pairs (log-sum-exp weights).
 //
+// The weights pw are stored tiled: the 64 history rows c of unit u form tile 4u + c, rows
+// (4u + c) * 256 + query, 64 columns, so every TMA box of them is one contiguous block.
 // Both passes give the P pairs contiguous ranges of the flattened unit index (units of example b
 // are [ustart[b], ustart[b+1])); a range cut inside an example makes a partial segment, stored
 // in slot 2p (the range's first segment) or 2p + 1 (its last).
@@ -32,7 +34,9 @@ namespace whale {
 
 constexpr int kAbsRows = 256;      // history rows per unit
 constexpr int kAbsQ = 256;         // absorbed queries per example (N * h)
+constexpr int kAbsMaxPairs = 74;   // CTA pairs of one launch (one CTA per SM)
 constexpr float kAbsLazy = 8.0f;   // log2 headroom before the softmax reference is raised
+constexpr float kAbsRedo = 64.0f;  // log2 excess above which a unit's weights are rewritten
 
 struct AbsArgs {
   const int* offsets;       // [B+1]
@@ -103,7 +107,7 @@ struct AbsWalk {
 };
 
 struct AbsUnit {
-  int b, t, nvalid, pcol0, slot;
+  int b, t, nvalid, ptile0, slot;  // ptile0: first 64-row weight tile of the unit (4 per unit)
   long long row0;            // first history row of the unit
   bool first, last, whole;   // first / last unit of its segment; segment = the whole example
 };
@@ -118,7 +122,7 @@ __device__ __forceinline__ AbsUnit abs_unit(const AbsArgs& a, const AbsWalk& w) 
   un.row0 = lo + (long long)kAbsRows * un.t;
   const long long nv = hi - un.row0;
   un.nvalid = nv > kAbsRows ? kAbsRows : (nv < 1 ? 1 : (int)nv);
-  un.pcol0 = w.u * kAbsRows;
+  un.ptile0 = w.u * (kAbsRows / 64);
   un.first = (w.u == w.u0) || (un.t == 0);
   un.last = (w.u == w.u1 - 1) || (w.u == w.ub1 - 1);
   un.whole = (w.u0 <= w.ub) && (w.u1 >= w.ub1);
@@ -355,6 +359,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
     }
   } else {
     // ---------------- softmax epilogue (warps 2..9, both CTAs) ----------------
+    // The first unit of a segment takes its reference from its own tile maximum (a pass over TMEM
+    // and an exchange with the partner half-warp). Later units write their weights with the
+    // current reference in one pass and exchange the tile maximum afterwards: above the lazy
+    // headroom the reference is raised for the following units (never at a segment's last unit,
+    // whose reference is the segment's), and above kAbsRedo the unit is rewritten with the new
+    // maximum so no weight exceeds 2^kAbsRedo.
     const int qd = warp & 3;
     const int hf = (warp - 2) >> 2;  // columns [128 hf, 128 hf + 128) of the unit
     const int row = qd * 32 + lane;
@@ -362,64 +372,72 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
     uint8_t* sbuf = epi + (warp - 2) * 4096;
     const uint32_t tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
     const uint32_t edone_peer0 = mapa_shared(smem_u32(&edone[0]), rank ^ 1);
-    float m_run = 0.f, l_part = 0.f;
-    int it = 0, nseg = 0;
-    for (; wk.valid(); wk.next(a), ++it) {
-      const AbsUnit un = abs_unit(a, wk);
-      const int acc = it & 1, ua = it >> 1;
-      if (!mbar_wait(&tfull[acc], ua & 1, abort_flag)) break;
-      if (!mbar_wait_cluster(&nfull[acc], ua & 1, abort_flag)) break;
-      tc_fence_after();
-      const float* r = rbuf + acc * 256 + hf * 128;
-      const uint32_t t0 = tmem_base + acc * 256 + hf * 128 + ((uint32_t)(qd * 32) << 16);
-      const int nv = un.nvalid - hf * 128;  // valid columns of this warp's half (may be <= 0)
-      // tile maximum of r_t * s over the valid columns
+
+    // maximum of r_t * s over the valid columns of this half
+    auto tile_max = [&](uint32_t t0, const float* r, int nv) -> float {
       float mx = -INFINITY;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(t0 + c * 32, v);
         tmem_ld_wait();
+        const float4* r4 = reinterpret_cast<const float4*>(r + c * 32);
+        const bool masked = c * 32 + 32 > nv;
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (c * 32 + j < nv) mx = fmaxf(mx, __uint_as_float(v[j]) * r[c * 32 + j]);
+        for (int i = 0; i < 8; ++i) {
+          const float4 rr = r4[i];
+          const float x0 = __uint_as_float(v[4 * i]) * rr.x, x1 = __uint_as_float(v[4 * i + 1]) * rr.y;
+          const float x2 = __uint_as_float(v[4 * i + 2]) * rr.z, x3 = __uint_as_float(v[4 * i + 3]) * rr.w;
+          if (!masked) {
+            mx = fmaxf(mx, fmaxf(fmaxf(x0, x1), fmaxf(x2, x3)));
+          } else {
+            const int col = c * 32 + 4 * i;
+            if (col < nv) mx = fmaxf(mx, x0);
+            if (col + 1 < nv) mx = fmaxf(mx, x1);
+            if (col + 2 < nv) mx = fmaxf(mx, x2);
+            if (col + 3 < nv) mx = fmaxf(mx, x3);
+          }
+        }
       }
-      // exchange with the other half-warp of this quadrant (bounded wait: no named barrier that a
-      // partner leaving on a timeout could strand)
-      xmax[(acc * 2 + hf) * 128 + row] = mx;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&xbar[qd * 2 + acc]);
-      if (!mbar_wait(&xbar[qd * 2 + acc], ua & 1, abort_flag)) break;
-      const float mt = fmaxf(xmax[(acc * 2) * 128 + row], xmax[(acc * 2 + 1) * 128 + row]);
-      if (un.first) {
-        m_run = mt;
-        l_part = 0.f;
-      } else if (mt > m_run + kAbsLazy) {
-        l_part *= fast_exp2(m_run - mt);
-        m_run = mt;
-      }
-      // weights p = 2^(r s - m), written as pw = p * r (bf16) through the staging tile
+      return mx;
+    };
+    // p = 2^(r s - m) over the valid columns (0 elsewhere): returns the local maximum of r s, adds
+    // sum(p) to lsum, and stores pw = p * r (bf16) through the staging tile, one 64-column tile
+    // of the tiled weight layout per store.
+    auto write_weights = [&](uint32_t t0, const float* r, int nv, float m, float& lsum, int tile_row0) -> float {
+      float mx = -INFINITY;
 #pragma unroll 1
       for (int cc = 0; cc < 2; ++cc) {
-        uint32_t v[32];
         if (lane == 0) bulk_wait_read<0>();  // the previous store from this buffer has read it
         __syncwarp();
         uint4* dst = reinterpret_cast<uint4*>(sbuf + lane * 128);
-#pragma unroll
+#pragma unroll 1
         for (int h2 = 0; h2 < 2; ++h2) {
           const int c0 = cc * 64 + h2 * 32;
+          uint32_t v[32];
           tmem_ld_32x32b_x32(t0 + c0, v);
           tmem_ld_wait();
+          const float4* r4 = reinterpret_cast<const float4*>(r + c0);
+          const bool masked = c0 + 32 > nv;
 #pragma unroll
           for (int j8 = 0; j8 < 4; ++j8) {
             float w[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int col = c0 + 8 * j8 + j;
-              const float rr = r[col];
-              const float p = col < nv ? fast_exp2(fmaf(__uint_as_float(v[8 * j8 + j]), rr, -m_run)) : 0.f;
-              l_part += p;
-              w[j] = p * rr;
+            for (int h = 0; h < 2; ++h) {
+              const float4 rr = r4[2 * j8 + h];
+              const float rv[4] = {rr.x, rr.y, rr.z, rr.w};
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const int j = 8 * j8 + 4 * h + k;
+                const float x = __uint_as_float(v[j]);
+                const bool ok = !masked || c0 + j < nv;
+                const float xr = x * rv[k];
+                mx = ok ? fmaxf(mx, xr) : mx;
+                const float pexp = fast_exp2(fmaf(x, rv[k], -m));
+                const float pv = ok ? pexp : 0.f;
+                lsum += pv;
+                w[4 * h + k] = pv * (ok ? rv[k] : 0.f);
+              }
             }
             uint4 pk;
             pk.x = pack_bf16x2(w[0], w[1]);
@@ -432,11 +450,64 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&tmP, sbuf, un.pcol0 + hf * 128 + cc * 64, (int)rank * 128 + qd * 32);
+          tma_store_2d(&tmP, sbuf, 0, (tile_row0 + hf * 2 + cc) * kAbsQ + (int)rank * 128 + qd * 32);
           bulk_commit();
         }
       }
-      if (hf == 0) a.mref[(size_t)wk.u * kAbsQ + qg] = m_run;
+      return mx;
+    };
+
+    float m_run = 0.f, l_part = 0.f;
+    int it = 0, nseg = 0;
+    bool ok = true;
+    for (; wk.valid() && ok; wk.next(a), ++it) {
+      const AbsUnit un = abs_unit(a, wk);
+      const int acc = it & 1, ua = it >> 1;
+      if (!mbar_wait(&tfull[acc], ua & 1, abort_flag)) break;
+      if (!mbar_wait_cluster(&nfull[acc], ua & 1, abort_flag)) break;
+      tc_fence_after();
+      const float* r = rbuf + acc * 256 + hf * 128;
+      const uint32_t t0 = tmem_base + acc * 256 + hf * 128 + ((uint32_t)(qd * 32) << 16);
+      const int nv = un.nvalid - hf * 128;  // valid columns of this half (may be <= 0)
+      // tile maximum of both halves, through the quadrant's exchange barrier (bounded wait)
+      auto exchange = [&](float mine) -> float {
+        xmax[(acc * 2 + hf) * 128 + row] = mine;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&xbar[qd * 2 + acc]);
+        if (!mbar_wait(&xbar[qd * 2 + acc], ua & 1, abort_flag)) {
+          ok = false;
+          return mine;
+        }
+        return fmaxf(xmax[(acc * 2) * 128 + row], xmax[(acc * 2 + 1) * 128 + row]);
+      };
+      float m_use, l_unit = 0.f;
+      if (un.first) {
+        m_use = exchange(tile_max(t0, r, nv));
+        if (!ok) break;
+        l_part = 0.f;
+        write_weights(t0, r, nv, m_use, l_unit, un.ptile0);
+        m_run = m_use;
+        l_part = l_unit;
+      } else {
+        m_use = m_run;
+        const float mt = exchange(write_weights(t0, r, nv, m_use, l_unit, un.ptile0));
+        if (!ok) break;
+        if (mt > m_use + kAbsRedo) {
+          // rewrite this unit with the new maximum (after the stores already issued completed)
+          if (lane == 0) bulk_wait<0>();
+          __syncwarp();
+          l_unit = 0.f;
+          write_weights(t0, r, nv, mt, l_unit, un.ptile0);
+          l_part = l_part * fast_exp2(m_use - mt) + l_unit;
+          m_use = m_run = mt;
+        } else if (mt > m_use + kAbsLazy && !un.last) {
+          l_part = (l_part + l_unit) * fast_exp2(m_use - mt);  // the following units use mt
+          m_run = mt;
+        } else {
+          l_part += l_unit;
+        }
+      }
+      if (hf == 0) a.mref[(size_t)wk.u * kAbsQ + qg] = m_use;
       if (un.last) {
         xsum[hf * 128 + row] = l_part;
         __syncwarp();
@@ -447,7 +518,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
           const float l = xsum[row] + xsum[128 + row];
           float2* st = un.whole ? reinterpret_cast<float2*>(a.stats_whole) + (size_t)un.b * kAbsQ + qg
                                 : reinterpret_cast<float2*>(a.stats_part) + (size_t)un.slot * kAbsQ + qg;
-          *st = make_float2(m_run, l);
+          *st = make_float2(m_use, l);
         }
       }
       tc_fence_before();
@@ -561,7 +632,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsBThreads, 1)
           uint8_t* st = smem + s * L::STAGE_BYTES;
           const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
           if (leader) mbar_arrive_expect_tx(&full[s], 2 * L::STAGE_BYTES);
-          tma_load_2d_cg2(st, &tmP, un.pcol0 + 64 * c, (int)rank * 128, bar);
+          tma_load_2d_cg2(st, &tmP, 0, (un.ptile0 + c) * kAbsQ + (int)rank * 128, bar);
           const int hrow = (int)un.row0 + 64 * c;
 #pragma unroll
           for (int e = 0; e < E; ++e)
@@ -702,12 +773,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsBThreads, 1)
 // ================================================================================================
 // merge of examples split across pairs; zero z for empty histories
 // ================================================================================================
-// grid (B, 256 / 8), 256 threads: one warp per absorbed query.
+// grid (B, 256 / 8), 256 threads: one warp per absorbed query. The lanes first gather the
+// (slot, weight) list of the example's partials (one pair each), then stream the partial z rows.
 __global__ void __launch_bounds__(256) abs_merge_kernel(const AbsArgs a) {
   pdl_wait();
   pdl_trigger();
+  __shared__ int s_slot[8][kAbsMaxPairs];
+  __shared__ float s_w[8][kAbsMaxPairs];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x;
-  const int q = blockIdx.y * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  const int q = blockIdx.y * 8 + warp;
   if (q >= kAbsQ) return;
   const int U = a.ustart[a.B];
   const int ub = a.ustart[b], ub1 = a.ustart[b + 1];
@@ -725,26 +800,38 @@ __global__ void __launch_bounds__(256) abs_merge_kernel(const AbsArgs a) {
   const int P = a.n_pairs;
   const int p0 = abs_pair_of(ub, U, P), p1 = abs_pair_of(ub1 - 1, U, P);
   if (p0 == p1) return;  // finished by pass B
-  auto slot_of = [&](int p) { return abs_range_start(U, P, p) >= ub ? 2 * p : 2 * p + 1; };
-  auto nonempty = [&](int p) { return abs_range_start(U, P, p) < abs_range_start(U, P, p + 1); };
+  const int cnt = p1 - p0 + 1;  // <= n_pairs <= kAbsMaxPairs
   const float2* st = reinterpret_cast<const float2*>(a.stats_part);
   float M = -INFINITY;
-  for (int p = p0; p <= p1; ++p)
-    if (nonempty(p)) M = fmaxf(M, st[(size_t)slot_of(p) * kAbsQ + q].x);
+  for (int j = lane; j < cnt; j += 32) {
+    const int p = p0 + j;
+    const int r0 = abs_range_start(U, P, p), r1 = abs_range_start(U, P, p + 1);
+    const int slot = r0 < r1 ? (r0 >= ub ? 2 * p : 2 * p + 1) : -1;
+    s_slot[warp][j] = slot;
+    const float m = slot >= 0 ? st[(size_t)slot * kAbsQ + q].x : -INFINITY;
+    s_w[warp][j] = m;
+    M = fmaxf(M, m);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   float l = 0.f;
-  for (int p = p0; p <= p1; ++p)
-    if (nonempty(p)) {
-      const float2 ml = st[(size_t)slot_of(p) * kAbsQ + q];
-      l += fast_exp2(ml.x - M) * ml.y;
-    }
+  for (int j = lane; j < cnt; j += 32) {
+    const int slot = s_slot[warp][j];
+    const float w = slot >= 0 ? fast_exp2(s_w[warp][j] - M) : 0.f;
+    s_w[warp][j] = w;
+    if (slot >= 0) l += w * st[(size_t)slot * kAbsQ + q].y;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+  __syncwarp();
   const float inv = 1.0f / l;
   for (int c = lane; c < a.d / 4; c += 32) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int p = p0; p <= p1; ++p) {
-      if (!nonempty(p)) continue;
-      const int sl = slot_of(p);
-      const float w = fast_exp2(st[(size_t)sl * kAbsQ + q].x - M);
-      const float4 z = __ldcg(reinterpret_cast<const float4*>(a.part_z + ((size_t)sl * kAbsQ + q) * a.d) + c);
+    for (int j = 0; j < cnt; ++j) {
+      const int slot = s_slot[warp][j];
+      if (slot < 0) continue;
+      const float w = s_w[warp][j];
+      const float4 z = __ldcg(reinterpret_cast<const float4*>(a.part_z + ((size_t)slot * kAbsQ + q) * a.d) + c);
       acc.x = fmaf(w, z.x, acc.x);
       acc.y = fmaf(w, z.y, acc.y);
       acc.z = fmaf(w, z.z, acc.z);

@@ -229,11 +229,12 @@ struct Layout {
   // absorbed attention: folded key weights, absorbed queries, weights pw, unit references,
   // segment statistics, partial z, unit starts, z as a bf16 pair
   size_t wkabs, qa, pw, mref, stw, stp, pz, ust, zh, zl;
-  long long units_max, pw_cols;
+  long long units_max;
   size_t total;
 };
 
-constexpr int kMaxPairs = kNumSM / 2;
+constexpr int kMaxPairs = kAbsMaxPairs;
+static_assert(kAbsMaxPairs == kNumSM / 2, "one CTA pair per two SMs");
 
 // Units of 256 history rows: sum_b ceil(L_b / 256) <= ceil(total_L / 256) + B.
 long long abs_units_max(const whale_shape_hint& h) { return cdiv<long long>(h.total_L, kAbsRows) + h.B; }
@@ -262,10 +263,9 @@ Layout make_layout(const Shape& s, const whale_shape_hint& hint) {
   L.kv = s.absorbed ? 0 : take(tl * s.kvw * s.es);
   if (s.absorbed) {
     L.units_max = abs_units_max(hint);
-    L.pw_cols = L.units_max * kAbsRows;
     L.wkabs = take((size_t)s.h * s.d * s.dh * 2);
     L.qa = take((size_t)hint.B * kAbsQ * s.d * 2);
-    L.pw = take((size_t)kAbsQ * L.pw_cols * 2);
+    L.pw = take((size_t)L.units_max * kAbsRows * kAbsQ * 2);
     L.mref = take((size_t)L.units_max * kAbsQ * 4);
     L.stw = take((size_t)hint.B * kAbsQ * 8);
     L.stp = take((size_t)2 * kMaxPairs * kAbsQ * 8);
@@ -736,11 +736,12 @@ whale_status attention_absorbed(const Shape& s, const void* q, const void* slab,
     CUtensorMap tq, th, tps;
     WCHECK(tmap_bf16(&tq, at(ws, L.qa), (long long)hint.B * kAbsQ, s.d, s.d, 128));
     WCHECK(tmap_bf16(&th, slab, hint.total_L, s.d, s.d, 128));
-    WCHECK(tmap_bf16(&tps, at(ws, L.pw), kAbsQ, L.pw_cols, L.pw_cols, 32));
+    const long long pw_rows = L.units_max * (kAbsRows / 64) * kAbsQ;  // tiled: [4 units_max * 256, 64]
+    WCHECK(tmap_bf16(&tps, at(ws, L.pw), pw_rows, 64, 64, 32));
     CUCHECK(cudaFuncSetAttribute(abs_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AbsASmem::BYTES));
     WCHECK(launch_pdl(abs_scores_kernel, dim3(2 * a.n_pairs), dim3(kAbsAThreads), AbsASmem::BYTES, st, tq, th, tps, a));
     CUtensorMap tpl, th64;
-    WCHECK(tmap_bf16(&tpl, at(ws, L.pw), kAbsQ, L.pw_cols, L.pw_cols, 128));
+    WCHECK(tmap_bf16(&tpl, at(ws, L.pw), pw_rows, 64, 64, 128));
     WCHECK(tmap_bf16(&th64, slab, hint.total_L, s.d, s.d, 64));
     if (E == 1) {
       CUCHECK(cudaFuncSetAttribute(abs_values_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1245,6 +1246,40 @@ whale_status whale_project_kv(const whale_config* cfg, long long rows, const voi
   WCHECK(row_rms(static_cast<const float*>(sx), rows, s.d, s.eps, r, st));
   return gemm_f32(static_cast<const float*>(sx), s.d, nullptr, 0, r, g_kv, static_cast<const float*>(w_kv), s.kvw,
                   static_cast<float*>(kv), rows, F32_NONE, nullptr, st);
+}
+
+whale_status whale_attend_states(const whale_config* cfg, const void* q, const void* layer_states,
+                                 const int* seq_offsets, const whale_layer_weights* w, void* a,
+                                 const whale_shape_hint* hint, void* ws, size_t ws_bytes, whale_stream_t stream) {
+  Shape s;
+  Layout L;
+  WCHECK(common_checks(cfg, hint, &s, ws, ws_bytes, &L));
+  if (!s.absorbed) return WHALE_ERR_UNSUPPORTED;
+  if (hint->B == 0) return WHALE_OK;
+  if (!q || !a || !seq_offsets || !w || !w->w_kv || (!s.prepared && !w->g_kv) || (hint->total_L > 0 && !layer_states))
+    return WHALE_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(a) || !aligned16(w->w_kv) || !aligned16(w->w_kabs) ||
+      (layer_states && !aligned16(layer_states)))
+    return WHALE_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  WCHECK(debug_check(s, seq_offsets, *hint, st));
+  const void* wkv = w->w_kv;
+  const void* wkabs = s.prepared ? w->w_kabs : nullptr;
+  auto* wkabs_ws = reinterpret_cast<__nv_bfloat16*>(at(ws, L.wkabs));
+  if (!s.prepared) {
+    wkv = at(ws, L.wkv);
+    wkabs = wkabs_ws;
+    WCHECK(fold_weights(s, nullptr, nullptr, static_cast<const __nv_bfloat16*>(w->w_kv), w->g_kv, nullptr, nullptr,
+                        nullptr, reinterpret_cast<__nv_bfloat16*>(at(ws, L.wkv)), nullptr, st,
+                        static_cast<const __nv_bfloat16*>(w->w_kv), w->g_kv, wkabs_ws));
+  } else if (!wkabs) {
+    wkabs = wkabs_ws;
+    WCHECK(fold_weights(s, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, st,
+                        static_cast<const __nv_bfloat16*>(w->w_kv), nullptr, wkabs_ws));
+  }
+  const void* wv = s.shared_kv ? wkv : static_cast<const char*>(wkv) + (size_t)s.d * s.d * 2;
+  WCHECK(abs_units(s, seq_offsets, *hint, ws, L, st));
+  return attention_absorbed(s, q, layer_states, seq_offsets, wkabs, wv, a, nullptr, *hint, ws, L, st);
 }
 
 whale_status whale_cross_attention(const whale_config* cfg, const void* q, const void* kv, const int* seq_offsets,

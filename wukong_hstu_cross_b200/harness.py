@@ -40,9 +40,15 @@ def weights_to_device(lws, w: I.Workload, device) -> list:
     return out
 
 
-def flags_of(shared_kv=False, tied_gate=False, debug=False) -> int:
+def flags_of(shared_kv=False, tied_gate=False, debug=False, materialized_kv=False) -> int:
     return (W.WHALE_SHARED_KV if shared_kv else 0) | (W.WHALE_TIED_GATE if tied_gate else 0) | \
-        (W.WHALE_DEBUG if debug else 0)
+        (W.WHALE_DEBUG if debug else 0) | (W.WHALE_MATERIALIZED_KV if materialized_kv else 0)
+
+
+def absorbed_applies(w: I.Workload, materialized_kv: bool = False) -> bool:
+    """Whether the library takes the absorbed attention path for this workload (whale_config)."""
+    return (w.dtype == "bf16" and not materialized_kv and w.n_tokens * w.n_heads == 256 and w.d_head == 64
+            and w.d in (256, 512))
 
 
 def config_of(w: I.Workload, flags: int = 0) -> W.whale_config:
@@ -73,7 +79,7 @@ class Problem:
 
 
 def build_problem(w: I.Workload, device="cuda", gains="ones", shared_kv=False, tied_gate=False, debug=False,
-                  lengths: np.ndarray | None = None, threads: int = 16) -> Problem:
+                  lengths: np.ndarray | None = None, threads: int = 16, materialized_kv=False) -> Problem:
     L = I.draw_lengths(w) if lengths is None else np.asarray(lengths, dtype=np.int64)
     off = I.offsets_of(L)
     total = int(off[-1])
@@ -89,7 +95,7 @@ def build_problem(w: I.Workload, device="cuda", gains="ones", shared_kv=False, t
         else:
             states[l, :total].copy_(torch.from_numpy(I.make_states_layer(w, l, L, threads=threads)))
     tokens = to_device(I.make_tokens(w), w, device)
-    fl = flags_of(shared_kv, tied_gate, debug)
+    fl = flags_of(shared_kv, tied_gate, debug, materialized_kv)
     cfg = config_of(w, fl)
     hint = W.make_hint(w.batch, int(L.max()) if len(L) else 0, total)
     ws_bytes = W.whale_workspace_size(cfg, hint)

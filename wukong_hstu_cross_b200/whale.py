@@ -66,6 +66,8 @@ _SIGS = {
     "whale_project_kv": ([POINTER(whale_config), c_longlong, _P, _P, _P, _P, _P, c_size_t, _P], c_int),
     "whale_cross_attention": ([POINTER(whale_config), _P, _P, _P, _P, POINTER(whale_shape_hint), _P, c_size_t,
                                _P], c_int),
+    "whale_attend_states": ([POINTER(whale_config), _P, _P, _P, POINTER(whale_layer_weights), _P,
+                             POINTER(whale_shape_hint), _P, c_size_t, _P], c_int),
     "whale_fusion_mlp": ([POINTER(whale_config), c_longlong, _P, _P, _P, _P, _P, _P, c_size_t, _P], c_int),
     "whale_swiglu_ffn": ([POINTER(whale_config), c_longlong, _P, _P, _P, _P, _P, _P, c_size_t, _P], c_int),
     "whale_get_device_error": ([_P, POINTER(c_int)], c_int),
@@ -229,6 +231,18 @@ def whale_cross_attention(cfg, q, kv, seq_offsets, a, hint, workspace, workspace
     if raw:
         return st
     _check(st, "whale_cross_attention")
+
+
+def whale_attend_states(cfg, q, layer_states, seq_offsets, weights, a, hint, workspace, workspace_bytes=None,
+                        stream=None, raw=False):
+    """S2 + S3 in absorbed form (no K|V tensor): `weights` is one layer's dict or whale_layer_weights."""
+    lw = layer_weights(weights)
+    st = _lib.whale_attend_states(ctypes.byref(cfg), _ptr(q), _ptr(layer_states), _ptr(seq_offsets),
+                                  ctypes.byref(lw), _ptr(a), ctypes.byref(hint), _ptr(workspace),
+                                  _ws_bytes(workspace, workspace_bytes), _stream(stream))
+    if raw:
+        return st
+    _check(st, "whale_attend_states")
 
 
 def whale_cross_attention_noalloc(cfg, q, kv, seq_offsets, a, hint, stream=None, raw=False):
