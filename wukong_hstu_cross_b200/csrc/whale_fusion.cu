@@ -26,6 +26,7 @@
 #include <mutex>
 
 #include "absorbed.cuh"
+#include "absorbed_fused.cuh"
 #include "aux_kernels.cuh"
 #include "attention.cuh"
 #include "fp32_path.cuh"
@@ -58,6 +59,14 @@ constexpr int kNumSM = 148;
 inline bool gemm_2sm_enabled() {
   const char* e = std::getenv("WHALE_GEMM_1SM");
   return !(e && e[0] == '1');
+}
+// The absorbed attention runs its two passes as two kernels by default; WHALE_ABS_FUSED=1 in the
+// environment selects the four-CTA-cluster kernel that runs both at once (absorbed_fused.cuh; it
+// reads each history row from HBM once, but its scorer pair is bound by the softmax, and it is
+// slower on the 15k-history workload). Read per call (comparison runs and tests).
+inline bool abs_fused_enabled() {
+  const char* e = std::getenv("WHALE_ABS_FUSED");
+  return e && e[0] == '1';
 }
 constexpr size_t kAlign = 256;
 inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -641,6 +650,40 @@ whale_status abs_max_pairs(int E, int* pairs) {
   return c > 0 ? WHALE_OK : WHALE_ERR_UNSUPPORTED;
 }
 
+// Co-resident four-CTA clusters of the fused kernel (cached per device).
+whale_status abs_max_clusters(int E, int* clusters) {
+  static std::mutex mu;
+  static int cache[64][2];
+  int dev = 0;
+  CUCHECK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return WHALE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(mu);
+  int& c = cache[dev][E - 1];
+  if (c == 0) {
+    const void* kern = E == 1 ? reinterpret_cast<const void*>(abs_fused_kernel<1>)
+                              : reinterpret_cast<const void*>(abs_fused_kernel<2>);
+    const size_t smem = E == 1 ? FuSmem<1>::BYTES : FuSmem<2>::BYTES;
+    CUCHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(4 * kFuMaxClusters, 1, 1);
+    lc.blockDim = dim3(kFuThreads, 1, 1);
+    lc.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 4;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    int n = 0;
+    CUCHECK(cudaOccupancyMaxActiveClusters(&n, kern, &lc));
+    n = std::min(n, kFuMaxClusters);
+    c = n > 0 ? n : -1;
+  }
+  *clusters = c;
+  return c > 0 ? WHALE_OK : WHALE_ERR_UNSUPPORTED;
+}
+
 // qa[b*256 + j*N + n, :] = q[b*N + n, j*64 : j*64 + 64] W~_j^T with W~ [h*d, 64] (one K block per
 // head: a block-diagonal GEMM over the h*d output columns, rows scattered per head).
 whale_status gemm_qabs(const Shape& s, const void* q, const void* wkabs, void* qa, long long rows, cudaStream_t st) {
@@ -729,6 +772,25 @@ whale_status attention_absorbed(const Shape& s, const void* q, const void* slab,
   a.part_z = reinterpret_cast<float*>(at(ws, L.pz));
   a.z_hi = reinterpret_cast<__nv_bfloat16*>(at(ws, L.zh));
   a.z_lo = reinterpret_cast<__nv_bfloat16*>(at(ws, L.zl));
+  if (abs_fused_enabled()) {
+    int clusters = 0;
+    WCHECK(abs_max_clusters(E, &clusters));
+    a.n_pairs = (int)std::max<long long>(1, std::min<long long>(clusters, L.units_max));
+    if (hint.total_L > 0) {
+      CUtensorMap tq, th, th64;
+      WCHECK(tmap_bf16(&tq, at(ws, L.qa), (long long)hint.B * kAbsQ, s.d, s.d, 128));
+      WCHECK(tmap_bf16(&th, slab, hint.total_L, s.d, s.d, 128));
+      WCHECK(tmap_bf16(&th64, slab, hint.total_L, s.d, s.d, 64));
+      if (E == 1)
+        WCHECK(launch_pdl(abs_fused_kernel<1>, dim3(4 * a.n_pairs), dim3(kFuThreads), FuSmem<1>::BYTES, st, tq, th,
+                          th64, a));
+      else
+        WCHECK(launch_pdl(abs_fused_kernel<2>, dim3(4 * a.n_pairs), dim3(kFuThreads), FuSmem<2>::BYTES, st, tq, th,
+                          th64, a));
+    }
+    WCHECK(launch_pdl(abs_merge_kernel, dim3(hint.B, kAbsQ / 8), dim3(256), 0, st, a));
+    return gemm_vabs(s, at(ws, L.zh), at(ws, L.zl), wv, out, out_lo, rows, st);
+  }
   int pairs = 0;
   WCHECK(abs_max_pairs(E, &pairs));
   a.n_pairs = (int)std::max<long long>(1, std::min<long long>(pairs, L.units_max));
