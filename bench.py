@@ -32,14 +32,15 @@ from wukong_hstu_cross_b200 import inputs as I  # noqa: E402
 
 METRIC = "WHALE fusion-layer examples/s @15k jagged history; % of HBM/TC roofline"
 # DRAM bytes per launch measured by ncu (dram__bytes_read.sum + dram__bytes_write.sum), per
-# history row, from the committed summary profiles/kv_proj_gemm_hist15k.md (d = 512; the 2-SM
-# default kernel and the one-SM kernel). Reported only for that width; null otherwise.
+# history row: one capture of the K|V projection GEMM at d = 512 on 109 605 rows (the 2-SM default
+# kernel and the one-SM kernel). Reported only for that width; null otherwise.
 KV_TRAFFIC_BYTES_PER_ROW_D512 = {"2sm": (113.378816e6 + 169.603840e6) / 109605,
                                  "1sm": (113.375488e6 + 168.328960e6) / 109605}
 
-# DRAM bytes per history row of one whale_attend_states call (pass A + pass B + the small kernels),
-# from the committed summary profiles/absorbed_attention_hist15k.md; None until captured.
-ABS_TRAFFIC_BYTES_PER_ROW_D512 = None
+# DRAM bytes per history row of one whale_attend_states call (qa GEMM, pass A, pass B, merge, W_V
+# GEMM, unit starts): one ncu capture of the six kernels at d = 512 on the full 403 481-row batch
+# (1167.7 MB read + 209.7 MB written per call). Two-kernel path only (the default).
+ABS_TRAFFIC_BYTES_PER_ROW_D512 = (1167.7e6 + 209.7e6) / 403481
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
 
@@ -405,13 +406,13 @@ def main():
         t_abs = timed(absorbed_step, reps)
         abs_tflops = work["attention_absorbed"]["flops"] / (t_abs * 1e-3) / 1e12
         abs_traffic = None
-        if w.d == 512 and not args.shared_kv and ABS_TRAFFIC_BYTES_PER_ROW_D512 is not None:
+        if w.d == 512 and not args.shared_kv and os.environ.get("WHALE_ABS_FUSED", "0") != "1":
             abs_traffic = ABS_TRAFFIC_BYTES_PER_ROW_D512 * total_L
         roof = {"kernel": "absorbed attention (pass A scores+softmax, pass B values: tcgen05 2-SM; with the "
                           "absorbed-query GEMM, merge and W_V GEMM of the same call)",
                 "bound": "tensor", "achieved": abs_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": abs_tflops / peaks["bf16_tflops"], "traffic": abs_traffic,
-                "traffic_source": "ncu capture scaled by rows (profiles/absorbed_attention_hist15k.md)",
+                "traffic_source": "ncu dram bytes of the six kernels of one call at the full batch, per row",
                 "frac_of_sustained": abs_tflops / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
                 "algorithmic_per_launch": work["attention_absorbed"]["flops"], "avg_launch_ms": t_abs,
                 "peak_source": f"{peak_src} bf16 burst"}
@@ -433,7 +434,7 @@ def main():
         roof = {"kernel": "K|V projection GEMM (tcgen05, RMSNorm row factor fused)", "bound": "tensor",
                 "achieved": kv_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": kv_tflops / peaks["bf16_tflops"], "traffic": kv_traffic,
-                "traffic_source": "ncu capture scaled by rows (profiles/kv_proj_gemm_hist15k.md)",
+                "traffic_source": "ncu dram bytes of one launch on 109605 rows, scaled by rows",
                 "frac_of_sustained": kv_tflops / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
                 "algorithmic_per_launch": work["kv_proj"]["flops"], "avg_launch_ms": t_kv,
                 "peak_source": f"{peak_src} bf16 burst"}
