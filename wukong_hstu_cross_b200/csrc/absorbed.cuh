@@ -58,7 +58,8 @@ __device__ __forceinline__ long long abs_off(const AbsArgs& a, int b) {
   return o < 0 ? 0 : (o > a.total_L ? a.total_L : o);
 }
 
-__device__ __forceinline__ int abs_range_start(int U, int P, int p) { return (int)(((long long)U * p) / P); }
+// U * p < 2^31: units_max < 2^31 / 256 (checked on the host) and P <= kAbsMaxPairs.
+__device__ __forceinline__ int abs_range_start(int U, int P, int p) { return (int)(((unsigned)U * (unsigned)p) / (unsigned)P); }
 
 // Pair whose range holds unit u (0 <= u < U).
 __device__ __forceinline__ int abs_pair_of(int u, int U, int P) {
