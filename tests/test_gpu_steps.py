@@ -120,6 +120,42 @@ def test_cross_attention_bf16(N, d, h, lengths):
     assert_parity(a, _attn_ref(q, kv, off, N, d, h), "bf16", rms_rel=1e-2, what="A")
 
 
+QTILE_CASES = [
+    # many queries per history: the query-tiled kernel (N >= 128); ragged query tiles, empty and
+    # one-row histories, blocks of 128 history rows with ragged tails, d_head 32 and 64
+    (128, 256, 8, [1, 127, 128, 129, 0, 700]),
+    (160, 256, 8, [300, 1, 2049]),
+    (256, 512, 8, [129, 0, 1500]),
+    (200, 128, 2, [64, 1000]),
+]
+
+
+@pytest.mark.parametrize("N,d,h,lengths", QTILE_CASES)
+@pytest.mark.parametrize("shared", [False, True])
+def test_cross_attention_many_queries(N, d, h, lengths, shared, monkeypatch):
+    rng = np.random.default_rng(N * 1000 + d + shared)
+    L = np.array(lengths, dtype=np.int64)
+    off = I.offsets_of(L)
+    B, total = len(L), int(off[-1])
+    q = bf16_randn(rng, B * N, d)
+    kv = bf16_randn(rng, max(total, 1), (1 if shared else 2) * d)
+    cfg = _cfg(d, h, N=N, flags=W.WHALE_SHARED_KV if shared else 0)
+    hint = W.make_hint(B, int(L.max()), total)
+    ws = _ws(W.whale_workspace_size(cfg, hint))
+    offs = torch.from_numpy(off).to(DEV)
+    a = torch.empty(B * N, d, dtype=torch.bfloat16, device=DEV)
+    W.whale_cross_attention(cfg, _t(q), _t(kv), offs, a, hint, ws)
+    torch.cuda.synchronize()
+    assert_parity(a, _attn_ref(q, kv, off, N, d, h, shared), "bf16", rms_rel=1e-2, what="A (query tiles)")
+    # the split-L kernel on the same inputs agrees within the bound
+    monkeypatch.setenv("WHALE_ATTN_SPLITL", "1")
+    a2 = torch.empty_like(a)
+    W.whale_cross_attention(cfg, _t(q), _t(kv), offs, a2, hint, ws)
+    torch.cuda.synchronize()
+    x, y = a.float(), a2.float()
+    assert bool(((x - y).abs() <= 2e-2 * (1 + y.abs())).all())
+
+
 def test_cross_attention_shared_kv_and_fp32():
     rng = np.random.default_rng(99)
     N, d, h = 32, 256, 8

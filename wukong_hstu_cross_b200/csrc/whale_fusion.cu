@@ -29,6 +29,7 @@
 #include "absorbed_fused.cuh"
 #include "aux_kernels.cuh"
 #include "attention.cuh"
+#include "attention_qtile.cuh"
 #include "fp32_path.cuh"
 #include "gemm_2sm.cuh"
 #include "gemm_persistent.cuh"
@@ -64,6 +65,12 @@ inline bool gemm_2sm_enabled() {
 // environment selects the four-CTA-cluster kernel that runs both at once (absorbed_fused.cuh; it
 // reads each history row from HBM once, but its scorer pair is bound by the softmax, and it is
 // slower on the 15k-history workload). Read per call (comparison runs and tests).
+// Histories attended by many queries (N >= 128 per example) take the query-tiled tcgen05 kernel;
+// WHALE_ATTN_SPLITL=1 in the environment keeps the split-L kernel for them (comparison runs, tests).
+inline bool qtile_enabled() {
+  const char* e = std::getenv("WHALE_ATTN_SPLITL");
+  return !(e && e[0] == '1');
+}
 inline bool abs_fused_enabled() {
   const char* e = std::getenv("WHALE_ABS_FUSED");
   return e && e[0] == '1';
@@ -563,6 +570,37 @@ whale_status launch_attn_hg(int hg, const CUtensorMap& tm, const AttnArgs& a, di
   return WHALE_ERR_UNSUPPORTED;
 }
 
+// Query-tiled attention (attention_qtile.cuh): one CTA per (example, 128 queries, head box).
+whale_status attention_qtile(const Shape& s, const void* q, const void* kv, const int* offsets, void* out,
+                             void* out_lo, int B, long long total_L, cudaStream_t st) {
+  QtArgs a{};
+  a.offsets = offsets;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.out_lo = static_cast<__nv_bfloat16*>(out_lo);
+  a.B = B;
+  a.N = s.N;
+  a.d = s.d;
+  a.n_qt = (int)cdiv<long long>(s.N, 128);
+  a.n_hb = s.h / (64 / s.dh);
+  a.v_col0 = s.shared_kv ? 0 : s.d;
+  a.total_L = total_L;
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)s.dh));
+  const long long grid = (long long)B * a.n_qt * a.n_hb;
+  if (grid <= 0) return WHALE_OK;
+  if (grid > 0x7fffffffll) return WHALE_ERR_UNSUPPORTED;
+  CUtensorMap tq, tkv;
+  WCHECK(tmap_bf16(&tq, q, (long long)B * s.N, s.d, s.d, 128));
+  WCHECK(tmap_bf16(&tkv, kv, total_L, s.kvw, s.kvw, 128));
+  if (s.dh == 32) {
+    CUCHECK(cudaFuncSetAttribute(attn_qtile_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)QtSmem<32>::BYTES));
+    return launch_pdl(attn_qtile_kernel<32>, dim3((unsigned)grid), dim3(kQtThreads), QtSmem<32>::BYTES, st, tq, tkv, a);
+  }
+  CUCHECK(cudaFuncSetAttribute(attn_qtile_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)QtSmem<64>::BYTES));
+  return launch_pdl(attn_qtile_kernel<64>, dim3((unsigned)grid), dim3(kQtThreads), QtSmem<64>::BYTES, st, tq, tkv, a);
+}
+
 whale_status attention_bf16(const Shape& s, const void* q, const void* kv, const int* offsets, void* out,
                             void* out_lo, int B, long long total_L, void* scratch, cudaStream_t st) {
   if (B == 0) return WHALE_OK;
@@ -573,6 +611,7 @@ whale_status attention_bf16(const Shape& s, const void* q, const void* kv, const
     if (out_lo) CUCHECK(cudaMemsetAsync(out_lo, 0, rows * s.d * 2, st));
     return WHALE_OK;
   }
+  if (s.N >= 128 && (s.dh == 32 || s.dh == 64) && qtile_enabled()) return attention_qtile(s, q, kv, offsets, out, out_lo, B, total_L, st);
   AttnArgs a{};
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.offsets = offsets;
