@@ -438,6 +438,18 @@ def main():
                 "frac_of_sustained": kv_tflops / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
                 "algorithmic_per_launch": work["kv_proj"]["flops"], "avg_launch_ms": t_kv,
                 "peak_source": f"{peak_src} bf16 burst"}
+    elif w.n_tokens >= 128:
+        # many queries per history (the serving shape): the query-tiled tensor-core attention is
+        # bound by its softmax exponentials. Peak = MUFU ex2 throughput: 16 per clock per SM x SMs x
+        # the maximum SM clock (nominal unit counts; sm_max_mhz is the measured maximum clock).
+        n_exp = float(w.n_heads) * w.n_tokens * total_L   # every query of an example against its rows
+        exp_peak = 16.0 * 148 * peaks.get("sm_max_mhz", 1965.0) * 1e6
+        exps = n_exp / (t_attn * 1e-3)
+        roof = {"kernel": "query-tiled attention (tcgen05 S and P V, softmax on MUFU + FMA polynomial)",
+                "bound": "alu", "achieved": exps / 1e12, "peak": exp_peak / 1e12, "unit": "Texp/s",
+                "frac": exps / exp_peak, "traffic": None, "algorithmic_per_launch": n_exp, "avg_launch_ms": t_attn,
+                "peak_source": "16 ex2/clk/SM x 148 SMs x max SM clock (nominal unit counts)",
+                "tensor_tflops": work["attention"]["flops"] / (t_attn * 1e-3) / 1e12}
     else:
         roof = {"kernel": "split-L cross-attention + combine", "bound": "hbm", "achieved": attn_gbs,
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": attn_gbs / peaks["hbm_gbs"], "traffic": None,
