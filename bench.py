@@ -18,6 +18,7 @@ from __future__ import annotations
 import argparse
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -41,6 +42,8 @@ KV_TRAFFIC_BYTES_PER_ROW_D512 = {"2sm": (113.378816e6 + 169.603840e6) / 109605,
 # GEMM, unit starts): one ncu capture of the six kernels at d = 512 on the full 403 481-row batch
 # (1167.7 MB read + 209.7 MB written per call). Two-kernel path only (the default).
 ABS_TRAFFIC_BYTES_PER_ROW_D512 = (1167.7e6 + 209.7e6) / 403481
+# ... and of its pass A kernel alone (abs_scores_kernel: 441.23 MB read + 174.07 MB written)
+ABS_PASSA_BYTES_PER_ROW_D512 = (441.23e6 + 174.07e6) / 403481
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
 
@@ -87,6 +90,22 @@ def step_work(w: I.Workload, total_L: int, shared_kv: bool = False, tied_gate: b
         "fusion_mlp": {"flops": 2.0 * rows * (2 * d * Fh + Fh * d), "bytes": e * (3 * rows * d + 2 * rows * Fh + 3 * d * Fh)},
         "swiglu_ffn": {"flops": 2.0 * rows * (d * ugw + H * d), "bytes": e * (3 * rows * d + 2 * rows * H + (ugw + H) * d)},
     }
+
+
+def kernel_name(mangled: str) -> str:
+    """Readable name of one of the library's kernels: `_ZN5whale17abs_scores_kernelE...` ->
+    `abs_scores_kernel`, with integer / bool template arguments as `<64,2,0,1>`."""
+    m = re.match(r"_ZN5whale(\d+)", mangled)
+    if not m:
+        return mangled
+    n = int(m.group(1))
+    rest = mangled[m.end():]
+    name, rest = rest[:n], rest[n:]
+    if rest.startswith("I"):
+        args = re.findall(r"L[ib](-?\d+)E", rest.split("EE")[0] + "E")
+        if args:
+            name += "<" + ",".join(args) + ">"
+    return name
 
 
 def launches_per_step(w: I.Workload, fold_per_call: bool, absorbed: bool) -> int:
@@ -362,6 +381,21 @@ def main():
     ms = max_over_ranks(ms, world)
     value = world * w.batch / (ms / 1e3)
 
+    # ---------------- every kernel of one step, live: the library's per-kernel events -------------
+    # (one extra step after the timed region; the events serialise launches, so each kernel's time
+    # is its own, and their sum is a little above the step time measured above)
+    Wb.whale_profile_begin(4096)
+    Hn.run_forward(p, stream)
+    recs = Wb.whale_profile_end()
+    kern = {}
+    for name, kms in recs:
+        e = kern.setdefault(kernel_name(name), [0, 0.0])
+        e[0] += 1
+        e[1] += kms
+    kern_total = sum(v[1] for v in kern.values()) or 1.0
+    kernels = {n: {"launches": c, "avg_ms": tt / c, "share": tt / kern_total}
+               for n, (c, tt) in sorted(kern.items(), key=lambda x: -x[1][1])}
+
     # ---------------- per-kernel timing of the heavy steps (same stream, CUDA events) ------
     work = step_work(w, total_L, args.shared_kv, args.tied_gate, absorbed)
     Hn_ws = p.workspace
@@ -408,14 +442,33 @@ def main():
         abs_traffic = None
         if w.d == 512 and not args.shared_kv and os.environ.get("WHALE_ABS_FUSED", "0") != "1":
             abs_traffic = ABS_TRAFFIC_BYTES_PER_ROW_D512 * total_L
-        roof = {"kernel": "absorbed attention (pass A scores+softmax, pass B values: tcgen05 2-SM; with the "
-                          "absorbed-query GEMM, merge and W_V GEMM of the same call)",
-                "bound": "tensor", "achieved": abs_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": abs_tflops / peaks["bf16_tflops"], "traffic": abs_traffic,
-                "traffic_source": "ncu dram bytes of the six kernels of one call at the full batch, per row",
-                "frac_of_sustained": abs_tflops / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
-                "algorithmic_per_launch": work["attention_absorbed"]["flops"], "avg_launch_ms": t_abs,
-                "peak_source": f"{peak_src} bf16 burst"}
+        call = {"entry_point": "whale_attend_states (qa GEMM, pass A, pass B, merge, W_V GEMM, unit starts)",
+                "tflops": abs_tflops, "frac": abs_tflops / peaks["bf16_tflops"], "avg_call_ms": t_abs,
+                "algorithmic_flops": work["attention_absorbed"]["flops"],
+                "algorithmic_bytes": work["attention_absorbed"]["bytes"], "traffic": abs_traffic,
+                "traffic_source": "ncu dram bytes of the six kernels of one call at the full batch, per row"}
+        pa = kernels.get("abs_scores_kernel")
+        if pa:
+            # the dominant kernel, pass A: S = qa H^T of N*h queries against every history row
+            # (2 (N h) d FLOP per row) with the softmax; its ncu DRAM bytes per row scaled by rows
+            fa = 2.0 * w.n_tokens * w.n_heads * total_L * w.d
+            ta = pa["avg_ms"]
+            a_tflops = fa / (ta * 1e-3) / 1e12
+            a_traffic = (ABS_PASSA_BYTES_PER_ROW_D512 * total_L) if abs_traffic is not None else None
+            roof = {"kernel": "abs_scores_kernel (absorbed pass A: scores on tcgen05 2-SM, online softmax, weights)",
+                    "bound": "tensor", "achieved": a_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": a_tflops / peaks["bf16_tflops"], "traffic": a_traffic,
+                    "traffic_source": "ncu dram bytes of one launch at the full batch, per row",
+                    "frac_of_sustained": a_tflops / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
+                    "algorithmic_per_launch": fa, "algorithmic_bytes_per_launch": 2.0 * total_L * w.d,
+                    "avg_launch_ms": ta, "timing": "library per-kernel events on the bench stream",
+                    "peak_source": f"{peak_src} bf16 burst", "call": call}
+        else:
+            roof = {"kernel": "whale_attend_states (the absorbed S2 + S3 call)", "bound": "tensor",
+                    "achieved": abs_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": abs_tflops / peaks["bf16_tflops"], "traffic": abs_traffic,
+                    "algorithmic_per_launch": work["attention_absorbed"]["flops"], "avg_launch_ms": t_abs,
+                    "peak_source": f"{peak_src} bf16 burst", "call": call}
     else:
         kv_step(0)
         torch.cuda.synchronize()
@@ -508,7 +561,8 @@ def main():
                               "path": "absorbed" if absorbed else "materialized K|V",
                               "kv_proj_ms": t_kv, "attention_ms": t_attn, "absorbed_attention_ms": t_abs,
                               "peaks": f"{peak_src}: {peaks['hbm_gbs']} GB/s, {peaks['bf16_tflops']} TFLOP/s"},
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step(w, args.fold_per_call, absorbed) * args.steps,
+            "kernels": kernels,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": (len(recs) or launches_per_step(w, args.fold_per_call, absorbed)) * args.steps,
             "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)

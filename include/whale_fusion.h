@@ -128,6 +128,22 @@ typedef struct {
 /* Human-readable name of a status code (static string). */
 const char* whale_status_string(whale_status s);
 
+/* Per-kernel timing, for profiling runs (no counterpart in the paper). Between
+ * whale_profile_begin and whale_profile_end, every kernel of the bf16 path that the library
+ * launches is followed by a CUDA event on its stream (at most max_kernels of them; the first
+ * launch is also preceded by one), so that kernel k's time is the time between event k-1 and
+ * event k. The events serialise the launches: a kernel no longer overlaps its prologue with its
+ * predecessor's tail, so the sum can exceed an unprofiled run slightly. whale_profile_end waits
+ * for the last event, writes up to `capacity` records {kernel name (owned by the CUDA runtime),
+ * milliseconds} in launch order, sets *count to the number recorded, and releases the events.
+ * Not thread-safe across concurrent forwards on different streams (one global record list). */
+typedef struct {
+  const char* kernel;
+  float ms;
+} whale_kernel_time;
+whale_status whale_profile_begin(int max_kernels);
+whale_status whale_profile_end(whale_kernel_time* out, int capacity, int* count);
+
 /* Bytes of device workspace needed by every entry point below for this config and
  * shape (0 if cfg/hint are invalid or unsupported). */
 size_t whale_workspace_size(const whale_config* cfg, const whale_shape_hint* hint);

@@ -17,6 +17,7 @@ EXPECTED = {
     "whale_fusion_forward_host", "whale_fusion_layer_forward", "whale_project_queries", "whale_project_kv",
     "whale_cross_attention", "whale_fusion_mlp", "whale_swiglu_ffn", "whale_get_device_error",
     "whale_attend_states", "whale_prepare_weights", "whale_prepared_weights_size", "whale_cross_attention_noalloc",
+    "whale_profile_begin", "whale_profile_end",
 }
 
 
@@ -116,3 +117,11 @@ def test_absorbed_path_selection_and_step_checks():
     # prepared weights carry the absorbed keys only where the path applies
     assert W.whale_prepared_weights_size(cfg) > W.whale_prepared_weights_size(
         Hn.config_of(w.replace(n_tokens=16)))
+
+
+def test_profile_records_nothing_without_launches():
+    assert W._lib.whale_profile_begin(0) == 1          # max_kernels must be positive
+    W.whale_profile_begin(16)
+    assert W.whale_profile_end() == []                  # no kernel launched: no records, no CUDA call
+    n = ctypes.c_int(-1)
+    assert W._lib.whale_profile_end(None, 4, ctypes.byref(n)) == 1   # records requested into a null buffer

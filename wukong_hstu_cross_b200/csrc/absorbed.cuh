@@ -48,9 +48,8 @@ struct AbsArgs {
   float* mref;              // [units_max, 256] softmax reference of each unit (log2 units)
   float* stats_whole;       // [B, 256] (m, l) of examples held by one pair
   float* stats_part;        // [2 * n_pairs, 256] (m, l) of partial segments
-  float* part_z;            // [2 * n_pairs, 256, d] unnormalised z of partial segments
-  __nv_bfloat16* z_hi;      // [h, B*N, d] z / l, bf16 pair (row j*B*N + b*N + n)
-  __nv_bfloat16* z_lo;
+  __nv_bfloat16* part_z;    // [2 * n_pairs, 256, d] unnormalised z of partial segments (bf16)
+  __nv_bfloat16* z_hi;      // [h, B*N, d] z / l, bf16 (row j*B*N + b*N + n)
 };
 
 __device__ __forceinline__ long long abs_off(const AbsArgs& a, int b) {
@@ -542,6 +541,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
   }
 }
 
+
+// 32 fp32 values scaled by `s` -> 32 bf16 at `dst` (16-byte aligned): four 16-byte stores.
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const uint32_t (&v)[32], float s) {
+  uint32_t w[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(__uint_as_float(v[2 * j]) * s, __uint_as_float(v[2 * j + 1]) * s);
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+}
+
 // ================================================================================================
 // pass B: z += pw H
 // ================================================================================================
@@ -718,44 +728,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsBThreads, 1)
       if (un.last) {
         if (!mbar_wait(&udone[it & 1], (it >> 1) & 1, abort_flag)) break;
         tc_fence_after();
-        if (un.whole) {
-          const float inv = 1.0f / reinterpret_cast<const float2*>(a.stats_whole)[(size_t)un.b * kAbsQ + qg].y;
-          const size_t zrow = ((size_t)head * a.B + un.b) * a.N + n;
+        // whole example: z / l; partial segment: unnormalised z (merged by abs_merge_kernel)
+        const float inv = un.whole
+                              ? 1.0f / reinterpret_cast<const float2*>(a.stats_whole)[(size_t)un.b * kAbsQ + qg].y
+                              : 1.0f;
+        __nv_bfloat16* dz = un.whole ? a.z_hi + (((size_t)head * a.B + un.b) * a.N + n) * a.d + hf * NC
+                                     : a.part_z + ((size_t)un.slot * kAbsQ + qg) * a.d + hf * NC;
 #pragma unroll 1
-          for (int c = 0; c < NC / 32; ++c) {
-            uint32_t v[32];
-            tmem_ld_32x32b_x32(t0 + c * 32, v);
-            tmem_ld_wait();
-            uint32_t hi[16], lo[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float x0 = __uint_as_float(v[2 * j]) * inv, x1 = __uint_as_float(v[2 * j + 1]) * inv;
-              const __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
-              hi[j] = *reinterpret_cast<const uint32_t*>(&hb);
-              const float2 hf2 = __bfloat1622float2(hb);
-              lo[j] = pack_bf16x2(x0 - hf2.x, x1 - hf2.y);
-            }
-            uint4* dh = reinterpret_cast<uint4*>(a.z_hi + zrow * a.d + hf * NC + c * 32);
-            uint4* dl = reinterpret_cast<uint4*>(a.z_lo + zrow * a.d + hf * NC + c * 32);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              dh[i] = make_uint4(hi[4 * i], hi[4 * i + 1], hi[4 * i + 2], hi[4 * i + 3]);
-              dl[i] = make_uint4(lo[4 * i], lo[4 * i + 1], lo[4 * i + 2], lo[4 * i + 3]);
-            }
-          }
-        } else {
-          float* dz = a.part_z + ((size_t)un.slot * kAbsQ + qg) * a.d + hf * NC;
-#pragma unroll 1
-          for (int c = 0; c < NC / 32; ++c) {
-            uint32_t v[32];
-            tmem_ld_32x32b_x32(t0 + c * 32, v);
-            tmem_ld_wait();
-            float4* d4 = reinterpret_cast<float4*>(dz + c * 32);
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              d4[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                  __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
-          }
+        for (int c = 0; c < NC / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(t0 + c * 32, v);
+          tmem_ld_wait();
+          store_bf16x32(dz + c * 32, v, inv);
         }
         tc_fence_before();
       }
@@ -790,12 +774,8 @@ __global__ void __launch_bounds__(256) abs_merge_kernel(const AbsArgs a) {
   const int head = q / a.N, n = q % a.N;
   const size_t zrow = ((size_t)head * a.B + b) * a.N + n;
   uint2* zh = reinterpret_cast<uint2*>(a.z_hi + zrow * a.d);
-  uint2* zl = reinterpret_cast<uint2*>(a.z_lo + zrow * a.d);
   if (ub >= ub1) {  // empty history: the attention output is the empty sum
-    for (int c = lane; c < a.d / 4; c += 32) {
-      zh[c] = make_uint2(0u, 0u);
-      zl[c] = make_uint2(0u, 0u);
-    }
+    for (int c = lane; c < a.d / 4; c += 32) zh[c] = make_uint2(0u, 0u);
     return;
   }
   const int P = a.n_pairs;
@@ -832,17 +812,15 @@ __global__ void __launch_bounds__(256) abs_merge_kernel(const AbsArgs a) {
       const int slot = s_slot[warp][j];
       if (slot < 0) continue;
       const float w = s_w[warp][j];
-      const float4 z = __ldcg(reinterpret_cast<const float4*>(a.part_z + ((size_t)slot * kAbsQ + q) * a.d) + c);
-      acc.x = fmaf(w, z.x, acc.x);
-      acc.y = fmaf(w, z.y, acc.y);
-      acc.z = fmaf(w, z.z, acc.z);
-      acc.w = fmaf(w, z.w, acc.w);
+      const uint2 zb = __ldcg(reinterpret_cast<const uint2*>(a.part_z + ((size_t)slot * kAbsQ + q) * a.d) + c);
+      const float2 z01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&zb.x));
+      const float2 z23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&zb.y));
+      acc.x = fmaf(w, z01.x, acc.x);
+      acc.y = fmaf(w, z01.y, acc.y);
+      acc.z = fmaf(w, z23.x, acc.z);
+      acc.w = fmaf(w, z23.y, acc.w);
     }
-    const float x[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
-    const __nv_bfloat162 h0 = __floats2bfloat162_rn(x[0], x[1]), h1 = __floats2bfloat162_rn(x[2], x[3]);
-    const float2 f0 = __bfloat1622float2(h0), f1 = __bfloat1622float2(h1);
-    zh[c] = make_uint2(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1));
-    zl[c] = make_uint2(pack_bf16x2(x[0] - f0.x, x[1] - f0.y), pack_bf16x2(x[2] - f1.x, x[3] - f1.y));
+    zh[c] = make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
   }
 }
 

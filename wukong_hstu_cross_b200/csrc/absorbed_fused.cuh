@@ -711,44 +711,15 @@ __device__ __forceinline__ void fu_value(uint8_t* smem, uint32_t rank, int cl, c
         }
         ++nseg;
         tc_fence_after();
-        if (un.whole) {
-          const float inv = 1.0f / lsg;
-          const size_t zrow = ((size_t)head * a.B + un.b) * a.N + n;
+        const float inv = un.whole ? 1.0f / lsg : 1.0f;
+        __nv_bfloat16* dz = un.whole ? a.z_hi + (((size_t)head * a.B + un.b) * a.N + n) * a.d + hf * NC
+                                     : a.part_z + ((size_t)un.slot * kAbsQ + qg) * a.d + hf * NC;
 #pragma unroll 1
-          for (int c = 0; c < NC / 32; ++c) {
-            uint32_t v[32];
-            tmem_ld_32x32b_x32(t0 + c * 32, v);
-            tmem_ld_wait();
-            uint32_t hi[16], lo[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float x0 = __uint_as_float(v[2 * j]) * inv, x1 = __uint_as_float(v[2 * j + 1]) * inv;
-              const __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
-              hi[j] = *reinterpret_cast<const uint32_t*>(&hb);
-              const float2 hf2 = __bfloat1622float2(hb);
-              lo[j] = pack_bf16x2(x0 - hf2.x, x1 - hf2.y);
-            }
-            uint4* dh = reinterpret_cast<uint4*>(a.z_hi + zrow * a.d + hf * NC + c * 32);
-            uint4* dl = reinterpret_cast<uint4*>(a.z_lo + zrow * a.d + hf * NC + c * 32);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              dh[i] = make_uint4(hi[4 * i], hi[4 * i + 1], hi[4 * i + 2], hi[4 * i + 3]);
-              dl[i] = make_uint4(lo[4 * i], lo[4 * i + 1], lo[4 * i + 2], lo[4 * i + 3]);
-            }
-          }
-        } else {
-          float* dz = a.part_z + ((size_t)un.slot * kAbsQ + qg) * a.d + hf * NC;
-#pragma unroll 1
-          for (int c = 0; c < NC / 32; ++c) {
-            uint32_t v[32];
-            tmem_ld_32x32b_x32(t0 + c * 32, v);
-            tmem_ld_wait();
-            float4* d4 = reinterpret_cast<float4*>(dz + c * 32);
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              d4[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                  __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
-          }
+        for (int c = 0; c < NC / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(t0 + c * 32, v);
+          tmem_ld_wait();
+          store_bf16x32(dz + c * 32, v, inv);
         }
         tc_fence_before();
       }

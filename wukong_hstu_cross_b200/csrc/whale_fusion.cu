@@ -24,6 +24,7 @@
 #include <functional>
 #include <utility>
 #include <mutex>
+#include <vector>
 
 #include "absorbed.cuh"
 #include "absorbed_fused.cuh"
@@ -90,9 +91,44 @@ inline bool pdl_enabled() {
   return !(e && e[0] == '1');
 }
 
+// Per-kernel timing (whale_profile_begin / whale_profile_end): while on, every kernel launched by
+// launch_pdl is followed by an event on its stream (the first one also by a start event). The
+// events serialise the launches (no overlap of a kernel's prologue with its predecessor's tail).
+struct ProfRec {
+  const void* fn;
+  cudaEvent_t ev;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+int g_prof_cap = 0;
+cudaEvent_t g_prof_start = nullptr;
+std::vector<ProfRec> g_prof;
+
+inline void prof_record(const void* fn, cudaStream_t st, bool before) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (!g_prof_on) return;
+  if (before) {
+    if (!g_prof_start && cudaEventCreate(&g_prof_start) == cudaSuccess) cudaEventRecord(g_prof_start, st);
+    return;
+  }
+  if ((int)g_prof.size() >= g_prof_cap) return;
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return;
+  cudaEventRecord(e, st);
+  g_prof.push_back({fn, e});
+}
+
 template <typename... KArgs, typename... Args>
 whale_status launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                         Args&&... args) {
+  if (g_prof_on) prof_record(reinterpret_cast<const void*>(kern), st, true);
+  struct After {
+    const void* fn;
+    cudaStream_t st;
+    ~After() {
+      if (g_prof_on) prof_record(fn, st, false);
+    }
+  } after{reinterpret_cast<const void*>(kern), st};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -244,7 +280,7 @@ struct Layout {
   size_t a_lo, g_lo, f_lo, u_lo, f32, x32[2], xhi[2], xlo[2];
   // absorbed attention: folded key weights, absorbed queries, weights pw, unit references,
   // segment statistics, partial z, unit starts, z as a bf16 pair
-  size_t wkabs, qa, pw, mref, stw, stp, pz, ust, zh, zl;
+  size_t wkabs, qa, pw, mref, stw, stp, pz, ust, zh;
   long long units_max;
   size_t total;
 };
@@ -285,10 +321,9 @@ Layout make_layout(const Shape& s, const whale_shape_hint& hint) {
     L.mref = take((size_t)L.units_max * kAbsQ * 4);
     L.stw = take((size_t)hint.B * kAbsQ * 8);
     L.stp = take((size_t)2 * kMaxPairs * kAbsQ * 8);
-    L.pz = take((size_t)2 * kMaxPairs * kAbsQ * s.d * 4);
+    L.pz = take((size_t)2 * kMaxPairs * kAbsQ * s.d * 2);
     L.ust = take(((size_t)hint.B + 1) * 4);
     L.zh = take((size_t)hint.B * kAbsQ * s.d * 2);
-    L.zl = take((size_t)hint.B * kAbsQ * s.d * 2);
   }
   L.a = take(rows * s.d * s.es);
   L.g = take(rows * (size_t)s.Fh * s.es);
@@ -751,16 +786,14 @@ whale_status gemm_qabs(const Shape& s, const void* q, const void* wkabs, void* q
   return launch_gemm_t<BN, EPI_QABS, false, false>(maps, g, tiles, st);
 }
 
-// A[:, j*64 : j*64 + 64] = z_j W'_V,j^T for every head j in one launch: z is the stack
-// [h, rows, d] (bf16 pair), W'_V the gain-folded [d, d] value weights (row j*64 + c).
-whale_status gemm_vabs(const Shape& s, const void* zh, const void* zl, const void* wv, void* a, void* a_lo,
-                       long long rows, cudaStream_t st) {
+// A[:, j*64 : j*64 + 64] = z_j W'_V,j^T for every head j in one launch: z is the stack [h, rows, d]
+// (bf16), W'_V the gain-folded [d, d] value weights (row j*64 + c); A as a bf16 pair.
+whale_status gemm_vabs(const Shape& s, const void* zh, const void* wv, void* a, void* a_lo, long long rows,
+                       cudaStream_t st) {
   if (s.dh != 64) return WHALE_ERR_UNSUPPORTED;
   CUtensorMap maps[5];
   WCHECK(tmap_bf16(&maps[0], zh, (long long)s.h * rows, s.d, s.d, 128));
-  WCHECK(tmap_bf16(&maps[1], zl, (long long)s.h * rows, s.d, s.d, 128));
-  maps[2] = maps[0];
-  maps[3] = maps[1];
+  maps[1] = maps[2] = maps[3] = maps[0];
   WCHECK(tmap_bf16(&maps[4], wv, s.d, s.d, s.d, 64));
   GemmArgs g{};
   g.M = (int)rows;
@@ -776,7 +809,7 @@ whale_status gemm_vabs(const Shape& s, const void* zh, const void* zl, const voi
   g.head_tiles = 1;
   g.a_kb_step = 0;
   g.a_row_step = rows;
-  return launch_gemm_t<64, EPI_STORE, false, true>(maps, g, tiles, st);
+  return launch_gemm_t<64, EPI_STORE, false, false>(maps, g, tiles, st);
 }
 
 // Unit starts of the batch (once per forward: the offsets are shared by every layer).
@@ -808,9 +841,8 @@ whale_status attention_absorbed(const Shape& s, const void* q, const void* slab,
   a.mref = reinterpret_cast<float*>(at(ws, L.mref));
   a.stats_whole = reinterpret_cast<float*>(at(ws, L.stw));
   a.stats_part = reinterpret_cast<float*>(at(ws, L.stp));
-  a.part_z = reinterpret_cast<float*>(at(ws, L.pz));
+  a.part_z = reinterpret_cast<__nv_bfloat16*>(at(ws, L.pz));
   a.z_hi = reinterpret_cast<__nv_bfloat16*>(at(ws, L.zh));
-  a.z_lo = reinterpret_cast<__nv_bfloat16*>(at(ws, L.zl));
   if (abs_fused_enabled()) {
     int clusters = 0;
     WCHECK(abs_max_clusters(E, &clusters));
@@ -828,7 +860,7 @@ whale_status attention_absorbed(const Shape& s, const void* q, const void* slab,
                           th64, a));
     }
     WCHECK(launch_pdl(abs_merge_kernel, dim3(hint.B, kAbsQ / 8), dim3(256), 0, st, a));
-    return gemm_vabs(s, at(ws, L.zh), at(ws, L.zl), wv, out, out_lo, rows, st);
+    return gemm_vabs(s, at(ws, L.zh), wv, out, out_lo, rows, st);
   }
   int pairs = 0;
   WCHECK(abs_max_pairs(E, &pairs));
@@ -857,7 +889,7 @@ whale_status attention_absorbed(const Shape& s, const void* q, const void* slab,
     }
   }
   WCHECK(launch_pdl(abs_merge_kernel, dim3(hint.B, kAbsQ / 8), dim3(256), 0, st, a));
-  return gemm_vabs(s, at(ws, L.zh), at(ws, L.zl), wv, out, out_lo, rows, st);
+  return gemm_vabs(s, at(ws, L.zh), wv, out, out_lo, rows, st);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -1139,6 +1171,48 @@ size_t host_staging_bytes(const Shape& s, const whale_shape_hint& h, size_t* o_t
 // C ABI
 // ============================================================================================
 extern "C" {
+
+whale_status whale_profile_begin(int max_kernels) {
+  if (max_kernels <= 0) return WHALE_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (auto& r : g_prof) cudaEventDestroy(r.ev);
+  g_prof.clear();
+  if (g_prof_start) cudaEventDestroy(g_prof_start);
+  g_prof_start = nullptr;
+  g_prof_cap = max_kernels;
+  g_prof_on = true;
+  return WHALE_OK;
+}
+
+whale_status whale_profile_end(whale_kernel_time* out, int capacity, int* count) {
+  if (!count || (capacity > 0 && !out)) return WHALE_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_on = false;
+  whale_status st = WHALE_OK;
+  int n = 0;
+  if (!g_prof.empty() && g_prof_start) {
+    if (cudaEventSynchronize(g_prof.back().ev) != cudaSuccess) st = WHALE_ERR_CUDA;
+    cudaEvent_t prev = g_prof_start;
+    for (const auto& r : g_prof) {
+      float ms = 0.f;
+      if (st == WHALE_OK && cudaEventElapsedTime(&ms, prev, r.ev) != cudaSuccess) st = WHALE_ERR_CUDA;
+      if (n < capacity) {
+        const char* name = nullptr;
+        if (cudaFuncGetName(&name, r.fn) != cudaSuccess) name = "?";
+        out[n] = whale_kernel_time{name, ms};
+      }
+      ++n;
+      prev = r.ev;
+    }
+  }
+  for (auto& r : g_prof) cudaEventDestroy(r.ev);
+  g_prof.clear();
+  if (g_prof_start) cudaEventDestroy(g_prof_start);
+  g_prof_start = nullptr;
+  (void)cudaGetLastError();
+  *count = n;
+  return st;
+}
 
 const char* whale_status_string(whale_status s) {
   switch (s) {

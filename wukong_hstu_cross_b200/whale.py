@@ -41,6 +41,10 @@ class whale_shape_hint(ctypes.Structure):
     _fields_ = [("B", c_int), ("max_L", c_int), ("total_L", c_longlong)]
 
 
+class whale_kernel_time(ctypes.Structure):
+    _fields_ = [("kernel", ctypes.c_char_p), ("ms", c_float)]
+
+
 class WhaleError(RuntimeError):
     def __init__(self, status: int, where: str):
         super().__init__(f"{where}: {STATUS.get(status, status)}")
@@ -54,6 +58,8 @@ _lib = ctypes.CDLL(LIB_PATH)
 _P = c_void_p
 _SIGS = {
     "whale_status_string": ([c_int], ctypes.c_char_p),
+    "whale_profile_begin": ([c_int], c_int),
+    "whale_profile_end": ([POINTER(whale_kernel_time), c_int, POINTER(c_int)], c_int),
     "whale_workspace_size": ([POINTER(whale_config), POINTER(whale_shape_hint)], c_size_t),
     "whale_host_workspace_size": ([POINTER(whale_config), POINTER(whale_shape_hint)], c_size_t),
     "whale_fusion_forward": ([POINTER(whale_config), _P, _P, _P, POINTER(whale_layer_weights), _P,
@@ -270,6 +276,18 @@ def whale_swiglu_ffn(cfg, rows, f, g_ffn, w_upgate, w_down, y, workspace, worksp
     if raw:
         return st
     _check(st, "whale_swiglu_ffn")
+
+
+def whale_profile_begin(max_kernels: int = 4096) -> None:
+    _check(_lib.whale_profile_begin(max_kernels), "whale_profile_begin")
+
+
+def whale_profile_end(capacity: int = 4096) -> list:
+    """[(kernel name, ms), ...] in launch order (see include/whale_fusion.h)."""
+    buf = (whale_kernel_time * capacity)()
+    n = c_int(0)
+    _check(_lib.whale_profile_end(buf, capacity, ctypes.byref(n)), "whale_profile_end")
+    return [((buf[i].kernel or b"?").decode(), float(buf[i].ms)) for i in range(min(n.value, capacity))]
 
 
 def whale_get_device_error(stream=None) -> int:
