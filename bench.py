@@ -38,12 +38,13 @@ METRIC = "WHALE fusion-layer examples/s @15k jagged history; % of HBM/TC rooflin
 KV_TRAFFIC_BYTES_PER_ROW_D512 = {"2sm": (113.378816e6 + 169.603840e6) / 109605,
                                  "1sm": (113.375488e6 + 168.328960e6) / 109605}
 
-# DRAM bytes per history row of one whale_attend_states call (qa GEMM, pass A, pass B, merge, W_V
-# GEMM, unit starts): one ncu capture of the six kernels at d = 512 on the full 403 481-row batch
-# (1167.7 MB read + 209.7 MB written per call). Two-kernel path only (the default).
-ABS_TRAFFIC_BYTES_PER_ROW_D512 = (1167.7e6 + 209.7e6) / 403481
-# ... and of its pass A kernel alone (abs_scores_kernel: 441.23 MB read + 174.07 MB written)
+# DRAM bytes per history row of the absorbed path's pass A kernel (abs_scores_kernel): one ncu
+# capture at d = 512 on the full 403 481-row batch (441.23 MB read + 174.07 MB written per launch).
+# Two-kernel path only (the default).
 ABS_PASSA_BYTES_PER_ROW_D512 = (441.23e6 + 174.07e6) / 403481
+# ... and of a whole whale_attend_states call (its six kernels); None until captured for the
+# current pass B, merge and W_V GEMM (single-bf16 z)
+ABS_TRAFFIC_BYTES_PER_ROW_D512 = None
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
 
@@ -440,7 +441,8 @@ def main():
         t_abs = timed(absorbed_step, reps)
         abs_tflops = work["attention_absorbed"]["flops"] / (t_abs * 1e-3) / 1e12
         abs_traffic = None
-        if w.d == 512 and not args.shared_kv and os.environ.get("WHALE_ABS_FUSED", "0") != "1":
+        passa_traffic_known = w.d == 512 and not args.shared_kv and os.environ.get("WHALE_ABS_FUSED", "0") != "1"
+        if passa_traffic_known and ABS_TRAFFIC_BYTES_PER_ROW_D512 is not None:
             abs_traffic = ABS_TRAFFIC_BYTES_PER_ROW_D512 * total_L
         call = {"entry_point": "whale_attend_states (qa GEMM, pass A, pass B, merge, W_V GEMM, unit starts)",
                 "tflops": abs_tflops, "frac": abs_tflops / peaks["bf16_tflops"], "avg_call_ms": t_abs,
@@ -454,7 +456,7 @@ def main():
             fa = 2.0 * w.n_tokens * w.n_heads * total_L * w.d
             ta = pa["avg_ms"]
             a_tflops = fa / (ta * 1e-3) / 1e12
-            a_traffic = (ABS_PASSA_BYTES_PER_ROW_D512 * total_L) if abs_traffic is not None else None
+            a_traffic = (ABS_PASSA_BYTES_PER_ROW_D512 * total_L) if passa_traffic_known else None
             roof = {"kernel": "abs_scores_kernel (absorbed pass A: scores on tcgen05 2-SM, online softmax, weights)",
                     "bound": "tensor", "achieved": a_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                     "frac": a_tflops / peaks["bf16_tflops"], "traffic": a_traffic,
