@@ -219,6 +219,35 @@ def test_swiglu_ffn(rows, d, tied):
     assert_parity(y, O.swiglu_ffn(f, g, wug, wd, 1e-6, tied_gate=tied), "bf16", rms_rel=1e-2, what="Y")
 
 
+@pytest.mark.parametrize("which,rows,d", [("fusion", 1000, 512), ("ffn", 1000, 512), ("ffn", 2000, 512),
+                                           ("ffn", 300, 256)])
+def test_residual_gemms_split_k(which, rows, d, monkeypatch):
+    """The split-K residual GEMM (clusters of 4 or 8 CTAs summing their K ranges through
+    distributed shared memory), enabled with WHALE_GEMM_SPLITK=1, on ragged row counts: Fusion
+    GEMM 2 (K = 2d) and the down projection (K = 4d)."""
+    monkeypatch.setenv("WHALE_GEMM_SPLITK", "1")
+    rng = np.random.default_rng(rows + d + len(which))
+    f = bf16_randn(rng, rows, d)
+    cfg = _cfg(d, d // 64)
+    out = torch.empty(rows, d, dtype=torch.bfloat16, device=DEV)
+    if which == "fusion":
+        x = bf16_randn(rng, rows, d)
+        w1 = I.bf16_round(I.xavier_uniform(rng, 2 * d, 2 * d))
+        w2 = I.bf16_round(I.xavier_uniform(rng, d, 2 * d))
+        cfg = _cfg(d, d // 64, Fh=2 * d)
+        W.whale_fusion_mlp(cfg, rows, _t(f), _t(x), _t(w1), _t(w2), out, _ws(64 << 20))
+        ref = O.fusion_mlp(f, x, w1, w2)
+    else:
+        H = 4 * d
+        g = rng.uniform(0.5, 1.5, d).astype(np.float32)
+        wug = np.concatenate([I.bf16_round(I.xavier_uniform(rng, H, d)), I.bf16_round(I.xavier_uniform(rng, H, d))])
+        wd = I.bf16_round(I.xavier_uniform(rng, d, H))
+        W.whale_swiglu_ffn(cfg, rows, _t(f), _g(g), _t(wug), _t(wd), out, _ws(64 << 20))
+        ref = O.swiglu_ffn(f, g, wug, wd, 1e-6)
+    torch.cuda.synchronize()
+    assert_parity(out, ref, "bf16", rms_rel=1e-2, what=which)
+
+
 def test_project_kv_one_and_two_sm_kernels():
     """Both persistent K|V GEMMs on a ragged large M: the 2-SM (cta_group::2) default and the
     one-SM kernel selected with WHALE_GEMM_1SM=1; they must agree bitwise (same fp32 sums)."""

@@ -72,6 +72,13 @@ inline bool qtile_enabled() {
   const char* e = std::getenv("WHALE_ATTN_SPLITL");
   return !(e && e[0] == '1');
 }
+// WHALE_GEMM_SPLITK=1 in the environment runs the residual-epilogue GEMMs with a long K split-K
+// across a cluster (gemm_splitk_kernel). Off by default: on the 2048-row token batch it measured
+// slower than one CTA per 128 x 64 tile (3.45-3.50 against 3.39-3.41 ms per 8-layer step).
+inline bool splitk_enabled() {
+  const char* e = std::getenv("WHALE_GEMM_SPLITK");
+  return e && e[0] == '1';
+}
 inline bool abs_fused_enabled() {
   const char* e = std::getenv("WHALE_ABS_FUSED");
   return e && e[0] == '1';
@@ -116,6 +123,31 @@ inline void prof_record(const void* fn, cudaStream_t st, bool before) {
   if (cudaEventCreate(&e) != cudaSuccess) return;
   cudaEventRecord(e, st);
   g_prof.push_back({fn, e});
+}
+
+// The same with a cluster shape given at launch (kernels without __cluster_dims__).
+template <typename... KArgs, typename... Args>
+whale_status launch_cluster_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                unsigned cluster_x, Args&&... args) {
+  if (g_prof_on) prof_record(reinterpret_cast<const void*>(kern), st, true);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cluster_x;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+  if (g_prof_on) prof_record(reinterpret_cast<const void*>(kern), st, false);
+  CUCHECK(e);
+  return WHALE_OK;
 }
 
 template <typename... KArgs, typename... Args>
@@ -488,6 +520,46 @@ whale_status gemm_bf16(const Opnd& a0, const Opnd& a1, const void* W, int N, con
     if (N % 256 == 0 && gemm_2sm_enabled()) WCHECK(g2_max_pairs(&pairs));
     if (pairs > 0) return gemm_rownorm_2sm(a0, W, N, out, M, eps, pairs, st);
     return gemm_rownorm_persistent(a0, W, N, out, M, eps, st);
+  }
+  // Residual epilogue, one hi/lo source, long K: split-K across a cluster of KS CTAs per 128 x 256 tile.
+  if (epi == EPI_RESID && split && a1.K == 0 && !rn && N % 256 == 0 && splitk_enabled()) {
+    const int KBs = a0.K / 64;
+    const long long tiles = tm * (N / 256);
+    int ks = 1;
+    for (int c : {2, 4, 8})
+      if (KBs % c == 0 && KBs / c >= 4 && tiles * c <= kNumSM) ks = c;
+    if (ks > 1) {
+      CUtensorMap ta, tl, tb;
+      WCHECK(tmap_bf16(&ta, a0.hi, M, a0.K, a0.ld, 128));
+      WCHECK(tmap_bf16(&tl, a0.lo, M, a0.K, a0.ld, 128));
+      WCHECK(tmap_bf16(&tb, W, N, a0.K, a0.K, 256));
+      GemmArgs g{};
+      g.M = (int)M;
+      g.N = N;
+      g.kb0 = KBs;
+      g.tiles_n = N / 256;
+      g.num_tiles = (int)tiles;
+      g.out_hi = static_cast<__nv_bfloat16*>(out.hi);
+      g.out_lo = static_cast<__nv_bfloat16*>(out.lo);
+      g.out32 = out.f32;
+      g.ldo = out.ld;
+      g.resid32 = resid32;
+      g.ldr = ldr;
+      const dim3 grid((unsigned)(tiles * ks));
+      if (ks == 2) {
+        CUCHECK(cudaFuncSetAttribute(gemm_splitk_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)SplitKSmem::BYTES));
+        return launch_cluster_pdl(gemm_splitk_kernel<2>, grid, dim3(192), SplitKSmem::BYTES, st, 2u, ta, tl, tb, g);
+      }
+      if (ks == 4) {
+        CUCHECK(cudaFuncSetAttribute(gemm_splitk_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)SplitKSmem::BYTES));
+        return launch_cluster_pdl(gemm_splitk_kernel<4>, grid, dim3(192), SplitKSmem::BYTES, st, 4u, ta, tl, tb, g);
+      }
+      CUCHECK(cudaFuncSetAttribute(gemm_splitk_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)SplitKSmem::BYTES));
+      return launch_cluster_pdl(gemm_splitk_kernel<8>, grid, dim3(192), SplitKSmem::BYTES, st, 8u, ta, tl, tb, g);
+    }
   }
   // Tile width by a small cost model (cycles): per-CTA fixed cost + tiles per persistent CTA x
   // (per 64-deep K block the larger of the MMA time and the operand bytes at ~80 B/clk, the rate
