@@ -169,31 +169,47 @@ __global__ void __launch_bounds__(1024) abs_units_kernel(const int* __restrict__
 // ================================================================================================
 // pass A: S = qa H^T, online softmax, pw = p * r
 // ================================================================================================
+// Columns of one weight store (the staging tile of an epilogue warp is 32 queries x kAbsEpiCols):
+// 64 (128-byte rows, 128-byte swizzle) or 32 (64-byte rows, 64-byte swizzle; half the staging
+// memory, one more stage of history rows at d = 512, twice the stores and proxy fences).
+constexpr int kAbsEpiCols = 32;
+
+template <int E>  // d = 256 E
 struct AbsASmem {
   static constexpr int BK = 64;
-  static constexpr uint32_t A_BYTES = 128 * BK * 2;   // 128 absorbed queries (this CTA's)
-  static constexpr uint32_t B_BYTES = 128 * BK * 2;   // this CTA's 128 history rows of the unit
-  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr uint32_t EPI_BYTES = 8 * 4096;     // one 32 x 64 bf16 staging tile per epilogue warp
+  static constexpr int KB = 4 * E;                     // 64-column blocks of d
+  static constexpr uint32_t BLK_BYTES = 128 * BK * 2;  // 128 rows x 64 columns
+  static constexpr uint32_t QA_BYTES = KB * BLK_BYTES; // this CTA's 128 absorbed queries, all of d
+  static constexpr uint32_t STAGE_BYTES = BLK_BYTES;   // this CTA's 128 history rows, one column block
+  static constexpr uint32_t EPI_WARP = 32 * kAbsEpiCols * 2;
+  static constexpr uint32_t EPI_BYTES = 8 * EPI_WARP;
   static constexpr int XCH = 2 * 256 * 4 + 2 * 2 * 128 * 4 + 2 * 128 * 4;  // r[2][256], max[2][2][128], l[2][128]
-  static constexpr int FIXED = 1024 + EPI_BYTES + XCH + 512;
+  static constexpr int FIXED = 1024 + QA_BYTES + EPI_BYTES + XCH + 512;
   static constexpr int STAGES = (232448 - FIXED) / (int)STAGE_BYTES > 8 ? 8 : (232448 - FIXED) / (int)STAGE_BYTES;
   static constexpr size_t BYTES = FIXED + STAGES * (size_t)STAGE_BYTES;
+  static_assert(STAGES >= 3, "at least three stages of history rows");
 };
 constexpr int kAbsAThreads = 480;
 
+// The absorbed queries of the example (the MMA's A operand, 128 per CTA) stay resident in shared
+// memory for the pair's whole segment of that example: the stage ring carries history rows only,
+// which halves the operand bytes streamed per MMA (TMA ingest bounds the loop, not the tensor pipe).
 // warps: 0 TMA producer (both CTAs), 1 TMEM (2 x 256 columns) + MMA issue (even CTA), 2..9 softmax
 // epilogue (two warps per lane quadrant, 128 columns each), 10..13 row statistics of this CTA's 128
 // history rows (r of all 256 columns reaches both CTAs through distributed shared memory), 14 relay
 // of "stage landed" (even CTA) as in the 2-SM projection GEMM.
+template <int E>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
     abs_scores_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmH,
                       const __grid_constant__ CUtensorMap tmP, const AbsArgs a) {
-  using L = AbsASmem;
+  using L = AbsASmem<E>;
   constexpr int ST = L::STAGES;
+  constexpr int KB = L::KB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* epi = smem + ST * L::STAGE_BYTES;
+  uint8_t* qsm = smem;                      // [KB][128 queries][64 columns], 128-byte swizzle
+  uint8_t* stages = smem + L::QA_BYTES;     // [ST][128 history rows][64 columns]
+  uint8_t* epi = stages + ST * L::STAGE_BYTES;
   float* rbuf = reinterpret_cast<float*>(epi + L::EPI_BYTES);  // [2][256]
   float* xmax = rbuf + 2 * 256;                                // [2 acc][2 half][128]
   float* xsum = xmax + 2 * 2 * 128;                            // [2 half][128]
@@ -206,14 +222,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
   uint64_t* edone = nfull + 2;    // [2] 8 local + 8 peer epilogue warps
   uint64_t* xbar = edone + 2;     // [4 quadrants][2 acc] tile maxima of both half-warps written
   uint64_t* lbar = xbar + 8;      // [4 quadrants] segment sums of both half-warps written
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lbar + 4);
+  uint64_t* qfull = lbar + 4;     // the segment's queries landed (both CTAs' copies, even CTA)
+  uint64_t* qempty = qfull + 1;   // the segment's last MMAs are done (commit to both CTAs)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qempty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1;
-  const int KB = a.d / 64;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < ST; ++s) {
@@ -221,6 +238,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
       mbar_init(&ready[s], 1);
       mbar_init(&empty[s], 1 + 4);
     }
+    mbar_init(qfull, 1);
+    mbar_init(qempty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], 16);
@@ -256,11 +275,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
   if (warp == 0) {
     // ---------------- TMA producer (both CTAs) ----------------
     if (lane == 0) {
-      int kg = 0;
+      int kg = 0, nseg = 0;
       bool stop = false;
+      const uint32_t qbar = mapa_shared(smem_u32(qfull), 0);
       for (; wk.valid() && !stop; wk.next(a)) {
         const AbsUnit un = abs_unit(a, wk);
-        const int qrow = un.b * kAbsQ + (int)rank * 128;
+        if (un.first) {
+          // a new segment: its queries replace the previous segment's once those MMAs are done
+          if (nseg > 0 && !mbar_wait(qempty, (nseg - 1) & 1, abort_flag)) break;
+          if (leader) mbar_arrive_expect_tx(qfull, 2 * L::QA_BYTES);
+          const int qrow = un.b * kAbsQ + (int)rank * 128;
+#pragma unroll
+          for (int kb = 0; kb < KB; ++kb) tma_load_2d_cg2(qsm + kb * L::BLK_BYTES, &tmQ, kb * L::BK, qrow, qbar);
+          ++nseg;
+        }
         const int hrow = (int)un.row0 + (int)rank * 128;
         for (int kb = 0; kb < KB; ++kb, ++kg) {
           const int s = kg % ST, u = kg / ST;
@@ -268,11 +296,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
             stop = true;
             break;
           }
-          uint8_t* st = smem + s * L::STAGE_BYTES;
           const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
           if (leader) mbar_arrive_expect_tx(&full[s], 2 * L::STAGE_BYTES);
-          tma_load_2d_cg2(st, &tmQ, kb * L::BK, qrow, bar);
-          tma_load_2d_cg2(st + L::A_BYTES, &tmH, kb * L::BK, hrow, bar);
+          tma_load_2d_cg2(stages + s * L::STAGE_BYTES, &tmH, kb * L::BK, hrow, bar);
         }
       }
     }
@@ -280,10 +306,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
     // ---------------- MMA issuer (even CTA) ----------------
     if (leader && lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(256, 256);
-      int kg = 0, it = 0;
+      int kg = 0, it = 0, nseg = 0;
       bool stop = false;
       for (; wk.valid() && !stop; wk.next(a), ++it) {
+        const AbsUnit un = abs_unit(a, wk);
         const int acc = it & 1, ua = it >> 1;
+        if (un.first) {
+          if (!mbar_wait(qfull, nseg & 1, abort_flag)) break;
+          ++nseg;
+        }
         if (it >= 2 && !mbar_wait(&tempty[acc], (ua - 1) & 1, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * 256;
@@ -294,8 +325,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a_base = smem_u32(smem + s * L::STAGE_BYTES);
-          const uint32_t b_base = a_base + L::A_BYTES;
+          const uint32_t a_base = smem_u32(qsm + kb * L::BLK_BYTES);
+          const uint32_t b_base = smem_u32(stages + s * L::STAGE_BYTES);
 #pragma unroll
           for (int kk = 0; kk < L::BK / 16; ++kk)
             umma_f16_cg2(d_tmem, sdesc_k_sw128(a_base + kk * 32), sdesc_k_sw128(b_base + kk * 32), idesc,
@@ -303,6 +334,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
           umma_commit_cg2_mc(&empty[s], 0x3);
         }
         umma_commit_cg2_mc(&tfull[acc], 0x3);
+        if (un.last) umma_commit_cg2_mc(qempty, 0x3);  // also on abort: arrives once issued MMAs are done
       }
     }
   } else if (warp == 14) {
@@ -333,7 +365,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
           ok = false;
           break;
         }
-        const uint4* rp = reinterpret_cast<const uint4*>(smem + s * L::STAGE_BYTES + L::A_BYTES + row * 128);
+        const uint4* rp = reinterpret_cast<const uint4*>(stages + s * L::STAGE_BYTES + row * 128);
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           float f[8];
@@ -369,7 +401,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
     const int hf = (warp - 2) >> 2;  // columns [128 hf, 128 hf + 128) of the unit
     const int row = qd * 32 + lane;
     const int qg = (int)rank * 128 + row;
-    uint8_t* sbuf = epi + (warp - 2) * 4096;
+    uint8_t* sbuf = epi + (warp - 2) * L::EPI_WARP;
     const uint32_t tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
     const uint32_t edone_peer0 = mapa_shared(smem_u32(&edone[0]), rank ^ 1);
 
@@ -402,17 +434,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
       return mx;
     };
     // p = 2^(r s - m) over the valid columns (0 elsewhere): returns the local maximum of r s, adds
-    // sum(p) to lsum, and stores pw = p * r (bf16) through the staging tile, one 64-column tile
-    // of the tiled weight layout per store.
+    // sum(p) to lsum, and stores pw = p * r (bf16) through the staging tile into the 64-column
+    // tiles of the tiled weight layout (kAbsEpiCols columns per store).
     auto write_weights = [&](uint32_t t0, const float* r, int nv, float m, float& lsum, int tile_row0) -> float {
       float mx = -INFINITY;
 #pragma unroll 1
       for (int cc = 0; cc < 2; ++cc) {
-        if (lane == 0) bulk_wait_read<0>();  // the previous store from this buffer has read it
-        __syncwarp();
-        uint4* dst = reinterpret_cast<uint4*>(sbuf + lane * 128);
 #pragma unroll 1
         for (int h2 = 0; h2 < 2; ++h2) {
+          if (kAbsEpiCols == 32 || h2 == 0) {
+            if (lane == 0) bulk_wait_read<0>();  // the previous store from this buffer has read it
+            __syncwarp();
+          }
           const int c0 = cc * 64 + h2 * 32;
           uint32_t v[32];
           tmem_ld_32x32b_x32(t0 + c0, v);
@@ -444,14 +477,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
             pk.y = pack_bf16x2(w[2], w[3]);
             pk.z = pack_bf16x2(w[4], w[5]);
             pk.w = pack_bf16x2(w[6], w[7]);
-            dst[(h2 * 4 + j8) ^ (lane & 7)] = pk;
+            // row = lane; 16-byte chunk positions follow the store's swizzle (128- or 64-byte)
+            if (kAbsEpiCols == 64)
+              reinterpret_cast<uint4*>(sbuf + lane * 128)[(h2 * 4 + j8) ^ (lane & 7)] = pk;
+            else
+              reinterpret_cast<uint4*>(sbuf + lane * 64)[j8 ^ ((lane >> 1) & 3)] = pk;
           }
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&tmP, sbuf, 0, (tile_row0 + hf * 2 + cc) * kAbsQ + (int)rank * 128 + qd * 32);
-          bulk_commit();
+          if (kAbsEpiCols == 32 || h2 == 1) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmP, sbuf, kAbsEpiCols == 32 ? h2 * 32 : 0,
+                           (tile_row0 + hf * 2 + cc) * kAbsQ + (int)rank * 128 + qd * 32);
+              bulk_commit();
+            }
+          }
         }
       }
       return mx;

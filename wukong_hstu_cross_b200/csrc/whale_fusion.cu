@@ -192,18 +192,27 @@ whale_status get_encoder() {
   return g_encode ? WHALE_OK : WHALE_ERR_CUDA;
 }
 
-// 2-D bf16 row-major tensor [rows, cols] with row stride ld, box [box_rows, 64 columns], 128-B swizzle.
-whale_status tmap_bf16(CUtensorMap* tm, const void* base, long long rows, long long cols, long long ld, int box_rows) {
+// 2-D bf16 row-major tensor [rows, cols] with row stride ld, box [box_rows, box_cols]; the swizzle
+// spans one box row (box_cols 64: 128-byte swizzle, 32: 64-byte swizzle).
+whale_status tmap_bf16_box(CUtensorMap* tm, const void* base, long long rows, long long cols, long long ld,
+                           int box_cols, int box_rows) {
   WCHECK(get_encoder());
   if ((reinterpret_cast<uintptr_t>(base) & 15) || (ld * 2) % 16 || rows <= 0 || cols <= 0) return WHALE_ERR_INVALID_ARG;
+  if (box_cols != 64 && box_cols != 32) return WHALE_ERR_INVALID_ARG;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
-  cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
   cuuint32_t es[2] = {1u, 1u};
   CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                        CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? WHALE_OK : WHALE_ERR_CUDA;
+}
+
+// Box [box_rows, 64 columns], 128-byte swizzle.
+whale_status tmap_bf16(CUtensorMap* tm, const void* base, long long rows, long long cols, long long ld, int box_rows) {
+  return tmap_bf16_box(tm, base, rows, cols, ld, 64, box_rows);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -786,9 +795,13 @@ whale_status abs_max_pairs(int E, int* pairs) {
       return WHALE_OK;
     };
     int na = 0, nb = 0;
-    WCHECK(query(reinterpret_cast<const void*>(abs_scores_kernel), AbsASmem::BYTES, kAbsAThreads, &na));
-    if (E == 1) WCHECK(query(reinterpret_cast<const void*>(abs_values_kernel<1>), AbsBSmem<1>::BYTES, kAbsBThreads, &nb));
-    else WCHECK(query(reinterpret_cast<const void*>(abs_values_kernel<2>), AbsBSmem<2>::BYTES, kAbsBThreads, &nb));
+    if (E == 1) {
+      WCHECK(query(reinterpret_cast<const void*>(abs_scores_kernel<1>), AbsASmem<1>::BYTES, kAbsAThreads, &na));
+      WCHECK(query(reinterpret_cast<const void*>(abs_values_kernel<1>), AbsBSmem<1>::BYTES, kAbsBThreads, &nb));
+    } else {
+      WCHECK(query(reinterpret_cast<const void*>(abs_scores_kernel<2>), AbsASmem<2>::BYTES, kAbsAThreads, &na));
+      WCHECK(query(reinterpret_cast<const void*>(abs_values_kernel<2>), AbsBSmem<2>::BYTES, kAbsBThreads, &nb));
+    }
     const int n = std::min(std::min(na, nb), kMaxPairs);
     c = n > 0 ? n : -1;
   }
@@ -942,9 +955,18 @@ whale_status attention_absorbed(const Shape& s, const void* q, const void* slab,
     WCHECK(tmap_bf16(&tq, at(ws, L.qa), (long long)hint.B * kAbsQ, s.d, s.d, 128));
     WCHECK(tmap_bf16(&th, slab, hint.total_L, s.d, s.d, 128));
     const long long pw_rows = L.units_max * (kAbsRows / 64) * kAbsQ;  // tiled: [4 units_max * 256, 64]
-    WCHECK(tmap_bf16(&tps, at(ws, L.pw), pw_rows, 64, 64, 32));
-    CUCHECK(cudaFuncSetAttribute(abs_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AbsASmem::BYTES));
-    WCHECK(launch_pdl(abs_scores_kernel, dim3(2 * a.n_pairs), dim3(kAbsAThreads), AbsASmem::BYTES, st, tq, th, tps, a));
+    WCHECK(tmap_bf16_box(&tps, at(ws, L.pw), pw_rows, 64, 64, kAbsEpiCols, 32));
+    if (E == 1) {
+      CUCHECK(cudaFuncSetAttribute(abs_scores_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)AbsASmem<1>::BYTES));
+      WCHECK(launch_pdl(abs_scores_kernel<1>, dim3(2 * a.n_pairs), dim3(kAbsAThreads), AbsASmem<1>::BYTES, st, tq, th,
+                        tps, a));
+    } else {
+      CUCHECK(cudaFuncSetAttribute(abs_scores_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)AbsASmem<2>::BYTES));
+      WCHECK(launch_pdl(abs_scores_kernel<2>, dim3(2 * a.n_pairs), dim3(kAbsAThreads), AbsASmem<2>::BYTES, st, tq, th,
+                        tps, a));
+    }
     CUtensorMap tpl, th64;
     WCHECK(tmap_bf16(&tpl, at(ws, L.pw), pw_rows, 64, 64, 128));
     WCHECK(tmap_bf16(&th64, slab, hint.total_L, s.d, s.d, 64));
