@@ -800,6 +800,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsBThreads, 1)
 // ================================================================================================
 // grid (B, 256 / 8), 256 threads: one warp per absorbed query. The lanes first gather the
 // (slot, weight) list of the example's partials (one pair each), then stream the partial z rows.
+// (Four queries per warp, with a quarter of the warps per SM, measured slower.)
 __global__ void __launch_bounds__(256) abs_merge_kernel(const AbsArgs a) {
   pdl_wait();
   pdl_trigger();
@@ -846,21 +847,41 @@ __global__ void __launch_bounds__(256) abs_merge_kernel(const AbsArgs a) {
   for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
   __syncwarp();
   const float inv = 1.0f / l;
-  for (int c = lane; c < a.d / 4; c += 32) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < cnt; ++j) {
-      const int slot = s_slot[warp][j];
-      if (slot < 0) continue;
-      const float w = s_w[warp][j];
-      const uint2 zb = __ldcg(reinterpret_cast<const uint2*>(a.part_z + ((size_t)slot * kAbsQ + q) * a.d) + c);
-      const float2 z01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&zb.x));
-      const float2 z23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&zb.y));
-      acc.x = fmaf(w, z01.x, acc.x);
-      acc.y = fmaf(w, z01.y, acc.y);
-      acc.z = fmaf(w, z23.x, acc.z);
-      acc.w = fmaf(w, z23.y, acc.w);
+  // Lane c holds columns [8c, 8c + 8) and, at d = 512, [256 + 8c, 256 + 8c + 8): one 16-byte
+  // load per chunk and partial, the loads of a partial issued together.
+  const int nch = a.d / 256;
+  float acc[2][8];
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[i][k] = 0.f;
+#pragma unroll 2
+  for (int j = 0; j < cnt; ++j) {
+    const int slot = s_slot[warp][j];
+    const float w = s_w[warp][j];  // 0 for an empty range
+    uint4 v[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+    if (slot >= 0) {
+      const uint4* src = reinterpret_cast<const uint4*>(a.part_z + ((size_t)slot * kAbsQ + q) * a.d);
+      v[0] = __ldcg(src + lane);
+      if (nch == 2) v[1] = __ldcg(src + 32 + lane);
     }
-    zh[c] = make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      if (i >= nch) break;
+      float f[8];
+      bf16x8_to_f32(v[i], f);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) acc[i][k] = fmaf(w, f[k], acc[i][k]);
+    }
+  }
+  uint4* zh16 = reinterpret_cast<uint4*>(a.z_hi + zrow * a.d);
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    if (i >= nch) break;
+    zh16[i * 32 + lane] = make_uint4(pack_bf16x2(acc[i][0] * inv, acc[i][1] * inv),
+                                     pack_bf16x2(acc[i][2] * inv, acc[i][3] * inv),
+                                     pack_bf16x2(acc[i][4] * inv, acc[i][5] * inv),
+                                     pack_bf16x2(acc[i][6] * inv, acc[i][7] * inv));
   }
 }
 

@@ -293,18 +293,29 @@ __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
     // ---------------- epilogue (warps 2..5): thread i of quadrant q owns row 32q + i ----------------
     const int q = warp & 3;
     const int row = q * 32 + lane;
+    // Residual tiles of 64 columns: the row's residual is loaded into registers before the
+    // accumulator is waited for, so its DRAM latency overlaps the MMAs.
+    constexpr bool kPre = EPI == EPI_RESID && BN <= 64;
+    float4 pre[kPre ? BN / 4 : 1];
     int it = 0;
     for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1, ua = it >> 1;
       const int m0 = (tile / args.tiles_n) * L::BM, n0 = (tile % args.tiles_n) * BN;
+      const long long gm = (long long)m0 + row;
+      const bool row_ok = gm < args.M;
+      if (kPre && row_ok) {
+        const float4* rp = reinterpret_cast<const float4*>(args.resid32 + gm * args.ldr + n0);
+#pragma unroll
+        for (int i = 0; i < (kPre ? BN / 4 : 1); ++i)
+          if (n0 + 4 * i < args.N) pre[i] = rp[i];
+      }
       if (!mbar_wait(&tfull[acc], ua & 1, abort_flag)) break;
       if (ROWNORM && !mbar_wait(&nfull[acc], ua & 1, abort_flag)) break;
       tc_fence_after();
       const float r = ROWNORM ? rbuf[acc * 128 + row] : 1.0f;
-      const long long gm = (long long)m0 + row;
-      const bool row_ok = gm < args.M;
       const uint32_t t_row = tmem_base + acc * BN + ((uint32_t)(q * 32) << 16);
-#pragma unroll 1
+      // (fully unrolled for the register-held residual, whose chunks need constant indices)
+#pragma unroll (kPre ? BN / 32 : 1)
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(t_row + c * 32, v);
@@ -324,7 +335,7 @@ __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
             const float4* rp = reinterpret_cast<const float4*>(args.resid32 + gm * args.ldr + col);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-              const float4 t = rp[i];
+              const float4 t = kPre ? pre[(c * 8 + i) % (kPre ? BN / 4 : 1)] : rp[i];
               x[4 * i] += t.x;
               x[4 * i + 1] += t.y;
               x[4 * i + 2] += t.z;
