@@ -27,6 +27,8 @@
 // in slot 2p (the range's first segment) or 2p + 1 (its last).
 #pragma once
 
+#include <type_traits>
+
 #include "gemm_tc.cuh"
 #include "ptx.cuh"
 
@@ -173,6 +175,11 @@ __global__ void __launch_bounds__(1024) abs_units_kernel(const int* __restrict__
 // 64 (128-byte rows, 128-byte swizzle) or 32 (64-byte rows, 64-byte swizzle; half the staging
 // memory, one more stage of history rows at d = 512, twice the stores and proxy fences).
 constexpr int kAbsEpiCols = 32;
+// Pass A prefetches history rows into L2 this many 64-column blocks ahead of its stage loads (one
+// prefetch per load): lookahead beyond what the shared-memory ring holds. 0 disables it.
+constexpr int kAbsPrefetchKb = 4;
+// Pass B: the same, in 64-row chunks (weights tile and this CTA's columns of the history rows).
+constexpr int kAbsBPrefetchCh = 1;
 
 template <int E>  // d = 256 E
 struct AbsASmem {
@@ -278,6 +285,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
       int kg = 0, nseg = 0;
       bool stop = false;
       const uint32_t qbar = mapa_shared(smem_u32(qfull), 0);
+      // prefetch cursor (unit pf, block pkb), kAbsPrefetchKb blocks ahead of the loads
+      AbsWalk pf = wk;
+      int pkb = 0, prow = pf.valid() ? (int)abs_unit(a, pf).row0 : 0;
+      auto pf_advance = [&]() {
+        if (++pkb == KB) {
+          pkb = 0;
+          pf.next(a);
+          if (pf.valid()) prow = (int)abs_unit(a, pf).row0;
+        }
+      };
+      for (int i = 0; i < kAbsPrefetchKb && pf.valid(); ++i) pf_advance();
       for (; wk.valid() && !stop; wk.next(a)) {
         const AbsUnit un = abs_unit(a, wk);
         if (un.first) {
@@ -299,6 +317,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
           const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
           if (leader) mbar_arrive_expect_tx(&full[s], 2 * L::STAGE_BYTES);
           tma_load_2d_cg2(stages + s * L::STAGE_BYTES, &tmH, kb * L::BK, hrow, bar);
+          if (kAbsPrefetchKb > 0 && pf.valid()) {
+            tma_prefetch_l2_2d(&tmH, pkb * L::BK, prow + (int)rank * 128);
+            pf_advance();
+          }
         }
       }
     }
@@ -415,14 +437,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
         tmem_ld_wait();
         const float4* r4 = reinterpret_cast<const float4*>(r + c * 32);
         const bool masked = c * 32 + 32 > nv;
+        if (!masked) {  // four independent chains
+          float m4[4] = {mx, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 rr = r4[i];
+            m4[0] = fmaxf(m4[0], __uint_as_float(v[4 * i]) * rr.x);
+            m4[1] = fmaxf(m4[1], __uint_as_float(v[4 * i + 1]) * rr.y);
+            m4[2] = fmaxf(m4[2], __uint_as_float(v[4 * i + 2]) * rr.z);
+            m4[3] = fmaxf(m4[3], __uint_as_float(v[4 * i + 3]) * rr.w);
+          }
+          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+          continue;
+        }
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const float4 rr = r4[i];
           const float x0 = __uint_as_float(v[4 * i]) * rr.x, x1 = __uint_as_float(v[4 * i + 1]) * rr.y;
           const float x2 = __uint_as_float(v[4 * i + 2]) * rr.z, x3 = __uint_as_float(v[4 * i + 3]) * rr.w;
-          if (!masked) {
-            mx = fmaxf(mx, fmaxf(fmaxf(x0, x1), fmaxf(x2, x3)));
-          } else {
+          {
             const int col = c * 32 + 4 * i;
             if (col < nv) mx = fmaxf(mx, x0);
             if (col + 1 < nv) mx = fmaxf(mx, x1);
@@ -451,38 +484,52 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
           tmem_ld_32x32b_x32(t0 + c0, v);
           tmem_ld_wait();
           const float4* r4 = reinterpret_cast<const float4*>(r + c0);
-          const bool masked = c0 + 32 > nv;
+          // Full 32-column chunks (all but the last of a ragged unit) skip the column test; four
+          // independent maximum / sum chains per chunk.
+          auto chunk = [&](auto masked_t) {
+            constexpr bool kMasked = decltype(masked_t)::value;
+            float mx4[4] = {mx, -INFINITY, -INFINITY, -INFINITY}, ls4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int j8 = 0; j8 < 4; ++j8) {
-            float w[8];
+            for (int j8 = 0; j8 < 4; ++j8) {
+              float w[8];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const float4 rr = r4[2 * j8 + h];
-              const float rv[4] = {rr.x, rr.y, rr.z, rr.w};
+              for (int h = 0; h < 2; ++h) {
+                const float4 rr = r4[2 * j8 + h];
+                const float rv[4] = {rr.x, rr.y, rr.z, rr.w};
 #pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const int j = 8 * j8 + 4 * h + k;
-                const float x = __uint_as_float(v[j]);
-                const bool ok = !masked || c0 + j < nv;
-                const float xr = x * rv[k];
-                mx = ok ? fmaxf(mx, xr) : mx;
-                const float pexp = fast_exp2(fmaf(x, rv[k], -m));
-                const float pv = ok ? pexp : 0.f;
-                lsum += pv;
-                w[4 * h + k] = pv * (ok ? rv[k] : 0.f);
+                for (int k = 0; k < 4; ++k) {
+                  const int j = 8 * j8 + 4 * h + k;
+                  const float x = __uint_as_float(v[j]);
+                  const float pexp = fast_exp2(fmaf(x, rv[k], -m));
+                  if (!kMasked) {
+                    mx4[k] = fmaxf(mx4[k], x * rv[k]);
+                    ls4[k] += pexp;
+                    w[4 * h + k] = pexp * rv[k];
+                  } else {
+                    const bool ok = c0 + j < nv;
+                    mx4[k] = ok ? fmaxf(mx4[k], x * rv[k]) : mx4[k];
+                    const float pv = ok ? pexp : 0.f;
+                    ls4[k] += pv;
+                    w[4 * h + k] = pv * (ok ? rv[k] : 0.f);
+                  }
+                }
               }
+              uint4 pk;
+              pk.x = pack_bf16x2(w[0], w[1]);
+              pk.y = pack_bf16x2(w[2], w[3]);
+              pk.z = pack_bf16x2(w[4], w[5]);
+              pk.w = pack_bf16x2(w[6], w[7]);
+              // row = lane; 16-byte chunk positions follow the store's swizzle (128- or 64-byte)
+              if (kAbsEpiCols == 64)
+                reinterpret_cast<uint4*>(sbuf + lane * 128)[(h2 * 4 + j8) ^ (lane & 7)] = pk;
+              else
+                reinterpret_cast<uint4*>(sbuf + lane * 64)[j8 ^ ((lane >> 1) & 3)] = pk;
             }
-            uint4 pk;
-            pk.x = pack_bf16x2(w[0], w[1]);
-            pk.y = pack_bf16x2(w[2], w[3]);
-            pk.z = pack_bf16x2(w[4], w[5]);
-            pk.w = pack_bf16x2(w[6], w[7]);
-            // row = lane; 16-byte chunk positions follow the store's swizzle (128- or 64-byte)
-            if (kAbsEpiCols == 64)
-              reinterpret_cast<uint4*>(sbuf + lane * 128)[(h2 * 4 + j8) ^ (lane & 7)] = pk;
-            else
-              reinterpret_cast<uint4*>(sbuf + lane * 64)[j8 ^ ((lane >> 1) & 3)] = pk;
-          }
+            mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+            lsum += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
+          };
+          if (c0 + 32 > nv) chunk(std::true_type{});
+          else chunk(std::false_type{});
           if (kAbsEpiCols == 32 || h2 == 1) {
             fence_proxy_async_smem();
             __syncwarp();
@@ -671,6 +718,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsBThreads, 1)
     if (lane == 0) {
       int kg = 0;
       bool stop = false;
+      // prefetch cursor (unit pf, chunk pc), kAbsBPrefetchCh valid chunks ahead of the loads
+      AbsWalk pf = wk;
+      int pc = 0;
+      AbsUnit pu{};
+      if (pf.valid()) pu = abs_unit(a, pf);
+      auto pf_advance = [&]() {
+        if (++pc == (pu.nvalid + 63) / 64) {
+          pc = 0;
+          pf.next(a);
+          if (pf.valid()) pu = abs_unit(a, pf);
+        }
+      };
+      for (int i = 0; i < kAbsBPrefetchCh && pf.valid(); ++i) pf_advance();
       for (; wk.valid() && !stop; wk.next(a)) {
         const AbsUnit un = abs_unit(a, wk);
         const int nch = (un.nvalid + 63) / 64;
@@ -691,6 +751,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsBThreads, 1)
             for (int j = 0; j < 2; ++j)
               tma_load_2d_cg2(st + L::A_BYTES + (e * 2 + j) * L::BOX_BYTES, &tmH, e * 256 + (int)rank * 128 + j * 64,
                               hrow, bar);
+          if (kAbsBPrefetchCh > 0 && pf.valid()) {
+            tma_prefetch_l2_2d(&tmP, 0, (pu.ptile0 + pc) * kAbsQ + (int)rank * 128);
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+#pragma unroll
+              for (int j = 0; j < 2; ++j)
+                tma_prefetch_l2_2d(&tmH, e * 256 + (int)rank * 128 + j * 64, (int)pu.row0 + 64 * pc);
+            pf_advance();
+          }
         }
       }
     }
