@@ -38,13 +38,12 @@ METRIC = "WHALE fusion-layer examples/s @15k jagged history; % of HBM/TC rooflin
 KV_TRAFFIC_BYTES_PER_ROW_D512 = {"2sm": (113.378816e6 + 169.603840e6) / 109605,
                                  "1sm": (113.375488e6 + 168.328960e6) / 109605}
 
-# DRAM bytes per history row of the absorbed path's pass A kernel (abs_scores_kernel): one ncu
-# capture at d = 512 on the full 403 481-row batch (441.23 MB read + 174.07 MB written per launch).
+# DRAM bytes per history row of the absorbed path's pass A kernel (abs_scores_kernel<2>): one ncu
+# capture at d = 512 on the full 403 481-row batch (444.91 MB read + 174.31 MB written per launch).
 # Two-kernel path only (the default).
-ABS_PASSA_BYTES_PER_ROW_D512 = (441.23e6 + 174.07e6) / 403481
-# ... and of a whole whale_attend_states call (its six kernels); None until captured for the
-# current pass B, merge and W_V GEMM (single-bf16 z)
-ABS_TRAFFIC_BYTES_PER_ROW_D512 = None
+ABS_PASSA_BYTES_PER_ROW_D512 = (444.91e6 + 174.31e6) / 403481
+# ... and of a whole whale_attend_states call (its six kernels: 1121.64 MB read + 193.49 MB written)
+ABS_TRAFFIC_BYTES_PER_ROW_D512 = (1121.64e6 + 193.49e6) / 403481
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
 
@@ -449,14 +448,15 @@ def main():
                 "algorithmic_flops": work["attention_absorbed"]["flops"],
                 "algorithmic_bytes": work["attention_absorbed"]["bytes"], "traffic": abs_traffic,
                 "traffic_source": "ncu dram bytes of the six kernels of one call at the full batch, per row"}
-        pa = kernels.get("abs_scores_kernel")
+        pa = next((v for k, v in kernels.items() if k.split("<")[0] == "abs_scores_kernel"), None)
         if pa:
             # the dominant kernel, pass A: S = qa H^T of N*h queries against every history row
             # (2 (N h) d FLOP per row) with the softmax; its ncu DRAM bytes per row scaled by rows
             fa = 2.0 * w.n_tokens * w.n_heads * total_L * w.d
             ta = pa["avg_ms"]
             a_tflops = fa / (ta * 1e-3) / 1e12
-            a_traffic = (ABS_PASSA_BYTES_PER_ROW_D512 * total_L) if passa_traffic_known else None
+            a_traffic = (ABS_PASSA_BYTES_PER_ROW_D512 * total_L
+                         if passa_traffic_known and ABS_PASSA_BYTES_PER_ROW_D512 is not None else None)
             roof = {"kernel": "abs_scores_kernel (absorbed pass A: scores on tcgen05 2-SM, online softmax, weights)",
                     "bound": "tensor", "achieved": a_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                     "frac": a_tflops / peaks["bf16_tflops"], "traffic": a_traffic,
