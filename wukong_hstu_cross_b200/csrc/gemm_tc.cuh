@@ -69,12 +69,17 @@ struct GemmSmem {
   static constexpr uint32_t A_ALL = SPLIT ? 2 * A_BYTES : A_BYTES;
   static constexpr uint32_t B_BYTES = BN * BK * 2;
   static constexpr uint32_t STAGE_BYTES = A_ALL + B_BYTES;
-  static constexpr int STAGES = (196608 / STAGE_BYTES) > 8 ? 8 : (196608 / STAGE_BYTES);
-  static constexpr size_t BYTES = 1024 /*alignment slack*/ + STAGES * (size_t)STAGE_BYTES + 2 * 128 * 4 /*row factors*/ +
-                                  256 /*barriers*/;
+  // stages fill what the 227 KB of shared memory leaves (one CTA per SM either way): five 40 KB
+  // stages for the 64-column hi/lo tiles
+  static constexpr int FIXED = 1024 /*alignment slack*/ + 2 * 128 * 4 /*row factors*/ + 256 /*barriers*/;
+  static constexpr int STAGES =
+      ((232448 - FIXED) / (int)STAGE_BYTES) > 8 ? 8 : ((232448 - FIXED) / (int)STAGE_BYTES);
+  static constexpr size_t BYTES = FIXED + STAGES * (size_t)STAGE_BYTES;
 };
 
-__device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
+// silu(x) = x / (1 + e^-x) with the fast (approximate-reciprocal) divide: a few ulp of fp32, far below
+// the 16 bits the hi/lo outputs keep; 0 once the denominator passes 2^126 (silu there is below 2^-119).
+__device__ __forceinline__ float silu_f(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 
 // bf16 -> fp32 is exact: the bf16 bits are the high half of the fp32 word (integer-pipe shift
 // and mask, no conversion instruction). The first element of each pair is the low half.
@@ -314,14 +319,9 @@ __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
       tc_fence_after();
       const float r = ROWNORM ? rbuf[acc * 128 + row] : 1.0f;
       const uint32_t t_row = tmem_base + acc * BN + ((uint32_t)(q * 32) << 16);
-      // (fully unrolled for the register-held residual, whose chunks need constant indices)
-#pragma unroll (kPre ? BN / 32 : 1)
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(t_row + c * 32, v);
-        tmem_ld_wait();
+      auto chunk = [&](const int c, const uint32_t (&v)[32]) {
         const int col = n0 + c * 32;
-        if (!row_ok || col >= args.N) continue;
+        if (!row_ok || col >= args.N) return;
         float x[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(v[j]) * r;
@@ -357,6 +357,18 @@ __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
             store_row_chunk<32>(args, gm * args.ldo + col, x);
           }
         }
+      };
+      // Two 32-column accumulator chunks per TMEM wait (BN / 32 is even); the loads are
+      // warp-collective, so every lane issues them. Fully unrolled for the register-held residual,
+      // whose chunks need constant indices.
+#pragma unroll (kPre ? BN / 64 : 1)
+      for (int c = 0; c < BN / 32; c += 2) {
+        uint32_t va[32], vb[32];
+        tmem_ld_32x32b_x32(t_row + c * 32, va);
+        tmem_ld_32x32b_x32(t_row + (c + 1) * 32, vb);
+        tmem_ld_wait();
+        chunk(c, va);
+        chunk(c + 1, vb);
       }
       // this accumulator buffer and its row factors may be reused
       tc_fence_before();
@@ -393,11 +405,12 @@ namespace whale {
 
 // ================================================================================================
 // Split-K variant for the residual-epilogue GEMMs with a long K (Fusion GEMM 2, K = 2d; the down
-// projection, K = 4d): a cluster of KS CTAs shares one 128 x 256 output tile, CTA r accumulating
-// K blocks [r KB/KS, (r+1) KB/KS) of hi/lo operand pairs into TMEM. Each CTA then puts its fp32
-// partial into its (now idle) stage memory; after a cluster barrier CTA r sums columns
+// projection, K = 4d): a cluster of KS = 4 or 8 CTAs shares one 128 x 256 output tile, CTA r
+// accumulating K blocks [r KB/KS, (r+1) KB/KS) of hi/lo operand pairs into TMEM. Each CTA then puts
+// its fp32 partial into its (now idle) stage memory; after a cluster barrier CTA r sums columns
 // [r 256/KS, (r+1) 256/KS) of the KS partials in rank order (the result does not depend on timing)
-// through distributed shared memory, adds the fp32 residual and writes the outputs. With 128 x 64
+// through distributed shared memory, adds the fp32 residual (loaded into registers while the MMAs
+// run) and writes the outputs. With 128 x 64
 // tiles each k-step of these GEMMs needs 40 KB of operands per 0.18 us of MMA, more than one SM
 // streams from L2; here a k-step is 64 KB per 0.72 us.
 // ================================================================================================
@@ -411,12 +424,13 @@ struct SplitKSmem {
   static constexpr size_t BYTES = 1024 + STAGES * (size_t)STAGE + 256;
 };
 
+// (No memory clobber, so several of these can be in flight at once; they are ordered after the
+// cluster barrier, itself volatile asm, that publishes the partials.)
 __device__ __forceinline__ float4 ld_shared_cluster_v4(uint32_t cluster_addr) {
   float4 v;
   asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
                : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(cluster_addr)
-               : "memory");
+               : "r"(cluster_addr));
   return v;
 }
 
@@ -502,7 +516,21 @@ __global__ void __launch_bounds__(192, 1)
       }
       umma_commit(tfull);  // also on abort: arrives once every issued MMA is done
     }
-  } else {
+  }
+  // This CTA reduces columns [kr NC, kr NC + NC) of the tile; the epilogue threads load their row's
+  // residual for them into registers while the MMAs run.
+  constexpr int NC = BN / KS;
+  static_assert(KS == 4 || KS == 8, "the residual of NC columns is held in registers");
+  float4 rres[NC / 4];
+  if (warp >= 2) {
+    const long long gm = (long long)m0 + (warp & 3) * 32 + lane;
+    if (gm < args.M) {
+      const float4* rp = reinterpret_cast<const float4*>(args.resid32 + gm * args.ldr + n0 + kr * NC);
+#pragma unroll
+      for (int i = 0; i < NC / 4; ++i) rres[i] = rp[i];
+    }
+  }
+  if (warp >= 2) {
     // epilogue warps 2..5: thread i of quadrant q owns row 32 q + i; the accumulator -> own partial
     const int q = warp & 3;
     const int row = q * 32 + lane;
@@ -530,16 +558,24 @@ __global__ void __launch_bounds__(192, 1)
     const int q = warp & 3;
     const int row = q * 32 + lane;
     const long long gm = (long long)m0 + row;
-    constexpr int NC = BN / KS;  // columns this CTA reduces
     const int c0 = kr * NC;
     const uint32_t base = smem_u32(part) + (uint32_t)(row * L::PSTRIDE * 4);
-#pragma unroll 1
-    for (int c = c0; c < c0 + NC; c += 8) {
+#pragma unroll
+    for (int g = 0; g < NC / 8; ++g) {
+      const int c = c0 + 8 * g;
+      // all KS partial chunks in flight first (remote loads), then summed in rank order (the sum
+      // does not depend on timing)
+      float4 pv[KS][2];
+#pragma unroll
+      for (int r = 0; r < KS; ++r) {
+        const uint32_t src = mapa_shared(base + (uint32_t)(c * 4), (uint32_t)r);
+        pv[r][0] = ld_shared_cluster_v4(src);
+        pv[r][1] = ld_shared_cluster_v4(src + 16);
+      }
       float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int r = 0; r < KS; ++r) {  // rank order: the sum does not depend on timing
-        const uint32_t src = mapa_shared(base + (uint32_t)(c * 4), (uint32_t)r);
-        const float4 v0 = ld_shared_cluster_v4(src), v1 = ld_shared_cluster_v4(src + 16);
+      for (int r = 0; r < KS; ++r) {
+        const float4 v0 = pv[r][0], v1 = pv[r][1];
         x[0] += v0.x;
         x[1] += v0.y;
         x[2] += v0.z;
@@ -551,8 +587,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (gm < args.M) {
         const int col = n0 + c;
-        const float4* rp = reinterpret_cast<const float4*>(args.resid32 + gm * args.ldr + col);
-        const float4 r0 = rp[0], r1 = rp[1];
+        const float4 r0 = rres[2 * g], r1 = rres[2 * g + 1];
         x[0] += r0.x;
         x[1] += r0.y;
         x[2] += r0.z;

@@ -535,7 +535,7 @@ whale_status gemm_bf16(const Opnd& a0, const Opnd& a1, const void* W, int N, con
     const int KBs = a0.K / 64;
     const long long tiles = tm * (N / 256);
     int ks = 1;
-    for (int c : {2, 4, 8})
+    for (int c : {4, 8})
       if (KBs % c == 0 && KBs / c >= 4 && tiles * c <= kNumSM) ks = c;
     if (ks > 1) {
       CUtensorMap ta, tl, tb;
@@ -555,11 +555,6 @@ whale_status gemm_bf16(const Opnd& a0, const Opnd& a1, const void* W, int N, con
       g.resid32 = resid32;
       g.ldr = ldr;
       const dim3 grid((unsigned)(tiles * ks));
-      if (ks == 2) {
-        CUCHECK(cudaFuncSetAttribute(gemm_splitk_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)SplitKSmem::BYTES));
-        return launch_cluster_pdl(gemm_splitk_kernel<2>, grid, dim3(192), SplitKSmem::BYTES, st, 2u, ta, tl, tb, g);
-      }
       if (ks == 4) {
         CUCHECK(cudaFuncSetAttribute(gemm_splitk_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)SplitKSmem::BYTES));
