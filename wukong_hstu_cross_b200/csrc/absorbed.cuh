@@ -172,8 +172,10 @@ __global__ void __launch_bounds__(1024) abs_units_kernel(const int* __restrict__
 // pass A: S = qa H^T, online softmax, pw = p * r
 // ================================================================================================
 // Columns of one weight store (the staging tile of an epilogue warp is 32 queries x kAbsEpiCols):
-// 64 (128-byte rows, 128-byte swizzle) or 32 (64-byte rows, 64-byte swizzle; half the staging
-// memory, one more stage of history rows at d = 512, twice the stores and proxy fences).
+// 64 (128-byte rows, 128-byte swizzle), 32 (64-byte rows, 64-byte swizzle) or 16 (32-byte rows,
+// 32-byte swizzle). Each halving of the staging memory leaves room for more stages of history rows
+// at d = 512 (3, 4, 5) at the price of twice the stores and proxy fences; 32 measured fastest
+// (4 us per layer ahead of 16, 9 us ahead of 64).
 constexpr int kAbsEpiCols = 32;
 // Pass A prefetches history rows into L2 this many 64-column blocks ahead of its stage loads (one
 // prefetch per load): lookahead beyond what the shared-memory ring holds. 0 disables it.
@@ -475,7 +477,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
       for (int cc = 0; cc < 2; ++cc) {
 #pragma unroll 1
         for (int h2 = 0; h2 < 2; ++h2) {
-          if (kAbsEpiCols == 32 || h2 == 0) {
+          if (kAbsEpiCols == 32 || (kAbsEpiCols == 64 && h2 == 0)) {
             if (lane == 0) bulk_wait_read<0>();  // the previous store from this buffer has read it
             __syncwarp();
           }
@@ -519,18 +521,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
               pk.y = pack_bf16x2(w[2], w[3]);
               pk.z = pack_bf16x2(w[4], w[5]);
               pk.w = pack_bf16x2(w[6], w[7]);
-              // row = lane; 16-byte chunk positions follow the store's swizzle (128- or 64-byte)
-              if (kAbsEpiCols == 64)
+              // row = lane; 16-byte chunk positions follow the store's swizzle (128-, 64- or 32-byte)
+              if (kAbsEpiCols == 64) {
                 reinterpret_cast<uint4*>(sbuf + lane * 128)[(h2 * 4 + j8) ^ (lane & 7)] = pk;
-              else
+              } else if (kAbsEpiCols == 32) {
                 reinterpret_cast<uint4*>(sbuf + lane * 64)[j8 ^ ((lane >> 1) & 3)] = pk;
+              } else {
+                if ((j8 & 1) == 0) {  // the previous store from this buffer has read it
+                  if (lane == 0) bulk_wait_read<0>();
+                  __syncwarp();
+                }
+                reinterpret_cast<uint4*>(sbuf + lane * 32)[(j8 & 1) ^ ((lane >> 2) & 1)] = pk;
+                if (j8 & 1) {
+                  fence_proxy_async_smem();
+                  __syncwarp();
+                  if (lane == 0) {
+                    tma_store_2d(&tmP, sbuf, h2 * 32 + (j8 >> 1) * 16,
+                                 (tile_row0 + hf * 2 + cc) * kAbsQ + (int)rank * 128 + qd * 32);
+                    bulk_commit();
+                  }
+                }
+              }
             }
             mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
             lsum += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
           };
           if (c0 + 32 > nv) chunk(std::true_type{});
           else chunk(std::false_type{});
-          if (kAbsEpiCols == 32 || h2 == 1) {
+          if (kAbsEpiCols == 32 || (kAbsEpiCols == 64 && h2 == 1)) {
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {

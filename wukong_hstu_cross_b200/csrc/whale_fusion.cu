@@ -193,19 +193,20 @@ whale_status get_encoder() {
 }
 
 // 2-D bf16 row-major tensor [rows, cols] with row stride ld, box [box_rows, box_cols]; the swizzle
-// spans one box row (box_cols 64: 128-byte swizzle, 32: 64-byte swizzle).
+// spans one box row (box_cols 64: 128-byte swizzle, 32: 64-byte, 16: 32-byte).
 whale_status tmap_bf16_box(CUtensorMap* tm, const void* base, long long rows, long long cols, long long ld,
                            int box_cols, int box_rows) {
   WCHECK(get_encoder());
   if ((reinterpret_cast<uintptr_t>(base) & 15) || (ld * 2) % 16 || rows <= 0 || cols <= 0) return WHALE_ERR_INVALID_ARG;
-  if (box_cols != 64 && box_cols != 32) return WHALE_ERR_INVALID_ARG;
+  if (box_cols != 64 && box_cols != 32 && box_cols != 16) return WHALE_ERR_INVALID_ARG;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
   cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
   cuuint32_t es[2] = {1u, 1u};
   CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
                         CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                        box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                       : (box_cols == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B),
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? WHALE_OK : WHALE_ERR_CUDA;
 }
