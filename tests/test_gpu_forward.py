@@ -176,3 +176,30 @@ def test_full_size_sampled(name):
     out3 = Hn.run_forward(p)
     torch.cuda.synchronize()
     assert torch.equal(out2, out3)
+
+
+def test_kernel_profile_records_every_launch():
+    """whale_profile_begin/end (the benchmark's per-kernel timing): one profiled forward of a
+    two-layer absorbed stack returns one record per launch, in launch order, each a kernel of this
+    library with a positive CUDA-event duration; profiling off again afterwards."""
+    w = I.WORKLOADS["hist15k_d512"].replace(**REDUCED["hist15k_d512"])
+    p = Hn.build_problem(w, device="cuda:0")
+    Hn.prepare_weights(p)
+    Hn.run_forward(p)  # first use outside the profile
+    torch.cuda.synchronize()
+    W.whale_profile_begin()
+    Hn.run_forward(p)
+    torch.cuda.synchronize()
+    recs = W.whale_profile_end()
+    names = [n for n, _ in recs]
+    assert len(recs) > 0 and all(ms > 0.0 for _, ms in recs)
+    assert all("whale" in n for n in names), names[:5]
+    # per layer: the absorbed passes run once each, in order
+    a = [i for i, n in enumerate(names) if "abs_scores_kernel" in n]
+    b = [i for i, n in enumerate(names) if "abs_values_kernel" in n]
+    assert len(a) == len(b) == w.n_layers and all(x < y for x, y in zip(a, b))
+    # nothing is recorded once profiling has ended
+    Hn.run_forward(p)
+    torch.cuda.synchronize()
+    W.whale_profile_begin()
+    assert W.whale_profile_end() == []
