@@ -68,6 +68,18 @@ def test_stack_reduced_workloads(name):
         _check(p, out)
 
 
+@pytest.mark.parametrize("name", ["stack_d256", "hist15k_d512"])
+def test_stack_on_cta_pair_gemms(name, monkeypatch):
+    """The whole stack with the token-side GEMMs on CTA pairs (WHALE_GEMM_PAIR=1): the row-norm
+    Q projection of the hi/lo residual stream, both Fusion GEMMs, up|gate and down."""
+    monkeypatch.setenv("WHALE_GEMM_PAIR", "1")
+    w = I.WORKLOADS[name].replace(**REDUCED[name])
+    p = Hn.build_problem(w, gains="random")
+    out = Hn.run_forward(p)
+    torch.cuda.synchronize()
+    _check(p, out)
+
+
 @pytest.mark.parametrize("shared_kv,tied_gate,fusion_mult", [(True, False, 2), (False, True, 2), (True, True, 0),
                                                               (False, False, 0)])
 def test_variants(shared_kv, tied_gate, fusion_mult):

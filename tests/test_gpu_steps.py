@@ -248,6 +248,38 @@ def test_residual_gemms_split_k(which, rows, d, monkeypatch):
     assert_parity(out, ref, "bf16", rms_rel=1e-2, what=which)
 
 
+@pytest.mark.parametrize("which,rows,d", [("fusion", 1000, 512), ("fusion", 130, 256), ("ffn", 1000, 512),
+                                           ("ffn", 300, 256), ("ffn", 2000, 512), ("tied", 257, 512)])
+def test_token_gemms_on_cta_pairs(which, rows, d, monkeypatch):
+    """The CTA-pair (cta_group::2) GEMM for hi/lo operand pairs, enabled with WHALE_GEMM_PAIR=1:
+    Fusion MLP (two K sources, SiLU and residual epilogues) and SwiGLU FFN (row-norm statistics with
+    the relay warp, SwiGLU / tied epilogues, residual), on row counts that leave the last 256-row
+    pair tile partly or wholly past the end."""
+    monkeypatch.setenv("WHALE_GEMM_PAIR", "1")
+    rng = np.random.default_rng(rows * 7 + d + len(which))
+    f = bf16_randn(rng, rows, d)
+    out = torch.empty(rows, d, dtype=torch.bfloat16, device=DEV)
+    if which == "fusion":
+        x = bf16_randn(rng, rows, d)
+        w1 = I.bf16_round(I.xavier_uniform(rng, 2 * d, 2 * d))
+        w2 = I.bf16_round(I.xavier_uniform(rng, d, 2 * d))
+        cfg = _cfg(d, d // 64, Fh=2 * d)
+        W.whale_fusion_mlp(cfg, rows, _t(f), _t(x), _t(w1), _t(w2), out, _ws(64 << 20))
+        ref = O.fusion_mlp(f, x, w1, w2)
+    else:
+        H = 4 * d
+        tied = which == "tied"
+        g = rng.uniform(0.5, 1.5, d).astype(np.float32)
+        wu = I.bf16_round(I.xavier_uniform(rng, H, d))
+        wug = wu if tied else np.concatenate([wu, I.bf16_round(I.xavier_uniform(rng, H, d))])
+        wd = I.bf16_round(I.xavier_uniform(rng, d, H))
+        cfg = _cfg(d, d // 64, flags=W.WHALE_TIED_GATE if tied else 0)
+        W.whale_swiglu_ffn(cfg, rows, _t(f), _g(g), _t(wug), _t(wd), out, _ws(64 << 20))
+        ref = O.swiglu_ffn(f, g, wug, wd, 1e-6, tied_gate=tied)
+    torch.cuda.synchronize()
+    assert_parity(out, ref, "bf16", rms_rel=1e-2, what=which)
+
+
 def test_project_kv_one_and_two_sm_kernels():
     """Both persistent K|V GEMMs on a ragged large M: the 2-SM (cta_group::2) default and the
     one-SM kernel selected with WHALE_GEMM_1SM=1; they must agree bitwise (same fp32 sums)."""

@@ -125,6 +125,85 @@ constexpr int gemm_threads() {
   return ROWNORM ? 320 : 192;
 }
 
+// ---- epilogue of one 128-row accumulator tile (shared by the one-CTA and the CTA-pair kernels) ----
+// Thread i of TMEM lane quadrant q owns output row 32q + i. Residual tiles of 64 columns: the row's
+// residual is loaded into registers before the accumulator is waited for, so its DRAM latency
+// overlaps the MMAs.
+template <int BN, int EPI>
+struct EpiPre {
+  static constexpr bool kOn = EPI == EPI_RESID && BN <= 64;
+  static constexpr int kN = kOn ? BN / 4 : 1;
+};
+
+template <int BN, int EPI>
+__device__ __forceinline__ void epi_load_resid(const GemmArgs& args, long long gm, bool row_ok, int n0,
+                                               float4 (&pre)[EpiPre<BN, EPI>::kN]) {
+  if (EpiPre<BN, EPI>::kOn && row_ok) {
+    const float4* rp = reinterpret_cast<const float4*>(args.resid32 + gm * args.ldr + n0);
+#pragma unroll
+    for (int i = 0; i < EpiPre<BN, EPI>::kN; ++i)
+      if (n0 + 4 * i < args.N) pre[i] = rp[i];
+  }
+}
+
+// t_row: TMEM address of this thread's lane at column 0 of the accumulator; r: row factor.
+template <int BN, int EPI>
+__device__ __forceinline__ void epi_tile(const GemmArgs& args, uint32_t t_row, float r, long long gm, bool row_ok,
+                                         int n0, const float4 (&pre)[EpiPre<BN, EPI>::kN]) {
+  constexpr bool kPre = EpiPre<BN, EPI>::kOn;
+  auto chunk = [&](const int c, const uint32_t (&v)[32]) {
+    const int col = n0 + c * 32;
+    if (!row_ok || col >= args.N) return;
+    float x[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(v[j]) * r;
+    if (EPI == EPI_SWIGLU) {
+      float h[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) h[j] = silu_f(x[16 + j]) * x[j];
+      store_row_chunk<16>(args, gm * args.ldo + col / 2, h);
+    } else {
+      if (EPI == EPI_RESID) {
+        const float4* rp = reinterpret_cast<const float4*>(args.resid32 + gm * args.ldr + col);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float4 t = kPre ? pre[(c * 8 + i) % EpiPre<BN, EPI>::kN] : rp[i];
+          x[4 * i] += t.x;
+          x[4 * i + 1] += t.y;
+          x[4 * i + 2] += t.z;
+          x[4 * i + 3] += t.w;
+        }
+      } else if (EPI == EPI_SILU) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[j] = silu_f(x[j]);
+      } else if (EPI == EPI_SWIGLU_TIED) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[j] = silu_f(x[j]) * x[j];
+      }
+      if (EPI == EPI_QABS) {
+        const int head = col / args.qabs_d;
+        const long long orow =
+            (gm / args.qabs_N) * args.qabs_rows + (long long)head * args.qabs_N + gm % args.qabs_N;
+        store_row_chunk<32>(args, orow * args.ldo + (col - head * args.qabs_d), x);
+      } else {
+        store_row_chunk<32>(args, gm * args.ldo + col, x);
+      }
+    }
+  };
+  // Two 32-column accumulator chunks per TMEM wait (BN / 32 is even); the loads are warp-collective,
+  // so every lane issues them. Fully unrolled for the register-held residual, whose chunks need
+  // constant indices.
+#pragma unroll (kPre ? BN / 64 : 1)
+  for (int c = 0; c < BN / 32; c += 2) {
+    uint32_t va[32], vb[32];
+    tmem_ld_32x32b_x32(t_row + c * 32, va);
+    tmem_ld_32x32b_x32(t_row + (c + 1) * 32, vb);
+    tmem_ld_wait();
+    chunk(c, va);
+    chunk(c + 1, vb);
+  }
+}
+
 template <int BN, int EPI, bool ROWNORM, bool SPLIT>
 __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA0lo,
@@ -298,78 +377,19 @@ __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
     // ---------------- epilogue (warps 2..5): thread i of quadrant q owns row 32q + i ----------------
     const int q = warp & 3;
     const int row = q * 32 + lane;
-    // Residual tiles of 64 columns: the row's residual is loaded into registers before the
-    // accumulator is waited for, so its DRAM latency overlaps the MMAs.
-    constexpr bool kPre = EPI == EPI_RESID && BN <= 64;
-    float4 pre[kPre ? BN / 4 : 1];
+    float4 pre[EpiPre<BN, EPI>::kN];
     int it = 0;
     for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1, ua = it >> 1;
       const int m0 = (tile / args.tiles_n) * L::BM, n0 = (tile % args.tiles_n) * BN;
       const long long gm = (long long)m0 + row;
       const bool row_ok = gm < args.M;
-      if (kPre && row_ok) {
-        const float4* rp = reinterpret_cast<const float4*>(args.resid32 + gm * args.ldr + n0);
-#pragma unroll
-        for (int i = 0; i < (kPre ? BN / 4 : 1); ++i)
-          if (n0 + 4 * i < args.N) pre[i] = rp[i];
-      }
+      epi_load_resid<BN, EPI>(args, gm, row_ok, n0, pre);
       if (!mbar_wait(&tfull[acc], ua & 1, abort_flag)) break;
       if (ROWNORM && !mbar_wait(&nfull[acc], ua & 1, abort_flag)) break;
       tc_fence_after();
       const float r = ROWNORM ? rbuf[acc * 128 + row] : 1.0f;
-      const uint32_t t_row = tmem_base + acc * BN + ((uint32_t)(q * 32) << 16);
-      auto chunk = [&](const int c, const uint32_t (&v)[32]) {
-        const int col = n0 + c * 32;
-        if (!row_ok || col >= args.N) return;
-        float x[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(v[j]) * r;
-        if (EPI == EPI_SWIGLU) {
-          float h[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) h[j] = silu_f(x[16 + j]) * x[j];
-          store_row_chunk<16>(args, gm * args.ldo + col / 2, h);
-        } else {
-          if (EPI == EPI_RESID) {
-            const float4* rp = reinterpret_cast<const float4*>(args.resid32 + gm * args.ldr + col);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float4 t = kPre ? pre[(c * 8 + i) % (kPre ? BN / 4 : 1)] : rp[i];
-              x[4 * i] += t.x;
-              x[4 * i + 1] += t.y;
-              x[4 * i + 2] += t.z;
-              x[4 * i + 3] += t.w;
-            }
-          } else if (EPI == EPI_SILU) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) x[j] = silu_f(x[j]);
-          } else if (EPI == EPI_SWIGLU_TIED) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) x[j] = silu_f(x[j]) * x[j];
-          }
-          if (EPI == EPI_QABS) {
-            const int head = col / args.qabs_d;
-            const long long orow =
-                (gm / args.qabs_N) * args.qabs_rows + (long long)head * args.qabs_N + gm % args.qabs_N;
-            store_row_chunk<32>(args, orow * args.ldo + (col - head * args.qabs_d), x);
-          } else {
-            store_row_chunk<32>(args, gm * args.ldo + col, x);
-          }
-        }
-      };
-      // Two 32-column accumulator chunks per TMEM wait (BN / 32 is even); the loads are
-      // warp-collective, so every lane issues them. Fully unrolled for the register-held residual,
-      // whose chunks need constant indices.
-#pragma unroll (kPre ? BN / 64 : 1)
-      for (int c = 0; c < BN / 32; c += 2) {
-        uint32_t va[32], vb[32];
-        tmem_ld_32x32b_x32(t_row + c * 32, va);
-        tmem_ld_32x32b_x32(t_row + (c + 1) * 32, vb);
-        tmem_ld_wait();
-        chunk(c, va);
-        chunk(c + 1, vb);
-      }
+      epi_tile<BN, EPI>(args, tmem_base + acc * BN + ((uint32_t)(q * 32) << 16), r, gm, row_ok, n0, pre);
       // this accumulator buffer and its row factors may be reused
       tc_fence_before();
       __syncwarp();

@@ -33,6 +33,7 @@
 #include "attention_qtile.cuh"
 #include "fp32_path.cuh"
 #include "gemm_2sm.cuh"
+#include "gemm_pair.cuh"
 #include "gemm_persistent.cuh"
 #include "gemm_tc.cuh"
 #include "ptx.cuh"
@@ -77,6 +78,13 @@ inline bool qtile_enabled() {
 // slower than one CTA per 128 x 64 tile (3.45-3.50 against 3.39-3.41 ms per 8-layer step).
 inline bool splitk_enabled() {
   const char* e = std::getenv("WHALE_GEMM_SPLITK");
+  return e && e[0] == '1';
+}
+// WHALE_GEMM_PAIR=1 in the environment runs the token-side GEMMs with hi/lo operand pairs on CTA
+// pairs (gemm_pair.cuh). Off by default: on the 2048-row token batch it measured no faster than
+// one CTA per tile (step 3.19-3.22 against 3.20-3.21 ms; Fusion GEMM 1 slower, up|gate even).
+inline bool gemm_pair_enabled() {
+  const char* e = std::getenv("WHALE_GEMM_PAIR");
   return e && e[0] == '1';
 }
 inline bool abs_fused_enabled() {
@@ -421,6 +429,59 @@ whale_status launch_gemm_t(const CUtensorMap* tm, const GemmArgs& g, long long t
   return launch_pdl(kern, dim3(grid), dim3(gemm_threads<RN>()), smem, st, tm[0], tm[1], tm[2], tm[3], tm[4], g);
 }
 
+// Co-resident two-CTA clusters of a pair kernel (cached per kernel and device).
+whale_status pair_max_clusters(const void* kern, size_t smem, int threads, int* clusters) {
+  static std::mutex mu;
+  static std::vector<std::pair<std::pair<const void*, int>, int>> cache;
+  int dev = 0;
+  CUCHECK(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lk(mu);
+  for (const auto& e : cache)
+    if (e.first.first == kern && e.first.second == dev) {
+      *clusters = e.second;
+      return e.second > 0 ? WHALE_OK : WHALE_ERR_UNSUPPORTED;
+    }
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(kNumSM, 1, 1);
+  lc.blockDim = dim3(threads, 1, 1);
+  lc.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  int n = 0;
+  CUCHECK(cudaOccupancyMaxActiveClusters(&n, kern, &lc));
+  n = std::min(n, kNumSM / 2);
+  cache.push_back({{kern, dev}, n > 0 ? n : -1});
+  *clusters = n;
+  return n > 0 ? WHALE_OK : WHALE_ERR_UNSUPPORTED;
+}
+
+template <int BN, int EPI, bool RN>
+whale_status launch_pair_t(const CUtensorMap* tm, const GemmArgs& g, cudaStream_t st) {
+  const size_t smem = PairSmem<BN>::BYTES;
+  auto kern = gemm_pair_kernel<BN, EPI, RN>;
+  CUCHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  int pairs = 0;
+  WCHECK(pair_max_clusters(reinterpret_cast<const void*>(kern), smem, pair_threads<RN>(), &pairs));
+  const long long np = std::min<long long>(g.num_tiles, pairs);
+  return launch_pdl(kern, dim3((unsigned)(2 * np)), dim3(pair_threads<RN>()), smem, st, tm[0], tm[1], tm[2], tm[3],
+                    tm[4], g);
+}
+
+template <int BN>
+whale_status launch_pair_bn(int epi, bool rn, const CUtensorMap* tm, const GemmArgs& g, cudaStream_t st) {
+  if (rn && epi == EPI_STORE) return launch_pair_t<BN, EPI_STORE, true>(tm, g, st);
+  if (rn && epi == EPI_SWIGLU) return launch_pair_t<BN, EPI_SWIGLU, true>(tm, g, st);
+  if (rn && epi == EPI_SWIGLU_TIED) return launch_pair_t<BN, EPI_SWIGLU_TIED, true>(tm, g, st);
+  if (!rn && epi == EPI_SILU) return launch_pair_t<BN, EPI_SILU, false>(tm, g, st);
+  if (!rn && epi == EPI_RESID) return launch_pair_t<BN, EPI_RESID, false>(tm, g, st);
+  return WHALE_ERR_UNSUPPORTED;
+}
+
 template <int BN>
 whale_status launch_gemm_bn(int epi, bool rn, bool split, const CUtensorMap* tm, const GemmArgs& g, long long tiles,
                             cudaStream_t st) {
@@ -565,6 +626,51 @@ whale_status gemm_bf16(const Opnd& a0, const Opnd& a1, const void* W, int N, con
                                    (int)SplitKSmem::BYTES));
       return launch_cluster_pdl(gemm_splitk_kernel<8>, grid, dim3(192), SplitKSmem::BYTES, st, 8u, ta, tl, tb, g);
     }
+  }
+  // hi/lo operand pairs: 256-row tiles on CTA pairs, each SM streaming half of the W tile. Tile
+  // width by the cost model below with pairs as the persistent unit and the per-SM streaming rate
+  // the per-CTA timelines show (~43 B/clk).
+  if (split && M > 128 && gemm_pair_enabled() &&
+      (rn ? (epi == EPI_STORE || epi == EPI_SWIGLU || epi == EPI_SWIGLU_TIED) : (epi == EPI_SILU || epi == EPI_RESID))) {
+    const int KBp = (a0.K + a1.K) / 64;
+    const long long tp = cdiv<long long>(M, 256);
+    auto pcost = [&](int bn) -> double {
+      if (N % bn) return 1e300;
+      const double per_pair = (double)cdiv<long long>(tp * (N / bn), kNumSM / 2);
+      return 5600.0 + per_pair * KBp * std::max(4.0 * bn, (32768.0 + bn * 64.0) / 43.0);
+    };
+    int bn = 64;
+    for (int cand : {128, 256})
+      if (pcost(cand) < pcost(bn)) bn = cand;
+    CUtensorMap maps[5];
+    WCHECK(tmap_bf16(&maps[0], a0.hi, M, a0.K, a0.ld, 128));
+    WCHECK(tmap_bf16(&maps[1], a0.lo, M, a0.K, a0.ld, 128));
+    if (a1.K > 0) {
+      WCHECK(tmap_bf16(&maps[2], a1.hi, M, a1.K, a1.ld, 128));
+      WCHECK(tmap_bf16(&maps[3], a1.lo, M, a1.K, a1.ld, 128));
+    } else {
+      maps[2] = maps[0];
+      maps[3] = maps[1];
+    }
+    WCHECK(tmap_bf16(&maps[4], W, N, a0.K + a1.K, a0.K + a1.K, bn / 2));
+    GemmArgs g{};
+    g.M = (int)M;
+    g.N = N;
+    g.kb0 = a0.K / 64;
+    g.kb1 = a1.K / 64;
+    g.tiles_n = N / bn;
+    g.num_tiles = (int)(tp * g.tiles_n);
+    g.inv_k = 1.0f / (float)a0.K;
+    g.eps = eps;
+    g.out_hi = static_cast<__nv_bfloat16*>(out.hi);
+    g.out_lo = static_cast<__nv_bfloat16*>(out.lo);
+    g.out32 = out.f32;
+    g.ldo = out.ld;
+    g.resid32 = resid32;
+    g.ldr = ldr;
+    if (bn == 256) return launch_pair_bn<256>(epi, rn, maps, g, st);
+    if (bn == 128) return launch_pair_bn<128>(epi, rn, maps, g, st);
+    return launch_pair_bn<64>(epi, rn, maps, g, st);
   }
   // Tile width by a small cost model (cycles): per-CTA fixed cost + tiles per persistent CTA x
   // (per 64-deep K block the larger of the MMA time and the operand bytes at ~80 B/clk, the rate
