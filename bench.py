@@ -176,35 +176,72 @@ class ClockSampler:
 # ------------------------------------------------------------------------------------------------
 # CPU baseline: the oracle on a bounded sample of the workload
 # ------------------------------------------------------------------------------------------------
+class OracleSampler:
+    """The fp64 oracle timed on whole examples of the workload, in batch order: lengths and weights
+    are drawn once; each example's inputs are generated outside the timed region. With `cycle`,
+    the sampler walks the first `cycle` examples over and over, their inputs generated once."""
+
+    def __init__(self, w: I.Workload, cycle: int = 0):
+        self.w = w
+        self.L = I.draw_lengths(w)
+        self.lws = I.make_all_weights(w)
+        # serving workload: time 64 of the request's candidate tokens, scale per example
+        self.sample_tokens = 64 if w.candidates else w.n_tokens
+        self.cycle = min(cycle, w.batch) if cycle > 0 else w.batch
+        self.cache = {}
+        self.next_b = 0
+        self.done, self.toks, self.t = 0, 0, 0.0
+
+    def inputs(self, b: int):
+        if b in self.cache:
+            return self.cache[b]
+        w = self.w
+        x = I.tokens_of_example(w, b)[:self.sample_tokens]
+        slabs = [I.states_of_example(w, l, b, int(self.L[b])) for l in range(w.n_layers)]
+        if self.cycle < w.batch:
+            self.cache[b] = (x, slabs)
+        return x, slabs
+
+    def run(self, budget_s: float, max_examples: int = None, count: bool = True) -> None:
+        """Examples from the rolling index on until budget_s of oracle time (at least one)."""
+        from oracle import whale_oracle as O
+        w = self.w
+        t_run, n = 0.0, 0
+        while True:
+            b = self.next_b
+            self.next_b = (self.next_b + 1) % self.cycle
+            x, slabs = self.inputs(b)
+            t0 = time.perf_counter()
+            O.fusion_stack_example(x, slabs, self.lws, w.n_heads, w.eps)
+            dt = time.perf_counter() - t0
+            t_run += dt
+            n += 1
+            if count:
+                self.t += dt
+                self.done += 1
+                self.toks += self.sample_tokens
+            if t_run >= budget_s or (max_examples is not None and n >= max_examples):
+                break
+
+    def summary(self, what: str) -> dict:
+        w = self.w
+        cores = len(os.sched_getaffinity(0))
+        if w.candidates:
+            # per-token cost: the sampled tokens share the K/V projections (amortised as in serving)
+            value = 1.0 / (self.t * (w.n_tokens / self.toks))
+            desc = f"{self.done} request(s), {self.sample_tokens} of {w.n_tokens} candidate tokens timed, scaled per request"
+        else:
+            value = self.done / self.t
+            where = f"examples 0..{self.cycle - 1} in turn" if self.cycle < w.batch else "examples in batch order"
+            desc = f"{what}: {self.done} timed, {where} (all {w.n_layers} layers, all {w.n_tokens} tokens each)"
+        return {"value": value, "unit": "examples/s", "cores": cores, "kind": "oracle",
+                "sample": desc + f"; fp64 numpy, {self.t:.1f} s of CPU time"}
+
+
 def oracle_sample(w: I.Workload, budget_s: float = 15.0, max_examples: int = 64):
-    from oracle import whale_oracle as O
-    L = I.draw_lengths(w)
-    lws = I.make_all_weights(w)
-    done, t_oracle = 0, 0.0
-    toks = 0
-    sample_tokens = w.n_tokens
-    if w.candidates:   # serving workload: time 64 of the request's candidate tokens, scale per example
-        sample_tokens = 64
-    for b in range(min(w.batch, max_examples)):
-        x = I.tokens_of_example(w, b)[:sample_tokens]
-        slabs = [I.states_of_example(w, l, b, int(L[b])) for l in range(w.n_layers)]
-        t0 = time.perf_counter()
-        O.fusion_stack_example(x, slabs, lws, w.n_heads, w.eps)
-        t_oracle += time.perf_counter() - t0
-        done += 1
-        toks += sample_tokens
-        if t_oracle >= budget_s:
-            break
-    cores = len(os.sched_getaffinity(0))
-    if w.candidates:
-        # per-token cost excluding nothing: the sampled tokens share the K/V projections (amortised as in serving)
-        value = 1.0 / (t_oracle * (w.n_tokens / toks))
-        desc = f"{done} request(s), {sample_tokens} of {w.n_tokens} candidate tokens timed, scaled per request"
-    else:
-        value = done / t_oracle
-        desc = f"first {done} of {w.batch} examples (all {w.n_layers} layers, all {w.n_tokens} tokens each)"
-    return {"value": value, "unit": "examples/s", "cores": cores, "kind": "oracle",
-            "sample": desc + f"; fp64 numpy, {t_oracle:.1f} s of CPU time"}
+    s = OracleSampler(w)
+    s.run(budget_s, max_examples=min(w.batch, max_examples))
+    return s.summary("first examples")
 
 
 # ------------------------------------------------------------------------------------------------
@@ -240,15 +277,20 @@ def run_reference(args):
         return 0
     w = I.WORKLOADS[args.workload]
     t0 = time.time()
-    vals = []
     steps = max(args.steps, 1)
+    sampler = OracleSampler(w, cycle=12)
+    for _ in range(max(args.warmup, 0)):   # untimed: one example each
+        sampler.run(0.0, count=False)
+    sampler.next_b = 0
+    # the whole run is bounded: each step gets an equal share of --ref-total seconds of oracle time
+    # (at least one whole example), cycling over the batch's first 12 examples (inputs generated once)
+    per_step = max(0.2, args.ref_total / steps)
     for _ in range(steps):
-        cb = oracle_sample(w, budget_s=args.ref_budget)
-        vals.append(cb["value"])
-    value = statistics.median(vals)
-    cb["value"] = value
+        sampler.run(per_step)
+    cb = sampler.summary("oracle")
+    value = cb["value"]
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "examples/s", "n_gpus": args.gpus,
-            "steps": steps, "warmup": 0, "ms_per_step": 1e3 * w.batch / value if value else None,
+            "steps": steps, "warmup": max(args.warmup, 0), "ms_per_step": 1e3 * w.batch / value if value else None,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, "batch": w.batch, "n_tokens": w.n_tokens, "d": w.d, "heads": w.n_heads,
                        "layers": w.n_layers},
@@ -325,7 +367,9 @@ def main():
     ap.add_argument("--workload", default="hist15k_d512", choices=list(I.WORKLOADS))
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
-    ap.add_argument("--ref-budget", type=float, default=15.0)
+    ap.add_argument("--ref-budget", type=float, default=15.0, help="oracle seconds of the cpu_baseline sample")
+    ap.add_argument("--ref-total", type=float, default=150.0,
+                    help="oracle seconds of the whole --impl reference run, split across its steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-case", choices=["kv", "attn", "ffn", "fusion", "absorbed"], default=None,
                     help="profiling aid: run only one step entry point on one layer of the workload")
