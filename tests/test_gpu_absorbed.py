@@ -201,3 +201,47 @@ def test_fused_kernel_agrees_with_two_passes(monkeypatch):
     one = Hn.run_forward(p).clone().float()
     torch.cuda.synchronize()
     assert bool(((one - two).abs() <= 2e-2 * (1 + two.abs())).all())
+
+
+def _states_host(p, b):
+    """Per-layer history rows of example b as they sit on the device (bf16 values, exact in fp64)."""
+    o0, o1 = int(p.offsets[b]), int(p.offsets[b + 1])
+    return [p.states[l, o0:o1].float().cpu().numpy() for l in range(p.w.n_layers)]
+
+
+def test_absorbed_long_history_of_identical_rows():
+    """A 15 000-row history whose rows are all equal (every score ties: the softmax is an average
+    over 59 units split across CTA pairs, each unit's weights exactly 1), next to a one-row and a
+    4 000-row copy-of-one-row history; checked against the oracle on the device's states."""
+    w = _workload(512, 3)
+    p = Hn.build_problem(w, lengths=np.array([15000, 1, 4000]), gains="random")
+    for b in (0, 2):
+        o0, o1 = int(p.offsets[b]), int(p.offsets[b + 1])
+        p.states[:, o0:o1] = p.states[:, o0:o0 + 1]
+    Hn.prepare_weights(p)
+    out = Hn.run_forward(p)
+    torch.cuda.synchronize()
+    o = out.float().cpu().numpy()
+    for b in range(3):
+        ref = O.fusion_stack_example(I.tokens_of_example(w, b), _states_host(p, b), p.host_weights, w.n_heads,
+                                     w.eps, **p.flags)
+        assert_parity(o[b], ref, "bf16", rms_rel=2e-2, what=f"example {b}")
+
+
+def test_absorbed_history_permutation_invariance_full_lengths():
+    """Permuting the rows of every example's history (the same permutation in every layer) leaves
+    the output unchanged up to summation order, at the 15k workload's length mix: the scores move
+    across units, CTA pairs and partial segments."""
+    w = _workload(512, 8, n_layers=2)
+    p = Hn.build_problem(w)
+    Hn.prepare_weights(p)
+    out1 = Hn.run_forward(p).clone()
+    rng = np.random.default_rng(11)
+    for b in range(w.batch):
+        o0, o1 = int(p.offsets[b]), int(p.offsets[b + 1])
+        perm = torch.from_numpy(rng.permutation(o1 - o0) + o0).to(p.states.device)
+        p.states[:, o0:o1] = p.states[:, perm]
+    out2 = Hn.run_forward(p)
+    torch.cuda.synchronize()
+    assert_parity(out2.float().cpu().numpy(), out1.float().cpu().numpy().astype(np.float64), "bf16", rms_rel=2e-2,
+                  what="permuted history")
