@@ -177,6 +177,10 @@ __global__ void __launch_bounds__(1024) abs_units_kernel(const int* __restrict__
 // at d = 512 (3, 4, 5) at the price of twice the stores and proxy fences; 32 measured fastest
 // (4 us per layer ahead of 16, 9 us ahead of 64).
 constexpr int kAbsEpiCols = 32;
+// The softmax of full 32-column chunks in packed f32x2 arithmetic (scale, shift, sums and weights of
+// two scores per instruction) with 3-input maxima: fewer issue slots in the epilogue that bounds
+// pass A.
+constexpr bool kAbsPackedSoftmax = true;
 // Pass A prefetches history rows into L2 this many 64-column blocks ahead of its stage loads (one
 // prefetch per load): lookahead beyond what the shared-memory ring holds. 0 disables it.
 constexpr int kAbsPrefetchKb = 4;
@@ -477,17 +481,71 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
       for (int cc = 0; cc < 2; ++cc) {
 #pragma unroll 1
         for (int h2 = 0; h2 < 2; ++h2) {
-          if (kAbsEpiCols == 32 || (kAbsEpiCols == 64 && h2 == 0)) {
+          const int c0 = cc * 64 + h2 * 32;
+          // the packed path of 32-column stores waits for the staging buffer only once its
+          // weights are in registers (the previous store's read then overlaps the arithmetic)
+          const bool late_wait = kAbsPackedSoftmax && kAbsEpiCols == 32 && c0 + 32 <= nv;
+          if (!late_wait && (kAbsEpiCols == 32 || (kAbsEpiCols == 64 && h2 == 0))) {
             if (lane == 0) bulk_wait_read<0>();  // the previous store from this buffer has read it
             __syncwarp();
           }
-          const int c0 = cc * 64 + h2 * 32;
           uint32_t v[32];
           tmem_ld_32x32b_x32(t0 + c0, v);
           tmem_ld_wait();
           const float4* r4 = reinterpret_cast<const float4*>(r + c0);
           // Full 32-column chunks (all but the last of a ragged unit) skip the column test; four
           // independent maximum / sum chains per chunk.
+          auto packed_chunk = [&]() {
+            const uint64_t nm2 = f2pack(-m, -m);
+            uint64_t lsa = f2pack(0.f, 0.f), lsb = lsa;
+            float mxa = mx, mxb = -INFINITY;
+            uint4 pks[4];
+#pragma unroll
+            for (int j8 = 0; j8 < 4; ++j8) {
+              uint32_t wpk[4];
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const float4 rr = r4[2 * j8 + h];
+                const int j = 8 * j8 + 4 * h;
+                const uint64_t r01 = f2pack(rr.x, rr.y), r23 = f2pack(rr.z, rr.w);
+                const uint64_t xr01 = fmul2(f2pack(__uint_as_float(v[j]), __uint_as_float(v[j + 1])), r01);
+                const uint64_t xr23 = fmul2(f2pack(__uint_as_float(v[j + 2]), __uint_as_float(v[j + 3])), r23);
+                float x0, x1, x2, x3, t0, t1, t2, t3;
+                f2unpack(xr01, x0, x1);
+                f2unpack(xr23, x2, x3);
+                mxa = fmax3(mxa, x0, x1);
+                mxb = fmax3(mxb, x2, x3);
+                f2unpack(fadd2(xr01, nm2), t0, t1);
+                f2unpack(fadd2(xr23, nm2), t2, t3);
+                const uint64_t p01 = f2pack(fast_exp2(t0), fast_exp2(t1));
+                const uint64_t p23 = f2pack(fast_exp2(t2), fast_exp2(t3));
+                lsa = fadd2(lsa, p01);
+                lsb = fadd2(lsb, p23);
+                float w0, w1, w2, w3;
+                f2unpack(fmul2(p01, r01), w0, w1);
+                f2unpack(fmul2(p23, r23), w2, w3);
+                wpk[2 * h] = pack_bf16x2(w0, w1);
+                wpk[2 * h + 1] = pack_bf16x2(w2, w3);
+              }
+              pks[j8] = make_uint4(wpk[0], wpk[1], wpk[2], wpk[3]);
+            }
+            if (kAbsEpiCols == 32) {
+              if (lane == 0) bulk_wait_read<0>();  // the previous store from this buffer has read it
+              __syncwarp();
+            }
+#pragma unroll
+            for (int j8 = 0; j8 < 4; ++j8) {
+              if (kAbsEpiCols == 64)
+                reinterpret_cast<uint4*>(sbuf + lane * 128)[(h2 * 4 + j8) ^ (lane & 7)] = pks[j8];
+              else
+                reinterpret_cast<uint4*>(sbuf + lane * 64)[j8 ^ ((lane >> 1) & 3)] = pks[j8];
+            }
+            mx = fmaxf(mxa, mxb);
+            float l0, l1, l2, l3;
+            f2unpack(lsa, l0, l1);
+            f2unpack(lsb, l2, l3);
+            lsum += (l0 + l1) + (l2 + l3);
+          };
           auto chunk = [&](auto masked_t) {
             constexpr bool kMasked = decltype(masked_t)::value;
             float mx4[4] = {mx, -INFINITY, -INFINITY, -INFINITY}, ls4[4] = {0.f, 0.f, 0.f, 0.f};
@@ -547,6 +605,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
             lsum += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
           };
           if (c0 + 32 > nv) chunk(std::true_type{});
+          else if (kAbsPackedSoftmax && kAbsEpiCols != 16) packed_chunk();
           else chunk(std::false_type{});
           if (kAbsEpiCols == 32 || (kAbsEpiCols == 64 && h2 == 1)) {
             fence_proxy_async_smem();
