@@ -671,19 +671,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
           l_part += l_unit;
         }
       }
-      if (hf == 0) a.mref[(size_t)wk.u * kAbsQ + qg] = m_use;
+      float l_seg = 0.f;
       if (un.last) {
         xsum[hf * 128 + row] = l_part;
         __syncwarp();
         if (lane == 0) mbar_arrive(&lbar[qd]);
         if (!mbar_wait(&lbar[qd], nseg & 1, abort_flag)) break;
         ++nseg;
-        if (hf == 0) {
-          const float l = xsum[row] + xsum[128 + row];
-          float2* st = un.whole ? reinterpret_cast<float2*>(a.stats_whole) + (size_t)un.b * kAbsQ + qg
-                                : reinterpret_cast<float2*>(a.stats_part) + (size_t)un.slot * kAbsQ + qg;
-          *st = make_float2(m_use, l);
-        }
+        l_seg = xsum[row] + xsum[128 + row];
       }
       tc_fence_before();
       __syncwarp();
@@ -691,6 +686,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
         mbar_arrive_cluster(tempty0 + acc * 8);  // the even CTA's MMA may reuse this accumulator
         mbar_arrive(&edone[acc]);
         mbar_arrive_cluster_release(edone_peer0 + acc * 8);
+      }
+      // The unit's reference and the segment's (m, l) are for pass B and the merge (later kernels):
+      // stored after the arrives, so the cluster-scope release above does not wait for them.
+      if (hf == 0) {
+        a.mref[(size_t)wk.u * kAbsQ + qg] = m_use;
+        if (un.last) {
+          float2* st = un.whole ? reinterpret_cast<float2*>(a.stats_whole) + (size_t)un.b * kAbsQ + qg
+                                : reinterpret_cast<float2*>(a.stats_part) + (size_t)un.slot * kAbsQ + qg;
+          *st = make_float2(m_use, l_seg);
+        }
       }
     }
     if (lane == 0) bulk_wait<0>();
