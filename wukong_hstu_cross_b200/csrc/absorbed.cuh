@@ -201,8 +201,11 @@ struct AbsASmem {
   static constexpr int STAGES = (232448 - FIXED) / (int)STAGE_BYTES > 8 ? 8 : (232448 - FIXED) / (int)STAGE_BYTES;
   static constexpr size_t BYTES = FIXED + STAGES * (size_t)STAGE_BYTES;
   static_assert(STAGES >= 3, "at least three stages of history rows");
+  // full/ready/empty per stage; tfull, tempty, nfull, edone, eloc [2]; xbar [8]; lbar [4]; qfull,
+  // qempty; then the TMEM address slot and the abort flag
+  static_assert(3 * STAGES * 8 + 24 * 8 + 8 <= 512, "barriers fit their area");
 };
-constexpr int kAbsAThreads = 480;
+constexpr int kAbsAThreads = 512;
 
 // The absorbed queries of the example (the MMA's A operand, 128 per CTA) stay resident in shared
 // memory for the pair's whole segment of that example: the stage ring carries history rows only,
@@ -210,7 +213,9 @@ constexpr int kAbsAThreads = 480;
 // warps: 0 TMA producer (both CTAs), 1 TMEM (2 x 256 columns) + MMA issue (even CTA), 2..9 softmax
 // epilogue (two warps per lane quadrant, 128 columns each), 10..13 row statistics of this CTA's 128
 // history rows (r of all 256 columns reaches both CTAs through distributed shared memory), 14 relay
-// of "stage landed" (even CTA) as in the 2-SM projection GEMM.
+// of "stage landed" (even CTA) as in the 2-SM projection GEMM, 15 forwarder of "epilogue done with
+// the unit's row factors" to the peer CTA: a cluster-scope release costs about 0.7 us, so the
+// epilogue warps arrive locally (CTA scope) and this warp issues the cluster-scope arrive.
 template <int E>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
     abs_scores_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmH,
@@ -237,7 +242,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
   uint64_t* lbar = xbar + 8;      // [4 quadrants] segment sums of both half-warps written
   uint64_t* qfull = lbar + 4;     // the segment's queries landed (both CTAs' copies, even CTA)
   uint64_t* qempty = qfull + 1;   // the segment's last MMAs are done (commit to both CTAs)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qempty + 1);
+  uint64_t* eloc = qempty + 1;    // [2] the 8 local epilogue warps are done with the row factors
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(eloc + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -257,7 +263,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], 16);
       mbar_init(&nfull[i], 8);
-      mbar_init(&edone[i], 16);
+      mbar_init(&edone[i], 2);  // the forwarders of both CTAs
+      mbar_init(&eloc[i], 8);
     }
     for (int i = 0; i < 8; ++i) mbar_init(&xbar[i], 2);
     for (int i = 0; i < 4; ++i) mbar_init(&lbar[i], 2);
@@ -365,6 +372,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
         if (un.last) umma_commit_cg2_mc(qempty, 0x3);  // also on abort: arrives once issued MMAs are done
       }
     }
+  } else if (warp == 15) {
+    // ---------------- forwarder (both CTAs): local epilogue done -> both CTAs' edone ----------------
+    if (lane == 0) {
+      const uint32_t edone_peer0 = mapa_shared(smem_u32(&edone[0]), rank ^ 1);
+      int it = 0;
+      for (; wk.valid(); wk.next(a), ++it) {
+        const int acc = it & 1, ua = it >> 1;
+        if (!mbar_wait(&eloc[acc], ua & 1, abort_flag)) break;
+        mbar_arrive(&edone[acc]);
+        mbar_arrive_cluster_release(edone_peer0 + acc * 8);
+      }
+    }
   } else if (warp == 14) {
     // ---------------- relay (even CTA) ----------------
     if (leader && lane == 0) {
@@ -431,7 +450,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
     const int qg = (int)rank * 128 + row;
     uint8_t* sbuf = epi + (warp - 2) * L::EPI_WARP;
     const uint32_t tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
-    const uint32_t edone_peer0 = mapa_shared(smem_u32(&edone[0]), rank ^ 1);
 
     // maximum of r_t * s over the valid columns of this half
     auto tile_max = [&](uint32_t t0, const float* r, int nv) -> float {
@@ -684,8 +702,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
       __syncwarp();
       if (lane == 0) {
         mbar_arrive_cluster(tempty0 + acc * 8);  // the even CTA's MMA may reuse this accumulator
-        mbar_arrive(&edone[acc]);
-        mbar_arrive_cluster_release(edone_peer0 + acc * 8);
+        mbar_arrive(&eloc[acc]);                 // forwarded to both CTAs' edone by warp 15
       }
       // The unit's reference and the segment's (m, l) are for pass B and the merge (later kernels):
       // stored after the arrives, so the cluster-scope release above does not wait for them.
