@@ -52,6 +52,7 @@ struct AbsArgs {
   float* stats_part;        // [2 * n_pairs, 256] (m, l) of partial segments
   __nv_bfloat16* part_z;    // [2 * n_pairs, 256, d] unnormalised z of partial segments (bf16)
   __nv_bfloat16* z_hi;      // [h, B*N, d] z / l, bf16 (row j*B*N + b*N + n)
+  const int* pstart;        // [n_pairs][8]: u0, u1, b, ub, ub1 of each pair's range (null: searched)
 };
 
 __device__ __forceinline__ long long abs_off(const AbsArgs& a, int b) {
@@ -77,6 +78,16 @@ struct AbsWalk {
   int b, ub, ub1;  // example of u and its unit range
   __device__ __forceinline__ void init(const AbsArgs& a, int p_) {
     p = p_;
+    if (a.pstart != nullptr) {  // tabulated once per forward by abs_units_kernel
+      const int4 e = *reinterpret_cast<const int4*>(a.pstart + 8 * p);
+      u0 = e.x;
+      u1 = e.y;
+      b = e.z;
+      ub = e.w;
+      ub1 = a.pstart[8 * p + 4];
+      u = u0;
+      return;
+    }
     const int U = a.ustart[a.B];
     u0 = abs_range_start(U, a.n_pairs, p);
     u1 = abs_range_start(U, a.n_pairs, p + 1);
@@ -134,8 +145,11 @@ __device__ __forceinline__ AbsUnit abs_unit(const AbsArgs& a, const AbsWalk& w) 
 
 // ustart[b] = sum_{b' < b} ceil(L_b' / 256), capped at units_max (only inconsistent offsets reach
 // the cap; they lose rows, never index past the buffers). One block of 1024 threads.
+// With P > 0 it also tabulates each of the P pairs' starting state for AbsWalk (pstart[p][0..4] =
+// u0, u1, the example b of unit u0, ustart[b], ustart[b + 1]), so the passes start without a search.
 __global__ void __launch_bounds__(1024) abs_units_kernel(const int* __restrict__ offsets, int B, long long total_L,
-                                                         int units_max, int* __restrict__ ustart) {
+                                                         int units_max, int* __restrict__ ustart, int P,
+                                                         int* __restrict__ pstart) {
   pdl_wait();
   pdl_trigger();
   __shared__ int part[1024];
@@ -166,6 +180,30 @@ __global__ void __launch_bounds__(1024) abs_units_kernel(const int* __restrict__
     if (run > units_max) run = units_max;
   }
   if (threadIdx.x == 1023) ustart[B] = part[1023];
+  if (P <= 0) return;
+  __syncthreads();  // ustart written by this block is visible to it
+  const int U = __ldcg(ustart + B);
+  for (int p = threadIdx.x; p < P; p += blockDim.x) {
+    const int u0 = abs_range_start(U, P, p), u1 = abs_range_start(U, P, p + 1);
+    int b = 0, ub = 0, ub1 = 0;
+    if (u0 < u1) {
+      int lo = 0, hi = B - 1;  // largest b with ustart[b] <= u0
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (__ldcg(ustart + mid) <= u0) lo = mid;
+        else hi = mid - 1;
+      }
+      b = lo;
+      ub = __ldcg(ustart + b);
+      ub1 = __ldcg(ustart + b + 1);
+    }
+    int* e = pstart + 8 * p;
+    e[0] = u0;
+    e[1] = u1;
+    e[2] = b;
+    e[3] = ub;
+    e[4] = ub1;
+  }
 }
 
 // ================================================================================================

@@ -330,7 +330,7 @@ struct Layout {
   size_t a_lo, g_lo, f_lo, u_lo, f32, x32[2], xhi[2], xlo[2];
   // absorbed attention: folded key weights, absorbed queries, weights pw, unit references,
   // segment statistics, partial z, unit starts, z as a bf16 pair
-  size_t wkabs, qa, pw, mref, stw, stp, pz, ust, zh;
+  size_t wkabs, qa, pw, mref, stw, stp, pz, ust, zh, pst;
   long long units_max;
   size_t total;
 };
@@ -373,6 +373,7 @@ Layout make_layout(const Shape& s, const whale_shape_hint& hint) {
     L.stp = take((size_t)2 * kMaxPairs * kAbsQ * 8);
     L.pz = take((size_t)2 * kMaxPairs * kAbsQ * s.d * 2);
     L.ust = take(((size_t)hint.B + 1) * 4);
+    L.pst = take((size_t)kMaxPairs * 8 * 4);
     L.zh = take((size_t)hint.B * kAbsQ * s.d * 2);
   }
   L.a = take(rows * s.d * s.es);
@@ -999,13 +1000,26 @@ whale_status gemm_vabs(const Shape& s, const void* zh, const void* wv, void* a, 
   return launch_gemm_t<64, EPI_STORE, false, false>(maps, g, tiles, st);
 }
 
-// Unit starts of the batch (once per forward: the offsets are shared by every layer).
+// CTA pairs of the two-pass kernels (0 with the one-pass kernel, whose clusters search their starts).
+whale_status abs_two_pass_pairs(const Shape& s, const Layout& L, int* P) {
+  *P = 0;
+  if (abs_fused_enabled()) return WHALE_OK;
+  int pairs = 0;
+  WCHECK(abs_max_pairs(s.d / 256, &pairs));
+  *P = (int)std::max<long long>(1, std::min<long long>(pairs, L.units_max));
+  return WHALE_OK;
+}
+
+// Unit starts of the batch and the pairs' starting states (once per forward: the offsets are shared
+// by every layer).
 whale_status abs_units(const Shape& s, const int* offsets, const whale_shape_hint& hint, void* ws, const Layout& L,
                        cudaStream_t st) {
   if (!s.absorbed || hint.B == 0) return WHALE_OK;
   if (L.units_max >= (1ll << 31) / kAbsRows) return WHALE_ERR_UNSUPPORTED;
+  int P = 0;
+  WCHECK(abs_two_pass_pairs(s, L, &P));
   return launch_pdl(abs_units_kernel, dim3(1), dim3(1024), 0, st, offsets, hint.B, (long long)hint.total_L,
-                    (int)L.units_max, reinterpret_cast<int*>(at(ws, L.ust)));
+                    (int)L.units_max, reinterpret_cast<int*>(at(ws, L.ust)), P, reinterpret_cast<int*>(at(ws, L.pst)));
 }
 
 // S3 through the absorbed path: q (bf16 [B*N, d]) -> A (bf16 pair [B*N, d]).
@@ -1049,9 +1063,10 @@ whale_status attention_absorbed(const Shape& s, const void* q, const void* slab,
     WCHECK(launch_pdl(abs_merge_kernel, dim3(hint.B, kAbsQ / 8), dim3(256), 0, st, a));
     return gemm_vabs(s, at(ws, L.zh), wv, out, out_lo, rows, st);
   }
-  int pairs = 0;
-  WCHECK(abs_max_pairs(E, &pairs));
-  a.n_pairs = (int)std::max<long long>(1, std::min<long long>(pairs, L.units_max));
+  int P = 0;
+  WCHECK(abs_two_pass_pairs(s, L, &P));
+  a.n_pairs = P;  // the pair count abs_units tabulated the starts for
+  a.pstart = reinterpret_cast<const int*>(at(ws, L.pst));
   if (hint.total_L > 0) {
     CUtensorMap tq, th, tps;
     WCHECK(tmap_bf16(&tq, at(ws, L.qa), (long long)hint.B * kAbsQ, s.d, s.d, 128));
