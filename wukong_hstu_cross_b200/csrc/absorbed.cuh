@@ -53,6 +53,9 @@ struct AbsArgs {
   __nv_bfloat16* part_z;    // [2 * n_pairs, 256, d] unnormalised z of partial segments (bf16)
   __nv_bfloat16* z_hi;      // [h, B*N, d] z / l, bf16 (row j*B*N + b*N + n)
   const int* pstart;        // [n_pairs][8]: u0, u1, b, ub, ub1 of each pair's range (null: searched)
+  // [2 + n_pairs]: pairs of pass A in the order they finished (p + 1; 0 = not yet) after two counters
+  // (entries published, entries taken). Null: pass B waits for the whole of pass A instead.
+  int* pq;
 };
 
 __device__ __forceinline__ long long abs_off(const AbsArgs& a, int b) {
@@ -146,10 +149,11 @@ __device__ __forceinline__ AbsUnit abs_unit(const AbsArgs& a, const AbsWalk& w) 
 // ustart[b] = sum_{b' < b} ceil(L_b' / 256), capped at units_max (only inconsistent offsets reach
 // the cap; they lose rows, never index past the buffers). One block of 1024 threads.
 // With P > 0 it also tabulates each of the P pairs' starting state for AbsWalk (pstart[p][0..4] =
-// u0, u1, the example b of unit u0, ustart[b], ustart[b + 1]), so the passes start without a search.
+// u0, u1, the example b of unit u0, ustart[b], ustart[b + 1]), so the passes start without a search,
+// and clears pq, the order in which the pairs of pass A finish.
 __global__ void __launch_bounds__(1024) abs_units_kernel(const int* __restrict__ offsets, int B, long long total_L,
                                                          int units_max, int* __restrict__ ustart, int P,
-                                                         int* __restrict__ pstart) {
+                                                         int* __restrict__ pstart, int* __restrict__ pq) {
   pdl_wait();
   pdl_trigger();
   __shared__ int part[1024];
@@ -181,6 +185,7 @@ __global__ void __launch_bounds__(1024) abs_units_kernel(const int* __restrict__
   }
   if (threadIdx.x == 1023) ustart[B] = part[1023];
   if (P <= 0) return;
+  for (int i = threadIdx.x; i < 2 + P; i += blockDim.x) pq[i] = 0;  // the finishing order of pass A
   __syncthreads();  // ustart written by this block is visible to it
   const int U = __ldcg(ustart + B);
   for (int p = threadIdx.x; p < P; p += blockDim.x) {
@@ -756,12 +761,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
     if (lane == 0) bulk_wait<0>();
   }
 
+  if (a.pq != nullptr) {  // weights (bulk stores, complete above), references, statistics: to gpu scope
+    fence_proxy_async_all();
+    __threadfence();
+  }
   tc_fence_before();
   __syncthreads();
   cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc_cg2(tmem_base, 512);
+  }
+  // Pass B reads only this pair's outputs: publish the pair as finished (both CTAs are past the
+  // cluster barrier, so their writes are ordered before the release).
+  if (a.pq != nullptr && leader && threadIdx.x == 0) {
+    __threadfence();
+    st_release_gpu(a.pq + 2 + atomicAdd(a.pq, 1), pair + 1);
   }
 }
 
@@ -812,6 +827,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsBThreads, 1)
   uint64_t* cready = udone + 2;   // [2] even CTA: unit released by 8 + 8 correction warps
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cready + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* ticket = reinterpret_cast<int*>(tmem_slot + 2);  // even CTA: this pair's place in pass A's order
+  int* src_slot = ticket + 1;                           // the pass A pair taken (+ 1; 0 = none)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -828,6 +845,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsBThreads, 1)
       mbar_init(&cready[i], 16);
     }
     *abort_flag = 0;
+    if (a.pq != nullptr && leader) *ticket = atomicAdd(a.pq + 1, 1);
     fence_mbar_init();
     fence_proxy_async_smem();
   }
@@ -844,11 +862,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsBThreads, 1)
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  pdl_wait();
+  int src = pair;  // the pass A pair whose units (weights, references, statistics) this pair reduces
+  if (a.pq != nullptr) {
+    // Pass A pairs are taken in the order they finish (the ticket drawn by the even CTA), each as
+    // soon as its outputs are published: no wait for the rest of pass A.
+    if (threadIdx.x == 0) {
+      const int t = leader ? *ticket : ld_shared_cluster_s32(mapa_shared(smem_u32(ticket), 0));
+      const int v = (t >= 0 && t < a.n_pairs) ? wait_nonzero_gpu(a.pq + 2 + t) : 0;
+      fence_proxy_async_all();  // the weights are read by TMA below
+      if (v == 0) *abort_flag = 1;
+      *src_slot = v;
+    }
+    __syncthreads();
+    src = *src_slot - 1;
+  } else {
+    pdl_wait();
+  }
   pdl_trigger();
 
   AbsWalk wk;
-  wk.init(a, pair);
+  wk.init(a, src < 0 ? pair : src);
+  if (src < 0) wk.u = wk.u1;  // nothing taken (timed out): no units
 
   if (warp == 0) {
     // ---------------- TMA producer (both CTAs): only the 64-row chunks holding valid rows ----------
@@ -1010,6 +1044,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsBThreads, 1)
 __global__ void __launch_bounds__(256) abs_merge_kernel(const AbsArgs a) {
   pdl_wait();
   pdl_trigger();
+  if (a.pq != nullptr && blockIdx.x == 0 && blockIdx.y == 0)  // both passes are complete: reset
+    for (int i = threadIdx.x; i < 2 + a.n_pairs; i += blockDim.x) a.pq[i] = 0;
   __shared__ int s_slot[8][kAbsMaxPairs];
   __shared__ float s_w[8][kAbsMaxPairs];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

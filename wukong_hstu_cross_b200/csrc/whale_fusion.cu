@@ -330,7 +330,7 @@ struct Layout {
   size_t a_lo, g_lo, f_lo, u_lo, f32, x32[2], xhi[2], xlo[2];
   // absorbed attention: folded key weights, absorbed queries, weights pw, unit references,
   // segment statistics, partial z, unit starts, z as a bf16 pair
-  size_t wkabs, qa, pw, mref, stw, stp, pz, ust, zh, pst;
+  size_t wkabs, qa, pw, mref, stw, stp, pz, ust, zh, pst, pq;
   long long units_max;
   size_t total;
 };
@@ -374,6 +374,7 @@ Layout make_layout(const Shape& s, const whale_shape_hint& hint) {
     L.pz = take((size_t)2 * kMaxPairs * kAbsQ * s.d * 2);
     L.ust = take(((size_t)hint.B + 1) * 4);
     L.pst = take((size_t)kMaxPairs * 8 * 4);
+    L.pq = take((size_t)(2 + kMaxPairs) * 4);
     L.zh = take((size_t)hint.B * kAbsQ * s.d * 2);
   }
   L.a = take(rows * s.d * s.es);
@@ -1019,7 +1020,8 @@ whale_status abs_units(const Shape& s, const int* offsets, const whale_shape_hin
   int P = 0;
   WCHECK(abs_two_pass_pairs(s, L, &P));
   return launch_pdl(abs_units_kernel, dim3(1), dim3(1024), 0, st, offsets, hint.B, (long long)hint.total_L,
-                    (int)L.units_max, reinterpret_cast<int*>(at(ws, L.ust)), P, reinterpret_cast<int*>(at(ws, L.pst)));
+                    (int)L.units_max, reinterpret_cast<int*>(at(ws, L.ust)), P, reinterpret_cast<int*>(at(ws, L.pst)),
+                    reinterpret_cast<int*>(at(ws, L.pq)));
 }
 
 // S3 through the absorbed path: q (bf16 [B*N, d]) -> A (bf16 pair [B*N, d]).
@@ -1067,6 +1069,7 @@ whale_status attention_absorbed(const Shape& s, const void* q, const void* slab,
   WCHECK(abs_two_pass_pairs(s, L, &P));
   a.n_pairs = P;  // the pair count abs_units tabulated the starts for
   a.pstart = reinterpret_cast<const int*>(at(ws, L.pst));
+  a.pq = reinterpret_cast<int*>(at(ws, L.pq));  // pass B takes each pair of pass A as it finishes
   if (hint.total_L > 0) {
     CUtensorMap tq, th, tps;
     WCHECK(tmap_bf16(&tq, at(ws, L.qa), (long long)hint.B * kAbsQ, s.d, s.d, 128));
