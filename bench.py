@@ -39,11 +39,11 @@ KV_TRAFFIC_BYTES_PER_ROW_D512 = {"2sm": (113.378816e6 + 169.603840e6) / 109605,
                                  "1sm": (113.375488e6 + 168.328960e6) / 109605}
 
 # DRAM bytes per history row of the absorbed path's pass A kernel (abs_scores_kernel<2>): one ncu
-# capture at d = 512 on the full 403 481-row batch (444.99 MB read + 178.94 MB written per launch).
+# capture at d = 512 on the full 403 481-row batch (444.77 MB read + 174.42 MB written per launch).
 # Two-kernel path only (the default).
-ABS_PASSA_BYTES_PER_ROW_D512 = (444.99e6 + 178.94e6) / 403481
-# ... and of a whole whale_attend_states call (its six kernels: 1121.64 MB read + 193.49 MB written)
-ABS_TRAFFIC_BYTES_PER_ROW_D512 = (1121.64e6 + 193.49e6) / 403481
+ABS_PASSA_BYTES_PER_ROW_D512 = (444.77e6 + 174.42e6) / 403481
+# ... and of a whole whale_attend_states call (its six kernels: 1121.52 MB read + 191.63 MB written)
+ABS_TRAFFIC_BYTES_PER_ROW_D512 = (1121.52e6 + 191.63e6) / 403481
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
 
