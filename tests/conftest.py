@@ -13,7 +13,7 @@ def pytest_configure(config):
 
 
 def pytest_collection_modifyitems(config, items):
-    # GPU tests are skipped (not failed) when no GPU is visible; on the GPU machine they run.
+    # GPU tests are skipped (not failed) when no GPU is visible; with a GPU they run.
     try:
         import torch
         has_gpu = torch.cuda.is_available()
