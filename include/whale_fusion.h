@@ -145,7 +145,10 @@ whale_status whale_profile_begin(int max_kernels);
 whale_status whale_profile_end(whale_kernel_time* out, int capacity, int* count);
 
 /* Bytes of device workspace needed by every entry point below for this config and
- * shape (0 if cfg/hint are invalid or unsupported). */
+ * shape (0 if cfg/hint are invalid or unsupported). The workspace holds one call's scratch
+ * tensors and the words its kernels synchronise through (the order in which the absorbed
+ * attention's first-pass CTA pairs finish, cleared by every call): calls in flight at the same
+ * time, on different streams, need separate workspaces; calls ordered on one stream may share one. */
 size_t whale_workspace_size(const whale_config* cfg, const whale_shape_hint* hint);
 
 /* One-time weight preparation (bf16 mode). RMSNorm(x; g) W^T = r(x) * (x (W diag(g))^T), so the
