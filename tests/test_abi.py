@@ -3,8 +3,6 @@ host-side checks return the documented status codes. No GPU work: every call bel
 returns before any CUDA call is made."""
 import ctypes
 
-import pytest
-
 from wukong_hstu_cross_b200 import build
 
 build.build()

@@ -18,7 +18,6 @@ if torch.cuda.is_available():
     from wukong_hstu_cross_b200 import build
     build.build()
     from wukong_hstu_cross_b200 import whale as W
-    from wukong_hstu_cross_b200 import harness as Hn
 
 DEV = "cuda"
 
