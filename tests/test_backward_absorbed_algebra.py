@@ -9,7 +9,8 @@ a backward kernel in the same layout would compute, per example:
   dz  = dA_j W'_V,j                       dW'_V,j = dA_j^T z
   dp  = r_t (dz . H_t)                    delta   = dz . z   (= sum_t p dp)
   ds  = p (dp - delta)                    dqa     = sum_t ds r_t H_t
-  dH_t = r_t sum_q (ds qa + p dz) - (r_t^2 H_t / d) sum_q (ds s + p dp)   (the second term: r_t)
+  dH_t = r_t sum_q (ds qa + p dz) - (r_t^2 H_t / d) sum_q (ds s + p dp)   (the second term: r_t;
+         its row sum equals H_t . (the first term), so it needs no reduction over queries)
 
 and the weight and gain gradients from dqa, q, dA and z alone (no pass over the history). This
 test states those formulas in plain numpy and checks them against oracle/whale_backward.py (which
@@ -120,3 +121,35 @@ def test_absorbed_backward_split_history_sums():
             dH_parts[lo:hi] += rp[:, None] * (ds.T @ qa + p.T @ dz) - (rp * rp / d)[:, None] * Hp * colsum[:, None]
     np.testing.assert_allclose(dq_parts, dq, rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(dH_parts, dH, rtol=1e-10, atol=1e-12)
+
+
+def test_rmsnorm_term_from_the_dH_product_rows():
+    """The RMSNorm term of dH needs no reduction over queries in the scoring pass: with
+    dH_raw_t = r_t sum_q (ds qa + p dz) (the dH product itself), sum_q (ds s + p dp) = H_t . dH_raw_t,
+    so dH_t = dH_raw_t - (r_t^2 / d) H_t (H_t . dH_raw_t): one dot product per history row in that
+    product's epilogue."""
+    rng = np.random.default_rng(43)
+    n, L, d, heads, eps = 5, 8, 16, 2, 1e-3
+    q, H = rng.standard_normal((n, d)), rng.standard_normal((L, d))
+    g = rng.uniform(0.5, 1.5, d)
+    w_k, w_v = rng.standard_normal((d, d)) * d ** -0.5, rng.standard_normal((d, d)) * d ** -0.5
+    dA = rng.standard_normal((n, d))
+    _, _, dH, _, _, _ = _absorbed_backward(q, H, g, w_k, w_v, dA, heads, eps)
+    dh = d // heads
+    r = 1.0 / np.sqrt(np.mean(H * H, axis=1) + eps)
+    raw = np.zeros_like(H)
+    for j in range(heads):
+        sl = slice(j * dh, (j + 1) * dh)
+        qa = q[:, sl] @ w_k[sl] / np.sqrt(dh) * g
+        s = r[None, :] * (qa @ H.T)
+        p = np.exp(s - s.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        z = (p * r[None, :]) @ H
+        dz = dA[:, sl] @ (w_v[sl] * g[None, :])
+        dp = r[None, :] * (dz @ H.T)
+        ds = p * (dp - np.sum(dz * z, axis=1, keepdims=True))
+        raw_j = r[:, None] * (ds.T @ qa + p.T @ dz)
+        np.testing.assert_allclose(np.sum(H * raw_j, axis=1), np.sum(ds * s + p * dp, axis=0), rtol=1e-10, atol=1e-12)
+        raw += raw_j
+    np.testing.assert_allclose(raw - (r * r / d)[:, None] * H * np.sum(H * raw, axis=1, keepdims=True), dH,
+                               rtol=1e-10, atol=1e-12)
