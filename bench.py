@@ -33,10 +33,9 @@ from wukong_hstu_cross_b200 import inputs as I  # noqa: E402
 
 METRIC = "WHALE fusion-layer examples/s @15k jagged history; % of HBM/TC roofline"
 # DRAM bytes per launch measured by ncu (dram__bytes_read.sum + dram__bytes_write.sum), per
-# history row: one capture of the K|V projection GEMM at d = 512 on 109 605 rows (the 2-SM default
-# kernel and the one-SM kernel). Reported only for that width; null otherwise.
-KV_TRAFFIC_BYTES_PER_ROW_D512 = {"2sm": (113.378816e6 + 169.603840e6) / 109605,
-                                 "1sm": (113.375488e6 + 168.328960e6) / 109605}
+# history row: one capture of the 2-SM K|V projection GEMM at d = 512 on 109 605 rows. Reported
+# only for that width; null otherwise.
+KV_TRAFFIC_BYTES_PER_ROW_D512 = (113.378816e6 + 169.603840e6) / 109605
 
 # DRAM bytes per history row of the absorbed path's pass A kernel (abs_scores_kernel<2>): one ncu
 # capture at d = 512 on the full 403 481-row batch (444.77 MB read + 174.42 MB written per launch).
@@ -55,6 +54,33 @@ def load_peaks():
         return p, "measured"
     except Exception:
         return PEAKS_FALLBACK, "fallback"
+
+
+def tensor_peak(peaks: dict, clocks) -> tuple:
+    """The bf16 tensor peak that applies to kernels timed in this run: the burst figure when the SM
+    clock sampled during the timed region stayed near its maximum (a short run, below the power
+    cap), else the sustained figure (a long run that settled under the power cap)."""
+    burst, sus = peaks["bf16_tflops"], peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    mx = peaks.get("sm_max_mhz", 1965.0)
+    if clocks and clocks.get("sm_mhz") and clocks["sm_mhz"] < 0.95 * mx:
+        return sus, f"bf16 sustained (median SM clock {clocks['sm_mhz']:.0f} of {mx:.0f} MHz under load)"
+    return burst, (f"bf16 burst (median SM clock {clocks['sm_mhz']:.0f} of {mx:.0f} MHz under load)" if clocks
+                   and clocks.get("sm_mhz") else "bf16 burst (no clock samples)")
+
+
+def roofline_of(flops: float, nbytes: float, t_ms: float, tc_peak: float, hbm_peak: float) -> dict:
+    """Roofline position of a kernel from its algorithmic work: the bound is the larger of its FLOP
+    time at the tensor peak and its byte time at the copy bandwidth; achieved and peak are in that
+    bound's unit, so frac = (bound's algorithmic time) / (measured time)."""
+    t_flop = flops / (tc_peak * 1e12)
+    t_byte = nbytes / (hbm_peak * 1e9)
+    t = t_ms * 1e-3
+    if t_flop >= t_byte:
+        return {"bound": "tensor", "achieved": flops / t / 1e12, "peak": tc_peak, "unit": "TFLOP/s",
+                "frac": t_flop / t, "t_flop_us": t_flop * 1e6, "t_byte_us": t_byte * 1e6,
+                "tensor_frac": t_flop / t, "hbm_frac": t_byte / t}
+    return {"bound": "hbm", "achieved": nbytes / t / 1e9, "peak": hbm_peak, "unit": "GB/s", "frac": t_byte / t,
+            "t_flop_us": t_flop * 1e6, "t_byte_us": t_byte * 1e6, "tensor_frac": t_flop / t, "hbm_frac": t_byte / t}
 
 
 # ------------------------------------------------------------------------------------------------
@@ -177,40 +203,39 @@ class ClockSampler:
 # CPU baseline: the oracle on a bounded sample of the workload
 # ------------------------------------------------------------------------------------------------
 class OracleSampler:
-    """The fp64 oracle timed on whole examples of the workload, in batch order: lengths and weights
-    are drawn once; each example's inputs are generated outside the timed region. With `cycle`,
-    the sampler walks the first `cycle` examples over and over, their inputs generated once."""
+    """The fp64 oracle timed on whole examples of the workload, walking the batch in order (and
+    round again): lengths and weights are drawn once; each example's inputs are generated outside
+    the timed region, the next example's in a background thread while the current one runs."""
 
-    def __init__(self, w: I.Workload, cycle: int = 0):
+    def __init__(self, w: I.Workload):
+        from concurrent.futures import ThreadPoolExecutor
         self.w = w
         self.L = I.draw_lengths(w)
         self.lws = I.make_all_weights(w)
         # serving workload: time 64 of the request's candidate tokens, scale per example
         self.sample_tokens = 64 if w.candidates else w.n_tokens
-        self.cycle = min(cycle, w.batch) if cycle > 0 else w.batch
-        self.cache = {}
         self.next_b = 0
         self.done, self.toks, self.t = 0, 0, 0.0
+        self.step_s = []
+        self.pool = ThreadPoolExecutor(1)
+        self.pending = self.pool.submit(self._inputs, 0)
 
-    def inputs(self, b: int):
-        if b in self.cache:
-            return self.cache[b]
+    def _inputs(self, b: int):
         w = self.w
         x = I.tokens_of_example(w, b)[:self.sample_tokens]
         slabs = [I.states_of_example(w, l, b, int(self.L[b])) for l in range(w.n_layers)]
-        if self.cycle < w.batch:
-            self.cache[b] = (x, slabs)
         return x, slabs
 
-    def run(self, budget_s: float, max_examples: int = None, count: bool = True) -> None:
-        """Examples from the rolling index on until budget_s of oracle time (at least one)."""
+    def run(self, budget_s: float, max_examples: int = None, count: bool = True) -> float:
+        """Examples from the rolling index on until budget_s of oracle time (at least one); returns
+        the oracle time spent."""
         from oracle import whale_oracle as O
         w = self.w
         t_run, n = 0.0, 0
         while True:
-            b = self.next_b
-            self.next_b = (self.next_b + 1) % self.cycle
-            x, slabs = self.inputs(b)
+            x, slabs = self.pending.result()
+            self.next_b = (self.next_b + 1) % w.batch
+            self.pending = self.pool.submit(self._inputs, self.next_b)
             t0 = time.perf_counter()
             O.fusion_stack_example(x, slabs, self.lws, w.n_heads, w.eps)
             dt = time.perf_counter() - t0
@@ -222,26 +247,45 @@ class OracleSampler:
                 self.toks += self.sample_tokens
             if t_run >= budget_s or (max_examples is not None and n >= max_examples):
                 break
+        if count:
+            self.step_s.append(t_run)
+        return t_run
+
+    def value(self) -> float:
+        w = self.w
+        if w.candidates:  # per-token cost: the sampled tokens share the K/V projections (as in serving)
+            return 1.0 / (self.t * (w.n_tokens / self.toks))
+        return self.done / self.t
 
     def summary(self, what: str) -> dict:
         w = self.w
         cores = len(os.sched_getaffinity(0))
         if w.candidates:
-            # per-token cost: the sampled tokens share the K/V projections (amortised as in serving)
-            value = 1.0 / (self.t * (w.n_tokens / self.toks))
             desc = f"{self.done} request(s), {self.sample_tokens} of {w.n_tokens} candidate tokens timed, scaled per request"
         else:
-            value = self.done / self.t
-            where = f"examples 0..{self.cycle - 1} in turn" if self.cycle < w.batch else "examples in batch order"
-            desc = f"{what}: {self.done} timed, {where} (all {w.n_layers} layers, all {w.n_tokens} tokens each)"
-        return {"value": value, "unit": "examples/s", "cores": cores, "kind": "oracle",
-                "sample": desc + f"; fp64 numpy, {self.t:.1f} s of CPU time"}
+            desc = (f"{what}: {self.done} examples timed, walking the batch in order from example 0 "
+                    f"(all {w.n_layers} layers, all {w.n_tokens} tokens each)")
+        return {"value": self.value(), "unit": "examples/s", "cores": cores, "kind": "oracle",
+                "sample": desc + f"; fp64 numpy on {cores} host threads, {self.t:.1f} s of oracle time"}
 
 
 def oracle_sample(w: I.Workload, budget_s: float = 15.0, max_examples: int = 64):
     s = OracleSampler(w)
     s.run(budget_s, max_examples=min(w.batch, max_examples))
-    return s.summary("first examples")
+    return s.summary("cpu baseline")
+
+
+def workload_config(w: I.Workload, total_L: int, max_L: int, world: int, args) -> dict:
+    """The `config` object of the JSON line (the same for both arms)."""
+    return {"workload": w.name, "batch": w.batch, "n_tokens": w.n_tokens, "d": w.d, "heads": w.n_heads,
+            "layers": w.n_layers, "total_L": int(total_L), "max_L": int(max_L),
+            "parallelism": f"dp{world} (independent examples per rank, no collective)",
+            "variant": ("shared K=V " if args.shared_kv else "") + ("tied gate" if args.tied_gate else "")
+                       or "separate W_K, W_V; untied up|gate",
+            "weights": ("gains folded per forward" if args.fold_per_call else
+                        "gains folded into the weights once at load (whale_prepare_weights)"),
+            "l2": "inputs larger than L2 (each layer reads its own "
+                  f"{total_L * w.d * 2 / 1e6:.0f} MB state slab), no flush"}
 
 
 # ------------------------------------------------------------------------------------------------
@@ -278,22 +322,22 @@ def run_reference(args):
     w = I.WORKLOADS[args.workload]
     t0 = time.time()
     steps = max(args.steps, 1)
-    sampler = OracleSampler(w, cycle=12)
+    sampler = OracleSampler(w)
     for _ in range(max(args.warmup, 0)):   # untimed: one example each
         sampler.run(0.0, count=False)
-    sampler.next_b = 0
     # the whole run is bounded: each step gets an equal share of --ref-total seconds of oracle time
-    # (at least one whole example), cycling over the batch's first 12 examples (inputs generated once)
+    # (at least one whole example), walking the batch in order from where the warm-up stopped
     per_step = max(0.2, args.ref_total / steps)
     for _ in range(steps):
         sampler.run(per_step)
-    cb = sampler.summary("oracle")
+    cb = sampler.summary("reference arm")
     value = cb["value"]
+    ms_step = 1e3 * statistics.mean(sampler.step_s)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "examples/s", "n_gpus": args.gpus,
-            "steps": steps, "warmup": max(args.warmup, 0), "ms_per_step": 1e3 * w.batch / value if value else None,
+            "steps": steps, "warmup": max(args.warmup, 0), "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "batch": w.batch, "n_tokens": w.n_tokens, "d": w.d, "heads": w.n_heads,
-                       "layers": w.n_layers},
+            "config": workload_config(w, int(sampler.L.sum()), int(sampler.L.max()), args.gpus, args),
+            "step": f"a bounded sample of the workload: {per_step:.1f} s of oracle time per step, whole examples",
             "cpu_baseline": cb, "e2e": {"value": value, "unit": "examples/s", "h2d_bytes_per_step": 0,
                                         "d2h_bytes_per_step": 0},
             "wall_s": time.time() - t0}
@@ -368,7 +412,7 @@ def main():
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--ref-budget", type=float, default=15.0, help="oracle seconds of the cpu_baseline sample")
-    ap.add_argument("--ref-total", type=float, default=150.0,
+    ap.add_argument("--ref-total", type=float, default=90.0,
                     help="oracle seconds of the whole --impl reference run, split across its steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-case", choices=["kv", "attn", "ffn", "fusion", "absorbed"], default=None,
@@ -421,6 +465,7 @@ def main():
         ev1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
+    clocks = clk.summary()
     ms = ev0.elapsed_time(ev1) / args.steps
     ms = max_over_ranks(ms, world)
     value = world * w.batch / (ms / 1e3)
@@ -482,67 +527,58 @@ def main():
     if absorbed:
         torch.cuda.synchronize()
         t_abs = timed(absorbed_step, reps)
-        abs_tflops = work["attention_absorbed"]["flops"] / (t_abs * 1e-3) / 1e12
         abs_traffic = None
-        passa_traffic_known = w.d == 512 and not args.shared_kv and os.environ.get("WHALE_ABS_FUSED", "0") != "1"
+        passa_traffic_known = w.d == 512 and not args.shared_kv
         if passa_traffic_known and ABS_TRAFFIC_BYTES_PER_ROW_D512 is not None:
             abs_traffic = ABS_TRAFFIC_BYTES_PER_ROW_D512 * total_L
         call = {"entry_point": "whale_attend_states (qa GEMM, pass A, pass B, merge, W_V GEMM, unit starts)",
-                "tflops": abs_tflops, "frac": abs_tflops / peaks["bf16_tflops"], "avg_call_ms": t_abs,
+                **roofline_of(work["attention_absorbed"]["flops"], work["attention_absorbed"]["bytes"], t_abs,
+                              tensor_peak(peaks, clocks)[0], peaks["hbm_gbs"]), "avg_call_ms": t_abs,
                 "algorithmic_flops": work["attention_absorbed"]["flops"],
                 "algorithmic_bytes": work["attention_absorbed"]["bytes"], "traffic": abs_traffic,
                 "traffic_source": "ncu dram bytes of the six kernels of one call at the full batch, per row"}
         pa = next((v for k, v in kernels.items() if k.split("<")[0] == "abs_scores_kernel"), None)
+        tc_peak, tc_src = tensor_peak(peaks, clocks)
         if pa:
             # the dominant kernel, pass A: S = qa H^T of N*h queries against every history row
-            # (2 (N h) d FLOP per row) with the softmax; its ncu DRAM bytes per row scaled by rows
+            # (2 (N h) d FLOP per row) with the softmax, reading the states once (2 d bytes per row);
+            # its ncu DRAM bytes per row scaled by rows
             fa = 2.0 * w.n_tokens * w.n_heads * total_L * w.d
+            ba = 2.0 * total_L * w.d
             ta = pa["avg_ms"]
-            a_tflops = fa / (ta * 1e-3) / 1e12
             a_traffic = (ABS_PASSA_BYTES_PER_ROW_D512 * total_L
                          if passa_traffic_known and ABS_PASSA_BYTES_PER_ROW_D512 is not None else None)
-            # Timed inside the long step, so the sustained tensor peak is the denominator; against
-            # it the FLOP time exceeds the time of the algorithmic bytes (the states read once).
-            sus = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-            ba = 2.0 * total_L * w.d
-            t_flop, t_byte = fa / (sus * 1e12), ba / (peaks["hbm_gbs"] * 1e9)
             roof = {"kernel": "abs_scores_kernel (absorbed pass A: scores on tcgen05 2-SM, online softmax, weights)",
-                    "bound": "tensor" if t_flop >= t_byte else "hbm", "achieved": a_tflops, "peak": sus,
-                    "unit": "TFLOP/s", "frac": a_tflops / sus, "traffic": a_traffic,
+                    **roofline_of(fa, ba, ta, tc_peak, peaks["hbm_gbs"]), "traffic": a_traffic,
                     "traffic_source": "ncu dram bytes of one launch at the full batch, per row",
-                    "frac_of_burst": a_tflops / peaks["bf16_tflops"],
-                    "hbm_frac": ba / (ta * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                    "algorithmic_per_launch": fa, "algorithmic_bytes_per_launch": ba,
+                    "algorithmic_flops_per_launch": fa, "algorithmic_bytes_per_launch": ba,
                     "avg_launch_ms": ta, "timing": "library per-kernel events on the bench stream",
-                    "peak_source": f"{peak_src} bf16 sustained (kernel timed inside the step loop)", "call": call}
+                    "peak_source": f"{peak_src}: {tc_src}; HBM copy {peaks['hbm_gbs']} GB/s", "call": call}
         else:
-            roof = {"kernel": "whale_attend_states (the absorbed S2 + S3 call)", "bound": "tensor",
-                    "achieved": abs_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                    "frac": abs_tflops / peaks["bf16_tflops"], "traffic": abs_traffic,
-                    "algorithmic_per_launch": work["attention_absorbed"]["flops"], "avg_launch_ms": t_abs,
-                    "peak_source": f"{peak_src} bf16 burst", "call": call}
+            roof = {"kernel": "whale_attend_states (the absorbed S2 + S3 call)",
+                    **roofline_of(work["attention_absorbed"]["flops"], work["attention_absorbed"]["bytes"], t_abs,
+                                  tc_peak, peaks["hbm_gbs"]), "traffic": abs_traffic,
+                    "algorithmic_flops_per_launch": work["attention_absorbed"]["flops"], "avg_launch_ms": t_abs,
+                    "peak_source": f"{peak_src}: {tc_src}", "call": call}
     else:
         kv_step(0)
         torch.cuda.synchronize()
         t_kv = timed(kv_step, reps)
         t_attn = timed(attn_step, reps)
-        kv_tflops = work["kv_proj"]["flops"] / (t_kv * 1e-3) / 1e12
-        attn_gbs = work["attention"]["bytes"] / (t_attn * 1e-3) / 1e9
         share_kv, share_attn = t_kv / layer_ms, t_attn / layer_ms
         kv_traffic = None
         if w.d == 512 and not args.shared_kv:
-            kv_traffic = KV_TRAFFIC_BYTES_PER_ROW_D512[
-                "1sm" if os.environ.get("WHALE_GEMM_1SM", "0") == "1" else "2sm"] * total_L
+            kv_traffic = KV_TRAFFIC_BYTES_PER_ROW_D512 * total_L
     if absorbed:
         pass
     elif share_kv >= share_attn:
-        roof = {"kernel": "K|V projection GEMM (tcgen05, RMSNorm row factor fused)", "bound": "tensor",
-                "achieved": kv_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": kv_tflops / peaks["bf16_tflops"], "traffic": kv_traffic,
-                "traffic_source": "ncu dram bytes of one launch on 109605 rows, scaled by rows",
-                "frac_of_sustained": kv_tflops / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
-                "algorithmic_per_launch": work["kv_proj"]["flops"], "avg_launch_ms": t_kv,
-                "peak_source": f"{peak_src} bf16 burst"}
+        tc_peak, tc_src = tensor_peak(peaks, clocks)
+        roof = {"kernel": "K|V projection GEMM (tcgen05, RMSNorm row factor fused)",
+                **roofline_of(work["kv_proj"]["flops"], work["kv_proj"]["bytes"], t_kv, tc_peak, peaks["hbm_gbs"]),
+                "traffic": kv_traffic, "traffic_source": "ncu dram bytes of one launch on 109605 rows, scaled by rows",
+                "algorithmic_flops_per_launch": work["kv_proj"]["flops"],
+                "algorithmic_bytes_per_launch": work["kv_proj"]["bytes"], "avg_launch_ms": t_kv,
+                "peak_source": f"{peak_src}: {tc_src}; HBM copy {peaks['hbm_gbs']} GB/s"}
     elif w.n_tokens >= 128:
         # many queries per history (the serving shape): the query-tiled tensor-core attention is
         # bound by its softmax exponentials. Peak = MUFU ex2 throughput: 16 per clock per SM x SMs x
@@ -556,14 +592,18 @@ def main():
                 "peak_source": "16 ex2/clk/SM x 148 SMs x max SM clock (nominal unit counts)",
                 "tensor_tflops": work["attention"]["flops"] / (t_attn * 1e-3) / 1e12}
     else:
-        roof = {"kernel": "split-L cross-attention + combine", "bound": "hbm", "achieved": attn_gbs,
-                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": attn_gbs / peaks["hbm_gbs"], "traffic": None,
-                "algorithmic_per_launch": work["attention"]["bytes"], "avg_launch_ms": t_attn,
-                "peak_source": f"{peak_src} HBM copy"}
+        tc_peak, tc_src = tensor_peak(peaks, clocks)
+        roof = {"kernel": "split-L cross-attention + combine",
+                **roofline_of(work["attention"]["flops"], work["attention"]["bytes"], t_attn, tc_peak,
+                              peaks["hbm_gbs"]), "traffic": None,
+                "algorithmic_flops_per_launch": work["attention"]["flops"],
+                "algorithmic_bytes_per_launch": work["attention"]["bytes"], "avg_launch_ms": t_attn,
+                "peak_source": f"{peak_src}: HBM copy {peaks['hbm_gbs']} GB/s; {tc_src}"}
     # roofline of the whole step: sum over kernels of max(flops / TC peak, bytes / HBM peak)
     t_star = 0.0
+    tc_step = tensor_peak(peaks, clocks)[0]
     for k, v in work.items():
-        t_star += max(v["flops"] / (peaks["bf16_tflops"] * 1e12), v["bytes"] / (peaks["hbm_gbs"] * 1e9))
+        t_star += max(v["flops"] / (tc_step * 1e12), v["bytes"] / (peaks["hbm_gbs"] * 1e9))
     t_star *= w.n_layers * 1e3
 
     # ---------------- end to end: host buffers through the C ABI, copies inside the timed region -----
@@ -599,23 +639,15 @@ def main():
             "metric": METRIC, "value": value, "unit": "examples/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) states and tokens, Xavier weights)",
-            "config": {"workload": w.name, "batch": w.batch, "n_tokens": w.n_tokens, "d": w.d, "heads": w.n_heads,
-                       "layers": w.n_layers, "total_L": total_L, "max_L": int(p.lengths.max()),
-                       "parallelism": f"dp{world} (independent examples per rank, no collective)",
-                       "variant": ("shared K=V " if args.shared_kv else "") + ("tied gate" if args.tied_gate else "")
-                                  or "separate W_K, W_V; untied up|gate",
-                       "weights": ("gains folded per forward" if args.fold_per_call else
-                                   "gains folded into the weights once at load (whale_prepare_weights)"),
-                       "l2": "inputs larger than L2 (each layer reads its own "
-                             f"{total_L * w.d * 2 / 1e6:.0f} MB state slab), no flush"},
+            "config": workload_config(w, total_L, int(p.lengths.max()), world, args),
             "roofline": roof,
             "step_roofline": {"t_star_ms": t_star, "frac": t_star / ms, "per_layer_ms": layer_ms,
                               "path": "absorbed" if absorbed else "materialized K|V",
                               "kv_proj_ms": t_kv, "attention_ms": t_attn, "absorbed_attention_ms": t_abs,
-                              "peaks": f"{peak_src}: {peaks['hbm_gbs']} GB/s, {peaks['bf16_tflops']} TFLOP/s"},
+                              "peaks": f"{peak_src}: {peaks['hbm_gbs']} GB/s, {tc_step} TFLOP/s"},
             "kernels": kernels,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": (len(recs) or launches_per_step(w, args.fold_per_call, absorbed)) * args.steps,
-            "clocks": clk.summary(),
+            "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -245,12 +245,15 @@ whale_status whale_attend_states(const whale_config* cfg, const void* q, const v
  * entry point takes no workspace: the attention partials live in one file-scope device array of
  * WHALE_NOALLOC_SCRATCH_BYTES (32 MiB) that every GPU which loads this library holds until the
  * process exits. It allocates nothing itself.
- *  - Limit: the partials of a call, (B * ceil(N / QB) + G) * n_heads * QB * (d_head + 2) * 4 bytes
+ *  - Limit: where the split-L kernel runs (fewer than 128 queries per example, or d_head not 32
+ *    or 64), its partials, (B * ceil(N / QB) + G) * n_heads * QB * (d_head + 2) * 4 bytes
  *    (QB = 16, 32 or 64 queries per block, G <= 148), must fit; a larger shape returns
  *    WHALE_ERR_WORKSPACE before any GPU work. The 15k-history stack (B 64, N 32, d 512, 8 heads)
- *    needs 14 MB; the 16384-query serving shape needs 28 MB.
- *  - The first call on a device looks up the array's device address (once per device, with that
- *    device current); make that first call before any stream capture.
+ *    needs 14 MB. Shapes with 128 or more queries per example and d_head 32 or 64 (the serving
+ *    shapes) take the query-tiled kernel, which keeps no partials: no limit applies to them.
+ *  - The first call in a CUDA context looks up the array's device address (once per context, with
+ *    that context's device current) and caches it under the context; make that first call before
+ *    any stream capture.
  *  - Every call shares the one array and overwrites it; nothing in it needs to start at zero (each
  *    partial is written before it is read within the same call). Calls whose kernels overlap on
  *    the GPU (other streams, other host threads) race on the array: serialise them.
@@ -259,6 +262,18 @@ whale_status whale_attend_states(const whale_config* cfg, const void* q, const v
 whale_status whale_cross_attention_noalloc(const whale_config* cfg, const void* q, const void* kv,
                                            const int* seq_offsets, void* a, const whale_shape_hint* hint,
                                            whale_stream_t stream);
+
+/* Failure detection. Every device-side wait of the library's kernels (a pipeline stage on an
+ * mbarrier, one CTA pair waiting for another's published results) gives up after a time limit
+ * (2 s in the kernels), records WHALE_DEVERR_TIMEOUT in the device error word and lets its kernel
+ * return instead of hanging the GPU; results of that call are then invalid, and the timeout is seen
+ * through whale_get_device_error (no entry point synchronises to check it on its own).
+ * whale_test_bounded_waits exercises that mechanism with no pipeline around it: it enqueues one
+ * small kernel whose two waits can never be satisfied (an mbarrier that no thread arrives on, a
+ * flag that no thread sets), each bounded by limit_ns (1 us .. 2 s, else WHALE_ERR_INVALID_ARG).
+ * Both give up after about limit_ns and record WHALE_DEVERR_TIMEOUT; the kernel returns and the
+ * context stays usable. No counterpart in the paper: a health check of the failure detection. */
+whale_status whale_test_bounded_waits(unsigned long long limit_ns, whale_stream_t stream);
 
 /* Synchronises `stream`, then reads and clears the device error word of the current
  * device (bits WHALE_DEVERR_*). Returns WHALE_ERR_DEVICE_CHECK if any bit was set. */

@@ -15,7 +15,7 @@ EXPECTED = {
     "whale_fusion_forward_host", "whale_fusion_layer_forward", "whale_project_queries", "whale_project_kv",
     "whale_cross_attention", "whale_fusion_mlp", "whale_swiglu_ffn", "whale_get_device_error",
     "whale_attend_states", "whale_prepare_weights", "whale_prepared_weights_size", "whale_cross_attention_noalloc",
-    "whale_profile_begin", "whale_profile_end",
+    "whale_profile_begin", "whale_profile_end", "whale_test_bounded_waits",
 }
 
 
@@ -25,6 +25,12 @@ def test_library_exports_every_declared_symbol():
     lib = ctypes.CDLL(W.LIB_PATH)
     for name in declared:
         assert hasattr(lib, name), name
+
+
+def test_bounded_wait_self_test_rejects_limits_out_of_range():
+    # 1 us .. 2 s; out-of-range limits are refused on the host before any launch
+    assert W.whale_test_bounded_waits(999, stream=0, raw=True) == 1
+    assert W.whale_test_bounded_waits(2_000_000_001, stream=0, raw=True) == 1
 
 
 def test_status_strings():

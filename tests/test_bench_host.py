@@ -79,9 +79,30 @@ def test_oracle_sampler_counts_whole_examples(bench):
     out = s.summary("first examples")
     assert out["unit"] == "examples/s" and out["kind"] == "oracle" and out["cores"] >= 1
     assert out["value"] == pytest.approx(s.done / s.t)
-    # the time budget ends a run (after one example at least); max_examples caps it
-    c = bench.OracleSampler(w, cycle=1)
+    # the time budget ends a run (after one example at least); max_examples caps it; the sampler
+    # walks the whole batch in order and starts again at example 0
+    c = bench.OracleSampler(w)
     c.run(60.0, max_examples=3)
-    assert c.done == 3 and list(c.cache) == [0]  # cycling over example 0 reuses its inputs
+    assert c.done == 3 and c.next_b == 3 % w.batch
+    assert len(c.step_s) == 1 and c.step_s[0] == pytest.approx(c.t)
     c.run(60.0, max_examples=2, count=False)  # an untimed warm-up run leaves the counts alone
-    assert c.done == 3
+    assert c.done == 3 and len(c.step_s) == 1
+
+
+def test_roofline_bound_is_the_larger_algorithmic_time(bench):
+    # pass A at the 15k-history batch: 105.8 GFLOP and 413 MB in 129.9 us against the burst figures
+    fa, ba = 2.0 * 256 * 403481 * 512, 2.0 * 403481 * 512
+    r = bench.roofline_of(fa, ba, 0.1299, 1717.8, 6456.5)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert r["frac"] == pytest.approx(ba / 6456.5e9 / 129.9e-6)
+    assert r["achieved"] / r["peak"] == pytest.approx(r["frac"])
+    # against the sustained figure the FLOP time is the larger one
+    r2 = bench.roofline_of(fa, ba, 0.1299, 1424.0, 6456.5)
+    assert r2["bound"] == "tensor" and r2["frac"] == pytest.approx(fa / 1424e12 / 129.9e-6)
+
+
+def test_tensor_peak_follows_the_sampled_clock(bench):
+    peaks = {"bf16_tflops": 1717.8, "bf16_tflops_sustained": 1424.0, "sm_max_mhz": 1965.0, "hbm_gbs": 6456.5}
+    assert bench.tensor_peak(peaks, {"sm_mhz": 1965.0})[0] == 1717.8
+    assert bench.tensor_peak(peaks, {"sm_mhz": 1372.0})[0] == 1424.0
+    assert bench.tensor_peak(peaks, None)[0] == 1717.8

@@ -3,8 +3,7 @@ oracle, through whale_fusion_forward: ragged lengths around the 256-row unit (1,
 513), empty histories, batches whose examples are split across CTA pairs and pairs holding many
 short examples, histories whose later rows raise pass A's softmax reference (so pass B rescales
 its accumulator), both widths the path takes (d = 512 with 8 heads, d = 256 with 4 heads), shared
-K = V, prepared weights, agreement with the materialising path, and the four-CTA-cluster kernel
-that runs both passes at once (WHALE_ABS_FUSED=1)."""
+K = V, prepared weights and agreement with the materialising path."""
 import numpy as np
 import pytest
 import torch
@@ -157,50 +156,6 @@ def test_absorbed_deterministic_and_all_empty():
     out0 = Hn.run_forward(p0)
     torch.cuda.synchronize()
     _oracle_check(p0, out0)
-
-
-# ------------------------------------------------------------------------------------------
-# the four-CTA-cluster kernel (WHALE_ABS_FUSED=1): both passes in one launch
-# ------------------------------------------------------------------------------------------
-@pytest.fixture
-def fused(monkeypatch):
-    monkeypatch.setenv("WHALE_ABS_FUSED", "1")
-
-
-@pytest.mark.parametrize("d", [512, 256])
-def test_fused_kernel_ragged_and_short_units(fused, d):
-    # one-chunk units in a row (lengths 1..64) make segment ends follow each other unit by unit
-    L = np.array([1, 255, 256, 257, 0, 513, 1800, 40, 3, 64, 65, 1, 2, 700])
-    w = _workload(d, len(L))
-    p = Hn.build_problem(w, gains="random", lengths=L)
-    out = Hn.run_forward(p)
-    torch.cuda.synchronize()
-    _oracle_check(p, out)
-
-
-def test_fused_kernel_many_ranges_and_reference_raised(fused):
-    w = _workload(512, 40, n_layers=2).replace(lengths=("uniform", 1, 2500))
-    L = I.draw_lengths(w)
-    L[7] = 0
-    p = Hn.build_problem(w, gains="random", lengths=L)
-    _scale_query_gain(p, 2.0)
-    out = Hn.run_forward(p)
-    torch.cuda.synchronize()
-    _oracle_check(p, out, examples=[0, 7, 13, 21, 39])
-    # deterministic: a second run gives bitwise the same output
-    again = Hn.run_forward(p)
-    torch.cuda.synchronize()
-    assert torch.equal(out, again)
-
-
-def test_fused_kernel_agrees_with_two_passes(monkeypatch):
-    w = _workload(512, 6).replace(lengths=("uniform", 200, 4000))
-    p = Hn.build_problem(w, gains="random")
-    two = Hn.run_forward(p).clone().float()
-    monkeypatch.setenv("WHALE_ABS_FUSED", "1")
-    one = Hn.run_forward(p).clone().float()
-    torch.cuda.synchronize()
-    assert bool(((one - two).abs() <= 2e-2 * (1 + two.abs())).all())
 
 
 def _states_host(p, b):

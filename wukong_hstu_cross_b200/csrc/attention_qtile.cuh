@@ -55,7 +55,7 @@ constexpr float kQtLazy = 8.0f;  // log2 headroom before the softmax reference i
 
 // 2^x on the FMA pipe, for x <= kQtLazy: Cody-Waite reduction x = n + f with n = round(x) (the
 // 1.5 * 2^23 rounding trick) and f in [-1/2, 1/2]; 2^f by a degree-3 polynomial fitted to minimise
-// the relative error on that interval (max relative error 7.5e-5, below the 2^-9 of the bf16
+// the relative error on that interval (max relative error 7.51e-5, below the 2^-9 of the bf16
 // weights it produces); 2^n added to the exponent bits. Arguments below -125 give 2^-125 (no
 // denormals or exponent wrap; used only for blocks without masked rows). Takes a share of the
 // exponentials off the MUFU unit.

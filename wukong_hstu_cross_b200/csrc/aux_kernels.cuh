@@ -1,4 +1,5 @@
-// aux_kernels.cuh — weight preparation for the bf16 path and the debug offset check.
+// aux_kernels.cuh — weight preparation for the bf16 path, the debug offset check and the self-test
+// of the bounded device waits.
 #pragma once
 
 #include "ptx.cuh"
@@ -86,6 +87,25 @@ __global__ void check_offsets_kernel(const int* __restrict__ off, int B, int max
     if (b == B) bad = bad || (long long)off[B] > total_L;
     if (bad) atomicOr(&g_device_error, kErrOffsets);
   }
+}
+
+// Self-test of the bounded waits every pipeline here relies on (mbar_wait, wait_nonzero_gpu):
+// thread 0 waits on an mbarrier that no thread arrives on, thread 32 on a word in global memory that
+// no thread sets, each for at most limit_ns. Both waits give up, record kErrTimeout in
+// g_device_error and return; the kernel then exits normally (nothing else is in flight).
+__device__ int g_wait_test_flag;  // never written by any kernel: stays 0
+__global__ void wait_selftest_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, &abort_flag, limit_ns);
+  if (threadIdx.x == 32) (void)wait_nonzero_gpu(&g_wait_test_flag, limit_ns);
+  __syncthreads();
 }
 
 }  // namespace whale

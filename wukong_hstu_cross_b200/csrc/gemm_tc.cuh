@@ -420,211 +420,3 @@ __global__ void pair_from_bf16_kernel(const __nv_bfloat16* __restrict__ x, float
 }
 
 }  // namespace whale
-
-namespace whale {
-
-// ================================================================================================
-// Split-K variant for the residual-epilogue GEMMs with a long K (Fusion GEMM 2, K = 2d; the down
-// projection, K = 4d): a cluster of KS = 4 or 8 CTAs shares one 128 x 256 output tile, CTA r
-// accumulating K blocks [r KB/KS, (r+1) KB/KS) of hi/lo operand pairs into TMEM. Each CTA then puts
-// its fp32 partial into its (now idle) stage memory; after a cluster barrier CTA r sums columns
-// [r 256/KS, (r+1) 256/KS) of the KS partials in rank order (the result does not depend on timing)
-// through distributed shared memory, adds the fp32 residual (loaded into registers while the MMAs
-// run) and writes the outputs. With 128 x 64
-// tiles each k-step of these GEMMs needs 40 KB of operands per 0.18 us of MMA, more than one SM
-// streams from L2; here a k-step is 64 KB per 0.72 us.
-// ================================================================================================
-struct SplitKSmem {
-  static constexpr uint32_t A_BYTES = 128 * 64 * 2;
-  static constexpr uint32_t B_BYTES = 256 * 64 * 2;
-  static constexpr uint32_t STAGE = 2 * A_BYTES + B_BYTES;  // A hi | A lo | W
-  static constexpr int STAGES = 3;
-  static constexpr int PSTRIDE = 256 + 4;                   // floats per partial row (bank spread)
-  static_assert(128 * PSTRIDE * 4 <= STAGES * (int)STAGE, "the partial fits in the stage memory");
-  static constexpr size_t BYTES = 1024 + STAGES * (size_t)STAGE + 256;
-};
-
-// (No memory clobber, so several of these can be in flight at once; they are ordered after the
-// cluster barrier, itself volatile asm, that publishes the partials.)
-__device__ __forceinline__ float4 ld_shared_cluster_v4(uint32_t cluster_addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(cluster_addr));
-  return v;
-}
-
-template <int KS>
-__global__ void __launch_bounds__(192, 1)
-    gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAlo,
-                       const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
-  using L = SplitKSmem;
-  constexpr int ST = L::STAGES;
-  constexpr int BN = 256;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * L::STAGE);
-  uint64_t* empty = full + ST;
-  uint64_t* tfull = empty + ST;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tfull + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* part = reinterpret_cast<float*>(smem);  // after the mainloop: [128][PSTRIDE] fp32
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kr = (int)cluster_ctarank();
-  const int tile = blockIdx.x / KS;
-  const int m0 = (tile / args.tiles_n) * 128, n0 = (tile % args.tiles_n) * BN;
-  const int KBc = args.kb0 / KS;
-  const int kb_begin = kr * KBc;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < ST; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    mbar_init(tfull, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-    fence_proxy_async_smem();
-  }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmAlo);
-    tma_prefetch_desc(&tmB);
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, BN);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-  pdl_wait();
-  pdl_trigger();
-
-  bool ok = true;
-  if (warp == 0) {
-    if (lane == 0) {
-      for (int i = 0; i < KBc; ++i) {
-        const int s = i % ST;
-        if (i >= ST && !mbar_wait(&empty[s], (i / ST - 1) & 1, abort_flag)) break;
-        uint8_t* st = smem + s * L::STAGE;
-        mbar_arrive_expect_tx(&full[s], L::STAGE);
-        const int kc = (kb_begin + i) * 64;
-        tma_load_2d(st, &tmA, kc, m0, &full[s]);
-        tma_load_2d(st + L::A_BYTES, &tmAlo, kc, m0, &full[s]);
-        tma_load_2d(st + 2 * L::A_BYTES, &tmB, kc, n0, &full[s]);
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
-      for (int i = 0; i < KBc; ++i) {
-        const int s = i % ST;
-        if (!mbar_wait(&full[s], (i / ST) & 1, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t a_base = smem_u32(smem + s * L::STAGE);
-        const uint32_t b_base = a_base + 2 * L::A_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bdesc = sdesc_k_sw128(b_base + kk * 32);
-          umma_f16(tmem_base, sdesc_k_sw128(a_base + kk * 32), bdesc, idesc, (i > 0 || kk > 0) ? 1u : 0u);
-          umma_f16(tmem_base, sdesc_k_sw128(a_base + L::A_BYTES + kk * 32), bdesc, idesc, 1u);
-        }
-        umma_commit(&empty[s]);
-      }
-      umma_commit(tfull);  // also on abort: arrives once every issued MMA is done
-    }
-  }
-  // This CTA reduces columns [kr NC, kr NC + NC) of the tile; the epilogue threads load their row's
-  // residual for them into registers while the MMAs run.
-  constexpr int NC = BN / KS;
-  static_assert(KS == 4 || KS == 8, "the residual of NC columns is held in registers");
-  float4 rres[NC / 4];
-  if (warp >= 2) {
-    const long long gm = (long long)m0 + (warp & 3) * 32 + lane;
-    if (gm < args.M) {
-      const float4* rp = reinterpret_cast<const float4*>(args.resid32 + gm * args.ldr + n0 + kr * NC);
-#pragma unroll
-      for (int i = 0; i < NC / 4; ++i) rres[i] = rp[i];
-    }
-  }
-  if (warp >= 2) {
-    // epilogue warps 2..5: thread i of quadrant q owns row 32 q + i; the accumulator -> own partial
-    const int q = warp & 3;
-    const int row = q * 32 + lane;
-    ok = mbar_wait(tfull, 0, abort_flag);
-    if (ok) {
-      tc_fence_after();
-      const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16);
-      float* prow = part + row * L::PSTRIDE;
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(t_row + c * 32, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          *reinterpret_cast<float4*>(prow + c * 32 + 4 * i) =
-              make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]), __uint_as_float(v[4 * i + 2]),
-                          __uint_as_float(v[4 * i + 3]));
-      }
-    }
-  }
-  tc_fence_before();
-  cluster_sync_all();  // every partial of the cluster is in shared memory
-  if (warp >= 2 && ok && !*abort_flag) {
-    const int q = warp & 3;
-    const int row = q * 32 + lane;
-    const long long gm = (long long)m0 + row;
-    const int c0 = kr * NC;
-    const uint32_t base = smem_u32(part) + (uint32_t)(row * L::PSTRIDE * 4);
-#pragma unroll
-    for (int g = 0; g < NC / 8; ++g) {
-      const int c = c0 + 8 * g;
-      // all KS partial chunks in flight first (remote loads), then summed in rank order (the sum
-      // does not depend on timing)
-      float4 pv[KS][2];
-#pragma unroll
-      for (int r = 0; r < KS; ++r) {
-        const uint32_t src = mapa_shared(base + (uint32_t)(c * 4), (uint32_t)r);
-        pv[r][0] = ld_shared_cluster_v4(src);
-        pv[r][1] = ld_shared_cluster_v4(src + 16);
-      }
-      float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int r = 0; r < KS; ++r) {
-        const float4 v0 = pv[r][0], v1 = pv[r][1];
-        x[0] += v0.x;
-        x[1] += v0.y;
-        x[2] += v0.z;
-        x[3] += v0.w;
-        x[4] += v1.x;
-        x[5] += v1.y;
-        x[6] += v1.z;
-        x[7] += v1.w;
-      }
-      if (gm < args.M) {
-        const int col = n0 + c;
-        const float4 r0 = rres[2 * g], r1 = rres[2 * g + 1];
-        x[0] += r0.x;
-        x[1] += r0.y;
-        x[2] += r0.z;
-        x[3] += r0.w;
-        x[4] += r1.x;
-        x[5] += r1.y;
-        x[6] += r1.z;
-        x[7] += r1.w;
-        store_row_chunk<8>(args, gm * args.ldo + col, x);
-      }
-    }
-  }
-  cluster_sync_all();  // no CTA leaves while a peer may still read its partial
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem_base, BN);
-  }
-}
-
-}  // namespace whale

@@ -69,7 +69,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Wait until the phase with the given parity has completed. Bounded: after kWaitLimitNs
 // (or as soon as *abort is raised by another thread of the CTA) it records the error
 // and returns false so the caller can unwind instead of hanging the GPU.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
@@ -77,7 +78,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       atomicOr(&g_device_error, kErrTimeout);
       *abort = 1;
       return false;
@@ -263,12 +264,12 @@ __device__ __forceinline__ int ld_shared_cluster_s32(uint32_t cluster_addr) {
 }
 // Bounded wait (gpu-scope acquire) for a word that another CTA publishes with a gpu-scope release:
 // its nonzero value, or 0 once kWaitLimitNs has passed (then g_device_error has kErrTimeout).
-__device__ __forceinline__ int wait_nonzero_gpu(const int* p) {
+__device__ __forceinline__ int wait_nonzero_gpu(const int* p, uint64_t limit_ns = kWaitLimitNs) {
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     const int v = ld_acquire_gpu(p);
     if (v != 0) return v;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       atomicOr(&g_device_error, kErrTimeout);
       return 0;
     }

@@ -27,14 +27,11 @@
 #include <vector>
 
 #include "absorbed.cuh"
-#include "absorbed_fused.cuh"
 #include "aux_kernels.cuh"
 #include "attention.cuh"
 #include "attention_qtile.cuh"
 #include "fp32_path.cuh"
 #include "gemm_2sm.cuh"
-#include "gemm_pair.cuh"
-#include "gemm_persistent.cuh"
 #include "gemm_tc.cuh"
 #include "ptx.cuh"
 
@@ -57,40 +54,6 @@ namespace {
   } while (0)
 
 constexpr int kNumSM = 148;
-// The 2-SM (cta_group::2) K|V GEMM is the default; WHALE_GEMM_1SM=1 in the environment selects the
-// one-SM persistent kernel instead (read per call; comparison runs and tests).
-inline bool gemm_2sm_enabled() {
-  const char* e = std::getenv("WHALE_GEMM_1SM");
-  return !(e && e[0] == '1');
-}
-// The absorbed attention runs its two passes as two kernels by default; WHALE_ABS_FUSED=1 in the
-// environment selects the four-CTA-cluster kernel that runs both at once (absorbed_fused.cuh; it
-// reads each history row from HBM once, but its scorer pair is bound by the softmax, and it is
-// slower on the 15k-history workload). Read per call (comparison runs and tests).
-// Histories attended by many queries (N >= 128 per example) take the query-tiled tcgen05 kernel;
-// WHALE_ATTN_SPLITL=1 in the environment keeps the split-L kernel for them (comparison runs, tests).
-inline bool qtile_enabled() {
-  const char* e = std::getenv("WHALE_ATTN_SPLITL");
-  return !(e && e[0] == '1');
-}
-// WHALE_GEMM_SPLITK=1 in the environment runs the residual-epilogue GEMMs with a long K split-K
-// across a cluster (gemm_splitk_kernel). Off by default: on the 2048-row token batch it measured
-// slower than one CTA per 128 x 64 tile (3.45-3.50 against 3.39-3.41 ms per 8-layer step).
-inline bool splitk_enabled() {
-  const char* e = std::getenv("WHALE_GEMM_SPLITK");
-  return e && e[0] == '1';
-}
-// WHALE_GEMM_PAIR=1 in the environment runs the token-side GEMMs with hi/lo operand pairs on CTA
-// pairs (gemm_pair.cuh). Off by default: on the 2048-row token batch it measured no faster than
-// one CTA per tile (step 3.19-3.22 against 3.20-3.21 ms; Fusion GEMM 1 slower, up|gate even).
-inline bool gemm_pair_enabled() {
-  const char* e = std::getenv("WHALE_GEMM_PAIR");
-  return e && e[0] == '1';
-}
-inline bool abs_fused_enabled() {
-  const char* e = std::getenv("WHALE_ABS_FUSED");
-  return e && e[0] == '1';
-}
 constexpr size_t kAlign = 256;
 inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 template <class T>
@@ -98,13 +61,8 @@ inline T cdiv(T a, T b) { return (a + b - 1) / b; }
 
 // ------------------------------------------------------------------------------------------
 // Launch with programmatic dependent launch (PDL): the kernel may start while the previous kernel
-// of the stream drains; it waits (griddepcontrol.wait) before touching global memory. Plain
-// launches when WHALE_NO_PDL=1 is set (comparison runs).
+// of the stream drains; it waits (griddepcontrol.wait) before touching global memory.
 // ------------------------------------------------------------------------------------------
-inline bool pdl_enabled() {
-  const char* e = std::getenv("WHALE_NO_PDL");
-  return !(e && e[0] == '1');
-}
 
 // Per-kernel timing (whale_profile_begin / whale_profile_end): while on, every kernel launched by
 // launch_pdl is followed by an event on its stream (the first one also by a start event). The
@@ -151,7 +109,7 @@ whale_status launch_cluster_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, s
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl_enabled() ? 2 : 1;
+  cfg.numAttrs = 2;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
   if (g_prof_on) prof_record(reinterpret_cast<const void*>(kern), st, false);
   CUCHECK(e);
@@ -178,7 +136,7 @@ whale_status launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sm
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  cfg.numAttrs = 1;
   CUCHECK(cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...));
   return WHALE_OK;
 }
@@ -431,59 +389,6 @@ whale_status launch_gemm_t(const CUtensorMap* tm, const GemmArgs& g, long long t
   return launch_pdl(kern, dim3(grid), dim3(gemm_threads<RN>()), smem, st, tm[0], tm[1], tm[2], tm[3], tm[4], g);
 }
 
-// Co-resident two-CTA clusters of a pair kernel (cached per kernel and device).
-whale_status pair_max_clusters(const void* kern, size_t smem, int threads, int* clusters) {
-  static std::mutex mu;
-  static std::vector<std::pair<std::pair<const void*, int>, int>> cache;
-  int dev = 0;
-  CUCHECK(cudaGetDevice(&dev));
-  std::lock_guard<std::mutex> lk(mu);
-  for (const auto& e : cache)
-    if (e.first.first == kern && e.first.second == dev) {
-      *clusters = e.second;
-      return e.second > 0 ? WHALE_OK : WHALE_ERR_UNSUPPORTED;
-    }
-  cudaLaunchConfig_t lc = {};
-  lc.gridDim = dim3(kNumSM, 1, 1);
-  lc.blockDim = dim3(threads, 1, 1);
-  lc.dynamicSmemBytes = smem;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  lc.attrs = attr;
-  lc.numAttrs = 1;
-  int n = 0;
-  CUCHECK(cudaOccupancyMaxActiveClusters(&n, kern, &lc));
-  n = std::min(n, kNumSM / 2);
-  cache.push_back({{kern, dev}, n > 0 ? n : -1});
-  *clusters = n;
-  return n > 0 ? WHALE_OK : WHALE_ERR_UNSUPPORTED;
-}
-
-template <int BN, int EPI, bool RN>
-whale_status launch_pair_t(const CUtensorMap* tm, const GemmArgs& g, cudaStream_t st) {
-  const size_t smem = PairSmem<BN>::BYTES;
-  auto kern = gemm_pair_kernel<BN, EPI, RN>;
-  CUCHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  int pairs = 0;
-  WCHECK(pair_max_clusters(reinterpret_cast<const void*>(kern), smem, pair_threads<RN>(), &pairs));
-  const long long np = std::min<long long>(g.num_tiles, pairs);
-  return launch_pdl(kern, dim3((unsigned)(2 * np)), dim3(pair_threads<RN>()), smem, st, tm[0], tm[1], tm[2], tm[3],
-                    tm[4], g);
-}
-
-template <int BN>
-whale_status launch_pair_bn(int epi, bool rn, const CUtensorMap* tm, const GemmArgs& g, cudaStream_t st) {
-  if (rn && epi == EPI_STORE) return launch_pair_t<BN, EPI_STORE, true>(tm, g, st);
-  if (rn && epi == EPI_SWIGLU) return launch_pair_t<BN, EPI_SWIGLU, true>(tm, g, st);
-  if (rn && epi == EPI_SWIGLU_TIED) return launch_pair_t<BN, EPI_SWIGLU_TIED, true>(tm, g, st);
-  if (!rn && epi == EPI_SILU) return launch_pair_t<BN, EPI_SILU, false>(tm, g, st);
-  if (!rn && epi == EPI_RESID) return launch_pair_t<BN, EPI_RESID, false>(tm, g, st);
-  return WHALE_ERR_UNSUPPORTED;
-}
-
 template <int BN>
 whale_status launch_gemm_bn(int epi, bool rn, bool split, const CUtensorMap* tm, const GemmArgs& g, long long tiles,
                             cudaStream_t st) {
@@ -495,16 +400,6 @@ whale_status launch_gemm_bn(int epi, bool rn, bool split, const CUtensorMap* tm,
   if (!rn && epi == EPI_SILU) return launch_gemm_t<BN, EPI_SILU, false, true>(tm, g, tiles, st);
   if (!rn && epi == EPI_RESID) return launch_gemm_t<BN, EPI_RESID, false, true>(tm, g, tiles, st);
   return WHALE_ERR_UNSUPPORTED;
-}
-
-template <int BN>
-whale_status launch_persistent_t(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
-                                 const PGemmArgs& g, cudaStream_t st) {
-  const size_t smem = PGemmSmem<BN>::BYTES;
-  auto kern = gemm_rownorm_persistent_kernel<BN>;
-  CUCHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  const int grid = g.num_tiles < kNumSM ? g.num_tiles : kNumSM;
-  return launch_pdl(kern, dim3(grid), dim3(kPGemmThreads), smem, st, ta, tb, to, g);
 }
 
 // Co-resident 2-CTA clusters of the 2-SM GEMM on the current device (cached per device).
@@ -558,26 +453,6 @@ whale_status gemm_rownorm_2sm(const Opnd& a0, const void* W, int N, const Outs& 
   return launch_pdl(kern, dim3(2 * pairs), dim3(kG2Threads), G2Smem::BYTES, st, ta, tb, to, g);
 }
 
-// out = r(A) * (A W^T) in bf16, persistent over 128 x BN tiles (BN = 256 when N allows).
-whale_status gemm_rownorm_persistent(const Opnd& a0, const void* W, int N, const Outs& out, long long M, float eps,
-                                     cudaStream_t st) {
-  const int bn = (N % 256 == 0) ? 256 : 128;
-  CUtensorMap ta, tb, to;
-  WCHECK(tmap_bf16(&ta, a0.hi, M, a0.K, a0.ld, 128));
-  WCHECK(tmap_bf16(&tb, W, N, a0.K, a0.K, bn));
-  WCHECK(tmap_bf16(&to, out.hi, M, N, out.ld, 32));
-  PGemmArgs g{};
-  g.M = (int)M;
-  g.N = N;
-  g.kb = a0.K / 64;
-  g.tiles_n = N / bn;
-  g.num_tiles = (int)(cdiv<long long>(M, 128) * g.tiles_n);
-  g.inv_k = 1.0f / (float)a0.K;
-  g.eps = eps;
-  if (bn == 256) return launch_persistent_t<256>(ta, tb, to, g, st);
-  return launch_persistent_t<128>(ta, tb, to, g, st);
-}
-
 // out = epi([A0 | A1] W^T), W [N, K0+K1] bf16; SPLIT when the operands carry lo halves.
 whale_status gemm_bf16(const Opnd& a0, const Opnd& a1, const void* W, int N, const Outs& out, const float* resid32,
                        long long ldr, long long M, int epi, bool rn, float eps, cudaStream_t st) {
@@ -586,93 +461,13 @@ whale_status gemm_bf16(const Opnd& a0, const Opnd& a1, const void* W, int N, con
   const bool split = a0.lo != nullptr;
   if (a0.K % 64 || a1.K % 64 || N % 64 || (a1.K > 0 && (a1.lo != nullptr) != split)) return WHALE_ERR_UNSUPPORTED;
   const long long tm = cdiv<long long>(M, 128);
-  // Large single-source row-norm projections (the history-side K|V GEMM): persistent kernel.
+  // Large single-source row-norm projections (the history-side K|V GEMM): the 2-SM persistent kernel
+  // (256 x 256 tiles on CTA pairs) where N allows; otherwise the one-CTA kernel below.
   if (!split && rn && epi == EPI_STORE && a1.K == 0 && out.hi && !out.lo && !out.f32 && N % 128 == 0 &&
       tm * (N / 128) >= 2 * kNumSM) {
     int pairs = 0;
-    if (N % 256 == 0 && gemm_2sm_enabled()) WCHECK(g2_max_pairs(&pairs));
+    if (N % 256 == 0) WCHECK(g2_max_pairs(&pairs));
     if (pairs > 0) return gemm_rownorm_2sm(a0, W, N, out, M, eps, pairs, st);
-    return gemm_rownorm_persistent(a0, W, N, out, M, eps, st);
-  }
-  // Residual epilogue, one hi/lo source, long K: split-K across a cluster of KS CTAs per 128 x 256 tile.
-  if (epi == EPI_RESID && split && a1.K == 0 && !rn && N % 256 == 0 && splitk_enabled()) {
-    const int KBs = a0.K / 64;
-    const long long tiles = tm * (N / 256);
-    int ks = 1;
-    for (int c : {4, 8})
-      if (KBs % c == 0 && KBs / c >= 4 && tiles * c <= kNumSM) ks = c;
-    if (ks > 1) {
-      CUtensorMap ta, tl, tb;
-      WCHECK(tmap_bf16(&ta, a0.hi, M, a0.K, a0.ld, 128));
-      WCHECK(tmap_bf16(&tl, a0.lo, M, a0.K, a0.ld, 128));
-      WCHECK(tmap_bf16(&tb, W, N, a0.K, a0.K, 256));
-      GemmArgs g{};
-      g.M = (int)M;
-      g.N = N;
-      g.kb0 = KBs;
-      g.tiles_n = N / 256;
-      g.num_tiles = (int)tiles;
-      g.out_hi = static_cast<__nv_bfloat16*>(out.hi);
-      g.out_lo = static_cast<__nv_bfloat16*>(out.lo);
-      g.out32 = out.f32;
-      g.ldo = out.ld;
-      g.resid32 = resid32;
-      g.ldr = ldr;
-      const dim3 grid((unsigned)(tiles * ks));
-      if (ks == 4) {
-        CUCHECK(cudaFuncSetAttribute(gemm_splitk_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)SplitKSmem::BYTES));
-        return launch_cluster_pdl(gemm_splitk_kernel<4>, grid, dim3(192), SplitKSmem::BYTES, st, 4u, ta, tl, tb, g);
-      }
-      CUCHECK(cudaFuncSetAttribute(gemm_splitk_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)SplitKSmem::BYTES));
-      return launch_cluster_pdl(gemm_splitk_kernel<8>, grid, dim3(192), SplitKSmem::BYTES, st, 8u, ta, tl, tb, g);
-    }
-  }
-  // hi/lo operand pairs: 256-row tiles on CTA pairs, each SM streaming half of the W tile. Tile
-  // width by the cost model below with pairs as the persistent unit and the per-SM streaming rate
-  // the per-CTA timelines show (~43 B/clk).
-  if (split && M > 128 && gemm_pair_enabled() &&
-      (rn ? (epi == EPI_STORE || epi == EPI_SWIGLU || epi == EPI_SWIGLU_TIED) : (epi == EPI_SILU || epi == EPI_RESID))) {
-    const int KBp = (a0.K + a1.K) / 64;
-    const long long tp = cdiv<long long>(M, 256);
-    auto pcost = [&](int bn) -> double {
-      if (N % bn) return 1e300;
-      const double per_pair = (double)cdiv<long long>(tp * (N / bn), kNumSM / 2);
-      return 5600.0 + per_pair * KBp * std::max(4.0 * bn, (32768.0 + bn * 64.0) / 43.0);
-    };
-    int bn = 64;
-    for (int cand : {128, 256})
-      if (pcost(cand) < pcost(bn)) bn = cand;
-    CUtensorMap maps[5];
-    WCHECK(tmap_bf16(&maps[0], a0.hi, M, a0.K, a0.ld, 128));
-    WCHECK(tmap_bf16(&maps[1], a0.lo, M, a0.K, a0.ld, 128));
-    if (a1.K > 0) {
-      WCHECK(tmap_bf16(&maps[2], a1.hi, M, a1.K, a1.ld, 128));
-      WCHECK(tmap_bf16(&maps[3], a1.lo, M, a1.K, a1.ld, 128));
-    } else {
-      maps[2] = maps[0];
-      maps[3] = maps[1];
-    }
-    WCHECK(tmap_bf16(&maps[4], W, N, a0.K + a1.K, a0.K + a1.K, bn / 2));
-    GemmArgs g{};
-    g.M = (int)M;
-    g.N = N;
-    g.kb0 = a0.K / 64;
-    g.kb1 = a1.K / 64;
-    g.tiles_n = N / bn;
-    g.num_tiles = (int)(tp * g.tiles_n);
-    g.inv_k = 1.0f / (float)a0.K;
-    g.eps = eps;
-    g.out_hi = static_cast<__nv_bfloat16*>(out.hi);
-    g.out_lo = static_cast<__nv_bfloat16*>(out.lo);
-    g.out32 = out.f32;
-    g.ldo = out.ld;
-    g.resid32 = resid32;
-    g.ldr = ldr;
-    if (bn == 256) return launch_pair_bn<256>(epi, rn, maps, g, st);
-    if (bn == 128) return launch_pair_bn<128>(epi, rn, maps, g, st);
-    return launch_pair_bn<64>(epi, rn, maps, g, st);
   }
   // Tile width by a small cost model (cycles): per-CTA fixed cost + tiles per persistent CTA x
   // (per 64-deep K block the larger of the MMA time and the operand bytes at ~80 B/clk, the rate
@@ -821,6 +616,10 @@ whale_status attention_qtile(const Shape& s, const void* q, const void* kv, cons
   return launch_pdl(attn_qtile_kernel<64>, dim3((unsigned)grid), dim3(kQtThreads), QtSmem<64>::BYTES, st, tq, tkv, a);
 }
 
+// Histories attended by many queries (N >= 128 per example) take the query-tiled tcgen05 kernel, which
+// needs no scratch; the split-L kernel (partials in the scratch of plan_attention) takes the rest.
+bool attention_is_query_tiled(const Shape& s) { return s.N >= 128 && (s.dh == 32 || s.dh == 64); }
+
 whale_status attention_bf16(const Shape& s, const void* q, const void* kv, const int* offsets, void* out,
                             void* out_lo, int B, long long total_L, void* scratch, cudaStream_t st) {
   if (B == 0) return WHALE_OK;
@@ -831,7 +630,7 @@ whale_status attention_bf16(const Shape& s, const void* q, const void* kv, const
     if (out_lo) CUCHECK(cudaMemsetAsync(out_lo, 0, rows * s.d * 2, st));
     return WHALE_OK;
   }
-  if (s.N >= 128 && (s.dh == 32 || s.dh == 64) && qtile_enabled()) return attention_qtile(s, q, kv, offsets, out, out_lo, B, total_L, st);
+  if (attention_is_query_tiled(s)) return attention_qtile(s, q, kv, offsets, out, out_lo, B, total_L, st);
   AttnArgs a{};
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.offsets = offsets;
@@ -913,40 +712,6 @@ whale_status abs_max_pairs(int E, int* pairs) {
   return c > 0 ? WHALE_OK : WHALE_ERR_UNSUPPORTED;
 }
 
-// Co-resident four-CTA clusters of the fused kernel (cached per device).
-whale_status abs_max_clusters(int E, int* clusters) {
-  static std::mutex mu;
-  static int cache[64][2];
-  int dev = 0;
-  CUCHECK(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= 64) return WHALE_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lk(mu);
-  int& c = cache[dev][E - 1];
-  if (c == 0) {
-    const void* kern = E == 1 ? reinterpret_cast<const void*>(abs_fused_kernel<1>)
-                              : reinterpret_cast<const void*>(abs_fused_kernel<2>);
-    const size_t smem = E == 1 ? FuSmem<1>::BYTES : FuSmem<2>::BYTES;
-    CUCHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    cudaLaunchConfig_t lc = {};
-    lc.gridDim = dim3(4 * kFuMaxClusters, 1, 1);
-    lc.blockDim = dim3(kFuThreads, 1, 1);
-    lc.dynamicSmemBytes = smem;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 4;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    lc.attrs = attr;
-    lc.numAttrs = 1;
-    int n = 0;
-    CUCHECK(cudaOccupancyMaxActiveClusters(&n, kern, &lc));
-    n = std::min(n, kFuMaxClusters);
-    c = n > 0 ? n : -1;
-  }
-  *clusters = c;
-  return c > 0 ? WHALE_OK : WHALE_ERR_UNSUPPORTED;
-}
-
 // qa[b*256 + j*N + n, :] = q[b*N + n, j*64 : j*64 + 64] W~_j^T with W~ [h*d, 64] (one K block per
 // head: a block-diagonal GEMM over the h*d output columns, rows scattered per head).
 whale_status gemm_qabs(const Shape& s, const void* q, const void* wkabs, void* qa, long long rows, cudaStream_t st) {
@@ -1001,10 +766,9 @@ whale_status gemm_vabs(const Shape& s, const void* zh, const void* wv, void* a, 
   return launch_gemm_t<64, EPI_STORE, false, false>(maps, g, tiles, st);
 }
 
-// CTA pairs of the two-pass kernels (0 with the one-pass kernel, whose clusters search their starts).
+// CTA pairs of the two-pass kernels.
 whale_status abs_two_pass_pairs(const Shape& s, const Layout& L, int* P) {
   *P = 0;
-  if (abs_fused_enabled()) return WHALE_OK;
   int pairs = 0;
   WCHECK(abs_max_pairs(s.d / 256, &pairs));
   *P = (int)std::max<long long>(1, std::min<long long>(pairs, L.units_max));
@@ -1046,25 +810,6 @@ whale_status attention_absorbed(const Shape& s, const void* q, const void* slab,
   a.stats_part = reinterpret_cast<float*>(at(ws, L.stp));
   a.part_z = reinterpret_cast<__nv_bfloat16*>(at(ws, L.pz));
   a.z_hi = reinterpret_cast<__nv_bfloat16*>(at(ws, L.zh));
-  if (abs_fused_enabled()) {
-    int clusters = 0;
-    WCHECK(abs_max_clusters(E, &clusters));
-    a.n_pairs = (int)std::max<long long>(1, std::min<long long>(clusters, L.units_max));
-    if (hint.total_L > 0) {
-      CUtensorMap tq, th, th64;
-      WCHECK(tmap_bf16(&tq, at(ws, L.qa), (long long)hint.B * kAbsQ, s.d, s.d, 128));
-      WCHECK(tmap_bf16(&th, slab, hint.total_L, s.d, s.d, 128));
-      WCHECK(tmap_bf16(&th64, slab, hint.total_L, s.d, s.d, 64));
-      if (E == 1)
-        WCHECK(launch_pdl(abs_fused_kernel<1>, dim3(4 * a.n_pairs), dim3(kFuThreads), FuSmem<1>::BYTES, st, tq, th,
-                          th64, a));
-      else
-        WCHECK(launch_pdl(abs_fused_kernel<2>, dim3(4 * a.n_pairs), dim3(kFuThreads), FuSmem<2>::BYTES, st, tq, th,
-                          th64, a));
-    }
-    WCHECK(launch_pdl(abs_merge_kernel, dim3(hint.B, kAbsQ / 8), dim3(256), 0, st, a));
-    return gemm_vabs(s, at(ws, L.zh), wv, out, out_lo, rows, st);
-  }
   int P = 0;
   WCHECK(abs_two_pass_pairs(s, L, &P));
   a.n_pairs = P;  // the pair count abs_units tabulated the starts for
@@ -1753,21 +1498,45 @@ whale_status whale_swiglu_ffn(const whale_config* cfg, long long rows, const voi
 namespace {
 __device__ __align__(256) unsigned char g_noalloc_scratch[WHALE_NOALLOC_SCRATCH_BYTES];
 
-// Device address of g_noalloc_scratch on the current device, looked up once per device (the
-// name is only a host-side stand-in for the array; kernels must get the real address).
+// The calling thread's current CUDA context, from the driver entry point (no link-time libcuda).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+whale_status current_context(CUcontext* ctx) {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(f);
+  });
+  if (!fn) return WHALE_ERR_CUDA;
+  *ctx = nullptr;
+  if (fn(ctx) != CUDA_SUCCESS) return WHALE_ERR_CUDA;
+  return WHALE_OK;  // *ctx is null if this thread has no current context yet
+}
+
+// Device address of g_noalloc_scratch in the current context (the name is only a host-side stand-in
+// for the array; kernels must get the real address). Looked up once per context, with the device
+// current, and cached under the context: a context created after cudaDeviceReset (a new primary
+// context) gets its own lookup, never the address from the old one.
 whale_status noalloc_scratch(void** out) {
   static std::mutex mu;
-  static void* addr[64];
-  int dev = 0;
-  CUCHECK(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= 64) return WHALE_ERR_UNSUPPORTED;
+  static std::vector<std::pair<CUcontext, void*>> cache;
+  CUcontext ctx = nullptr;
+  WCHECK(current_context(&ctx));
   std::lock_guard<std::mutex> lk(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    CUCHECK(cudaGetSymbolAddress(&p, g_noalloc_scratch));
-    addr[dev] = p;
-  }
-  *out = addr[dev];
+  if (ctx)
+    for (const auto& e : cache)
+      if (e.first == ctx) {
+        *out = e.second;
+        return WHALE_OK;
+      }
+  void* p = nullptr;
+  CUCHECK(cudaGetSymbolAddress(&p, g_noalloc_scratch));  // initialises the runtime's context if needed
+  if (!ctx) WCHECK(current_context(&ctx));
+  if (ctx) cache.push_back({ctx, p});
+  *out = p;
   return WHALE_OK;
 }
 }  // namespace
@@ -1788,12 +1557,20 @@ whale_status whale_cross_attention_noalloc(const whale_config* cfg, const void* 
     return attention_f32(s, static_cast<const float*>(q), static_cast<const float*>(kv), seq_offsets,
                          static_cast<float*>(a), hint->B, hint->total_L, st);
   }
+  // only the split-L kernel keeps partials in the scratch; the query-tiled kernel uses none
   const AttnPlan p = plan_attention(s, hint->B, hint->total_L);
-  if (p.bytes() > (size_t)WHALE_NOALLOC_SCRATCH_BYTES) return WHALE_ERR_WORKSPACE;
+  if (!attention_is_query_tiled(s) && p.bytes() > (size_t)WHALE_NOALLOC_SCRATCH_BYTES) return WHALE_ERR_WORKSPACE;
   void* scratch = nullptr;
   WCHECK(noalloc_scratch(&scratch));
   WCHECK(debug_check(s, seq_offsets, *hint, st));
   return attention_bf16(s, q, kv, seq_offsets, a, nullptr, hint->B, hint->total_L, scratch, st);
+}
+
+whale_status whale_test_bounded_waits(unsigned long long limit_ns, whale_stream_t stream) {
+  if (limit_ns < 1000ull || limit_ns > kWaitLimitNs) return WHALE_ERR_INVALID_ARG;
+  wait_selftest_kernel<<<1, 64, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_ns);
+  CUCHECK(cudaGetLastError());
+  return WHALE_OK;
 }
 
 whale_status whale_get_device_error(whale_stream_t stream, int* code) {

@@ -81,6 +81,7 @@ _SIGS = {
     "whale_prepare_weights": ([POINTER(whale_config), POINTER(whale_layer_weights), _P, c_size_t,
                                POINTER(whale_layer_weights), _P], c_int),
     "whale_cross_attention_noalloc": ([POINTER(whale_config), _P, _P, _P, _P, POINTER(whale_shape_hint), _P], c_int),
+    "whale_test_bounded_waits": ([ctypes.c_ulonglong, _P], c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -288,6 +289,14 @@ def whale_profile_end(capacity: int = 4096) -> list:
     n = c_int(0)
     _check(_lib.whale_profile_end(buf, capacity, ctypes.byref(n)), "whale_profile_end")
     return [((buf[i].kernel or b"?").decode(), float(buf[i].ms)) for i in range(min(n.value, capacity))]
+
+
+def whale_test_bounded_waits(limit_ns: int, stream=None, raw=False):
+    """Enqueue the self-test of the bounded device waits (see include/whale_fusion.h)."""
+    st = _lib.whale_test_bounded_waits(int(limit_ns), _stream(stream))
+    if raw:
+        return st
+    _check(st, "whale_test_bounded_waits")
 
 
 def whale_get_device_error(stream=None) -> int:
