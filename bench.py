@@ -359,6 +359,13 @@ def run_kernel_case(args):
         w = w.replace(batch=args.batch)
     p = Hn.build_problem(w, device="cuda")
     lw = p.weights[0]
+    if args.kernel_case == "backward":  # one layer's backward (all of its kernels)
+        import torch
+        res = time_backward(p, p.weights, w, p.total_L, load_peaks()[0], None, torch.cuda.current_stream(),
+                            reps=args.steps)
+        print(json.dumps({"kernel_case": "backward", "workload": w.name, "total_L": p.total_L,
+                          "ms_per_layer": res.get("ms_per_layer")}), flush=True)
+        return 0
     if args.kernel_case == "absorbed":
         Hn.prepare_weights(p)   # as the forward runs it: gains folded, absorbed keys formed at load
     T = p.total_L
@@ -403,6 +410,66 @@ def run_kernel_case(args):
     return 0
 
 
+def time_backward(p, raw_weights, w, total_L, peaks, clocks, stream, reps=10):
+    """One layer's backward (whale_fusion_layer_backward, raw weights, an N(0,1) upstream gradient)
+    timed with CUDA events over `reps` calls, its kernels from the library's per-kernel events, and
+    the roofline of its attention kernel (KV-parallel: reads K|V and writes dK|dV once, plus the
+    example's queries per history chunk: HBM-bound at N <= 32)."""
+    import torch
+    from wukong_hstu_cross_b200 import harness as Hn
+    from wukong_hstu_cross_b200 import whale as Wb
+    cfg = Hn.config_of(w, Hn.flags_of(p.flags.get("shared_kv", False), p.flags.get("tied_gate", False)))
+    nbytes = Wb.whale_backward_workspace_size(cfg, p.hint)
+    if nbytes == 0:
+        return {"unsupported": "shape outside the backward pass's support"}
+    lw = raw_weights[0]
+    dev = p.tokens.device
+    grads = {k: torch.empty(tuple(v.shape), dtype=torch.float32, device=dev) for k, v in lw.items()
+             if v is not None and k != "w_kabs"}
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    d_out = torch.randn(p.tokens.shape, dtype=torch.float32, device=dev, generator=torch.Generator(dev).manual_seed(1))
+    d_tok = torch.empty(p.tokens.shape, dtype=torch.float32, device=dev)
+    d_st = torch.empty(p.states.shape[1:], dtype=p.states.dtype, device=dev)
+
+    def call():
+        Wb.whale_fusion_layer_backward(cfg, p.tokens, p.states[0], p.offsets_t, lw, d_out, d_tok, d_st, grads, p.hint,
+                                       ws, stream=stream)
+    for _ in range(2):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    Wb.whale_profile_begin(4096)
+    call()
+    recs = Wb.whale_profile_end()
+    kern = {}
+    for name, kms in recs:
+        e = kern.setdefault(kernel_name(name), [0, 0.0])
+        e[0] += 1
+        e[1] += kms
+    tot = sum(v[1] for v in kern.values()) or 1.0
+    kernels = {n: {"launches": c, "avg_ms": t / c, "share": t / tot}
+               for n, (c, t) in sorted(kern.items(), key=lambda x: -x[1][1])}
+    out = {"entry_point": "whale_fusion_layer_backward (one layer, forward recomputed inside)", "ms_per_layer": ms,
+           "reps": reps, "kernels": kernels}
+    ab = next((v for k, v in kernels.items() if k.split("<")[0] == "attn_bwd_kernel"), None)
+    if ab:
+        kvw = w.d if p.flags.get("shared_kv") else 2 * w.d
+        nb = 2.0 * total_L * kvw * 2          # K|V read once, dK|dV written once (bf16)
+        fl = 10.0 * w.n_tokens * total_L * w.d  # S, dP, dV, dK, dQ: five contractions of 2 N L d
+        tc, tc_src = tensor_peak(peaks, clocks)
+        out["roofline"] = {"kernel": "attn_bwd_kernel (KV-parallel attention backward, mma.sync)",
+                           **roofline_of(fl, nb, ab["avg_ms"], tc, peaks["hbm_gbs"]),
+                           "algorithmic_flops_per_launch": fl, "algorithmic_bytes_per_launch": nb,
+                           "avg_launch_ms": ab["avg_ms"], "peak_source": tc_src}
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -415,13 +482,14 @@ def main():
     ap.add_argument("--ref-total", type=float, default=90.0,
                     help="oracle seconds of the whole --impl reference run, split across its steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel-case", choices=["kv", "attn", "ffn", "fusion", "absorbed"], default=None,
+    ap.add_argument("--kernel-case", choices=["kv", "attn", "ffn", "fusion", "absorbed", "backward"], default=None,
                     help="profiling aid: run only one step entry point on one layer of the workload")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (kernel cases)")
     ap.add_argument("--shared-kv", action="store_true", help="variant: K = V (one W_K), the pages' shared key/value")
     ap.add_argument("--tied-gate", action="store_true", help="variant: W_gate = W_up, the pages' shared-gate SwiGLU")
     ap.add_argument("--fold-per-call", action="store_true",
                     help="fold the RMSNorm gains into the weights inside every forward instead of once at load")
+    ap.add_argument("--no-backward", action="store_true", help="skip the one-layer backward measurement")
     ap.add_argument("--materialized-kv", action="store_true",
                     help="project K|V and attend over them even where the absorbed attention applies")
     args = ap.parse_args()
@@ -606,6 +674,11 @@ def main():
         t_star += max(v["flops"] / (tc_step * 1e12), v["bytes"] / (peaks["hbm_gbs"] * 1e9))
     t_star *= w.n_layers * 1e3
 
+    # ---------------- backward pass of one layer (the training path), device-resident ----------------
+    bwd = None
+    if not args.no_backward:
+        bwd = time_backward(p, raw_weights, w, total_L, peaks, clocks, stream, reps=max(3, min(args.steps, 20)))
+
     # ---------------- end to end: host buffers through the C ABI, copies inside the timed region -----
     e2e = None
     if args.e2e_steps > 0:
@@ -646,6 +719,7 @@ def main():
                               "kv_proj_ms": t_kv, "attention_ms": t_attn, "absorbed_attention_ms": t_abs,
                               "peaks": f"{peak_src}: {peaks['hbm_gbs']} GB/s, {tc_step} TFLOP/s"},
             "kernels": kernels,
+            "backward": bwd,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": (len(recs) or launches_per_step(w, args.fold_per_call, absorbed)) * args.steps,
             "clocks": clocks,
         }

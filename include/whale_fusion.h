@@ -263,6 +263,51 @@ whale_status whale_cross_attention_noalloc(const whale_config* cfg, const void* 
                                            const int* seq_offsets, void* a, const whale_shape_hint* hint,
                                            whale_stream_t stream);
 
+/* ---- backward pass (training) -------------------------------------------------------------
+ *
+ * The gradients of one fusion layer for an upstream gradient d_out = dLoss/dH_f: the
+ * vector-Jacobian product of the forward above, step by step in reverse (the pages give the
+ * forward's steps, gist.science section 2.1, and name the backward's schedule, section 2.2
+ * "Asymmetric Backward Variants": the attention's backward is KV-parallel here, since a few queries
+ * per example meet thousands of history rows; paper-daily.com digest, section 2). The forward is
+ * recomputed inside the call (with K|V materialised and the softmax's log-sum-exp kept), so the
+ * caller passes only the layer's inputs.
+ *
+ *   tokens_in     device [B, N, d]    the layer's H_w (cfg->dtype)
+ *   layer_states  device [total_L, d] the layer's H_s (cfg->dtype)
+ *   seq_offsets   device int32 [B+1]
+ *   w             the layer's RAW weights and gains (WHALE_PREPARED_WEIGHTS is not accepted)
+ *   d_out         device fp32 [B, N, d]      dLoss/dH_f
+ *   d_tokens      device fp32 [B, N, d]      dLoss/dH_w (written)
+ *   d_states      device [total_L, d]        dLoss/dH_s in cfg->dtype (written)
+ *   grads         HOST struct of device fp32 pointers, each overwritten with dLoss/d(parameter),
+ *                 summed over the batch, in the parameter's own layout (w_f1 may be null when
+ *                 fusion_hidden is 0)
+ *   workspace     device, >= whale_backward_workspace_size bytes, 256-byte aligned
+ *
+ * Supported: bf16 with n_tokens <= 32, d_head 32 or 64, d % 64 == 0, d <= 1024; fp32 with d_head
+ * <= 64 (the SIMT correctness mode). Other shapes return WHALE_ERR_UNSUPPORTED (the many-candidate
+ * serving shape is an inference shape). Asynchronous on `stream`; no device-to-host reads. In bf16
+ * mode dq is summed with fp32 atomics across history chunks, so repeated calls can differ in the
+ * last bits of d_tokens and of the gradients downstream of it. */
+typedef struct {
+  float* g_q;      /* [d] */
+  float* g_kv;     /* [d] */
+  float* w_q;      /* [d, d] */
+  float* w_kv;     /* [2d, d] ([d, d] with WHALE_SHARED_KV) */
+  float* w_f1;     /* [fusion_hidden, 2d] (null if fusion_hidden 0) */
+  float* w_f2;     /* [d, fusion_hidden] ([d, 2d] if fusion_hidden 0) */
+  float* g_ffn;    /* [d] */
+  float* w_upgate; /* [2H, d] ([H, d] with WHALE_TIED_GATE) */
+  float* w_down;   /* [d, H] */
+} whale_layer_grads;
+size_t whale_backward_workspace_size(const whale_config* cfg, const whale_shape_hint* hint);
+whale_status whale_fusion_layer_backward(const whale_config* cfg, const void* tokens_in, const void* layer_states,
+                                         const int* seq_offsets, const whale_layer_weights* w, const float* d_out,
+                                         float* d_tokens, void* d_states, const whale_layer_grads* grads,
+                                         const whale_shape_hint* hint, void* workspace, size_t workspace_bytes,
+                                         whale_stream_t stream);
+
 /* Failure detection. Every device-side wait of the library's kernels (a pipeline stage on an
  * mbarrier, one CTA pair waiting for another's published results) gives up after a time limit
  * (2 s in the kernels), records WHALE_DEVERR_TIMEOUT in the device error word and lets its kernel

@@ -15,7 +15,8 @@ EXPECTED = {
     "whale_fusion_forward_host", "whale_fusion_layer_forward", "whale_project_queries", "whale_project_kv",
     "whale_cross_attention", "whale_fusion_mlp", "whale_swiglu_ffn", "whale_get_device_error",
     "whale_attend_states", "whale_prepare_weights", "whale_prepared_weights_size", "whale_cross_attention_noalloc",
-    "whale_profile_begin", "whale_profile_end", "whale_test_bounded_waits",
+    "whale_profile_begin", "whale_profile_end", "whale_test_bounded_waits", "whale_backward_workspace_size",
+    "whale_fusion_layer_backward",
 }
 
 
@@ -25,6 +26,44 @@ def test_library_exports_every_declared_symbol():
     lib = ctypes.CDLL(W.LIB_PATH)
     for name in declared:
         assert hasattr(lib, name), name
+
+
+def test_backward_workspace_size_and_supported_shapes():
+    # the training workloads are supported; the many-candidate serving shape (N = 16384) is not
+    for name in ("tiny_fp32", "stack_d128", "stack_d256", "hist15k_d512"):
+        w, cfg = _cfg(name)
+        assert W.whale_backward_workspace_size(cfg, W.make_hint(w.batch, 3000, w.batch * 3000)) > 0, name
+    w, cfg = _cfg("serve_15k")
+    assert W.whale_backward_workspace_size(cfg, W.make_hint(1, 15000, 15000)) == 0
+    # prepared (gain-folded, re-packed) weights are not accepted: the backward needs the raw ones
+    w, cfg = _cfg("stack_d128")
+    prep = W.make_config(cfg.n_layers, cfg.d, cfg.n_heads, cfg.n_tokens, cfg.ffn_hidden, cfg.fusion_hidden, cfg.dtype,
+                         cfg.flags | W.WHALE_PREPARED_WEIGHTS, cfg.eps)
+    assert W.whale_backward_workspace_size(prep, W.make_hint(4, 100, 400)) == 0
+    # the workspace grows with the history (K|V, its gradient, the states' gradient terms)
+    small = W.whale_backward_workspace_size(cfg, W.make_hint(4, 100, 400))
+    large = W.whale_backward_workspace_size(cfg, W.make_hint(4, 100, 40000))
+    assert large - small >= (40000 - 400) * cfg.d * (2 * 2 + 2 * 2 + 4 + 2)
+
+
+def test_backward_host_side_errors():
+    w, cfg = _cfg("stack_d128")
+    hint = W.make_hint(2, 10, 20)
+    fake = 1 << 20  # never dereferenced: every call below fails its checks first
+    lw = dict.fromkeys(["g_q", "g_kv", "w_q", "w_kv", "w_f1", "w_f2", "g_ffn", "w_upgate", "w_down"], fake)
+    gr = dict(lw)
+    nbytes = W.whale_backward_workspace_size(cfg, hint)
+    # workspace too small
+    assert W.whale_fusion_layer_backward(cfg, fake, fake, fake, lw, fake, fake, fake, gr, hint, fake, nbytes - 1,
+                                         stream=0, raw=True) == 4
+    # a missing gradient buffer
+    bad = dict(gr, w_down=None)
+    assert W.whale_fusion_layer_backward(cfg, fake, fake, fake, lw, fake, fake, fake, bad, hint, fake, nbytes,
+                                         stream=0, raw=True) == 1
+    # unsupported: more than 32 tokens per example in bf16
+    w2, cfg2 = _cfg("stack_d128", n_tokens=64)
+    assert W.whale_fusion_layer_backward(cfg2, fake, fake, fake, lw, fake, fake, fake, gr, hint, fake, 1 << 30,
+                                         stream=0, raw=True) == 2
 
 
 def test_bounded_wait_self_test_rejects_limits_out_of_range():

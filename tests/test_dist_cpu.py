@@ -1,6 +1,8 @@
 """Multi-rank plumbing on CPU: two gloo ranks (world_size 2) shard the examples of a workload
 with no data exchange, keep the weights replicated, and reduce the per-rank device time with a
-max, exactly as bench.py does under torchrun on GPUs."""
+max, exactly as bench.py does under torchrun on GPUs. One batch split across the ranks by
+history rows (shard_batch) and run through the oracle on each rank gives, gathered, bitwise the
+unsharded result."""
 import os
 import socket
 
@@ -65,3 +67,61 @@ def test_single_process_defaults():
     w = I.WORKLOADS["stack_d128"]
     assert D.shard_workload(w, 0, 1) is w
     assert D.max_over_ranks(3.5, 1) == 3.5
+
+
+def _shard_worker(rank, world, port, out):
+    import torch.distributed as dist
+    from oracle import whale_oracle as O
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    w = I.WORKLOADS["stack_d128"].replace(batch=7, n_layers=2, lengths=("uniform", 1, 120))
+    L = I.draw_lengths(w)
+    L[3] = 0
+    off = I.offsets_of(L)
+    tokens = I.make_tokens(w)
+    states = np.stack([I.make_states_layer(w, l, L, threads=1) for l in range(w.n_layers)])
+    lws = I.make_all_weights(w, gains="random")
+    tok_r, st_r, off_r, (b0, b1) = D.shard_batch(tokens, states, off, rank, world)
+    y = O.fusion_stack(tok_r, st_r, off_r, lws, w.n_heads, w.eps) if b1 > b0 else np.zeros((0, w.n_tokens, w.d))
+    objs = [None] * world
+    dist.all_gather_object(objs, (b0, b1, int(st_r.shape[1]), y))
+    if rank == 0:
+        full = O.fusion_stack(tokens, states, off, lws, w.n_heads, w.eps)
+        out.put((objs, full, L.tolist()))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_one_batch_sharded_by_history_rows_equals_unsharded():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    objs, full, L = q.get(timeout=180)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    (a0, a1, rows0, y0), (c0, c1, rows1, y1) = objs
+    assert (a0, a1, c1) == (0, c0, len(L))                 # contiguous, covering the batch
+    assert rows0 + rows1 == sum(L) and abs(rows0 - rows1) <= max(L)   # balanced within one example
+    assert np.array_equal(np.concatenate([y0, y1]), full)  # bitwise the unsharded oracle
+
+
+def test_balanced_ranges_edge_cases():
+    assert D.balanced_ranges([5, 5, 5, 5], 2) == [(0, 2), (2, 4)]
+    assert D.balanced_ranges([100, 1, 1, 1], 2) == [(0, 1), (1, 4)]
+    assert D.balanced_ranges([3], 4) == [(0, 0), (0, 1), (1, 1), (1, 1)] or \
+        sum(b - a for a, b in D.balanced_ranges([3], 4)) == 1
+    assert D.balanced_ranges([], 2) == [(0, 0), (0, 0)]
+    assert D.balanced_ranges([0, 0, 7, 0], 1) == [(0, 4)]
+    # every example lands in exactly one range, ranges in order
+    rng = np.random.default_rng(0)
+    for world in (2, 3, 8):
+        L = rng.integers(0, 5000, size=37)
+        rr = D.balanced_ranges(L, world)
+        assert rr[0][0] == 0 and rr[-1][1] == 37 and all(rr[k][1] == rr[k + 1][0] for k in range(world - 1))
+        loads = [int(L[a:b].sum()) for a, b in rr]
+        assert max(loads) - min(loads) <= 2 * int(L.max())

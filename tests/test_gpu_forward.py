@@ -129,6 +129,51 @@ def test_prepared_weights_match_per_call_fold():
         assert torch.equal(out, ref)
 
 
+def test_prepared_weights_outlive_the_raw_weight_list():
+    """Prepared weights point into the caller's raw w_f1, w_f2, w_down and gains: once the problem's
+    weight list is replaced by the prepared array, those tensors must stay alive. Repeated forwards
+    with allocations and a cache flush in between give bitwise the same output (a dangling pointer
+    here once made later forwards read freed memory)."""
+    w = I.WORKLOADS["stack_d128"].replace(batch=4, n_layers=2, lengths=("uniform", 1, 400))
+    p = Hn.build_problem(w, gains="random")
+    Hn.prepare_weights(p)
+    ref = Hn.run_forward(p).clone()
+    torch.cuda.synchronize()
+    _check(p, ref)
+    for _ in range(3):
+        junk = [torch.full((1 << 20,), 7.0, device="cuda") for _ in range(8)]  # reuse freed memory, if any
+        del junk
+        torch.cuda.empty_cache()
+        out = Hn.run_forward(p)
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref)
+
+
+def test_cuda_graph_replay_matches_stream_launches():
+    """One forward of the absorbed 15k-history path (prepared weights) captured in a CUDA graph: the
+    programmatic-dependent launches become graph edges; replays give bitwise the stream result."""
+    w = I.WORKLOADS["hist15k_d512"].replace(**REDUCED["hist15k_d512"])
+    p = Hn.build_problem(w, gains="random")
+    Hn.prepare_weights(p)
+    st = torch.cuda.Stream()
+    with torch.cuda.stream(st):
+        for _ in range(2):
+            Hn.run_forward(p, st)
+    torch.cuda.synchronize()
+    ref = p.out.clone()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=st):
+        Hn.run_forward(p, st)
+    torch.cuda.synchronize()
+    for _ in range(3):
+        p.out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(p.out, ref)
+    del g
+    _check(p, ref)
+
+
 def test_host_buffer_entry_point_matches_device_entry_point():
     w = I.WORKLOADS["stack_d256"].replace(batch=4, n_layers=3, lengths=("uniform", 10, 1200))
     p = Hn.build_problem(w, gains="random")

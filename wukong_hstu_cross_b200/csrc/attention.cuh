@@ -44,6 +44,8 @@ struct AttnArgs {
   int* counters;           // [B * n_qblocks] finished-slice counts, zero at launch
   __nv_bfloat16* out;      // A [B*N, d] (bf16)
   __nv_bfloat16* out_lo;   // bf16 residue of A (may be null)
+  float* lse;              // [B*N, h] log2 of each softmax denominator, in scaled units (may be null):
+                           // p_t = 2^(s_t * scale_log2 - lse); the backward pass reuses it
 };
 
 // Offsets clamped into the slab [0, total_L]: example b owns rows [lo_b, hi_b).
@@ -478,6 +480,8 @@ __global__ void __launch_bounds__(32 * (HG + 1), 1)
           if (n >= a.N) continue;
           const float inv = 1.0f / lq[mt][hr];
           const long long row = ((long long)sg.b * a.N + n) * a.d + head * DH;
+          if (a.lse != nullptr && qd == 0)
+            a.lse[((long long)sg.b * a.N + n) * a.n_heads + head] = m_run[mt][hr] + __log2f(lq[mt][hr]);
 #pragma unroll
           for (int nt = 0; nt < DH / 8; ++nt) {
             const float x0 = o[mt][nt][2 * hr] * inv, x1 = o[mt][nt][2 * hr + 1] * inv;

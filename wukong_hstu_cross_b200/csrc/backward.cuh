@@ -1,0 +1,427 @@
+// backward.cuh — the element-wise, row-wise and reduction kernels of the fusion layer's backward
+// pass (the vector-Jacobian product of the forward for an upstream gradient dY = dLoss/dH_f), and
+// the SIMT kernels of its fp32 (correctness) mode. The dense contractions of the bf16 mode run on
+// the tcgen05 GEMM (gemm_tc.cuh, MN-major operands and split-K) and the attention's backward on
+// attention_bwd.cuh.
+//
+// The derivatives are the forward's steps differentiated one by one (gist.science technical summary
+// of WHALE, section 2.2 "Efficiency Optimizations", Asymmetric Backward Variants, names the
+// backward's schedules; the formulas follow from the forward of section 2.1):
+//   RMSNorm  n = r x g, r = (mean(x^2) + eps)^-1/2:  dx = r (dn g) - x r^3 / d * sum(dn g x),
+//                                                    dg = sum over rows of dn x r
+//   SiLU     silu'(z) = s(z) (1 + z (1 - s(z))), s = sigmoid
+//   SwiGLU   m = silu(gate) up:  dup = dm silu(gate), dgate = dm up silu'(gate)
+//            (tied gate, up = gate = u: du = dup + dgate)
+#pragma once
+
+#include "ptx.cuh"
+
+namespace whale {
+
+__device__ __forceinline__ float sigmoid_f(float z) { return 1.0f / (1.0f + __expf(-z)); }
+__device__ __forceinline__ float silu_grad_f(float z) {
+  const float s = sigmoid_f(z);
+  return s * (1.0f + z * (1.0f - s));
+}
+
+// x (fp32, row stride ldx) -> bf16 hi = bf16(x) and lo = bf16(x - hi) (lo may be null), row stride ldo.
+__global__ void split_pair_kernel(const float* __restrict__ x, long long ldx, __nv_bfloat16* __restrict__ hi,
+                                  __nv_bfloat16* __restrict__ lo, long long ldo, long long rows, int cols) {
+  pdl_wait();
+  pdl_trigger();
+  const long long n = rows * cols;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const long long r = i / cols, c = i - r * cols;
+    const float v = x[r * ldx + c];
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    hi[r * ldo + c] = h;
+    if (lo) lo[r * ldo + c] = __float2bfloat16_rn(v - __bfloat162float(h));
+  }
+}
+
+// G = SiLU(Z); Z fp32 [n]; outputs (each may be null): fp32, and a bf16 pair (hi, lo).
+__global__ void silu_pair_kernel(const float* __restrict__ z, float* __restrict__ g32, __nv_bfloat16* __restrict__ hi,
+                                 __nv_bfloat16* __restrict__ lo, long long n) {
+  pdl_wait();
+  pdl_trigger();
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const float zz = z[i];
+    const float v = zz * sigmoid_f(zz);
+    if (g32) g32[i] = v;
+    if (hi) {
+      const __nv_bfloat16 h = __float2bfloat16_rn(v);
+      hi[i] = h;
+      if (lo) lo[i] = __float2bfloat16_rn(v - __bfloat162float(h));
+    }
+  }
+}
+
+// dZ = dH * silu'(Z) as fp32 (optional) and a bf16 pair (optional).
+__global__ void silu_bwd_kernel(const float* __restrict__ dh, const float* __restrict__ z, float* __restrict__ dz32,
+                                __nv_bfloat16* __restrict__ hi, __nv_bfloat16* __restrict__ lo, long long n) {
+  pdl_wait();
+  pdl_trigger();
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const float v = dh[i] * silu_grad_f(z[i]);
+    if (dz32) dz32[i] = v;
+    if (hi) {
+      const __nv_bfloat16 h = __float2bfloat16_rn(v);
+      hi[i] = h;
+      if (lo) lo[i] = __float2bfloat16_rn(v - __bfloat162float(h));
+    }
+  }
+}
+
+// SwiGLU backward. ug: fp32 [rows, ugw] pre-activations ([up | gate], or u alone with a tied gate);
+// dm: fp32 [rows, H] gradient of m = SiLU(gate) * up. Outputs (each may be null): m as bf16 [rows, H],
+// and dug = [dup | dgate] (or du) as fp32 and as a bf16 pair, [rows, ugw]; m also as fp32 (m32) and
+// as the bf16 residue of m_out (m_lo).
+__global__ void swiglu_bwd_kernel(const float* __restrict__ ug, const float* __restrict__ dm, long long rows, int H,
+                                  int tied, __nv_bfloat16* __restrict__ m_out, __nv_bfloat16* __restrict__ m_lo,
+                                  float* __restrict__ m32,
+                                  float* __restrict__ dug32, __nv_bfloat16* __restrict__ dug_hi,
+                                  __nv_bfloat16* __restrict__ dug_lo) {
+  pdl_wait();
+  pdl_trigger();
+  const int ugw = tied ? H : 2 * H;
+  const long long n = rows * H;
+  auto put = [&](long long idx, float v) {
+    if (dug32) dug32[idx] = v;
+    if (dug_hi) {
+      const __nv_bfloat16 h = __float2bfloat16_rn(v);
+      dug_hi[idx] = h;
+      if (dug_lo) dug_lo[idx] = __float2bfloat16_rn(v - __bfloat162float(h));
+    }
+  };
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const long long r = i / H;
+    const int c = (int)(i - r * H);
+    const float up = ug[r * ugw + c];
+    const float gate = tied ? up : ug[r * ugw + H + c];
+    const float s = sigmoid_f(gate);
+    const float sg = gate * s;  // silu(gate)
+    const float g = dm[i];
+    const float mv = sg * up;
+    if (m_out) {
+      const __nv_bfloat16 mh = __float2bfloat16_rn(mv);
+      m_out[i] = mh;
+      if (m_lo) m_lo[i] = __float2bfloat16_rn(mv - __bfloat162float(mh));
+    }
+    if (m32) m32[i] = mv;
+    const float dup = g * sg;
+    const float dgate = g * up * s * (1.0f + gate * (1.0f - s));
+    if (tied) {
+      put(r * ugw + c, dup + dgate);
+    } else {
+      put(r * ugw + c, dup);
+      put(r * ugw + H + c, dgate);
+    }
+  }
+}
+
+// RMSNorm backward, one warp per row (d a multiple of 32, at most 1024), for n = r x g:
+//   dx = r (dn g) - x (r^3 / d) sum_c (dn g x)_c  [+ resid1 + resid2]
+// x: bf16 or fp32 [rows, d] (row stride d); dn fp32 [rows, d]; outputs (each may be null): dx as fp32,
+// as bf16 (dx_hi, with its residue dx_lo), n = r x g as a bf16 pair (n_out, n_lo) or fp32 (n32). colp [gridDim.x, d]: this
+// block's column sums of dn x r (the gain's gradient, summed over the block's rows; a second pass
+// sums the blocks in order).
+template <typename TX>
+__global__ void __launch_bounds__(256) rms_bwd_kernel(const TX* __restrict__ x, const float* __restrict__ g,
+                                                      const float* __restrict__ dn, long long rows, int d, float eps,
+                                                      const float* __restrict__ resid1, long long ld1,
+                                                      const float* __restrict__ resid2, long long ld2,
+                                                      float* __restrict__ dx32, __nv_bfloat16* __restrict__ dx_hi,
+                                                      __nv_bfloat16* __restrict__ dx_lo,
+                                                      __nv_bfloat16* __restrict__ n_out,
+                                                      __nv_bfloat16* __restrict__ n_lo, float* __restrict__ n32,
+                                                      float* __restrict__ colp) {
+  constexpr int MAXC = 32;  // columns per lane (d <= 1024)
+  __shared__ float red[8][1024];
+  pdl_wait();
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nc = d >> 5;
+  float cg[MAXC];
+#pragma unroll
+  for (int i = 0; i < MAXC; ++i) cg[i] = 0.f;
+  const long long per = (rows + gridDim.x - 1) / gridDim.x;
+  const long long r0 = (long long)blockIdx.x * per, r1 = min(rows, r0 + per);
+  for (long long r = r0 + warp; r < r1; r += 8) {
+    float xv[MAXC], u[MAXC];
+    float ss = 0.f, sux = 0.f;
+#pragma unroll
+    for (int i = 0; i < MAXC; ++i) {
+      if (i < nc) {
+        const int c = lane + 32 * i;
+        xv[i] = (float)x[r * d + c];
+        ss = fmaf(xv[i], xv[i], ss);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float rr = rsqrtf(ss / (float)d + eps);
+#pragma unroll
+    for (int i = 0; i < MAXC; ++i) {
+      if (i < nc) {
+        const int c = lane + 32 * i;
+        const float dv = dn[r * d + c];
+        u[i] = dv * g[c];
+        sux = fmaf(u[i], xv[i], sux);
+        cg[i] = fmaf(dv, xv[i] * rr, cg[i]);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sux += __shfl_xor_sync(0xffffffffu, sux, o);
+    const float k = rr * rr * rr / (float)d * sux;
+#pragma unroll
+    for (int i = 0; i < MAXC; ++i) {
+      if (i < nc) {
+        const int c = lane + 32 * i;
+        float v = rr * u[i] - xv[i] * k;
+        if (resid1) v += resid1[r * ld1 + c];
+        if (resid2) v += resid2[r * ld2 + c];
+        if (dx32) dx32[r * d + c] = v;
+        if (dx_hi) {
+          const __nv_bfloat16 h = __float2bfloat16_rn(v);
+          dx_hi[r * d + c] = h;
+          if (dx_lo) dx_lo[r * d + c] = __float2bfloat16_rn(v - __bfloat162float(h));
+        }
+        const float nv = xv[i] * rr * g[c];
+        if (n_out) {
+          const __nv_bfloat16 nh = __float2bfloat16_rn(nv);
+          n_out[r * d + c] = nh;
+          if (n_lo) n_lo[r * d + c] = __float2bfloat16_rn(nv - __bfloat162float(nh));
+        }
+        if (n32) n32[r * d + c] = nv;
+      }
+    }
+  }
+  if (colp) {
+#pragma unroll
+    for (int i = 0; i < MAXC; ++i)
+      if (i < nc) red[warp][lane + 32 * i] = cg[i];
+    __syncthreads();
+    for (int c = threadIdx.x; c < d; c += blockDim.x) {
+      float sum = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) sum += red[w][c];
+      colp[(long long)blockIdx.x * d + c] = sum;
+    }
+  }
+}
+
+// n = r x g as a bf16 pair (n_out, n_lo) and/or fp32 (n32): the normalised rows the weight gradients
+// contract with, one warp per row.
+template <typename TX>
+__global__ void __launch_bounds__(256) rms_rows_kernel(const TX* __restrict__ x, const float* __restrict__ g,
+                                                       long long rows, int d, float eps,
+                                                       __nv_bfloat16* __restrict__ n_out,
+                                                       __nv_bfloat16* __restrict__ n_lo, float* __restrict__ n32) {
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  const long long warps = (long long)gridDim.x * 8;
+  for (long long r = (long long)blockIdx.x * 8 + (threadIdx.x >> 5); r < rows; r += warps) {
+    float ss = 0.f;
+    for (int c = lane; c < d; c += 32) {
+      const float v = (float)x[r * d + c];
+      ss = fmaf(v, v, ss);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float rr = rsqrtf(ss / (float)d + eps);
+    for (int c = lane; c < d; c += 32) {
+      const float v = (float)x[r * d + c] * rr * g[c];
+      if (n_out) {
+        const __nv_bfloat16 nh = __float2bfloat16_rn(v);
+        n_out[r * d + c] = nh;
+        if (n_lo) n_lo[r * d + c] = __float2bfloat16_rn(v - __bfloat162float(nh));
+      }
+      if (n32) n32[r * d + c] = v;
+    }
+  }
+}
+
+// out[r, c] (row stride ldo) = sum_b part[b][r][c] over b = 0..nb-1 in order (deterministic);
+// part holds nb dense [rows, cols] blocks.
+__global__ void sum_partials_kernel(const float* __restrict__ part, int nb, long long rows, int cols,
+                                    float* __restrict__ out, long long ldo) {
+  pdl_wait();
+  pdl_trigger();
+  const long long n = rows * cols;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    float s = 0.f;
+    for (int b = 0; b < nb; ++b) s += part[(long long)b * n + i];
+    const long long r = i / cols;
+    out[r * ldo + (i - r * cols)] = s;
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// fp32 (correctness) mode
+// ---------------------------------------------------------------------------------------------
+// C[m, n] = sum_k A[m sam + k sak] * B[k sbk + n sbn] (+ C if accumulate), fp32, any strides: 64 x 64
+// tiles, 256 threads with 4 x 4 outputs each, K in steps of 16 through shared memory.
+__global__ void __launch_bounds__(256) gemm_strided_f32_kernel(const float* __restrict__ A, long long sam,
+                                                               long long sak, const float* __restrict__ B,
+                                                               long long sbk, long long sbn, float* __restrict__ C,
+                                                               long long ldc, long long M, long long N, long long K,
+                                                               int accumulate) {
+  __shared__ float As[16][64 + 1];
+  __shared__ float Bs[16][64 + 1];
+  const long long m0 = (long long)blockIdx.y * 64, n0 = (long long)blockIdx.x * 64;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float acc[4][4] = {};
+  for (long long k0 = 0; k0 < K; k0 += 16) {
+    for (int i = threadIdx.x; i < 16 * 64; i += 256) {
+      const int kk = i / 64, mm = i % 64;
+      const long long gm = m0 + mm, gk = k0 + kk;
+      As[kk][mm] = (gm < M && gk < K) ? A[gm * sam + gk * sak] : 0.f;
+      const long long gn = n0 + mm;
+      Bs[kk][mm] = (gn < N && gk < K) ? B[gk * sbk + gn * sbn] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        a[i] = As[kk][ty * 4 + i];
+        b[i] = Bs[kk][tx * 4 + i];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const long long gm = m0 + ty * 4 + i;
+    if (gm >= M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const long long gn = n0 + tx * 4 + j;
+      if (gn >= N) continue;
+      float* c = C + gm * ldc + gn;
+      *c = accumulate ? *c + acc[i][j] : acc[i][j];
+    }
+  }
+}
+
+// fp32 attention backward, one block per (example, head): all of the example's queries stay in
+// shared memory; each thread takes history rows in turn and writes their dK, dV rows itself (one
+// block holds every query of the pair, so no reduction over queries is needed), while dQ collects
+// in shared memory. Phase 1 recomputes each query's softmax statistics and delta = sum_t p_t dp_t
+// (warp per query). kv rows: K in columns [head*DH, ...), V at v_col0 + head*DH; dkv the same
+// layout (shared K = V: dK + dV in the K columns). Needs N * (3 DH + 3) floats of shared memory.
+template <int DH>
+__global__ void __launch_bounds__(256) attn_bwd_f32_kernel(const float* __restrict__ q, const float* __restrict__ kv,
+                                                           int kvw, int v_col0, const float* __restrict__ da,
+                                                           long long ld_da, const int* __restrict__ offsets,
+                                                           long long total_L, int N,
+                                                           int d, int n_heads, float scale, float* __restrict__ dq,
+                                                           float* __restrict__ dkv, int shared_kv) {
+  extern __shared__ float sm[];
+  float* qs = sm;                 // [N][DH]
+  float* das = qs + N * DH;       // [N][DH]
+  float* dqs = das + N * DH;      // [N][DH]
+  float* mx = dqs + N * DH;       // [N]
+  float* ls = mx + N;             // [N] sum of exp(s - mx)
+  float* del = ls + N;            // [N]
+  const int b = blockIdx.x, head = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  long long lo = offsets[b], hi = offsets[b + 1];
+  lo = lo < 0 ? 0 : (lo > total_L ? total_L : lo);
+  hi = hi < lo ? lo : (hi > total_L ? total_L : hi);
+  const int hc = head * DH;
+  for (int i = threadIdx.x; i < N * DH; i += blockDim.x) {
+    const int n = i / DH, c = i % DH;
+    qs[i] = q[((long long)b * N + n) * d + hc + c];
+    das[i] = da[((long long)b * N + n) * ld_da + hc + c];
+    dqs[i] = 0.f;
+  }
+  __syncthreads();
+  const float* kcol = kv + hc;
+  const float* vcol = kv + v_col0 + hc;
+  // phase 1: statistics and delta, one warp per query
+  for (int n = warp; n < N; n += 8) {
+    float m = -INFINITY, l = 0.f;
+    for (long long t = lo + lane; t < hi; t += 32) {
+      float s = 0.f;
+      for (int c = 0; c < DH; ++c) s = fmaf(qs[n * DH + c], kcol[t * kvw + c], s);
+      s *= scale;
+      const float mn = fmaxf(m, s);
+      l = l * __expf(m - mn) + __expf(s - mn);
+      m = mn;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, m, o), l2 = __shfl_xor_sync(0xffffffffu, l, o);
+      const float mn = fmaxf(m, m2);
+      l = (m == -INFINITY ? 0.f : l * __expf(m - mn)) + (m2 == -INFINITY ? 0.f : l2 * __expf(m2 - mn));
+      m = mn;
+    }
+    float dl = 0.f;
+    for (long long t = lo + lane; t < hi; t += 32) {
+      float s = 0.f, dp = 0.f;
+      for (int c = 0; c < DH; ++c) {
+        s = fmaf(qs[n * DH + c], kcol[t * kvw + c], s);
+        dp = fmaf(das[n * DH + c], vcol[t * kvw + c], dp);
+      }
+      dl += __expf(s * scale - m) / l * dp;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, o);
+    if (lane == 0) {
+      mx[n] = m;
+      ls[n] = l;
+      del[n] = dl;
+    }
+  }
+  __syncthreads();
+  // phase 2: one history row per thread
+  for (long long t = lo + threadIdx.x; t < hi; t += blockDim.x) {
+    float kr[DH], vr[DH], dk[DH], dv[DH];
+#pragma unroll
+    for (int c = 0; c < DH; ++c) {
+      kr[c] = kcol[t * kvw + c];
+      vr[c] = vcol[t * kvw + c];
+      dk[c] = 0.f;
+      dv[c] = 0.f;
+    }
+    for (int n = 0; n < N; ++n) {
+      float s = 0.f, dp = 0.f;
+#pragma unroll
+      for (int c = 0; c < DH; ++c) {
+        s = fmaf(qs[n * DH + c], kr[c], s);
+        dp = fmaf(das[n * DH + c], vr[c], dp);
+      }
+      const float p = __expf(s * scale - mx[n]) / ls[n];
+      const float ds = p * (dp - del[n]);
+#pragma unroll
+      for (int c = 0; c < DH; ++c) {
+        dv[c] = fmaf(p, das[n * DH + c], dv[c]);
+        dk[c] = fmaf(ds * scale, qs[n * DH + c], dk[c]);
+        atomicAdd(&dqs[n * DH + c], ds * scale * kr[c]);
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < DH; ++c) {
+      if (shared_kv) {
+        dkv[t * kvw + hc + c] = dk[c] + dv[c];
+      } else {
+        dkv[t * kvw + hc + c] = dk[c];
+        dkv[t * kvw + v_col0 + hc + c] = dv[c];
+      }
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < N * DH; i += blockDim.x) {
+    const int n = i / DH, c = i % DH;
+    dq[((long long)b * N + n) * d + hc + c] = dqs[i];
+  }
+}
+
+}  // namespace whale

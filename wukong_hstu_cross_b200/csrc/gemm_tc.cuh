@@ -9,6 +9,14 @@
 // as an fp32 activation times the weight. The token-side (residual-stream) GEMMs use this;
 // the history-side K|V projection reads bf16 states directly.
 //
+// Operand layouts. An operand is K-major (rows of the operand along M or N, K contiguous: the
+// nn.Linear layout of W, and the activations of the forward) or, with A_MN / B_MN, MN-major (stored
+// [K, M] or [K, N] row-major: M or N contiguous). MN-major tiles are loaded as 64-element-wide TMA
+// boxes of 64 K rows (128-byte swizzle) and described to the MMA with the transpose bit of the
+// instruction descriptor; they let the backward pass contract over the token or history rows
+// (weight gradients dW = dY^T X: both operands MN-major) and multiply by an untransposed weight
+// (dX = dY W: W [K, N] is an MN-major B) without transposing anything in memory.
+//
 // Persistent: CTA c walks the 128 x BN tiles c, c + gridDim.x, ... (N-tiles of a row block are
 // adjacent, so A is re-read from L2, not HBM). Warp roles (192 threads, 320 with ROWNORM):
 //   warp 0      TMA producer: A (hi, lo) and W tiles (64 columns = 128 B, 128-byte swizzle)
@@ -59,16 +67,21 @@ struct GemmArgs {
   // EPI_QABS: the accumulator row m = b * qabs_N + n of head block j (qabs_d columns) is written to
   // row b * qabs_rows + j * qabs_N + n, columns relative to the head block.
   int qabs_N, qabs_d, qabs_rows;
+  // Split-K (ksplit > 1, one K source): tile t of num_tiles = ksplit * tiles_m * tiles_n takes K blocks
+  // [s kb_split, (s + 1) kb_split) of split s = t / (tiles_m tiles_n) and writes its fp32 partial at
+  // out32 + s * split_stride (a later pass sums the partials in split order).
+  int ksplit, kb_split;
+  long long split_stride;
 };
 
 
-template <int BN, bool SPLIT>
+template <int BN, bool SPLIT, bool SPLIT_B = false>
 struct GemmSmem {
   static constexpr int BM = 128, BK = 64;
   static constexpr uint32_t A_BYTES = BM * BK * 2;
   static constexpr uint32_t A_ALL = SPLIT ? 2 * A_BYTES : A_BYTES;
   static constexpr uint32_t B_BYTES = BN * BK * 2;
-  static constexpr uint32_t STAGE_BYTES = A_ALL + B_BYTES;
+  static constexpr uint32_t STAGE_BYTES = A_ALL + (SPLIT_B ? 2 : 1) * B_BYTES;
   // stages fill what the 227 KB of shared memory leaves (one CTA per SM either way): five 40 KB
   // stages for the 64-column hi/lo tiles
   static constexpr int FIXED = 1024 /*alignment slack*/ + 2 * 128 * 4 /*row factors*/ + 256 /*barriers*/;
@@ -94,9 +107,10 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* f) {
 
 // Write NV consecutive fp32 values (NV multiple of 8) of one row to the requested outputs.
 template <int NV>
-__device__ __forceinline__ void store_row_chunk(const GemmArgs& g, long long off, const float* x) {
+__device__ __forceinline__ void store_row_chunk(const GemmArgs& g, long long off, const float* x,
+                                                long long off32 = 0) {
   if (g.out32) {
-    float4* d = reinterpret_cast<float4*>(g.out32 + off);
+    float4* d = reinterpret_cast<float4*>(g.out32 + off32 + off);
 #pragma unroll
     for (int i = 0; i < NV / 4; ++i) d[i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
   }
@@ -147,9 +161,10 @@ __device__ __forceinline__ void epi_load_resid(const GemmArgs& args, long long g
 }
 
 // t_row: TMEM address of this thread's lane at column 0 of the accumulator; r: row factor.
+// off32: extra offset of the fp32 output (a split-K partial's place).
 template <int BN, int EPI>
 __device__ __forceinline__ void epi_tile(const GemmArgs& args, uint32_t t_row, float r, long long gm, bool row_ok,
-                                         int n0, const float4 (&pre)[EpiPre<BN, EPI>::kN]) {
+                                         int n0, const float4 (&pre)[EpiPre<BN, EPI>::kN], long long off32 = 0) {
   constexpr bool kPre = EpiPre<BN, EPI>::kOn;
   auto chunk = [&](const int c, const uint32_t (&v)[32]) {
     const int col = n0 + c * 32;
@@ -186,7 +201,7 @@ __device__ __forceinline__ void epi_tile(const GemmArgs& args, uint32_t t_row, f
             (gm / args.qabs_N) * args.qabs_rows + (long long)head * args.qabs_N + gm % args.qabs_N;
         store_row_chunk<32>(args, orow * args.ldo + (col - head * args.qabs_d), x);
       } else {
-        store_row_chunk<32>(args, gm * args.ldo + col, x);
+        store_row_chunk<32>(args, gm * args.ldo + col, x, off32);
       }
     }
   };
@@ -204,14 +219,23 @@ __device__ __forceinline__ void epi_tile(const GemmArgs& args, uint32_t t_row, f
   }
 }
 
-template <int BN, int EPI, bool ROWNORM, bool SPLIT>
+// Instruction-descriptor bit selecting an MN-major A operand.
+constexpr uint32_t kIdescAMnMajor = 1u << 15;
+
+// SPLIT_B: B is a hi/lo pair too (single A source: tmA1 then holds B's lo half), and every k-step
+// issues A_hi B_hi, A_lo B_hi and A_hi B_lo (the A_lo B_lo term is below 2^-16 of the product):
+// the weight gradients of the token side, whose sums over rows cancel, need both operands at ~16 bits.
+template <int BN, int EPI, bool ROWNORM, bool SPLIT, bool A_MN = false, bool B_MN = false, bool SPLIT_B = false>
 __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA0lo,
                    const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmA1lo,
                    const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
-  using L = GemmSmem<BN, SPLIT>;
+  using L = GemmSmem<BN, SPLIT, SPLIT_B>;
   constexpr int STAGES = L::STAGES;
   constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators: 128, 256 or 512 columns
+  static_assert(!(ROWNORM && A_MN), "row statistics read K-major A rows");
+  static_assert(!(ROWNORM && SPLIT_B), "row-normalised GEMMs have one B");
+  constexpr uint32_t MN_BOX = 64 * 64 * 2;  // one MN-major box: 64 K rows x 64 elements
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   // stage s: [A hi | A lo (SPLIT) | W]; then row factors [2][128]; then barriers
@@ -227,6 +251,17 @@ __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int KB = args.kb0 + args.kb1;
+  const int nsplit = args.ksplit > 1 ? args.ksplit : 1;
+  const int tiles_mn = args.num_tiles / nsplit;
+  // tile -> (split, m0, n0) and the split's K blocks [kb_lo, kb_hi)
+  auto tile_of = [&](int tile, int& m0, int& n0, int& kb_lo, int& kb_hi, int& split) {
+    split = tile / tiles_mn;
+    const int tmn = tile - split * tiles_mn;
+    m0 = (tmn / args.tiles_n) * L::BM;
+    n0 = (tmn % args.tiles_n) * BN;
+    kb_lo = nsplit > 1 ? split * args.kb_split : 0;
+    kb_hi = nsplit > 1 ? min(KB, kb_lo + args.kb_split) : KB;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -247,6 +282,7 @@ __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
     tma_prefetch_desc(&tmA0);
     tma_prefetch_desc(&tmB);
     if (SPLIT) tma_prefetch_desc(&tmA0lo);
+    if (SPLIT_B) tma_prefetch_desc(&tmA1);
     if (args.kb1 > 0) {
       tma_prefetch_desc(&tmA1);
       if (SPLIT) tma_prefetch_desc(&tmA1lo);
@@ -269,8 +305,9 @@ __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
       int kg = 0;
       bool stop = false;
       for (int tile = blockIdx.x; tile < args.num_tiles && !stop; tile += gridDim.x) {
-        const int m0 = (tile / args.tiles_n) * L::BM, n0 = (tile % args.tiles_n) * BN;
-        for (int kb = 0; kb < KB; ++kb, ++kg) {
+        int m0, n0, kb_lo, kb_hi, split;
+        tile_of(tile, m0, n0, kb_lo, kb_hi, split);
+        for (int kb = kb_lo; kb < kb_hi; ++kb, ++kg) {
           const int s = kg % STAGES, u = kg / STAGES;
           if (kg >= STAGES && !mbar_wait(&empty[s], (u - 1) & 1, abort_flag)) {
             stop = true;
@@ -285,9 +322,26 @@ __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
             kc += head * args.a_kb_step * L::BK;
             ma += (int)(head * args.a_row_step);
           }
-          tma_load_2d(st, first ? &tmA0 : &tmA1, kc, ma, &full[s]);
-          if (SPLIT) tma_load_2d(st + L::A_BYTES, first ? &tmA0lo : &tmA1lo, kc, ma, &full[s]);
-          tma_load_2d(st + L::A_ALL, &tmB, kb * L::BK, n0, &full[s]);
+          if (A_MN) {
+#pragma unroll
+            for (int i = 0; i < L::BM / 64; ++i) {
+              tma_load_2d(st + i * MN_BOX, first ? &tmA0 : &tmA1, ma + 64 * i, kc, &full[s]);
+              if (SPLIT) tma_load_2d(st + L::A_BYTES + i * MN_BOX, first ? &tmA0lo : &tmA1lo, ma + 64 * i, kc, &full[s]);
+            }
+          } else {
+            tma_load_2d(st, first ? &tmA0 : &tmA1, kc, ma, &full[s]);
+            if (SPLIT) tma_load_2d(st + L::A_BYTES, first ? &tmA0lo : &tmA1lo, kc, ma, &full[s]);
+          }
+          if (B_MN) {
+#pragma unroll
+            for (int i = 0; i < BN / 64; ++i) {
+              tma_load_2d(st + L::A_ALL + i * MN_BOX, &tmB, n0 + 64 * i, kb * L::BK, &full[s]);
+              if (SPLIT_B) tma_load_2d(st + L::A_ALL + L::B_BYTES + i * MN_BOX, &tmA1, n0 + 64 * i, kb * L::BK, &full[s]);
+            }
+          } else {
+            tma_load_2d(st + L::A_ALL, &tmB, kb * L::BK, n0, &full[s]);
+            if (SPLIT_B) tma_load_2d(st + L::A_ALL + L::B_BYTES, &tmA1, kb * L::BK, n0, &full[s]);
+          }
         }
       }
       if (*abort_flag) {
@@ -300,7 +354,8 @@ __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
   } else if (warp == 1) {
     // ---------------- MMA issuer: tile i accumulates into buffer i % 2 ----------------
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
+      constexpr uint32_t idesc =
+          idesc_bf16_f32(128, BN) | (A_MN ? kIdescAMnMajor : 0u) | (B_MN ? kIdescBMnMajor : 0u);
       int kg = 0, it = 0;
       bool stop = false;
       for (int tile = blockIdx.x; tile < args.num_tiles && !stop; tile += gridDim.x, ++it) {
@@ -308,7 +363,9 @@ __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
         if (it >= 2 && !mbar_wait(&tempty[acc], (ua - 1) & 1, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int kb = 0; kb < KB; ++kb, ++kg) {
+        int m0, n0, kb_lo, kb_hi, split;
+        tile_of(tile, m0, n0, kb_lo, kb_hi, split);
+        for (int kb = kb_lo; kb < kb_hi; ++kb, ++kg) {
           const int s = kg % STAGES, u = kg / STAGES;
           if (!mbar_wait(&full[s], u & 1, abort_flag)) {
             stop = true;
@@ -319,9 +376,17 @@ __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
           const uint32_t b_base = a_base + L::A_ALL;
 #pragma unroll
           for (int kk = 0; kk < L::BK / 16; ++kk) {
-            const uint64_t bdesc = sdesc_k_sw128(b_base + kk * 32);
-            umma_f16(d_tmem, sdesc_k_sw128(a_base + kk * 32), bdesc, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
-            if (SPLIT) umma_f16(d_tmem, sdesc_k_sw128(a_base + L::A_BYTES + kk * 32), bdesc, idesc, 1u);
+            // MN-major: 16 K rows of 128 bytes per k-step; 64-element MN groups one box apart
+            auto bd = [&](uint32_t base) {
+              return B_MN ? sdesc_mn_sw128(base + kk * 2048, MN_BOX, 1024) : sdesc_k_sw128(base + kk * 32);
+            };
+            auto ad = [&](uint32_t base) {
+              return A_MN ? sdesc_mn_sw128(base + kk * 2048, MN_BOX, 1024) : sdesc_k_sw128(base + kk * 32);
+            };
+            const uint64_t bdesc = bd(b_base), adesc = ad(a_base);
+            umma_f16(d_tmem, adesc, bdesc, idesc, (kb > kb_lo || kk > 0) ? 1u : 0u);
+            if (SPLIT) umma_f16(d_tmem, ad(a_base + L::A_BYTES), bdesc, idesc, 1u);
+            if (SPLIT_B) umma_f16(d_tmem, adesc, bd(b_base + L::B_BYTES), idesc, 1u);
           }
           umma_commit(&empty[s]);
         }
@@ -381,7 +446,8 @@ __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
     int it = 0;
     for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1, ua = it >> 1;
-      const int m0 = (tile / args.tiles_n) * L::BM, n0 = (tile % args.tiles_n) * BN;
+      int m0, n0, kb_lo, kb_hi, split;
+      tile_of(tile, m0, n0, kb_lo, kb_hi, split);
       const long long gm = (long long)m0 + row;
       const bool row_ok = gm < args.M;
       epi_load_resid<BN, EPI>(args, gm, row_ok, n0, pre);
@@ -389,7 +455,8 @@ __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
       if (ROWNORM && !mbar_wait(&nfull[acc], ua & 1, abort_flag)) break;
       tc_fence_after();
       const float r = ROWNORM ? rbuf[acc * 128 + row] : 1.0f;
-      epi_tile<BN, EPI>(args, tmem_base + acc * BN + ((uint32_t)(q * 32) << 16), r, gm, row_ok, n0, pre);
+      epi_tile<BN, EPI>(args, tmem_base + acc * BN + ((uint32_t)(q * 32) << 16), r, gm, row_ok, n0, pre,
+                        nsplit > 1 ? split * args.split_stride : 0ll);
       // this accumulator buffer and its row factors may be reused
       tc_fence_before();
       __syncwarp();

@@ -30,6 +30,8 @@
 #include "aux_kernels.cuh"
 #include "attention.cuh"
 #include "attention_qtile.cuh"
+#include "attention_bwd.cuh"
+#include "backward.cuh"
 #include "fp32_path.cuh"
 #include "gemm_2sm.cuh"
 #include "gemm_tc.cuh"
@@ -380,10 +382,10 @@ struct Outs {
   long long ld;
 };
 
-template <int BN, int EPI, bool RN, bool SPLIT>
+template <int BN, int EPI, bool RN, bool SPLIT, bool A_MN = false, bool B_MN = false, bool SPLIT_B = false>
 whale_status launch_gemm_t(const CUtensorMap* tm, const GemmArgs& g, long long tiles, cudaStream_t st) {
-  const size_t smem = GemmSmem<BN, SPLIT>::BYTES;
-  auto kern = gemm_tc_kernel<BN, EPI, RN, SPLIT>;
+  const size_t smem = GemmSmem<BN, SPLIT, SPLIT_B>::BYTES;
+  auto kern = gemm_tc_kernel<BN, EPI, RN, SPLIT, A_MN, B_MN, SPLIT_B>;
   CUCHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   const unsigned grid = (unsigned)(tiles < kNumSM ? tiles : kNumSM);
   return launch_pdl(kern, dim3(grid), dim3(gemm_threads<RN>()), smem, st, tm[0], tm[1], tm[2], tm[3], tm[4], g);
@@ -395,6 +397,7 @@ whale_status launch_gemm_bn(int epi, bool rn, bool split, const CUtensorMap* tm,
   if (rn && epi == EPI_STORE && !split) return launch_gemm_t<BN, EPI_STORE, true, false>(tm, g, tiles, st);
   if (rn && epi == EPI_STORE && split) return launch_gemm_t<BN, EPI_STORE, true, true>(tm, g, tiles, st);
   if (!split) return WHALE_ERR_UNSUPPORTED;
+  if (!rn && epi == EPI_STORE) return launch_gemm_t<BN, EPI_STORE, false, true>(tm, g, tiles, st);
   if (rn && epi == EPI_SWIGLU) return launch_gemm_t<BN, EPI_SWIGLU, true, true>(tm, g, tiles, st);
   if (rn && epi == EPI_SWIGLU_TIED) return launch_gemm_t<BN, EPI_SWIGLU_TIED, true, true>(tm, g, tiles, st);
   if (!rn && epi == EPI_SILU) return launch_gemm_t<BN, EPI_SILU, false, true>(tm, g, tiles, st);
@@ -517,6 +520,123 @@ whale_status gemm_bf16(const Opnd& a0, const Opnd& a1, const void* W, int N, con
   return launch_gemm_bn<64>(epi, rn, split, maps, g, tiles, st);
 }
 
+// ------------------------------------------------------------------------------------------
+// General bf16 contraction into fp32 for the backward pass: C[M, N] = sum_k A(m, k) B(k, n).
+//   A: K-major [M, K] (a.hi, optional bf16 residue a.lo: two MMAs per k-step; row stride a.ld), or
+//      with a_mn MN-major [K, M] (a.hi only, row stride a.ld);
+//   B: K-major [N, K] (row stride ldb) or, with b_mn, MN-major [K, N] (row stride ldb).
+// K need not be a multiple of 64 (the TMA boxes read zeros past K). Output tiles that would leave SMs
+// idle with a long K take split-K: fp32 partials of ksplit K ranges in `part` (part_cap floats), then
+// summed in split order (deterministic).
+// ------------------------------------------------------------------------------------------
+template <int BN>
+whale_status launch_acc32_bn(bool split, bool split_b, bool a_mn, bool b_mn, const CUtensorMap* tm, const GemmArgs& g,
+                             long long tiles, cudaStream_t st) {
+  if (!b_mn) return WHALE_ERR_UNSUPPORTED;
+  if (!a_mn && split && !split_b) return launch_gemm_t<BN, EPI_STORE, false, true, false, true>(tm, g, tiles, st);
+  if (!a_mn && !split && !split_b) return launch_gemm_t<BN, EPI_STORE, false, false, false, true>(tm, g, tiles, st);
+  if (a_mn && !split && !split_b) return launch_gemm_t<BN, EPI_STORE, false, false, true, true>(tm, g, tiles, st);
+  if (a_mn && split && !split_b) return launch_gemm_t<BN, EPI_STORE, false, true, true, true>(tm, g, tiles, st);
+  if (a_mn && split && split_b) return launch_gemm_t<BN, EPI_STORE, false, true, true, true, true>(tm, g, tiles, st);
+  return WHALE_ERR_UNSUPPORTED;
+}
+
+whale_status gemm_acc32(const void* a_hi, const void* a_lo, long long lda, bool a_mn, const void* b, long long ldb,
+                        bool b_mn, long long M, int N, long long K, float* c, long long ldc, float* part,
+                        size_t part_cap, cudaStream_t st, const void* b_lo = nullptr) {
+  if (M <= 0 || N <= 0) return WHALE_OK;
+  if (K <= 0) {
+    for (long long r = 0; r < M; ++r) CUCHECK(cudaMemsetAsync(c + r * ldc, 0, (size_t)N * 4, st));
+    return WHALE_OK;
+  }
+  if (M >= (1ll << 31) || K >= (1ll << 31) || N % 64) return WHALE_ERR_UNSUPPORTED;
+  const bool split = a_lo != nullptr, split_b = b_lo != nullptr;
+  if (split_b && !split) return WHALE_ERR_UNSUPPORTED;
+  const long long tm = cdiv<long long>(M, 128);
+  const long long KB = cdiv<long long>(K, 64);
+  // tile width: the cost model of gemm_bf16 (per persistent CTA: tiles x K blocks x max(MMA, bytes))
+  auto cost = [&](int bn) -> double {
+    if (N % bn) return 1e300;
+    const double per_cta = (double)cdiv<long long>(tm * (N / bn), kNumSM);
+    const double mma = (split ? (split_b ? 6.0 : 4.0) : 2.0) * bn;
+    const double bytes = (split ? 32768.0 : 16384.0) + bn * 128.0 * (split_b ? 2 : 1);
+    return 5600.0 + per_cta * KB * std::max(mma, bytes / 80.0);
+  };
+  int bn = 64;
+  for (int cand : {128, 256})
+    if (cost(cand) < cost(bn) && (!split_b || cand <= 128)) bn = cand;  // pairs on both: stages of 64 KB at most
+  const long long tiles_mn = tm * (N / bn);
+  // split-K: enough tiles to fill the SMs once, at least 8 K blocks per split, partials within part_cap
+  int ks = 1;
+  if (tiles_mn < kNumSM && KB >= 16 && part) {
+    long long want = std::min<long long>(cdiv<long long>(kNumSM, tiles_mn), KB / 8);
+    while (want > 1 && (size_t)want * M * N > part_cap) --want;
+    ks = (int)std::max<long long>(1, std::min<long long>(want, 64));
+  }
+  int kb_split = (int)cdiv<long long>(KB, ks);
+  ks = (int)cdiv<long long>(KB, kb_split);  // no empty split
+  CUtensorMap maps[5];
+  if (a_mn) {
+    WCHECK(tmap_bf16_box(&maps[0], a_hi, K, M, lda, 64, 64));
+    if (split) WCHECK(tmap_bf16_box(&maps[1], a_lo, K, M, lda, 64, 64));
+    else maps[1] = maps[0];
+  } else {
+    WCHECK(tmap_bf16(&maps[0], a_hi, M, K, lda, 128));
+    if (split) WCHECK(tmap_bf16(&maps[1], a_lo, M, K, lda, 128));
+    else maps[1] = maps[0];
+  }
+  maps[2] = maps[0];
+  maps[3] = maps[1];
+  if (b_mn) {
+    WCHECK(tmap_bf16_box(&maps[4], b, K, N, ldb, 64, 64));
+    if (split_b) WCHECK(tmap_bf16_box(&maps[2], b_lo, K, N, ldb, 64, 64));  // B's lo half rides in the A1 slot
+  } else {
+    WCHECK(tmap_bf16(&maps[4], b, N, K, ldb, bn));
+    if (split_b) WCHECK(tmap_bf16(&maps[2], b_lo, N, K, ldb, bn));
+  }
+  GemmArgs g{};
+  g.M = (int)M;
+  g.N = N;
+  g.kb0 = (int)KB;
+  g.kb1 = 0;
+  g.tiles_n = N / bn;
+  g.num_tiles = (int)(tiles_mn * ks);
+  g.ksplit = ks;
+  g.kb_split = kb_split;
+  if (ks > 1) {
+    g.out32 = part;
+    g.ldo = N;
+    g.split_stride = M * N;
+  } else {
+    g.out32 = c;
+    g.ldo = ldc;
+  }
+  const long long tiles = tiles_mn * ks;
+  whale_status r;
+  if (bn == 256) r = launch_acc32_bn<256>(split, split_b, a_mn, b_mn, maps, g, tiles, st);
+  else if (bn == 128) r = launch_acc32_bn<128>(split, split_b, a_mn, b_mn, maps, g, tiles, st);
+  else r = launch_acc32_bn<64>(split, split_b, a_mn, b_mn, maps, g, tiles, st);
+  WCHECK(r);
+  if (ks > 1) {
+    const unsigned grid = (unsigned)std::min<long long>(cdiv<long long>(M * N, 256), 8 * kNumSM);
+    WCHECK(launch_pdl(sum_partials_kernel, dim3(grid), dim3(256), 0, st, (const float*)part, ks, M, N, c, ldc));
+  }
+  return WHALE_OK;
+}
+
+// fp32 (SIMT) contraction with arbitrary strides: C[m, n] = sum_k A[m sam + k sak] B[k sbk + n sbn].
+whale_status gemm_strided_f32(const float* A, long long sam, long long sak, const float* B, long long sbk,
+                              long long sbn, float* C, long long ldc, long long M, long long N, long long K,
+                              cudaStream_t st) {
+  if (M <= 0 || N <= 0) return WHALE_OK;
+  const long long gy = cdiv<long long>(M, 64);
+  if (gy > 65535) return WHALE_ERR_UNSUPPORTED;
+  gemm_strided_f32_kernel<<<dim3((unsigned)cdiv<long long>(N, 64), (unsigned)gy), 256, 0, st>>>(
+      A, sam, sak, B, sbk, sbn, C, ldc, M, N, K, 0);
+  CUCHECK(cudaGetLastError());
+  return WHALE_OK;
+}
+
 inline Opnd opnd(const void* hi, const void* lo, long long ld, int K) { return Opnd{hi, lo, ld, K}; }
 inline Opnd no_opnd() { return Opnd{nullptr, nullptr, 0, 0}; }
 
@@ -620,8 +740,10 @@ whale_status attention_qtile(const Shape& s, const void* q, const void* kv, cons
 // needs no scratch; the split-L kernel (partials in the scratch of plan_attention) takes the rest.
 bool attention_is_query_tiled(const Shape& s) { return s.N >= 128 && (s.dh == 32 || s.dh == 64); }
 
+// lse (optional, split-L kernel only): [B*N, h] log2 softmax denominators for the backward pass.
 whale_status attention_bf16(const Shape& s, const void* q, const void* kv, const int* offsets, void* out,
-                            void* out_lo, int B, long long total_L, void* scratch, cudaStream_t st) {
+                            void* out_lo, int B, long long total_L, void* scratch, cudaStream_t st,
+                            float* lse = nullptr) {
   if (B == 0) return WHALE_OK;
   const AttnPlan p = plan_attention(s, B, total_L);
   const size_t rows = (size_t)B * s.N;
@@ -630,8 +752,12 @@ whale_status attention_bf16(const Shape& s, const void* q, const void* kv, const
     if (out_lo) CUCHECK(cudaMemsetAsync(out_lo, 0, rows * s.d * 2, st));
     return WHALE_OK;
   }
-  if (attention_is_query_tiled(s)) return attention_qtile(s, q, kv, offsets, out, out_lo, B, total_L, st);
+  if (attention_is_query_tiled(s)) {
+    if (lse) return WHALE_ERR_UNSUPPORTED;
+    return attention_qtile(s, q, kv, offsets, out, out_lo, B, total_L, st);
+  }
   AttnArgs a{};
+  a.lse = lse;
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.offsets = offsets;
   a.part_o = reinterpret_cast<float*>(at(scratch, p.po_off()));
@@ -1124,6 +1250,396 @@ size_t host_staging_bytes(const Shape& s, const whale_shape_hint& h, size_t* o_t
   return o;
 }
 
+// ============================================================================================
+// Backward pass of one fusion layer (the vector-Jacobian product for dY = dLoss/dH_f): the forward
+// is recomputed (materialised K|V path, with the softmax log-sum-exp kept), then its steps are
+// reversed. bf16 mode: tcgen05 GEMMs (MN-major operands for the untransposed weights and for the
+// weight gradients, which contract over token or history rows; split-K where the output is small),
+// the KV-parallel tensor-core attention backward, fused element-wise and RMSNorm-backward row
+// kernels. fp32 mode: the same steps with SIMT kernels.
+// ============================================================================================
+constexpr int kColpBlocks = 8 * kNumSM;  // row-kernel blocks (column partials of the gain gradients)
+
+inline int rows_blocks(long long rows) {
+  return (int)std::max<long long>(1, std::min<long long>(cdiv<long long>(rows, 32), kColpBlocks));
+}
+
+struct BwdBufs {
+  // forward recompute
+  void *x32, *xlo, *r, *q, *q_lo, *sn, *sn_lo, *kv, *kv_lo, *attn, *a, *a_lo, *lse, *z1, *g, *g_lo, *f32, *f, *f_lo,
+      *ug;
+  // backward
+  void *dy, *dy_lo, *dm, *msw, *msw_lo, *dug, *dug_lo, *dn, *nrm, *nrm_lo, *nq, *nq_lo, *df32, *df, *df_lo, *dhid,
+      *dz, *dz_lo, *dc, *da16, *da_lo, *delta, *dq, *dq_hi, *dq_lo, *cst, *dkv, *dkv_lo, *dsn, *colp, *part;
+  size_t part_floats;
+};
+
+// Buffers of the backward workspace (null pointers when base is null); returns its size in bytes.
+size_t bwd_buffers(const Shape& s, const whale_shape_hint& h, char* base, BwdBufs* b) {
+  size_t o = 0;
+  auto take = [&](size_t bytes) -> void* {
+    void* p = base ? base + o : nullptr;
+    o = align_up(o + bytes);
+    return p;
+  };
+  const size_t rows = (size_t)h.B * s.N, T = (size_t)h.total_L, d = s.d, H = s.H, Fh = s.Fh;
+  const size_t ugw = s.ugw, kvw = s.kvw, nh = s.h;
+  const size_t e = s.bf16 ? 2 : 4;  // element size of the operand copies
+  *b = BwdBufs{};
+  if (s.bf16) {
+    b->x32 = take(rows * d * 4);
+    b->xlo = take(rows * d * 2);
+    b->attn = take(plan_attention(s, h.B, h.total_L).bytes());
+    b->lse = take(rows * nh * 4);
+  } else {
+    b->r = take(std::max(rows, T) * 4);
+  }
+  b->q = take(rows * d * e);
+  b->kv = take(T * kvw * e);
+  b->sn = take(T * d * e);
+  if (s.bf16) {
+    b->q_lo = take(rows * d * 2);
+    b->kv_lo = take(T * kvw * 2);
+    b->sn_lo = take(T * d * 2);
+  }
+  b->a = take(rows * d * e);
+  if (s.bf16) b->a_lo = take(rows * d * 2);
+  if (Fh) {
+    b->z1 = take(rows * Fh * 4);
+    b->g = take(rows * Fh * e);
+    if (s.bf16) b->g_lo = take(rows * Fh * 2);
+  }
+  b->f32 = take(rows * d * 4);
+  if (s.bf16) {
+    b->f = take(rows * d * 2);
+    b->f_lo = take(rows * d * 2);
+  }
+  b->ug = take(rows * ugw * 4);
+  if (s.bf16) {
+    b->dy = take(rows * d * 2);
+    b->dy_lo = take(rows * d * 2);
+  }
+  b->dm = take(rows * H * 4);
+  b->msw = take(rows * H * e);
+  if (s.bf16) b->msw_lo = take(rows * H * 2);
+  b->dug = take(rows * ugw * e);
+  if (s.bf16) b->dug_lo = take(rows * ugw * 2);
+  b->dn = take(rows * d * 4);
+  b->nrm = take(rows * d * e);
+  if (s.bf16) {
+    b->nrm_lo = take(rows * d * 2);
+    b->nq = take(rows * d * 2);
+    b->nq_lo = take(rows * d * 2);
+  }
+  b->df32 = take(rows * d * 4);
+  if (s.bf16) {
+    b->df = take(rows * d * 2);
+    b->df_lo = take(rows * d * 2);
+  }
+  if (Fh) {
+    b->dhid = take(rows * Fh * 4);
+    b->dz = take(rows * Fh * e);
+    if (s.bf16) b->dz_lo = take(rows * Fh * 2);
+  }
+  b->dc = take(rows * 2 * d * 4);
+  if (s.bf16) {
+    b->da16 = take(rows * d * 2);
+    b->da_lo = take(rows * d * 2);
+    b->delta = take(rows * nh * 4);
+    b->dq_hi = take(rows * d * 2);
+    b->dq_lo = take(rows * d * 2);
+    b->cst = take(((size_t)h.B + 1) * 4);
+  }
+  b->dq = take(rows * d * 4);
+  b->dkv = take(T * kvw * e);
+  if (s.bf16) b->dkv_lo = take(T * kvw * 2);
+  b->dsn = take(T * d * 4);
+  b->colp = take((size_t)kColpBlocks * d * 4);
+  const size_t mn = std::max({d * H, ugw * d, d * std::max(Fh, d), kvw * d});
+  b->part_floats = s.bf16 ? 16 * mn : 0;
+  b->part = s.bf16 ? take(b->part_floats * 4) : nullptr;
+  return o;
+}
+
+// Gain gradient: the row kernel's column partials summed in block order.
+whale_status gain_grad(const float* colp, int blocks, int d, float* dg, cudaStream_t st) {
+  if (!dg) return WHALE_OK;
+  return launch_pdl(sum_partials_kernel, dim3((unsigned)cdiv(d, 256)), dim3(256), 0, st, colp, blocks, 1ll, d, dg,
+                    (long long)d);
+}
+
+template <typename TX>
+whale_status rms_bwd(const TX* x, const float* g, const float* dn, long long rows, int d, float eps,
+                     const float* r1, long long ld1, const float* r2, long long ld2, float* dx32, void* dx_hi,
+                     void* dx_lo, void* n_out, void* n_lo, float* n32, float* colp, float* dg, cudaStream_t st) {
+  if (rows <= 0) {
+    if (dg) CUCHECK(cudaMemsetAsync(dg, 0, (size_t)d * 4, st));
+    return WHALE_OK;
+  }
+  const int blocks = rows_blocks(rows);
+  WCHECK(launch_pdl(rms_bwd_kernel<TX>, dim3(blocks), dim3(256), 0, st, x, g, dn, rows, d, eps, r1, ld1, r2, ld2, dx32,
+                    static_cast<__nv_bfloat16*>(dx_hi), static_cast<__nv_bfloat16*>(dx_lo),
+                    static_cast<__nv_bfloat16*>(n_out), static_cast<__nv_bfloat16*>(n_lo), n32, colp));
+  return gain_grad(colp, blocks, d, dg, st);
+}
+
+template <typename F, typename... A>
+whale_status ew_launch(F kern, long long n, cudaStream_t st, A... args) {
+  if (n <= 0) return WHALE_OK;
+  const unsigned grid = (unsigned)std::min<long long>(cdiv<long long>(n, 256), 8 * kNumSM);
+  return launch_pdl(kern, dim3(grid), dim3(256), 0, st, args...);
+}
+
+template <int DH, int NQ>
+whale_status launch_attn_bwd(const AttnBwdArgs& a, unsigned chunks, cudaStream_t st) {
+  using C = AttnBwdCfg<DH, NQ>;
+  if (a.n_heads % C::HG) return WHALE_ERR_UNSUPPORTED;
+  CUCHECK(cudaFuncSetAttribute(attn_bwd_kernel<DH, NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::BYTES));
+  return launch_pdl(attn_bwd_kernel<DH, NQ>, dim3(chunks, a.n_heads / C::HG), dim3(C::THREADS), C::BYTES, st, a);
+}
+
+// Shapes the backward pass supports: bf16 with at most 32 queries per example (the KV-parallel
+// attention backward keeps all of an example's queries resident), d a multiple of 128 (its head
+// groups span 128 columns) and d <= 1024 (row kernels); fp32 with d_head <= 64.
+bool backward_shape_ok(const Shape& s) {
+  if (s.d > 1024 || s.d % 32) return false;
+  if (s.bf16) return s.N <= 32 && (s.dh == 32 || s.dh == 64) && s.d % 128 == 0;
+  return s.dh == 8 || s.dh == 16 || s.dh == 32 || s.dh == 64;
+}
+
+whale_status layer_backward_bf16(const Shape& s, const void* x, const void* slab, const int* offsets,
+                                 const whale_layer_weights& w, const float* dy, float* dx, void* ds,
+                                 const whale_layer_grads& gr, const whale_shape_hint& h, const BwdBufs& b,
+                                 cudaStream_t st) {
+  using bf = __nv_bfloat16;
+  const long long rows = (long long)h.B * s.N, T = h.total_L;
+  const int d = s.d, H = s.H, Fh = s.Fh, ugw = s.ugw, kvw = s.kvw;
+  auto F = [](void* p) { return static_cast<float*>(p); };
+  // ---- forward recompute ----
+  WCHECK(pair_from_bf16(x, F(b.x32), b.xlo, rows * d, st));
+  const Opnd X = opnd(x, b.xlo, d, d);
+  // Token side: the normalised rows n = r x g as a hi/lo pair times the raw (exact) weights; folding g
+  // into a bf16 weight would round every product's weight by up to 2^-9, an error the weight
+  // gradients (sums over rows) would carry.
+  WCHECK(launch_pdl(rms_rows_kernel<bf>, dim3(rows_blocks(rows)), dim3(256), 0, st, static_cast<const bf*>(x), w.g_q,
+                    rows, d, s.eps, static_cast<bf*>(b.nq), static_cast<bf*>(b.nq_lo), (float*)nullptr));
+  WCHECK(gemm_bf16(opnd(b.nq, b.nq_lo, d, d), no_opnd(), w.w_q, d, Outs{b.q, b.q_lo, nullptr, d}, nullptr, 0, rows,
+                   EPI_STORE, false, 0.f, st));
+  // History side the same way: K|V = (r s g) W_kv^T from the normalised states as a pair, written as a
+  // pair (the attention backward reads both halves; the forward attention below reads hi).
+  if (T > 0) {
+    WCHECK(launch_pdl(rms_rows_kernel<bf>, dim3(rows_blocks(T)), dim3(256), 0, st, static_cast<const bf*>(slab),
+                      w.g_kv, T, d, s.eps, static_cast<bf*>(b.sn), static_cast<bf*>(b.sn_lo), (float*)nullptr));
+    WCHECK(gemm_bf16(opnd(b.sn, b.sn_lo, d, d), no_opnd(), w.w_kv, kvw, Outs{b.kv, b.kv_lo, nullptr, kvw}, nullptr, 0,
+                     T, EPI_STORE, false, 0.f, st));
+  }
+  WCHECK(attention_bf16(s, b.q, b.kv, offsets, b.a, b.a_lo, h.B, T, b.attn, st, F(b.lse)));
+  const Opnd A = opnd(b.a, b.a_lo, d, d);
+  if (Fh > 0) {
+    WCHECK(gemm_bf16(A, X, w.w_f1, Fh, Outs{nullptr, nullptr, F(b.z1), Fh}, nullptr, 0, rows, EPI_STORE, false, 0.f,
+                     st));
+    WCHECK(ew_launch(silu_pair_kernel, rows * Fh, st, (const float*)F(b.z1), (float*)nullptr, static_cast<bf*>(b.g),
+                     static_cast<bf*>(b.g_lo), rows * Fh));
+    WCHECK(gemm_bf16(opnd(b.g, b.g_lo, Fh, Fh), no_opnd(), w.w_f2, d, Outs{b.f, b.f_lo, F(b.f32), d}, F(b.x32), d,
+                     rows, EPI_RESID, false, 0.f, st));
+  } else {
+    WCHECK(gemm_bf16(A, X, w.w_f2, d, Outs{b.f, b.f_lo, F(b.f32), d}, F(b.x32), d, rows, EPI_RESID, false, 0.f, st));
+  }
+  WCHECK(launch_pdl(rms_rows_kernel<float>, dim3(rows_blocks(rows)), dim3(256), 0, st, (const float*)F(b.f32),
+                    w.g_ffn, rows, d, s.eps, static_cast<bf*>(b.nrm), static_cast<bf*>(b.nrm_lo), (float*)nullptr));
+  WCHECK(gemm_bf16(opnd(b.nrm, b.nrm_lo, d, d), no_opnd(), w.w_upgate, ugw, Outs{nullptr, nullptr, F(b.ug), ugw},
+                   nullptr, 0, rows, EPI_STORE, false, 0.f, st));
+  // ---- S5 backward: SwiGLU FFN ----
+  float* part = F(b.part);
+  const size_t pc = b.part_floats;
+  WCHECK(ew_launch(split_pair_kernel, rows * d, st, dy, (long long)d, static_cast<bf*>(b.dy), static_cast<bf*>(b.dy_lo),
+                   (long long)d, rows, d));
+  WCHECK(gemm_acc32(b.dy, b.dy_lo, d, false, w.w_down, H, true, rows, H, d, F(b.dm), H, part, pc, st));
+  WCHECK(ew_launch(swiglu_bwd_kernel, rows * H, st, (const float*)F(b.ug), (const float*)F(b.dm), rows, H,
+                   s.tied ? 1 : 0, static_cast<bf*>(b.msw), static_cast<bf*>(b.msw_lo), (float*)nullptr,
+                   (float*)nullptr, static_cast<bf*>(b.dug), static_cast<bf*>(b.dug_lo)));
+  // token-side weight gradients: both operands as hi/lo pairs (their sums over rows cancel)
+  WCHECK(gemm_acc32(b.dy, b.dy_lo, d, true, b.msw, H, true, d, H, rows, gr.w_down, H, part, pc, st, b.msw_lo));
+  WCHECK(gemm_acc32(b.dug, b.dug_lo, ugw, false, w.w_upgate, d, true, rows, d, ugw, F(b.dn), d, part, pc, st));
+  WCHECK(rms_bwd<float>(F(b.f32), w.g_ffn, F(b.dn), rows, d, s.eps, dy, d, nullptr, 0, F(b.df32), b.df, b.df_lo,
+                        nullptr, nullptr, nullptr, F(b.colp), gr.g_ffn, st));
+  WCHECK(gemm_acc32(b.dug, b.dug_lo, ugw, true, b.nrm, d, true, ugw, d, rows, gr.w_upgate, d, part, pc, st, b.nrm_lo));
+  // ---- S4 backward: Fusion MLP (dc = d[A | H_w]) ----
+  if (Fh > 0) {
+    WCHECK(gemm_acc32(b.df, b.df_lo, d, false, w.w_f2, Fh, true, rows, Fh, d, F(b.dhid), Fh, part, pc, st));
+    WCHECK(ew_launch(silu_bwd_kernel, rows * Fh, st, (const float*)F(b.dhid), (const float*)F(b.z1), (float*)nullptr,
+                     static_cast<bf*>(b.dz), static_cast<bf*>(b.dz_lo), rows * Fh));
+    WCHECK(gemm_acc32(b.df, b.df_lo, d, true, b.g, Fh, true, d, Fh, rows, gr.w_f2, Fh, part, pc, st, b.g_lo));
+    WCHECK(gemm_acc32(b.dz, b.dz_lo, Fh, false, w.w_f1, 2 * d, true, rows, 2 * d, Fh, F(b.dc), 2 * d, part, pc, st));
+    WCHECK(gemm_acc32(b.dz, b.dz_lo, Fh, true, b.a, d, true, Fh, d, rows, gr.w_f1, 2 * d, part, pc, st, b.a_lo));
+    WCHECK(gemm_acc32(b.dz, b.dz_lo, Fh, true, x, d, true, Fh, d, rows, gr.w_f1 + d, 2 * d, part, pc, st));
+  } else {
+    WCHECK(gemm_acc32(b.df, b.df_lo, d, false, w.w_f2, 2 * d, true, rows, 2 * d, d, F(b.dc), 2 * d, part, pc, st));
+    WCHECK(gemm_acc32(b.df, b.df_lo, d, true, b.a, d, true, d, d, rows, gr.w_f2, 2 * d, part, pc, st, b.a_lo));
+    WCHECK(gemm_acc32(b.df, b.df_lo, d, true, x, d, true, d, d, rows, gr.w_f2 + d, 2 * d, part, pc, st));
+  }
+  // ---- S3 backward: attention (KV-parallel) ----
+  WCHECK(ew_launch(attn_bwd_prep_kernel, rows * s.h, st, (const float*)F(b.dc), (long long)(2 * d),
+                   (const bf*)b.a, (const bf*)b.a_lo, rows, d, s.h, F(b.delta), static_cast<bf*>(b.da16),
+                   static_cast<bf*>(b.da_lo)));
+  CUCHECK(cudaMemsetAsync(b.dq, 0, (size_t)rows * d * 4, st));
+  if (T > 0) {
+    const long long cmax = cdiv<long long>(T, kBwdChunk) + h.B;
+    if (cmax >= (1ll << 31)) return WHALE_ERR_UNSUPPORTED;
+    WCHECK(launch_pdl(chunk_starts_kernel, dim3(1), dim3(1024), 0, st, offsets, h.B, T, kBwdChunk, (int)cmax,
+                      static_cast<int*>(b.cst)));
+    AttnBwdArgs aa{};
+    aa.q = static_cast<const bf*>(b.q);
+    aa.q_lo = static_cast<const bf*>(b.q_lo);
+    aa.kv = static_cast<const bf*>(b.kv);
+    aa.kv_lo = static_cast<const bf*>(b.kv_lo);
+    aa.da = static_cast<const bf*>(b.da16);
+    aa.da_lo = static_cast<const bf*>(b.da_lo);
+    aa.dkv_lo = static_cast<bf*>(b.dkv_lo);
+    aa.lse = F(b.lse);
+    aa.delta = F(b.delta);
+    aa.offsets = offsets;
+    aa.cstart = static_cast<const int*>(b.cst);
+    aa.dq = F(b.dq);
+    aa.dkv = static_cast<bf*>(b.dkv);
+    aa.B = h.B;
+    aa.N = s.N;
+    aa.d = d;
+    aa.n_heads = s.h;
+    aa.kvw = kvw;
+    aa.v_col0 = s.shared_kv ? 0 : d;
+    aa.shared_kv = s.shared_kv ? 1 : 0;
+    aa.total_L = T;
+    aa.scale = (float)(1.0 / std::sqrt((double)s.dh));
+    aa.scale_log2 = scale_log2_of(s);
+    whale_status r;
+    if (s.dh == 64) r = s.N <= 16 ? launch_attn_bwd<64, 16>(aa, (unsigned)cmax, st) : launch_attn_bwd<64, 32>(aa, (unsigned)cmax, st);
+    else r = s.N <= 16 ? launch_attn_bwd<32, 16>(aa, (unsigned)cmax, st) : launch_attn_bwd<32, 32>(aa, (unsigned)cmax, st);
+    WCHECK(r);
+  }
+  // ---- S1 backward: query projection and its RMSNorm; d_tokens ----
+  WCHECK(ew_launch(split_pair_kernel, rows * d, st, (const float*)F(b.dq), (long long)d, static_cast<bf*>(b.dq_hi),
+                   static_cast<bf*>(b.dq_lo), (long long)d, rows, d));
+  WCHECK(gemm_acc32(b.dq_hi, b.dq_lo, d, false, w.w_q, d, true, rows, d, d, F(b.dn), d, part, pc, st));
+  WCHECK(gemm_acc32(b.dq_hi, b.dq_lo, d, true, b.nq, d, true, d, d, rows, gr.w_q, d, part, pc, st, b.nq_lo));
+  WCHECK(rms_bwd<bf>(static_cast<const bf*>(x), w.g_q, F(b.dn), rows, d, s.eps, F(b.df32), d, F(b.dc) + d, 2 * d, dx,
+                     nullptr, nullptr, nullptr, nullptr, nullptr, F(b.colp), gr.g_q, st));
+  // ---- S2 backward: K|V projection and the states' RMSNorm ----
+  if (T > 0) {
+    WCHECK(gemm_acc32(b.dkv, b.dkv_lo, kvw, false, w.w_kv, d, true, T, d, kvw, F(b.dsn), d, part, pc, st));
+    WCHECK(rms_bwd<bf>(static_cast<const bf*>(slab), w.g_kv, F(b.dsn), T, d, s.eps, nullptr, 0, nullptr, 0, nullptr, ds,
+                       nullptr, nullptr, nullptr, nullptr, F(b.colp), gr.g_kv, st));
+    WCHECK(gemm_acc32(b.dkv, b.dkv_lo, kvw, true, b.sn, d, true, kvw, d, T, gr.w_kv, d, part, pc, st, b.sn_lo));
+  } else {
+    CUCHECK(cudaMemsetAsync(gr.g_kv, 0, (size_t)d * 4, st));
+    CUCHECK(cudaMemsetAsync(gr.w_kv, 0, (size_t)kvw * d * 4, st));
+  }
+  return WHALE_OK;
+}
+
+whale_status layer_backward_f32(const Shape& s, const float* x, const float* slab, const int* offsets,
+                                const whale_layer_weights& w, const float* dy, float* dx, float* ds,
+                                const whale_layer_grads& gr, const whale_shape_hint& h, const BwdBufs& b,
+                                cudaStream_t st) {
+  const long long rows = (long long)h.B * s.N, T = h.total_L;
+  const int d = s.d, H = s.H, Fh = s.Fh, ugw = s.ugw, kvw = s.kvw;
+  auto F = [](void* p) { return static_cast<float*>(p); };
+  auto W32 = [](const void* p) { return static_cast<const float*>(p); };
+  // C = A B with A [M, K] and B [K, N] row-major (dX = dY W)
+  auto mm = [&](const float* A, long long lda, const float* B, long long ldb, float* C, long long ldc, long long M,
+                long long N, long long K) { return gemm_strided_f32(A, lda, 1, B, ldb, 1, C, ldc, M, N, K, st); };
+  // C = A^T B with A [K, M] and B [K, N] row-major (dW = dY^T X)
+  auto mtm = [&](const float* A, long long lda, const float* B, long long ldb, float* C, long long ldc, long long M,
+                 long long N, long long K) { return gemm_strided_f32(A, 1, lda, B, ldb, 1, C, ldc, M, N, K, st); };
+  // ---- forward recompute ----
+  WCHECK(row_rms(x, rows, d, s.eps, F(b.r), st));
+  WCHECK(gemm_f32(x, d, nullptr, 0, F(b.r), w.g_q, W32(w.w_q), d, F(b.q), rows, F32_NONE, nullptr, st));
+  WCHECK(row_rms(slab, T, d, s.eps, F(b.r), st));
+  WCHECK(gemm_f32(slab, d, nullptr, 0, F(b.r), w.g_kv, W32(w.w_kv), kvw, F(b.kv), T, F32_NONE, nullptr, st));
+  WCHECK(attention_f32(s, F(b.q), F(b.kv), offsets, F(b.a), h.B, T, st));
+  if (Fh > 0) {
+    WCHECK(gemm_f32(F(b.a), d, x, d, nullptr, nullptr, W32(w.w_f1), Fh, F(b.z1), rows, F32_NONE, nullptr, st));
+    WCHECK(ew_launch(silu_pair_kernel, rows * Fh, st, (const float*)F(b.z1), F(b.g), (__nv_bfloat16*)nullptr,
+                     (__nv_bfloat16*)nullptr, rows * Fh));
+    WCHECK(gemm_f32(F(b.g), Fh, nullptr, 0, nullptr, nullptr, W32(w.w_f2), d, F(b.f32), rows, F32_RESID, x, st));
+  } else {
+    WCHECK(gemm_f32(F(b.a), d, x, d, nullptr, nullptr, W32(w.w_f2), d, F(b.f32), rows, F32_RESID, x, st));
+  }
+  WCHECK(row_rms(F(b.f32), rows, d, s.eps, F(b.r), st));
+  WCHECK(gemm_f32(F(b.f32), d, nullptr, 0, F(b.r), w.g_ffn, W32(w.w_upgate), ugw, F(b.ug), rows, F32_NONE, nullptr,
+                  st));
+  // ---- S5 backward ----
+  WCHECK(mm(dy, d, W32(w.w_down), H, F(b.dm), H, rows, H, d));
+  WCHECK(ew_launch(swiglu_bwd_kernel, rows * H, st, (const float*)F(b.ug), (const float*)F(b.dm), rows, H,
+                   s.tied ? 1 : 0, (__nv_bfloat16*)nullptr, (__nv_bfloat16*)nullptr, F(b.msw), F(b.dug),
+                   (__nv_bfloat16*)nullptr, (__nv_bfloat16*)nullptr));
+  WCHECK(mtm(dy, d, F(b.msw), H, gr.w_down, H, d, H, rows));
+  WCHECK(mm(F(b.dug), ugw, W32(w.w_upgate), d, F(b.dn), d, rows, d, ugw));
+  WCHECK(rms_bwd<float>(F(b.f32), w.g_ffn, F(b.dn), rows, d, s.eps, dy, d, nullptr, 0, F(b.df32), nullptr, nullptr,
+                        nullptr, nullptr, F(b.nrm), F(b.colp), gr.g_ffn, st));
+  WCHECK(mtm(F(b.dug), ugw, F(b.nrm), d, gr.w_upgate, d, ugw, d, rows));
+  // ---- S4 backward ----
+  if (Fh > 0) {
+    WCHECK(mm(F(b.df32), d, W32(w.w_f2), Fh, F(b.dhid), Fh, rows, Fh, d));
+    WCHECK(ew_launch(silu_bwd_kernel, rows * Fh, st, (const float*)F(b.dhid), (const float*)F(b.z1), F(b.dz),
+                     (__nv_bfloat16*)nullptr, (__nv_bfloat16*)nullptr, rows * Fh));
+    WCHECK(mtm(F(b.df32), d, F(b.g), Fh, gr.w_f2, Fh, d, Fh, rows));
+    WCHECK(mm(F(b.dz), Fh, W32(w.w_f1), 2 * d, F(b.dc), 2 * d, rows, 2 * d, Fh));
+    WCHECK(mtm(F(b.dz), Fh, F(b.a), d, gr.w_f1, 2 * d, Fh, d, rows));
+    WCHECK(mtm(F(b.dz), Fh, x, d, gr.w_f1 + d, 2 * d, Fh, d, rows));
+  } else {
+    WCHECK(mm(F(b.df32), d, W32(w.w_f2), 2 * d, F(b.dc), 2 * d, rows, 2 * d, d));
+    WCHECK(mtm(F(b.df32), d, F(b.a), d, gr.w_f2, 2 * d, d, d, rows));
+    WCHECK(mtm(F(b.df32), d, x, d, gr.w_f2 + d, 2 * d, d, d, rows));
+  }
+  // ---- S3 backward ----
+  if (h.B > 0) {
+    const size_t smem = (size_t)s.N * (3 * s.dh + 3) * 4;
+    if (smem > 227 * 1024) return WHALE_ERR_UNSUPPORTED;
+    const dim3 grid((unsigned)h.B, (unsigned)s.h);
+    const float scale = (float)(1.0 / std::sqrt((double)s.dh));
+    const int v0 = s.shared_kv ? 0 : d;
+#define ATTB32(DH)                                                                                                    \
+  do {                                                                                                                \
+    CUCHECK(cudaFuncSetAttribute(attn_bwd_f32_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));   \
+    attn_bwd_f32_kernel<DH><<<grid, 256, smem, st>>>(F(b.q), F(b.kv), kvw, v0, F(b.dc), 2ll * d, offsets, T, s.N, d,   \
+                                                     s.h, scale, F(b.dq), F(b.dkv), s.shared_kv ? 1 : 0);             \
+  } while (0)
+    switch (s.dh) {
+      case 8: ATTB32(8); break;
+      case 16: ATTB32(16); break;
+      case 32: ATTB32(32); break;
+      case 64: ATTB32(64); break;
+      default: return WHALE_ERR_UNSUPPORTED;
+    }
+#undef ATTB32
+    CUCHECK(cudaGetLastError());
+  }
+  // ---- S1 backward ----
+  WCHECK(mm(F(b.dq), d, W32(w.w_q), d, F(b.dn), d, rows, d, d));
+  WCHECK(launch_pdl(rms_rows_kernel<float>, dim3(rows_blocks(rows)), dim3(256), 0, st, x, w.g_q, rows, d, s.eps,
+                    (__nv_bfloat16*)nullptr, (__nv_bfloat16*)nullptr, F(b.nrm)));
+  WCHECK(mtm(F(b.dq), d, F(b.nrm), d, gr.w_q, d, d, d, rows));
+  WCHECK(rms_bwd<float>(x, w.g_q, F(b.dn), rows, d, s.eps, F(b.df32), d, F(b.dc) + d, 2 * d, dx, nullptr, nullptr,
+                        nullptr, nullptr, nullptr, F(b.colp), gr.g_q, st));
+  // ---- S2 backward ----
+  if (T > 0) {
+    WCHECK(mm(F(b.dkv), kvw, W32(w.w_kv), d, F(b.dsn), d, T, d, kvw));
+    WCHECK(rms_bwd<float>(slab, w.g_kv, F(b.dsn), T, d, s.eps, nullptr, 0, nullptr, 0, ds, nullptr, nullptr, nullptr,
+                          nullptr, F(b.sn), F(b.colp), gr.g_kv, st));
+    WCHECK(mtm(F(b.dkv), kvw, F(b.sn), d, gr.w_kv, d, kvw, d, T));
+  } else {
+    CUCHECK(cudaMemsetAsync(gr.g_kv, 0, (size_t)d * 4, st));
+    CUCHECK(cudaMemsetAsync(gr.w_kv, 0, (size_t)kvw * d * 4, st));
+  }
+  return WHALE_OK;
+}
+
+bool grads_ok(const Shape& s, const whale_layer_grads* g) {
+  return g && g->g_q && g->g_kv && g->g_ffn && g->w_q && g->w_kv && g->w_f2 && g->w_upgate && g->w_down &&
+         (s.Fh == 0 || g->w_f1);
+}
+
 }  // namespace
 
 // ============================================================================================
@@ -1564,6 +2080,54 @@ whale_status whale_cross_attention_noalloc(const whale_config* cfg, const void* 
   WCHECK(noalloc_scratch(&scratch));
   WCHECK(debug_check(s, seq_offsets, *hint, st));
   return attention_bf16(s, q, kv, seq_offsets, a, nullptr, hint->B, hint->total_L, scratch, st);
+}
+
+size_t whale_backward_workspace_size(const whale_config* cfg, const whale_shape_hint* hint) {
+  Shape s;
+  if (validate(cfg, &s) != WHALE_OK || check_hint(hint) != WHALE_OK || !backward_shape_ok(s) || s.prepared) return 0;
+  BwdBufs b;
+  return bwd_buffers(s, *hint, nullptr, &b);
+}
+
+whale_status whale_fusion_layer_backward(const whale_config* cfg, const void* tokens_in, const void* layer_states,
+                                         const int* seq_offsets, const whale_layer_weights* w, const float* d_out,
+                                         float* d_tokens, void* d_states, const whale_layer_grads* grads,
+                                         const whale_shape_hint* hint, void* ws, size_t ws_bytes,
+                                         whale_stream_t stream) {
+  Shape s;
+  WCHECK(validate(cfg, &s));
+  WCHECK(check_hint(hint));
+  if (s.prepared) return WHALE_ERR_UNSUPPORTED;
+  if (!backward_shape_ok(s)) return WHALE_ERR_UNSUPPORTED;
+  if (!weights_ok(s, w) || !grads_ok(s, grads)) return WHALE_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  BwdBufs b;
+  const size_t need = bwd_buffers(s, *hint, nullptr, &b);
+  if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1))) return WHALE_ERR_WORKSPACE;
+  if (hint->B == 0) {  // no examples: every gradient is zero
+    const size_t d = s.d;
+    const float* zs[] = {grads->g_q, grads->g_kv, grads->g_ffn};
+    for (const float* z : zs) CUCHECK(cudaMemsetAsync(const_cast<float*>(z), 0, d * 4, st));
+    CUCHECK(cudaMemsetAsync(grads->w_q, 0, d * d * 4, st));
+    CUCHECK(cudaMemsetAsync(grads->w_kv, 0, (size_t)s.kvw * d * 4, st));
+    if (s.Fh > 0) CUCHECK(cudaMemsetAsync(grads->w_f1, 0, (size_t)s.Fh * 2 * d * 4, st));
+    CUCHECK(cudaMemsetAsync(grads->w_f2, 0, d * (size_t)(s.Fh > 0 ? s.Fh : 2 * s.d) * 4, st));
+    CUCHECK(cudaMemsetAsync(grads->w_upgate, 0, (size_t)s.ugw * d * 4, st));
+    CUCHECK(cudaMemsetAsync(grads->w_down, 0, d * (size_t)s.H * 4, st));
+    return WHALE_OK;
+  }
+  if (!tokens_in || !seq_offsets || !d_out || !d_tokens || (hint->total_L > 0 && (!layer_states || !d_states)))
+    return WHALE_ERR_INVALID_ARG;
+  if (!aligned16(tokens_in) || !aligned16(d_out) || !aligned16(d_tokens) ||
+      (layer_states && !aligned16(layer_states)) || (d_states && !aligned16(d_states)))
+    return WHALE_ERR_INVALID_ARG;
+  bwd_buffers(s, *hint, static_cast<char*>(ws), &b);
+  WCHECK(debug_check(s, seq_offsets, *hint, st));
+  if (s.bf16)
+    return layer_backward_bf16(s, tokens_in, layer_states, seq_offsets, *w, d_out, d_tokens, d_states, *grads, *hint, b,
+                               st);
+  return layer_backward_f32(s, static_cast<const float*>(tokens_in), static_cast<const float*>(layer_states),
+                            seq_offsets, *w, d_out, d_tokens, static_cast<float*>(d_states), *grads, *hint, b, st);
 }
 
 whale_status whale_test_bounded_waits(unsigned long long limit_ns, whale_stream_t stream) {

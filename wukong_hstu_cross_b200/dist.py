@@ -1,8 +1,10 @@
 """Rank plumbing for multi-GPU runs (one process per GPU, torch.distributed).
 
 The fusion forward shards with no exchange: examples are independent, so each rank runs the
-whole stack on its own batch (weak scaling) with replicated weights, and nothing crosses ranks
-on the data path. The only collective is the timing reduction (max over ranks).
+whole stack on its own examples with replicated weights, and nothing crosses ranks on the data
+path. Two ways to give ranks their examples: a fresh batch per rank (weak scaling, as the
+benchmark runs), or one batch split into contiguous example ranges balanced by history rows
+(shard_batch). The only collective is the timing reduction (max over ranks).
 """
 from __future__ import annotations
 
@@ -27,6 +29,40 @@ def shard_workload(w: I.Workload, rank: int, world: int) -> I.Workload:
     if world <= 1 or rank == 0:
         return w
     return w.replace(seed=w.seed + 1000 * rank, weight_seed=w.weight_seed if w.weight_seed is not None else w.seed)
+
+
+def balanced_ranges(lengths, world: int) -> list:
+    """Split one batch's examples into `world` contiguous ranges [b0, b1), balanced by history rows.
+
+    The rows each rank streams through the history-side kernels are its sum of L_b, so the cut
+    after rank k's range is put at the example boundary whose prefix sum of lengths lies closest to
+    (k + 1) / world of the total. Ranges are contiguous, so a rank's history rows are one slice of
+    the layer slab and its offsets only shift. A rank may get no examples (more ranks than examples)."""
+    import numpy as np
+    L = np.asarray(lengths, dtype=np.int64)
+    B = len(L)
+    pre = np.concatenate([[0], np.cumsum(L)])
+    total = int(pre[-1])
+    cuts = [0]
+    for k in range(1, world):
+        target = total * k / world
+        b = int(np.searchsorted(pre, target))        # first boundary with prefix >= target
+        if b > 0 and abs(pre[b - 1] - target) <= abs(pre[min(b, B)] - target):
+            b -= 1
+        cuts.append(min(max(b, cuts[-1]), B))
+    cuts.append(B)
+    return [(cuts[k], cuts[k + 1]) for k in range(world)]
+
+
+def shard_batch(tokens, states, offsets, rank: int, world: int):
+    """Rank `rank`'s part of one batch: (tokens [b1-b0, N, d], states [n_layers, rows, d],
+    offsets rebased to start at 0 (int32 [b1-b0+1]), (b0, b1)). Works on numpy arrays and torch
+    tensors alike (slices of the inputs; the offsets are a new array)."""
+    import numpy as np
+    off = np.asarray(offsets.cpu() if hasattr(offsets, "cpu") else offsets, dtype=np.int64)
+    b0, b1 = balanced_ranges(np.diff(off), world)[rank]
+    o0, o1 = int(off[b0]), int(off[b1])
+    return tokens[b0:b1], states[:, o0:o1], (off[b0:b1 + 1] - o0).astype(np.int32), (b0, b1)
 
 
 def max_over_ranks(x: float, world: int, device=None) -> float:

@@ -72,6 +72,7 @@ class Problem:
     workspace: torch.Tensor
     flags: dict
     prepared_buf: torch.Tensor | None = None
+    raw_weights: list | None = None     # the unprepared weights (kept alive once prepared)
 
     @property
     def total_L(self) -> int:
@@ -113,6 +114,8 @@ def prepare_weights(p: Problem) -> None:
     if p.w.dtype != "bf16":
         return
     p.prepared_buf = torch.empty(W.whale_prepared_weights_size(p.cfg), dtype=torch.uint8, device=p.out.device)
+    # the prepared array still points at the raw w_f1, w_f2, w_down and gains: keep them alive
+    p.raw_weights = p.weights
     p.weights = W.whale_prepare_weights(p.cfg, p.weights, p.prepared_buf)
     p.cfg = W.make_config(p.cfg.n_layers, p.cfg.d, p.cfg.n_heads, p.cfg.n_tokens, p.cfg.ffn_hidden,
                           p.cfg.fusion_hidden, p.cfg.dtype, p.cfg.flags | W.WHALE_PREPARED_WEIGHTS, p.cfg.eps)
@@ -127,3 +130,24 @@ def run_forward(p: Problem, stream=None) -> torch.Tensor:
 def states_of_example_host(p: Problem, b: int) -> list:
     """Per-layer H_s rows of example b, regenerated on the host (float32)."""
     return [I.states_of_example(p.w, l, b, int(p.lengths[b])) for l in range(p.w.n_layers)]
+
+
+def run_layer_backward(p: Problem, layer: int, d_out: torch.Tensor, stream=None) -> dict:
+    """Gradients of layer `layer` for the upstream gradient d_out (fp32 [B, N, d]) through
+    whale_fusion_layer_backward, with the layer's raw weights; the layer's input is the problem's
+    tokens. Returns {"d_tokens", "d_states", and one fp32 tensor per parameter}."""
+    w = p.w
+    lw = (p.raw_weights or p.weights)[layer]
+    dev = p.tokens.device
+    grads = {k: torch.empty(tuple(v.shape), dtype=torch.float32, device=dev) for k, v in lw.items()
+             if v is not None and k != "w_kabs"}
+    cfg = config_of(w, flags_of(p.flags.get("shared_kv", False), p.flags.get("tied_gate", False)))
+    nbytes = W.whale_backward_workspace_size(cfg, p.hint)
+    if nbytes == 0:
+        raise ValueError("shape not supported by the backward pass")
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    d_tokens = torch.empty(p.tokens.shape, dtype=torch.float32, device=dev)
+    d_states = torch.empty(p.states.shape[1:], dtype=p.states.dtype, device=dev)
+    W.whale_fusion_layer_backward(cfg, p.tokens, p.states[layer], p.offsets_t, lw, d_out, d_tokens, d_states, grads,
+                                  p.hint, ws, stream=stream)
+    return {"d_tokens": d_tokens, "d_states": d_states, **grads}

@@ -37,6 +37,13 @@ class whale_layer_weights(ctypes.Structure):
     _fields_ = [(n, c_void_p) for n in _WNAMES]
 
 
+_GNAMES = ("g_q", "g_kv", "w_q", "w_kv", "w_f1", "w_f2", "g_ffn", "w_upgate", "w_down")
+
+
+class whale_layer_grads(ctypes.Structure):
+    _fields_ = [(n, c_void_p) for n in _GNAMES]
+
+
 class whale_shape_hint(ctypes.Structure):
     _fields_ = [("B", c_int), ("max_L", c_int), ("total_L", c_longlong)]
 
@@ -82,6 +89,9 @@ _SIGS = {
                                POINTER(whale_layer_weights), _P], c_int),
     "whale_cross_attention_noalloc": ([POINTER(whale_config), _P, _P, _P, _P, POINTER(whale_shape_hint), _P], c_int),
     "whale_test_bounded_waits": ([ctypes.c_ulonglong, _P], c_int),
+    "whale_backward_workspace_size": ([POINTER(whale_config), POINTER(whale_shape_hint)], c_size_t),
+    "whale_fusion_layer_backward": ([POINTER(whale_config), _P, _P, _P, POINTER(whale_layer_weights), _P, _P, _P,
+                                     POINTER(whale_layer_grads), POINTER(whale_shape_hint), _P, c_size_t, _P], c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -171,7 +181,9 @@ def whale_prepared_weights_size(cfg: whale_config) -> int:
 
 def whale_prepare_weights(cfg, weights, prepared, prepared_bytes=None, stream=None, raw=False):
     """Fold gains / pack up|gate once; returns the ctypes array of prepared layer weights (use it
-    with cfg.flags | WHALE_PREPARED_WEIGHTS). Keep `prepared` alive while it is used."""
+    with cfg.flags | WHALE_PREPARED_WEIGHTS). The array points into `prepared` and, for the matrices
+    that are not re-packed (w_f1, w_f2, w_down, the gains), into the caller's original tensors: it
+    keeps references to both, so neither is freed while the array is alive."""
     w = weights if isinstance(weights, ctypes.Array) else weights_array(weights)
     out = (whale_layer_weights * len(w))()
     st = _lib.whale_prepare_weights(ctypes.byref(cfg), w, _ptr(prepared), _ws_bytes(prepared, prepared_bytes), out,
@@ -179,6 +191,7 @@ def whale_prepare_weights(cfg, weights, prepared, prepared_bytes=None, stream=No
     if raw:
         return st
     _check(st, "whale_prepare_weights")
+    out._keepalive = (weights, w, prepared)
     return out
 
 
@@ -289,6 +302,31 @@ def whale_profile_end(capacity: int = 4096) -> list:
     n = c_int(0)
     _check(_lib.whale_profile_end(buf, capacity, ctypes.byref(n)), "whale_profile_end")
     return [((buf[i].kernel or b"?").decode(), float(buf[i].ms)) for i in range(min(n.value, capacity))]
+
+
+def whale_backward_workspace_size(cfg: whale_config, hint: whale_shape_hint) -> int:
+    return int(_lib.whale_backward_workspace_size(ctypes.byref(cfg), ctypes.byref(hint)))
+
+
+def layer_grads(g) -> whale_layer_grads:
+    """A whale_layer_grads from a dict of fp32 tensors (w_f1 may be absent or None)."""
+    if isinstance(g, whale_layer_grads):
+        return g
+    return whale_layer_grads(*[_ptr(g.get(n)) for n in _GNAMES])
+
+
+def whale_fusion_layer_backward(cfg, tokens_in, layer_states, seq_offsets, layer_weights_, d_out, d_tokens, d_states,
+                                grads, hint, workspace, workspace_bytes=None, stream=None, raw=False):
+    """Gradients of one fusion layer (see include/whale_fusion.h); `grads` is a dict of fp32 tensors."""
+    lw = layer_weights(layer_weights_)
+    gr = layer_grads(grads)
+    st = _lib.whale_fusion_layer_backward(ctypes.byref(cfg), _ptr(tokens_in), _ptr(layer_states), _ptr(seq_offsets),
+                                          ctypes.byref(lw), _ptr(d_out), _ptr(d_tokens), _ptr(d_states),
+                                          ctypes.byref(gr), ctypes.byref(hint), _ptr(workspace),
+                                          _ws_bytes(workspace, workspace_bytes), _stream(stream))
+    if raw:
+        return st
+    _check(st, "whale_fusion_layer_backward")
 
 
 def whale_test_bounded_waits(limit_ns: int, stream=None, raw=False):
