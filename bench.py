@@ -204,11 +204,11 @@ class ClockSampler:
 # ------------------------------------------------------------------------------------------------
 class OracleSampler:
     """The fp64 oracle timed on whole examples of the workload, walking the batch in order (and
-    round again): lengths and weights are drawn once; each example's inputs are generated outside
-    the timed region, the next example's in a background thread while the current one runs."""
+    round again): lengths and weights are drawn once; each example's inputs are generated before
+    its timed region (not concurrently: a generator thread beside the oracle's BLAS threads
+    oversubscribes the cores and slows the oracle down)."""
 
     def __init__(self, w: I.Workload):
-        from concurrent.futures import ThreadPoolExecutor
         self.w = w
         self.L = I.draw_lengths(w)
         self.lws = I.make_all_weights(w)
@@ -217,8 +217,6 @@ class OracleSampler:
         self.next_b = 0
         self.done, self.toks, self.t = 0, 0, 0.0
         self.step_s = []
-        self.pool = ThreadPoolExecutor(1)
-        self.pending = self.pool.submit(self._inputs, 0)
 
     def _inputs(self, b: int):
         w = self.w
@@ -233,9 +231,8 @@ class OracleSampler:
         w = self.w
         t_run, n = 0.0, 0
         while True:
-            x, slabs = self.pending.result()
+            x, slabs = self._inputs(self.next_b)
             self.next_b = (self.next_b + 1) % w.batch
-            self.pending = self.pool.submit(self._inputs, self.next_b)
             t0 = time.perf_counter()
             O.fusion_stack_example(x, slabs, self.lws, w.n_heads, w.eps)
             dt = time.perf_counter() - t0
@@ -456,7 +453,8 @@ def time_backward(p, raw_weights, w, total_L, peaks, clocks, stream, reps=10):
     kernels = {n: {"launches": c, "avg_ms": t / c, "share": t / tot}
                for n, (c, t) in sorted(kern.items(), key=lambda x: -x[1][1])}
     out = {"entry_point": "whale_fusion_layer_backward (one layer, forward recomputed inside)", "ms_per_layer": ms,
-           "reps": reps, "kernels": kernels}
+           "reps": reps, "kernels": kernels,
+           "launch_order": [[kernel_name(n), round(t, 4)] for n, t in recs]}
     ab = next((v for k, v in kernels.items() if k.split("<")[0] == "attn_bwd_kernel"), None)
     if ab:
         kvw = w.d if p.flags.get("shared_kv") else 2 * w.d

@@ -301,12 +301,33 @@ typedef struct {
   float* w_upgate; /* [2H, d] ([H, d] with WHALE_TIED_GATE) */
   float* w_down;   /* [d, H] */
 } whale_layer_grads;
+/* Workspace of whale_fusion_backward for cfg->n_layers layers (also enough for
+ * whale_fusion_layer_backward; 0 for unsupported shapes). */
 size_t whale_backward_workspace_size(const whale_config* cfg, const whale_shape_hint* hint);
 whale_status whale_fusion_layer_backward(const whale_config* cfg, const void* tokens_in, const void* layer_states,
                                          const int* seq_offsets, const whale_layer_weights* w, const float* d_out,
                                          float* d_tokens, void* d_states, const whale_layer_grads* grads,
                                          const whale_shape_hint* hint, void* workspace, size_t workspace_bytes,
                                          whale_stream_t stream);
+
+/* The whole stack's backward: the forward is run once more, keeping every layer's input (the
+ * residual stream between layers in fp32 and its hi/lo pair, as the forward carries it), then each
+ * layer's backward, last layer first, each layer's d_tokens being the upstream gradient of the layer
+ * below (the Wukong module between layers is the identity, as in the forward).
+ *   wukong_tokens  device [B, N, d]               H_w of layer 0 (cfg->dtype)
+ *   seq_states     device [n_layers, total_L, d]  H_s slab of each layer
+ *   weights        HOST array of n_layers raw whale_layer_weights
+ *   d_out          device fp32 [B, N, d]          dLoss/d(last layer's H_f)
+ *   d_tokens       device fp32 [B, N, d]          dLoss/d(layer 0's H_w) (written)
+ *   d_states       device [n_layers, total_L, d]  dLoss/dH_s of each layer, cfg->dtype (written)
+ *   grads          HOST array of n_layers whale_layer_grads (device fp32 pointers, overwritten)
+ *   workspace      device, >= whale_backward_workspace_size bytes, 256-byte aligned
+ * Supported shapes as for whale_fusion_layer_backward, n_layers <= 64. */
+whale_status whale_fusion_backward(const whale_config* cfg, const void* wukong_tokens, const void* seq_states,
+                                   const int* seq_offsets, const whale_layer_weights* weights, const float* d_out,
+                                   float* d_tokens, void* d_states, const whale_layer_grads* grads,
+                                   const whale_shape_hint* hint, void* workspace, size_t workspace_bytes,
+                                   whale_stream_t stream);
 
 /* Failure detection. Every device-side wait of the library's kernels (a pipeline stage on an
  * mbarrier, one CTA pair waiting for another's published results) gives up after a time limit

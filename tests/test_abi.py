@@ -16,7 +16,7 @@ EXPECTED = {
     "whale_cross_attention", "whale_fusion_mlp", "whale_swiglu_ffn", "whale_get_device_error",
     "whale_attend_states", "whale_prepare_weights", "whale_prepared_weights_size", "whale_cross_attention_noalloc",
     "whale_profile_begin", "whale_profile_end", "whale_test_bounded_waits", "whale_backward_workspace_size",
-    "whale_fusion_layer_backward",
+    "whale_fusion_layer_backward", "whale_fusion_backward",
 }
 
 
@@ -53,9 +53,11 @@ def test_backward_host_side_errors():
     lw = dict.fromkeys(["g_q", "g_kv", "w_q", "w_kv", "w_f1", "w_f2", "g_ffn", "w_upgate", "w_down"], fake)
     gr = dict(lw)
     nbytes = W.whale_backward_workspace_size(cfg, hint)
-    # workspace too small
-    assert W.whale_fusion_layer_backward(cfg, fake, fake, fake, lw, fake, fake, fake, gr, hint, fake, nbytes - 1,
+    # workspace too small (for one layer, and for the stack)
+    assert W.whale_fusion_layer_backward(cfg, fake, fake, fake, lw, fake, fake, fake, gr, hint, fake, 1024,
                                          stream=0, raw=True) == 4
+    assert W.whale_fusion_backward(cfg, fake, fake, fake, [lw] * cfg.n_layers, fake, fake, fake, [gr] * cfg.n_layers,
+                                   hint, fake, nbytes - 1, stream=0, raw=True) == 4
     # a missing gradient buffer
     bad = dict(gr, w_down=None)
     assert W.whale_fusion_layer_backward(cfg, fake, fake, fake, lw, fake, fake, fake, bad, hint, fake, nbytes,

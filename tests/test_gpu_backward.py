@@ -119,3 +119,36 @@ def test_layer_backward_is_repeatable():
     for k in ("d_tokens", "w_q", "g_q"):
         x, y = a[k].float(), b[k].float()
         assert bool(((x - y).abs() <= 1e-4 * (1 + y.abs())).all()), k
+
+
+STACK_CASES = {
+    "tiny_fp32_2layers": ("tiny_fp32", dict(batch=3, n_layers=2), {}),
+    "d128_3layers": ("stack_d128", dict(batch=4, n_layers=3, lengths=("uniform", 1, 600)), {}),
+    "d512_2layers": ("hist15k_d512", dict(batch=3, n_layers=2, lengths=("lognormal", 1500.0, 0.5, 64, 3000)), {}),
+}
+
+
+@pytest.mark.parametrize("case", list(STACK_CASES))
+def test_stack_backward_matches_oracle(case):
+    """The whole stack's backward (whale_fusion_backward) against the oracle's stack VJP: every
+    layer's state and weight gradients and the tokens' gradient through all layers."""
+    from oracle import whale_oracle as O  # noqa: F401  (the stack VJP below re-runs its forward)
+    base, over, flags = STACK_CASES[case]
+    w = I.WORKLOADS[base].replace(**over)
+    L = I.draw_lengths(w)
+    if case == "d128_3layers":
+        L[1] = 0
+    p = Hn.build_problem(w, gains="random", lengths=L, **flags)
+    dy = np.random.default_rng(11).standard_normal((w.batch, w.n_tokens, w.d)).astype(np.float32)
+    out = Hn.run_stack_backward(p, torch.from_numpy(dy).cuda())
+    torch.cuda.synchronize()
+    assert W.whale_get_device_error() == 0
+    tokens = I.make_tokens(w)
+    states = np.stack([I.make_states_layer(w, l, L, threads=4) for l in range(w.n_layers)])
+    d_tok, d_st, d_w = OB.fusion_stack_backward(tokens, states, p.offsets, p.host_weights, w.n_heads, w.eps, dy,
+                                                **flags)
+    _check("d_tokens", to_np(out["d_tokens"]), d_tok, w.dtype)
+    for l in range(w.n_layers):
+        _check(f"d_states[{l}]", to_np(out["d_states"][l, :p.total_L]), d_st[l], w.dtype)
+        for k, v in d_w[l].items():
+            _check(f"{k}[{l}]", to_np(out["grads"][l][k]), v, w.dtype)

@@ -14,6 +14,7 @@
 //            (tied gate, up = gate = u: du = dup + dgate)
 #pragma once
 
+#include "gemm_tc.cuh"
 #include "ptx.cuh"
 
 namespace whale {
@@ -119,13 +120,40 @@ __global__ void swiglu_bwd_kernel(const float* __restrict__ ug, const float* __r
   }
 }
 
-// RMSNorm backward, one warp per row (d a multiple of 32, at most 1024), for n = r x g:
+// 8 consecutive values of a row as fp32 (16-byte loads: one of bf16, two of fp32).
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
+  bf16x8_to_f32(*reinterpret_cast<const uint4*>(p), v);
+}
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+  const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void store8(float* p, const float (&v)[8]) {
+  reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+  reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+// bf16 of 8 values (hi) and, if lo is set, the bf16 of their rounding residues
+__device__ __forceinline__ void store8_pair(__nv_bfloat16* hi, __nv_bfloat16* lo, const float (&v)[8]) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const __nv_bfloat162 hh = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+    h[j] = *reinterpret_cast<const uint32_t*>(&hh);
+    const float2 hf = __bfloat1622float2(hh);
+    l[j] = pack_bf16x2(v[2 * j] - hf.x, v[2 * j + 1] - hf.y);
+  }
+  *reinterpret_cast<uint4*>(hi) = make_uint4(h[0], h[1], h[2], h[3]);
+  if (lo) *reinterpret_cast<uint4*>(lo) = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// RMSNorm backward, one warp per row (d a multiple of 8, at most 1024; lane l takes the 8-column
+// chunks l, l + 32, ...: 16-byte loads and stores), for n = r x g:
 //   dx = r (dn g) - x (r^3 / d) sum_c (dn g x)_c  [+ resid1 + resid2]
 // x: bf16 or fp32 [rows, d] (row stride d); dn fp32 [rows, d]; outputs (each may be null): dx as fp32,
-// as bf16 (dx_hi, with its residue dx_lo), n = r x g as a bf16 pair (n_out, n_lo) or fp32 (n32). colp [gridDim.x, d]: this
-// block's column sums of dn x r (the gain's gradient, summed over the block's rows; a second pass
-// sums the blocks in order).
-template <typename TX>
+// as bf16 (dx_hi, with its residue dx_lo), n = r x g as a bf16 pair (n_out, n_lo) or fp32 (n32).
+// colp [gridDim.x, d]: this block's column sums of dn x r (the gain's gradient, summed over the
+// block's rows; a second pass sums the blocks in order).
+template <typename TX, int MAXCH>
 __global__ void __launch_bounds__(256) rms_bwd_kernel(const TX* __restrict__ x, const float* __restrict__ g,
                                                       const float* __restrict__ dn, long long rows, int d, float eps,
                                                       const float* __restrict__ resid1, long long ld1,
@@ -135,71 +163,87 @@ __global__ void __launch_bounds__(256) rms_bwd_kernel(const TX* __restrict__ x, 
                                                       __nv_bfloat16* __restrict__ n_out,
                                                       __nv_bfloat16* __restrict__ n_lo, float* __restrict__ n32,
                                                       float* __restrict__ colp) {
-  constexpr int MAXC = 32;  // columns per lane (d <= 1024)
-  __shared__ float red[8][1024];
+  // MAXCH: 8-column chunks per lane (d <= 256 MAXCH); fewer registers for narrower rows, more blocks per SM
+  __shared__ float red[8][256 * MAXCH];
   pdl_wait();
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nc = d >> 5;
-  float cg[MAXC];
+  const int nch = d >> 3;
+  float cg[MAXCH][8];
 #pragma unroll
-  for (int i = 0; i < MAXC; ++i) cg[i] = 0.f;
+  for (int i = 0; i < MAXCH; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) cg[i][j] = 0.f;
   const long long per = (rows + gridDim.x - 1) / gridDim.x;
   const long long r0 = (long long)blockIdx.x * per, r1 = min(rows, r0 + per);
   for (long long r = r0 + warp; r < r1; r += 8) {
-    float xv[MAXC], u[MAXC];
+    float xv[MAXCH][8], u[MAXCH][8];
     float ss = 0.f, sux = 0.f;
 #pragma unroll
-    for (int i = 0; i < MAXC; ++i) {
-      if (i < nc) {
-        const int c = lane + 32 * i;
-        xv[i] = (float)x[r * d + c];
-        ss = fmaf(xv[i], xv[i], ss);
+    for (int i = 0; i < MAXCH; ++i) {
+      const int c8 = lane + 32 * i;
+      if (c8 < nch) {
+        load8(x + r * d + 8 * c8, xv[i]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) ss = fmaf(xv[i][j], xv[i][j], ss);
       }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     const float rr = rsqrtf(ss / (float)d + eps);
 #pragma unroll
-    for (int i = 0; i < MAXC; ++i) {
-      if (i < nc) {
-        const int c = lane + 32 * i;
-        const float dv = dn[r * d + c];
-        u[i] = dv * g[c];
-        sux = fmaf(u[i], xv[i], sux);
-        cg[i] = fmaf(dv, xv[i] * rr, cg[i]);
+    for (int i = 0; i < MAXCH; ++i) {
+      const int c8 = lane + 32 * i;
+      if (c8 < nch) {
+        float dv[8], gv[8];
+        load8(dn + r * d + 8 * c8, dv);
+        load8(g + 8 * c8, gv);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          u[i][j] = dv[j] * gv[j];
+          sux = fmaf(u[i][j], xv[i][j], sux);
+          cg[i][j] = fmaf(dv[j], xv[i][j] * rr, cg[i][j]);
+        }
       }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sux += __shfl_xor_sync(0xffffffffu, sux, o);
     const float k = rr * rr * rr / (float)d * sux;
 #pragma unroll
-    for (int i = 0; i < MAXC; ++i) {
-      if (i < nc) {
-        const int c = lane + 32 * i;
-        float v = rr * u[i] - xv[i] * k;
-        if (resid1) v += resid1[r * ld1 + c];
-        if (resid2) v += resid2[r * ld2 + c];
-        if (dx32) dx32[r * d + c] = v;
-        if (dx_hi) {
-          const __nv_bfloat16 h = __float2bfloat16_rn(v);
-          dx_hi[r * d + c] = h;
-          if (dx_lo) dx_lo[r * d + c] = __float2bfloat16_rn(v - __bfloat162float(h));
+    for (int i = 0; i < MAXCH; ++i) {
+      const int c8 = lane + 32 * i;
+      if (c8 < nch) {
+        const int c = 8 * c8;
+        float v[8], r1v[8], r2v[8];
+        if (resid1) load8(resid1 + r * ld1 + c, r1v);
+        if (resid2) load8(resid2 + r * ld2 + c, r2v);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          v[j] = rr * u[i][j] - xv[i][j] * k;
+          if (resid1) v[j] += r1v[j];
+          if (resid2) v[j] += r2v[j];
         }
-        const float nv = xv[i] * rr * g[c];
-        if (n_out) {
-          const __nv_bfloat16 nh = __float2bfloat16_rn(nv);
-          n_out[r * d + c] = nh;
-          if (n_lo) n_lo[r * d + c] = __float2bfloat16_rn(nv - __bfloat162float(nh));
+        if (dx32) store8(dx32 + r * d + c, v);
+        if (dx_hi) store8_pair(dx_hi + r * d + c, dx_lo ? dx_lo + r * d + c : nullptr, v);
+        if (n_out || n32) {
+          float gv[8], nv[8];
+          load8(g + c, gv);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) nv[j] = xv[i][j] * rr * gv[j];
+          if (n_out) store8_pair(n_out + r * d + c, n_lo ? n_lo + r * d + c : nullptr, nv);
+          if (n32) store8(n32 + r * d + c, nv);
         }
-        if (n32) n32[r * d + c] = nv;
       }
     }
   }
   if (colp) {
 #pragma unroll
-    for (int i = 0; i < MAXC; ++i)
-      if (i < nc) red[warp][lane + 32 * i] = cg[i];
+    for (int i = 0; i < MAXCH; ++i) {
+      const int c8 = lane + 32 * i;
+      if (c8 < nch)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) red[warp][8 * c8 + j] = cg[i][j];
+    }
     __syncthreads();
     for (int c = threadIdx.x; c < d; c += blockDim.x) {
       float sum = 0.f;
@@ -211,34 +255,88 @@ __global__ void __launch_bounds__(256) rms_bwd_kernel(const TX* __restrict__ x, 
 }
 
 // n = r x g as a bf16 pair (n_out, n_lo) and/or fp32 (n32): the normalised rows the weight gradients
-// contract with, one warp per row.
+// contract with, one warp per row (8-column chunks per lane, as above).
 template <typename TX>
 __global__ void __launch_bounds__(256) rms_rows_kernel(const TX* __restrict__ x, const float* __restrict__ g,
                                                        long long rows, int d, float eps,
                                                        __nv_bfloat16* __restrict__ n_out,
                                                        __nv_bfloat16* __restrict__ n_lo, float* __restrict__ n32) {
+  constexpr int MAXCH = 4;  // 8-column chunks per lane (d <= 1024)
   pdl_wait();
   pdl_trigger();
   const int lane = threadIdx.x & 31;
+  const int nch = d >> 3;
   const long long warps = (long long)gridDim.x * 8;
   for (long long r = (long long)blockIdx.x * 8 + (threadIdx.x >> 5); r < rows; r += warps) {
+    float xv[MAXCH][8];
     float ss = 0.f;
-    for (int c = lane; c < d; c += 32) {
-      const float v = (float)x[r * d + c];
-      ss = fmaf(v, v, ss);
+#pragma unroll
+    for (int i = 0; i < MAXCH; ++i) {
+      const int c8 = lane + 32 * i;
+      if (c8 < nch) {
+        load8(x + r * d + 8 * c8, xv[i]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) ss = fmaf(xv[i][j], xv[i][j], ss);
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     const float rr = rsqrtf(ss / (float)d + eps);
-    for (int c = lane; c < d; c += 32) {
-      const float v = (float)x[r * d + c] * rr * g[c];
-      if (n_out) {
-        const __nv_bfloat16 nh = __float2bfloat16_rn(v);
-        n_out[r * d + c] = nh;
-        if (n_lo) n_lo[r * d + c] = __float2bfloat16_rn(v - __bfloat162float(nh));
+#pragma unroll
+    for (int i = 0; i < MAXCH; ++i) {
+      const int c8 = lane + 32 * i;
+      if (c8 < nch) {
+        const int c = 8 * c8;
+        float gv[8], nv[8];
+        load8(g + c, gv);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) nv[j] = xv[i][j] * rr * gv[j];
+        if (n_out) store8_pair(n_out + r * d + c, n_lo ? n_lo + r * d + c : nullptr, nv);
+        if (n32) store8(n32 + r * d + c, nv);
       }
-      if (n32) n32[r * d + c] = v;
     }
+  }
+}
+
+// out[c] = sum_b part[b * n + c] over b = 0..nb-1, for n columns: a block per 32 columns, its eight
+// warps summing row stripes b = w, w + 8, ... and then combined in warp order (deterministic).
+__global__ void __launch_bounds__(256) col_sums_kernel(const float* __restrict__ part, int nb, int n,
+                                                       float* __restrict__ out) {
+  __shared__ float red[8][32];
+  pdl_wait();
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.x * 32 + lane;
+  float s = 0.f;
+  if (c < n)
+    for (int b = warp; b < nb; b += 8) s += part[(long long)b * n + c];
+  red[warp][lane] = s;
+  __syncthreads();
+  if (warp == 0 && c < n) {
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) t += red[w][lane];
+    out[c] = t;
+  }
+}
+
+// SwiGLU forward: m = SiLU(gate) * up from the pre-activations ug fp32 [rows, ugw] ([up | gate], or u
+// alone with a tied gate), as a bf16 pair [rows, H].
+__global__ void swiglu_pair_kernel(const float* __restrict__ ug, long long rows, int H, int tied,
+                                   __nv_bfloat16* __restrict__ m_hi, __nv_bfloat16* __restrict__ m_lo) {
+  pdl_wait();
+  pdl_trigger();
+  const int ugw = tied ? H : 2 * H;
+  const long long n = rows * H;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const long long r = i / H;
+    const int c = (int)(i - r * H);
+    const float up = ug[r * ugw + c];
+    const float gate = tied ? up : ug[r * ugw + H + c];
+    const float v = gate * sigmoid_f(gate) * up;
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    m_hi[i] = h;
+    m_lo[i] = __float2bfloat16_rn(v - __bfloat162float(h));
   }
 }
 

@@ -554,25 +554,36 @@ whale_status gemm_acc32(const void* a_hi, const void* a_lo, long long lda, bool 
   if (split_b && !split) return WHALE_ERR_UNSUPPORTED;
   const long long tm = cdiv<long long>(M, 128);
   const long long KB = cdiv<long long>(K, 64);
-  // tile width: the cost model of gemm_bf16 (per persistent CTA: tiles x K blocks x max(MMA, bytes))
-  auto cost = [&](int bn) -> double {
+  // Tile width and split-K together, by a cost model (cycles): waves of CTAs x K blocks per CTA x
+  // max(MMA time, operand bytes at ~80 B/clk per SM). When the output has fewer tiles than SMs and K
+  // is long, ks K ranges per tile (fp32 partials within part_cap, at least 8 K blocks each) fill the
+  // SMs in one wave; wider tiles then re-read the operands fewer times.
+  const double mma_per_col = split ? (split_b ? 6.0 : 4.0) : 2.0;
+  auto plan = [&](int bn, int* ks_out) -> double {
     if (N % bn) return 1e300;
-    const double per_cta = (double)cdiv<long long>(tm * (N / bn), kNumSM);
-    const double mma = (split ? (split_b ? 6.0 : 4.0) : 2.0) * bn;
+    const long long tiles = tm * (N / bn);
+    int k = 1;
+    if (tiles < kNumSM && KB >= 16 && part) {
+      long long want = std::min<long long>(std::max<long long>(1, kNumSM / tiles), KB / 8);
+      while (want > 1 && (size_t)want * M * N > part_cap) --want;
+      k = (int)std::max<long long>(1, std::min<long long>(want, 64));
+    }
+    *ks_out = k;
+    const double waves = (double)cdiv<long long>(tiles * k, kNumSM);
     const double bytes = (split ? 32768.0 : 16384.0) + bn * 128.0 * (split_b ? 2 : 1);
-    return 5600.0 + per_cta * KB * std::max(mma, bytes / 80.0);
+    return 5600.0 + waves * (double)cdiv<long long>(KB, k) * std::max(mma_per_col * bn, bytes / 80.0);
   };
-  int bn = 64;
-  for (int cand : {128, 256})
-    if (cost(cand) < cost(bn) && (!split_b || cand <= 128)) bn = cand;  // pairs on both: stages of 64 KB at most
-  const long long tiles_mn = tm * (N / bn);
-  // split-K: enough tiles to fill the SMs once, at least 8 K blocks per split, partials within part_cap
-  int ks = 1;
-  if (tiles_mn < kNumSM && KB >= 16 && part) {
-    long long want = std::min<long long>(cdiv<long long>(kNumSM, tiles_mn), KB / 8);
-    while (want > 1 && (size_t)want * M * N > part_cap) --want;
-    ks = (int)std::max<long long>(1, std::min<long long>(want, 64));
+  int bn = 64, ks = 1, ks_c = 1;
+  double best = plan(64, &ks);
+  for (int cand : {128, 256}) {
+    const double cost = plan(cand, &ks_c);
+    if (cost < best) {
+      best = cost;
+      bn = cand;
+      ks = ks_c;
+    }
   }
+  const long long tiles_mn = tm * (N / bn);
   int kb_split = (int)cdiv<long long>(KB, ks);
   ks = (int)cdiv<long long>(KB, kb_split);  // no empty split
   CUtensorMap maps[5];
@@ -1364,8 +1375,7 @@ size_t bwd_buffers(const Shape& s, const whale_shape_hint& h, char* base, BwdBuf
 // Gain gradient: the row kernel's column partials summed in block order.
 whale_status gain_grad(const float* colp, int blocks, int d, float* dg, cudaStream_t st) {
   if (!dg) return WHALE_OK;
-  return launch_pdl(sum_partials_kernel, dim3((unsigned)cdiv(d, 256)), dim3(256), 0, st, colp, blocks, 1ll, d, dg,
-                    (long long)d);
+  return launch_pdl(col_sums_kernel, dim3((unsigned)cdiv(d, 32)), dim3(256), 0, st, colp, blocks, d, dg);
 }
 
 template <typename TX>
@@ -1377,9 +1387,14 @@ whale_status rms_bwd(const TX* x, const float* g, const float* dn, long long row
     return WHALE_OK;
   }
   const int blocks = rows_blocks(rows);
-  WCHECK(launch_pdl(rms_bwd_kernel<TX>, dim3(blocks), dim3(256), 0, st, x, g, dn, rows, d, eps, r1, ld1, r2, ld2, dx32,
-                    static_cast<__nv_bfloat16*>(dx_hi), static_cast<__nv_bfloat16*>(dx_lo),
-                    static_cast<__nv_bfloat16*>(n_out), static_cast<__nv_bfloat16*>(n_lo), n32, colp));
+  auto go = [&](auto kern) {
+    return launch_pdl(kern, dim3(blocks), dim3(256), 0, st, x, g, dn, rows, d, eps, r1, ld1, r2, ld2, dx32,
+                      static_cast<__nv_bfloat16*>(dx_hi), static_cast<__nv_bfloat16*>(dx_lo),
+                      static_cast<__nv_bfloat16*>(n_out), static_cast<__nv_bfloat16*>(n_lo), n32, colp);
+  };
+  if (d <= 256) WCHECK(go(rms_bwd_kernel<TX, 1>));
+  else if (d <= 512) WCHECK(go(rms_bwd_kernel<TX, 2>));
+  else WCHECK(go(rms_bwd_kernel<TX, 4>));
   return gain_grad(colp, blocks, d, dg, st);
 }
 
@@ -1407,22 +1422,24 @@ bool backward_shape_ok(const Shape& s) {
   return s.dh == 8 || s.dh == 16 || s.dh == 32 || s.dh == 64;
 }
 
-whale_status layer_backward_bf16(const Shape& s, const void* x, const void* slab, const int* offsets,
-                                 const whale_layer_weights& w, const float* dy, float* dx, void* ds,
-                                 const whale_layer_grads& gr, const whale_shape_hint& h, const BwdBufs& b,
-                                 cudaStream_t st) {
+// The forward of one layer in bf16 mode as the backward pass recomputes it, into the backward buffers
+// (q, K|V, A and its log-sum-exp, z1, G, F, UG). The layer input is a residual-stream tensor `in`:
+// fp32 plus its bf16 hi/lo pair (a layer of the stack gets its exact input, the layer entry point its
+// bf16 tokens with lo = 0).
+whale_status recompute_bf16(const Shape& s, const Stream3& in, const void* slab, const int* offsets,
+                            const whale_layer_weights& w, const whale_shape_hint& h, const BwdBufs& b,
+                            cudaStream_t st) {
   using bf = __nv_bfloat16;
   const long long rows = (long long)h.B * s.N, T = h.total_L;
-  const int d = s.d, H = s.H, Fh = s.Fh, ugw = s.ugw, kvw = s.kvw;
+  const int d = s.d, Fh = s.Fh, ugw = s.ugw, kvw = s.kvw;
   auto F = [](void* p) { return static_cast<float*>(p); };
-  // ---- forward recompute ----
-  WCHECK(pair_from_bf16(x, F(b.x32), b.xlo, rows * d, st));
-  const Opnd X = opnd(x, b.xlo, d, d);
+  const float* x32 = in.f32;
+  const Opnd X = opnd(in.hi, in.lo, d, d);
   // Token side: the normalised rows n = r x g as a hi/lo pair times the raw (exact) weights; folding g
   // into a bf16 weight would round every product's weight by up to 2^-9, an error the weight
   // gradients (sums over rows) would carry.
-  WCHECK(launch_pdl(rms_rows_kernel<bf>, dim3(rows_blocks(rows)), dim3(256), 0, st, static_cast<const bf*>(x), w.g_q,
-                    rows, d, s.eps, static_cast<bf*>(b.nq), static_cast<bf*>(b.nq_lo), (float*)nullptr));
+  WCHECK(launch_pdl(rms_rows_kernel<float>, dim3(rows_blocks(rows)), dim3(256), 0, st, x32, w.g_q, rows, d, s.eps,
+                    static_cast<bf*>(b.nq), static_cast<bf*>(b.nq_lo), (float*)nullptr));
   WCHECK(gemm_bf16(opnd(b.nq, b.nq_lo, d, d), no_opnd(), w.w_q, d, Outs{b.q, b.q_lo, nullptr, d}, nullptr, 0, rows,
                    EPI_STORE, false, 0.f, st));
   // History side the same way: K|V = (r s g) W_kv^T from the normalised states as a pair, written as a
@@ -1440,15 +1457,41 @@ whale_status layer_backward_bf16(const Shape& s, const void* x, const void* slab
                      st));
     WCHECK(ew_launch(silu_pair_kernel, rows * Fh, st, (const float*)F(b.z1), (float*)nullptr, static_cast<bf*>(b.g),
                      static_cast<bf*>(b.g_lo), rows * Fh));
-    WCHECK(gemm_bf16(opnd(b.g, b.g_lo, Fh, Fh), no_opnd(), w.w_f2, d, Outs{b.f, b.f_lo, F(b.f32), d}, F(b.x32), d,
+    WCHECK(gemm_bf16(opnd(b.g, b.g_lo, Fh, Fh), no_opnd(), w.w_f2, d, Outs{b.f, b.f_lo, F(b.f32), d}, x32, d,
                      rows, EPI_RESID, false, 0.f, st));
   } else {
-    WCHECK(gemm_bf16(A, X, w.w_f2, d, Outs{b.f, b.f_lo, F(b.f32), d}, F(b.x32), d, rows, EPI_RESID, false, 0.f, st));
+    WCHECK(gemm_bf16(A, X, w.w_f2, d, Outs{b.f, b.f_lo, F(b.f32), d}, x32, d, rows, EPI_RESID, false, 0.f, st));
   }
   WCHECK(launch_pdl(rms_rows_kernel<float>, dim3(rows_blocks(rows)), dim3(256), 0, st, (const float*)F(b.f32),
                     w.g_ffn, rows, d, s.eps, static_cast<bf*>(b.nrm), static_cast<bf*>(b.nrm_lo), (float*)nullptr));
-  WCHECK(gemm_bf16(opnd(b.nrm, b.nrm_lo, d, d), no_opnd(), w.w_upgate, ugw, Outs{nullptr, nullptr, F(b.ug), ugw},
-                   nullptr, 0, rows, EPI_STORE, false, 0.f, st));
+  return gemm_bf16(opnd(b.nrm, b.nrm_lo, d, d), no_opnd(), w.w_upgate, ugw, Outs{nullptr, nullptr, F(b.ug), ugw},
+                   nullptr, 0, rows, EPI_STORE, false, 0.f, st);
+}
+
+// The layer's output from the recomputed intermediates: H_f = F + W_down (SiLU(gate) * up), as a
+// residual-stream tensor (fp32 and its pair): the next layer's input in the stack backward.
+whale_status layer_output_bf16(const Shape& s, const whale_layer_weights& w, const whale_shape_hint& h,
+                               const BwdBufs& b, const Stream3& out, cudaStream_t st) {
+  using bf = __nv_bfloat16;
+  const long long rows = (long long)h.B * s.N;
+  WCHECK(ew_launch(swiglu_pair_kernel, rows * s.H, st, (const float*)static_cast<float*>(b.ug), rows, s.H,
+                   s.tied ? 1 : 0, static_cast<bf*>(b.msw), static_cast<bf*>(b.msw_lo)));
+  return gemm_bf16(opnd(b.msw, b.msw_lo, s.H, s.H), no_opnd(), w.w_down, s.d, Outs{out.hi, out.lo, out.f32, s.d},
+                   static_cast<const float*>(b.f32), s.d, rows, EPI_RESID, false, 0.f, st);
+}
+
+// One layer's backward in bf16 mode (input as for recompute_bf16).
+whale_status layer_backward_bf16(const Shape& s, const Stream3& in, const void* slab, const int* offsets,
+                                 const whale_layer_weights& w, const float* dy, float* dx, void* ds,
+                                 const whale_layer_grads& gr, const whale_shape_hint& h, const BwdBufs& b,
+                                 cudaStream_t st) {
+  using bf = __nv_bfloat16;
+  const long long rows = (long long)h.B * s.N, T = h.total_L;
+  const int d = s.d, H = s.H, Fh = s.Fh, ugw = s.ugw, kvw = s.kvw;
+  auto F = [](void* p) { return static_cast<float*>(p); };
+  const void* x = in.hi;
+  const float* x32 = in.f32;
+  WCHECK(recompute_bf16(s, in, slab, offsets, w, h, b, st));
   // ---- S5 backward: SwiGLU FFN ----
   float* part = F(b.part);
   const size_t pc = b.part_floats;
@@ -1472,11 +1515,11 @@ whale_status layer_backward_bf16(const Shape& s, const void* x, const void* slab
     WCHECK(gemm_acc32(b.df, b.df_lo, d, true, b.g, Fh, true, d, Fh, rows, gr.w_f2, Fh, part, pc, st, b.g_lo));
     WCHECK(gemm_acc32(b.dz, b.dz_lo, Fh, false, w.w_f1, 2 * d, true, rows, 2 * d, Fh, F(b.dc), 2 * d, part, pc, st));
     WCHECK(gemm_acc32(b.dz, b.dz_lo, Fh, true, b.a, d, true, Fh, d, rows, gr.w_f1, 2 * d, part, pc, st, b.a_lo));
-    WCHECK(gemm_acc32(b.dz, b.dz_lo, Fh, true, x, d, true, Fh, d, rows, gr.w_f1 + d, 2 * d, part, pc, st));
+    WCHECK(gemm_acc32(b.dz, b.dz_lo, Fh, true, x, d, true, Fh, d, rows, gr.w_f1 + d, 2 * d, part, pc, st, in.lo));
   } else {
     WCHECK(gemm_acc32(b.df, b.df_lo, d, false, w.w_f2, 2 * d, true, rows, 2 * d, d, F(b.dc), 2 * d, part, pc, st));
     WCHECK(gemm_acc32(b.df, b.df_lo, d, true, b.a, d, true, d, d, rows, gr.w_f2, 2 * d, part, pc, st, b.a_lo));
-    WCHECK(gemm_acc32(b.df, b.df_lo, d, true, x, d, true, d, d, rows, gr.w_f2 + d, 2 * d, part, pc, st));
+    WCHECK(gemm_acc32(b.df, b.df_lo, d, true, x, d, true, d, d, rows, gr.w_f2 + d, 2 * d, part, pc, st, in.lo));
   }
   // ---- S3 backward: attention (KV-parallel) ----
   WCHECK(ew_launch(attn_bwd_prep_kernel, rows * s.h, st, (const float*)F(b.dc), (long long)(2 * d),
@@ -1522,8 +1565,8 @@ whale_status layer_backward_bf16(const Shape& s, const void* x, const void* slab
                    static_cast<bf*>(b.dq_lo), (long long)d, rows, d));
   WCHECK(gemm_acc32(b.dq_hi, b.dq_lo, d, false, w.w_q, d, true, rows, d, d, F(b.dn), d, part, pc, st));
   WCHECK(gemm_acc32(b.dq_hi, b.dq_lo, d, true, b.nq, d, true, d, d, rows, gr.w_q, d, part, pc, st, b.nq_lo));
-  WCHECK(rms_bwd<bf>(static_cast<const bf*>(x), w.g_q, F(b.dn), rows, d, s.eps, F(b.df32), d, F(b.dc) + d, 2 * d, dx,
-                     nullptr, nullptr, nullptr, nullptr, nullptr, F(b.colp), gr.g_q, st));
+  WCHECK(rms_bwd<float>(x32, w.g_q, F(b.dn), rows, d, s.eps, F(b.df32), d, F(b.dc) + d, 2 * d, dx, nullptr, nullptr,
+                        nullptr, nullptr, nullptr, F(b.colp), gr.g_q, st));
   // ---- S2 backward: K|V projection and the states' RMSNorm ----
   if (T > 0) {
     WCHECK(gemm_acc32(b.dkv, b.dkv_lo, kvw, false, w.w_kv, d, true, T, d, kvw, F(b.dsn), d, part, pc, st));
@@ -1633,6 +1676,42 @@ whale_status layer_backward_f32(const Shape& s, const float* x, const float* sla
     CUCHECK(cudaMemsetAsync(gr.w_kv, 0, (size_t)kvw * d * 4, st));
   }
   return WHALE_OK;
+}
+
+// Workspace of the stack backward (also enough for one layer): the backward buffers, the forward's
+// workspace for the fp32 mode's layer inputs, every layer's input as a residual-stream tensor (fp32,
+// plus its bf16 pair in bf16 mode), and a ping-pong pair of fp32 token gradients.
+struct StackBwd {
+  BwdBufs b;
+  char* fwd;
+  Layout fl;
+  Stream3 in[64];
+  float* g[2];
+};
+size_t stack_bwd_bytes(const Shape& s, const whale_shape_hint& h, char* base, StackBwd* sb = nullptr) {
+  StackBwd local;
+  StackBwd& k = sb ? *sb : local;
+  size_t o = align_up(bwd_buffers(s, h, base, &k.b));
+  k.fwd = nullptr;
+  if (!s.bf16) {  // the fp32 stack's forward runs the forward's own layer (its workspace); bf16 recomputes
+    k.fl = make_layout(s, h);
+    k.fwd = base ? base + o : nullptr;
+    o = align_up(o + k.fl.total);
+  }
+  const size_t rows = (size_t)h.B * s.N;
+  auto take = [&](size_t bytes) -> char* {
+    char* p = base ? base + o : nullptr;
+    o = align_up(o + bytes);
+    return p;
+  };
+  const int nl = std::min(s.layers, 64);
+  for (int l = 0; l < nl; ++l) {
+    k.in[l].f32 = reinterpret_cast<float*>(take(rows * s.d * 4));
+    k.in[l].hi = s.bf16 ? take(rows * s.d * 2) : nullptr;
+    k.in[l].lo = s.bf16 ? take(rows * s.d * 2) : nullptr;
+  }
+  for (int i = 0; i < 2; ++i) k.g[i] = reinterpret_cast<float*>(take(rows * s.d * 4));
+  return o;
 }
 
 bool grads_ok(const Shape& s, const whale_layer_grads* g) {
@@ -2085,8 +2164,7 @@ whale_status whale_cross_attention_noalloc(const whale_config* cfg, const void* 
 size_t whale_backward_workspace_size(const whale_config* cfg, const whale_shape_hint* hint) {
   Shape s;
   if (validate(cfg, &s) != WHALE_OK || check_hint(hint) != WHALE_OK || !backward_shape_ok(s) || s.prepared) return 0;
-  BwdBufs b;
-  return bwd_buffers(s, *hint, nullptr, &b);
+  return stack_bwd_bytes(s, *hint, nullptr);
 }
 
 whale_status whale_fusion_layer_backward(const whale_config* cfg, const void* tokens_in, const void* layer_states,
@@ -2102,7 +2180,7 @@ whale_status whale_fusion_layer_backward(const whale_config* cfg, const void* to
   if (!weights_ok(s, w) || !grads_ok(s, grads)) return WHALE_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   BwdBufs b;
-  const size_t need = bwd_buffers(s, *hint, nullptr, &b);
+  const size_t need = bwd_buffers(s, *hint, nullptr, &b);  // the prefix of whale_backward_workspace_size
   if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1))) return WHALE_ERR_WORKSPACE;
   if (hint->B == 0) {  // no examples: every gradient is zero
     const size_t d = s.d;
@@ -2123,11 +2201,74 @@ whale_status whale_fusion_layer_backward(const whale_config* cfg, const void* to
     return WHALE_ERR_INVALID_ARG;
   bwd_buffers(s, *hint, static_cast<char*>(ws), &b);
   WCHECK(debug_check(s, seq_offsets, *hint, st));
-  if (s.bf16)
-    return layer_backward_bf16(s, tokens_in, layer_states, seq_offsets, *w, d_out, d_tokens, d_states, *grads, *hint, b,
-                               st);
+  if (s.bf16) {
+    WCHECK(pair_from_bf16(tokens_in, static_cast<float*>(b.x32), b.xlo, (long long)hint->B * s.N * s.d, st));
+    const Stream3 in{static_cast<float*>(b.x32), const_cast<void*>(tokens_in), b.xlo};
+    return layer_backward_bf16(s, in, layer_states, seq_offsets, *w, d_out, d_tokens, d_states, *grads, *hint, b, st);
+  }
   return layer_backward_f32(s, static_cast<const float*>(tokens_in), static_cast<const float*>(layer_states),
                             seq_offsets, *w, d_out, d_tokens, static_cast<float*>(d_states), *grads, *hint, b, st);
+}
+
+whale_status whale_fusion_backward(const whale_config* cfg, const void* tokens, const void* seq_states,
+                                   const int* seq_offsets, const whale_layer_weights* weights, const float* d_out,
+                                   float* d_tokens, void* d_states, const whale_layer_grads* grads,
+                                   const whale_shape_hint* hint, void* ws, size_t ws_bytes, whale_stream_t stream) {
+  Shape s;
+  WCHECK(validate(cfg, &s));
+  WCHECK(check_hint(hint));
+  if (s.prepared || !backward_shape_ok(s) || s.layers > 64) return WHALE_ERR_UNSUPPORTED;
+  if (!weights || !grads) return WHALE_ERR_INVALID_ARG;
+  for (int l = 0; l < s.layers; ++l)
+    if (!weights_ok(s, &weights[l]) || !grads_ok(s, &grads[l])) return WHALE_ERR_INVALID_ARG;
+  const size_t need = stack_bwd_bytes(s, *hint, nullptr);
+  if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1))) return WHALE_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const long long rows = (long long)hint->B * s.N, T = hint->total_L;
+  if (hint->B == 0) {
+    for (int l = 0; l < s.layers; ++l)
+      WCHECK(whale_fusion_layer_backward(cfg, nullptr, nullptr, nullptr, &weights[l], nullptr, nullptr, nullptr,
+                                         &grads[l], hint, ws, ws_bytes, stream));
+    return WHALE_OK;
+  }
+  if (!tokens || !seq_offsets || !d_out || !d_tokens || (T > 0 && (!seq_states || !d_states)))
+    return WHALE_ERR_INVALID_ARG;
+  if (!aligned16(tokens) || !aligned16(d_out) || !aligned16(d_tokens) || (seq_states && !aligned16(seq_states)) ||
+      (d_states && !aligned16(d_states)))
+    return WHALE_ERR_INVALID_ARG;
+  StackBwd k;
+  stack_bwd_bytes(s, *hint, static_cast<char*>(ws), &k);
+  WCHECK(debug_check(s, seq_offsets, *hint, st));
+  const size_t slab_bytes = (size_t)T * s.d * s.es;
+  auto slab = [&](int l) { return T > 0 ? static_cast<const char*>(seq_states) + l * slab_bytes : nullptr; };
+  // forward, keeping every layer's input (the residual stream: fp32 and, in bf16 mode, its pair)
+  if (s.bf16) {
+    // the recompute path of the backward (hi/lo pairs, raw weights, K|V as pairs), so that every
+    // layer's input carries the precision its gradients need
+    WCHECK(pair_from_bf16(tokens, k.in[0].f32, k.in[0].lo, rows * s.d, st));
+    CUCHECK(cudaMemcpyAsync(k.in[0].hi, tokens, (size_t)rows * s.d * 2, cudaMemcpyDeviceToDevice, st));
+    for (int l = 0; l + 1 < s.layers; ++l) {
+      WCHECK(recompute_bf16(s, k.in[l], slab(l), seq_offsets, weights[l], *hint, k.b, st));
+      WCHECK(layer_output_bf16(s, weights[l], *hint, k.b, k.in[l + 1], st));
+    }
+  } else {
+    CUCHECK(cudaMemcpyAsync(k.in[0].f32, tokens, (size_t)rows * s.d * 4, cudaMemcpyDeviceToDevice, st));
+    for (int l = 0; l + 1 < s.layers; ++l)
+      WCHECK(layer_f32(s, k.in[l].f32, slab(l), seq_offsets, weights[l], k.in[l + 1].f32, *hint, k.fwd, k.fl, st));
+  }
+  // backward, last layer first: each layer's token gradient is the next one's upstream gradient
+  const float* g = d_out;
+  for (int l = s.layers - 1; l >= 0; --l) {
+    float* dx = l == 0 ? d_tokens : k.g[l & 1];
+    void* dsl = T > 0 ? static_cast<char*>(d_states) + l * slab_bytes : nullptr;
+    if (s.bf16)
+      WCHECK(layer_backward_bf16(s, k.in[l], slab(l), seq_offsets, weights[l], g, dx, dsl, grads[l], *hint, k.b, st));
+    else
+      WCHECK(layer_backward_f32(s, k.in[l].f32, reinterpret_cast<const float*>(slab(l)), seq_offsets, weights[l], g, dx,
+                                static_cast<float*>(dsl), grads[l], *hint, k.b, st));
+    g = dx;
+  }
+  return WHALE_OK;
 }
 
 whale_status whale_test_bounded_waits(unsigned long long limit_ns, whale_stream_t stream) {

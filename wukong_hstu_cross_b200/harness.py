@@ -151,3 +151,23 @@ def run_layer_backward(p: Problem, layer: int, d_out: torch.Tensor, stream=None)
     W.whale_fusion_layer_backward(cfg, p.tokens, p.states[layer], p.offsets_t, lw, d_out, d_tokens, d_states, grads,
                                   p.hint, ws, stream=stream)
     return {"d_tokens": d_tokens, "d_states": d_states, **grads}
+
+
+def run_stack_backward(p: Problem, d_out: torch.Tensor, stream=None) -> dict:
+    """Gradients of the whole stack for d_out (fp32 [B, N, d]) through whale_fusion_backward, with the
+    raw weights. Returns {"d_tokens", "d_states" [n_layers, total_L, d], "grads": one dict per layer}."""
+    w = p.w
+    dev = p.tokens.device
+    raw = p.raw_weights or p.weights
+    grads = [{k: torch.empty(tuple(v.shape), dtype=torch.float32, device=dev) for k, v in lw.items()
+              if v is not None and k != "w_kabs"} for lw in raw]
+    cfg = config_of(w, flags_of(p.flags.get("shared_kv", False), p.flags.get("tied_gate", False)))
+    nbytes = W.whale_backward_workspace_size(cfg, p.hint)
+    if nbytes == 0:
+        raise ValueError("shape not supported by the backward pass")
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    d_tokens = torch.empty(p.tokens.shape, dtype=torch.float32, device=dev)
+    d_states = torch.empty(p.states.shape, dtype=p.states.dtype, device=dev)
+    W.whale_fusion_backward(cfg, p.tokens, p.states, p.offsets_t, raw, d_out, d_tokens, d_states, grads, p.hint, ws,
+                            stream=stream)
+    return {"d_tokens": d_tokens, "d_states": d_states, "grads": grads}

@@ -92,6 +92,8 @@ _SIGS = {
     "whale_backward_workspace_size": ([POINTER(whale_config), POINTER(whale_shape_hint)], c_size_t),
     "whale_fusion_layer_backward": ([POINTER(whale_config), _P, _P, _P, POINTER(whale_layer_weights), _P, _P, _P,
                                      POINTER(whale_layer_grads), POINTER(whale_shape_hint), _P, c_size_t, _P], c_int),
+    "whale_fusion_backward": ([POINTER(whale_config), _P, _P, _P, POINTER(whale_layer_weights), _P, _P, _P,
+                               POINTER(whale_layer_grads), POINTER(whale_shape_hint), _P, c_size_t, _P], c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -327,6 +329,20 @@ def whale_fusion_layer_backward(cfg, tokens_in, layer_states, seq_offsets, layer
     if raw:
         return st
     _check(st, "whale_fusion_layer_backward")
+
+
+def whale_fusion_backward(cfg, wukong_tokens, seq_states, seq_offsets, weights, d_out, d_tokens, d_states, grads,
+                          hint, workspace, workspace_bytes=None, stream=None, raw=False):
+    """Gradients of the whole stack (see include/whale_fusion.h): `weights` one dict per layer (raw),
+    `grads` one dict of fp32 tensors per layer."""
+    w = weights if isinstance(weights, ctypes.Array) else weights_array(weights)
+    g = (whale_layer_grads * len(grads))(*[layer_grads(x) for x in grads])
+    st = _lib.whale_fusion_backward(ctypes.byref(cfg), _ptr(wukong_tokens), _ptr(seq_states), _ptr(seq_offsets), w,
+                                    _ptr(d_out), _ptr(d_tokens), _ptr(d_states), g, ctypes.byref(hint),
+                                    _ptr(workspace), _ws_bytes(workspace, workspace_bytes), _stream(stream))
+    if raw:
+        return st
+    _check(st, "whale_fusion_backward")
 
 
 def whale_test_bounded_waits(limit_ns: int, stream=None, raw=False):
