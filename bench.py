@@ -488,6 +488,7 @@ def main():
     ap.add_argument("--fold-per-call", action="store_true",
                     help="fold the RMSNorm gains into the weights inside every forward instead of once at load")
     ap.add_argument("--no-backward", action="store_true", help="skip the one-layer backward measurement")
+    ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay measurement")
     ap.add_argument("--materialized-kv", action="store_true",
                     help="project K|V and attend over them even where the absorbed attention applies")
     args = ap.parse_args()
@@ -518,22 +519,55 @@ def main():
     total_L = p.total_L
 
     # ---------------- device-resident timed region: the whole stack per step ----------------
+    # A deployment replays a captured CUDA graph of the forward (launches, their programmatic
+    # dependencies and arguments recorded once, the same kernels); that replay is the timed step.
+    # The same step launched call by call is timed beside it (`stream_launch`); --no-graph makes the
+    # call-by-call launches the timed step.
     for _ in range(args.warmup):
         Hn.run_forward(p, stream)
     torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
-        barrier(world)
+
+    def timed(step_fn, steps, sample_clocks):
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        clk = ClockSampler(local) if sample_clocks else None
+        if clk:
+            clk.__enter__()
+        try:
+            barrier(world)
+            torch.cuda.synchronize()
+            ev0.record(stream)
+            for _ in range(steps):
+                step_fn()
+            ev1.record(stream)
+            torch.cuda.synchronize()
+            barrier(world)
+        finally:
+            if clk:
+                clk.__exit__(None, None, None)
+        return max_over_ranks(ev0.elapsed_time(ev1) / steps, world), (clk.summary() if clk else None)
+
+    stream_launch = None
+    if args.no_graph:
+        ms, clocks = timed(lambda: Hn.run_forward(p, stream), args.steps, True)
+        launch = "call by call (programmatic dependent launches on one stream)"
+    else:
+        side = torch.cuda.Stream()
+        with torch.cuda.stream(side):
+            Hn.run_forward(p, side)
         torch.cuda.synchronize()
-        ev0.record(stream)
-        for _ in range(args.steps):
-            Hn.run_forward(p, stream)
-        ev1.record(stream)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            Hn.run_forward(p, side)
         torch.cuda.synchronize()
-        barrier(world)
-    clocks = clk.summary()
-    ms = ev0.elapsed_time(ev1) / args.steps
-    ms = max_over_ranks(ms, world)
+        for _ in range(args.warmup):
+            g.replay()
+        torch.cuda.synchronize()
+        ms, clocks = timed(g.replay, args.steps, True)
+        s_ms, _ = timed(lambda: Hn.run_forward(p, stream), args.steps, False)
+        stream_launch = {"ms_per_step": s_ms, "value": world * w.batch / (s_ms / 1e3), "steps": args.steps,
+                         "what": "the same step launched call by call (whale_fusion_forward per step)"}
+        launch = "captured CUDA graph of whale_fusion_forward, replayed once per step"
+        del g
     value = world * w.batch / (ms / 1e3)
 
     # ---------------- every kernel of one step, live: the library's per-kernel events -------------
@@ -717,6 +751,8 @@ def main():
                               "kv_proj_ms": t_kv, "attention_ms": t_attn, "absorbed_attention_ms": t_abs,
                               "peaks": f"{peak_src}: {peaks['hbm_gbs']} GB/s, {tc_step} TFLOP/s"},
             "kernels": kernels,
+            "launch": launch,
+            "stream_launch": stream_launch,
             "backward": bwd,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": (len(recs) or launches_per_step(w, args.fold_per_call, absorbed)) * args.steps,
             "clocks": clocks,

@@ -75,15 +75,17 @@ struct GemmArgs {
 };
 
 
-template <int BN, bool SPLIT, bool SPLIT_B = false>
+// A pipeline stage holds KPS consecutive 64-column K blocks: [A hi: KPS blocks][A lo: KPS blocks]
+// [W: KPS blocks][W lo: KPS blocks], each block a 128-byte-swizzled [rows][64] tile.
+template <int BN, bool SPLIT, bool SPLIT_B = false, int KPS = 1>
 struct GemmSmem {
   static constexpr int BM = 128, BK = 64;
-  static constexpr uint32_t A_BYTES = BM * BK * 2;
-  static constexpr uint32_t A_ALL = SPLIT ? 2 * A_BYTES : A_BYTES;
-  static constexpr uint32_t B_BYTES = BN * BK * 2;
-  static constexpr uint32_t STAGE_BYTES = A_ALL + (SPLIT_B ? 2 : 1) * B_BYTES;
+  static constexpr uint32_t A_BYTES = BM * BK * 2;  // one K block of A (hi or lo)
+  static constexpr uint32_t A_ALL = (SPLIT ? 2 : 1) * KPS * A_BYTES;
+  static constexpr uint32_t B_BYTES = BN * BK * 2;  // one K block of W
+  static constexpr uint32_t STAGE_BYTES = A_ALL + (SPLIT_B ? 2 : 1) * KPS * B_BYTES;
   // stages fill what the 227 KB of shared memory leaves (one CTA per SM either way): five 40 KB
-  // stages for the 64-column hi/lo tiles
+  // stages for the 64-column hi/lo tiles, two 80 KB ones when a stage holds two K blocks
   static constexpr int FIXED = 1024 /*alignment slack*/ + 2 * 128 * 4 /*row factors*/ + 256 /*barriers*/;
   static constexpr int STAGES =
       ((232448 - FIXED) / (int)STAGE_BYTES) > 8 ? 8 : ((232448 - FIXED) / (int)STAGE_BYTES);
@@ -225,16 +227,23 @@ constexpr uint32_t kIdescAMnMajor = 1u << 15;
 // SPLIT_B: B is a hi/lo pair too (single A source: tmA1 then holds B's lo half), and every k-step
 // issues A_hi B_hi, A_lo B_hi and A_hi B_lo (the A_lo B_lo term is below 2^-16 of the product):
 // the weight gradients of the token side, whose sums over rows cancel, need both operands at ~16 bits.
-template <int BN, int EPI, bool ROWNORM, bool SPLIT, bool A_MN = false, bool B_MN = false, bool SPLIT_B = false>
+//
+// KPS = 2: each stage carries two K blocks, loaded with 3-D tensor maps (the view {64 columns, rows,
+// K / 64 blocks} of each K-major operand, box {64, rows, 2}), so a stage costs three copies instead of
+// six. The K blocks of every tile, of A0 and of each split-K range are then even in number.
+template <int BN, int EPI, bool ROWNORM, bool SPLIT, bool A_MN = false, bool B_MN = false, bool SPLIT_B = false,
+          int KPS = 1>
 __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA0lo,
                    const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmA1lo,
                    const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
-  using L = GemmSmem<BN, SPLIT, SPLIT_B>;
+  using L = GemmSmem<BN, SPLIT, SPLIT_B, KPS>;
   constexpr int STAGES = L::STAGES;
   constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators: 128, 256 or 512 columns
   static_assert(!(ROWNORM && A_MN), "row statistics read K-major A rows");
   static_assert(!(ROWNORM && SPLIT_B), "row-normalised GEMMs have one B");
+  static_assert(KPS == 1 || (KPS == 2 && !A_MN && !B_MN && !SPLIT_B), "two-block stages: K-major operands");
+  static_assert(STAGES >= 2, "pipeline depth");
   constexpr uint32_t MN_BOX = 64 * 64 * 2;  // one MN-major box: 64 K rows x 64 elements
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -302,12 +311,26 @@ __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
   if (warp == 0) {
     // ---------------- TMA producer: every K block of every tile of this CTA ----------------
     if (lane == 0) {
+      auto load_b = [&](uint8_t* st, int kb, int n0, uint64_t* bar) {
+        if (B_MN) {
+#pragma unroll
+          for (int i = 0; i < BN / 64; ++i) {
+            tma_load_2d(st + L::A_ALL + i * MN_BOX, &tmB, n0 + 64 * i, kb * L::BK, bar);
+            if (SPLIT_B) tma_load_2d(st + L::A_ALL + L::B_BYTES + i * MN_BOX, &tmA1, n0 + 64 * i, kb * L::BK, bar);
+          }
+        } else if (KPS == 1) {
+          tma_load_2d(st + L::A_ALL, &tmB, kb * L::BK, n0, bar);
+          if (SPLIT_B) tma_load_2d(st + L::A_ALL + L::B_BYTES, &tmA1, kb * L::BK, n0, bar);
+        } else {
+          tma_load_3d(st + L::A_ALL, &tmB, 0, n0, kb, bar);
+        }
+      };
       int kg = 0;
       bool stop = false;
       for (int tile = blockIdx.x; tile < args.num_tiles && !stop; tile += gridDim.x) {
         int m0, n0, kb_lo, kb_hi, split;
         tile_of(tile, m0, n0, kb_lo, kb_hi, split);
-        for (int kb = kb_lo; kb < kb_hi; ++kb, ++kg) {
+        for (int kb = kb_lo; kb < kb_hi; kb += KPS, ++kg) {
           const int s = kg % STAGES, u = kg / STAGES;
           if (kg >= STAGES && !mbar_wait(&empty[s], (u - 1) & 1, abort_flag)) {
             stop = true;
@@ -328,20 +351,14 @@ __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
               tma_load_2d(st + i * MN_BOX, first ? &tmA0 : &tmA1, ma + 64 * i, kc, &full[s]);
               if (SPLIT) tma_load_2d(st + L::A_BYTES + i * MN_BOX, first ? &tmA0lo : &tmA1lo, ma + 64 * i, kc, &full[s]);
             }
-          } else {
+          } else if (KPS == 1) {
             tma_load_2d(st, first ? &tmA0 : &tmA1, kc, ma, &full[s]);
             if (SPLIT) tma_load_2d(st + L::A_BYTES, first ? &tmA0lo : &tmA1lo, kc, ma, &full[s]);
-          }
-          if (B_MN) {
-#pragma unroll
-            for (int i = 0; i < BN / 64; ++i) {
-              tma_load_2d(st + L::A_ALL + i * MN_BOX, &tmB, n0 + 64 * i, kb * L::BK, &full[s]);
-              if (SPLIT_B) tma_load_2d(st + L::A_ALL + L::B_BYTES + i * MN_BOX, &tmA1, n0 + 64 * i, kb * L::BK, &full[s]);
-            }
           } else {
-            tma_load_2d(st + L::A_ALL, &tmB, kb * L::BK, n0, &full[s]);
-            if (SPLIT_B) tma_load_2d(st + L::A_ALL + L::B_BYTES, &tmA1, kb * L::BK, n0, &full[s]);
+            tma_load_3d(st, first ? &tmA0 : &tmA1, 0, ma, kc / L::BK, &full[s]);
+            if (SPLIT) tma_load_3d(st + KPS * L::A_BYTES, first ? &tmA0lo : &tmA1lo, 0, ma, kc / L::BK, &full[s]);
           }
+          load_b(st, kb, n0, &full[s]);
         }
       }
       if (*abort_flag) {
@@ -365,28 +382,32 @@ __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
         const uint32_t d_tmem = tmem_base + acc * BN;
         int m0, n0, kb_lo, kb_hi, split;
         tile_of(tile, m0, n0, kb_lo, kb_hi, split);
-        for (int kb = kb_lo; kb < kb_hi; ++kb, ++kg) {
+        for (int kb = kb_lo; kb < kb_hi; kb += KPS, ++kg) {
           const int s = kg % STAGES, u = kg / STAGES;
           if (!mbar_wait(&full[s], u & 1, abort_flag)) {
             stop = true;
             break;
           }
           tc_fence_after();
-          const uint32_t a_base = smem_u32(smem + s * L::STAGE_BYTES);
-          const uint32_t b_base = a_base + L::A_ALL;
+          const uint32_t st_base = smem_u32(smem + s * L::STAGE_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < L::BK / 16; ++kk) {
-            // MN-major: 16 K rows of 128 bytes per k-step; 64-element MN groups one box apart
-            auto bd = [&](uint32_t base) {
-              return B_MN ? sdesc_mn_sw128(base + kk * 2048, MN_BOX, 1024) : sdesc_k_sw128(base + kk * 32);
-            };
-            auto ad = [&](uint32_t base) {
-              return A_MN ? sdesc_mn_sw128(base + kk * 2048, MN_BOX, 1024) : sdesc_k_sw128(base + kk * 32);
-            };
-            const uint64_t bdesc = bd(b_base), adesc = ad(a_base);
-            umma_f16(d_tmem, adesc, bdesc, idesc, (kb > kb_lo || kk > 0) ? 1u : 0u);
-            if (SPLIT) umma_f16(d_tmem, ad(a_base + L::A_BYTES), bdesc, idesc, 1u);
-            if (SPLIT_B) umma_f16(d_tmem, adesc, bd(b_base + L::B_BYTES), idesc, 1u);
+          for (int j = 0; j < KPS; ++j) {
+            const uint32_t a_base = st_base + j * L::A_BYTES;
+            const uint32_t b_base = st_base + L::A_ALL + j * L::B_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < L::BK / 16; ++kk) {
+              // MN-major: 16 K rows of 128 bytes per k-step; 64-element MN groups one box apart
+              auto bd = [&](uint32_t base) {
+                return B_MN ? sdesc_mn_sw128(base + kk * 2048, MN_BOX, 1024) : sdesc_k_sw128(base + kk * 32);
+              };
+              auto ad = [&](uint32_t base) {
+                return A_MN ? sdesc_mn_sw128(base + kk * 2048, MN_BOX, 1024) : sdesc_k_sw128(base + kk * 32);
+              };
+              const uint64_t bdesc = bd(b_base), adesc = ad(a_base);
+              umma_f16(d_tmem, adesc, bdesc, idesc, (kb > kb_lo || j > 0 || kk > 0) ? 1u : 0u);
+              if (SPLIT) umma_f16(d_tmem, ad(a_base + KPS * L::A_BYTES), bdesc, idesc, 1u);
+              if (SPLIT_B) umma_f16(d_tmem, adesc, bd(b_base + KPS * L::B_BYTES), idesc, 1u);
+            }
           }
           umma_commit(&empty[s]);
         }
@@ -402,30 +423,33 @@ __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
         const int acc = it & 1, ua = it >> 1;
         float ss = 0.f;
         bool ok = true;
-        for (int kb = 0; kb < KB; ++kb, ++kg) {
+        for (int kb = 0; kb < KB; kb += KPS, ++kg) {
           const int s = kg % STAGES, u = kg / STAGES;
           if (!mbar_wait(&full[s], u & 1, abort_flag)) {
             ok = false;
             break;
           }
-          if (kb < args.kb0) {
-            // The row's 128 bytes are contiguous; the 128-byte swizzle stores its logical 16-byte
-            // chunk c at position c ^ (row % 8) (identically in the hi and lo tiles). Summing in
-            // logical order keeps the row factor independent of the row's position in the tile.
-            const uint8_t* st = smem + s * L::STAGE_BYTES + row * 128;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const int pc = c ^ (row & 7);
-              float f[8];
-              bf16x8_to_f32(reinterpret_cast<const uint4*>(st)[pc], f);
-              if (SPLIT) {
-                float fl[8];
-                bf16x8_to_f32(reinterpret_cast<const uint4*>(st + L::A_BYTES)[pc], fl);
+          for (int jb = 0; jb < KPS; ++jb) {
+            if (kb + jb < args.kb0) {
+              // The row's 128 bytes are contiguous; the 128-byte swizzle stores its logical 16-byte
+              // chunk c at position c ^ (row % 8) (identically in the hi and lo tiles). Summing in
+              // logical order keeps the row factor independent of the row's position in the tile.
+              const uint8_t* st = smem + s * L::STAGE_BYTES + jb * L::A_BYTES + row * 128;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) f[j] += fl[j];
+              for (int c = 0; c < 8; ++c) {
+                const int pc = c ^ (row & 7);
+                float f[8];
+                bf16x8_to_f32(reinterpret_cast<const uint4*>(st)[pc], f);
+                if (SPLIT) {
+                  float fl[8];
+                  bf16x8_to_f32(reinterpret_cast<const uint4*>(st + KPS * L::A_BYTES)[pc], fl);
+#pragma unroll
+                  for (int j = 0; j < 8; ++j) f[j] += fl[j];
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) ss = fmaf(f[j], f[j], ss);
               }
-#pragma unroll
-              for (int j = 0; j < 8; ++j) ss = fmaf(f[j], f[j], ss);
             }
           }
           __syncwarp();

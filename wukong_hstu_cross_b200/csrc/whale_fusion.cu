@@ -184,6 +184,30 @@ whale_status tmap_bf16(CUtensorMap* tm, const void* base, long long rows, long l
   return tmap_bf16_box(tm, base, rows, cols, ld, 64, box_rows);
 }
 
+// A K-major bf16 operand [rows, K] (row stride ld, K a multiple of 64) seen as {64 columns, rows,
+// K / 64 blocks}: one box {64, box_rows, kps} brings kps consecutive 64-column blocks, each a
+// 128-byte-swizzled [box_rows][64] tile.
+whale_status tmap_bf16_kblocks(CUtensorMap* tm, const void* base, long long rows, long long K, long long ld,
+                               int box_rows, int kps) {
+  WCHECK(get_encoder());
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || (ld * 2) % 16 || rows <= 0 || K <= 0 || K % 64 || K > ld)
+    return WHALE_ERR_INVALID_ARG;
+  cuuint64_t dims[3] = {64u, (cuuint64_t)rows, (cuuint64_t)(K / 64)};
+  cuuint64_t strides[2] = {(cuuint64_t)(ld * 2), 128u};
+  cuuint32_t box[3] = {64u, (cuuint32_t)box_rows, (cuuint32_t)kps};
+  cuuint32_t es[3] = {1u, 1u, 1u};
+  CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? WHALE_OK : WHALE_ERR_CUDA;
+}
+
+// A K-major operand's map for stages of kps K blocks (kps 1: the 2-D map).
+whale_status tmap_operand(CUtensorMap* tm, const void* base, long long rows, long long K, long long ld, int box_rows,
+                          int kps) {
+  return kps == 1 ? tmap_bf16(tm, base, rows, K, ld, box_rows) : tmap_bf16_kblocks(tm, base, rows, K, ld, box_rows, kps);
+}
+
 // ------------------------------------------------------------------------------------------
 // Validated shape
 // ------------------------------------------------------------------------------------------
@@ -382,27 +406,54 @@ struct Outs {
   long long ld;
 };
 
-template <int BN, int EPI, bool RN, bool SPLIT, bool A_MN = false, bool B_MN = false, bool SPLIT_B = false>
+template <int BN, int EPI, bool RN, bool SPLIT, bool A_MN = false, bool B_MN = false, bool SPLIT_B = false,
+          int KPS = 1>
 whale_status launch_gemm_t(const CUtensorMap* tm, const GemmArgs& g, long long tiles, cudaStream_t st) {
-  const size_t smem = GemmSmem<BN, SPLIT, SPLIT_B>::BYTES;
-  auto kern = gemm_tc_kernel<BN, EPI, RN, SPLIT, A_MN, B_MN, SPLIT_B>;
-  CUCHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  const unsigned grid = (unsigned)(tiles < kNumSM ? tiles : kNumSM);
-  return launch_pdl(kern, dim3(grid), dim3(gemm_threads<RN>()), smem, st, tm[0], tm[1], tm[2], tm[3], tm[4], g);
+  if constexpr (GemmSmem<BN, SPLIT, SPLIT_B, KPS>::STAGES < 2) {
+    return WHALE_ERR_UNSUPPORTED;  // two stages of this tile do not fit in shared memory
+  } else {
+    const size_t smem = GemmSmem<BN, SPLIT, SPLIT_B, KPS>::BYTES;
+    auto kern = gemm_tc_kernel<BN, EPI, RN, SPLIT, A_MN, B_MN, SPLIT_B, KPS>;
+    CUCHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    const unsigned grid = (unsigned)(tiles < kNumSM ? tiles : kNumSM);
+    return launch_pdl(kern, dim3(grid), dim3(gemm_threads<RN>()), smem, st, tm[0], tm[1], tm[2], tm[3], tm[4], g);
+  }
 }
 
-template <int BN>
+template <int BN, int KPS>
 whale_status launch_gemm_bn(int epi, bool rn, bool split, const CUtensorMap* tm, const GemmArgs& g, long long tiles,
                             cudaStream_t st) {
-  if (rn && epi == EPI_STORE && !split) return launch_gemm_t<BN, EPI_STORE, true, false>(tm, g, tiles, st);
-  if (rn && epi == EPI_STORE && split) return launch_gemm_t<BN, EPI_STORE, true, true>(tm, g, tiles, st);
+  if (rn && epi == EPI_STORE && !split)
+    return launch_gemm_t<BN, EPI_STORE, true, false, false, false, false, KPS>(tm, g, tiles, st);
+  if (rn && epi == EPI_STORE && split)
+    return launch_gemm_t<BN, EPI_STORE, true, true, false, false, false, KPS>(tm, g, tiles, st);
   if (!split) return WHALE_ERR_UNSUPPORTED;
-  if (!rn && epi == EPI_STORE) return launch_gemm_t<BN, EPI_STORE, false, true>(tm, g, tiles, st);
-  if (rn && epi == EPI_SWIGLU) return launch_gemm_t<BN, EPI_SWIGLU, true, true>(tm, g, tiles, st);
-  if (rn && epi == EPI_SWIGLU_TIED) return launch_gemm_t<BN, EPI_SWIGLU_TIED, true, true>(tm, g, tiles, st);
-  if (!rn && epi == EPI_SILU) return launch_gemm_t<BN, EPI_SILU, false, true>(tm, g, tiles, st);
-  if (!rn && epi == EPI_RESID) return launch_gemm_t<BN, EPI_RESID, false, true>(tm, g, tiles, st);
+  if (!rn && epi == EPI_STORE) return launch_gemm_t<BN, EPI_STORE, false, true, false, false, false, KPS>(tm, g, tiles, st);
+  if (rn && epi == EPI_SWIGLU) return launch_gemm_t<BN, EPI_SWIGLU, true, true, false, false, false, KPS>(tm, g, tiles, st);
+  if (rn && epi == EPI_SWIGLU_TIED)
+    return launch_gemm_t<BN, EPI_SWIGLU_TIED, true, true, false, false, false, KPS>(tm, g, tiles, st);
+  if (!rn && epi == EPI_SILU) return launch_gemm_t<BN, EPI_SILU, false, true, false, false, false, KPS>(tm, g, tiles, st);
+  if (!rn && epi == EPI_RESID) return launch_gemm_t<BN, EPI_RESID, false, true, false, false, false, KPS>(tm, g, tiles, st);
   return WHALE_ERR_UNSUPPORTED;
+}
+
+// Pipeline cost of one stage in SM cycles, as measured for TMA tensor copies of L2-resident tiles on
+// B200 (one CTA per SM, rings of 2 to 8 stages of 1 to 8 copies): each stage (one mbarrier) costs a
+// fixed ~470 cycles, each copy ~160 more and its bytes one cycle per ~240, almost independent of how
+// many stages are in flight. Two-K-block stages took the K loop of the Fusion MLP's GEMMs from 0.51
+// to 0.40 us per K block when run alone.
+inline double gemm_stage_cycles(int bn, bool split, int kps) {
+  const double copies = split ? 3.0 : 2.0;
+  const double bytes = kps * ((split ? 32768.0 : 16384.0) + bn * 128.0);
+  const double load = 470.0 + 160.0 * copies + bytes / 240.0;
+  const double mma = kps * (split ? 4.0 : 2.0) * bn;
+  return std::max(load, mma);
+}
+
+// Shared memory of a tile configuration holds at least two stages.
+template <int BN>
+bool gemm_kps2_fits(bool split) {
+  return split ? GemmSmem<BN, true, false, 2>::STAGES >= 2 : GemmSmem<BN, false, false, 2>::STAGES >= 2;
 }
 
 // Co-resident 2-CTA clusters of the 2-SM GEMM on the current device (cached per device).
@@ -472,33 +523,40 @@ whale_status gemm_bf16(const Opnd& a0, const Opnd& a1, const void* W, int N, con
     if (N % 256 == 0) WCHECK(g2_max_pairs(&pairs));
     if (pairs > 0) return gemm_rownorm_2sm(a0, W, N, out, M, eps, pairs, st);
   }
-  // Tile width by a small cost model (cycles): per-CTA fixed cost + tiles per persistent CTA x
-  // (per 64-deep K block the larger of the MMA time and the operand bytes at ~80 B/clk, the rate
-  // one latency-bound CTA streams from L2).
+  // Tile width and K blocks per stage by a small cost model (cycles): per-CTA fixed cost + tiles per
+  // persistent CTA x stages per tile x the larger of a stage's MMA time and its TMA cost.
   const int KB = (a0.K + a1.K) / 64;
-  auto cost = [&](int bn) -> double {
+  const bool kps2_ok = KB % 2 == 0 && (a0.K / 64) % 2 == 0;
+  auto cost = [&](int bn, int kps) -> double {
     if (N % bn) return 1e300;
+    if (kps == 2) {
+      const bool fits = bn == 64 ? gemm_kps2_fits<64>(split) : bn == 128 ? gemm_kps2_fits<128>(split)
+                                                                         : gemm_kps2_fits<256>(split);
+      if (!kps2_ok || !fits) return 1e300;
+    }
     const double per_cta = (double)cdiv<long long>(tm * (N / bn), kNumSM);  // tiles per persistent CTA
-    const double mma = (split ? 4.0 : 2.0) * bn;
-    const double bytes = (split ? 32768.0 : 16384.0) + bn * 128.0;
-    return 5600.0 + per_cta * KB * std::max(mma, bytes / 80.0);
+    return 5600.0 + per_cta * (KB / kps) * gemm_stage_cycles(bn, split, kps);
   };
-  int bn = 64;
-  for (int cand : {128, 256})
-    if (cost(cand) < cost(bn)) bn = cand;
+  int bn = 64, kps = 1;
+  for (int cand : {64, 128, 256})
+    for (int kc : {1, 2})
+      if (cost(cand, kc) < cost(bn, kps)) {
+        bn = cand;
+        kps = kc;
+      }
   CUtensorMap maps[5];
-  WCHECK(tmap_bf16(&maps[0], a0.hi, M, a0.K, a0.ld, 128));
-  if (split) WCHECK(tmap_bf16(&maps[1], a0.lo, M, a0.K, a0.ld, 128));
+  WCHECK(tmap_operand(&maps[0], a0.hi, M, a0.K, a0.ld, 128, kps));
+  if (split) WCHECK(tmap_operand(&maps[1], a0.lo, M, a0.K, a0.ld, 128, kps));
   else maps[1] = maps[0];
   if (a1.K > 0) {
-    WCHECK(tmap_bf16(&maps[2], a1.hi, M, a1.K, a1.ld, 128));
-    if (split) WCHECK(tmap_bf16(&maps[3], a1.lo, M, a1.K, a1.ld, 128));
+    WCHECK(tmap_operand(&maps[2], a1.hi, M, a1.K, a1.ld, 128, kps));
+    if (split) WCHECK(tmap_operand(&maps[3], a1.lo, M, a1.K, a1.ld, 128, kps));
     else maps[3] = maps[2];
   } else {
     maps[2] = maps[0];
     maps[3] = maps[1];
   }
-  WCHECK(tmap_bf16(&maps[4], W, N, a0.K + a1.K, a0.K + a1.K, bn));
+  WCHECK(tmap_operand(&maps[4], W, N, a0.K + a1.K, a0.K + a1.K, bn, kps));
   GemmArgs g{};
   g.M = (int)M;
   g.N = N;
@@ -515,9 +573,14 @@ whale_status gemm_bf16(const Opnd& a0, const Opnd& a1, const void* W, int N, con
   g.resid32 = resid32;
   g.ldr = ldr;
   const long long tiles = tm * g.tiles_n;
-  if (bn == 256) return launch_gemm_bn<256>(epi, rn, split, maps, g, tiles, st);
-  if (bn == 128) return launch_gemm_bn<128>(epi, rn, split, maps, g, tiles, st);
-  return launch_gemm_bn<64>(epi, rn, split, maps, g, tiles, st);
+  if (kps == 2) {
+    if (bn == 256) return launch_gemm_bn<256, 2>(epi, rn, split, maps, g, tiles, st);
+    if (bn == 128) return launch_gemm_bn<128, 2>(epi, rn, split, maps, g, tiles, st);
+    return launch_gemm_bn<64, 2>(epi, rn, split, maps, g, tiles, st);
+  }
+  if (bn == 256) return launch_gemm_bn<256, 1>(epi, rn, split, maps, g, tiles, st);
+  if (bn == 128) return launch_gemm_bn<128, 1>(epi, rn, split, maps, g, tiles, st);
+  return launch_gemm_bn<64, 1>(epi, rn, split, maps, g, tiles, st);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -882,10 +945,11 @@ whale_status gemm_qabs(const Shape& s, const void* q, const void* wkabs, void* q
 whale_status gemm_vabs(const Shape& s, const void* zh, const void* wv, void* a, void* a_lo, long long rows,
                        cudaStream_t st) {
   if (s.dh != 64) return WHALE_ERR_UNSUPPORTED;
+  const int kps = (s.d / 64) % 2 == 0 ? 2 : 1;
   CUtensorMap maps[5];
-  WCHECK(tmap_bf16(&maps[0], zh, (long long)s.h * rows, s.d, s.d, 128));
+  WCHECK(tmap_operand(&maps[0], zh, (long long)s.h * rows, s.d, s.d, 128, kps));
   maps[1] = maps[2] = maps[3] = maps[0];
-  WCHECK(tmap_bf16(&maps[4], wv, s.d, s.d, s.d, 64));
+  WCHECK(tmap_operand(&maps[4], wv, s.d, s.d, s.d, 64, kps));
   GemmArgs g{};
   g.M = (int)rows;
   g.N = s.d;
@@ -900,6 +964,7 @@ whale_status gemm_vabs(const Shape& s, const void* zh, const void* wv, void* a, 
   g.head_tiles = 1;
   g.a_kb_step = 0;
   g.a_row_step = rows;
+  if (kps == 2) return launch_gemm_t<64, EPI_STORE, false, false, false, false, false, 2>(maps, g, tiles, st);
   return launch_gemm_t<64, EPI_STORE, false, false>(maps, g, tiles, st);
 }
 
