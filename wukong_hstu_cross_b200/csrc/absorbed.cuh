@@ -185,7 +185,9 @@ __global__ void __launch_bounds__(1024) abs_units_kernel(const int* __restrict__
   }
   if (threadIdx.x == 1023) ustart[B] = part[1023];
   if (P <= 0) return;
-  for (int i = threadIdx.x; i < 2 + P; i += blockDim.x) pq[i] = 0;  // the finishing order of pass A
+  // The finishing order of pass A (ordering: this clear -> pass A, which waits on its predecessor,
+  // so on this kernel transitively -> pass A publishes -> pass B acquires -> the merge clears again).
+  for (int i = threadIdx.x; i < 2 + P; i += blockDim.x) pq[i] = 0;
   __syncthreads();  // ustart written by this block is visible to it
   const int U = __ldcg(ustart + B);
   for (int p = threadIdx.x; p < P; p += blockDim.x) {
@@ -773,7 +775,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsAThreads, 1)
     tmem_dealloc_cg2(tmem_base, 512);
   }
   // Pass B reads only this pair's outputs: publish the pair as finished (both CTAs are past the
-  // cluster barrier, so their writes are ordered before the release).
+  // cluster barrier, so their writes are ordered before the release). The queue was cleared by a
+  // kernel this one waited for (the unit starts, or the previous layer's merge), and pass B can only
+  // have started after this grid's trigger, which follows its dependency wait.
   if (a.pq != nullptr && leader && threadIdx.x == 0) {
     __threadfence();
     st_release_gpu(a.pq + 2 + atomicAdd(a.pq, 1), pair + 1);
@@ -845,6 +849,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsBThreads, 1)
       mbar_init(&cready[i], 16);
     }
     *abort_flag = 0;
+    // The ticket counter is read without a dependency wait: pass B launches only after pass A's
+    // trigger, which pass A issues after its own wait, so the clear of the queue (a kernel before
+    // pass A) has completed; the atomic is performed at L2, where that completed clear is.
     if (a.pq != nullptr && leader) *ticket = atomicAdd(a.pq + 1, 1);
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -1044,7 +1051,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAbsBThreads, 1)
 __global__ void __launch_bounds__(256) abs_merge_kernel(const AbsArgs a) {
   pdl_wait();
   pdl_trigger();
-  if (a.pq != nullptr && blockIdx.x == 0 && blockIdx.y == 0)  // both passes are complete: reset
+  // Pass B is complete (this kernel waited for it), and with it every pass A pair it acquired, so
+  // every pass A pair has published: the queue can be reset for the next layer's passes.
+  if (a.pq != nullptr && blockIdx.x == 0 && blockIdx.y == 0)
     for (int i = threadIdx.x; i < 2 + a.n_pairs; i += blockDim.x) a.pq[i] = 0;
   __shared__ int s_slot[8][kAbsMaxPairs];
   __shared__ float s_w[8][kAbsMaxPairs];
