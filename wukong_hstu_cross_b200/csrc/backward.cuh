@@ -154,7 +154,7 @@ __device__ __forceinline__ void store8_pair(__nv_bfloat16* hi, __nv_bfloat16* lo
 // colp [gridDim.x, d]: this block's column sums of dn x r (the gain's gradient, summed over the
 // block's rows; a second pass sums the blocks in order).
 template <typename TX, int MAXCH>
-__global__ void __launch_bounds__(256) rms_bwd_kernel(const TX* __restrict__ x, const float* __restrict__ g,
+__global__ void __launch_bounds__(256, MAXCH <= 2 ? 2 : 1) rms_bwd_kernel(const TX* __restrict__ x, const float* __restrict__ g,
                                                       const float* __restrict__ dn, long long rows, int d, float eps,
                                                       const float* __restrict__ resid1, long long ld1,
                                                       const float* __restrict__ resid2, long long ld2,
@@ -174,16 +174,31 @@ __global__ void __launch_bounds__(256) rms_bwd_kernel(const TX* __restrict__ x, 
   for (int i = 0; i < MAXCH; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) cg[i][j] = 0.f;
+  // the gains of this lane's columns, once for all rows
+  float gr[MAXCH][8];
+#pragma unroll
+  for (int i = 0; i < MAXCH; ++i) {
+    const int c8 = lane + 32 * i;
+    if (c8 < nch) load8(g + 8 * c8, gr[i]);
+  }
   const long long per = (rows + gridDim.x - 1) / gridDim.x;
   const long long r0 = (long long)blockIdx.x * per, r1 = min(rows, r0 + per);
   for (long long r = r0 + warp; r < r1; r += 8) {
-    float xv[MAXCH][8], u[MAXCH][8];
+    float xv[MAXCH][8], dv[MAXCH][8], u[MAXCH][8];
     float ss = 0.f, sux = 0.f;
+    // the row of x and of dn in one round of loads
 #pragma unroll
     for (int i = 0; i < MAXCH; ++i) {
       const int c8 = lane + 32 * i;
       if (c8 < nch) {
         load8(x + r * d + 8 * c8, xv[i]);
+        load8(dn + r * d + 8 * c8, dv[i]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < MAXCH; ++i) {
+      const int c8 = lane + 32 * i;
+      if (c8 < nch) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) ss = fmaf(xv[i][j], xv[i][j], ss);
       }
@@ -195,14 +210,11 @@ __global__ void __launch_bounds__(256) rms_bwd_kernel(const TX* __restrict__ x, 
     for (int i = 0; i < MAXCH; ++i) {
       const int c8 = lane + 32 * i;
       if (c8 < nch) {
-        float dv[8], gv[8];
-        load8(dn + r * d + 8 * c8, dv);
-        load8(g + 8 * c8, gv);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          u[i][j] = dv[j] * gv[j];
+          u[i][j] = dv[i][j] * gr[i][j];
           sux = fmaf(u[i][j], xv[i][j], sux);
-          cg[i][j] = fmaf(dv[j], xv[i][j] * rr, cg[i][j]);
+          cg[i][j] = fmaf(dv[i][j], xv[i][j] * rr, cg[i][j]);
         }
       }
     }
@@ -226,10 +238,9 @@ __global__ void __launch_bounds__(256) rms_bwd_kernel(const TX* __restrict__ x, 
         if (dx32) store8(dx32 + r * d + c, v);
         if (dx_hi) store8_pair(dx_hi + r * d + c, dx_lo ? dx_lo + r * d + c : nullptr, v);
         if (n_out || n32) {
-          float gv[8], nv[8];
-          load8(g + c, gv);
+          float nv[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) nv[j] = xv[i][j] * rr * gv[j];
+          for (int j = 0; j < 8; ++j) nv[j] = xv[i][j] * rr * gr[i][j];
           if (n_out) store8_pair(n_out + r * d + c, n_lo ? n_lo + r * d + c : nullptr, nv);
           if (n32) store8(n32 + r * d + c, nv);
         }
