@@ -46,6 +46,7 @@ struct AttnBwdArgs {
   const int* cstart;         // [B+1] first chunk of each example; cstart[B] = number of chunks
   float* dq;                 // [B*N, d] fp32, zero at launch (atomics)
   __nv_bfloat16 *dkv, *dkv_lo;  // [total_L, kvw]: dK in columns [0, d), dV from v_col0 (shared K = V: dK + dV)
+  const float* row_scale;     // [total_L] or null: dK and dV of history row t are stored times row_scale[t]
   int B, N, d, n_heads, kvw, v_col0, shared_kv;
   long long total_L;
   float scale_log2;          // log2(e) / sqrt(d_h)
@@ -365,10 +366,11 @@ __global__ void __launch_bounds__(AttnBwdCfg<DH, NQ>::THREADS, 1) attn_bwd_kerne
         if (row >= k1) continue;
         __nv_bfloat16* dst = a.dkv + row * a.kvw + col;
         __nv_bfloat16* dstl = a.dkv_lo + row * a.kvw + col;
+        const float rs = a.row_scale ? a.row_scale[row] : 1.0f;
 #pragma unroll
         for (int nt = 0; nt < DH / 8; ++nt) {
           uint32_t h, l;
-          split2(acc[nt][2 * hr], acc[nt][2 * hr + 1], h, l);
+          split2(acc[nt][2 * hr] * rs, acc[nt][2 * hr + 1] * rs, h, l);
           *reinterpret_cast<uint32_t*>(dst + 8 * nt + 2 * qd) = h;
           *reinterpret_cast<uint32_t*>(dstl + 8 * nt + 2 * qd) = l;
         }

@@ -153,7 +153,9 @@ __device__ __forceinline__ void store8_pair(__nv_bfloat16* hi, __nv_bfloat16* lo
 // as bf16 (dx_hi, with its residue dx_lo), n = r x g as a bf16 pair (n_out, n_lo) or fp32 (n32).
 // colp [gridDim.x, d]: this block's column sums of dn x r (the gain's gradient, summed over the
 // block's rows; a second pass sums the blocks in order).
-template <typename TX, int MAXCH>
+// PRE: dn is already scaled by the row factor (dn' = r dn, as the history side's backward forms it):
+// dx = dn' g - x r^2/d sum(dn' g x) and the gain's column sums are of dn' x.
+template <typename TX, int MAXCH, bool PRE = false>
 __global__ void __launch_bounds__(256, MAXCH <= 2 ? 2 : 1) rms_bwd_kernel(const TX* __restrict__ x, const float* __restrict__ g,
                                                       const float* __restrict__ dn, long long rows, int d, float eps,
                                                       const float* __restrict__ resid1, long long ld1,
@@ -214,13 +216,14 @@ __global__ void __launch_bounds__(256, MAXCH <= 2 ? 2 : 1) rms_bwd_kernel(const 
         for (int j = 0; j < 8; ++j) {
           u[i][j] = dv[i][j] * gr[i][j];
           sux = fmaf(u[i][j], xv[i][j], sux);
-          cg[i][j] = fmaf(dv[i][j], xv[i][j] * rr, cg[i][j]);
+          cg[i][j] = fmaf(dv[i][j], PRE ? xv[i][j] : xv[i][j] * rr, cg[i][j]);
         }
       }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sux += __shfl_xor_sync(0xffffffffu, sux, o);
-    const float k = rr * rr * rr / (float)d * sux;
+    const float k = (PRE ? rr * rr : rr * rr * rr) / (float)d * sux;
+    const float ru = PRE ? 1.0f : rr;
 #pragma unroll
     for (int i = 0; i < MAXCH; ++i) {
       const int c8 = lane + 32 * i;
@@ -231,7 +234,7 @@ __global__ void __launch_bounds__(256, MAXCH <= 2 ? 2 : 1) rms_bwd_kernel(const 
         if (resid2) load8(resid2 + r * ld2 + c, r2v);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          v[j] = rr * u[i][j] - xv[i][j] * k;
+          v[j] = ru * u[i][j] - xv[i][j] * k;
           if (resid1) v[j] += r1v[j];
           if (resid2) v[j] += r2v[j];
         }
@@ -530,6 +533,35 @@ __global__ void __launch_bounds__(256) attn_bwd_f32_kernel(const float* __restri
   for (int i = threadIdx.x; i < N * DH; i += blockDim.x) {
     const int n = i / DH, c = i % DH;
     dq[((long long)b * N + n) * d + hc + c] = dqs[i];
+  }
+}
+
+// hi/lo pair of W diag(g): w [rows, cols] bf16, g [cols] fp32 (the history-side projection weights
+// with the states' RMSNorm gain, for the backward's recompute).
+__global__ void scale_cols_pair_kernel(const __nv_bfloat16* __restrict__ w, const float* __restrict__ g,
+                                       long long rows, int cols, __nv_bfloat16* __restrict__ hi,
+                                       __nv_bfloat16* __restrict__ lo) {
+  pdl_wait();
+  pdl_trigger();
+  const long long n = rows * cols;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const float v = __bfloat162float(w[i]) * g[i % cols];
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    hi[i] = h;
+    lo[i] = __float2bfloat16_rn(v - __bfloat162float(h));
+  }
+}
+
+// c[r, col] *= g[col] for a row-major fp32 [rows, cols] matrix (row stride ld).
+__global__ void scale_cols_kernel(float* __restrict__ c, long long ld, const float* __restrict__ g, long long rows,
+                                  int cols) {
+  pdl_wait();
+  pdl_trigger();
+  const long long n = rows * cols;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const long long r = i / cols;
+    const int col = (int)(i - r * cols);
+    c[r * ld + col] *= g[col];
   }
 }
 

@@ -72,6 +72,8 @@ struct GemmArgs {
   // out32 + s * split_stride (a later pass sums the partials in split order).
   int ksplit, kb_split;
   long long split_stride;
+  // ROWNORM: the row factors r are also written here (by the tiles of the first output columns; may be null).
+  float* rows_r;
 };
 
 
@@ -227,6 +229,8 @@ constexpr uint32_t kIdescAMnMajor = 1u << 15;
 // SPLIT_B: B is a hi/lo pair too (single A source: tmA1 then holds B's lo half), and every k-step
 // issues A_hi B_hi, A_lo B_hi and A_hi B_lo (the A_lo B_lo term is below 2^-16 of the product):
 // the weight gradients of the token side, whose sums over rows cancel, need both operands at ~16 bits.
+// With an exact bf16 A (SPLIT off) it issues A B_hi and A B_lo: the backward's recompute of the
+// history-side projection multiplies the raw states by W diag(g) carried as a pair.
 //
 // KPS = 2: each stage carries two K blocks, loaded with 3-D tensor maps (the view {64 columns, rows,
 // K / 64 blocks} of each K-major operand, box {64, rows, 2}), so a stage costs three copies instead of
@@ -241,7 +245,6 @@ __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
   constexpr int STAGES = L::STAGES;
   constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators: 128, 256 or 512 columns
   static_assert(!(ROWNORM && A_MN), "row statistics read K-major A rows");
-  static_assert(!(ROWNORM && SPLIT_B), "row-normalised GEMMs have one B");
   static_assert(KPS == 1 || (KPS == 2 && !A_MN && !B_MN && !SPLIT_B), "two-block stages: K-major operands");
   static_assert(STAGES >= 2, "pipeline depth");
   constexpr uint32_t MN_BOX = 64 * 64 * 2;  // one MN-major box: 64 K rows x 64 elements
@@ -479,6 +482,7 @@ __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
       if (ROWNORM && !mbar_wait(&nfull[acc], ua & 1, abort_flag)) break;
       tc_fence_after();
       const float r = ROWNORM ? rbuf[acc * 128 + row] : 1.0f;
+      if (ROWNORM && args.rows_r && n0 == 0 && row_ok) args.rows_r[gm] = r;
       epi_tile<BN, EPI>(args, tmem_base + acc * BN + ((uint32_t)(q * 32) << 16), r, gm, row_ok, n0, pre,
                         nsplit > 1 ? split * args.split_stride : 0ll);
       // this accumulator buffer and its row factors may be reused

@@ -1340,10 +1340,42 @@ inline int rows_blocks(long long rows) {
   return (int)std::max<long long>(1, std::min<long long>(cdiv<long long>(rows, 32), kColpBlocks));
 }
 
+// out = r(x) (x W^T) as a bf16 pair, W given as a pair (w_hi + w_lo, [N, K] K-major), x bf16 [M, K]
+// (row stride K); r = 1/sqrt(mean(x^2) + eps) per row, also written to rows_r. Two MMAs per k-step.
+whale_status gemm_rownorm_wpair(const void* x, long long M, int K, const void* w_hi, const void* w_lo, int N,
+                                void* out_hi, void* out_lo, float* rows_r, float eps, cudaStream_t st) {
+  if (M <= 0) return WHALE_OK;
+  if (M >= (1ll << 31) || K % 64 || N % 64) return WHALE_ERR_UNSUPPORTED;
+  const int bn = N % 256 == 0 ? 256 : (N % 128 == 0 ? 128 : 64);
+  CUtensorMap maps[5];
+  WCHECK(tmap_bf16(&maps[0], x, M, K, K, 128));
+  maps[1] = maps[0];
+  WCHECK(tmap_bf16(&maps[2], w_lo, N, K, K, bn));  // B's lo half rides in the A1 slot
+  maps[3] = maps[2];
+  WCHECK(tmap_bf16(&maps[4], w_hi, N, K, K, bn));
+  GemmArgs g{};
+  g.M = (int)M;
+  g.N = N;
+  g.kb0 = K / 64;
+  g.kb1 = 0;
+  g.tiles_n = N / bn;
+  const long long tiles = cdiv<long long>(M, 128) * g.tiles_n;
+  g.num_tiles = (int)tiles;
+  g.inv_k = 1.0f / (float)K;
+  g.eps = eps;
+  g.out_hi = static_cast<__nv_bfloat16*>(out_hi);
+  g.out_lo = static_cast<__nv_bfloat16*>(out_lo);
+  g.ldo = N;
+  g.rows_r = rows_r;
+  if (bn == 256) return launch_gemm_t<256, EPI_STORE, true, false, false, false, true>(maps, g, tiles, st);
+  if (bn == 128) return launch_gemm_t<128, EPI_STORE, true, false, false, false, true>(maps, g, tiles, st);
+  return launch_gemm_t<64, EPI_STORE, true, false, false, false, true>(maps, g, tiles, st);
+}
+
 struct BwdBufs {
   // forward recompute
-  void *x32, *xlo, *r, *q, *q_lo, *sn, *sn_lo, *kv, *kv_lo, *attn, *a, *a_lo, *lse, *z1, *g, *g_lo, *f32, *f, *f_lo,
-      *ug;
+  void *x32, *xlo, *r, *q, *q_lo, *sn, *wg, *wg_lo, *rkv, *kv, *kv_lo, *attn, *a, *a_lo, *lse, *z1, *g, *g_lo, *f32,
+      *f, *f_lo, *ug;
   // backward
   void *dy, *dy_lo, *dm, *msw, *msw_lo, *dug, *dug_lo, *dn, *nrm, *nrm_lo, *nq, *nq_lo, *df32, *df, *df_lo, *dhid,
       *dz, *dz_lo, *dc, *da16, *da_lo, *delta, *dq, *dq_hi, *dq_lo, *cst, *dkv, *dkv_lo, *dsn, *colp, *part;
@@ -1372,11 +1404,14 @@ size_t bwd_buffers(const Shape& s, const whale_shape_hint& h, char* base, BwdBuf
   }
   b->q = take(rows * d * e);
   b->kv = take(T * kvw * e);
-  b->sn = take(T * d * e);
   if (s.bf16) {
     b->q_lo = take(rows * d * 2);
     b->kv_lo = take(T * kvw * 2);
-    b->sn_lo = take(T * d * 2);
+    b->wg = take(kvw * d * 2);  // W_kv diag(g_kv) as a pair
+    b->wg_lo = take(kvw * d * 2);
+    b->rkv = take(T * 4);       // the history rows' RMSNorm factors
+  } else {
+    b->sn = take(T * d * 4);
   }
   b->a = take(rows * d * e);
   if (s.bf16) b->a_lo = take(rows * d * 2);
@@ -1446,7 +1481,8 @@ whale_status gain_grad(const float* colp, int blocks, int d, float* dg, cudaStre
 template <typename TX>
 whale_status rms_bwd(const TX* x, const float* g, const float* dn, long long rows, int d, float eps,
                      const float* r1, long long ld1, const float* r2, long long ld2, float* dx32, void* dx_hi,
-                     void* dx_lo, void* n_out, void* n_lo, float* n32, float* colp, float* dg, cudaStream_t st) {
+                     void* dx_lo, void* n_out, void* n_lo, float* n32, float* colp, float* dg, cudaStream_t st,
+                     bool pre = false) {
   if (rows <= 0) {
     if (dg) CUCHECK(cudaMemsetAsync(dg, 0, (size_t)d * 4, st));
     return WHALE_OK;
@@ -1457,9 +1493,15 @@ whale_status rms_bwd(const TX* x, const float* g, const float* dn, long long row
                       static_cast<__nv_bfloat16*>(dx_hi), static_cast<__nv_bfloat16*>(dx_lo),
                       static_cast<__nv_bfloat16*>(n_out), static_cast<__nv_bfloat16*>(n_lo), n32, colp);
   };
-  if (d <= 256) WCHECK(go(rms_bwd_kernel<TX, 1>));
-  else if (d <= 512) WCHECK(go(rms_bwd_kernel<TX, 2>));
-  else WCHECK(go(rms_bwd_kernel<TX, 4>));
+  if (pre) {
+    if (d <= 256) WCHECK(go(rms_bwd_kernel<TX, 1, true>));
+    else if (d <= 512) WCHECK(go(rms_bwd_kernel<TX, 2, true>));
+    else WCHECK(go(rms_bwd_kernel<TX, 4, true>));
+  } else {
+    if (d <= 256) WCHECK(go(rms_bwd_kernel<TX, 1>));
+    else if (d <= 512) WCHECK(go(rms_bwd_kernel<TX, 2>));
+    else WCHECK(go(rms_bwd_kernel<TX, 4>));
+  }
   return gain_grad(colp, blocks, d, dg, st);
 }
 
@@ -1507,13 +1549,13 @@ whale_status recompute_bf16(const Shape& s, const Stream3& in, const void* slab,
                     static_cast<bf*>(b.nq), static_cast<bf*>(b.nq_lo), (float*)nullptr));
   WCHECK(gemm_bf16(opnd(b.nq, b.nq_lo, d, d), no_opnd(), w.w_q, d, Outs{b.q, b.q_lo, nullptr, d}, nullptr, 0, rows,
                    EPI_STORE, false, 0.f, st));
-  // History side the same way: K|V = (r s g) W_kv^T from the normalised states as a pair, written as a
-  // pair (the attention backward reads both halves; the forward attention below reads hi).
+  // History side: K|V = r (s (W_kv diag(g))^T) with the raw states s (exact bf16) times W_kv diag(g) as
+  // a pair, the row factor r in the epilogue (and kept for the backward), written as a pair (the
+  // attention backward reads both halves; the forward attention below reads hi).
   if (T > 0) {
-    WCHECK(launch_pdl(rms_rows_kernel<bf>, dim3(rows_blocks(T)), dim3(256), 0, st, static_cast<const bf*>(slab),
-                      w.g_kv, T, d, s.eps, static_cast<bf*>(b.sn), static_cast<bf*>(b.sn_lo), (float*)nullptr));
-    WCHECK(gemm_bf16(opnd(b.sn, b.sn_lo, d, d), no_opnd(), w.w_kv, kvw, Outs{b.kv, b.kv_lo, nullptr, kvw}, nullptr, 0,
-                     T, EPI_STORE, false, 0.f, st));
+    WCHECK(ew_launch(scale_cols_pair_kernel, (long long)kvw * d, st, static_cast<const bf*>(w.w_kv), w.g_kv,
+                     (long long)kvw, d, static_cast<bf*>(b.wg), static_cast<bf*>(b.wg_lo)));
+    WCHECK(gemm_rownorm_wpair(slab, T, d, b.wg, b.wg_lo, kvw, b.kv, b.kv_lo, F(b.rkv), s.eps, st));
   }
   WCHECK(attention_bf16(s, b.q, b.kv, offsets, b.a, b.a_lo, h.B, T, b.attn, st, F(b.lse)));
   const Opnd A = opnd(b.a, b.a_lo, d, d);
@@ -1610,6 +1652,7 @@ whale_status layer_backward_bf16(const Shape& s, const Stream3& in, const void* 
     aa.cstart = static_cast<const int*>(b.cst);
     aa.dq = F(b.dq);
     aa.dkv = static_cast<bf*>(b.dkv);
+    aa.row_scale = F(b.rkv);  // dK|V' = r dK|V: what both history-side products below contract with
     aa.B = h.B;
     aa.N = s.N;
     aa.d = d;
@@ -1633,11 +1676,15 @@ whale_status layer_backward_bf16(const Shape& s, const Stream3& in, const void* 
   WCHECK(rms_bwd<float>(x32, w.g_q, F(b.dn), rows, d, s.eps, F(b.df32), d, F(b.dc) + d, 2 * d, dx, nullptr, nullptr,
                         nullptr, nullptr, nullptr, F(b.colp), gr.g_q, st));
   // ---- S2 backward: K|V projection and the states' RMSNorm ----
+  // With dK|V' = r dK|V (rows scaled by the attention backward): dsn' = dK|V' W_kv = r dsn feeds the
+  // RMSNorm backward in its prescaled form, and dW_kv = dK|V^T (r s g) = (dK|V'^T s) diag(g) contracts
+  // with the raw states (exact bf16: two MMAs per k-step instead of three with a normalised pair).
   if (T > 0) {
     WCHECK(gemm_acc32(b.dkv, b.dkv_lo, kvw, false, w.w_kv, d, true, T, d, kvw, F(b.dsn), d, part, pc, st));
     WCHECK(rms_bwd<bf>(static_cast<const bf*>(slab), w.g_kv, F(b.dsn), T, d, s.eps, nullptr, 0, nullptr, 0, nullptr, ds,
-                       nullptr, nullptr, nullptr, nullptr, F(b.colp), gr.g_kv, st));
-    WCHECK(gemm_acc32(b.dkv, b.dkv_lo, kvw, true, b.sn, d, true, kvw, d, T, gr.w_kv, d, part, pc, st, b.sn_lo));
+                       nullptr, nullptr, nullptr, nullptr, F(b.colp), gr.g_kv, st, true));
+    WCHECK(gemm_acc32(b.dkv, b.dkv_lo, kvw, true, slab, d, true, kvw, d, T, gr.w_kv, d, part, pc, st));
+    WCHECK(ew_launch(scale_cols_kernel, (long long)kvw * d, st, gr.w_kv, (long long)d, w.g_kv, (long long)kvw, d));
   } else {
     CUCHECK(cudaMemsetAsync(gr.g_kv, 0, (size_t)d * 4, st));
     CUCHECK(cudaMemsetAsync(gr.w_kv, 0, (size_t)kvw * d * 4, st));
