@@ -79,7 +79,7 @@ struct GemmArgs {
 
 // A pipeline stage holds KPS consecutive 64-column K blocks: [A hi: KPS blocks][A lo: KPS blocks]
 // [W: KPS blocks][W lo: KPS blocks], each block a 128-byte-swizzled [rows][64] tile.
-template <int BN, bool SPLIT, bool SPLIT_B = false, int KPS = 1>
+template <int BN, bool SPLIT, bool SPLIT_B = false, int KPS = 1, bool TST = false>
 struct GemmSmem {
   static constexpr int BM = 128, BK = 64;
   static constexpr uint32_t A_BYTES = BM * BK * 2;  // one K block of A (hi or lo)
@@ -88,7 +88,9 @@ struct GemmSmem {
   static constexpr uint32_t STAGE_BYTES = A_ALL + (SPLIT_B ? 2 : 1) * KPS * B_BYTES;
   // stages fill what the 227 KB of shared memory leaves (one CTA per SM either way): five 40 KB
   // stages for the 64-column hi/lo tiles, two 80 KB ones when a stage holds two K blocks
-  static constexpr int FIXED = 1024 /*alignment slack*/ + 2 * 128 * 4 /*row factors*/ + 256 /*barriers*/;
+  // TST: the epilogue's staging buffers for tensor stores, 8 KB per epilogue warp (after the stages)
+  static constexpr int STG_BYTES = TST ? 4 * 8192 : 0;
+  static constexpr int FIXED = 1024 /*alignment slack*/ + STG_BYTES + 2 * 128 * 4 /*row factors*/ + 256 /*barriers*/;
   static constexpr int STAGES =
       ((232448 - FIXED) / (int)STAGE_BYTES) > 8 ? 8 : ((232448 - FIXED) / (int)STAGE_BYTES);
   static constexpr size_t BYTES = FIXED + STAGES * (size_t)STAGE_BYTES;
@@ -223,6 +225,112 @@ __device__ __forceinline__ void epi_tile(const GemmArgs& args, uint32_t t_row, f
   }
 }
 
+// The epilogue through shared memory (TST): each 32-column chunk of the warp's 32 rows is staged in
+// the warp's 8 KB buffer (fp32: 128-byte rows, 128-byte swizzle; bf16 hi and lo: 64-byte rows,
+// 64-byte swizzle) and written by one lane with tensor stores: whole lines per copy, where direct
+// stores write 32 rows' 16-byte pieces per instruction. Rows past M are clipped by the tensor maps.
+struct EpiStage {
+  uint8_t* buf;
+  const CUtensorMap *o32, *ohi, *olo;
+  int orow;   // first output row of this warp
+  int split;  // split-K range of the tile (the fp32 output's third coordinate)
+  int lane;
+};
+
+template <int BN, int EPI>
+__device__ __forceinline__ void epi_tile_tma(const GemmArgs& args, uint32_t t_row, float r, long long gm, bool row_ok,
+                                             int n0, const float4 (&pre)[EpiPre<BN, EPI>::kN], const EpiStage& es) {
+  constexpr bool kPre = EpiPre<BN, EPI>::kOn;
+  const int lane = es.lane;
+  uint8_t* s32 = es.buf;
+  uint8_t* shi = es.buf + 4096;
+  uint8_t* slo = es.buf + 6144;
+  // stage 32 values of this lane's row (all lanes) and store them at output column ocol
+  auto emit = [&](const float (&x)[32], int ocol) {
+    if (lane == 0) bulk_wait_read<0>();  // the previous chunk's stores have read the buffer
+    __syncwarp();
+    if (args.out32) {
+      uint4* d = reinterpret_cast<uint4*>(s32 + lane * 128);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        d[j ^ (lane & 7)] = make_uint4(__float_as_uint(x[4 * j]), __float_as_uint(x[4 * j + 1]),
+                                       __float_as_uint(x[4 * j + 2]), __float_as_uint(x[4 * j + 3]));
+    }
+    if (args.out_hi) {
+      uint32_t hi[16], lo[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * j], x[2 * j + 1]);
+        hi[j] = *reinterpret_cast<const uint32_t*>(&h);
+        const float2 hf = __bfloat1622float2(h);
+        lo[j] = pack_bf16x2(x[2 * j] - hf.x, x[2 * j + 1] - hf.y);
+      }
+      uint4* dh = reinterpret_cast<uint4*>(shi + lane * 64);
+      uint4* dl = reinterpret_cast<uint4*>(slo + lane * 64);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        dh[j ^ ((lane >> 1) & 3)] = make_uint4(hi[4 * j], hi[4 * j + 1], hi[4 * j + 2], hi[4 * j + 3]);
+        if (args.out_lo) dl[j ^ ((lane >> 1) & 3)] = make_uint4(lo[4 * j], lo[4 * j + 1], lo[4 * j + 2], lo[4 * j + 3]);
+      }
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      if (args.out32) tma_store_3d(es.o32, s32, ocol, es.orow, es.split);
+      if (args.out_hi) tma_store_2d(es.ohi, shi, ocol, es.orow);
+      if (args.out_hi && args.out_lo) tma_store_2d(es.olo, slo, ocol, es.orow);
+      bulk_commit();
+    }
+  };
+  // the 32 values of accumulator chunk c (all epilogues but SwiGLU)
+  auto values = [&](const int c, const uint32_t (&v)[32], float (&x)[32]) {
+    const int col = n0 + c * 32;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(v[j]) * r;
+    if (EPI == EPI_RESID) {
+      if (row_ok) {
+        const float4* rp = reinterpret_cast<const float4*>(args.resid32 + gm * args.ldr + col);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float4 t = kPre ? pre[(c * 8 + i) % EpiPre<BN, EPI>::kN] : rp[i];
+          x[4 * i] += t.x;
+          x[4 * i + 1] += t.y;
+          x[4 * i + 2] += t.z;
+          x[4 * i + 3] += t.w;
+        }
+      }
+    } else if (EPI == EPI_SILU) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) x[j] = silu_f(x[j]);
+    } else if (EPI == EPI_SWIGLU_TIED) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) x[j] = silu_f(x[j]) * x[j];
+    }
+  };
+#pragma unroll (kPre ? BN / 64 : 1)
+  for (int c = 0; c < BN / 32; c += 2) {
+    uint32_t va[32], vb[32];
+    tmem_ld_32x32b_x32(t_row + c * 32, va);
+    tmem_ld_32x32b_x32(t_row + (c + 1) * 32, vb);
+    tmem_ld_wait();
+    if (EPI == EPI_SWIGLU) {  // 16 up and 16 gate columns per chunk: the pair gives 32 outputs
+      float h[32];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        h[j] = silu_f(__uint_as_float(va[16 + j]) * r) * (__uint_as_float(va[j]) * r);
+        h[16 + j] = silu_f(__uint_as_float(vb[16 + j]) * r) * (__uint_as_float(vb[j]) * r);
+      }
+      emit(h, (n0 + c * 32) / 2);
+    } else {
+      float x[32];
+      values(c, va, x);
+      emit(x, n0 + c * 32);
+      values(c + 1, vb, x);
+      emit(x, n0 + (c + 1) * 32);
+    }
+  }
+}
+
 // Instruction-descriptor bit selecting an MN-major A operand.
 constexpr uint32_t kIdescAMnMajor = 1u << 15;
 
@@ -235,13 +343,20 @@ constexpr uint32_t kIdescAMnMajor = 1u << 15;
 // KPS = 2: each stage carries two K blocks, loaded with 3-D tensor maps (the view {64 columns, rows,
 // K / 64 blocks} of each K-major operand, box {64, rows, 2}), so a stage costs three copies instead of
 // six. The K blocks of every tile, of A0 and of each split-K range are then even in number.
+//
+// TST: the epilogue writes through shared memory with tensor stores (maps tmO32, tmOhi, tmOlo over
+// the fp32 output {columns, rows, split} and the bf16 hi and lo outputs, boxes of 32 x 32); the QABS
+// row scatter keeps direct stores.
 template <int BN, int EPI, bool ROWNORM, bool SPLIT, bool A_MN = false, bool B_MN = false, bool SPLIT_B = false,
-          int KPS = 1>
+          int KPS = 1, bool TST = false>
 __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA0lo,
                    const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmA1lo,
-                   const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
-  using L = GemmSmem<BN, SPLIT, SPLIT_B, KPS>;
+                   const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmO32,
+                   const __grid_constant__ CUtensorMap tmOhi, const __grid_constant__ CUtensorMap tmOlo,
+                   const GemmArgs args) {
+  using L = GemmSmem<BN, SPLIT, SPLIT_B, KPS, TST>;
+  static_assert(!(TST && EPI == EPI_QABS), "the per-head row scatter stores directly");
   constexpr int STAGES = L::STAGES;
   constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators: 128, 256 or 512 columns
   static_assert(!(ROWNORM && A_MN), "row statistics read K-major A rows");
@@ -250,8 +365,9 @@ __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
   constexpr uint32_t MN_BOX = 64 * 64 * 2;  // one MN-major box: 64 K rows x 64 elements
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  // stage s: [A hi | A lo (SPLIT) | W]; then row factors [2][128]; then barriers
-  float* rbuf = reinterpret_cast<float*>(smem + STAGES * L::STAGE_BYTES);
+  // stage s: [A hi | A lo (SPLIT) | W]; then the epilogue staging (TST); row factors [2][128]; barriers
+  uint8_t* stg = smem + STAGES * L::STAGE_BYTES;
+  float* rbuf = reinterpret_cast<float*>(stg + L::STG_BYTES);
   uint64_t* full = reinterpret_cast<uint64_t*>(rbuf + 2 * 128);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;  // [2] accumulator ready (MMA commit)
@@ -483,8 +599,14 @@ __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
       tc_fence_after();
       const float r = ROWNORM ? rbuf[acc * 128 + row] : 1.0f;
       if (ROWNORM && args.rows_r && n0 == 0 && row_ok) args.rows_r[gm] = r;
-      epi_tile<BN, EPI>(args, tmem_base + acc * BN + ((uint32_t)(q * 32) << 16), r, gm, row_ok, n0, pre,
-                        nsplit > 1 ? split * args.split_stride : 0ll);
+      if constexpr (TST) {
+        const int orow = m0 + q * 32;
+        const EpiStage es{stg + (warp - 2) * 8192, &tmO32, &tmOhi, &tmOlo, orow, nsplit > 1 ? split : 0, lane};
+        epi_tile_tma<BN, EPI>(args, tmem_base + acc * BN + ((uint32_t)(q * 32) << 16), r, gm, row_ok, n0, pre, es);
+      } else {
+        epi_tile<BN, EPI>(args, tmem_base + acc * BN + ((uint32_t)(q * 32) << 16), r, gm, row_ok, n0, pre,
+                          nsplit > 1 ? split * args.split_stride : 0ll);
+      }
       // this accumulator buffer and its row factors may be reused
       tc_fence_before();
       __syncwarp();
@@ -493,6 +615,7 @@ __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
         mbar_arrive(&edone[acc]);
       }
     }
+    if (TST && lane == 0) bulk_wait<0>();  // this warp's tensor stores are complete before the CTA exits
   }
 
   tc_fence_before();

@@ -202,6 +202,35 @@ whale_status tmap_bf16_kblocks(CUtensorMap* tm, const void* base, long long rows
   return r == CUDA_SUCCESS ? WHALE_OK : WHALE_ERR_CUDA;
 }
 
+// fp32 splits x [rows, cols] row-major (row stride ld, split stride rows * ld) as {cols, rows, splits}
+// with a box of 32 x 32 x 1 (128-byte rows, 128-byte swizzle): the GEMM epilogue's tensor stores,
+// which clip rows past `rows` within each split.
+whale_status tmap_f32_32(CUtensorMap* tm, const void* base, long long rows, long long cols, long long ld,
+                         long long splits) {
+  WCHECK(get_encoder());
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || (ld * 4) % 16 || rows <= 0 || cols <= 0 || splits <= 0)
+    return WHALE_ERR_INVALID_ARG;
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)splits};
+  cuuint64_t strides[2] = {(cuuint64_t)(ld * 4), (cuuint64_t)(rows * ld * 4)};
+  cuuint32_t box[3] = {32u, 32u, 1u};
+  cuuint32_t es[3] = {1u, 1u, 1u};
+  CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? WHALE_OK : WHALE_ERR_CUDA;
+}
+
+// The epilogue's store maps o[0..2] (fp32, bf16 hi, bf16 lo) over the GEMM's outputs: cols output
+// columns (N, or N / 2 for the SwiGLU epilogue), M rows; the fp32 output holds `splits` split-K
+// partials of M rows each. A missing output gets a copy of `any` (never stored through).
+whale_status epi_maps(CUtensorMap* o, const GemmArgs& g, long long cols, long long splits, const CUtensorMap& any) {
+  o[0] = o[1] = o[2] = any;
+  if (g.out32) WCHECK(tmap_f32_32(&o[0], g.out32, g.M, cols, g.ldo, splits));
+  if (g.out_hi) WCHECK(tmap_bf16_box(&o[1], g.out_hi, g.M, cols, g.ldo, 32, 32));
+  if (g.out_lo) WCHECK(tmap_bf16_box(&o[2], g.out_lo, g.M, cols, g.ldo, 32, 32));
+  return WHALE_OK;
+}
+
 // A K-major operand's map for stages of kps K blocks (kps 1: the 2-D map).
 whale_status tmap_operand(CUtensorMap* tm, const void* base, long long rows, long long K, long long ld, int box_rows,
                           int kps) {
@@ -406,17 +435,19 @@ struct Outs {
   long long ld;
 };
 
+// tm: the operand maps [A0, A0 lo, A1, A1 lo, W] and, for TST, the store maps [fp32, hi, lo] (eight).
 template <int BN, int EPI, bool RN, bool SPLIT, bool A_MN = false, bool B_MN = false, bool SPLIT_B = false,
-          int KPS = 1>
+          int KPS = 1, bool TST = true>
 whale_status launch_gemm_t(const CUtensorMap* tm, const GemmArgs& g, long long tiles, cudaStream_t st) {
-  if constexpr (GemmSmem<BN, SPLIT, SPLIT_B, KPS>::STAGES < 2) {
+  if constexpr (GemmSmem<BN, SPLIT, SPLIT_B, KPS, TST>::STAGES < 2) {
     return WHALE_ERR_UNSUPPORTED;  // two stages of this tile do not fit in shared memory
   } else {
-    const size_t smem = GemmSmem<BN, SPLIT, SPLIT_B, KPS>::BYTES;
-    auto kern = gemm_tc_kernel<BN, EPI, RN, SPLIT, A_MN, B_MN, SPLIT_B, KPS>;
+    const size_t smem = GemmSmem<BN, SPLIT, SPLIT_B, KPS, TST>::BYTES;
+    auto kern = gemm_tc_kernel<BN, EPI, RN, SPLIT, A_MN, B_MN, SPLIT_B, KPS, TST>;
     CUCHECK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     const unsigned grid = (unsigned)(tiles < kNumSM ? tiles : kNumSM);
-    return launch_pdl(kern, dim3(grid), dim3(gemm_threads<RN>()), smem, st, tm[0], tm[1], tm[2], tm[3], tm[4], g);
+    return launch_pdl(kern, dim3(grid), dim3(gemm_threads<RN>()), smem, st, tm[0], tm[1], tm[2], tm[3], tm[4], tm[5],
+                      tm[6], tm[7], g);
   }
 }
 
@@ -453,7 +484,7 @@ inline double gemm_stage_cycles(int bn, bool split, int kps) {
 // Shared memory of a tile configuration holds at least two stages.
 template <int BN>
 bool gemm_kps2_fits(bool split) {
-  return split ? GemmSmem<BN, true, false, 2>::STAGES >= 2 : GemmSmem<BN, false, false, 2>::STAGES >= 2;
+  return split ? GemmSmem<BN, true, false, 2, true>::STAGES >= 2 : GemmSmem<BN, false, false, 2, true>::STAGES >= 2;
 }
 
 // Co-resident 2-CTA clusters of the 2-SM GEMM on the current device (cached per device).
@@ -544,7 +575,7 @@ whale_status gemm_bf16(const Opnd& a0, const Opnd& a1, const void* W, int N, con
         bn = cand;
         kps = kc;
       }
-  CUtensorMap maps[5];
+  CUtensorMap maps[8];
   WCHECK(tmap_operand(&maps[0], a0.hi, M, a0.K, a0.ld, 128, kps));
   if (split) WCHECK(tmap_operand(&maps[1], a0.lo, M, a0.K, a0.ld, 128, kps));
   else maps[1] = maps[0];
@@ -572,6 +603,7 @@ whale_status gemm_bf16(const Opnd& a0, const Opnd& a1, const void* W, int N, con
   g.ldo = out.ld;
   g.resid32 = resid32;
   g.ldr = ldr;
+  WCHECK(epi_maps(maps + 5, g, epi == EPI_SWIGLU ? N / 2 : N, 1, maps[0]));
   const long long tiles = tm * g.tiles_n;
   if (kps == 2) {
     if (bn == 256) return launch_gemm_bn<256, 2>(epi, rn, split, maps, g, tiles, st);
@@ -649,7 +681,7 @@ whale_status gemm_acc32(const void* a_hi, const void* a_lo, long long lda, bool 
   const long long tiles_mn = tm * (N / bn);
   int kb_split = (int)cdiv<long long>(KB, ks);
   ks = (int)cdiv<long long>(KB, kb_split);  // no empty split
-  CUtensorMap maps[5];
+  CUtensorMap maps[8];
   if (a_mn) {
     WCHECK(tmap_bf16_box(&maps[0], a_hi, K, M, lda, 64, 64));
     if (split) WCHECK(tmap_bf16_box(&maps[1], a_lo, K, M, lda, 64, 64));
@@ -685,6 +717,7 @@ whale_status gemm_acc32(const void* a_hi, const void* a_lo, long long lda, bool 
     g.out32 = c;
     g.ldo = ldc;
   }
+  WCHECK(epi_maps(maps + 5, g, N, ks, maps[0]));
   const long long tiles = tiles_mn * ks;
   whale_status r;
   if (bn == 256) r = launch_acc32_bn<256>(split, split_b, a_mn, b_mn, maps, g, tiles, st);
@@ -917,9 +950,9 @@ whale_status abs_max_pairs(int E, int* pairs) {
 whale_status gemm_qabs(const Shape& s, const void* q, const void* wkabs, void* qa, long long rows, cudaStream_t st) {
   constexpr int BN = 256;
   if (s.d % BN || s.dh != 64) return WHALE_ERR_UNSUPPORTED;
-  CUtensorMap maps[5];
+  CUtensorMap maps[8];
   WCHECK(tmap_bf16(&maps[0], q, rows, s.d, s.d, 128));
-  maps[1] = maps[2] = maps[3] = maps[0];
+  maps[1] = maps[2] = maps[3] = maps[5] = maps[6] = maps[7] = maps[0];
   WCHECK(tmap_bf16(&maps[4], wkabs, (long long)s.h * s.d, s.dh, s.dh, BN));
   GemmArgs g{};
   g.M = (int)rows;
@@ -937,7 +970,7 @@ whale_status gemm_qabs(const Shape& s, const void* q, const void* wkabs, void* q
   g.qabs_N = s.N;
   g.qabs_d = s.d;
   g.qabs_rows = kAbsQ;
-  return launch_gemm_t<BN, EPI_QABS, false, false>(maps, g, tiles, st);
+  return launch_gemm_t<BN, EPI_QABS, false, false, false, false, false, 1, false>(maps, g, tiles, st);
 }
 
 // A[:, j*64 : j*64 + 64] = z_j W'_V,j^T for every head j in one launch: z is the stack [h, rows, d]
@@ -946,7 +979,7 @@ whale_status gemm_vabs(const Shape& s, const void* zh, const void* wv, void* a, 
                        cudaStream_t st) {
   if (s.dh != 64) return WHALE_ERR_UNSUPPORTED;
   const int kps = (s.d / 64) % 2 == 0 ? 2 : 1;
-  CUtensorMap maps[5];
+  CUtensorMap maps[8];
   WCHECK(tmap_operand(&maps[0], zh, (long long)s.h * rows, s.d, s.d, 128, kps));
   maps[1] = maps[2] = maps[3] = maps[0];
   WCHECK(tmap_operand(&maps[4], wv, s.d, s.d, s.d, 64, kps));
@@ -964,6 +997,7 @@ whale_status gemm_vabs(const Shape& s, const void* zh, const void* wv, void* a, 
   g.head_tiles = 1;
   g.a_kb_step = 0;
   g.a_row_step = rows;
+  WCHECK(epi_maps(maps + 5, g, s.d, 1, maps[0]));
   if (kps == 2) return launch_gemm_t<64, EPI_STORE, false, false, false, false, false, 2>(maps, g, tiles, st);
   return launch_gemm_t<64, EPI_STORE, false, false>(maps, g, tiles, st);
 }
@@ -1347,7 +1381,7 @@ whale_status gemm_rownorm_wpair(const void* x, long long M, int K, const void* w
   if (M <= 0) return WHALE_OK;
   if (M >= (1ll << 31) || K % 64 || N % 64) return WHALE_ERR_UNSUPPORTED;
   const int bn = N % 256 == 0 ? 256 : (N % 128 == 0 ? 128 : 64);
-  CUtensorMap maps[5];
+  CUtensorMap maps[8];
   WCHECK(tmap_bf16(&maps[0], x, M, K, K, 128));
   maps[1] = maps[0];
   WCHECK(tmap_bf16(&maps[2], w_lo, N, K, K, bn));  // B's lo half rides in the A1 slot
@@ -1367,6 +1401,7 @@ whale_status gemm_rownorm_wpair(const void* x, long long M, int K, const void* w
   g.out_lo = static_cast<__nv_bfloat16*>(out_lo);
   g.ldo = N;
   g.rows_r = rows_r;
+  WCHECK(epi_maps(maps + 5, g, N, 1, maps[0]));
   if (bn == 256) return launch_gemm_t<256, EPI_STORE, true, false, false, false, true>(maps, g, tiles, st);
   if (bn == 128) return launch_gemm_t<128, EPI_STORE, true, false, false, false, true>(maps, g, tiles, st);
   return launch_gemm_t<64, EPI_STORE, true, false, false, false, true>(maps, g, tiles, st);
