@@ -246,7 +246,7 @@ __device__ __forceinline__ void epi_tile_tma(const GemmArgs& args, uint32_t t_ro
   uint8_t* shi = es.buf + 4096;
   uint8_t* slo = es.buf + 6144;
   // stage 32 values of this lane's row (all lanes) and store them at output column ocol
-  auto emit = [&](const float (&x)[32], int ocol) {
+  auto emit = [&](const float (&x)[32], int ocol, int orow) {
     if (lane == 0) bulk_wait_read<0>();  // the previous chunk's stores have read the buffer
     __syncwarp();
     if (args.out32) {
@@ -276,9 +276,9 @@ __device__ __forceinline__ void epi_tile_tma(const GemmArgs& args, uint32_t t_ro
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      if (args.out32) tma_store_3d(es.o32, s32, ocol, es.orow, es.split);
-      if (args.out_hi) tma_store_2d(es.ohi, shi, ocol, es.orow);
-      if (args.out_hi && args.out_lo) tma_store_2d(es.olo, slo, ocol, es.orow);
+      if (args.out32) tma_store_3d(es.o32, s32, ocol, orow, es.split);
+      if (args.out_hi) tma_store_2d(es.ohi, shi, ocol, orow);
+      if (args.out_hi && args.out_lo) tma_store_2d(es.olo, slo, ocol, orow);
       bulk_commit();
     }
   };
@@ -320,13 +320,23 @@ __device__ __forceinline__ void epi_tile_tma(const GemmArgs& args, uint32_t t_ro
         h[j] = silu_f(__uint_as_float(va[16 + j]) * r) * (__uint_as_float(va[j]) * r);
         h[16 + j] = silu_f(__uint_as_float(vb[16 + j]) * r) * (__uint_as_float(vb[j]) * r);
       }
-      emit(h, (n0 + c * 32) / 2);
+      emit(h, (n0 + c * 32) / 2, es.orow);
+    } else if (EPI == EPI_QABS) {  // head block j of the warp's example: rows b qabs_rows + j qabs_N + n
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int col = n0 + (c + h2) * 32;
+        const int head = col / args.qabs_d;
+        const int orow = (es.orow / args.qabs_N) * args.qabs_rows + head * args.qabs_N + es.orow % args.qabs_N;
+        float x[32];
+        values(c + h2, h2 ? vb : va, x);
+        emit(x, col - head * args.qabs_d, orow);
+      }
     } else {
       float x[32];
       values(c, va, x);
-      emit(x, n0 + c * 32);
+      emit(x, n0 + c * 32, es.orow);
       values(c + 1, vb, x);
-      emit(x, n0 + (c + 1) * 32);
+      emit(x, n0 + (c + 1) * 32, es.orow);
     }
   }
 }
@@ -345,8 +355,8 @@ constexpr uint32_t kIdescAMnMajor = 1u << 15;
 // six. The K blocks of every tile, of A0 and of each split-K range are then even in number.
 //
 // TST: the epilogue writes through shared memory with tensor stores (maps tmO32, tmOhi, tmOlo over
-// the fp32 output {columns, rows, split} and the bf16 hi and lo outputs, boxes of 32 x 32); the QABS
-// row scatter keeps direct stores.
+// the fp32 output {columns, rows, split} and the bf16 hi and lo outputs, boxes of 32 x 32). The QABS
+// row scatter takes it when a warp's 32 rows stay within one example (qabs_N a multiple of 32).
 template <int BN, int EPI, bool ROWNORM, bool SPLIT, bool A_MN = false, bool B_MN = false, bool SPLIT_B = false,
           int KPS = 1, bool TST = false>
 __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
@@ -356,7 +366,6 @@ __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
                    const __grid_constant__ CUtensorMap tmOhi, const __grid_constant__ CUtensorMap tmOlo,
                    const GemmArgs args) {
   using L = GemmSmem<BN, SPLIT, SPLIT_B, KPS, TST>;
-  static_assert(!(TST && EPI == EPI_QABS), "the per-head row scatter stores directly");
   constexpr int STAGES = L::STAGES;
   constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators: 128, 256 or 512 columns
   static_assert(!(ROWNORM && A_MN), "row statistics read K-major A rows");

@@ -221,13 +221,16 @@ whale_status tmap_f32_32(CUtensorMap* tm, const void* base, long long rows, long
 }
 
 // The epilogue's store maps o[0..2] (fp32, bf16 hi, bf16 lo) over the GEMM's outputs: cols output
-// columns (N, or N / 2 for the SwiGLU epilogue), M rows; the fp32 output holds `splits` split-K
-// partials of M rows each. A missing output gets a copy of `any` (never stored through).
-whale_status epi_maps(CUtensorMap* o, const GemmArgs& g, long long cols, long long splits, const CUtensorMap& any) {
+// columns (N, or N / 2 for the SwiGLU epilogue), out_rows rows (M but for the per-head row scatter);
+// the fp32 output holds `splits` split-K partials of M rows each. A missing output gets a copy of
+// `any` (never stored through).
+whale_status epi_maps(CUtensorMap* o, const GemmArgs& g, long long cols, long long splits, const CUtensorMap& any,
+                      long long out_rows = 0) {
+  if (out_rows <= 0) out_rows = g.M;
   o[0] = o[1] = o[2] = any;
   if (g.out32) WCHECK(tmap_f32_32(&o[0], g.out32, g.M, cols, g.ldo, splits));
-  if (g.out_hi) WCHECK(tmap_bf16_box(&o[1], g.out_hi, g.M, cols, g.ldo, 32, 32));
-  if (g.out_lo) WCHECK(tmap_bf16_box(&o[2], g.out_lo, g.M, cols, g.ldo, 32, 32));
+  if (g.out_hi) WCHECK(tmap_bf16_box(&o[1], g.out_hi, out_rows, cols, g.ldo, 32, 32));
+  if (g.out_lo) WCHECK(tmap_bf16_box(&o[2], g.out_lo, out_rows, cols, g.ldo, 32, 32));
   return WHALE_OK;
 }
 
@@ -970,6 +973,10 @@ whale_status gemm_qabs(const Shape& s, const void* q, const void* wkabs, void* q
   g.qabs_N = s.N;
   g.qabs_d = s.d;
   g.qabs_rows = kAbsQ;
+  if (s.N % 32 == 0) {  // a warp's 32 rows are one example's: tensor stores
+    WCHECK(epi_maps(maps + 5, g, s.d, 1, maps[0], rows / s.N * kAbsQ));
+    return launch_gemm_t<BN, EPI_QABS, false, false>(maps, g, tiles, st);
+  }
   return launch_gemm_t<BN, EPI_QABS, false, false, false, false, false, 1, false>(maps, g, tiles, st);
 }
 
