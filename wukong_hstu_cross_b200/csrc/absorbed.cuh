@@ -1057,6 +1057,7 @@ __global__ void __launch_bounds__(256) abs_merge_kernel(const AbsArgs a) {
     for (int i = threadIdx.x; i < 2 + a.n_pairs; i += blockDim.x) a.pq[i] = 0;
   __shared__ int s_slot[8][kAbsMaxPairs];
   __shared__ float s_w[8][kAbsMaxPairs];
+  __shared__ float s_l[8][kAbsMaxPairs];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x;
   const int q = blockIdx.y * 8 + warp;
@@ -1081,9 +1082,10 @@ __global__ void __launch_bounds__(256) abs_merge_kernel(const AbsArgs a) {
     const int r0 = abs_range_start(U, P, p), r1 = abs_range_start(U, P, p + 1);
     const int slot = r0 < r1 ? (r0 >= ub ? 2 * p : 2 * p + 1) : -1;
     s_slot[warp][j] = slot;
-    const float m = slot >= 0 ? st[(size_t)slot * kAbsQ + q].x : -INFINITY;
-    s_w[warp][j] = m;
-    M = fmaxf(M, m);
+    const float2 ml = slot >= 0 ? st[(size_t)slot * kAbsQ + q] : make_float2(-INFINITY, 0.f);  // (m, l) at once
+    s_w[warp][j] = ml.x;
+    s_l[warp][j] = ml.y;
+    M = fmaxf(M, ml.x);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
@@ -1092,7 +1094,7 @@ __global__ void __launch_bounds__(256) abs_merge_kernel(const AbsArgs a) {
     const int slot = s_slot[warp][j];
     const float w = slot >= 0 ? fast_exp2(s_w[warp][j] - M) : 0.f;
     s_w[warp][j] = w;
-    if (slot >= 0) l += w * st[(size_t)slot * kAbsQ + q].y;
+    if (slot >= 0) l += w * s_l[warp][j];
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
