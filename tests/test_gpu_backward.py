@@ -2,7 +2,8 @@
 (oracle/whale_backward.py, itself pinned by finite differences of the forward oracle): every
 gradient, d_tokens, d_states and each parameter's, summed over the batch. Reduced copies of the
 training workloads (d = 128 with 4 heads of 32, d = 512 with 8 heads of 64, ragged histories, an
-empty one), every variant (shared K = V, tied gate, single-map Fusion MLP) and the fp32 mode.
+empty one, 16 tokens with histories over several 1024-row chunks), every variant (shared K = V, tied
+gate, single-map Fusion MLP) and the fp32 mode.
 Every case's worst error over bound, per tensor, goes to the JSON-lines file named by
 WHALE_PARITY_REPORT when it is set.
 
@@ -74,6 +75,8 @@ CASES = {
     "d512_reduced": ("hist15k_d512", dict(batch=3, n_layers=1, lengths=("lognormal", 1500.0, 0.5, 64, 3000)), {}),
     "d128_shared_kv": ("stack_d128", dict(batch=4, n_layers=1, lengths=("uniform", 1, 900)), {"shared_kv": True}),
     "d512_tied_gate": ("hist15k_d512", dict(batch=3, n_layers=1, lengths=("uniform", 1, 900)), {"tied_gate": True}),
+    "d512_shared_kv": ("hist15k_d512", dict(batch=3, n_layers=1, lengths=("uniform", 1, 1300)), {"shared_kv": True}),
+    "d512_n16_long": ("hist15k_d512", dict(batch=2, n_layers=1, n_tokens=16, lengths=("uniform", 1100, 2600)), {}),
     "d128_single_map": ("stack_d128", dict(batch=4, n_layers=1, lengths=("uniform", 1, 900), fusion_mult=0), {}),
     "fp32_variants": ("tiny_fp32", dict(batch=3, fusion_mult=0), {"shared_kv": True, "tied_gate": True}),
 }

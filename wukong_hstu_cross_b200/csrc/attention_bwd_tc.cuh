@@ -1,0 +1,358 @@
+// attention_bwd_tc.cuh — backward of Eq. (4) on the 5th-generation tensor cores (bf16 mode, d_h = 64,
+// up to 32 queries per example), the same products and schedule as attention_bwd.cuh:
+//   S^T = K Q^T,  dP^T = V dA^T,  P^T = 2^(S^T log2(e)/sqrt(d_h) - lse),  dS^T = P^T (dP^T - delta),
+//   dV = P^T dA,  dK = (dS^T / sqrt(d_h)) Q,  dQ^T += K^T (dS^T / sqrt(d_h)).
+// KV-parallel (gist.science technical summary of WHALE, section 2.2, Asymmetric Backward Variants):
+// a CTA owns one head of a chunk of up to 1024 history rows of one example, keeps the example's
+// queries (q, dA as bf16 pairs) in shared memory and walks the chunk in blocks of 128 rows, so dK and
+// dV of a block are complete inside the CTA and only dQ (N d_h values per chunk) is added to global
+// memory with fp32 atomics.
+//
+// Per block, with every operand a hi/lo bf16 pair and every product three MMAs (hi hi, lo hi, hi lo):
+//   tensor memory: S^T | dP^T (double-buffered, 32 + 32 columns), dV and dK (64 columns each) and
+//   the running dQ^T (64 columns; lanes 0-63 = d_h, lanes 64-127 unused products of the second
+//   MN group), all fp32;
+//   shared memory: the K|V block ring (TMA, 128-byte swizzle), and P^T and dS^T written by the
+//   epilogue threads in the K-major 128-byte-swizzled layout the MMA reads — the same bytes serve
+//   dS^T as the MN-major B operand of dQ^T.
+// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM allocation + MMA issue (one thread),
+// warps 2..5 the softmax backward and the dK|dV stores (thread i of TMEM lane quadrant q owns block
+// row 32q + i).
+// Rows past the chunk (the next example's, or past the states) and queries past N are read but give
+// P = 0 and dS = 0: lse is +inf for the missing queries and the rows past the chunk are masked.
+#pragma once
+
+#include "attention_bwd.cuh"
+#include "gemm_tc.cuh"
+#include "ptx.cuh"
+
+namespace whale {
+
+struct AttnBwdTcSmem {
+  static constexpr uint32_t TILE_Q = 32 * 128;    // 32 queries x 64 d_h bf16
+  static constexpr uint32_t TILE_KV = 128 * 128;  // 128 rows x 64 d_h bf16
+  static constexpr uint32_t OFF_Q = 0;            // q, q_lo, da, da_lo
+  static constexpr uint32_t OFF_KV = 4 * TILE_Q;  // [2 stages][k, k_lo, v, v_lo]
+  static constexpr uint32_t OFF_STG = OFF_KV + 2 * 4 * TILE_KV;  // p, p_lo, ds, ds_lo
+  static constexpr uint32_t OFF_LSE = OFF_STG + 4 * TILE_KV;     // lse[32], delta[32]
+  static constexpr uint32_t OFF_BAR = OFF_LSE + 256;
+  static constexpr uint32_t BYTES = OFF_BAR + 256 + 1024;  // + alignment slack
+};
+static_assert(AttnBwdTcSmem::BYTES <= 232448, "shared memory");
+constexpr int kAttnBwdTcThreads = 192;
+
+__global__ void __launch_bounds__(kAttnBwdTcThreads, 1)
+    attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const __grid_constant__ CUtensorMap tmKVlo,
+                       const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQlo,
+                       const __grid_constant__ CUtensorMap tmDA, const __grid_constant__ CUtensorMap tmDAlo,
+                       const AttnBwdArgs a) {
+  using L = AttnBwdTcSmem;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* lse_s = reinterpret_cast<float*>(smem + L::OFF_LSE);
+  float* del_s = lse_s + 32;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* q_full = bars;           // queries landed
+  uint64_t* kv_full = bars + 1;      // [2]
+  uint64_t* kv_empty = bars + 3;     // [2]
+  uint64_t* sp_full = bars + 5;      // [2] S^T | dP^T computed
+  uint64_t* sp_empty = bars + 7;     // [2] S^T | dP^T read by the 4 epilogue warps
+  uint64_t* pd_full = bars + 9;      // P^T, dS^T staged by the 4 epilogue warps
+  uint64_t* dvk_full = bars + 10;    // dV, dK (and dQ^T so far) computed; the staging may be rewritten
+  uint64_t* dvk_empty = bars + 11;   // dV, dK read by the 4 epilogue warps
+  uint64_t* fin = bars + 12;         // every MMA issued has completed (unwinding)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = blockIdx.x, head = blockIdx.y;
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+      mbar_init(&sp_full[i], 1);
+      mbar_init(&sp_empty[i], 4);
+    }
+    mbar_init(pd_full, 4);
+    mbar_init(dvk_full, 1);
+    mbar_init(dvk_empty, 4);
+    mbar_init(fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
+
+  // ---- this CTA's example and rows (uniform across the CTA) ----
+  const int U = a.cstart[a.B];
+  bool active = chunk < U;
+  int b = 0;
+  long long k0 = 0, k1 = 0;
+  if (active) {
+    int lo = 0, hi = a.B - 1;  // largest b with cstart[b] <= chunk
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (a.cstart[mid] <= chunk) lo = mid;
+      else hi = mid - 1;
+    }
+    b = lo;
+    auto clampo = [&](int e) -> long long {
+      long long o = a.offsets[e];
+      return o < 0 ? 0 : (o > a.total_L ? a.total_L : o);
+    };
+    const long long lo_b = clampo(b);
+    long long hi_b = clampo(b + 1);
+    if (hi_b < lo_b) hi_b = lo_b;
+    k0 = lo_b + (long long)(chunk - a.cstart[b]) * kBwdChunk;
+    k1 = min(hi_b, k0 + kBwdChunk);
+    active = k0 < k1;
+  }
+  const int nblk = active ? (int)((k1 - k0 + 127) / 128) : 0;
+  const int colk = head * 64, colv = a.v_col0 + head * 64;
+
+  // TMEM columns
+  const uint32_t t_sp = tmem_base;          // [2][S^T 32 | dP^T 32]
+  const uint32_t t_dv = tmem_base + 128;    // 64
+  const uint32_t t_dk = tmem_base + 192;    // 64
+  const uint32_t t_dq = tmem_base + 256;    // 64 (dQ^T: lanes = d_h, columns = queries)
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0 && nblk > 0) {
+      tma_prefetch_desc(&tmKV);
+      tma_prefetch_desc(&tmKVlo);
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmDA);
+      const int qrow = b * a.N;
+      mbar_arrive_expect_tx(q_full, 4 * L::TILE_Q);
+      tma_load_2d(smem + L::OFF_Q + 0 * L::TILE_Q, &tmQ, colk, qrow, q_full);
+      tma_load_2d(smem + L::OFF_Q + 1 * L::TILE_Q, &tmQlo, colk, qrow, q_full);
+      tma_load_2d(smem + L::OFF_Q + 2 * L::TILE_Q, &tmDA, colk, qrow, q_full);
+      tma_load_2d(smem + L::OFF_Q + 3 * L::TILE_Q, &tmDAlo, colk, qrow, q_full);
+      const uint32_t kv_bytes = (a.shared_kv ? 2 : 4) * L::TILE_KV;
+      int issued = 0;
+      for (int blk = 0; blk < nblk; ++blk, ++issued) {
+        const int s = blk & 1, u = blk >> 1;
+        if (blk >= 2 && !mbar_wait(&kv_empty[s], (u - 1) & 1, abort_flag)) break;
+        uint8_t* st = smem + L::OFF_KV + s * 4 * L::TILE_KV;
+        const int r0 = (int)(k0 + 128ll * blk);
+        mbar_arrive_expect_tx(&kv_full[s], kv_bytes);
+        tma_load_2d(st + 0 * L::TILE_KV, &tmKV, colk, r0, &kv_full[s]);
+        tma_load_2d(st + 1 * L::TILE_KV, &tmKVlo, colk, r0, &kv_full[s]);
+        if (!a.shared_kv) {
+          tma_load_2d(st + 2 * L::TILE_KV, &tmKV, colv, r0, &kv_full[s]);
+          tma_load_2d(st + 3 * L::TILE_KV, &tmKVlo, colv, r0, &kv_full[s]);
+        }
+      }
+      if (*abort_flag) {  // let the copies in flight land before the CTA exits
+        volatile int quiet = 0;
+        mbar_wait(q_full, 0, &quiet, 100000000ull);
+        for (int k = (issued > 2 ? issued - 2 : 0); k < issued; ++k)
+          mbar_wait(&kv_full[k & 1], (k >> 1) & 1, &quiet, 100000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0 && nblk > 0) {
+      constexpr uint32_t id_sp = idesc_bf16_f32(128, 32);                            // K-major A and B
+      constexpr uint32_t id_kv = idesc_bf16_f32(128, 64) | kIdescBMnMajor;           // dV, dK
+      constexpr uint32_t id_dq = idesc_bf16_f32(128, 64) | kIdescAMnMajor | kIdescBMnMajor;  // dQ^T
+      const uint32_t q_s = smem_u32(smem + L::OFF_Q);
+      const uint32_t ql_s = q_s + L::TILE_Q, da_s = q_s + 2 * L::TILE_Q, dal_s = q_s + 3 * L::TILE_Q;
+      const uint32_t stg = smem_u32(smem + L::OFF_STG);
+      const uint32_t p_s = stg, pl_s = stg + L::TILE_KV, ds_s = stg + 2 * L::TILE_KV, dsl_s = stg + 3 * L::TILE_KV;
+      bool ok = mbar_wait(q_full, 0, abort_flag);
+      // S^T and dP^T of block `blk` into buffer blk & 1
+      auto issue_sp = [&](int blk) -> bool {
+        const int s = blk & 1, u = blk >> 1;
+        if (!mbar_wait(&kv_full[s], u & 1, abort_flag)) return false;
+        if (blk >= 2 && !mbar_wait(&sp_empty[s], (u - 1) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t kst = smem_u32(smem + L::OFF_KV + s * 4 * L::TILE_KV);
+        const uint32_t k_s = kst, kl_s = kst + L::TILE_KV;
+        const uint32_t v_s = a.shared_kv ? k_s : kst + 2 * L::TILE_KV;
+        const uint32_t vl_s = a.shared_kv ? kl_s : kst + 3 * L::TILE_KV;
+        const uint32_t d_s = t_sp + s * 64, d_p = t_sp + s * 64 + 32;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint32_t acc = kk > 0 ? 1u : 0u;
+          umma_f16(d_s, sdesc_k_sw128(k_s + kk * 32), sdesc_k_sw128(q_s + kk * 32), id_sp, acc);
+          umma_f16(d_s, sdesc_k_sw128(kl_s + kk * 32), sdesc_k_sw128(q_s + kk * 32), id_sp, 1u);
+          umma_f16(d_s, sdesc_k_sw128(k_s + kk * 32), sdesc_k_sw128(ql_s + kk * 32), id_sp, 1u);
+          umma_f16(d_p, sdesc_k_sw128(v_s + kk * 32), sdesc_k_sw128(da_s + kk * 32), id_sp, acc);
+          umma_f16(d_p, sdesc_k_sw128(vl_s + kk * 32), sdesc_k_sw128(da_s + kk * 32), id_sp, 1u);
+          umma_f16(d_p, sdesc_k_sw128(v_s + kk * 32), sdesc_k_sw128(dal_s + kk * 32), id_sp, 1u);
+        }
+        umma_commit(&sp_full[s]);
+        return true;
+      };
+      if (ok) ok = issue_sp(0);
+      for (int blk = 0; blk < nblk && ok; ++blk) {
+        if (blk + 1 < nblk && !issue_sp(blk + 1)) break;
+        if (!mbar_wait(pd_full, blk & 1, abort_flag)) break;
+        if (blk >= 1 && !mbar_wait(dvk_empty, (blk - 1) & 1, abort_flag)) break;
+        tc_fence_after();
+        const int s = blk & 1;
+        const uint32_t kst = smem_u32(smem + L::OFF_KV + s * 4 * L::TILE_KV);
+        const uint32_t k_s = kst, kl_s = kst + L::TILE_KV;
+        // dV = P^T dA and dK = (dS^T / sqrt(d_h)) Q: K = 32 queries (two k-steps); with shared K = V
+        // both accumulate into dV's columns
+        const uint32_t d_k = a.shared_kv ? t_dv : t_dk;
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          const uint32_t acc = kk > 0 ? 1u : 0u;
+          const uint64_t bda = sdesc_mn_sw128(da_s + kk * 2048, 8192, 1024);
+          const uint64_t bdal = sdesc_mn_sw128(dal_s + kk * 2048, 8192, 1024);
+          const uint64_t bq = sdesc_mn_sw128(q_s + kk * 2048, 8192, 1024);
+          const uint64_t bql = sdesc_mn_sw128(ql_s + kk * 2048, 8192, 1024);
+          umma_f16(t_dv, sdesc_k_sw128(p_s + kk * 32), bda, id_kv, acc);
+          umma_f16(t_dv, sdesc_k_sw128(pl_s + kk * 32), bda, id_kv, 1u);
+          umma_f16(t_dv, sdesc_k_sw128(p_s + kk * 32), bdal, id_kv, 1u);
+          const uint32_t acck = a.shared_kv ? 1u : acc;
+          umma_f16(d_k, sdesc_k_sw128(ds_s + kk * 32), bq, id_kv, acck);
+          umma_f16(d_k, sdesc_k_sw128(dsl_s + kk * 32), bq, id_kv, 1u);
+          umma_f16(d_k, sdesc_k_sw128(ds_s + kk * 32), bql, id_kv, 1u);
+        }
+        // dQ^T += K^T (dS^T / sqrt(d_h)): A = the K tile MN-major (M = d_h; its second 64-element MN
+        // group, lanes 64-127, reads the K lo tile and is not used), B = dS^T MN-major (N = queries,
+        // 64 wide: columns 32-63 are not used), K = the block's 128 rows
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t acc = (blk > 0 || kk > 0) ? 1u : 0u;
+          const uint64_t bds = sdesc_mn_sw128(ds_s + kk * 2048, 8192, 1024);
+          const uint64_t bdsl = sdesc_mn_sw128(dsl_s + kk * 2048, 8192, 1024);
+          umma_f16(t_dq, sdesc_mn_sw128(k_s + kk * 2048, L::TILE_KV, 1024), bds, id_dq, acc);
+          umma_f16(t_dq, sdesc_mn_sw128(kl_s + kk * 2048, L::TILE_KV, 1024), bds, id_dq, 1u);
+          umma_f16(t_dq, sdesc_mn_sw128(k_s + kk * 2048, L::TILE_KV, 1024), bdsl, id_dq, 1u);
+        }
+        umma_commit(dvk_full);      // dV, dK, dQ^T so far; the staging tiles are free again
+        umma_commit(&kv_empty[s]);  // the K|V stage may be refilled
+      }
+      umma_commit(fin);  // arrives once every MMA issued above has completed
+      volatile int quiet = 0;
+      mbar_wait(fin, 0, &quiet, 100000000ull);
+    }
+  } else if (nblk > 0) {
+    // ---------------- softmax backward and the dK|dV stores (warps 2..5) ----------------
+    const int qd = warp & 3;
+    const int rloc = qd * 32 + lane;  // block row of this thread (= TMEM lane)
+    const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+    // lse (+inf past N: p = 0) and delta of this head
+    if (warp == 2) {
+      const long long idx = ((long long)b * a.N + lane) * a.n_heads + head;
+      lse_s[lane] = lane < a.N ? a.lse[idx] : INFINITY;
+      del_s[lane] = lane < a.N ? a.delta[idx] : 0.f;
+    }
+    named_bar_sync(1, 128);
+    uint8_t* stg = smem + L::OFF_STG;
+    const uint32_t sw = (uint32_t)(rloc & 7);
+    int done = 0;  // blocks completed (all of them unless a wait ran out)
+    for (int blk = 0; blk < nblk; ++blk) {
+      const int s = blk & 1, u = blk >> 1;
+      const long long row = k0 + 128ll * blk + rloc;
+      const bool row_ok = row < k1;
+      if (!mbar_wait(&sp_full[s], u & 1, abort_flag)) break;
+      tc_fence_after();
+      uint32_t sv[32], dpv[32];
+      tmem_ld_32x32b_x32(t_sp + s * 64 + lane_off, sv);
+      tmem_ld_32x32b_x32(t_sp + s * 64 + 32 + lane_off, dpv);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sp_empty[s]);
+      // P^T and dS^T / sqrt(d_h) of this row as bf16 pairs, in the K-major 128-byte-swizzled layout
+      // (row rloc: 16-byte chunk c at position c ^ (rloc % 8)); queries 0..31 fill chunks 0..3
+      uint32_t ph[16], pl[16], dh[16], dl[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        float p0 = 0.f, p1 = 0.f, g0 = 0.f, g1 = 0.f;
+        if (row_ok) {
+          p0 = fast_exp2(fmaf(__uint_as_float(sv[2 * j]), a.scale_log2, -lse_s[2 * j]));
+          p1 = fast_exp2(fmaf(__uint_as_float(sv[2 * j + 1]), a.scale_log2, -lse_s[2 * j + 1]));
+          g0 = p0 * (__uint_as_float(dpv[2 * j]) - del_s[2 * j]) * a.scale;
+          g1 = p1 * (__uint_as_float(dpv[2 * j + 1]) - del_s[2 * j + 1]) * a.scale;
+        }
+        split2(p0, p1, ph[j], pl[j]);
+        split2(g0, g1, dh[j], dl[j]);
+      }
+      // the staging is free: the previous block's MMAs completed (its dvk_full, waited below)
+      {
+        uint8_t* rowp = stg + rloc * 128;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t off = ((uint32_t)c ^ sw) * 16;
+          *reinterpret_cast<uint4*>(rowp + 0 * L::TILE_KV + off) = make_uint4(ph[4 * c], ph[4 * c + 1], ph[4 * c + 2], ph[4 * c + 3]);
+          *reinterpret_cast<uint4*>(rowp + 1 * L::TILE_KV + off) = make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
+          *reinterpret_cast<uint4*>(rowp + 2 * L::TILE_KV + off) = make_uint4(dh[4 * c], dh[4 * c + 1], dh[4 * c + 2], dh[4 * c + 3]);
+          *reinterpret_cast<uint4*>(rowp + 3 * L::TILE_KV + off) = make_uint4(dl[4 * c], dl[4 * c + 1], dl[4 * c + 2], dl[4 * c + 3]);
+        }
+      }
+      fence_proxy_async_smem();  // the MMAs read the staging through the async proxy
+      __syncwarp();
+      if (lane == 0) mbar_arrive(pd_full);
+      // dV and dK of this block: rows scaled by row_scale, stored as pairs
+      if (!mbar_wait(dvk_full, blk & 1, abort_flag)) break;
+      tc_fence_after();
+      const float rs = (a.row_scale && row_ok) ? a.row_scale[row] : 1.0f;
+#pragma unroll 1
+      for (int which = 0; which < (a.shared_kv ? 1 : 2); ++which) {
+        const uint32_t tcol = which == 0 ? t_dk : t_dv;
+        const int gcol = which == 0 ? colk : colv;
+        const uint32_t tsrc = a.shared_kv ? t_dv : tcol;  // shared K = V: dK + dV in dV's columns
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tsrc + h2 * 32 + lane_off, v);
+          tmem_ld_wait();
+          if (row_ok) {
+            uint32_t hw[16], lw[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              split2(__uint_as_float(v[2 * j]) * rs, __uint_as_float(v[2 * j + 1]) * rs, hw[j], lw[j]);
+            uint4* dst = reinterpret_cast<uint4*>(a.dkv + row * a.kvw + gcol + h2 * 32);
+            uint4* dstl = reinterpret_cast<uint4*>(a.dkv_lo + row * a.kvw + gcol + h2 * 32);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              dst[c] = make_uint4(hw[4 * c], hw[4 * c + 1], hw[4 * c + 2], hw[4 * c + 3]);
+              dstl[c] = make_uint4(lw[4 * c], lw[4 * c + 1], lw[4 * c + 2], lw[4 * c + 3]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dvk_empty);
+      done = blk + 1;
+    }
+    // dq += this chunk's share: dQ^T lanes 0..63 (d_h) x columns 0..31 (queries), read by the warps of
+    // lane quadrants 0 and 1 once the last block's MMAs are complete (its dvk_full, waited above)
+    if (done == nblk && *abort_flag == 0 && qd < 2) {
+      tc_fence_after();
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(t_dq + lane_off, v);
+      tmem_ld_wait();
+      const int m = qd * 32 + lane;  // d_h index
+      for (int n = 0; n < a.N && n < 32; ++n)
+        atomicAdd(a.dq + ((long long)b * a.N + n) * a.d + colk + m, __uint_as_float(v[n]));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+}  // namespace whale

@@ -31,6 +31,7 @@
 #include "attention.cuh"
 #include "attention_qtile.cuh"
 #include "attention_bwd.cuh"
+#include "attention_bwd_tc.cuh"
 #include "backward.cuh"
 #include "fp32_path.cuh"
 #include "gemm_2sm.cuh"
@@ -1562,6 +1563,24 @@ whale_status launch_attn_bwd(const AttnBwdArgs& a, unsigned chunks, cudaStream_t
   return launch_pdl(attn_bwd_kernel<DH, NQ>, dim3(chunks, a.n_heads / C::HG), dim3(C::THREADS), C::BYTES, st, a);
 }
 
+// The tensor-core attention backward (d_h = 64, N <= 32): one CTA per (chunk, head); K|V, q, dA
+// (all bf16 pairs) read through tensor maps.
+whale_status launch_attn_bwd_tc(const AttnBwdArgs& a, unsigned chunks, cudaStream_t st) {
+  if (a.d % 64 || a.N > 32 || a.N < 1 || a.kvw % 64 || a.total_L <= 0) return WHALE_ERR_UNSUPPORTED;
+  const long long rows = (long long)a.B * a.N;
+  CUtensorMap m[6];
+  WCHECK(tmap_bf16(&m[0], a.kv, a.total_L, a.kvw, a.kvw, 128));
+  WCHECK(tmap_bf16(&m[1], a.kv_lo, a.total_L, a.kvw, a.kvw, 128));
+  WCHECK(tmap_bf16(&m[2], a.q, rows, a.d, a.d, 32));
+  WCHECK(tmap_bf16(&m[3], a.q_lo, rows, a.d, a.d, 32));
+  WCHECK(tmap_bf16(&m[4], a.da, rows, a.d, a.d, 32));
+  WCHECK(tmap_bf16(&m[5], a.da_lo, rows, a.d, a.d, 32));
+  CUCHECK(cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)AttnBwdTcSmem::BYTES));
+  return launch_pdl(attn_bwd_tc_kernel, dim3(chunks, a.n_heads), dim3(kAttnBwdTcThreads), AttnBwdTcSmem::BYTES, st,
+                    m[0], m[1], m[2], m[3], m[4], m[5], a);
+}
+
 // Shapes the backward pass supports: bf16 with at most 32 queries per example (the KV-parallel
 // attention backward keeps all of an example's queries resident), d a multiple of 128 (its head
 // groups span 128 columns) and d <= 1024 (row kernels); fp32 with d_head <= 64.
@@ -1706,7 +1725,7 @@ whale_status layer_backward_bf16(const Shape& s, const Stream3& in, const void* 
     aa.scale = (float)(1.0 / std::sqrt((double)s.dh));
     aa.scale_log2 = scale_log2_of(s);
     whale_status r;
-    if (s.dh == 64) r = s.N <= 16 ? launch_attn_bwd<64, 16>(aa, (unsigned)cmax, st) : launch_attn_bwd<64, 32>(aa, (unsigned)cmax, st);
+    if (s.dh == 64) r = launch_attn_bwd_tc(aa, (unsigned)cmax, st);
     else r = s.N <= 16 ? launch_attn_bwd<32, 16>(aa, (unsigned)cmax, st) : launch_attn_bwd<32, 32>(aa, (unsigned)cmax, st);
     WCHECK(r);
   }
