@@ -9,15 +9,18 @@
 // memory with fp32 atomics.
 //
 // Per block, with every operand a hi/lo bf16 pair and every product three MMAs (hi hi, lo hi, hi lo):
-//   tensor memory: S^T | dP^T (double-buffered, 32 + 32 columns), dV and dK (64 columns each) and
-//   the running dQ^T (64 columns; lanes 0-63 = d_h, lanes 64-127 unused products of the second
-//   MN group), all fp32;
+//   tensor memory: S^T | dP^T (double-buffered, 32 + 32 columns), dV and dK (double-buffered, 64
+//   columns each) and the running dQ^T (64 columns; lanes 0-63 = d_h, lanes 64-127 unused products
+//   of the second MN group), all fp32;
 //   shared memory: the K|V block ring (TMA, 128-byte swizzle), and P^T and dS^T written by the
 //   epilogue threads in the K-major 128-byte-swizzled layout the MMA reads — the same bytes serve
 //   dS^T as the MN-major B operand of dQ^T.
-// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM allocation + MMA issue (one thread),
-// warps 2..5 the softmax backward and the dK|dV stores (thread i of TMEM lane quadrant q owns block
-// row 32q + i).
+// Warp roles (320 threads): warp 0 TMA producer, warp 1 TMEM allocation + MMA issue (one thread),
+// warps 2..5 the softmax backward (the next block's while a block's MMAs run), warps 6..9 the dK|dV
+// drain while the next block is computed: rows scaled by r, split into pairs, written into the block's
+// own K|V stage (free once the block's MMAs are done) and stored from there with tensor stores (boxes
+// of 32 rows x 64 columns: tmDKV, tmDKVlo); the producer refills the stage after those stores have
+// read it. Thread i of TMEM lane quadrant q owns block row 32q + i.
 // Rows past the chunk (the next example's, or past the states) and queries past N are read but give
 // P = 0 and dS = 0: lse is +inf for the missing queries and the rows past the chunk are masked.
 #pragma once
@@ -39,12 +42,13 @@ struct AttnBwdTcSmem {
   static constexpr uint32_t BYTES = OFF_BAR + 256 + 1024;  // + alignment slack
 };
 static_assert(AttnBwdTcSmem::BYTES <= 232448, "shared memory");
-constexpr int kAttnBwdTcThreads = 192;
+constexpr int kAttnBwdTcThreads = 320;
 
 __global__ void __launch_bounds__(kAttnBwdTcThreads, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const __grid_constant__ CUtensorMap tmKVlo,
                        const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQlo,
                        const __grid_constant__ CUtensorMap tmDA, const __grid_constant__ CUtensorMap tmDAlo,
+                       const __grid_constant__ CUtensorMap tmDKV, const __grid_constant__ CUtensorMap tmDKVlo,
                        const AttnBwdArgs a) {
   using L = AttnBwdTcSmem;
   extern __shared__ uint8_t smem_raw[];
@@ -54,14 +58,14 @@ __global__ void __launch_bounds__(kAttnBwdTcThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* q_full = bars;           // queries landed
   uint64_t* kv_full = bars + 1;      // [2]
-  uint64_t* kv_empty = bars + 3;     // [2]
+  uint64_t* kv_empty = bars + 3;     // [2] the stage's dK|dV stores have read it (4 drain warps)
   uint64_t* sp_full = bars + 5;      // [2] S^T | dP^T computed
   uint64_t* sp_empty = bars + 7;     // [2] S^T | dP^T read by the 4 epilogue warps
-  uint64_t* pd_full = bars + 9;      // P^T, dS^T staged by the 4 epilogue warps
-  uint64_t* dvk_full = bars + 10;    // dV, dK (and dQ^T so far) computed; the staging may be rewritten
-  uint64_t* dvk_empty = bars + 11;   // dV, dK read by the 4 epilogue warps
-  uint64_t* fin = bars + 12;         // every MMA issued has completed (unwinding)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  uint64_t* pd_full = bars + 9;      // P^T, dS^T staged by the 4 softmax warps
+  uint64_t* dvk_full = bars + 10;    // [2] dV, dK (and dQ^T so far) computed; the staging is free again
+  uint64_t* dvk_empty = bars + 12;   // [2] dV, dK read by the 4 drain warps
+  uint64_t* fin = bars + 14;         // every MMA issued has completed (unwinding)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -70,13 +74,15 @@ __global__ void __launch_bounds__(kAttnBwdTcThreads, 1)
     mbar_init(q_full, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&kv_empty[i], 4);
       mbar_init(&sp_full[i], 1);
       mbar_init(&sp_empty[i], 4);
     }
     mbar_init(pd_full, 4);
-    mbar_init(dvk_full, 1);
-    mbar_init(dvk_empty, 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&dvk_full[i], 1);
+      mbar_init(&dvk_empty[i], 4);
+    }
     mbar_init(fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -122,9 +128,9 @@ __global__ void __launch_bounds__(kAttnBwdTcThreads, 1)
 
   // TMEM columns
   const uint32_t t_sp = tmem_base;          // [2][S^T 32 | dP^T 32]
-  const uint32_t t_dv = tmem_base + 128;    // 64
-  const uint32_t t_dk = tmem_base + 192;    // 64
-  const uint32_t t_dq = tmem_base + 256;    // 64 (dQ^T: lanes = d_h, columns = queries)
+  const uint32_t t_dv = tmem_base + 128;    // [2][64]
+  const uint32_t t_dk = tmem_base + 256;    // [2][64]
+  const uint32_t t_dq = tmem_base + 384;    // 64 (dQ^T: lanes = d_h, columns = queries)
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -197,17 +203,29 @@ __global__ void __launch_bounds__(kAttnBwdTcThreads, 1)
         return true;
       };
       if (ok) ok = issue_sp(0);
+      int sp_next = 1;  // the next block whose S^T | dP^T is to be issued
+      // S^T | dP^T of the next block goes ahead of this block's products when its K|V stage has landed
+      // (the stage is refilled only after the dK|dV stores of two blocks back have read it)
+      auto sp_ready = [&](int nb) {
+        return mbar_test(&kv_full[nb & 1], (nb >> 1) & 1) &&
+               (nb < 2 || mbar_test(&sp_empty[nb & 1], ((nb >> 1) - 1) & 1));
+      };
       for (int blk = 0; blk < nblk && ok; ++blk) {
-        if (blk + 1 < nblk && !issue_sp(blk + 1)) break;
+        if (sp_next == blk + 1 && sp_next < nblk && sp_ready(sp_next)) {
+          if (!issue_sp(sp_next)) break;
+          ++sp_next;
+        }
         if (!mbar_wait(pd_full, blk & 1, abort_flag)) break;
-        if (blk >= 1 && !mbar_wait(dvk_empty, (blk - 1) & 1, abort_flag)) break;
+        const int db = blk & 1;  // dV|dK buffer
+        if (blk >= 2 && !mbar_wait(&dvk_empty[db], ((blk >> 1) - 1) & 1, abort_flag)) break;
         tc_fence_after();
         const int s = blk & 1;
         const uint32_t kst = smem_u32(smem + L::OFF_KV + s * 4 * L::TILE_KV);
         const uint32_t k_s = kst, kl_s = kst + L::TILE_KV;
         // dV = P^T dA and dK = (dS^T / sqrt(d_h)) Q: K = 32 queries (two k-steps); with shared K = V
         // both accumulate into dV's columns
-        const uint32_t d_k = a.shared_kv ? t_dv : t_dk;
+        const uint32_t d_v = t_dv + db * 64;
+        const uint32_t d_k = a.shared_kv ? d_v : t_dk + db * 64;
 #pragma unroll
         for (int kk = 0; kk < 2; ++kk) {
           const uint32_t acc = kk > 0 ? 1u : 0u;
@@ -215,9 +233,9 @@ __global__ void __launch_bounds__(kAttnBwdTcThreads, 1)
           const uint64_t bdal = sdesc_mn_sw128(dal_s + kk * 2048, 8192, 1024);
           const uint64_t bq = sdesc_mn_sw128(q_s + kk * 2048, 8192, 1024);
           const uint64_t bql = sdesc_mn_sw128(ql_s + kk * 2048, 8192, 1024);
-          umma_f16(t_dv, sdesc_k_sw128(p_s + kk * 32), bda, id_kv, acc);
-          umma_f16(t_dv, sdesc_k_sw128(pl_s + kk * 32), bda, id_kv, 1u);
-          umma_f16(t_dv, sdesc_k_sw128(p_s + kk * 32), bdal, id_kv, 1u);
+          umma_f16(d_v, sdesc_k_sw128(p_s + kk * 32), bda, id_kv, acc);
+          umma_f16(d_v, sdesc_k_sw128(pl_s + kk * 32), bda, id_kv, 1u);
+          umma_f16(d_v, sdesc_k_sw128(p_s + kk * 32), bdal, id_kv, 1u);
           const uint32_t acck = a.shared_kv ? 1u : acc;
           umma_f16(d_k, sdesc_k_sw128(ds_s + kk * 32), bq, id_kv, acck);
           umma_f16(d_k, sdesc_k_sw128(dsl_s + kk * 32), bq, id_kv, 1u);
@@ -235,15 +253,18 @@ __global__ void __launch_bounds__(kAttnBwdTcThreads, 1)
           umma_f16(t_dq, sdesc_mn_sw128(kl_s + kk * 2048, L::TILE_KV, 1024), bds, id_dq, 1u);
           umma_f16(t_dq, sdesc_mn_sw128(k_s + kk * 2048, L::TILE_KV, 1024), bdsl, id_dq, 1u);
         }
-        umma_commit(dvk_full);      // dV, dK, dQ^T so far; the staging tiles are free again
-        umma_commit(&kv_empty[s]);  // the K|V stage may be refilled
+        umma_commit(&dvk_full[db]);  // dV, dK, dQ^T so far; the staging tiles and the K|V stage are free
+        if (sp_next == blk + 1 && sp_next < nblk) {
+          if (!issue_sp(sp_next)) break;
+          ++sp_next;
+        }
       }
       umma_commit(fin);  // arrives once every MMA issued above has completed
       volatile int quiet = 0;
       mbar_wait(fin, 0, &quiet, 100000000ull);
     }
-  } else if (nblk > 0) {
-    // ---------------- softmax backward and the dK|dV stores (warps 2..5) ----------------
+  } else if (warp < 6 && nblk > 0) {
+    // ---------------- softmax backward (warps 2..5) ----------------
     const int qd = warp & 3;
     const int rloc = qd * 32 + lane;  // block row of this thread (= TMEM lane)
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
@@ -254,14 +275,13 @@ __global__ void __launch_bounds__(kAttnBwdTcThreads, 1)
       del_s[lane] = lane < a.N ? a.delta[idx] : 0.f;
     }
     named_bar_sync(1, 128);
-    uint8_t* stg = smem + L::OFF_STG;
+    uint8_t* rowp = smem + L::OFF_STG + rloc * 128;  // this thread's row of each staging tile
     const uint32_t sw = (uint32_t)(rloc & 7);
-    int done = 0;  // blocks completed (all of them unless a wait ran out)
-    for (int blk = 0; blk < nblk; ++blk) {
+    // P^T and dS^T / sqrt(d_h) of one block for this row as bf16 pairs
+    uint32_t ph[16], pl[16], dh[16], dl[16];
+    auto softmax = [&](int blk) -> bool {
       const int s = blk & 1, u = blk >> 1;
-      const long long row = k0 + 128ll * blk + rloc;
-      const bool row_ok = row < k1;
-      if (!mbar_wait(&sp_full[s], u & 1, abort_flag)) break;
+      if (!mbar_wait(&sp_full[s], u & 1, abort_flag)) return false;
       tc_fence_after();
       uint32_t sv[32], dpv[32];
       tmem_ld_32x32b_x32(t_sp + s * 64 + lane_off, sv);
@@ -270,9 +290,7 @@ __global__ void __launch_bounds__(kAttnBwdTcThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sp_empty[s]);
-      // P^T and dS^T / sqrt(d_h) of this row as bf16 pairs, in the K-major 128-byte-swizzled layout
-      // (row rloc: 16-byte chunk c at position c ^ (rloc % 8)); queries 0..31 fill chunks 0..3
-      uint32_t ph[16], pl[16], dh[16], dl[16];
+      const bool row_ok = k0 + 128ll * blk + rloc < k1;
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         float p0 = 0.f, p1 = 0.f, g0 = 0.f, g1 = 0.f;
@@ -285,55 +303,95 @@ __global__ void __launch_bounds__(kAttnBwdTcThreads, 1)
         split2(p0, p1, ph[j], pl[j]);
         split2(g0, g1, dh[j], dl[j]);
       }
-      // the staging is free: the previous block's MMAs completed (its dvk_full, waited below)
-      {
-        uint8_t* rowp = stg + rloc * 128;
+      return true;
+    };
+    bool ok = softmax(0);
+    for (int blk = 0; blk < nblk && ok; ++blk) {
+      // the staging is free once the previous block's MMAs have completed
+      if (blk >= 1 && !mbar_wait(&dvk_full[(blk - 1) & 1], ((blk - 1) >> 1) & 1, abort_flag)) break;
+      // P^T and dS^T in the K-major 128-byte-swizzled layout (row rloc: 16-byte chunk c at position
+      // c ^ (rloc % 8)); queries 0..31 fill chunks 0..3
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint32_t off = ((uint32_t)c ^ sw) * 16;
-          *reinterpret_cast<uint4*>(rowp + 0 * L::TILE_KV + off) = make_uint4(ph[4 * c], ph[4 * c + 1], ph[4 * c + 2], ph[4 * c + 3]);
-          *reinterpret_cast<uint4*>(rowp + 1 * L::TILE_KV + off) = make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
-          *reinterpret_cast<uint4*>(rowp + 2 * L::TILE_KV + off) = make_uint4(dh[4 * c], dh[4 * c + 1], dh[4 * c + 2], dh[4 * c + 3]);
-          *reinterpret_cast<uint4*>(rowp + 3 * L::TILE_KV + off) = make_uint4(dl[4 * c], dl[4 * c + 1], dl[4 * c + 2], dl[4 * c + 3]);
-        }
+      for (int c = 0; c < 4; ++c) {
+        const uint32_t off = ((uint32_t)c ^ sw) * 16;
+        *reinterpret_cast<uint4*>(rowp + 0 * L::TILE_KV + off) = make_uint4(ph[4 * c], ph[4 * c + 1], ph[4 * c + 2], ph[4 * c + 3]);
+        *reinterpret_cast<uint4*>(rowp + 1 * L::TILE_KV + off) = make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
+        *reinterpret_cast<uint4*>(rowp + 2 * L::TILE_KV + off) = make_uint4(dh[4 * c], dh[4 * c + 1], dh[4 * c + 2], dh[4 * c + 3]);
+        *reinterpret_cast<uint4*>(rowp + 3 * L::TILE_KV + off) = make_uint4(dl[4 * c], dl[4 * c + 1], dl[4 * c + 2], dl[4 * c + 3]);
       }
       fence_proxy_async_smem();  // the MMAs read the staging through the async proxy
       __syncwarp();
       if (lane == 0) mbar_arrive(pd_full);
-      // dV and dK of this block: rows scaled by row_scale, stored as pairs
-      if (!mbar_wait(dvk_full, blk & 1, abort_flag)) break;
+      // the next block's softmax runs while this block's MMAs do
+      if (blk + 1 < nblk) ok = softmax(blk + 1);
+    }
+  } else if (nblk > 0) {
+    // ---------------- dK|dV drain (warps 6..9) ----------------
+    const int qd = warp & 3;
+    const int rloc = qd * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+    const int nw = a.shared_kv ? 1 : 2;
+    const uint32_t sw = (uint32_t)(rloc & 7);
+    int done = 0;  // blocks drained (all of them unless a wait ran out)
+    for (int blk = 0; blk < nblk; ++blk) {
+      const int db = blk & 1, s = blk & 1;
+      const long long row = k0 + 128ll * blk + rloc;
+      const bool row_ok = row < k1;
+      const float rs = (a.row_scale && row_ok) ? a.row_scale[row] : 1.0f;  // before the wait
+      const long long slice0 = k0 + 128ll * blk + qd * 32;
+      const bool full_slice = slice0 + 32 <= k1;  // uniform across the warp
+      uint8_t* rowp = smem + L::OFF_KV + s * 4 * L::TILE_KV + rloc * 128;  // this row of the block's stage
+      if (!mbar_wait(&dvk_full[db], (blk >> 1) & 1, abort_flag)) break;
       tc_fence_after();
-      const float rs = (a.row_scale && row_ok) ? a.row_scale[row] : 1.0f;
 #pragma unroll 1
-      for (int which = 0; which < (a.shared_kv ? 1 : 2); ++which) {
-        const uint32_t tcol = which == 0 ? t_dk : t_dv;
+      for (int which = 0; which < nw; ++which) {
+        // dK (which 0; with shared K = V, dK + dV in dV's columns) and dV (which 1), rows scaled by r
+        const uint32_t tsrc = a.shared_kv ? t_dv + db * 64 : (which == 0 ? t_dk : t_dv) + db * 64;
         const int gcol = which == 0 ? colk : colv;
-        const uint32_t tsrc = a.shared_kv ? t_dv : tcol;  // shared K = V: dK + dV in dV's columns
+        uint32_t v0[32], v1[32];
+        tmem_ld_32x32b_x32(tsrc + lane_off, v0);
+        tmem_ld_32x32b_x32(tsrc + 32 + lane_off, v1);
+        tmem_ld_wait();
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(tsrc + h2 * 32 + lane_off, v);
-          tmem_ld_wait();
-          if (row_ok) {
-            uint32_t hw[16], lw[16];
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t* v = c < 4 ? v0 + 8 * c : v1 + 8 * (c - 4);
+          uint32_t h[4], l[4];
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-              split2(__uint_as_float(v[2 * j]) * rs, __uint_as_float(v[2 * j + 1]) * rs, hw[j], lw[j]);
-            uint4* dst = reinterpret_cast<uint4*>(a.dkv + row * a.kvw + gcol + h2 * 32);
-            uint4* dstl = reinterpret_cast<uint4*>(a.dkv_lo + row * a.kvw + gcol + h2 * 32);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              dst[c] = make_uint4(hw[4 * c], hw[4 * c + 1], hw[4 * c + 2], hw[4 * c + 3]);
-              dstl[c] = make_uint4(lw[4 * c], lw[4 * c + 1], lw[4 * c + 2], lw[4 * c + 3]);
-            }
+          for (int j = 0; j < 4; ++j)
+            split2(__uint_as_float(v[2 * j]) * rs, __uint_as_float(v[2 * j + 1]) * rs, h[j], l[j]);
+          if (full_slice) {  // 128-byte-swizzled rows of the stage's tiles (dK hi, dK lo, dV hi, dV lo)
+            const uint32_t off = ((uint32_t)c ^ sw) * 16;
+            *reinterpret_cast<uint4*>(rowp + (2 * which) * L::TILE_KV + off) = make_uint4(h[0], h[1], h[2], h[3]);
+            *reinterpret_cast<uint4*>(rowp + (2 * which + 1) * L::TILE_KV + off) = make_uint4(l[0], l[1], l[2], l[3]);
+          } else if (row_ok) {
+            reinterpret_cast<uint4*>(a.dkv + row * a.kvw + gcol)[c] = make_uint4(h[0], h[1], h[2], h[3]);
+            reinterpret_cast<uint4*>(a.dkv_lo + row * a.kvw + gcol)[c] = make_uint4(l[0], l[1], l[2], l[3]);
           }
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(dvk_empty);
+      if (lane == 0) mbar_arrive(&dvk_empty[db]);  // this TMEM buffer may take block blk + 2
+      if (full_slice) {
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          uint8_t* st = smem + L::OFF_KV + s * 4 * L::TILE_KV + qd * 4096;
+          for (int which = 0; which < nw; ++which) {
+            const int gcol = which == 0 ? colk : colv;
+            tma_store_2d(&tmDKV, st + (2 * which) * L::TILE_KV, gcol, (int)slice0);
+            tma_store_2d(&tmDKVlo, st + (2 * which + 1) * L::TILE_KV, gcol, (int)slice0);
+          }
+          bulk_commit();
+          bulk_wait_read<0>();  // the stores have read the stage
+        }
+        __syncwarp();
+      }
+      if (lane == 0) mbar_arrive(&kv_empty[s]);  // the producer may refill the stage
       done = blk + 1;
     }
+    if (lane == 0) bulk_wait<0>();  // this warp's tensor stores are complete
+    __syncwarp();
     // dq += this chunk's share: dQ^T lanes 0..63 (d_h) x columns 0..31 (queries), read by the warps of
     // lane quadrants 0 and 1 once the last block's MMAs are complete (its dvk_full, waited above)
     if (done == nblk && *abort_flag == 0 && qd < 2) {

@@ -1568,17 +1568,19 @@ whale_status launch_attn_bwd(const AttnBwdArgs& a, unsigned chunks, cudaStream_t
 whale_status launch_attn_bwd_tc(const AttnBwdArgs& a, unsigned chunks, cudaStream_t st) {
   if (a.d % 64 || a.N > 32 || a.N < 1 || a.kvw % 64 || a.total_L <= 0) return WHALE_ERR_UNSUPPORTED;
   const long long rows = (long long)a.B * a.N;
-  CUtensorMap m[6];
+  CUtensorMap m[8];
   WCHECK(tmap_bf16(&m[0], a.kv, a.total_L, a.kvw, a.kvw, 128));
   WCHECK(tmap_bf16(&m[1], a.kv_lo, a.total_L, a.kvw, a.kvw, 128));
   WCHECK(tmap_bf16(&m[2], a.q, rows, a.d, a.d, 32));
   WCHECK(tmap_bf16(&m[3], a.q_lo, rows, a.d, a.d, 32));
   WCHECK(tmap_bf16(&m[4], a.da, rows, a.d, a.d, 32));
   WCHECK(tmap_bf16(&m[5], a.da_lo, rows, a.d, a.d, 32));
+  WCHECK(tmap_bf16(&m[6], a.dkv, a.total_L, a.kvw, a.kvw, 32));
+  WCHECK(tmap_bf16(&m[7], a.dkv_lo, a.total_L, a.kvw, a.kvw, 32));
   CUCHECK(cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)AttnBwdTcSmem::BYTES));
   return launch_pdl(attn_bwd_tc_kernel, dim3(chunks, a.n_heads), dim3(kAttnBwdTcThreads), AttnBwdTcSmem::BYTES, st,
-                    m[0], m[1], m[2], m[3], m[4], m[5], a);
+                    m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], a);
 }
 
 // Shapes the backward pass supports: bf16 with at most 32 queries per example (the KV-parallel
