@@ -455,13 +455,15 @@ def time_backward(p, raw_weights, w, total_L, peaks, clocks, stream, reps=10):
     out = {"entry_point": "whale_fusion_layer_backward (one layer, forward recomputed inside)", "ms_per_layer": ms,
            "reps": reps, "kernels": kernels,
            "launch_order": [[kernel_name(n), round(t, 4)] for n, t in recs]}
-    ab = next((v for k, v in kernels.items() if k.split("<")[0] == "attn_bwd_kernel"), None)
+    abk = next((k for k in kernels if k.split("<")[0] in ("attn_bwd_tc_kernel", "attn_bwd_kernel")), None)
+    ab = kernels[abk] if abk else None
     if ab:
         kvw = w.d if p.flags.get("shared_kv") else 2 * w.d
         nb = 2.0 * total_L * kvw * 2          # K|V read once, dK|dV written once (bf16)
         fl = 10.0 * w.n_tokens * total_L * w.d  # S, dP, dV, dK, dQ: five contractions of 2 N L d
         tc, tc_src = tensor_peak(peaks, clocks)
-        out["roofline"] = {"kernel": "attn_bwd_kernel (KV-parallel attention backward, mma.sync)",
+        what = ("tcgen05, TMEM accumulators" if abk.startswith("attn_bwd_tc") else "mma.sync")
+        out["roofline"] = {"kernel": f"{abk} (KV-parallel attention backward, {what})",
                            **roofline_of(fl, nb, ab["avg_ms"], tc, peaks["hbm_gbs"]),
                            "algorithmic_flops_per_launch": fl, "algorithmic_bytes_per_launch": nb,
                            "avg_launch_ms": ab["avg_ms"], "peak_source": tc_src}
