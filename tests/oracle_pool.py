@@ -63,3 +63,39 @@ def oracle_outputs(name, lengths, gains="ones", overrides=(), shared_kv=False, t
                 os.environ.pop(k, None)
             else:
                 os.environ[k] = v
+
+
+def _one_bwd(task):
+    from oracle import whale_backward as OB
+    from wukong_hstu_cross_b200 import inputs as I
+    key, b, length, dy_b = task
+    w, lws = _setup(key)
+    _, _, _, shared_kv, tied_gate = key
+    x = I.tokens_of_example(w, b)
+    s = I.states_of_example(w, 0, b, length)
+    dx, ds, dlw = OB.fusion_layer_backward(x, s, lws[0], w.n_heads, w.eps, dy_b, shared_kv=shared_kv,
+                                           tied_gate=tied_gate)
+    return b, dx, ds, dlw
+
+
+def oracle_layer_backward(name, lengths, dy, gains="ones", overrides=(), shared_kv=False, tied_gate=False):
+    """The fp64 VJP of layer 0 for every example (upstream gradient dy [B, N, d]): yields (b, d_tokens,
+    d_states [L_b, d], {parameter: this example's share of its gradient})."""
+    from wukong_hstu_cross_b200 import inputs as I
+    key = (name, tuple(sorted(dict(overrides).items())), gains, shared_kv, tied_gate)
+    w = I.WORKLOADS[name].replace(**dict(overrides))
+    tasks = [(key, b, int(lengths[b]), dy[b]) for b in range(w.batch)]
+    tasks.sort(key=lambda t: -t[2])  # longest first
+    env = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
+    for k in env:
+        os.environ[k] = "1"
+    try:
+        with ProcessPoolExecutor(workers(), mp_context=mp.get_context("spawn")) as ex:
+            for res in ex.map(_one_bwd, tasks, chunksize=1):
+                yield res
+    finally:
+        for k, v in env.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v

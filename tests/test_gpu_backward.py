@@ -155,3 +155,44 @@ def test_stack_backward_matches_oracle(case):
         _check(f"d_states[{l}]", to_np(out["d_states"][l, :p.total_L]), d_st[l], w.dtype)
         for k, v in d_w[l].items():
             _check(f"{k}[{l}]", to_np(out["grads"][l][k]), v, w.dtype)
+
+
+def test_layer_backward_full_size():
+    """The 15k-history layer at full size (B 64, 403 481 history rows, random gains) against the fp64
+    VJP on every element: d_tokens and d_states example by example, and each parameter's gradient (a
+    sum over all examples). The oracle runs per example in a process pool."""
+    from tests import oracle_pool
+    w_name = "hist15k_d512"
+    w = I.WORKLOADS[w_name].replace(n_layers=1)
+    p = Hn.build_problem(w, gains="random")
+    dy = np.random.default_rng(17).standard_normal((w.batch, w.n_tokens, w.d)).astype(np.float32)
+    out = Hn.run_layer_backward(p, 0, torch.from_numpy(dy).cuda())
+    torch.cuda.synchronize()
+    assert W.whale_get_device_error() == 0
+    d_tok = to_np(out["d_tokens"])
+    d_st = to_np(out["d_states"][:p.total_L])
+    lw = p.host_weights[0]
+    d_w = {k: np.zeros(np.shape(v)) for k, v in lw.items() if v is not None}
+    worst = {}
+    seen = 0
+    for b, dx, ds, dlw in oracle_pool.oracle_layer_backward(w_name, p.lengths, dy, gains="random",
+                                                            overrides=(("n_layers", 1),)):
+        lo, hi = int(p.offsets[b]), int(p.offsets[b + 1])
+        _check(f"d_tokens[{b}]", d_tok[b], dx, "bf16")
+        _check(f"d_states[{b}]", d_st[lo:hi], ds, "bf16")
+        for k, v in dlw.items():
+            d_w[k] += v
+        for name, g, r in (("d_tokens", d_tok[b], dx), ("d_states", d_st[lo:hi], ds)):
+            if r.size:
+                worst[name] = max(worst.get(name, 0.0), float((np.abs(g - r) / (2e-2 * (1 + np.abs(r)))).max()))
+        seen += 1
+    assert seen == w.batch
+    for k, v in d_w.items():
+        g = to_np(out[k])
+        _check(k, g, v, "bf16")
+        worst[k] = float((np.abs(g - v) / (2e-2 * (1 + np.abs(v)))).max())
+    path = os.environ.get("WHALE_PARITY_REPORT")
+    if path:
+        with open(path, "a") as fh:
+            fh.write(json.dumps({"backward": f"{w_name} full size (B 64, total_L {p.total_L})",
+                                 "bound": "2e-2*(1+|oracle|)", "max_err_over_bound": worst}) + "\n")
