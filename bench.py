@@ -467,6 +467,29 @@ def time_backward(p, raw_weights, w, total_L, peaks, clocks, stream, reps=10):
                            **roofline_of(fl, nb, ab["avg_ms"], tc, peaks["hbm_gbs"]),
                            "algorithmic_flops_per_launch": fl, "algorithmic_bytes_per_launch": nb,
                            "avg_launch_ms": ab["avg_ms"], "peak_source": tc_src}
+    del ws, grads, d_st
+    # the whole stack's backward (whale_fusion_backward: its forward on the recompute path, then every
+    # layer's backward, last layer first), timed over two calls after one warm-up call
+    if w.n_layers > 1:
+        raw = raw_weights
+        sgrads = [{k: torch.empty(tuple(v.shape), dtype=torch.float32, device=dev) for k, v in lwl.items()
+                   if v is not None and k != "w_kabs"} for lwl in raw]
+        sws = torch.empty(Wb.whale_backward_workspace_size(cfg, p.hint), dtype=torch.uint8, device=dev)
+        s_st = torch.empty(p.states.shape, dtype=p.states.dtype, device=dev)
+
+        def scall():
+            Wb.whale_fusion_backward(cfg, p.tokens, p.states, p.offsets_t, raw, d_out, d_tok, s_st, sgrads, p.hint,
+                                     sws, stream=stream)
+        scall()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(2):
+            scall()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        out["stack"] = {"entry_point": "whale_fusion_backward (all layers, forward recomputed inside)",
+                        "ms": e0.elapsed_time(e1) / 2, "layers": w.n_layers, "calls": 2}
+        del sgrads, sws, s_st
     return out
 
 
@@ -712,6 +735,10 @@ def main():
     bwd = None
     if not args.no_backward:
         bwd = time_backward(p, raw_weights, w, total_L, peaks, clocks, stream, reps=max(3, min(args.steps, 20)))
+        if isinstance(bwd, dict) and "stack" in bwd:
+            tr = ms + bwd["stack"]["ms"]  # one forward (the timed step) and the stack's backward
+            bwd["training_step"] = {"ms": tr, "examples_per_s": world * w.batch / (tr / 1e3),
+                                    "what": "forward step + whale_fusion_backward, per rank"}
 
     # ---------------- end to end: host buffers through the C ABI, copies inside the timed region -----
     e2e = None
