@@ -452,7 +452,7 @@ def time_backward(p, raw_weights, w, total_L, peaks, clocks, stream, reps=10):
     tot = sum(v[1] for v in kern.values()) or 1.0
     kernels = {n: {"launches": c, "avg_ms": t / c, "share": t / tot}
                for n, (c, t) in sorted(kern.items(), key=lambda x: -x[1][1])}
-    out = {"entry_point": "whale_fusion_layer_backward (one layer, forward recomputed inside)", "ms_per_layer": ms,
+    out = {"entry_point": "whale_fusion_layer_backward (one layer, its forward recomputed inside)", "ms_per_layer": ms,
            "reps": reps, "kernels": kernels,
            "launch_order": [[kernel_name(n), round(t, 4)] for n, t in recs]}
     abk = next((k for k in kernels if k.split("<")[0] in ("attn_bwd_tc_kernel", "attn_bwd_kernel")), None)
@@ -487,7 +487,8 @@ def time_backward(p, raw_weights, w, total_L, peaks, clocks, stream, reps=10):
             scall()
         e1.record(stream)
         torch.cuda.synchronize()
-        out["stack"] = {"entry_point": "whale_fusion_backward (all layers, forward recomputed inside)",
+        out["stack"] = {"entry_point": ("whale_fusion_backward (all layers; the forward once, each layer's "
+                                        "activations kept for its backward)"),
                         "ms": e0.elapsed_time(e1) / 2, "layers": w.n_layers, "calls": 2}
         del sgrads, sws, s_st
     return out

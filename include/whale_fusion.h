@@ -311,9 +311,12 @@ whale_status whale_fusion_layer_backward(const whale_config* cfg, const void* to
                                          whale_stream_t stream);
 
 /* The whole stack's backward: the forward is run once more, keeping every layer's input (the
- * residual stream between layers in fp32 and its hi/lo pair, as the forward carries it), then each
- * layer's backward, last layer first, each layer's d_tokens being the upstream gradient of the layer
- * below (the Wukong module between layers is the identity, as in the forward).
+ * residual stream between layers in fp32 and its hi/lo pair, as the forward carries it) and, in bf16
+ * mode, every layer's forward activations (its K|V pair over the history above all, about 4 bytes per
+ * K|V element), then each layer's backward, last layer first, each layer's d_tokens being the upstream
+ * gradient of the layer below (the Wukong module between layers is the identity, as in the forward).
+ * In bf16 mode each layer's forward thus runs once; the fp32 mode recomputes it inside the layer's
+ * backward.
  *   wukong_tokens  device [B, N, d]               H_w of layer 0 (cfg->dtype)
  *   seq_states     device [n_layers, total_L, d]  H_s slab of each layer
  *   weights        HOST array of n_layers raw whale_layer_weights

@@ -1425,6 +1425,35 @@ struct BwdBufs {
   size_t part_floats;
 };
 
+// The forward activations one layer's backward reads (bf16 mode): q and its normalised rows, K|V and
+// the history rows' factors, A and its log-sum-exp, z1 and G, F, UG and the FFN's normalised rows.
+// The stack backward keeps one set per layer so that each layer's forward runs once.
+template <typename Take>
+void act_buffers(const Shape& s, const whale_shape_hint& h, Take take, BwdBufs* b) {
+  const size_t rows = (size_t)h.B * s.N, T = (size_t)h.total_L, d = s.d, Fh = s.Fh;
+  b->lse = take(rows * s.h * 4);
+  b->nq = take(rows * d * 2);
+  b->nq_lo = take(rows * d * 2);
+  b->q = take(rows * d * 2);
+  b->q_lo = take(rows * d * 2);
+  b->kv = take(T * s.kvw * 2);
+  b->kv_lo = take(T * s.kvw * 2);
+  b->rkv = take(T * 4);
+  b->a = take(rows * d * 2);
+  b->a_lo = take(rows * d * 2);
+  if (Fh) {
+    b->z1 = take(rows * Fh * 4);
+    b->g = take(rows * Fh * 2);
+    b->g_lo = take(rows * Fh * 2);
+  }
+  b->f32 = take(rows * d * 4);
+  b->f = take(rows * d * 2);
+  b->f_lo = take(rows * d * 2);
+  b->ug = take(rows * s.ugw * 4);
+  b->nrm = take(rows * d * 2);
+  b->nrm_lo = take(rows * d * 2);
+}
+
 // Buffers of the backward workspace (null pointers when base is null); returns its size in bytes.
 size_t bwd_buffers(const Shape& s, const whale_shape_hint& h, char* base, BwdBufs* b) {
   size_t o = 0;
@@ -1438,37 +1467,26 @@ size_t bwd_buffers(const Shape& s, const whale_shape_hint& h, char* base, BwdBuf
   const size_t e = s.bf16 ? 2 : 4;  // element size of the operand copies
   *b = BwdBufs{};
   if (s.bf16) {
+    act_buffers(s, h, take, b);
     b->x32 = take(rows * d * 4);
     b->xlo = take(rows * d * 2);
     b->attn = take(plan_attention(s, h.B, h.total_L).bytes());
-    b->lse = take(rows * nh * 4);
-  } else {
-    b->r = take(std::max(rows, T) * 4);
-  }
-  b->q = take(rows * d * e);
-  b->kv = take(T * kvw * e);
-  if (s.bf16) {
-    b->q_lo = take(rows * d * 2);
-    b->kv_lo = take(T * kvw * 2);
     b->wg = take(kvw * d * 2);  // W_kv diag(g_kv) as a pair
     b->wg_lo = take(kvw * d * 2);
-    b->rkv = take(T * 4);       // the history rows' RMSNorm factors
   } else {
+    b->r = take(std::max(rows, T) * 4);
+    b->q = take(rows * d * 4);
+    b->kv = take(T * kvw * 4);
     b->sn = take(T * d * 4);
+    b->a = take(rows * d * 4);
+    if (Fh) {
+      b->z1 = take(rows * Fh * 4);
+      b->g = take(rows * Fh * 4);
+    }
+    b->f32 = take(rows * d * 4);
+    b->ug = take(rows * ugw * 4);
+    b->nrm = take(rows * d * 4);
   }
-  b->a = take(rows * d * e);
-  if (s.bf16) b->a_lo = take(rows * d * 2);
-  if (Fh) {
-    b->z1 = take(rows * Fh * 4);
-    b->g = take(rows * Fh * e);
-    if (s.bf16) b->g_lo = take(rows * Fh * 2);
-  }
-  b->f32 = take(rows * d * 4);
-  if (s.bf16) {
-    b->f = take(rows * d * 2);
-    b->f_lo = take(rows * d * 2);
-  }
-  b->ug = take(rows * ugw * 4);
   if (s.bf16) {
     b->dy = take(rows * d * 2);
     b->dy_lo = take(rows * d * 2);
@@ -1479,12 +1497,6 @@ size_t bwd_buffers(const Shape& s, const whale_shape_hint& h, char* base, BwdBuf
   b->dug = take(rows * ugw * e);
   if (s.bf16) b->dug_lo = take(rows * ugw * 2);
   b->dn = take(rows * d * 4);
-  b->nrm = take(rows * d * e);
-  if (s.bf16) {
-    b->nrm_lo = take(rows * d * 2);
-    b->nq = take(rows * d * 2);
-    b->nq_lo = take(rows * d * 2);
-  }
   b->df32 = take(rows * d * 4);
   if (s.bf16) {
     b->df = take(rows * d * 2);
@@ -1650,18 +1662,19 @@ whale_status layer_output_bf16(const Shape& s, const whale_layer_weights& w, con
                    static_cast<const float*>(b.f32), s.d, rows, EPI_RESID, false, 0.f, st);
 }
 
-// One layer's backward in bf16 mode (input as for recompute_bf16).
+// One layer's backward in bf16 mode (input as for recompute_bf16). With recompute false the forward
+// activations in b are those of this layer's input already (the stack backward's forward loop).
 whale_status layer_backward_bf16(const Shape& s, const Stream3& in, const void* slab, const int* offsets,
                                  const whale_layer_weights& w, const float* dy, float* dx, void* ds,
                                  const whale_layer_grads& gr, const whale_shape_hint& h, const BwdBufs& b,
-                                 cudaStream_t st) {
+                                 cudaStream_t st, bool recompute = true) {
   using bf = __nv_bfloat16;
   const long long rows = (long long)h.B * s.N, T = h.total_L;
   const int d = s.d, H = s.H, Fh = s.Fh, ugw = s.ugw, kvw = s.kvw;
   auto F = [](void* p) { return static_cast<float*>(p); };
   const void* x = in.hi;
   const float* x32 = in.f32;
-  WCHECK(recompute_bf16(s, in, slab, offsets, w, h, b, st));
+  if (recompute) WCHECK(recompute_bf16(s, in, slab, offsets, w, h, b, st));
   // ---- S5 backward: SwiGLU FFN ----
   float* part = F(b.part);
   const size_t pc = b.part_floats;
@@ -1855,9 +1868,12 @@ whale_status layer_backward_f32(const Shape& s, const float* x, const float* sla
 
 // Workspace of the stack backward (also enough for one layer): the backward buffers, the forward's
 // workspace for the fp32 mode's layer inputs, every layer's input as a residual-stream tensor (fp32,
-// plus its bf16 pair in bf16 mode), and a ping-pong pair of fp32 token gradients.
+// plus its bf16 pair in bf16 mode), a ping-pong pair of fp32 token gradients and, in bf16 mode, the
+// forward activations of every layer but the first (lb[l]: the backward buffers with layer l's
+// activations; lb[0] is b itself).
 struct StackBwd {
   BwdBufs b;
+  BwdBufs lb[64];
   char* fwd;
   Layout fl;
   Stream3 in[64];
@@ -1886,6 +1902,11 @@ size_t stack_bwd_bytes(const Shape& s, const whale_shape_hint& h, char* base, St
     k.in[l].lo = s.bf16 ? take(rows * s.d * 2) : nullptr;
   }
   for (int i = 0; i < 2; ++i) k.g[i] = reinterpret_cast<float*>(take(rows * s.d * 4));
+  if (s.bf16)
+    for (int l = 0; l < nl; ++l) {
+      k.lb[l] = k.b;
+      if (l > 0) act_buffers(s, h, [&](size_t bytes) -> void* { return take(bytes); }, &k.lb[l]);
+    }
   return o;
 }
 
@@ -2419,12 +2440,13 @@ whale_status whale_fusion_backward(const whale_config* cfg, const void* tokens, 
   // forward, keeping every layer's input (the residual stream: fp32 and, in bf16 mode, its pair)
   if (s.bf16) {
     // the recompute path of the backward (hi/lo pairs, raw weights, K|V as pairs), so that every
-    // layer's input carries the precision its gradients need
+    // layer's input carries the precision its gradients need; each layer's activations stay in
+    // lb[l] for its backward below
     WCHECK(pair_from_bf16(tokens, k.in[0].f32, k.in[0].lo, rows * s.d, st));
     CUCHECK(cudaMemcpyAsync(k.in[0].hi, tokens, (size_t)rows * s.d * 2, cudaMemcpyDeviceToDevice, st));
-    for (int l = 0; l + 1 < s.layers; ++l) {
-      WCHECK(recompute_bf16(s, k.in[l], slab(l), seq_offsets, weights[l], *hint, k.b, st));
-      WCHECK(layer_output_bf16(s, weights[l], *hint, k.b, k.in[l + 1], st));
+    for (int l = 0; l < s.layers; ++l) {
+      WCHECK(recompute_bf16(s, k.in[l], slab(l), seq_offsets, weights[l], *hint, k.lb[l], st));
+      if (l + 1 < s.layers) WCHECK(layer_output_bf16(s, weights[l], *hint, k.lb[l], k.in[l + 1], st));
     }
   } else {
     CUCHECK(cudaMemcpyAsync(k.in[0].f32, tokens, (size_t)rows * s.d * 4, cudaMemcpyDeviceToDevice, st));
@@ -2437,7 +2459,8 @@ whale_status whale_fusion_backward(const whale_config* cfg, const void* tokens, 
     float* dx = l == 0 ? d_tokens : k.g[l & 1];
     void* dsl = T > 0 ? static_cast<char*>(d_states) + l * slab_bytes : nullptr;
     if (s.bf16)
-      WCHECK(layer_backward_bf16(s, k.in[l], slab(l), seq_offsets, weights[l], g, dx, dsl, grads[l], *hint, k.b, st));
+      WCHECK(layer_backward_bf16(s, k.in[l], slab(l), seq_offsets, weights[l], g, dx, dsl, grads[l], *hint, k.lb[l], st,
+                                 false));
     else
       WCHECK(layer_backward_f32(s, k.in[l].f32, reinterpret_cast<const float*>(slab(l)), seq_offsets, weights[l], g, dx,
                                 static_cast<float*>(dsl), grads[l], *hint, k.b, st));
