@@ -8,19 +8,23 @@
 // dV of a block are complete inside the CTA and only dQ (N d_h values per chunk) is added to global
 // memory with fp32 atomics.
 //
-// Per block, with every operand a hi/lo bf16 pair and every product three MMAs (hi hi, lo hi, hi lo):
+// Per block, with every operand a hi/lo bf16 pair:
 //   tensor memory: S^T | dP^T (double-buffered, 32 + 32 columns), dV and dK (double-buffered, 64
-//   columns each) and the running dQ^T (64 columns; lanes 0-63 = d_h, lanes 64-127 unused products
-//   of the second MN group), all fp32;
-//   shared memory: the K|V block ring (TMA, 128-byte swizzle), and P^T and dS^T written by the
-//   epilogue threads in the K-major 128-byte-swizzled layout the MMA reads — the same bytes serve
-//   dS^T as the MN-major B operand of dQ^T.
+//   columns each) and the running dQ^T (64 x 128: see below), all fp32;
+//   shared memory: the K|V block ring (TMA, 128-byte swizzle); P^T and dS^T written by the softmax
+//   threads in the K-major 128-byte-swizzled layout the MMA reads, each as one tile whose 128-byte
+//   rows hold the hi half (queries 0-31) then the lo half; and the dK|dV drain's staging.
+// S^T, dP^T, dV and dK take three MMAs per k-step (hi hi, lo hi, hi lo). dQ^T takes one: its A
+// operand is the K tile MN-major with M = 128, whose two 64-element MN groups are the K hi and K lo
+// tiles (adjacent in the stage), and its B operand the dS^T tile MN-major with N = 64 (the hi and lo
+// halves side by side), so TMEM lane (g 64 + m), column (h 32 + n) holds K_g^T dS_h for d_h index m
+// and query n, and dQ is the sum of the four (g, h) products.
 // Warp roles (320 threads): warp 0 TMA producer, warp 1 TMEM allocation + MMA issue (one thread),
 // warps 2..5 the softmax backward (the next block's while a block's MMAs run), warps 6..9 the dK|dV
-// drain while the next block is computed: rows scaled by r, split into pairs, written into the block's
-// own K|V stage (free once the block's MMAs are done) and stored from there with tensor stores (boxes
-// of 32 rows x 64 columns: tmDKV, tmDKVlo); the producer refills the stage after those stores have
-// read it. Thread i of TMEM lane quadrant q owns block row 32q + i.
+// drain while the next block is computed: rows scaled by r, split into pairs, written into the warp's
+// staging and stored from there with tensor stores (boxes of 32 rows x 64 columns: tmDKV, tmDKVlo).
+// A K|V stage is refilled as soon as the MMAs of its block are complete. Thread i of TMEM lane
+// quadrant q owns block row 32q + i.
 // Rows past the chunk (the next example's, or past the states) and queries past N are read but give
 // P = 0 and dS = 0: lse is +inf for the missing queries and the rows past the chunk are masked.
 #pragma once
@@ -36,8 +40,9 @@ struct AttnBwdTcSmem {
   static constexpr uint32_t TILE_KV = 128 * 128;  // 128 rows x 64 d_h bf16
   static constexpr uint32_t OFF_Q = 0;            // q, q_lo, da, da_lo
   static constexpr uint32_t OFF_KV = 4 * TILE_Q;  // [2 stages][k, k_lo, v, v_lo]
-  static constexpr uint32_t OFF_STG = OFF_KV + 2 * 4 * TILE_KV;  // p, p_lo, ds, ds_lo
-  static constexpr uint32_t OFF_LSE = OFF_STG + 4 * TILE_KV;     // lse[32], delta[32]
+  static constexpr uint32_t OFF_STG = OFF_KV + 2 * 4 * TILE_KV;  // [p | p_lo], [ds | ds_lo]
+  static constexpr uint32_t OFF_DST = OFF_STG + 2 * TILE_KV;     // drain: [4 warps][hi 32 rows | lo 32 rows]
+  static constexpr uint32_t OFF_LSE = OFF_DST + 4 * 8192;        // lse[32], delta[32]
   static constexpr uint32_t OFF_BAR = OFF_LSE + 256;
   static constexpr uint32_t BYTES = OFF_BAR + 256 + 1024;  // + alignment slack
 };
@@ -58,11 +63,11 @@ __global__ void __launch_bounds__(kAttnBwdTcThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* q_full = bars;           // queries landed
   uint64_t* kv_full = bars + 1;      // [2]
-  uint64_t* kv_empty = bars + 3;     // [2] the stage's dK|dV stores have read it (4 drain warps)
   uint64_t* sp_full = bars + 5;      // [2] S^T | dP^T computed
   uint64_t* sp_empty = bars + 7;     // [2] S^T | dP^T read by the 4 epilogue warps
   uint64_t* pd_full = bars + 9;      // P^T, dS^T staged by the 4 softmax warps
-  uint64_t* dvk_full = bars + 10;    // [2] dV, dK (and dQ^T so far) computed; the staging is free again
+  uint64_t* dvk_full = bars + 10;    // [2] dV, dK (and dQ^T so far) computed; the staging and the K|V
+                                     //     stage of the block are free again
   uint64_t* dvk_empty = bars + 12;   // [2] dV, dK read by the 4 drain warps
   uint64_t* fin = bars + 14;         // every MMA issued has completed (unwinding)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
@@ -74,7 +79,6 @@ __global__ void __launch_bounds__(kAttnBwdTcThreads, 1)
     mbar_init(q_full, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], 4);
       mbar_init(&sp_full[i], 1);
       mbar_init(&sp_empty[i], 4);
     }
@@ -130,7 +134,7 @@ __global__ void __launch_bounds__(kAttnBwdTcThreads, 1)
   const uint32_t t_sp = tmem_base;          // [2][S^T 32 | dP^T 32]
   const uint32_t t_dv = tmem_base + 128;    // [2][64]
   const uint32_t t_dk = tmem_base + 256;    // [2][64]
-  const uint32_t t_dq = tmem_base + 384;    // 64 (dQ^T: lanes = d_h, columns = queries)
+  const uint32_t t_dq = tmem_base + 384;    // 64 (dQ^T: lanes = (K hi | K lo) x d_h, columns = (dS hi | dS lo) x queries)
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -149,7 +153,7 @@ __global__ void __launch_bounds__(kAttnBwdTcThreads, 1)
       int issued = 0;
       for (int blk = 0; blk < nblk; ++blk, ++issued) {
         const int s = blk & 1, u = blk >> 1;
-        if (blk >= 2 && !mbar_wait(&kv_empty[s], (u - 1) & 1, abort_flag)) break;
+        if (blk >= 2 && !mbar_wait(&dvk_full[s], (u - 1) & 1, abort_flag)) break;  // block blk - 2 is done
         uint8_t* st = smem + L::OFF_KV + s * 4 * L::TILE_KV;
         const int r0 = (int)(k0 + 128ll * blk);
         mbar_arrive_expect_tx(&kv_full[s], kv_bytes);
@@ -176,7 +180,7 @@ __global__ void __launch_bounds__(kAttnBwdTcThreads, 1)
       const uint32_t q_s = smem_u32(smem + L::OFF_Q);
       const uint32_t ql_s = q_s + L::TILE_Q, da_s = q_s + 2 * L::TILE_Q, dal_s = q_s + 3 * L::TILE_Q;
       const uint32_t stg = smem_u32(smem + L::OFF_STG);
-      const uint32_t p_s = stg, pl_s = stg + L::TILE_KV, ds_s = stg + 2 * L::TILE_KV, dsl_s = stg + 3 * L::TILE_KV;
+      const uint32_t p_s = stg, pl_s = stg + 64, ds_s = stg + L::TILE_KV, dsl_s = stg + L::TILE_KV + 64;
       bool ok = mbar_wait(q_full, 0, abort_flag);
       // S^T and dP^T of block `blk` into buffer blk & 1
       auto issue_sp = [&](int blk) -> bool {
@@ -205,7 +209,7 @@ __global__ void __launch_bounds__(kAttnBwdTcThreads, 1)
       if (ok) ok = issue_sp(0);
       int sp_next = 1;  // the next block whose S^T | dP^T is to be issued
       // S^T | dP^T of the next block goes ahead of this block's products when its K|V stage has landed
-      // (the stage is refilled only after the dK|dV stores of two blocks back have read it)
+      // (the stage is refilled only after the MMAs of two blocks back are complete)
       auto sp_ready = [&](int nb) {
         return mbar_test(&kv_full[nb & 1], (nb >> 1) & 1) &&
                (nb < 2 || mbar_test(&sp_empty[nb & 1], ((nb >> 1) - 1) & 1));
@@ -220,8 +224,7 @@ __global__ void __launch_bounds__(kAttnBwdTcThreads, 1)
         if (blk >= 2 && !mbar_wait(&dvk_empty[db], ((blk >> 1) - 1) & 1, abort_flag)) break;
         tc_fence_after();
         const int s = blk & 1;
-        const uint32_t kst = smem_u32(smem + L::OFF_KV + s * 4 * L::TILE_KV);
-        const uint32_t k_s = kst, kl_s = kst + L::TILE_KV;
+        const uint32_t k_s = smem_u32(smem + L::OFF_KV + s * 4 * L::TILE_KV);
         // dV = P^T dA and dK = (dS^T / sqrt(d_h)) Q: K = 32 queries (two k-steps); with shared K = V
         // both accumulate into dV's columns
         const uint32_t d_v = t_dv + db * 64;
@@ -241,17 +244,14 @@ __global__ void __launch_bounds__(kAttnBwdTcThreads, 1)
           umma_f16(d_k, sdesc_k_sw128(dsl_s + kk * 32), bq, id_kv, 1u);
           umma_f16(d_k, sdesc_k_sw128(ds_s + kk * 32), bql, id_kv, 1u);
         }
-        // dQ^T += K^T (dS^T / sqrt(d_h)): A = the K tile MN-major (M = d_h; its second 64-element MN
-        // group, lanes 64-127, reads the K lo tile and is not used), B = dS^T MN-major (N = queries,
-        // 64 wide: columns 32-63 are not used), K = the block's 128 rows
+        // dQ^T += K^T (dS^T / sqrt(d_h)), all four hi/lo products in one MMA per k-step: A = the K
+        // tile MN-major (M = 128: the K hi tile's 64 d_h, then the K lo tile's, one tile apart), B =
+        // the dS^T tile MN-major (N = 64: its hi then lo queries), K = the block's 128 rows
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t acc = (blk > 0 || kk > 0) ? 1u : 0u;
-          const uint64_t bds = sdesc_mn_sw128(ds_s + kk * 2048, 8192, 1024);
-          const uint64_t bdsl = sdesc_mn_sw128(dsl_s + kk * 2048, 8192, 1024);
-          umma_f16(t_dq, sdesc_mn_sw128(k_s + kk * 2048, L::TILE_KV, 1024), bds, id_dq, acc);
-          umma_f16(t_dq, sdesc_mn_sw128(kl_s + kk * 2048, L::TILE_KV, 1024), bds, id_dq, 1u);
-          umma_f16(t_dq, sdesc_mn_sw128(k_s + kk * 2048, L::TILE_KV, 1024), bdsl, id_dq, 1u);
+          umma_f16(t_dq, sdesc_mn_sw128(k_s + kk * 2048, L::TILE_KV, 1024), sdesc_mn_sw128(ds_s + kk * 2048, 8192, 1024),
+                   id_dq, acc);
         }
         umma_commit(&dvk_full[db]);  // dV, dK, dQ^T so far; the staging tiles and the K|V stage are free
         if (sp_next == blk + 1 && sp_next < nblk) {
@@ -310,14 +310,14 @@ __global__ void __launch_bounds__(kAttnBwdTcThreads, 1)
       // the staging is free once the previous block's MMAs have completed
       if (blk >= 1 && !mbar_wait(&dvk_full[(blk - 1) & 1], ((blk - 1) >> 1) & 1, abort_flag)) break;
       // P^T and dS^T in the K-major 128-byte-swizzled layout (row rloc: 16-byte chunk c at position
-      // c ^ (rloc % 8)); queries 0..31 fill chunks 0..3
+      // c ^ (rloc % 8)); the hi halves of queries 0..31 fill chunks 0..3, the lo halves chunks 4..7
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const uint32_t off = ((uint32_t)c ^ sw) * 16;
-        *reinterpret_cast<uint4*>(rowp + 0 * L::TILE_KV + off) = make_uint4(ph[4 * c], ph[4 * c + 1], ph[4 * c + 2], ph[4 * c + 3]);
-        *reinterpret_cast<uint4*>(rowp + 1 * L::TILE_KV + off) = make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
-        *reinterpret_cast<uint4*>(rowp + 2 * L::TILE_KV + off) = make_uint4(dh[4 * c], dh[4 * c + 1], dh[4 * c + 2], dh[4 * c + 3]);
-        *reinterpret_cast<uint4*>(rowp + 3 * L::TILE_KV + off) = make_uint4(dl[4 * c], dl[4 * c + 1], dl[4 * c + 2], dl[4 * c + 3]);
+        const uint32_t oh = ((uint32_t)c ^ sw) * 16, ol = ((uint32_t)(c + 4) ^ sw) * 16;
+        *reinterpret_cast<uint4*>(rowp + oh) = make_uint4(ph[4 * c], ph[4 * c + 1], ph[4 * c + 2], ph[4 * c + 3]);
+        *reinterpret_cast<uint4*>(rowp + ol) = make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
+        *reinterpret_cast<uint4*>(rowp + L::TILE_KV + oh) = make_uint4(dh[4 * c], dh[4 * c + 1], dh[4 * c + 2], dh[4 * c + 3]);
+        *reinterpret_cast<uint4*>(rowp + L::TILE_KV + ol) = make_uint4(dl[4 * c], dl[4 * c + 1], dl[4 * c + 2], dl[4 * c + 3]);
       }
       fence_proxy_async_smem();  // the MMAs read the staging through the async proxy
       __syncwarp();
@@ -331,16 +331,17 @@ __global__ void __launch_bounds__(kAttnBwdTcThreads, 1)
     const int rloc = qd * 32 + lane;
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
     const int nw = a.shared_kv ? 1 : 2;
-    const uint32_t sw = (uint32_t)(rloc & 7);
+    const uint32_t sw = (uint32_t)(lane & 7);
+    uint8_t* dst = smem + L::OFF_DST + qd * 8192;  // this warp's staging: hi then lo, 32 rows of 128 bytes
+    uint8_t* rowp = dst + lane * 128;
     int done = 0;  // blocks drained (all of them unless a wait ran out)
     for (int blk = 0; blk < nblk; ++blk) {
-      const int db = blk & 1, s = blk & 1;
+      const int db = blk & 1;
       const long long row = k0 + 128ll * blk + rloc;
       const bool row_ok = row < k1;
       const float rs = (a.row_scale && row_ok) ? a.row_scale[row] : 1.0f;  // before the wait
       const long long slice0 = k0 + 128ll * blk + qd * 32;
       const bool full_slice = slice0 + 32 <= k1;  // uniform across the warp
-      uint8_t* rowp = smem + L::OFF_KV + s * 4 * L::TILE_KV + rloc * 128;  // this row of the block's stage
       if (!mbar_wait(&dvk_full[db], (blk >> 1) & 1, abort_flag)) break;
       tc_fence_after();
 #pragma unroll 1
@@ -352,6 +353,15 @@ __global__ void __launch_bounds__(kAttnBwdTcThreads, 1)
         tmem_ld_32x32b_x32(tsrc + lane_off, v0);
         tmem_ld_32x32b_x32(tsrc + 32 + lane_off, v1);
         tmem_ld_wait();
+        if (which == nw - 1) {  // this TMEM buffer may take block blk + 2
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&dvk_empty[db]);
+        }
+        if (full_slice) {  // the staging's previous stores have read it
+          if (lane == 0) bulk_wait_read<0>();
+          __syncwarp();
+        }
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           const uint32_t* v = c < 4 ? v0 + 8 * c : v1 + 8 * (c - 4);
@@ -359,49 +369,59 @@ __global__ void __launch_bounds__(kAttnBwdTcThreads, 1)
 #pragma unroll
           for (int j = 0; j < 4; ++j)
             split2(__uint_as_float(v[2 * j]) * rs, __uint_as_float(v[2 * j + 1]) * rs, h[j], l[j]);
-          if (full_slice) {  // 128-byte-swizzled rows of the stage's tiles (dK hi, dK lo, dV hi, dV lo)
+          if (full_slice) {  // 128-byte-swizzled rows of the staging (hi, lo)
             const uint32_t off = ((uint32_t)c ^ sw) * 16;
-            *reinterpret_cast<uint4*>(rowp + (2 * which) * L::TILE_KV + off) = make_uint4(h[0], h[1], h[2], h[3]);
-            *reinterpret_cast<uint4*>(rowp + (2 * which + 1) * L::TILE_KV + off) = make_uint4(l[0], l[1], l[2], l[3]);
+            *reinterpret_cast<uint4*>(rowp + off) = make_uint4(h[0], h[1], h[2], h[3]);
+            *reinterpret_cast<uint4*>(rowp + 4096 + off) = make_uint4(l[0], l[1], l[2], l[3]);
           } else if (row_ok) {
             reinterpret_cast<uint4*>(a.dkv + row * a.kvw + gcol)[c] = make_uint4(h[0], h[1], h[2], h[3]);
             reinterpret_cast<uint4*>(a.dkv_lo + row * a.kvw + gcol)[c] = make_uint4(l[0], l[1], l[2], l[3]);
           }
         }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&dvk_empty[db]);  // this TMEM buffer may take block blk + 2
-      if (full_slice) {
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          uint8_t* st = smem + L::OFF_KV + s * 4 * L::TILE_KV + qd * 4096;
-          for (int which = 0; which < nw; ++which) {
-            const int gcol = which == 0 ? colk : colv;
-            tma_store_2d(&tmDKV, st + (2 * which) * L::TILE_KV, gcol, (int)slice0);
-            tma_store_2d(&tmDKVlo, st + (2 * which + 1) * L::TILE_KV, gcol, (int)slice0);
+        if (full_slice) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmDKV, dst, gcol, (int)slice0);
+            tma_store_2d(&tmDKVlo, dst + 4096, gcol, (int)slice0);
+            bulk_commit();
           }
-          bulk_commit();
-          bulk_wait_read<0>();  // the stores have read the stage
         }
-        __syncwarp();
       }
-      if (lane == 0) mbar_arrive(&kv_empty[s]);  // the producer may refill the stage
       done = blk + 1;
     }
-    if (lane == 0) bulk_wait<0>();  // this warp's tensor stores are complete
+    if (lane == 0) bulk_wait<0>();  // this warp's tensor stores are complete: its staging is free
     __syncwarp();
-    // dq += this chunk's share: dQ^T lanes 0..63 (d_h) x columns 0..31 (queries), read by the warps of
-    // lane quadrants 0 and 1 once the last block's MMAs are complete (its dvk_full, waited above)
-    if (done == nblk && *abort_flag == 0 && qd < 2) {
+    // dq += this chunk's share once the last block's MMAs are complete (its dvk_full, waited above):
+    // quadrant qd holds d_h indices 32 (qd % 2) + lane of K hi (qd < 2) or K lo (qd >= 2); columns
+    // 0..31 are the dS hi products of queries 0..31, columns 32..63 the dS lo ones. Quadrants 2 and 3
+    // hand their sums to quadrants 0 and 1 through their staging; those add them to dq.
+    const bool ok_dq = done == nblk && *abort_flag == 0;
+    float* xch = reinterpret_cast<float*>(smem + L::OFF_DST + ((qd & 1) + 2) * 8192);  // [32 queries][32 lanes]
+    int* xok = reinterpret_cast<int*>(xch + 32 * 32);
+    float sum[32];
+    if (ok_dq) {
       tc_fence_after();
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(t_dq + lane_off, v);
+      uint32_t v0[32], v1[32];
+      tmem_ld_32x32b_x32(t_dq + lane_off, v0);
+      tmem_ld_32x32b_x32(t_dq + 32 + lane_off, v1);
       tmem_ld_wait();
+#pragma unroll
+      for (int n = 0; n < 32; ++n) sum[n] = __uint_as_float(v0[n]) + __uint_as_float(v1[n]);
+    }
+    if (qd >= 2) {
+      if (ok_dq) {
+#pragma unroll
+        for (int n = 0; n < 32; ++n) xch[n * 32 + lane] = sum[n];
+      }
+      if (lane == 0) *xok = ok_dq ? 1 : 0;
+    }
+    named_bar_sync(2, 128);  // the four drain warps (every one reaches it)
+    if (qd < 2 && ok_dq && *xok) {
       const int m = qd * 32 + lane;  // d_h index
-      for (int n = 0; n < a.N && n < 32; ++n)
-        atomicAdd(a.dq + ((long long)b * a.N + n) * a.d + colk + m, __uint_as_float(v[n]));
+#pragma unroll
+      for (int n = 0; n < 32; ++n)
+        if (n < a.N) atomicAdd(a.dq + ((long long)b * a.N + n) * a.d + colk + m, sum[n] + xch[n * 32 + lane]);
     }
   }
 
