@@ -44,6 +44,7 @@ struct AttnBwdArgs {
   const float* delta;        // [B*N, h]
   const int* offsets;        // [B+1]
   const int* cstart;         // [B+1] first chunk of each example; cstart[B] = number of chunks
+  int chunk;                 // history rows per chunk (the tensor-core kernel; the other takes kBwdChunk)
   float* dq;                 // [B*N, d] fp32, zero at launch (atomics)
   __nv_bfloat16 *dkv, *dkv_lo;  // [total_L, kvw]: dK in columns [0, d), dV from v_col0 (shared K = V: dK + dV)
   const float* row_scale;     // [total_L] or null: dK and dV of history row t are stored times row_scale[t]
@@ -114,28 +115,54 @@ __global__ void __launch_bounds__(1024) chunk_starts_kernel(const int* __restric
 }
 
 // delta[row, j] = sum over head j's columns of da * a (a = a_hi + a_lo, the forward's output as a
-// bf16 pair), and da as a bf16 pair: da32 fp32 with row stride ld_da.
+// bf16 pair), and da as a bf16 pair: da32 fp32 with row stride ld_da. A thread takes 8 consecutive
+// columns; the d_h / 8 threads of one (row, head) are consecutive lanes of one warp (d_h / 8 a power
+// of two dividing 32) and add their partial sums with shuffles.
 __global__ void attn_bwd_prep_kernel(const float* __restrict__ da32, long long ld_da, const __nv_bfloat16* __restrict__ a_hi,
                                      const __nv_bfloat16* __restrict__ a_lo, long long rows, int d, int n_heads,
                                      float* __restrict__ delta, __nv_bfloat16* __restrict__ da_hi,
                                      __nv_bfloat16* __restrict__ da_lo) {
   pdl_wait();
   pdl_trigger();
-  const int dh = d / n_heads;
-  const long long n = rows * n_heads;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
-    const long long r = i / n_heads;
-    const int j = (int)(i - r * n_heads);
+  const int gph = (d / n_heads) >> 3;  // threads per (row, head)
+  const int cg = d >> 3;
+  const long long n = rows * cg;
+  const int lane = threadIdx.x & 31;
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  // warp-uniform trip count: every lane of a warp takes part in the shuffles
+  for (long long base = (long long)blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < n; base += stride) {
+    const long long i = base + lane;
+    const bool act = i < n;
     float s = 0.f;
-    for (int c = j * dh; c < (j + 1) * dh; ++c) {
-      const float g = da32[r * ld_da + c];
-      const float av = __bfloat162float(a_hi[r * d + c]) + (a_lo ? __bfloat162float(a_lo[r * d + c]) : 0.f);
-      s = fmaf(g, av, s);
-      const __nv_bfloat16 gh = __float2bfloat16_rn(g);
-      da_hi[r * d + c] = gh;
-      da_lo[r * d + c] = __float2bfloat16_rn(g - __bfloat162float(gh));
+    long long r = 0;
+    int c = 0;
+    if (act) {
+      r = n < (1ll << 31) ? (long long)((unsigned)i / (unsigned)cg) : i / cg;
+      c = (int)(i - r * cg) * 8;
+      const float4 g0 = *reinterpret_cast<const float4*>(da32 + r * ld_da + c);
+      const float4 g1 = *reinterpret_cast<const float4*>(da32 + r * ld_da + c + 4);
+      const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+      const uint4 ah = *reinterpret_cast<const uint4*>(a_hi + r * d + c);
+      const uint4 al = a_lo ? *reinterpret_cast<const uint4*>(a_lo + r * d + c) : make_uint4(0u, 0u, 0u, 0u);
+      const uint32_t wh[4] = {ah.x, ah.y, ah.z, ah.w}, wl[4] = {al.x, al.y, al.z, al.w};
+      uint32_t h[4], l[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        // bf16 -> fp32: the bf16 bits are the high half of the fp32 word
+        const float a0 = __uint_as_float(wh[j] << 16) + __uint_as_float(wl[j] << 16);
+        const float a1 = __uint_as_float(wh[j] & 0xffff0000u) + __uint_as_float(wl[j] & 0xffff0000u);
+        s = fmaf(g[2 * j], a0, s);
+        s = fmaf(g[2 * j + 1], a1, s);
+        const __nv_bfloat162 gh = __floats2bfloat162_rn(g[2 * j], g[2 * j + 1]);
+        h[j] = *reinterpret_cast<const uint32_t*>(&gh);
+        const float2 gf = __bfloat1622float2(gh);
+        l[j] = pack_bf16x2(g[2 * j] - gf.x, g[2 * j + 1] - gf.y);
+      }
+      *reinterpret_cast<uint4*>(da_hi + r * d + c) = make_uint4(h[0], h[1], h[2], h[3]);
+      *reinterpret_cast<uint4*>(da_lo + r * d + c) = make_uint4(l[0], l[1], l[2], l[3]);
     }
-    delta[i] = s;
+    for (int o = gph >> 1; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (act && (lane & (gph - 1)) == 0) delta[r * n_heads + c / (d / n_heads)] = s;
   }
 }
 

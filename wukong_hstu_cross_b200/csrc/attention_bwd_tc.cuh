@@ -3,7 +3,7 @@
 //   S^T = K Q^T,  dP^T = V dA^T,  P^T = 2^(S^T log2(e)/sqrt(d_h) - lse),  dS^T = P^T (dP^T - delta),
 //   dV = P^T dA,  dK = (dS^T / sqrt(d_h)) Q,  dQ^T += K^T (dS^T / sqrt(d_h)).
 // KV-parallel (gist.science technical summary of WHALE, section 2.2, Asymmetric Backward Variants):
-// a CTA owns one head of a chunk of up to 1024 history rows of one example, keeps the example's
+// a CTA owns one head of a chunk of history rows of one example (kBwdChunkTc rows at most), keeps the example's
 // queries (q, dA as bf16 pairs) in shared memory and walks the chunk in blocks of 128 rows, so dK and
 // dV of a block are complete inside the CTA and only dQ (N d_h values per chunk) is added to global
 // memory with fp32 atomics.
@@ -34,6 +34,8 @@
 #include "ptx.cuh"
 
 namespace whale {
+
+constexpr int kBwdChunkTc = 2048;  // history rows per CTA (sixteen blocks of 128)
 
 struct AttnBwdTcSmem {
   static constexpr uint32_t TILE_Q = 32 * 128;    // 32 queries x 64 d_h bf16
@@ -123,8 +125,8 @@ __global__ void __launch_bounds__(kAttnBwdTcThreads, 1)
     const long long lo_b = clampo(b);
     long long hi_b = clampo(b + 1);
     if (hi_b < lo_b) hi_b = lo_b;
-    k0 = lo_b + (long long)(chunk - a.cstart[b]) * kBwdChunk;
-    k1 = min(hi_b, k0 + kBwdChunk);
+    k0 = lo_b + (long long)(chunk - a.cstart[b]) * a.chunk;
+    k1 = min(hi_b, k0 + a.chunk);
     active = k0 < k1;
   }
   const int nblk = active ? (int)((k1 - k0 + 127) / 128) : 0;

@@ -25,18 +25,59 @@ __device__ __forceinline__ float silu_grad_f(float z) {
   return s * (1.0f + z * (1.0f - s));
 }
 
+// The element-wise kernels below take 8 consecutive values per thread and step (32-byte fp32 and
+// 16-byte bf16 accesses), so that enough bytes are in flight per SM to approach the HBM bandwidth.
+__device__ __forceinline__ void ld8f(const float* p, float (&v)[8]) {
+  const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void st8f(float* p, const float (&v)[8]) {
+  reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+  reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+// bf16 hi = bf16(v) and lo = bf16(v - hi) of 8 values, each as one 16-byte word
+__device__ __forceinline__ void split8(const float (&v)[8], uint4& hi, uint4& lo) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const __nv_bfloat162 hh = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+    h[j] = *reinterpret_cast<const uint32_t*>(&hh);
+    const float2 hf = __bfloat1622float2(hh);
+    l[j] = pack_bf16x2(v[2 * j] - hf.x, v[2 * j + 1] - hf.y);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+// Writes 8 values at element offset idx of any of: fp32, bf16 hi, bf16 lo (each may be null).
+__device__ __forceinline__ void put8(long long idx, const float (&v)[8], float* f32, __nv_bfloat16* hi,
+                                     __nv_bfloat16* lo) {
+  if (f32) st8f(f32 + idx, v);
+  if (hi) {
+    uint4 h, l;
+    split8(v, h, l);
+    *reinterpret_cast<uint4*>(hi + idx) = h;
+    if (lo) *reinterpret_cast<uint4*>(lo + idx) = l;
+  }
+}
+// i / m for the index range of one launch (32-bit division when the range allows)
+__device__ __forceinline__ long long div_idx(long long i, long long m, long long n) {
+  return n < (1ll << 31) ? (long long)((unsigned)i / (unsigned)m) : i / m;
+}
+
 // x (fp32, row stride ldx) -> bf16 hi = bf16(x) and lo = bf16(x - hi) (lo may be null), row stride ldo.
+// cols, ldx and ldo multiples of 8.
 __global__ void split_pair_kernel(const float* __restrict__ x, long long ldx, __nv_bfloat16* __restrict__ hi,
                                   __nv_bfloat16* __restrict__ lo, long long ldo, long long rows, int cols) {
   pdl_wait();
   pdl_trigger();
-  const long long n = rows * cols;
+  const int cg = cols >> 3;
+  const long long n = rows * cg;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
-    const long long r = i / cols, c = i - r * cols;
-    const float v = x[r * ldx + c];
-    const __nv_bfloat16 h = __float2bfloat16_rn(v);
-    hi[r * ldo + c] = h;
-    if (lo) lo[r * ldo + c] = __float2bfloat16_rn(v - __bfloat162float(h));
+    const long long r = div_idx(i, cg, n);
+    const int c = (int)(i - r * cg) * 8;
+    float v[8];
+    ld8f(x + r * ldx + c, v);
+    put8(r * ldo + c, v, nullptr, hi, lo);
   }
 }
 
@@ -45,9 +86,17 @@ __global__ void silu_pair_kernel(const float* __restrict__ z, float* __restrict_
                                  __nv_bfloat16* __restrict__ lo, long long n) {
   pdl_wait();
   pdl_trigger();
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
-    const float zz = z[i];
-    const float v = zz * sigmoid_f(zz);
+  const long long n8 = n >> 3, t0 = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  for (long long i = t0; i < n8; i += (long long)gridDim.x * blockDim.x) {
+    float v[8];
+    ld8f(z + 8 * i, v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] *= sigmoid_f(v[j]);
+    put8(8 * i, v, g32, hi, lo);
+  }
+  if (t0 < n - 8 * n8) {  // the last n % 8 values
+    const long long i = 8 * n8 + t0;
+    const float v = z[i] * sigmoid_f(z[i]);
     if (g32) g32[i] = v;
     if (hi) {
       const __nv_bfloat16 h = __float2bfloat16_rn(v);
@@ -62,7 +111,17 @@ __global__ void silu_bwd_kernel(const float* __restrict__ dh, const float* __res
                                 __nv_bfloat16* __restrict__ hi, __nv_bfloat16* __restrict__ lo, long long n) {
   pdl_wait();
   pdl_trigger();
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+  const long long n8 = n >> 3, t0 = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  for (long long i = t0; i < n8; i += (long long)gridDim.x * blockDim.x) {
+    float g[8], zz[8];
+    ld8f(dh + 8 * i, g);
+    ld8f(z + 8 * i, zz);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) g[j] *= silu_grad_f(zz[j]);
+    put8(8 * i, g, dz32, hi, lo);
+  }
+  if (t0 < n - 8 * n8) {
+    const long long i = 8 * n8 + t0;
     const float v = dh[i] * silu_grad_f(z[i]);
     if (dz32) dz32[i] = v;
     if (hi) {
@@ -76,7 +135,7 @@ __global__ void silu_bwd_kernel(const float* __restrict__ dh, const float* __res
 // SwiGLU backward. ug: fp32 [rows, ugw] pre-activations ([up | gate], or u alone with a tied gate);
 // dm: fp32 [rows, H] gradient of m = SiLU(gate) * up. Outputs (each may be null): m as bf16 [rows, H],
 // and dug = [dup | dgate] (or du) as fp32 and as a bf16 pair, [rows, ugw]; m also as fp32 (m32) and
-// as the bf16 residue of m_out (m_lo).
+// as the bf16 residue of m_out (m_lo). H a multiple of 8.
 __global__ void swiglu_bwd_kernel(const float* __restrict__ ug, const float* __restrict__ dm, long long rows, int H,
                                   int tied, __nv_bfloat16* __restrict__ m_out, __nv_bfloat16* __restrict__ m_lo,
                                   float* __restrict__ m32,
@@ -85,37 +144,37 @@ __global__ void swiglu_bwd_kernel(const float* __restrict__ ug, const float* __r
   pdl_wait();
   pdl_trigger();
   const int ugw = tied ? H : 2 * H;
-  const long long n = rows * H;
-  auto put = [&](long long idx, float v) {
-    if (dug32) dug32[idx] = v;
-    if (dug_hi) {
-      const __nv_bfloat16 h = __float2bfloat16_rn(v);
-      dug_hi[idx] = h;
-      if (dug_lo) dug_lo[idx] = __float2bfloat16_rn(v - __bfloat162float(h));
-    }
-  };
+  const int hg = H >> 3;
+  const long long n = rows * hg;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
-    const long long r = i / H;
-    const int c = (int)(i - r * H);
-    const float up = ug[r * ugw + c];
-    const float gate = tied ? up : ug[r * ugw + H + c];
-    const float s = sigmoid_f(gate);
-    const float sg = gate * s;  // silu(gate)
-    const float g = dm[i];
-    const float mv = sg * up;
-    if (m_out) {
-      const __nv_bfloat16 mh = __float2bfloat16_rn(mv);
-      m_out[i] = mh;
-      if (m_lo) m_lo[i] = __float2bfloat16_rn(mv - __bfloat162float(mh));
-    }
-    if (m32) m32[i] = mv;
-    const float dup = g * sg;
-    const float dgate = g * up * s * (1.0f + gate * (1.0f - s));
+    const long long r = div_idx(i, hg, n);
+    const int c = (int)(i - r * hg) * 8;
+    float up[8], gate[8], g[8];
+    ld8f(ug + r * ugw + c, up);
     if (tied) {
-      put(r * ugw + c, dup + dgate);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) gate[j] = up[j];
     } else {
-      put(r * ugw + c, dup);
-      put(r * ugw + H + c, dgate);
+      ld8f(ug + r * ugw + H + c, gate);
+    }
+    ld8f(dm + r * H + c, g);
+    float mv[8], dup[8], dgate[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float sg0 = sigmoid_f(gate[j]);
+      const float sg = gate[j] * sg0;  // silu(gate)
+      mv[j] = sg * up[j];
+      dup[j] = g[j] * sg;
+      dgate[j] = g[j] * up[j] * sg0 * (1.0f + gate[j] * (1.0f - sg0));
+    }
+    put8(r * H + c, mv, m32, m_out, m_lo);
+    if (tied) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) dup[j] += dgate[j];
+      put8(r * ugw + c, dup, dug32, dug_hi, dug_lo);
+    } else {
+      put8(r * ugw + c, dup, dug32, dug_hi, dug_lo);
+      put8(r * ugw + H + c, dgate, dug32, dug_hi, dug_lo);
     }
   }
 }
@@ -355,7 +414,31 @@ __global__ void swiglu_pair_kernel(const float* __restrict__ ug, long long rows,
 }
 
 // out[r, c] (row stride ldo) = sum_b part[b][r][c] over b = 0..nb-1 in order (deterministic);
-// part holds nb dense [rows, cols] blocks.
+// part holds nb dense [rows, cols] blocks. sum_partials4_kernel: the same four columns at a time
+// (cols and ldo multiples of 4, out 16-byte aligned), the same sums.
+__global__ void sum_partials4_kernel(const float* __restrict__ part, int nb, long long rows, int cols,
+                                     float* __restrict__ out, long long ldo) {
+  pdl_wait();
+  pdl_trigger();
+  const int c4 = cols >> 2;
+  const long long n4 = rows * c4, nn = rows * cols;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
+    const long long r = div_idx(i, c4, n4);
+    const int c = (int)(i - r * c4) * 4;
+    const float* src = part + r * cols + c;
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int b = 0; b < nb; ++b) {
+      const float4 v = *reinterpret_cast<const float4*>(src + (long long)b * nn);
+      s.x += v.x;
+      s.y += v.y;
+      s.z += v.z;
+      s.w += v.w;
+    }
+    *reinterpret_cast<float4*>(out + r * ldo + c) = s;
+  }
+}
+
 __global__ void sum_partials_kernel(const float* __restrict__ part, int nb, long long rows, int cols,
                                     float* __restrict__ out, long long ldo) {
   pdl_wait();

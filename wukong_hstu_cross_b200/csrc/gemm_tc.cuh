@@ -646,4 +646,28 @@ __global__ void pair_from_bf16_kernel(const __nv_bfloat16* __restrict__ x, float
   }
 }
 
+// The same, 8 values per thread and step (x, x32 and lo 16-byte aligned); the last n % 8 values by
+// the first threads.
+__global__ void pair_from_bf16_8_kernel(const __nv_bfloat16* __restrict__ x, float* __restrict__ x32,
+                                        __nv_bfloat16* __restrict__ lo, long long n) {
+  pdl_wait();
+  pdl_trigger();
+  const long long n8 = n >> 3, t0 = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  for (long long i = t0; i < n8; i += (long long)gridDim.x * blockDim.x) {
+    if (x32) {
+      float f[8];
+      bf16x8_to_f32(reinterpret_cast<const uint4*>(x)[i], f);
+      float4* d = reinterpret_cast<float4*>(x32 + 8 * i);
+      d[0] = make_float4(f[0], f[1], f[2], f[3]);
+      d[1] = make_float4(f[4], f[5], f[6], f[7]);
+    }
+    if (lo) reinterpret_cast<uint4*>(lo)[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  if (t0 < n - 8 * n8) {
+    const long long i = 8 * n8 + t0;
+    if (x32) x32[i] = __bfloat162float(x[i]);
+    if (lo) lo[i] = __float2bfloat16_rn(0.f);
+  }
+}
+
 }  // namespace whale

@@ -729,8 +729,13 @@ whale_status gemm_acc32(const void* a_hi, const void* a_lo, long long lda, bool 
   else r = launch_acc32_bn<64>(split, split_b, a_mn, b_mn, maps, g, tiles, st);
   WCHECK(r);
   if (ks > 1) {
-    const unsigned grid = (unsigned)std::min<long long>(cdiv<long long>(M * N, 256), 8 * kNumSM);
-    WCHECK(launch_pdl(sum_partials_kernel, dim3(grid), dim3(256), 0, st, (const float*)part, ks, M, N, c, ldc));
+    if (N % 4 == 0 && ldc % 4 == 0 && !(reinterpret_cast<uintptr_t>(c) & 15)) {
+      const unsigned grid = (unsigned)std::min<long long>(cdiv<long long>(M * N / 4, 256), 8 * kNumSM);
+      WCHECK(launch_pdl(sum_partials4_kernel, dim3(grid), dim3(256), 0, st, (const float*)part, ks, M, N, c, ldc));
+    } else {
+      const unsigned grid = (unsigned)std::min<long long>(cdiv<long long>(M * N, 256), 8 * kNumSM);
+      WCHECK(launch_pdl(sum_partials_kernel, dim3(grid), dim3(256), 0, st, (const float*)part, ks, M, N, c, ldc));
+    }
   }
   return WHALE_OK;
 }
@@ -751,8 +756,15 @@ whale_status gemm_strided_f32(const float* A, long long sam, long long sak, cons
 inline Opnd opnd(const void* hi, const void* lo, long long ld, int K) { return Opnd{hi, lo, ld, K}; }
 inline Opnd no_opnd() { return Opnd{nullptr, nullptr, 0, 0}; }
 
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
 whale_status pair_from_bf16(const void* x, float* x32, void* lo, long long n, cudaStream_t st) {
   if (n <= 0) return WHALE_OK;
+  if (aligned16(x) && aligned16(x32) && aligned16(lo)) {
+    const unsigned grid = (unsigned)std::min<long long>(cdiv<long long>(cdiv<long long>(n, 8), 256), 8 * kNumSM);
+    return launch_pdl(pair_from_bf16_8_kernel, dim3(grid), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(x),
+                      x32, static_cast<__nv_bfloat16*>(lo), n);
+  }
   const unsigned grid = (unsigned)std::min<long long>(cdiv<long long>(n, 256), 8 * kNumSM);
   return launch_pdl(pair_from_bf16_kernel, dim3(grid), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(x), x32,
                     static_cast<__nv_bfloat16*>(lo), n);
@@ -1317,7 +1329,6 @@ whale_status common_checks(const whale_config* cfg, const whale_shape_hint* hint
   return WHALE_OK;
 }
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 whale_status debug_check(const Shape& s, const int* offsets, const whale_shape_hint& hint, cudaStream_t st) {
   if (!s.debug) return WHALE_OK;
@@ -1566,6 +1577,11 @@ whale_status ew_launch(F kern, long long n, cudaStream_t st, A... args) {
   const unsigned grid = (unsigned)std::min<long long>(cdiv<long long>(n, 256), 8 * kNumSM);
   return launch_pdl(kern, dim3(grid), dim3(256), 0, st, args...);
 }
+// The same for the kernels that take 8 elements per thread and step (n elements in all).
+template <typename F, typename... A>
+whale_status ew8_launch(F kern, long long n, cudaStream_t st, A... args) {
+  return ew_launch(kern, cdiv<long long>(n, 8), st, args...);
+}
 
 template <int DH, int NQ>
 whale_status launch_attn_bwd(const AttnBwdArgs& a, unsigned chunks, cudaStream_t st) {
@@ -1597,9 +1613,10 @@ whale_status launch_attn_bwd_tc(const AttnBwdArgs& a, unsigned chunks, cudaStrea
 
 // Shapes the backward pass supports: bf16 with at most 32 queries per example (the KV-parallel
 // attention backward keeps all of an example's queries resident), d a multiple of 128 (its head
-// groups span 128 columns) and d <= 1024 (row kernels); fp32 with d_head <= 64.
+// groups span 128 columns) and d <= 1024 (row kernels); fp32 with d_head <= 64. The SwiGLU backward
+// takes 8 hidden columns per thread: ffn_hidden a multiple of 8.
 bool backward_shape_ok(const Shape& s) {
-  if (s.d > 1024 || s.d % 32) return false;
+  if (s.d > 1024 || s.d % 32 || s.H % 8) return false;
   if (s.bf16) return s.N <= 32 && (s.dh == 32 || s.dh == 64) && s.d % 128 == 0;
   return s.dh == 8 || s.dh == 16 || s.dh == 32 || s.dh == 64;
 }
@@ -1637,7 +1654,7 @@ whale_status recompute_bf16(const Shape& s, const Stream3& in, const void* slab,
   if (Fh > 0) {
     WCHECK(gemm_bf16(A, X, w.w_f1, Fh, Outs{nullptr, nullptr, F(b.z1), Fh}, nullptr, 0, rows, EPI_STORE, false, 0.f,
                      st));
-    WCHECK(ew_launch(silu_pair_kernel, rows * Fh, st, (const float*)F(b.z1), (float*)nullptr, static_cast<bf*>(b.g),
+    WCHECK(ew8_launch(silu_pair_kernel, rows * Fh, st, (const float*)F(b.z1), (float*)nullptr, static_cast<bf*>(b.g),
                      static_cast<bf*>(b.g_lo), rows * Fh));
     WCHECK(gemm_bf16(opnd(b.g, b.g_lo, Fh, Fh), no_opnd(), w.w_f2, d, Outs{b.f, b.f_lo, F(b.f32), d}, x32, d,
                      rows, EPI_RESID, false, 0.f, st));
@@ -1678,10 +1695,10 @@ whale_status layer_backward_bf16(const Shape& s, const Stream3& in, const void* 
   // ---- S5 backward: SwiGLU FFN ----
   float* part = F(b.part);
   const size_t pc = b.part_floats;
-  WCHECK(ew_launch(split_pair_kernel, rows * d, st, dy, (long long)d, static_cast<bf*>(b.dy), static_cast<bf*>(b.dy_lo),
+  WCHECK(ew8_launch(split_pair_kernel, rows * d, st, dy, (long long)d, static_cast<bf*>(b.dy), static_cast<bf*>(b.dy_lo),
                    (long long)d, rows, d));
   WCHECK(gemm_acc32(b.dy, b.dy_lo, d, false, w.w_down, H, true, rows, H, d, F(b.dm), H, part, pc, st));
-  WCHECK(ew_launch(swiglu_bwd_kernel, rows * H, st, (const float*)F(b.ug), (const float*)F(b.dm), rows, H,
+  WCHECK(ew8_launch(swiglu_bwd_kernel, rows * H, st, (const float*)F(b.ug), (const float*)F(b.dm), rows, H,
                    s.tied ? 1 : 0, static_cast<bf*>(b.msw), static_cast<bf*>(b.msw_lo), (float*)nullptr,
                    (float*)nullptr, static_cast<bf*>(b.dug), static_cast<bf*>(b.dug_lo)));
   // token-side weight gradients: both operands as hi/lo pairs (their sums over rows cancel)
@@ -1693,7 +1710,7 @@ whale_status layer_backward_bf16(const Shape& s, const Stream3& in, const void* 
   // ---- S4 backward: Fusion MLP (dc = d[A | H_w]) ----
   if (Fh > 0) {
     WCHECK(gemm_acc32(b.df, b.df_lo, d, false, w.w_f2, Fh, true, rows, Fh, d, F(b.dhid), Fh, part, pc, st));
-    WCHECK(ew_launch(silu_bwd_kernel, rows * Fh, st, (const float*)F(b.dhid), (const float*)F(b.z1), (float*)nullptr,
+    WCHECK(ew8_launch(silu_bwd_kernel, rows * Fh, st, (const float*)F(b.dhid), (const float*)F(b.z1), (float*)nullptr,
                      static_cast<bf*>(b.dz), static_cast<bf*>(b.dz_lo), rows * Fh));
     WCHECK(gemm_acc32(b.df, b.df_lo, d, true, b.g, Fh, true, d, Fh, rows, gr.w_f2, Fh, part, pc, st, b.g_lo));
     WCHECK(gemm_acc32(b.dz, b.dz_lo, Fh, false, w.w_f1, 2 * d, true, rows, 2 * d, Fh, F(b.dc), 2 * d, part, pc, st));
@@ -1705,14 +1722,15 @@ whale_status layer_backward_bf16(const Shape& s, const Stream3& in, const void* 
     WCHECK(gemm_acc32(b.df, b.df_lo, d, true, x, d, true, d, d, rows, gr.w_f2 + d, 2 * d, part, pc, st, in.lo));
   }
   // ---- S3 backward: attention (KV-parallel) ----
-  WCHECK(ew_launch(attn_bwd_prep_kernel, rows * s.h, st, (const float*)F(b.dc), (long long)(2 * d),
+  WCHECK(ew8_launch(attn_bwd_prep_kernel, rows * d, st, (const float*)F(b.dc), (long long)(2 * d),
                    (const bf*)b.a, (const bf*)b.a_lo, rows, d, s.h, F(b.delta), static_cast<bf*>(b.da16),
                    static_cast<bf*>(b.da_lo)));
   CUCHECK(cudaMemsetAsync(b.dq, 0, (size_t)rows * d * 4, st));
   if (T > 0) {
-    const long long cmax = cdiv<long long>(T, kBwdChunk) + h.B;
+    const int chunk = s.dh == 64 ? kBwdChunkTc : kBwdChunk;
+    const long long cmax = cdiv<long long>(T, chunk) + h.B;
     if (cmax >= (1ll << 31)) return WHALE_ERR_UNSUPPORTED;
-    WCHECK(launch_pdl(chunk_starts_kernel, dim3(1), dim3(1024), 0, st, offsets, h.B, T, kBwdChunk, (int)cmax,
+    WCHECK(launch_pdl(chunk_starts_kernel, dim3(1), dim3(1024), 0, st, offsets, h.B, T, chunk, (int)cmax,
                       static_cast<int*>(b.cst)));
     AttnBwdArgs aa{};
     aa.q = static_cast<const bf*>(b.q);
@@ -1726,6 +1744,7 @@ whale_status layer_backward_bf16(const Shape& s, const Stream3& in, const void* 
     aa.delta = F(b.delta);
     aa.offsets = offsets;
     aa.cstart = static_cast<const int*>(b.cst);
+    aa.chunk = chunk;
     aa.dq = F(b.dq);
     aa.dkv = static_cast<bf*>(b.dkv);
     aa.row_scale = F(b.rkv);  // dK|V' = r dK|V: what both history-side products below contract with
@@ -1745,7 +1764,7 @@ whale_status layer_backward_bf16(const Shape& s, const Stream3& in, const void* 
     WCHECK(r);
   }
   // ---- S1 backward: query projection and its RMSNorm; d_tokens ----
-  WCHECK(ew_launch(split_pair_kernel, rows * d, st, (const float*)F(b.dq), (long long)d, static_cast<bf*>(b.dq_hi),
+  WCHECK(ew8_launch(split_pair_kernel, rows * d, st, (const float*)F(b.dq), (long long)d, static_cast<bf*>(b.dq_hi),
                    static_cast<bf*>(b.dq_lo), (long long)d, rows, d));
   WCHECK(gemm_acc32(b.dq_hi, b.dq_lo, d, false, w.w_q, d, true, rows, d, d, F(b.dn), d, part, pc, st));
   WCHECK(gemm_acc32(b.dq_hi, b.dq_lo, d, true, b.nq, d, true, d, d, rows, gr.w_q, d, part, pc, st, b.nq_lo));
@@ -1790,7 +1809,7 @@ whale_status layer_backward_f32(const Shape& s, const float* x, const float* sla
   WCHECK(attention_f32(s, F(b.q), F(b.kv), offsets, F(b.a), h.B, T, st));
   if (Fh > 0) {
     WCHECK(gemm_f32(F(b.a), d, x, d, nullptr, nullptr, W32(w.w_f1), Fh, F(b.z1), rows, F32_NONE, nullptr, st));
-    WCHECK(ew_launch(silu_pair_kernel, rows * Fh, st, (const float*)F(b.z1), F(b.g), (__nv_bfloat16*)nullptr,
+    WCHECK(ew8_launch(silu_pair_kernel, rows * Fh, st, (const float*)F(b.z1), F(b.g), (__nv_bfloat16*)nullptr,
                      (__nv_bfloat16*)nullptr, rows * Fh));
     WCHECK(gemm_f32(F(b.g), Fh, nullptr, 0, nullptr, nullptr, W32(w.w_f2), d, F(b.f32), rows, F32_RESID, x, st));
   } else {
@@ -1801,7 +1820,7 @@ whale_status layer_backward_f32(const Shape& s, const float* x, const float* sla
                   st));
   // ---- S5 backward ----
   WCHECK(mm(dy, d, W32(w.w_down), H, F(b.dm), H, rows, H, d));
-  WCHECK(ew_launch(swiglu_bwd_kernel, rows * H, st, (const float*)F(b.ug), (const float*)F(b.dm), rows, H,
+  WCHECK(ew8_launch(swiglu_bwd_kernel, rows * H, st, (const float*)F(b.ug), (const float*)F(b.dm), rows, H,
                    s.tied ? 1 : 0, (__nv_bfloat16*)nullptr, (__nv_bfloat16*)nullptr, F(b.msw), F(b.dug),
                    (__nv_bfloat16*)nullptr, (__nv_bfloat16*)nullptr));
   WCHECK(mtm(dy, d, F(b.msw), H, gr.w_down, H, d, H, rows));
@@ -1812,7 +1831,7 @@ whale_status layer_backward_f32(const Shape& s, const float* x, const float* sla
   // ---- S4 backward ----
   if (Fh > 0) {
     WCHECK(mm(F(b.df32), d, W32(w.w_f2), Fh, F(b.dhid), Fh, rows, Fh, d));
-    WCHECK(ew_launch(silu_bwd_kernel, rows * Fh, st, (const float*)F(b.dhid), (const float*)F(b.z1), F(b.dz),
+    WCHECK(ew8_launch(silu_bwd_kernel, rows * Fh, st, (const float*)F(b.dhid), (const float*)F(b.z1), F(b.dz),
                      (__nv_bfloat16*)nullptr, (__nv_bfloat16*)nullptr, rows * Fh));
     WCHECK(mtm(F(b.df32), d, F(b.g), Fh, gr.w_f2, Fh, d, Fh, rows));
     WCHECK(mm(F(b.dz), Fh, W32(w.w_f1), 2 * d, F(b.dc), 2 * d, rows, 2 * d, Fh));
