@@ -74,6 +74,10 @@ struct GemmArgs {
   long long split_stride;
   // ROWNORM: the row factors r are also written here (by the tiles of the first output columns; may be null).
   float* rows_r;
+  // SPLIT, K-major A: tmA0 and tmA1 each cover both halves of their pair as two planes (3-D with one
+  // K block per stage, 4-D with two), so one copy per source and stage brings hi and lo (in either
+  // order: the kernel only ever sums the two halves' products and squares).
+  int a_planes;
 };
 
 
@@ -479,6 +483,9 @@ __global__ void __launch_bounds__(gemm_threads<ROWNORM>(), 1)
               tma_load_2d(st + i * MN_BOX, first ? &tmA0 : &tmA1, ma + 64 * i, kc, &full[s]);
               if (SPLIT) tma_load_2d(st + L::A_BYTES + i * MN_BOX, first ? &tmA0lo : &tmA1lo, ma + 64 * i, kc, &full[s]);
             }
+          } else if (SPLIT && args.a_planes) {
+            if (KPS == 1) tma_load_3d(st, first ? &tmA0 : &tmA1, kc, ma, 0, &full[s]);
+            else tma_load_4d(st, first ? &tmA0 : &tmA1, 0, ma, kc / L::BK, 0, &full[s]);
           } else if (KPS == 1) {
             tma_load_2d(st, first ? &tmA0 : &tmA1, kc, ma, &full[s]);
             if (SPLIT) tma_load_2d(st + L::A_BYTES, first ? &tmA0lo : &tmA1lo, kc, ma, &full[s]);

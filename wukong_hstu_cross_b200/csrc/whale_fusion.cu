@@ -235,6 +235,45 @@ whale_status epi_maps(CUtensorMap* o, const GemmArgs& g, long long cols, long lo
   return WHALE_OK;
 }
 
+// Both halves of a K-major bf16 pair [rows, K] (row stride ld) as two planes one byte stride apart:
+// base = the lower of the two addresses, pstride = their distance (a multiple of 16, below 2^40).
+// kps 1: {K, rows, 2} with box {64, box_rows, 2}; kps 2: {64, rows, K / 64, 2} with box {64,
+// box_rows, 2, 2}. One copy then brings [plane][block][row][64], the layout of a stage's A halves.
+whale_status tmap_bf16_pair(CUtensorMap* tm, const void* base, long long pstride, long long rows, long long K,
+                            long long ld, int box_rows, int kps) {
+  WCHECK(get_encoder());
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || (ld * 2) % 16 || rows <= 0 || K <= 0 || K % 64 || K > ld ||
+      pstride <= 0 || pstride % 16 || pstride >= (1ll << 40))
+    return WHALE_ERR_INVALID_ARG;
+  CUresult r;
+  cuuint32_t es[4] = {1u, 1u, 1u, 1u};
+  if (kps == 1) {
+    cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)rows, 2u};
+    cuuint64_t strides[2] = {(cuuint64_t)(ld * 2), (cuuint64_t)pstride};
+    cuuint32_t box[3] = {64u, (cuuint32_t)box_rows, 2u};
+    r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  } else {
+    cuuint64_t dims[4] = {64u, (cuuint64_t)rows, (cuuint64_t)(K / 64), 2u};
+    cuuint64_t strides[3] = {(cuuint64_t)(ld * 2), 128u, (cuuint64_t)pstride};
+    cuuint32_t box[4] = {64u, (cuuint32_t)box_rows, (cuuint32_t)kps, 2u};
+    r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  }
+  return r == CUDA_SUCCESS ? WHALE_OK : WHALE_ERR_CUDA;
+}
+
+// The pair map of an operand when its halves allow one (see tmap_bf16_pair); false otherwise.
+bool pair_map(CUtensorMap* tm, const void* hi, const void* lo, long long rows, long long K, long long ld, int box_rows,
+              int kps) {
+  if (!hi || !lo) return false;
+  const uintptr_t h = reinterpret_cast<uintptr_t>(hi), l = reinterpret_cast<uintptr_t>(lo);
+  const long long d = h < l ? (long long)(l - h) : (long long)(h - l);
+  return tmap_bf16_pair(tm, h < l ? hi : lo, d, rows, K, ld, box_rows, kps) == WHALE_OK;
+}
+
 // A K-major operand's map for stages of kps K blocks (kps 1: the 2-D map).
 whale_status tmap_operand(CUtensorMap* tm, const void* base, long long rows, long long K, long long ld, int box_rows,
                           int kps) {
@@ -580,16 +619,25 @@ whale_status gemm_bf16(const Opnd& a0, const Opnd& a1, const void* W, int N, con
         kps = kc;
       }
   CUtensorMap maps[8];
-  WCHECK(tmap_operand(&maps[0], a0.hi, M, a0.K, a0.ld, 128, kps));
-  if (split) WCHECK(tmap_operand(&maps[1], a0.lo, M, a0.K, a0.ld, 128, kps));
-  else maps[1] = maps[0];
-  if (a1.K > 0) {
-    WCHECK(tmap_operand(&maps[2], a1.hi, M, a1.K, a1.ld, 128, kps));
-    if (split) WCHECK(tmap_operand(&maps[3], a1.lo, M, a1.K, a1.ld, 128, kps));
-    else maps[3] = maps[2];
+  // hi/lo pairs: one two-plane map per source where both sources allow it (one copy per stage each)
+  bool planes = split && pair_map(&maps[0], a0.hi, a0.lo, M, a0.K, a0.ld, 128, kps) &&
+                (a1.K == 0 || pair_map(&maps[2], a1.hi, a1.lo, M, a1.K, a1.ld, 128, kps));
+  if (planes) {
+    maps[1] = maps[0];
+    if (a1.K == 0) maps[2] = maps[0];
+    maps[3] = maps[2];
   } else {
-    maps[2] = maps[0];
-    maps[3] = maps[1];
+    WCHECK(tmap_operand(&maps[0], a0.hi, M, a0.K, a0.ld, 128, kps));
+    if (split) WCHECK(tmap_operand(&maps[1], a0.lo, M, a0.K, a0.ld, 128, kps));
+    else maps[1] = maps[0];
+    if (a1.K > 0) {
+      WCHECK(tmap_operand(&maps[2], a1.hi, M, a1.K, a1.ld, 128, kps));
+      if (split) WCHECK(tmap_operand(&maps[3], a1.lo, M, a1.K, a1.ld, 128, kps));
+      else maps[3] = maps[2];
+    } else {
+      maps[2] = maps[0];
+      maps[3] = maps[1];
+    }
   }
   WCHECK(tmap_operand(&maps[4], W, N, a0.K + a1.K, a0.K + a1.K, bn, kps));
   GemmArgs g{};
@@ -607,6 +655,7 @@ whale_status gemm_bf16(const Opnd& a0, const Opnd& a1, const void* W, int N, con
   g.ldo = out.ld;
   g.resid32 = resid32;
   g.ldr = ldr;
+  g.a_planes = planes ? 1 : 0;
   WCHECK(epi_maps(maps + 5, g, epi == EPI_SWIGLU ? N / 2 : N, 1, maps[0]));
   const long long tiles = tm * g.tiles_n;
   if (kps == 2) {
