@@ -46,6 +46,33 @@ def test_backward_workspace_size_and_supported_shapes():
     assert large - small >= (40000 - 400) * cfg.d * (2 * 2 + 2 * 2 + 4 + 2)
 
 
+def test_stack_backward_keeps_each_layers_activations():
+    # bf16: every layer past the first adds its own forward activations to the stack's workspace
+    # (its K|V pair over the history above all: 4 bytes per K|V element), so that the stack runs each
+    # layer's forward once; fp32 adds only the layer's input (it recomputes inside each layer)
+    T, B = 40000, 4
+    for name in ("stack_d128", "tiny_fp32"):
+        _, cfg = _cfg(name)
+        kvw = 2 * cfg.d
+        sizes = []
+        for nl in (1, 2, 3):
+            c = W.make_config(nl, cfg.d, cfg.n_heads, cfg.n_tokens, cfg.ffn_hidden, cfg.fusion_hidden, cfg.dtype,
+                              cfg.flags, cfg.eps)
+            sizes.append(W.whale_backward_workspace_size(c, W.make_hint(B, T // B, T)))
+        step = sizes[2] - sizes[1]
+        assert step == sizes[1] - sizes[0], name  # the same for every added layer
+        rows = B * cfg.n_tokens
+        if cfg.dtype == W.WHALE_BF16:
+            assert step >= T * kvw * 4 + rows * cfg.d * (4 + 2 + 2), name
+        else:
+            assert rows * cfg.d * 4 <= step < T * kvw * 4, name
+    # the SwiGLU backward takes 8 hidden columns per thread: other hidden sizes are not supported
+    w, cfg = _cfg("stack_d128")
+    odd = W.make_config(cfg.n_layers, cfg.d, cfg.n_heads, cfg.n_tokens, cfg.ffn_hidden + 4, cfg.fusion_hidden,
+                        W.WHALE_FP32, cfg.flags, cfg.eps)
+    assert W.whale_backward_workspace_size(odd, W.make_hint(4, 100, 400)) == 0
+
+
 def test_backward_host_side_errors():
     w, cfg = _cfg("stack_d128")
     hint = W.make_hint(2, 10, 20)
