@@ -125,3 +125,60 @@ def test_balanced_ranges_edge_cases():
         assert rr[0][0] == 0 and rr[-1][1] == 37 and all(rr[k][1] == rr[k + 1][0] for k in range(world - 1))
         loads = [int(L[a:b].sum()) for a, b in rr]
         assert max(loads) - min(loads) <= 2 * int(L.max())
+
+
+def _cand_worker(rank, world, port, out):
+    import torch.distributed as dist
+    from oracle import whale_oracle as O
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    # a reduced serving request: one shared history, 7 candidates x 4 tokens (7 does not divide by 2)
+    w = I.WORKLOADS["serve_15k"].replace(n_tokens=7 * 4, candidates=7, d=64, n_heads=2, n_layers=2,
+                                         lengths=("fixed", 150))
+    L = I.draw_lengths(w)
+    off = I.offsets_of(L)
+    tokens = I.make_tokens(w)
+    states = np.stack([I.make_states_layer(w, l, L, threads=1) for l in range(w.n_layers)])
+    lws = I.make_all_weights(w, gains="random")
+    tok_r, (c0, c1) = D.shard_candidates(tokens, 4, rank, world)
+    y = O.fusion_stack(tok_r, states, off, lws, w.n_heads, w.eps)     # the history replicated
+    objs = [None] * world
+    dist.all_gather_object(objs, (c0, c1, y))
+    if rank == 0:
+        out.put((objs, O.fusion_stack(tokens, states, off, lws, w.n_heads, w.eps)))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_serving_request_sharded_by_candidates_equals_unsharded():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_cand_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    objs, full = q.get(timeout=180)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    (a0, a1, y0), (c0, c1, y1) = objs
+    assert (a0, a1, c0, c1) == (0, 4, 4, 7)
+    got = np.concatenate([y0, y1], axis=1)
+    assert got.shape == full.shape
+    # each token's result depends on its own row and the shared history only; the fp64 products of
+    # fewer rows may be blocked differently by BLAS, so agreement is to fp64 rounding, not bitwise
+    assert np.allclose(got, full, rtol=1e-12, atol=1e-12), float(np.abs(got - full).max())
+
+
+def test_candidate_ranges():
+    assert [D.candidate_range(1024, r, 8) for r in (0, 7)] == [(0, 128), (896, 1024)]
+    assert [D.candidate_range(7, r, 3) for r in range(3)] == [(0, 3), (3, 5), (5, 7)]
+    assert [D.candidate_range(2, r, 4) for r in range(4)] == [(0, 1), (1, 2), (2, 2), (2, 2)]
+    x = np.zeros((1, 12, 3))
+    assert D.shard_candidates(x, 4, 1, 2)[0].shape == (1, 4, 3)
+    try:
+        D.shard_candidates(x, 5, 0, 2)
+        raise AssertionError("12 tokens are not whole candidates of 5")
+    except ValueError:
+        pass

@@ -4,7 +4,9 @@ The fusion forward shards with no exchange: examples are independent, so each ra
 whole stack on its own examples with replicated weights, and nothing crosses ranks on the data
 path. Two ways to give ranks their examples: a fresh batch per rank (weak scaling, as the
 benchmark runs), or one batch split into contiguous example ranges balanced by history rows
-(shard_batch). The only collective is the timing reduction (max over ranks).
+(shard_batch). A serving request, one history shared by many candidates, splits along its
+candidates instead, the history replicated (shard_candidates). The only collective is the timing
+reduction (max over ranks).
 """
 from __future__ import annotations
 
@@ -63,6 +65,30 @@ def shard_batch(tokens, states, offsets, rank: int, world: int):
     b0, b1 = balanced_ranges(np.diff(off), world)[rank]
     o0, o1 = int(off[b0]), int(off[b1])
     return tokens[b0:b1], states[:, o0:o1], (off[b0:b1 + 1] - o0).astype(np.int32), (b0, b1)
+
+
+def candidate_range(n_candidates: int, rank: int, world: int) -> tuple:
+    """Rank `rank`'s contiguous range [c0, c1) of one request's candidates, as even as whole
+    candidates allow (the first n_candidates % world ranks take one more)."""
+    base, extra = divmod(max(int(n_candidates), 0), world)
+    c0 = rank * base + min(rank, extra)
+    return c0, c0 + base + (1 if rank < extra else 0)
+
+
+def shard_candidates(tokens, tokens_per_candidate: int, rank: int, world: int):
+    """Rank `rank`'s part of a serving request whose one history is shared by every candidate.
+
+    Each query token attends over the request's whole history, and the Fusion MLP and the FFN act
+    on each token alone, so the request splits along its queries with no exchange: every rank keeps
+    the history (and the weights) whole and runs its own candidates' tokens, with n_tokens set to
+    that count in its config. tokens: [1, n_candidates * tokens_per_candidate, d] (numpy or torch).
+    Returns (tokens [1, (c1-c0) * tokens_per_candidate, d], (c0, c1)); the ranks' outputs, put back
+    in rank order along the token axis, are the request's output."""
+    n = int(tokens.shape[1])
+    if tokens_per_candidate < 1 or n % tokens_per_candidate:
+        raise ValueError(f"{n} tokens are not whole candidates of {tokens_per_candidate}")
+    c0, c1 = candidate_range(n // tokens_per_candidate, rank, world)
+    return tokens[:, c0 * tokens_per_candidate:c1 * tokens_per_candidate], (c0, c1)
 
 
 def max_over_ranks(x: float, world: int, device=None) -> float:
