@@ -183,7 +183,9 @@ whale_status whale_fusion_forward(const whale_config* cfg, const void* wukong_to
  * host_tokens [B,N,d], host_seq_states [n_layers,total_L,d], host_offsets int32 [B+1],
  * host_out [B,N,d] are host pointers (pin them for asynchronous copies); weights as above.
  * The workspace must hold whale_host_workspace_size bytes. Returns after enqueueing;
- * synchronise `stream` before reading host_out. */
+ * synchronise `stream` before reading host_out. Calls on one device share one copy stream: calls
+ * from several host threads take turns to enqueue (their GPU work may still overlap, each with its
+ * own workspace). At most 64 layers. */
 size_t whale_host_workspace_size(const whale_config* cfg, const whale_shape_hint* hint);
 whale_status whale_fusion_forward_host(const whale_config* cfg, const void* host_tokens,
                                        const void* host_seq_states, const int* host_offsets,

@@ -197,3 +197,22 @@ def test_profile_records_nothing_without_launches():
     assert W.whale_profile_end() == []                  # no kernel launched: no records, no CUDA call
     n = ctypes.c_int(-1)
     assert W._lib.whale_profile_end(None, 4, ctypes.byref(n)) == 1   # records requested into a null buffer
+
+
+def test_host_buffer_forward_checks_before_any_copy():
+    # the host-buffer forward checks its layer count and workspace before it enqueues a copy
+    w, cfg = _cfg("stack_d128")
+    hint = W.make_hint(2, 10, 20)
+    fake = 1 << 20
+    lw = dict.fromkeys(["g_q", "g_kv", "w_q", "w_kv", "w_f1", "w_f2", "g_ffn", "w_upgate", "w_down"], fake)
+    deep = W.make_config(65, cfg.d, cfg.n_heads, cfg.n_tokens, cfg.ffn_hidden, cfg.fusion_hidden, cfg.dtype,
+                         cfg.flags, cfg.eps)
+    ws = W.whale_host_workspace_size(deep, hint)
+    assert ws > W.whale_workspace_size(deep, hint)          # the staging buffers come first
+    assert W.whale_fusion_forward_host(deep, fake, fake, fake, [lw] * 65, fake, hint, fake, ws, stream=0,
+                                       raw=True) == 2        # more than 64 layers
+    ws4 = W.whale_host_workspace_size(cfg, hint)
+    assert W.whale_fusion_forward_host(cfg, fake, fake, fake, [lw] * 4, fake, hint, fake, ws4 - 1, stream=0,
+                                       raw=True) == 4
+    assert W.whale_fusion_forward_host(cfg, None, fake, fake, [lw] * 4, fake, hint, fake, ws4, stream=0,
+                                       raw=True) == 1

@@ -1386,10 +1386,14 @@ whale_status debug_check(const Shape& s, const int* offsets, const whale_shape_h
   return WHALE_OK;
 }
 
-// Per-device copy stream and events of the host-buffer forward (created once, kept).
+// Per-device copy stream and events of the host-buffer forward (created once, kept). A call holds
+// `mu` while it enqueues: each of its waits must see its own event records, not another call's
+// recorded in between on another stream (a copy into a staging buffer would then not wait for the
+// layer of its own call that still reads that buffer).
 struct HostPipe {
   cudaStream_t copy = nullptr;
   cudaEvent_t copied[2] = {nullptr, nullptr}, consumed[2] = {nullptr, nullptr};
+  std::mutex mu;
 };
 std::mutex g_pipe_mu;
 HostPipe g_pipes[64];
@@ -2145,6 +2149,7 @@ whale_status whale_fusion_forward_host(const whale_config* cfg, const void* host
   Shape s;
   WCHECK(validate(cfg, &s));
   WCHECK(check_hint(hint));
+  if (s.layers > 64) return WHALE_ERR_UNSUPPORTED;  // the per-layer slab table below
   size_t o_tok, o_s0, o_s1, o_off, o_out;
   const size_t staging = align_up(host_staging_bytes(s, *hint, &o_tok, &o_s0, &o_s1, &o_off, &o_out));
   const Layout L = make_layout(s, *hint);
@@ -2158,6 +2163,7 @@ whale_status whale_fusion_forward_host(const whale_config* cfg, const void* host
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   HostPipe* pipe = nullptr;
   WCHECK(host_pipe(&pipe));
+  std::lock_guard<std::mutex> enqueue(pipe->mu);
   void* fws = at(ws, staging);
   const size_t rows = (size_t)hint->B * s.N;
   const size_t tok_bytes = rows * s.d * s.es;
@@ -2183,7 +2189,6 @@ whale_status whale_fusion_forward_host(const whale_config* cfg, const void* host
   };
   WCHECK(copy_slab(0));
   const void* slabs[64];
-  if (s.layers > 64) return WHALE_ERR_UNSUPPORTED;
   for (int l = 0; l < s.layers; ++l) slabs[l] = slab_bytes ? d_slab[l & 1] : nullptr;
   auto hook = [&](int l, bool before) -> whale_status {
     if (before) {
