@@ -281,7 +281,8 @@ whale_status whale_cross_attention_noalloc(const whale_config* cfg, const void* 
  *   w             the layer's RAW weights and gains (WHALE_PREPARED_WEIGHTS is not accepted)
  *   d_out         device fp32 [B, N, d]      dLoss/dH_f
  *   d_tokens      device fp32 [B, N, d]      dLoss/dH_w (written)
- *   d_states      device [total_L, d]        dLoss/dH_s in cfg->dtype (written)
+ *   d_states      device [total_L, d]        dLoss/dH_s in cfg->dtype (written; rows past offsets[B],
+ *                                            which no example reads, get 0)
  *   grads         HOST struct of device fp32 pointers, each overwritten with dLoss/d(parameter),
  *                 summed over the batch, in the parameter's own layout (w_f1 may be null when
  *                 fusion_hidden is 0)

@@ -635,6 +635,26 @@ __global__ void scale_cols_pair_kernel(const __nv_bfloat16* __restrict__ w, cons
   }
 }
 
+// Rows [offsets[B], total_L) of a history slab belong to no example, so their K|V gradient is zero;
+// the attention backward writes the examples' rows only. This clears the others in x and, if given,
+// x_lo (each [total_L, width] row-major). Nothing is written when the examples cover the slab.
+template <typename T>
+__global__ void zero_tail_rows_kernel(const int* __restrict__ offsets, int B, long long total_L, int width,
+                                      T* __restrict__ x, T* __restrict__ x_lo) {
+  pdl_wait();
+  pdl_trigger();
+  long long r0 = offsets[B];
+  r0 = r0 < 0 ? 0 : (r0 > total_L ? total_L : r0);
+  const long long n = (total_L - r0) * width;
+  T* p = x + r0 * width;
+  T* q = x_lo ? x_lo + r0 * width : nullptr;
+  const T zero = T(0.0f);
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    p[i] = zero;
+    if (q) q[i] = zero;
+  }
+}
+
 // c[r, col] *= g[col] for a row-major fp32 [rows, cols] matrix (row stride ld).
 __global__ void scale_cols_kernel(float* __restrict__ c, long long ld, const float* __restrict__ g, long long rows,
                                   int cols) {

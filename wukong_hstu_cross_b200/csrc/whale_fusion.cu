@@ -1783,6 +1783,8 @@ whale_status layer_backward_bf16(const Shape& s, const Stream3& in, const void* 
     const int chunk = s.dh == 64 ? kBwdChunkTc : kBwdChunk;
     const long long cmax = cdiv<long long>(T, chunk) + h.B;
     if (cmax >= (1ll << 31)) return WHALE_ERR_UNSUPPORTED;
+    WCHECK(ew_launch(zero_tail_rows_kernel<bf>, T * kvw, st, offsets, h.B, T, kvw, static_cast<bf*>(b.dkv),
+                     static_cast<bf*>(b.dkv_lo)));
     WCHECK(launch_pdl(chunk_starts_kernel, dim3(1), dim3(1024), 0, st, offsets, h.B, T, chunk, (int)cmax,
                       static_cast<int*>(b.cst)));
     AttnBwdArgs aa{};
@@ -1902,6 +1904,8 @@ whale_status layer_backward_f32(const Shape& s, const float* x, const float* sla
     const dim3 grid((unsigned)h.B, (unsigned)s.h);
     const float scale = (float)(1.0 / std::sqrt((double)s.dh));
     const int v0 = s.shared_kv ? 0 : d;
+    if (T > 0)
+      WCHECK(ew_launch(zero_tail_rows_kernel<float>, T * kvw, st, offsets, h.B, T, kvw, F(b.dkv), (float*)nullptr));
 #define ATTB32(DH)                                                                                                    \
   do {                                                                                                                \
     CUCHECK(cudaFuncSetAttribute(attn_bwd_f32_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));   \
@@ -2461,6 +2465,8 @@ whale_status whale_fusion_layer_backward(const whale_config* cfg, const void* to
     CUCHECK(cudaMemsetAsync(grads->w_f2, 0, d * (size_t)(s.Fh > 0 ? s.Fh : 2 * s.d) * 4, st));
     CUCHECK(cudaMemsetAsync(grads->w_upgate, 0, (size_t)s.ugw * d * 4, st));
     CUCHECK(cudaMemsetAsync(grads->w_down, 0, d * (size_t)s.H * 4, st));
+    if (hint->total_L > 0 && d_states)  // rows of no example
+      CUCHECK(cudaMemsetAsync(d_states, 0, (size_t)hint->total_L * s.d * s.es, st));
     return WHALE_OK;
   }
   if (!tokens_in || !seq_offsets || !d_out || !d_tokens || (hint->total_L > 0 && (!layer_states || !d_states)))
@@ -2496,7 +2502,9 @@ whale_status whale_fusion_backward(const whale_config* cfg, const void* tokens, 
   const long long rows = (long long)hint->B * s.N, T = hint->total_L;
   if (hint->B == 0) {
     for (int l = 0; l < s.layers; ++l)
-      WCHECK(whale_fusion_layer_backward(cfg, nullptr, nullptr, nullptr, &weights[l], nullptr, nullptr, nullptr,
+      WCHECK(whale_fusion_layer_backward(cfg, nullptr, nullptr, nullptr, &weights[l], nullptr, nullptr,
+                                         T > 0 && d_states ? static_cast<char*>(d_states) + l * T * s.d * s.es
+                                                           : nullptr,
                                          &grads[l], hint, ws, ws_bytes, stream));
     return WHALE_OK;
   }
