@@ -1,10 +1,11 @@
 """History rows that no example reads. The C ABI lets a slab hold more rows than the examples use
-(offsets[B] < total_L); the forward never reads those rows, so their gradient is zero and they add
-nothing to the K|V weight and gain gradients. Checked through whale_fusion_layer_backward (bf16 with
-both attention backward kernels, d_head 32 and 64, and the fp32 mode) and whale_fusion_backward (a
-two-layer stack, each layer's slab with its own unread rows) against the fp64 VJP oracle, with the
-unread rows holding random values; and a batch of no examples over a non-empty slab, whose every
-gradient is zero."""
+(offsets[B] < total_L). The forward never reads those rows: its output is the oracle's for the
+examples' own rows, on the split-L, the query-tiled and the absorbed attention and in fp32 mode. Their
+gradient is zero and they add nothing to the K|V weight and gain gradients: checked through
+whale_fusion_layer_backward (bf16 with both attention backward kernels, d_head 32 and 64, and the
+fp32 mode) and whale_fusion_backward (a two-layer stack, each layer's slab with its own unread rows)
+against the fp64 VJP oracle. The unread rows hold random values. A batch of no examples over a
+non-empty slab gets every gradient zero."""
 import dataclasses
 
 import numpy as np
@@ -12,7 +13,8 @@ import pytest
 import torch
 
 from oracle import whale_backward as OB
-from tests.gpu_util import to_np
+from oracle import whale_oracle as O
+from tests.gpu_util import assert_parity, to_np
 from tests.test_gpu_backward import _check, _oracle
 from wukong_hstu_cross_b200 import inputs as I
 
@@ -28,8 +30,8 @@ EXTRA = 300  # unread rows after the last example's
 
 
 def _with_unread_rows(p, extra, seed):
-    """The problem with `extra` random rows appended to every layer's slab and total_L raised to match
-    (offsets unchanged)."""
+    """The problem with `extra` random rows appended to every layer's slab, total_L raised to match
+    (offsets unchanged) and the forward's workspace sized for it."""
     w = p.w
     T = p.total_L + extra
     tail = I.bf16_round(np.random.default_rng(seed).standard_normal((w.n_layers, extra, w.d)).astype(np.float32))
@@ -38,7 +40,29 @@ def _with_unread_rows(p, extra, seed):
     for l in range(w.n_layers):
         states[l, p.total_L:].copy_(Hn.to_device(tail[l], w, p.states.device))
     hint = W.make_hint(w.batch, int(p.lengths.max()), T)
-    return dataclasses.replace(p, states=states, hint=hint)
+    ws = torch.empty(W.whale_workspace_size(p.cfg, hint), dtype=torch.uint8, device=p.states.device)
+    return dataclasses.replace(p, states=states, hint=hint, workspace=ws)
+
+
+FORWARD_CASES = {
+    "d128_splitl": ("stack_d128", dict(batch=4, n_layers=2, lengths=("uniform", 1, 500))),
+    "d512_absorbed": ("hist15k_d512", dict(batch=3, n_layers=2, lengths=("uniform", 100, 900))),
+    "d256_query_tiled": ("serve_15k", dict(n_tokens=16 * 16, n_layers=1, lengths=("fixed", 700))),
+    "tiny_fp32": ("tiny_fp32", dict(batch=3)),
+}
+
+
+@pytest.mark.parametrize("case", list(FORWARD_CASES))
+def test_forward_ignores_unread_rows(case):
+    base, over = FORWARD_CASES[case]
+    w = I.WORKLOADS[base].replace(**over)
+    p = _with_unread_rows(Hn.build_problem(w, gains="random"), EXTRA, seed=4)
+    out = Hn.run_forward(p).float().cpu().numpy()
+    torch.cuda.synchronize()
+    for b in range(w.batch):
+        ref = O.fusion_stack_example(I.tokens_of_example(w, b), Hn.states_of_example_host(p, b), p.host_weights,
+                                     w.n_heads, w.eps)
+        assert_parity(out[b], ref, w.dtype, what=f"{case} example {b}")
 
 
 LAYER_CASES = {
