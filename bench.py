@@ -619,7 +619,7 @@ def main():
     a = torch.empty_like(q)
     reps = max(args.steps, 3)
 
-    def timed(fn, n):
+    def timed_per_layer(fn, n):
         for l in range(min(2, w.n_layers)):
             fn(l)
         torch.cuda.synchronize()
@@ -652,7 +652,7 @@ def main():
     t_kv = t_attn = t_abs = None
     if absorbed:
         torch.cuda.synchronize()
-        t_abs = timed(absorbed_step, reps)
+        t_abs = timed_per_layer(absorbed_step, reps)
         abs_traffic = None
         passa_traffic_known = w.d == 512 and not args.shared_kv
         if passa_traffic_known and ABS_TRAFFIC_BYTES_PER_ROW_D512 is not None:
@@ -689,8 +689,8 @@ def main():
     else:
         kv_step(0)
         torch.cuda.synchronize()
-        t_kv = timed(kv_step, reps)
-        t_attn = timed(attn_step, reps)
+        t_kv = timed_per_layer(kv_step, reps)
+        t_attn = timed_per_layer(attn_step, reps)
         share_kv, share_attn = t_kv / layer_ms, t_attn / layer_ms
         kv_traffic = None
         if w.d == 512 and not args.shared_kv:
