@@ -86,7 +86,7 @@ typedef struct {
                          WHALE_MATERIALIZED_KV */
   float eps;          /* RMSNorm epsilon */
 } whale_config;
-/* Supported: fp32 — any d with d % n_heads == 0, d_head <= 128 (SIMT correctness path).
+/* Supported: fp32 — any d with d % n_heads == 0 and d_head in {8, 16, 32, 64, 128} (SIMT correctness path).
  *            bf16 — d % 64 == 0, d_head in {32, 64}, n_heads / (heads per CTA) integral
  *            (heads per CTA = min(n_heads, 8), its d_head multiple of 64 columns),
  *            ffn_hidden % 64 == 0, fusion_hidden % 64 == 0. Any n_tokens >= 1.

@@ -216,3 +216,11 @@ def test_host_buffer_forward_checks_before_any_copy():
                                        raw=True) == 4
     assert W.whale_fusion_forward_host(cfg, None, fake, fake, [lw] * 4, fake, hint, fake, ws4, stream=0,
                                        raw=True) == 1
+
+
+def test_fp32_head_sizes():
+    # fp32 mode takes d_head 8, 16, 32, 64 or 128 (any d those divide); other head sizes are refused
+    hint = W.make_hint(2, 10, 20)
+    for d, h, ok in ((64, 8, True), (24, 3, True), (64, 1, True), (128, 1, True), (96, 2, False), (256, 1, False)):
+        cfg = W.make_config(1, d, h, 8, 4 * d, 2 * d, W.WHALE_FP32, 0, 1e-6)
+        assert (W.whale_workspace_size(cfg, hint) > 0) == ok, (d, h)
