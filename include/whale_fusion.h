@@ -87,9 +87,9 @@ typedef struct {
   float eps;          /* RMSNorm epsilon */
 } whale_config;
 /* Supported: fp32 — any d with d % n_heads == 0 and d_head in {8, 16, 32, 64, 128} (SIMT correctness path).
- *            bf16 — d % 64 == 0, d_head in {32, 64}, n_heads / (heads per CTA) integral
- *            (heads per CTA = min(n_heads, 8), its d_head multiple of 64 columns),
- *            ffn_hidden % 64 == 0, fusion_hidden % 64 == 0. Any n_tokens >= 1.
+ *            bf16 — d % 64 == 0, d_head in {32, 64}, n_heads 2, 4 or a multiple of 8 (the
+ *            attention kernels take min(n_heads, 8) heads per CTA), ffn_hidden % 64 == 0,
+ *            fusion_hidden % 64 == 0. Any n_tokens >= 1.
  *
  * Absorbed attention (bf16, the default where it applies: n_tokens * n_heads == 256, d_head == 64,
  * d in {256, 512}, WHALE_MATERIALIZED_KV not set). The key and value projections are folded into

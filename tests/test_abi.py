@@ -224,3 +224,15 @@ def test_fp32_head_sizes():
     for d, h, ok in ((64, 8, True), (24, 3, True), (64, 1, True), (128, 1, True), (96, 2, False), (256, 1, False)):
         cfg = W.make_config(1, d, h, 8, 4 * d, 2 * d, W.WHALE_FP32, 0, 1e-6)
         assert (W.whale_workspace_size(cfg, hint) > 0) == ok, (d, h)
+
+
+def test_bf16_head_counts():
+    # bf16 mode: d_head 32 or 64 with 2, 4 or a multiple of 8 heads
+    hint = W.make_hint(2, 10, 20)
+    for h in range(1, 33):
+        for dh in (32, 64):
+            d = h * dh
+            if d % 64:
+                continue
+            cfg = W.make_config(1, d, h, 8, 4 * d, 2 * d, W.WHALE_BF16, 0, 1e-6)
+            assert (W.whale_workspace_size(cfg, hint) > 0) == (h in (2, 4) or h % 8 == 0), (h, dh)
