@@ -288,8 +288,8 @@ whale_status whale_cross_attention_noalloc(const whale_config* cfg, const void* 
  *                 fusion_hidden is 0)
  *   workspace     device, >= whale_backward_workspace_size bytes, 256-byte aligned
  *
- * Supported: bf16 with n_tokens <= 32, d_head 32 or 64, d % 128 == 0, d <= 1024; fp32 with d_head
- * <= 64 (the SIMT correctness mode); ffn_hidden a multiple of 8. Other shapes return
+ * Supported: d <= 1024, d % 32 == 0 and ffn_hidden a multiple of 8; bf16 also with n_tokens <= 32,
+ * d_head 32 or 64 and d % 128 == 0; fp32 with d_head 8, 16, 32 or 64 (the SIMT correctness mode). Other shapes return
  * WHALE_ERR_UNSUPPORTED (the many-candidate serving shape is an inference shape). Asynchronous on `stream`; no device-to-host reads. In bf16
  * mode dq is summed with fp32 atomics across history chunks, so repeated calls can differ in the
  * last bits of d_tokens and of the gradients downstream of it. */

@@ -236,3 +236,18 @@ def test_bf16_head_counts():
                 continue
             cfg = W.make_config(1, d, h, 8, 4 * d, 2 * d, W.WHALE_BF16, 0, 1e-6)
             assert (W.whale_workspace_size(cfg, hint) > 0) == (h in (2, 4) or h % 8 == 0), (h, dh)
+
+
+def test_backward_shapes():
+    hint = W.make_hint(2, 10, 20)
+    cases = [  # (dtype, d, heads, n_tokens, ffn_hidden, supported)
+        (W.WHALE_BF16, 512, 8, 32, 2048, True), (W.WHALE_BF16, 128, 4, 16, 512, True),
+        (W.WHALE_BF16, 1024, 16, 32, 4096, True), (W.WHALE_BF16, 2048, 32, 32, 8192, False),   # d > 1024
+        (W.WHALE_BF16, 512, 8, 33, 2048, False), (W.WHALE_BF16, 192, 2, 16, 768, False),     # N > 32; d % 128
+        (W.WHALE_FP32, 64, 2, 8, 256, True), (W.WHALE_FP32, 96, 12, 8, 384, True),
+        (W.WHALE_FP32, 128, 1, 8, 512, False), (W.WHALE_FP32, 48, 6, 8, 192, False),          # d_head 128; d % 32
+        (W.WHALE_FP32, 64, 2, 8, 260, False),                                               # ffn_hidden % 8
+    ]
+    for dt, d, h, n, ffn, ok in cases:
+        cfg = W.make_config(1, d, h, n, ffn, 2 * d, dt, 0, 1e-6)
+        assert (W.whale_backward_workspace_size(cfg, hint) > 0) == ok, (dt, d, h, n, ffn)
