@@ -185,7 +185,8 @@ whale_status whale_fusion_forward(const whale_config* cfg, const void* wukong_to
  * The workspace must hold whale_host_workspace_size bytes. Returns after enqueueing;
  * synchronise `stream` before reading host_out. Calls on one device share one copy stream: calls
  * from several host threads take turns to enqueue (their GPU work may still overlap, each with its
- * own workspace). At most 64 layers. */
+ * own workspace). That stream and its events are created on the device's first call and kept, so
+ * this entry point is not usable after cudaDeviceReset in the same process. At most 64 layers. */
 size_t whale_host_workspace_size(const whale_config* cfg, const whale_shape_hint* hint);
 whale_status whale_fusion_forward_host(const whale_config* cfg, const void* host_tokens,
                                        const void* host_seq_states, const int* host_offsets,
