@@ -16,10 +16,12 @@
 #include "whale_fusion.h"
 
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
 #include <cstdlib>
+#include <cstdio>
 #include <cstring>
 #include <functional>
 #include <utility>
@@ -55,6 +57,15 @@ namespace {
       return WHALE_ERR_CUDA;               \
     }                                      \
   } while (0)
+
+// An NVTX range over one entry point or one layer, for timeline tools (Nsight Systems); with no
+// tool attached the push and pop return at once.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 constexpr int kNumSM = 148;
 constexpr size_t kAlign = 256;
@@ -1344,6 +1355,9 @@ whale_status stack_impl(const Shape& s, const void* tokens, const void* seq_stat
   if (!s.bf16) {
     const void* x = tokens;
     for (int l = 0; l < n_layers; ++l) {
+      char name[32];
+      snprintf(name, sizeof name, "whale layer %d", first_layer + l);
+      NvtxRange range(name);
       void* y = (l == n_layers - 1) ? out : at(ws, (l & 1) ? L.x1 : L.x0);
       if (hook) WCHECK(hook(l, true));
       WCHECK(layer_f32(s, x, slab_of(l), offsets, weights[first_layer + l], y, hint, ws, L, st));
@@ -1360,6 +1374,9 @@ whale_status stack_impl(const Shape& s, const void* tokens, const void* seq_stat
   WCHECK(pair_from_bf16(tokens, in.f32, in.lo, rows * s.d, st));
   WCHECK(abs_units(s, offsets, hint, ws, L, st));
   for (int l = 0; l < n_layers; ++l) {
+    char name[32];
+    snprintf(name, sizeof name, "whale layer %d", first_layer + l);
+    NvtxRange range(name);
     const Stream3 y = (l == n_layers - 1) ? Stream3{nullptr, out, nullptr} : buf((l + 1) & 1);
     if (hook) WCHECK(hook(l, true));
     WCHECK(layer_bf16(s, in, slab_of(l), offsets, weights[first_layer + l], y, hint, ws, L, st));
@@ -2062,6 +2079,7 @@ size_t whale_prepared_weights_size(const whale_config* cfg) {
 
 whale_status whale_prepare_weights(const whale_config* cfg, const whale_layer_weights* weights, void* prepared,
                                    size_t prepared_bytes, whale_layer_weights* out_weights, whale_stream_t stream) {
+  NvtxRange range("whale_prepare_weights");
   Shape s;
   WCHECK(validate(cfg, &s));
   if (!s.bf16) return WHALE_ERR_UNSUPPORTED;
@@ -2109,6 +2127,7 @@ whale_status whale_fusion_layer_forward(const whale_config* cfg, const void* tok
                                         const int* seq_offsets, const whale_layer_weights* w, void* tokens_out,
                                         const whale_shape_hint* hint, void* ws, size_t ws_bytes,
                                         whale_stream_t stream) {
+  NvtxRange range("whale_fusion_layer_forward");
   Shape s;
   Layout L;
   WCHECK(common_checks(cfg, hint, &s, ws, ws_bytes, &L));
@@ -2126,6 +2145,7 @@ whale_status whale_fusion_layer_forward(const whale_config* cfg, const void* tok
 whale_status whale_fusion_forward(const whale_config* cfg, const void* tokens, const void* seq_states,
                                   const int* seq_offsets, const whale_layer_weights* weights, void* out,
                                   const whale_shape_hint* hint, void* ws, size_t ws_bytes, whale_stream_t stream) {
+  NvtxRange range("whale_fusion_forward");
   Shape s;
   Layout L;
   WCHECK(common_checks(cfg, hint, &s, ws, ws_bytes, &L));
@@ -2150,6 +2170,7 @@ whale_status whale_fusion_forward_host(const whale_config* cfg, const void* host
                                        const int* host_offsets, const whale_layer_weights* weights, void* host_out,
                                        const whale_shape_hint* hint, void* ws, size_t ws_bytes,
                                        whale_stream_t stream) {
+  NvtxRange range("whale_fusion_forward_host");
   Shape s;
   WCHECK(validate(cfg, &s));
   WCHECK(check_hint(hint));
@@ -2210,6 +2231,7 @@ whale_status whale_fusion_forward_host(const whale_config* cfg, const void* host
 
 whale_status whale_project_queries(const whale_config* cfg, long long rows, const void* x, const float* g_q,
                                    const void* w_q, void* q, void* ws, size_t ws_bytes, whale_stream_t stream) {
+  NvtxRange range("whale_project_queries");
   Shape s;
   WCHECK(validate(cfg, &s));
   if (rows < 0 || !x || !g_q || !w_q || !q) return WHALE_ERR_INVALID_ARG;
@@ -2231,6 +2253,7 @@ whale_status whale_project_queries(const whale_config* cfg, long long rows, cons
 
 whale_status whale_project_kv(const whale_config* cfg, long long rows, const void* sx, const float* g_kv,
                               const void* w_kv, void* kv, void* ws, size_t ws_bytes, whale_stream_t stream) {
+  NvtxRange range("whale_project_kv");
   Shape s;
   WCHECK(validate(cfg, &s));
   if (rows < 0 || !sx || !g_kv || !w_kv || !kv) return WHALE_ERR_INVALID_ARG;
@@ -2253,6 +2276,7 @@ whale_status whale_project_kv(const whale_config* cfg, long long rows, const voi
 whale_status whale_attend_states(const whale_config* cfg, const void* q, const void* layer_states,
                                  const int* seq_offsets, const whale_layer_weights* w, void* a,
                                  const whale_shape_hint* hint, void* ws, size_t ws_bytes, whale_stream_t stream) {
+  NvtxRange range("whale_attend_states");
   Shape s;
   Layout L;
   WCHECK(common_checks(cfg, hint, &s, ws, ws_bytes, &L));
@@ -2287,6 +2311,7 @@ whale_status whale_attend_states(const whale_config* cfg, const void* q, const v
 whale_status whale_cross_attention(const whale_config* cfg, const void* q, const void* kv, const int* seq_offsets,
                                    void* a, const whale_shape_hint* hint, void* ws, size_t ws_bytes,
                                    whale_stream_t stream) {
+  NvtxRange range("whale_cross_attention");
   Shape s;
   WCHECK(validate(cfg, &s));
   WCHECK(check_hint(hint));
@@ -2306,6 +2331,7 @@ whale_status whale_cross_attention(const whale_config* cfg, const void* q, const
 
 whale_status whale_fusion_mlp(const whale_config* cfg, long long rows, const void* a, const void* x, const void* w_f1,
                               const void* w_f2, void* f, void* ws, size_t ws_bytes, whale_stream_t stream) {
+  NvtxRange range("whale_fusion_mlp");
   Shape s;
   WCHECK(validate(cfg, &s));
   if (rows < 0 || !a || !x || !w_f2 || !f || (s.Fh > 0 && !w_f1)) return WHALE_ERR_INVALID_ARG;
@@ -2330,6 +2356,7 @@ whale_status whale_fusion_mlp(const whale_config* cfg, long long rows, const voi
 whale_status whale_swiglu_ffn(const whale_config* cfg, long long rows, const void* f, const float* g_ffn,
                               const void* w_upgate, const void* w_down, void* y, void* ws, size_t ws_bytes,
                               whale_stream_t stream) {
+  NvtxRange range("whale_swiglu_ffn");
   Shape s;
   WCHECK(validate(cfg, &s));
   if (rows < 0 || !f || !g_ffn || !w_upgate || !w_down || !y) return WHALE_ERR_INVALID_ARG;
@@ -2445,6 +2472,7 @@ whale_status whale_fusion_layer_backward(const whale_config* cfg, const void* to
                                          float* d_tokens, void* d_states, const whale_layer_grads* grads,
                                          const whale_shape_hint* hint, void* ws, size_t ws_bytes,
                                          whale_stream_t stream) {
+  NvtxRange range("whale_fusion_layer_backward");
   Shape s;
   WCHECK(validate(cfg, &s));
   WCHECK(check_hint(hint));
@@ -2489,6 +2517,7 @@ whale_status whale_fusion_backward(const whale_config* cfg, const void* tokens, 
                                    const int* seq_offsets, const whale_layer_weights* weights, const float* d_out,
                                    float* d_tokens, void* d_states, const whale_layer_grads* grads,
                                    const whale_shape_hint* hint, void* ws, size_t ws_bytes, whale_stream_t stream) {
+  NvtxRange range("whale_fusion_backward");
   Shape s;
   WCHECK(validate(cfg, &s));
   WCHECK(check_hint(hint));
