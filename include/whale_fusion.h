@@ -89,7 +89,8 @@ typedef struct {
                          WHALE_MATERIALIZED_KV */
   float eps;          /* RMSNorm epsilon */
 } whale_config;
-/* Supported: fp32 — any d with d % n_heads == 0 and d_head in {8, 16, 32, 64, 128} (SIMT correctness path).
+/* Supported: fp32 — any d with d % n_heads == 0 and d_head in {8, 16, 32, 64, 128} (SIMT correctness path;
+ *            its GEMMs take at most 65535 * 64 rows, so total_L and B * n_tokens up to 4 194 240).
  *            bf16 — d % 64 == 0, d_head in {32, 64}, n_heads 2, 4 or a multiple of 8 (the
  *            attention kernels take min(n_heads, 8) heads per CTA), ffn_hidden % 64 == 0,
  *            fusion_hidden % 64 == 0. Any n_tokens >= 1.
